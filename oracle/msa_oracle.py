@@ -1,0 +1,337 @@
+"""Plain fp64 CPU oracle for the memory path of one Memory Sparse Attention layer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or run
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` use it.  It shares no code with the CUDA library.
+
+What the method computes, and where it is stated
+-------------------------------------------------
+* "MSA: Memory Sparse Attention" README, section "Architecture": document latent
+  states K / V / K_r are compressed by chunk-mean pooling; a router scores
+  relevance by cosine similarity, averaged over router heads and then maximised
+  over the query's tokens; the top-k documents are selected and their compressed
+  K / V are concatenated with the query's local K / V for attention.
+* Same README, Figure 2 caption: the MSA layer uses document-wise ("parallel")
+  RoPE on the memory side.  The blog post "MSA" (moses-y.github.io), section
+  "What This Does": document-wise RoPE keeps positions from drifting between
+  training and inference.
+* Same README, section "Inference Pipeline", stages 1-2: memory is encoded
+  offline into chunk-pooled (K̄, V̄, K̄_r); online, the query's Q_r is matched
+  against K̄_r, the top-k documents are picked, and only their K̄ / V̄ are loaded
+  and concatenated with the local context.
+* "MSA × Qwen3.5" model card, section "Architecture summary": full-attention MSA
+  layers concatenate the top-k chunks' K / V with the local KV in sparse
+  attention.
+
+The pages print no formulas.  Where they leave a step open this module takes
+the plainest reading and says so at the function (the list of readings):
+  R1 RoPE is the rotate-half form, ω_i = θ^(-2i/d) for i < d/2, applied to K only
+     (not V, not K_r), at the token's position inside its own document.
+  R2 A chunk is P consecutive tokens of one document; the last chunk of a
+     document may be shorter and is averaged over its actual token count.
+  R3 Cosine uses max(‖x‖, 1e-12) as the norm (only artificial zero vectors reach it).
+  R4 A document's score is the maximum of its chunks' scores; every token of one
+     query shares one top-k set; batch rows are independent.
+  R5 Top-k output is sorted by score descending, ties broken by lower index.
+  R6 Attention keys are [selected memory rows (no mask)] ++ [local rows, causal,
+     bottom-right aligned: query token i sits at local position Lloc - Tq + i];
+     q-head h reads KV head floor(h / (Hq / Hkv)); the scale is 1/sqrt(d).
+  R7 Stored bf16 values are the fp64 result rounded to nearest, ties to even.
+
+Layouts are row-major with the innermost dimension last:
+  K, V [Ntok, Hkv, d]; Kr [Ntok, Hr, dr]; doc_tok_off int64 [D+1]
+  Kbar, Vbar [C, Hkv, d]; Krbar [C, Hr, dr]; doc_chunk_off int64 [D+1]
+  Qr [B, Tq, Hr, dr]; doc_scores [B, D]; topk_idx int [B, k]
+  Q [B, Tq, Hq, d]; Kloc, Vloc [B, Lloc, Hkv, d]; Kmem, Vmem [B, M, Hkv, d]
+
+Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
+closed forms, textbook special cases, an independent library routine or brute
+force (see the docstring of each function for which).
+"""
+from __future__ import annotations
+
+import itertools
+import math
+
+import numpy as np
+
+NORM_EPS = 1e-12  # reading R3
+
+
+# ----------------------------------------------------------------------------
+# storage rounding (reading R7)
+# ----------------------------------------------------------------------------
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """fp64 values rounded to the nearest bfloat16 (8 significant bits), ties to even.
+
+    Written from the definition of the format: 1 sign bit, 8 exponent bits, 7
+    stored mantissa bits.  Values below the smallest normal bf16 are rounded on
+    the subnormal grid (spacing 2^-133).  Pinned by exhaustive comparison with
+    the bit pattern decoding in tests.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = x != 0
+    m, e = np.frexp(x[nz])  # x = m * 2**e, 0.5 <= |m| < 1
+    # normal bf16: 8 significant bits -> scale the mantissa by 2**8
+    e_min = -125  # frexp exponent of the smallest normal bf16 (2**-126 = 0.5 * 2**-125)
+    shift = np.where(e < e_min, 8 - (e_min - e), 8)
+    r = np.round(np.ldexp(m, shift))  # np.round is round-half-to-even
+    out[nz] = np.ldexp(r, e - shift)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# step 1: document-wise RoPE + chunk-mean pooling
+# ----------------------------------------------------------------------------
+def rope_angles(positions: np.ndarray, d: int, theta: float) -> np.ndarray:
+    """Angle p * ω_i for each position p and i < d/2, with ω_i = θ^(-2i/d) (reading R1)."""
+    i = np.arange(d // 2, dtype=np.float64)
+    omega = theta ** (-2.0 * i / d)
+    return np.asarray(positions, dtype=np.float64)[:, None] * omega[None, :]
+
+
+def rope_rotate(x: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate-half RoPE of x [T, H, d] with token positions [T] (reading R1).
+
+    For i < d/2 the pair (x_i, x_{i+d/2}) turns by the angle p * ω_i:
+      x_i'       = x_i cos - x_{i+d/2} sin
+      x_{i+d/2}' = x_{i+d/2} cos + x_i sin
+    Pins: position 0 is the identity; each pair keeps its length; the
+    relative-position identity <R_m q, R_n k> = <R_{m-n} q, k>; a hand-made
+    quarter turn.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    ang = rope_angles(positions, d, theta)[:, None, :]  # [T, 1, d/2]
+    c, s = np.cos(ang), np.sin(ang)
+    lo, hi = x[..., : d // 2], x[..., d // 2 :]
+    return np.concatenate([lo * c - hi * s, hi * c + lo * s], axis=-1)
+
+
+def chunk_offsets(doc_tok_off: np.ndarray, P: int) -> np.ndarray:
+    """doc_chunk_off [D+1]: document j owns chunks [off[j], off[j+1]), n_j = ceil(L_j / P) (R2)."""
+    L = np.diff(np.asarray(doc_tok_off, dtype=np.int64))
+    n = (L + P - 1) // P
+    return np.concatenate([[0], np.cumsum(n)]).astype(np.int64)
+
+
+def chunk_token_ranges(doc_tok_off: np.ndarray, P: int):
+    """List of (start, end, doc) token ranges, one per chunk, in chunk order (R2)."""
+    out = []
+    for j in range(len(doc_tok_off) - 1):
+        s, e = int(doc_tok_off[j]), int(doc_tok_off[j + 1])
+        for c0 in range(s, e, P):
+            out.append((c0, min(c0 + P, e), j))
+    return out
+
+
+def doc_positions(doc_tok_off: np.ndarray) -> np.ndarray:
+    """Position of every token inside its own document, restarting at 0 (R1, document-wise RoPE)."""
+    off = np.asarray(doc_tok_off, dtype=np.int64)
+    ntok = int(off[-1])
+    pos = np.arange(ntok, dtype=np.int64)
+    doc = np.searchsorted(off, pos, side="right") - 1
+    return pos - off[doc]
+
+
+def pool(K, V, Kr, doc_tok_off, P: int, theta: float, out_bf16: bool = False):
+    """Step 1, offline memory encoding: RoPE on K, then chunk means of K', V and Kr.
+
+    "MSA: Memory Sparse Attention" README, "Architecture" (chunk-mean pooling of
+    K / V / K_r) and "Inference Pipeline" stage 1 (cache chunk-pooled K̄, V̄, K̄_r);
+    Figure 2 caption (document-wise RoPE).  Readings R1, R2, R7.
+
+    Returns (Kbar, Vbar, Krbar, doc_chunk_off, kr_rnorm) with kr_rnorm[c, h] =
+    1 / max(‖Krbar[c, h]‖, 1e-12) taken from the (possibly bf16-rounded) stored Krbar.
+    Pins: a constant input pools to itself; pooling is linear; a ramp 0..n-1 pools
+    to (n-1)/2; a 52-token tail chunk averages over 52 tokens.
+    """
+    off = np.asarray(doc_tok_off, dtype=np.int64)
+    Kp = rope_rotate(K, doc_positions(off), theta)
+    V = np.asarray(V, dtype=np.float64)
+    Kr = np.asarray(Kr, dtype=np.float64)
+    ranges = chunk_token_ranges(off, P)
+    starts = np.array([r[0] for r in ranges], dtype=np.int64)
+    counts = np.array([r[1] - r[0] for r in ranges], dtype=np.float64)
+    if len(ranges) == 0:
+        z = lambda a: np.zeros((0,) + a.shape[1:])
+        return z(K), z(V), z(Kr), chunk_offsets(off, P), np.zeros((0, Kr.shape[1]))
+    # np.add.reduceat sums each [starts[c], starts[c+1]) slice; chunks tile the
+    # token axis contiguously, so these are exactly the chunk sums.
+    mean = lambda a: np.add.reduceat(a, starts, axis=0) / counts[:, None, None]
+    Kbar, Vbar, Krbar = mean(Kp), mean(V), mean(Kr)
+    if out_bf16:
+        Kbar, Vbar, Krbar = round_to_bf16(Kbar), round_to_bf16(Vbar), round_to_bf16(Krbar)
+    rnorm = 1.0 / np.maximum(np.sqrt((Krbar * Krbar).sum(-1)), NORM_EPS)
+    return Kbar, Vbar, Krbar, chunk_offsets(off, P), rnorm
+
+
+# ----------------------------------------------------------------------------
+# step 2: cosine routing
+# ----------------------------------------------------------------------------
+def cosine_scores(Qr, Krbar) -> np.ndarray:
+    """s[b, t, c] = (1/Hr) Σ_h cos(Qr[b, t, h], Krbar[c, h]).
+
+    README "Architecture": relevance by cosine similarity, mean-pooled over heads
+    (reading R3 for the norm clamp).  Pins: values in [-1, 1]; identical vectors
+    give 1, negated give -1; invariant to positive scaling of either side; Hr = 1
+    is the textbook cosine (scipy).
+    """
+    Qr = np.asarray(Qr, dtype=np.float64)
+    Kb = np.asarray(Krbar, dtype=np.float64)
+    qn = Qr / np.maximum(np.linalg.norm(Qr, axis=-1, keepdims=True), NORM_EPS)
+    kn = Kb / np.maximum(np.linalg.norm(Kb, axis=-1, keepdims=True), NORM_EPS)
+    Hr = Qr.shape[2]
+    s = np.zeros(Qr.shape[:2] + (Kb.shape[0],))
+    for h in range(Hr):
+        s += qn[:, :, h, :] @ kn[:, h, :].T  # [B, Tq, C]
+    return s / Hr
+
+
+def route(Qr, Krbar, doc_chunk_off) -> np.ndarray:
+    """Step 2: doc_score[b, j] = max over chunks c of document j of max over tokens t of s[b, t, c].
+
+    README "Architecture": head mean first, then the token-wise max; the document
+    score is the max over the document's chunks (reading R4).  A document with no
+    chunks scores -inf.  Pins: the order head-mean-then-max matters and is checked
+    on a hand case; a document whose K_r tokens all equal a query token scores 1.
+    """
+    s = cosine_scores(Qr, Krbar)          # [B, Tq, C]
+    m = s.max(axis=1)                     # token-wise max -> [B, C]
+    off = np.asarray(doc_chunk_off, dtype=np.int64)
+    D = len(off) - 1
+    out = np.full((m.shape[0], D), -np.inf)
+    for j in range(D):
+        if off[j + 1] > off[j]:
+            out[:, j] = m[:, off[j] : off[j + 1]].max(axis=1)
+    return out
+
+
+def route_docs(Qr, Krbar, doc_chunk_off, docs) -> np.ndarray:
+    """route() restricted to the listed documents: [B, len(docs)] (for sampled full-size checks)."""
+    off = np.asarray(doc_chunk_off, dtype=np.int64)
+    Kb = np.asarray(Krbar)
+    out = np.full((np.asarray(Qr).shape[0], len(docs)), -np.inf)
+    for n, j in enumerate(docs):
+        a, b = int(off[j]), int(off[j + 1])
+        if b > a:
+            out[:, n] = cosine_scores(Qr, Kb[a:b]).max(axis=(1, 2))
+    return out
+
+
+# ----------------------------------------------------------------------------
+# step 3: top-k documents
+# ----------------------------------------------------------------------------
+def topk(doc_scores, k: int):
+    """Step 3: the k best documents per row, sorted by (score desc, index asc) (reading R5).
+
+    README "Architecture" / "Inference Pipeline" stage 2: select the top-k
+    documents.  Pins: brute force over every k-subset on small rows; agreement
+    with a full stable sort.
+    """
+    sc = np.asarray(doc_scores, dtype=np.float64)
+    B, D = sc.shape
+    idx = np.zeros((B, k), dtype=np.int64)
+    val = np.zeros((B, k))
+    for b in range(B):
+        order = sorted(range(D), key=lambda j: (-sc[b, j], j))[:k]
+        idx[b] = order
+        val[b] = sc[b, order]
+    return idx, val
+
+
+def topk_bruteforce(doc_scores_row, k: int):
+    """Reference for tiny rows: the k-subset with the largest score sum, then sorted (R5)."""
+    row = list(doc_scores_row)
+    best, best_key = None, None
+    for sub in itertools.combinations(range(len(row)), k):
+        # maximise the sum; among equal sums prefer the lexicographically smallest index set
+        key = (sum(row[j] for j in sub), tuple(-j for j in sub))
+        if best_key is None or key > best_key:
+            best, best_key = sub, key
+    return sorted(best, key=lambda j: (-row[j], j))
+
+
+# ----------------------------------------------------------------------------
+# step 4: gather the selected documents' chunks
+# ----------------------------------------------------------------------------
+def gather(topk_idx, doc_chunk_off, Kbar, Vbar, Mmax: int):
+    """Step 4: concatenate the selected documents' chunks, in rank order (README stage 2).
+
+    Within a document the chunks keep their order.  Rows past mem_len[b] are zero.
+    Pins: the copy is exact; mem_len equals the sum of the selected n_j.
+    """
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    off = np.asarray(doc_chunk_off, dtype=np.int64)
+    Kb, Vb = np.asarray(Kbar), np.asarray(Vbar)
+    B = idx.shape[0]
+    Km = np.zeros((B, Mmax) + Kb.shape[1:], dtype=Kb.dtype)
+    Vm = np.zeros((B, Mmax) + Vb.shape[1:], dtype=Vb.dtype)
+    mem_len = np.zeros(B, dtype=np.int64)
+    for b in range(B):
+        rows = [c for j in idx[b] for c in range(off[j], off[j + 1])]
+        n = len(rows)
+        if n > Mmax:
+            raise ValueError("selected documents exceed Mmax rows")
+        Km[b, :n], Vm[b, :n] = Kb[rows], Vb[rows]
+        mem_len[b] = n
+    return Km, Vm, mem_len
+
+
+# ----------------------------------------------------------------------------
+# step 5: sparse attention over [memory ++ causal local]
+# ----------------------------------------------------------------------------
+def attention(Q, Kloc, Vloc, Kmem, Vmem, mem_len, scale=None):
+    """Step 5: softmax(scale q·kᵀ) v over [memory rows ++ causal local rows] (reading R6).
+
+    "MSA × Qwen3.5" card, "Architecture summary" (full layers: concat top-k
+    chunks' K/V with local KV in sparse attention); README "Architecture".
+    Returns (O [B, Tq, Hq, d], lse [B, Hq, Tq]) with lse the natural-log
+    normaliser of the scaled logits.
+    Pins: no memory rows equals plain causal attention and matches torch's
+    scaled_dot_product_attention in fp64; identical keys return the mean of V;
+    Hq = Hkv is plain multi-head attention; every row's weights sum to 1.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    Kl, Vl = np.asarray(Kloc, dtype=np.float64), np.asarray(Vloc, dtype=np.float64)
+    Km, Vm = np.asarray(Kmem, dtype=np.float64), np.asarray(Vmem, dtype=np.float64)
+    B, Tq, Hq, d = Q.shape
+    Lloc, Hkv = Kl.shape[1], Kl.shape[2]
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    group = Hq // Hkv
+    O = np.zeros_like(Q)
+    lse = np.zeros((B, Hq, Tq))
+    for b in range(B):
+        M = int(mem_len[b])
+        for h in range(Hq):
+            g = h // group
+            keys = np.concatenate([Km[b, :M, g], Kl[b, :, g]], axis=0)   # [M + Lloc, d]
+            vals = np.concatenate([Vm[b, :M, g], Vl[b, :, g]], axis=0)
+            logits = scale * (Q[b, :, h] @ keys.T)                       # [Tq, M + Lloc]
+            pos = Lloc - Tq + np.arange(Tq)
+            visible = np.concatenate(
+                [np.ones((Tq, M), bool), np.arange(Lloc)[None, :] <= pos[:, None]], axis=1)
+            logits = np.where(visible, logits, -np.inf)
+            mx = logits.max(axis=1, keepdims=True)
+            w = np.exp(logits - mx)
+            den = w.sum(axis=1, keepdims=True)
+            O[b, :, h] = (w / den) @ vals
+            lse[b, h] = (mx + np.log(den))[:, 0]
+    return O, lse
+
+
+# ----------------------------------------------------------------------------
+# steps 2-5 composed: one MSA layer's query path over a pooled bank
+# ----------------------------------------------------------------------------
+def layer_forward(Qr, Krbar, doc_chunk_off, k: int, Q, Kloc, Vloc, Kbar, Vbar, Mmax: int, scale=None):
+    """Route -> top-k -> gather -> attention, in the README's "Inference Pipeline" order.
+
+    Returns a dict with doc_scores, topk_idx, topk_score, mem_len, O, lse.
+    """
+    ds = route(Qr, Krbar, doc_chunk_off)
+    ti, ts = topk(ds, k)
+    Km, Vm, ml = gather(ti, doc_chunk_off, Kbar, Vbar, Mmax)
+    O, lse = attention(Q, Kloc, Vloc, Km, Vm, ml, scale)
+    return dict(doc_scores=ds, topk_idx=ti, topk_score=ts, mem_len=ml, O=O, lse=lse)

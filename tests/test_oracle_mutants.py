@@ -1,0 +1,59 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that a pin catches each one.
+
+Each mutant is the oracle function's own source with one textual edit, compiled
+into the oracle module's namespace; the pin that should catch it must then fail.
+"""
+import inspect
+import textwrap
+
+import pytest
+
+from oracle import msa_oracle as O
+import tests.test_oracle_pins as pins
+
+MUTANTS = [
+    # (function, original text, planted mistake, pin that must fail, pin args)
+    ("rope_rotate", "lo * c - hi * s, hi * c + lo * s", "lo * c + hi * s, hi * c - lo * s",
+     "test_rope_quarter_turn_by_hand", ()),
+    ("doc_positions", "return pos - off[doc]", "return pos",
+     "test_pool_rotates_k_at_document_local_positions", ()),
+    ("pool", "/ counts[:, None, None]", "/ float(P)",
+     "test_pool_ramp_mean_closed_form_and_tail", ()),
+    ("route", "m = s.max(axis=1)", "m = s.max(axis=1) * 0 + s.mean(axis=1)",
+     "test_planted_document_scores_one_and_is_selected", ()),
+    ("route", "s = cosine_scores(Qr, Krbar)",
+     "s = np.mean([cosine_scores(Qr[:, :, h:h + 1], Krbar[:, h:h + 1]).max(axis=1, keepdims=True)"
+     " for h in range(np.asarray(Qr).shape[2])], axis=0)",
+     "test_head_mean_then_token_max_hand_case", ()),
+    ("cosine_scores", "s / Hr", "s",
+     "test_cosine_identical_negated_and_scale_invariant", ()),
+    ("cosine_scores", "qn[:, :, h, :] @ kn[:, h, :].T", "Qr[:, :, h, :] @ Kb[:, h, :].T",
+     "test_cosine_identical_negated_and_scale_invariant", ()),
+    ("topk", "key=lambda j: (-sc[b, j], j)", "key=lambda j: (-sc[b, j], -j)",
+     "test_topk_sorted_and_ties_prefer_lower_index", ()),
+    ("gather", "for c in range(off[j], off[j + 1])", "for c in range(off[j], off[j + 1] - 1)",
+     "test_gather_copies_selected_chunks_in_rank_order", ()),
+    ("attention", "<= pos[:, None]", "< pos[:, None]",
+     "test_attention_matches_sdpa", (7, 7, 0, 4, 2)),
+    ("attention", "g = h // group", "g = h % Hkv",
+     "test_attention_matches_sdpa", (6, 9, 13, 8, 2)),
+    ("attention", "pos = Lloc - Tq + np.arange(Tq)", "pos = np.arange(Tq)",
+     "test_attention_matches_sdpa", (5, 11, 0, 2, 2)),
+    ("attention", "[np.ones((Tq, M), bool),", "[np.arange(M)[None, :] <= np.arange(Tq)[:, None],",
+     "test_attention_matches_sdpa", (6, 9, 13, 8, 2)),
+]
+
+
+def _mutant(fn_name, old, new):
+    src = textwrap.dedent(inspect.getsource(getattr(O, fn_name)))
+    assert old in src, f"mutation anchor not found in {fn_name}"
+    ns = {}
+    exec(compile(src.replace(old, new, 1), f"<mutant {fn_name}>", "exec"), O.__dict__, ns)
+    return ns[fn_name]
+
+
+@pytest.mark.parametrize("fn,old,new,pin,args", MUTANTS, ids=[f"{m[0]}:{i}" for i, m in enumerate(MUTANTS)])
+def test_pin_catches_planted_mistake(monkeypatch, fn, old, new, pin, args):
+    monkeypatch.setattr(O, fn, _mutant(fn, old, new))
+    with pytest.raises(AssertionError):
+        getattr(pins, pin)(*args)

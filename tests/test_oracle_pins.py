@@ -1,0 +1,330 @@
+"""Pins for the fp64 oracle: closed forms, textbook cases, a library routine, brute force.
+
+None of these re-types an oracle formula: each checks the oracle against a fact
+that the pages or the mathematics fix independently of how the oracle computes it.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.spatial.distance as ssd
+import torch
+import torch.nn.functional as F
+
+from oracle import msa_oracle as O
+from workloads import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(1234)
+
+
+def load_golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, rest = line.split("=", 1)
+            vals[key.strip()] = np.array([float(x) for x in rest.split()])
+    return vals
+
+
+# ------------------------------------------------------------------ bf16 rounding
+def _bf16_decode(bits):
+    """Value of a bf16 bit pattern from the format's definition (1 / 8 / 7 bits)."""
+    s = (bits >> 15) & 1
+    e = (bits >> 7) & 0xFF
+    m = bits & 0x7F
+    if e == 0:
+        v = m * 2.0 ** (-133)
+    else:
+        v = (1 + m / 128.0) * 2.0 ** (e - 127)
+    return -v if s else v
+
+
+def test_bf16_rounding_fixed_points_and_midpoints():
+    finite = [b for b in range(0x0000, 0x7F80)]  # every non-negative finite pattern
+    vals = np.array([_bf16_decode(b) for b in finite])
+    assert np.array_equal(O.round_to_bf16(vals), vals)
+    assert np.array_equal(O.round_to_bf16(-vals), -vals)
+    lo, hi = vals[:-1], vals[1:]
+    mid = (lo + hi) / 2
+    even = np.array([(b & 1) == 0 for b in finite[:-1]])
+    expect = np.where(even, lo, hi)
+    assert np.array_equal(O.round_to_bf16(mid), expect)
+    gap = hi - lo
+    assert np.array_equal(O.round_to_bf16(mid - gap * 1e-3), lo)
+    assert np.array_equal(O.round_to_bf16(mid + gap * 1e-3), hi)
+
+
+# ------------------------------------------------------------------ RoPE
+def test_rope_position_zero_is_identity():
+    x = rng.standard_normal((5, 3, 16))
+    assert np.array_equal(O.rope_rotate(x, np.zeros(5, int), 1e6), x)
+
+
+def test_rope_keeps_pair_lengths():
+    x = rng.standard_normal((7, 2, 32))
+    y = O.rope_rotate(x, np.arange(7) * 37, 1e4)
+    n = lambda a: a[..., :16] ** 2 + a[..., 16:] ** 2
+    np.testing.assert_allclose(n(y), n(x), rtol=1e-12)
+
+
+def test_rope_relative_position_identity():
+    d = 64
+    q, k = rng.standard_normal((1, 1, d)), rng.standard_normal((1, 1, d))
+    for m, n in [(5, 3), (100, 7), (511, 510), (9, 0)]:
+        lhs = np.sum(O.rope_rotate(q, [m], 1e6) * O.rope_rotate(k, [n], 1e6))
+        rhs = np.sum(O.rope_rotate(q, [m - n], 1e6) * k)
+        assert abs(lhs - rhs) < 1e-10
+
+
+def test_rope_quarter_turn_by_hand():
+    g = load_golden("rope_quarter_turn.txt")
+    theta = float(g["theta"][0])
+    x = g["x"].reshape(1, 1, 4)
+    y = O.rope_rotate(x, [1], theta)[0, 0]
+    np.testing.assert_allclose(y, g["expected"], atol=1e-12)
+
+
+def test_document_positions_restart():
+    off = np.array([0, 3, 3, 8])
+    assert O.doc_positions(off).tolist() == [0, 1, 2, 0, 1, 2, 3, 4]
+
+
+# ------------------------------------------------------------------ pooling
+def _ragged_offsets():
+    return np.array([0, 500, 1000, 1064, 1065, 1200], dtype=np.int64)
+
+
+def test_chunk_offsets_ceil():
+    off = _ragged_offsets()
+    assert O.chunk_offsets(off, 64).tolist() == [0, 8, 16, 17, 18, 21]
+
+
+def test_pool_constant_input_pools_to_itself():
+    off = _ragged_offsets()
+    n = int(off[-1])
+    c = rng.standard_normal((1, 2, 8))
+    V = np.repeat(c, n, axis=0)
+    Kz = np.zeros((n, 2, 8))
+    Kb, Vb, Krb, _, _ = O.pool(Kz, V, V, off, 64, 1e6)
+    np.testing.assert_allclose(Vb, np.repeat(c, len(Vb), 0), rtol=1e-14)
+    np.testing.assert_allclose(Krb, np.repeat(c, len(Vb), 0), rtol=1e-14)
+
+
+def test_pool_ramp_mean_closed_form_and_tail():
+    off = _ragged_offsets()
+    n = int(off[-1])
+    ranges = O.chunk_token_ranges(off, 64)
+    V = np.zeros((n, 1, 4))
+    for s, e, _ in ranges:
+        V[s:e, 0, :] = np.arange(e - s)[:, None]      # 0, 1, ..., |c|-1 inside each chunk
+    _, Vb, _, _, _ = O.pool(np.zeros_like(V), V, V, off, 64, 1e6)
+    expect = np.array([(e - s - 1) / 2 for s, e, _ in ranges])
+    np.testing.assert_allclose(Vb[:, 0, 0], expect, rtol=1e-14)
+    # document 0 has 500 tokens: 7 full chunks and a 52-token tail averaging 0..51
+    assert ranges[7][1] - ranges[7][0] == 52 and Vb[7, 0, 0] == 25.5
+
+
+def test_pool_is_linear():
+    off = _ragged_offsets()
+    n = int(off[-1])
+    X = [rng.standard_normal((n, 2, 8)) for _ in range(6)]
+    a, b = 0.7, -1.9
+    P1 = O.pool(X[0], X[1], X[2], off, 64, 1e6)
+    P2 = O.pool(X[3], X[4], X[5], off, 64, 1e6)
+    P3 = O.pool(a * X[0] + b * X[3], a * X[1] + b * X[4], a * X[2] + b * X[5], off, 64, 1e6)
+    for i in range(3):
+        np.testing.assert_allclose(P3[i], a * P1[i] + b * P2[i], atol=1e-12)
+
+
+def test_pool_rotates_k_at_document_local_positions():
+    # With P = 1 each chunk is one token: K̄ is that token rotated at its position
+    # inside its own document, V̄ and K̄r are not rotated.
+    off = np.array([0, 3, 7])
+    K = rng.standard_normal((7, 2, 8))
+    Kb, Vb, Krb, _, _ = O.pool(K, K, K, off, 1, 10.0)
+    np.testing.assert_array_equal(Vb, K)
+    np.testing.assert_array_equal(Krb, K)
+    for t, p in enumerate([0, 1, 2, 0, 1, 2, 3]):
+        ang = p * 10.0 ** (-2 * np.arange(4) / 8)
+        lo, hi = K[t, :, :4], K[t, :, 4:]
+        exp = np.concatenate([lo * np.cos(ang) - hi * np.sin(ang), hi * np.cos(ang) + lo * np.sin(ang)], -1)
+        np.testing.assert_allclose(Kb[t], exp, atol=1e-12)
+
+
+def test_pool_rnorm_is_inverse_norm_of_stored_bank():
+    off = np.array([0, 64, 130])
+    X = rng.standard_normal((130, 3, 16))
+    _, _, Krb, _, rn = O.pool(X, X, X, off, 64, 1e6, out_bf16=True)
+    assert np.array_equal(O.round_to_bf16(Krb), Krb)
+    for c in range(Krb.shape[0]):
+        for h in range(3):
+            assert abs(rn[c, h] * math.sqrt(sum(v * v for v in Krb[c, h])) - 1) < 1e-13
+
+
+# ------------------------------------------------------------------ cosine routing
+def test_cosine_in_range_and_textbook_for_one_head():
+    Qr = rng.standard_normal((2, 5, 1, 12))
+    Kb = rng.standard_normal((9, 1, 12))
+    s = O.cosine_scores(Qr, Kb)
+    assert np.all(np.abs(s) <= 1 + 1e-15)
+    for b, t, c in itertools.product(range(2), range(5), range(9)):
+        assert abs(s[b, t, c] - (1 - ssd.cosine(Qr[b, t, 0], Kb[c, 0]))) < 1e-12
+
+
+def test_cosine_identical_negated_and_scale_invariant():
+    Kb = rng.standard_normal((4, 3, 16))
+    Qr = np.stack([Kb[2], -Kb[1]])[None]                  # [1, 2, 3, 16]
+    s = O.cosine_scores(Qr, Kb)
+    assert abs(s[0, 0, 2] - 1) < 1e-14 and abs(s[0, 1, 1] + 1) < 1e-14
+    s2 = O.cosine_scores(3.7 * Qr, 0.2 * Kb)
+    np.testing.assert_allclose(s2, s, atol=1e-14)
+
+
+def test_head_mean_then_token_max_hand_case():
+    g = load_golden("route_hand_case.txt")
+    Qr = g["Qr"].reshape(1, 2, 2, 2)
+    Kb = g["Krbar"].reshape(1, 2, 2)
+    ds = O.route(Qr, Kb, np.array([0, 1]))
+    assert abs(ds[0, 0] - g["doc_score"][0]) < 1e-12
+    assert abs(ds[0, 0] - g["max_then_mean"][0]) > 0.2   # the other order gives a different number
+
+
+def test_document_score_is_max_over_its_chunks():
+    Kb = rng.standard_normal((6, 2, 8))
+    Qr = rng.standard_normal((1, 3, 2, 8))
+    off = np.array([0, 2, 2, 6])                          # doc 1 is empty
+    ds = O.route(Qr, Kb, off)
+    per_chunk = [max(np.mean([1 - ssd.cosine(Qr[0, t, h], Kb[c, h]) for h in range(2)])
+                     for t in range(3)) for c in range(6)]
+    assert abs(ds[0, 0] - max(per_chunk[0:2])) < 1e-12
+    assert ds[0, 1] == -np.inf
+    assert abs(ds[0, 2] - max(per_chunk[2:6])) < 1e-12
+
+
+def test_planted_document_scores_one_and_is_selected():
+    cfg = synth.get_config("tiny")
+    q = synth.gen_query(cfg)
+    K, V, Kr = synth.gen_raw_slab(cfg, 0, cfg.D, Qr0=q["Qr"][0])
+    off = synth.doc_tok_offsets(cfg)
+    _, _, Krb, coff, _ = O.pool(K.numpy(), V.numpy(), Kr.numpy(), off, cfg.P, cfg.theta)
+    ds = O.route(q["Qr"].numpy(), Krb, coff)
+    assert abs(ds[0, 17] - 1.0) < 1e-12
+    assert ds[0].max() == ds[0, 17]
+    idx, _ = O.topk(ds, cfg.k)
+    assert idx[0, 0] == 17
+
+
+# ------------------------------------------------------------------ top-k
+@pytest.mark.parametrize("D,k", [(5, 1), (6, 2), (9, 3), (12, 3)])
+def test_topk_equals_bruteforce(D, k):
+    for trial in range(20):
+        row = rng.integers(-4, 5, size=D).astype(float) if trial % 2 else rng.standard_normal(D)
+        idx, val = O.topk(row[None], k)
+        assert list(idx[0]) == O.topk_bruteforce(row, k)
+        assert np.array_equal(val[0], row[idx[0]])
+
+
+def test_topk_sorted_and_ties_prefer_lower_index():
+    row = np.array([0.5, 0.9, 0.5, 0.9, 0.1, 0.5])
+    idx, _ = O.topk(row[None], 4)
+    assert idx[0].tolist() == [1, 3, 0, 2]
+    full = np.lexsort((np.arange(6), -row))
+    assert idx[0].tolist() == full[:4].tolist()
+
+
+# ------------------------------------------------------------------ gather
+def test_gather_copies_selected_chunks_in_rank_order():
+    off = np.array([0, 3, 4, 4, 9])
+    Kb = rng.standard_normal((9, 2, 4))
+    Vb = rng.standard_normal((9, 2, 4))
+    Km, Vm, ml = O.gather(np.array([[3, 0, 2], [1, 3, 0]]), off, Kb, Vb, 10)
+    assert ml.tolist() == [8, 9]
+    assert np.array_equal(Km[0, :8], Kb[[4, 5, 6, 7, 8, 0, 1, 2]])
+    assert np.array_equal(Vm[1, :9], Vb[[3, 4, 5, 6, 7, 8, 0, 1, 2]])
+    assert not Km[0, 8:].any()
+
+
+# ------------------------------------------------------------------ attention
+def _sdpa(Q, K, V, mask, scale):
+    """torch's fp64 CPU scaled_dot_product_attention as the independent routine. Q [Tq,H,d]."""
+    q = torch.from_numpy(Q).permute(1, 0, 2)[None]
+    k = torch.from_numpy(K).permute(1, 0, 2)[None]
+    v = torch.from_numpy(V).permute(1, 0, 2)[None]
+    o = F.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(mask),
+                                       scale=scale, enable_gqa=q.shape[1] != k.shape[1])
+    return o[0].permute(1, 0, 2).numpy()
+
+
+@pytest.mark.parametrize("Tq,Lloc,M,Hq,Hkv", [(7, 7, 0, 4, 2), (5, 11, 0, 2, 2), (6, 9, 13, 8, 2), (1, 20, 4, 4, 1)])
+def test_attention_matches_sdpa(Tq, Lloc, M, Hq, Hkv):
+    d = 16
+    Q = rng.standard_normal((1, Tq, Hq, d))
+    Kl, Vl = rng.standard_normal((2, 1, Lloc, Hkv, d))
+    Km, Vm = rng.standard_normal((2, 1, M + 3, Hkv, d))   # 3 pad rows past mem_len
+    Oo, lse = O.attention(Q, Kl, Vl, Km, Vm, [M])
+    pos = Lloc - Tq + np.arange(Tq)
+    mask = np.concatenate([np.ones((Tq, M), bool), np.arange(Lloc)[None] <= pos[:, None]], 1)
+    ref = _sdpa(Q[0], np.concatenate([Km[0, :M], Kl[0]]), np.concatenate([Vm[0, :M], Vl[0]]),
+                mask, 1 / math.sqrt(d))
+    np.testing.assert_allclose(Oo[0], ref, atol=1e-12)
+
+
+def test_attention_no_memory_is_plain_causal_attention():
+    Q = rng.standard_normal((1, 9, 2, 8))
+    Kl, Vl = rng.standard_normal((2, 1, 9, 2, 8))
+    Oo, _ = O.attention(Q, Kl, Vl, np.zeros((1, 4, 2, 8)), np.zeros((1, 4, 2, 8)), [0])
+    q = torch.from_numpy(Q[0]).permute(1, 0, 2)
+    ref = F.scaled_dot_product_attention(q, torch.from_numpy(Kl[0]).permute(1, 0, 2),
+                                         torch.from_numpy(Vl[0]).permute(1, 0, 2), is_causal=True)
+    np.testing.assert_allclose(Oo[0], ref.permute(1, 0, 2).numpy(), atol=1e-12)
+
+
+def test_attention_identical_keys_give_mean_of_values_and_weights_sum_to_one():
+    Tq, Lloc, M, d = 4, 6, 5, 8
+    key = rng.standard_normal(d)
+    Kl = np.broadcast_to(key, (1, Lloc, 1, d)).copy()
+    Km = np.broadcast_to(key, (1, M, 1, d)).copy()
+    Vl, Vm = rng.standard_normal((1, Lloc, 1, d)), rng.standard_normal((1, M, 1, d))
+    Q = rng.standard_normal((1, Tq, 2, d))
+    Oo, lse = O.attention(Q, Kl, Vl, Km, Vm, [M])
+    for i in range(Tq):
+        vis = np.concatenate([Vm[0, :, 0], Vl[0, : Lloc - Tq + i + 1, 0]])
+        np.testing.assert_allclose(Oo[0, i, 0], vis.mean(0), atol=1e-12)
+        # equal logits: the normaliser is logit + log(number of visible keys)
+        logit = Q[0, i, 1] @ key / math.sqrt(d)
+        assert abs(lse[0, 1, i] - (logit + math.log(len(vis)))) < 1e-12
+
+
+def test_attention_hand_case():
+    g = load_golden("attention_hand_case.txt")
+    d = 2
+    Q = g["q"].reshape(1, 1, 1, d)
+    Kl = g["k_local"].reshape(1, 1, 1, d)
+    Vl = g["v_local"].reshape(1, 1, 1, d)
+    Km = g["k_mem"].reshape(1, 1, 1, d)
+    Vm = g["v_mem"].reshape(1, 1, 1, d)
+    Oo, _ = O.attention(Q, Kl, Vl, Km, Vm, [1], scale=1.0)
+    np.testing.assert_allclose(Oo[0, 0, 0], g["out"], atol=1e-12)
+
+
+# ------------------------------------------------------------------ composed layer
+def test_layer_with_all_documents_is_dense_attention_over_bank():
+    cfg = synth.get_config("tiny").scaled(D=6, L=100, k=6)
+    q = synth.gen_query(cfg)
+    K, V, Kr = synth.gen_raw_slab(cfg, 0, cfg.D, Qr0=q["Qr"][0])
+    off = synth.doc_tok_offsets(cfg)
+    Kb, Vb, Krb, coff, _ = O.pool(K.numpy(), V.numpy(), Kr.numpy(), off, cfg.P, cfg.theta)
+    r = O.layer_forward(q["Qr"].numpy(), Krb, coff, cfg.k, q["Q"].numpy(), q["Kloc"].numpy(),
+                        q["Vloc"].numpy(), Kb, Vb, Mmax=int(coff[-1]))
+    assert r["mem_len"][0] == coff[-1]
+    # attention is invariant to the order of the (unmasked) memory rows: compare with
+    # dense attention over the whole bank in natural order
+    Od, _ = O.attention(q["Q"].numpy(), q["Kloc"].numpy(), q["Vloc"].numpy(), Kb[None], Vb[None],
+                        [int(coff[-1])])
+    np.testing.assert_allclose(r["O"], Od, atol=1e-12)
