@@ -1,0 +1,232 @@
+/*
+ * msa.h - C ABI of the Memory Sparse Attention (MSA) memory-path library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * One MSA layer's memory path, as the "MSA: Memory Sparse Attention" README
+ * describes it ("Architecture" and "Inference Pipeline" sections):
+ *   1. msa_pool         - document-wise RoPE on K, then chunk-mean pooling of
+ *                         K, V and the router keys Kr into the memory bank.
+ *   2.+3. msa_route_topk - cosine routing of the query's router projections Qr
+ *                         against the bank's pooled router keys (mean over
+ *                         router heads, max over query tokens, max over a
+ *                         document's chunks), then the top-k documents.
+ *   4. msa_gather       - copy the selected documents' pooled K/V chunks.
+ *   5. msa_sparse_attn  - GQA softmax attention of the query tokens over
+ *                         [selected memory rows ++ causal local KV].
+ *   msa_layer_forward   - steps 2-5 fused: the attention reads the selected
+ *                         chunks straight from the bank by index.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.  Every tensor argument is a DEVICE pointer (to memory the caller
+ *   allocated and owns) unless its comment says "host".  Tensors are dense,
+ *   row-major, innermost dimension last, and 16-byte aligned.  The library
+ *   never allocates, frees or synchronises inside these calls.
+ * Types.  msa_dtype names the storage type of the float tensors (bf16 or fp32);
+ *   every accumulation is fp32.  Offsets are int64, selected indices int32,
+ *   scores and normalisers fp32.
+ * Streams.  All device work is enqueued on `stream` (a cudaStream_t; NULL is
+ *   the legacy default stream), in call order.
+ * Errors.  Arguments are checked on the host before anything is launched; a
+ *   bad argument returns an error and launches nothing.  A failed launch
+ *   returns MSA_ERR_CUDA.  Problems only the device can see (an index out of
+ *   range, inconsistent offsets, a bounded wait that ran out) are OR-ed as
+ *   MSA_FLAG_* bits into *err_flag (an int32 the caller zeroes beforehand and
+ *   reads after synchronising; NULL turns the reporting off); the offending
+ *   item is skipped and no kernel traps.
+ *   No C++ exception crosses this interface.
+ * Reading of the pages (they print no formulas): RoPE is the rotate-half form
+ *   with angle p * theta^(-2i/d) for the pair (x_i, x_{i+d/2}), p the token's
+ *   position inside its document; it is applied to K only.  The last chunk of
+ *   a document may be shorter than P and is averaged over its own tokens.
+ *   Attention is bottom-right causal on the local rows (query token i sits at
+ *   local position Lloc - Tq + i) and unmasked on memory rows; q-head h reads
+ *   KV head h / (Hq / Hkv).
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* msa_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned pointer */
+  MSA_ERR_UNSUPPORTED = -2, /* a shape or dtype this build has no kernel for */
+  MSA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than *_workspace_size */
+  MSA_ERR_CUDA = -4,        /* a CUDA launch or runtime call failed */
+} msa_status;
+
+/* Bits of the device-side error flag. */
+enum {
+  MSA_FLAG_INDEX_OOB = 1, /* a document / chunk / row index outside its tensor */
+  MSA_FLAG_OFFSETS = 2,   /* offsets that are not non-decreasing or disagree with P */
+  MSA_FLAG_TIMEOUT = 4,   /* a bounded wait on a barrier ran out */
+  MSA_FLAG_OVERFLOW = 8,  /* selected rows exceed the Mmax rows of the output */
+};
+
+typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype;
+
+/* Text for a status code; never NULL. */
+const char* msa_status_string(int status);
+
+/* Library version, "major.minor.patch". */
+const char* msa_version(void);
+
+/* Number of CUDA kernels this library has launched in this process so far
+ * (memsets and copies are not kernels and are not counted).  For accounting:
+ * the difference across a region is the number of library kernels it ran. */
+uint64_t msa_kernel_launch_count(void);
+
+/* ------------------------------------------------------------------------
+ * RoPE table (host).  Fills host_out[max_len][d/2][2] with (cos, sin) of the
+ * angle p * theta^(-2i/d), computed in fp64 by the C library and stored as
+ * fp32, for p < max_len and i < d/2.  The caller copies it to the device for
+ * msa_pool.  "MSA: Memory Sparse Attention" README, Figure 2 caption
+ * (document-wise RoPE); the rotate-half form is this library's reading.
+ * Errors: MSA_ERR_INVALID_ARG for d odd or < 2, max_len < 1, theta <= 0, or a
+ * NULL host_out.
+ * ---------------------------------------------------------------------- */
+msa_status msa_rope_table_host(double theta, int d, int max_len, float* host_out);
+
+/* ------------------------------------------------------------------------
+ * Chunk offsets (host).  out[0] = 0 and out[j+1] = out[j] + ceil(L_j / P) with
+ * L_j = doc_tok_off[j+1] - doc_tok_off[j]: document j owns chunks
+ * [out[j], out[j+1]) of the bank.  doc_tok_off and out are HOST arrays of D+1
+ * int64.  Errors: MSA_ERR_INVALID_ARG for NULL arrays, D < 0, P < 1 or a
+ * decreasing doc_tok_off.
+ * ---------------------------------------------------------------------- */
+msa_status msa_chunk_offsets_host(const int64_t* doc_tok_off, int64_t D, int P, int64_t* out);
+
+/* ------------------------------------------------------------------------
+ * Step 1: offline memory encoding ("Inference Pipeline", stage 1; "Architecture":
+ * chunk-mean pooling of K / V / Kr).  For document j (tokens
+ * [doc_tok_off[j], doc_tok_off[j+1]), chunks [doc_chunk_off[j], doc_chunk_off[j+1]))
+ * and its chunk c covering tokens [s, e) (P tokens; the last chunk of a document
+ * may be shorter):
+ *   Kbar[c]  = mean over t in [s,e) of RoPE_{t - doc_tok_off[j]}(K[t])
+ *   Vbar[c]  = mean V[t],   Krbar[c] = mean Kr[t]   (not rotated)
+ *   kr_rnorm[c, h] = 1 / max(||Krbar_stored[c, h]||, 1e-12)   (fp32, optional)
+ * The norm is taken from the stored (rounded) Krbar so that routing sees exactly
+ * the bank it reads.
+ *   K, V     [Ntok, Hkv, d]   dtype dt
+ *   Kr       [Ntok, Hr, dr]   dtype dt
+ *   doc_tok_off, doc_chunk_off  int64 [D+1], both starting at 0; document j must
+ *            own exactly ceil(L_j / P) chunks and doc_chunk_off[D] == C.
+ *   rope_cs  fp32 [max_len, d/2, 2] from msa_rope_table_host; every document
+ *            must be at most max_len tokens long.
+ *   Kbar, Vbar [C, Hkv, d], Krbar [C, Hr, dr] (dtype dt, outputs)
+ *   kr_rnorm fp32 [C, Hr] or NULL.
+ * To pool a corpus slab by slab, pass each slab's pointers with offsets that
+ * are relative to the slab.  Supported: d, dr in {64, 128}; P in [1, 4096].
+ * Device flags: MSA_FLAG_OFFSETS for offsets that disagree with P, Ntok or C,
+ * MSA_FLAG_INDEX_OOB for a document longer than max_len (its chunks are skipped).
+ * ---------------------------------------------------------------------- */
+msa_status msa_pool(msa_dtype dt, const void* K, const void* V, const void* Kr,
+                    const int64_t* doc_tok_off, const int64_t* doc_chunk_off,
+                    int64_t D, int64_t Ntok, int64_t C, int Hkv, int d, int Hr, int dr, int P,
+                    const float* rope_cs, int max_len,
+                    void* Kbar, void* Vbar, void* Krbar, float* kr_rnorm,
+                    int32_t* err_flag, msa_stream_t stream);
+
+/* kr_rnorm[c, h] = 1 / max(||Krbar[c, h]||, 1e-12) for a bank built elsewhere.
+ * Krbar [C, Hr, dr] dtype dt; kr_rnorm fp32 [C, Hr].  dr in {64, 128}. */
+msa_status msa_bank_rnorm(msa_dtype dt, const void* Krbar, int64_t C, int Hr, int dr,
+                          float* kr_rnorm, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Steps 2 and 3: routing and top-k ("Architecture": cosine similarity,
+ * mean-pooled over heads, then token-wise max, then Top-k documents;
+ * "Inference Pipeline" stage 2).
+ *   s[b, t, c]       = (1/Hr) sum_h cos(Qr[b, t, h], Krbar[c, h])
+ *   doc_score[b, j]  = max over chunks c of document j, max over t < Tq, of s
+ *   topk_idx[b, :]   = the k documents with the largest doc_score, sorted by
+ *                      score descending, equal scores by lower index first.
+ *   Qr        [B, Tq, Hr, dr] dtype dt
+ *   Krbar     [C, Hr, dr] dtype dt;  kr_rnorm fp32 [C, Hr] (from msa_pool or
+ *             msa_bank_rnorm)
+ *   doc_chunk_off int64 [D+1] (a document with no chunks scores -inf)
+ *   doc_scores fp32 [B, D] or NULL;  topk_idx int32 [B, k];  topk_score fp32
+ *             [B, k] or NULL.
+ *   ws / ws_bytes  device scratch of at least msa_route_topk_workspace_size();
+ *             its contents need no initialisation and are not kept.
+ * Supported: dr in {64, 128}, Hr in [1, 8], 1 <= k <= min(D, 256).
+ * Device flags: MSA_FLAG_OFFSETS for decreasing offsets or doc_chunk_off[D] != C.
+ * ---------------------------------------------------------------------- */
+size_t msa_route_topk_workspace_size(int64_t B, int64_t D, int k);
+msa_status msa_route_topk(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr,
+                          const void* Krbar, const float* kr_rnorm,
+                          const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
+                          float* doc_scores, int32_t* topk_idx, float* topk_score,
+                          void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Step 4: context assembly ("Inference Pipeline" stage 2: load only the
+ * selected K̄ / V̄).  For query b, the chunks of documents topk_idx[b, 0..k-1]
+ * are copied in rank order (each document's chunks in ascending order) into
+ * rows [0, mem_len[b]) of Kmem / Vmem; rows past mem_len[b] are left untouched.
+ *   topk_idx int32 [B, k];  doc_chunk_off int64 [D+1]
+ *   Kbar, Vbar [C, Hkv, d] dtype dt;  Kmem, Vmem [B, Mmax, Hkv, d];  mem_len int32 [B]
+ * Device flags: MSA_FLAG_INDEX_OOB for a document index outside [0, D) or a
+ * chunk outside [0, C) (that document is skipped), MSA_FLAG_OVERFLOW when the
+ * selected chunks exceed Mmax (the rows that do not fit are dropped).
+ * ---------------------------------------------------------------------- */
+msa_status msa_gather(msa_dtype dt, const int32_t* topk_idx, int64_t B, int k,
+                      const int64_t* doc_chunk_off, int64_t D, int64_t C,
+                      const void* Kbar, const void* Vbar, int Hkv, int d, int Mmax,
+                      void* Kmem, void* Vmem, int32_t* mem_len,
+                      int32_t* err_flag, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Step 5: sparse attention ("MSA x Qwen3.5" card, "Architecture summary": the
+ * top-k chunks' K/V concatenated with the local KV in softmax attention).
+ * For batch b, q-head h (KV head g = h / (Hq / Hkv)) and query token i at local
+ * position pos_i = Lloc - Tq + i, the keys are memory rows [0, mem_len[b]) of
+ * Kmem/Vmem (all visible) followed by local rows [0, pos_i] of Kloc/Vloc:
+ *   O[b, i, h] = softmax_j(scale * q . k_j) v_j
+ *   lse[b, h, i] = log sum_j exp(scale * q . k_j)    (natural log, optional)
+ *   Q [B, Tq, Hq, d];  Kloc, Vloc [B, Lloc, Hkv, d];  Kmem, Vmem [B, Mmax, Hkv, d]
+ *   mem_len int32 [B] (each in [0, Mmax]);  O [B, Tq, Hq, d];  lse fp32 [B, Hq, Tq] or NULL
+ *   scale <= 0 means 1/sqrt(d).
+ * Requires Lloc >= Tq >= 1, Hq % Hkv == 0, d in {64, 128}.
+ * Device flags: MSA_FLAG_INDEX_OOB when a mem_len is outside [0, Mmax] (that
+ * batch row is computed with mem_len clamped into range).
+ * ---------------------------------------------------------------------- */
+size_t msa_sparse_attn_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Mmax);
+msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const void* Vloc,
+                           int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d,
+                           const void* Kmem, const void* Vmem, const int32_t* mem_len, int Mmax,
+                           float scale, void* O, float* lse,
+                           void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Steps 2-5 fused for one layer: route + top-k, then attention whose memory
+ * rows are read directly from Kbar / Vbar through the selected documents'
+ * chunk ranges (no gathered copy).  Arguments as in msa_route_topk and
+ * msa_sparse_attn; Mmax bounds the memory rows per query (selected chunks past
+ * it are dropped and flagged MSA_FLAG_OVERFLOW).  topk_idx is required (it is
+ * the layer's routing output); doc_scores, topk_score and lse may be NULL.
+ * ---------------------------------------------------------------------- */
+size_t msa_layer_forward_workspace_size(int64_t B, int64_t D, int k, int Tq, int Lloc,
+                                        int Hq, int Hkv, int d, int Mmax);
+msa_status msa_layer_forward(msa_dtype dt,
+                             const void* Qr, int Hr, int dr,
+                             const void* Krbar, const float* kr_rnorm,
+                             const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
+                             const void* Q, const void* Kloc, const void* Vloc,
+                             int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d,
+                             const void* Kbar, const void* Vbar, int Mmax, float scale,
+                             void* O, float* lse, int32_t* topk_idx, float* topk_score,
+                             float* doc_scores,
+                             void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSA_H_ */

@@ -1,0 +1,148 @@
+"""Python binding of the MSA memory-path library (include/msa.h) for B200.
+
+Argument marshalling only: every function takes caller-allocated torch tensors,
+checks that they are contiguous CUDA tensors of the right dtype, and passes raw
+pointers and sizes to the C ABI in libmsa.so on the current (or given) stream.
+All computation happens in the library's CUDA kernels; there is no fallback.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+
+F32, BF16 = 0, 1
+FLAG_INDEX_OOB, FLAG_OFFSETS, FLAG_TIMEOUT, FLAG_OVERFLOW = 1, 2, 4, 8
+DTYPES = {torch.float32: F32, torch.bfloat16: BF16}
+
+
+class MSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = _lib.load().msa_status_string(status).decode()
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = status
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype not in DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return DTYPES[t.dtype]
+
+
+def _p(t, dtype=None):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("the MSA library takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("the MSA library takes contiguous tensors")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _s(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _call(name: str, *args) -> None:
+    st = getattr(_lib.load(), name)(*args)
+    if st != 0:
+        raise MSAError(name, st)
+
+
+def version() -> str:
+    return _lib.load().msa_version().decode()
+
+
+def kernel_launch_count() -> int:
+    """Kernels the library has launched in this process (msa_kernel_launch_count)."""
+    return int(_lib.load().msa_kernel_launch_count())
+
+
+def rope_table(theta: float, d: int, max_len: int) -> torch.Tensor:
+    """Host fp32 [max_len, d/2, 2] table of (cos, sin) built in fp64 by the library."""
+    out = torch.empty((max_len, d // 2, 2), dtype=torch.float32)
+    _call("msa_rope_table_host", float(theta), d, max_len, out.data_ptr())
+    return out
+
+
+def chunk_offsets(doc_tok_off, P: int):
+    """Host int64 [D+1] chunk offsets for host int64 token offsets (msa_chunk_offsets_host)."""
+    import numpy as np
+    tok = np.ascontiguousarray(np.asarray(doc_tok_off, dtype=np.int64))
+    out = np.empty_like(tok)
+    _call("msa_chunk_offsets_host", tok.ctypes.data, len(tok) - 1, P, out.ctypes.data)
+    return out
+
+
+def pool(K, V, Kr, doc_tok_off, doc_chunk_off, P, rope_cs, Kbar, Vbar, Krbar, kr_rnorm=None,
+         err_flag=None, stream=None):
+    """Step 1: RoPE + chunk-mean pooling (msa_pool)."""
+    D = doc_tok_off.numel() - 1
+    _call("msa_pool", _dt(K), _p(K), _p(V, K.dtype), _p(Kr, K.dtype), _p(doc_tok_off, torch.int64),
+          _p(doc_chunk_off, torch.int64), D, K.shape[0], Kbar.shape[0], K.shape[1], K.shape[2],
+          Kr.shape[1], Kr.shape[2], P, _p(rope_cs, torch.float32), rope_cs.shape[0],
+          _p(Kbar, K.dtype), _p(Vbar, K.dtype), _p(Krbar, K.dtype), _p(kr_rnorm, torch.float32),
+          _p(err_flag, torch.int32), _s(stream))
+
+
+def bank_rnorm(Krbar, kr_rnorm, stream=None):
+    _call("msa_bank_rnorm", _dt(Krbar), _p(Krbar), Krbar.shape[0], Krbar.shape[1], Krbar.shape[2],
+          _p(kr_rnorm, torch.float32), _s(stream))
+
+
+def route_topk_workspace_size(B: int, D: int, k: int) -> int:
+    return _lib.load().msa_route_topk_workspace_size(B, D, k)
+
+
+def route_topk(Qr, Krbar, kr_rnorm, doc_chunk_off, k, topk_idx, ws, topk_score=None, doc_scores=None,
+               err_flag=None, stream=None):
+    """Steps 2+3: cosine routing and top-k (msa_route_topk).  Qr [B, Tq, Hr, dr]."""
+    B, Tq, Hr, dr = Qr.shape
+    _call("msa_route_topk", _dt(Qr), _p(Qr), B, Tq, Hr, dr, _p(Krbar, Qr.dtype), _p(kr_rnorm, torch.float32),
+          _p(doc_chunk_off, torch.int64), doc_chunk_off.numel() - 1, Krbar.shape[0], k,
+          _p(doc_scores, torch.float32), _p(topk_idx, torch.int32), _p(topk_score, torch.float32),
+          _p(ws), ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))
+
+
+def gather(topk_idx, doc_chunk_off, Kbar, Vbar, Kmem, Vmem, mem_len, err_flag=None, stream=None):
+    """Step 4: copy the selected documents' chunks (msa_gather).  Kmem [B, Mmax, Hkv, d]."""
+    B, k = topk_idx.shape
+    _call("msa_gather", _dt(Kbar), _p(topk_idx, torch.int32), B, k, _p(doc_chunk_off, torch.int64),
+          doc_chunk_off.numel() - 1, Kbar.shape[0], _p(Kbar), _p(Vbar, Kbar.dtype), Kbar.shape[1],
+          Kbar.shape[2], Kmem.shape[1], _p(Kmem, Kbar.dtype), _p(Vmem, Kbar.dtype),
+          _p(mem_len, torch.int32), _p(err_flag, torch.int32), _s(stream))
+
+
+def sparse_attn_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Mmax) -> int:
+    return _lib.load().msa_sparse_attn_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Mmax)
+
+
+def sparse_attn(Q, Kloc, Vloc, Kmem, Vmem, mem_len, O, lse=None, scale=0.0, ws=None, err_flag=None,
+                stream=None):
+    """Step 5: attention over [memory ++ causal local] (msa_sparse_attn).  Q [B, Tq, Hq, d]."""
+    B, Tq, Hq, d = Q.shape
+    _call("msa_sparse_attn", _dt(Q), _p(Q), _p(Kloc, Q.dtype), _p(Vloc, Q.dtype), B, Tq, Kloc.shape[1], Hq,
+          Kloc.shape[2], d, _p(Kmem, Q.dtype), _p(Vmem, Q.dtype), _p(mem_len, torch.int32), Kmem.shape[1],
+          float(scale), _p(O, Q.dtype), _p(lse, torch.float32), _p(ws),
+          0 if ws is None else ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))
+
+
+def layer_forward_workspace_size(B, D, k, Tq, Lloc, Hq, Hkv, d, Mmax) -> int:
+    return _lib.load().msa_layer_forward_workspace_size(B, D, k, Tq, Lloc, Hq, Hkv, d, Mmax)
+
+
+def layer_forward(Qr, Krbar, kr_rnorm, doc_chunk_off, k, Q, Kloc, Vloc, Kbar, Vbar, Mmax, O, topk_idx, ws,
+                  lse=None, topk_score=None, doc_scores=None, scale=0.0, err_flag=None, stream=None):
+    """Steps 2-5 fused (msa_layer_forward): memory rows read from the bank by index."""
+    B, Tq, Hr, dr = Qr.shape
+    Hq, d = Q.shape[2], Q.shape[3]
+    _call("msa_layer_forward", _dt(Qr), _p(Qr), Hr, dr, _p(Krbar, Qr.dtype), _p(kr_rnorm, torch.float32),
+          _p(doc_chunk_off, torch.int64), doc_chunk_off.numel() - 1, Krbar.shape[0], k,
+          _p(Q, Qr.dtype), _p(Kloc, Qr.dtype), _p(Vloc, Qr.dtype), B, Tq, Kloc.shape[1], Hq, Kloc.shape[2], d,
+          _p(Kbar, Qr.dtype), _p(Vbar, Qr.dtype), Mmax, float(scale), _p(O, Qr.dtype), _p(lse, torch.float32),
+          _p(topk_idx, torch.int32), _p(topk_score, torch.float32), _p(doc_scores, torch.float32),
+          _p(ws), ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))

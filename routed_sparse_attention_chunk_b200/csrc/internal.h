@@ -1,0 +1,99 @@
+// Launchers behind the C ABI (host side, C++ linkage).  Each returns the
+// cudaError_t of its launches; the entry points in api.cu validate first.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "msa.h"
+
+namespace msa {
+
+// Counts every kernel launch of the library (read by msa_kernel_launch_count).
+void count_launch(int n = 1);
+
+struct PoolArgs {
+  const void *K, *V, *Kr;
+  const int64_t *doc_tok_off, *doc_chunk_off;
+  int64_t D, Ntok, C;
+  int Hkv, d, Hr, dr, P;
+  const float* rope_cs;
+  int max_len;
+  void *Kbar, *Vbar, *Krbar;
+  float* kr_rnorm;
+  int32_t* err_flag;
+};
+cudaError_t launch_pool(msa_dtype dt, const PoolArgs& a, cudaStream_t s);
+cudaError_t launch_bank_rnorm(msa_dtype dt, const void* Krbar, int64_t C, int Hr, int dr,
+                              float* kr_rnorm, cudaStream_t s);
+
+struct RouteArgs {
+  const void* Qr;
+  int64_t B;
+  int Tq, Hr, dr;
+  const void* Krbar;
+  const float* kr_rnorm;
+  const int64_t* doc_chunk_off;
+  int64_t D, C;
+  uint32_t* doc_key;  // [B, D] ordered keys, zeroed by the launcher
+  int32_t* err_flag;
+};
+cudaError_t launch_route(msa_dtype dt, const RouteArgs& a, cudaStream_t s);
+
+// Top-k over ordered document keys [B, D]: writes idx / score (score may be null)
+// and optionally decodes every document score into doc_scores.
+struct TopkArgs {
+  const uint32_t* doc_key;
+  int64_t B, D;
+  int k;
+  uint64_t* cand;  // workspace [B, nslice, k]
+  int nslice;
+  int32_t* topk_idx;
+  float* topk_score;
+  float* doc_scores;
+};
+int topk_num_slices(int64_t D, int k);
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+
+struct GatherArgs {
+  const int32_t* topk_idx;
+  int64_t B;
+  int k;
+  const int64_t* doc_chunk_off;
+  int64_t D, C;
+  const void *Kbar, *Vbar;
+  int Hkv, d, Mmax;
+  void *Kmem, *Vmem;
+  int32_t* mem_len;
+  int32_t* err_flag;
+};
+cudaError_t launch_gather(msa_dtype dt, const GatherArgs& a, cudaStream_t s);
+
+// Memory rows come either from dense [B, Mmax, Hkv, d] tensors (Kmem/Vmem) or,
+// when row_map is set, from bank rows row_map[b, m] of Kbank/Vbank [C, Hkv, d].
+struct AttnArgs {
+  const void *Q, *Kloc, *Vloc;
+  int64_t B;
+  int Tq, Lloc, Hq, Hkv, d;
+  const void *Kmem, *Vmem;  // dense memory rows, or the bank when row_map != null
+  const int32_t* row_map;   // [B, Mmax] bank chunk per memory row, or null
+  const int32_t* mem_len;   // [B]
+  int Mmax;
+  float scale;
+  void* O;
+  float* lse;
+  void* ws;
+  size_t ws_bytes;
+  int32_t* err_flag;
+};
+size_t attn_workspace_size(msa_dtype dt, int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Mmax);
+cudaError_t launch_attn(msa_dtype dt, const AttnArgs& a, cudaStream_t s);
+
+// Bank chunk index of every memory row of the selected documents (the index
+// form of msa_gather, used by the fused layer).
+cudaError_t launch_row_map(const int32_t* topk_idx, int64_t B, int k, const int64_t* doc_chunk_off,
+                           int64_t D, int64_t C, int Mmax, int32_t* row_map, int32_t* mem_len,
+                           int32_t* err_flag, cudaStream_t s);
+
+}  // namespace msa

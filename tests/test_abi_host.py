@@ -1,0 +1,148 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point that include/msa.h declares, its host helpers agree with the
+oracle, and bad arguments are rejected before anything is launched.
+
+Every rejected call below has exactly one bad argument, and that argument is
+checked before any CUDA call in the entry point, so no device work is queued
+even when a GPU is present (the fake device pointers are never dereferenced).
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import routed_sparse_attention_chunk_b200 as msa
+from routed_sparse_attention_chunk_b200 import _lib
+from oracle import msa_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, -1, -2, -3
+FAKE = 0x10000  # 16-byte aligned, never dereferenced (validation fails first)
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "msa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_function():
+    lib = _lib.load()
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), f"libmsa.so does not export {n}"
+    assert set(names) == set(_lib.SIGNATURES), "binding signatures out of step with msa.h"
+
+
+def test_status_strings_and_version():
+    lib = _lib.load()
+    for st in (OK, INVALID, UNSUPPORTED, WORKSPACE, -4, 12345):
+        assert lib.msa_status_string(st)
+    assert re.fullmatch(rb"\d+\.\d+\.\d+", lib.msa_version())
+
+
+def test_rope_table_matches_oracle_angles():
+    t = msa.rope_table(1e6, 128, 600).numpy()
+    ang = O.rope_angles(np.arange(600), 128, 1e6)
+    np.testing.assert_allclose(t[..., 0], np.cos(ang).astype(np.float32), rtol=0, atol=1.2e-7)
+    np.testing.assert_allclose(t[..., 1], np.sin(ang).astype(np.float32), rtol=0, atol=1.2e-7)
+    lib = _lib.load()
+    buf = (ctypes.c_float * 8)()
+    assert lib.msa_rope_table_host(1e6, 3, 4, buf) == INVALID
+    assert lib.msa_rope_table_host(-1.0, 4, 1, buf) == INVALID
+    assert lib.msa_rope_table_host(1e6, 4, 0, buf) == INVALID
+
+
+def test_chunk_offsets_match_oracle():
+    off = np.array([0, 500, 1000, 1064, 1065, 1065, 1200], dtype=np.int64)
+    for P in (1, 7, 64, 4096):
+        assert np.array_equal(msa.chunk_offsets(off, P), O.chunk_offsets(off, P))
+    with pytest.raises(msa.MSAError):
+        msa.chunk_offsets(np.array([0, 5, 3]), 64)
+
+
+def _pool(**kw):
+    a = dict(dt=1, K=FAKE, V=FAKE, Kr=FAKE, tok=FAKE, chk=FAKE, D=4, Ntok=100, C=4, Hkv=8, d=128, Hr=8,
+             dr=128, P=64, rope=FAKE, max_len=64, Kb=FAKE, Vb=FAKE, Krb=FAKE, rn=None, flag=None)
+    a.update(kw)
+    return _lib.load().msa_pool(*a.values(), None)
+
+
+def test_pool_rejects_bad_arguments():
+    assert _pool(d=96) == UNSUPPORTED
+    assert _pool(dr=32) == UNSUPPORTED
+    assert _pool(P=0) == INVALID
+    assert _pool(P=5000) == UNSUPPORTED
+    assert _pool(K=None) == INVALID
+    assert _pool(V=FAKE + 8) == INVALID           # misaligned
+    assert _pool(dt=7) == INVALID
+    assert _pool(C=0, K=None) == OK                # nothing to do, nothing launched
+
+
+def _route(**kw):
+    a = dict(dt=1, Qr=FAKE, B=1, Tq=4, Hr=8, dr=128, Krb=FAKE, rn=FAKE, chk=FAKE, D=10, C=20, k=3,
+             ds=None, idx=FAKE, sc=None, ws=FAKE, wsb=1 << 20, flag=None)
+    a.update(kw)
+    return _lib.load().msa_route_topk(*a.values(), None)
+
+
+def test_route_rejects_bad_arguments():
+    assert _route(k=11) == INVALID          # k > D
+    assert _route(k=0) == INVALID
+    assert _route(Hr=9) == UNSUPPORTED
+    assert _route(dr=96) == UNSUPPORTED
+    assert _route(Tq=0) == INVALID
+    assert _route(idx=None) == INVALID
+    assert _route(Qr=FAKE + 2) == INVALID
+    assert _route(ws=None) == WORKSPACE
+    need = _lib.load().msa_route_topk_workspace_size(1, 10, 3)
+    assert need > 0 and _route(wsb=need - 1) == WORKSPACE
+    assert _route(B=0) == OK
+
+
+def _attn(**kw):
+    a = dict(dt=1, Q=FAKE, Kl=FAKE, Vl=FAKE, B=1, Tq=8, Lloc=8, Hq=32, Hkv=8, d=128, Km=FAKE, Vm=FAKE,
+             ml=FAKE, Mmax=16, scale=0.0, O=FAKE, lse=None, ws=FAKE, wsb=1 << 20, flag=None)
+    a.update(kw)
+    return _lib.load().msa_sparse_attn(*a.values(), None)
+
+
+def test_attention_rejects_bad_arguments():
+    assert _attn(Hq=30) == INVALID          # Hq % Hkv != 0
+    assert _attn(Lloc=4) == INVALID         # Lloc < Tq
+    assert _attn(d=80) == UNSUPPORTED
+    assert _attn(Mmax=-1) == INVALID
+    assert _attn(O=None) == INVALID
+    assert _attn(ml=None) == INVALID
+    assert _attn(Kl=FAKE + 4) == INVALID
+    assert _attn(B=0) == OK
+
+
+def test_gather_and_layer_reject_bad_arguments():
+    lib = _lib.load()
+    g = dict(dt=1, idx=FAKE, B=2, k=4, chk=FAKE, D=10, C=30, Kb=FAKE, Vb=FAKE, Hkv=8, d=128, Mmax=32,
+             Km=FAKE, Vm=FAKE, ml=FAKE, flag=None)
+    assert lib.msa_gather(*dict(g, d=100).values(), None) == UNSUPPORTED
+    assert lib.msa_gather(*dict(g, ml=None).values(), None) == INVALID
+    assert lib.msa_gather(*dict(g, Km=FAKE + 1).values(), None) == INVALID
+    need = lib.msa_layer_forward_workspace_size(1, 10, 3, 8, 8, 32, 8, 128, 24)
+    assert need > lib.msa_route_topk_workspace_size(1, 10, 3)
+    L = dict(dt=1, Qr=FAKE, Hr=8, dr=128, Krb=FAKE, rn=FAKE, chk=FAKE, D=10, C=20, k=3, Q=FAKE, Kl=FAKE,
+             Vl=FAKE, B=1, Tq=8, Lloc=8, Hq=32, Hkv=8, d=128, Kb=FAKE, Vb=FAKE, Mmax=24, scale=0.0, O=FAKE,
+             lse=None, idx=FAKE, sc=None, ds=None, ws=FAKE, wsb=need, flag=None)
+    assert lib.msa_layer_forward(*dict(L, wsb=need - 1).values(), None) == WORKSPACE
+    assert lib.msa_layer_forward(*dict(L, Hq=33).values(), None) == INVALID
+    assert lib.msa_layer_forward(*dict(L, k=0).values(), None) == INVALID
+    assert lib.msa_layer_forward(*dict(L, Kb=None).values(), None) == INVALID
+
+
+def test_binding_rejects_host_and_strided_tensors():
+    x = torch.zeros((4, 8, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        msa.bank_rnorm(x, torch.zeros((4, 8)))
+    with pytest.raises(TypeError):
+        msa._dt(torch.zeros(2, dtype=torch.float16))
