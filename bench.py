@@ -168,7 +168,7 @@ class MSAWorkload:
         B = cfg.B
         self.O = [torch.empty_like(L["Q"]) for L in self.layers]
         self.idx = [torch.empty((B, cfg.k), dtype=torch.int32, device=device) for _ in self.layers]
-        nws = msa.layer_forward_workspace_size(B, self.D, cfg.k, cfg.Tq, cfg.Lloc, cfg.Hq, cfg.Hkv, cfg.d, cfg.Mmax)
+        nws = msa.layer_forward_workspace_size(B, cfg.Tq, cfg.Lloc, cfg.Hq, cfg.Hkv, cfg.d, cfg.Hr, self.D, cfg.k, cfg.Mmax)
         self.ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=device)
 
     def input_tensors(self):
@@ -201,7 +201,7 @@ def breakdown(w: MSAWorkload, counts: dict, peaks: dict, reps: int = 10) -> dict
     msa, c, dev = w.msa, w.cfg, w.dev
     L = w.layers[0]
     B = c.B
-    ws = torch.empty(msa.route_topk_workspace_size(B, w.D, c.k), dtype=torch.uint8, device=dev)
+    ws = torch.empty(msa.route_topk_workspace_size(B, c.Tq, c.Hr, w.D, c.k), dtype=torch.uint8, device=dev)
     idx = torch.empty((B, c.k), dtype=torch.int32, device=dev)
     Km = torch.zeros((B, c.Mmax, c.Hkv, c.d), dtype=c.torch_dtype, device=dev)
     Vm = torch.zeros_like(Km)

@@ -13,8 +13,8 @@
  *   4. msa_gather       - copy the selected documents' pooled K/V chunks.
  *   5. msa_sparse_attn  - GQA softmax attention of the query tokens over
  *                         [selected memory rows ++ causal local KV].
- *   msa_layer_forward   - steps 2-5 fused: the attention reads the selected
- *                         chunks straight from the bank by index.
+ *   msa_layer_forward   - steps 2-5 in one call, with the gathered chunks kept
+ *                         in the caller's workspace.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -159,7 +159,7 @@ msa_status msa_bank_rnorm(msa_dtype dt, const void* Krbar, int64_t C, int Hr, in
  * Supported: dr in {64, 128}, Hr in [1, 8], 1 <= k <= min(D, 256).
  * Device flags: MSA_FLAG_OFFSETS for decreasing offsets or doc_chunk_off[D] != C.
  * ---------------------------------------------------------------------- */
-size_t msa_route_topk_workspace_size(int64_t B, int64_t D, int k);
+size_t msa_route_topk_workspace_size(int64_t B, int Tq, int Hr, int64_t D, int k);
 msa_status msa_route_topk(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr,
                           const void* Krbar, const float* kr_rnorm,
                           const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
@@ -206,15 +206,16 @@ msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const 
                            void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * Steps 2-5 fused for one layer: route + top-k, then attention whose memory
- * rows are read directly from Kbar / Vbar through the selected documents'
- * chunk ranges (no gathered copy).  Arguments as in msa_route_topk and
- * msa_sparse_attn; Mmax bounds the memory rows per query (selected chunks past
- * it are dropped and flagged MSA_FLAG_OVERFLOW).  topk_idx is required (it is
- * the layer's routing output); doc_scores, topk_score and lse may be NULL.
+ * Steps 2-5 for one layer in one call: route + top-k, the selected chunks
+ * copied into the workspace (the msa_gather kernel), then attention over them
+ * and the local KV.  Arguments as in msa_route_topk and msa_sparse_attn; Mmax
+ * bounds the memory rows per query (selected chunks past it are dropped and
+ * flagged MSA_FLAG_OVERFLOW).  topk_idx is required (it is the layer's routing
+ * output); doc_scores, topk_score and lse may be NULL.  The workspace size is
+ * computed for fp32 storage and so also covers bf16.
  * ---------------------------------------------------------------------- */
-size_t msa_layer_forward_workspace_size(int64_t B, int64_t D, int k, int Tq, int Lloc,
-                                        int Hq, int Hkv, int d, int Mmax);
+size_t msa_layer_forward_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d,
+                                        int Hr, int64_t D, int k, int Mmax);
 msa_status msa_layer_forward(msa_dtype dt,
                              const void* Qr, int Hr, int dr,
                              const void* Krbar, const float* kr_rnorm,

@@ -81,8 +81,7 @@ __global__ void __launch_bounds__(kNT) attn_generic_kernel(AttnArgs a) {
         int64_t off;
         const T *kp, *vp;
         if (kk < M) {
-          const int64_t ridx = a.row_map ? (int64_t)__ldg(a.row_map + b * a.Mmax + kk) : b * a.Mmax + kk;
-          off = (ridx * a.Hkv + g) * (int64_t)DH + col;
+          off = ((b * a.Mmax + kk) * a.Hkv + g) * (int64_t)DH + col;
           kp = Km; vp = Vm;
         } else {
           off = ((b * a.Lloc + (kk - M)) * a.Hkv + g) * (int64_t)DH + col;

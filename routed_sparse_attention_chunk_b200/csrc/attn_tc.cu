@@ -1,18 +1,397 @@
-// Tensor-core (tcgen05) attention for bf16: not built yet; every shape goes to
-// the CUDA-core kernel in attn.cu.
+// Step 5 of the MSA memory path on the 5th-generation tensor cores: softmax
+// attention of the query tokens over [selected memory rows ++ causal local rows]
+// ("MSA x Qwen3.5" model card, "Architecture summary"; "MSA: Memory Sparse
+// Attention" README, "Architecture").
+//
+// Flash-style forward, one CTA per (query block, KV head, batch row):
+//   * the CTA's 128 rows are the GQA group's G q-heads x (128 / G) tokens, so one
+//     K/V tile serves every head of the group;
+//   * key tiles of 128 rows: first the memory rows (all visible; rows past
+//     mem_len are masked), then the local rows up to the block's last causal
+//     position (bottom-right aligned: token i sits at Lloc - Tq + i);
+//   * S = Q K^T by tcgen05.mma into one of two TMEM buffers (the tensor core
+//     computes S_{j+1} while the softmax warps work on S_j), P = exp2(S - m) in
+//     bf16 written to shared memory in the swizzled K-major layout, and
+//     O += P V with V read MN-major straight from its TMA tile;
+//   * the running max is only moved (and O rescaled in TMEM) when it grows by
+//     more than 2^8, so most tiles skip the rescale; the final 1/l and the
+//     log-sum-exp use the same max, which keeps the result exact.
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..5 softmax / correction / output (one row per thread).
+// Every wait is bounded and ends the CTA with MSA_FLAG_TIMEOUT on expiry.
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
+#include "tma_host.h"
 
 namespace msa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kRows = 128;   // MMA M: query rows per CTA
+constexpr int kKeys = 128;   // keys per tile
+constexpr int kThreads = 192;
+constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr float kRescaleLog2 = 8.0f;  // move the running max only when it grows by more than this
+
+struct AttnTcParams {
+  const int32_t* mem_len;
+  int32_t* err_flag;
+  __nv_bfloat16* O;
+  float* lse;
+  int Tq, Lloc, Hq, Hkv, Mmax, G, TB, n_qblk;
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+template <int DH>
+struct ALayout {
+  static constexpr int kBoxes = DH / 64;
+  static constexpr int kQ = kRows * DH * 2;
+  static constexpr int kK = kKeys * DH * 2;
+  static constexpr int kStage = 2 * kK;  // K then V
+  static constexpr int kP = kRows * kKeys * 2;
+  static constexpr int kBar = 8 * 16;
+  static constexpr int kSmem = 1024 + kQ + 2 * kStage + kP + kBar;
+  static constexpr uint32_t kTmemCols = 512;  // S0, S1 (128 each), O (DH)
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for an MN-major operand in 128-byte swizzle
+// (rows of 128 bytes along N, consecutive K rows 128 bytes apart, groups of 8
+// K rows 1024 bytes apart, 64-wide N blocks `lbo` bytes apart).
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3fffu);
+  d |= (uint64_t)((lbo >> 4) & 0x3fffu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKm,
+               const __grid_constant__ CUtensorMap tmVm, const __grid_constant__ CUtensorMap tmKl,
+               const __grid_constant__ CUtensorMap tmVl, AttnTcParams p) {
+  using L = ALayout<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Qs = smem;
+  uint8_t* KV = Qs + L::kQ;                  // [2 stages][K, V]
+  uint8_t* Ps = KV + 2 * L::kStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Ps + L::kP);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* o_done = bars + 10;
+  uint64_t* drain = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // longest blocks first: block index 0 takes the last query block
+  const int qb = p.n_qblk - 1 - (int)blockIdx.x;
+  const int g = blockIdx.y;
+  const int b = blockIdx.z;
+  const int t0 = qb * p.TB;
+  const int tlast = min(t0 + p.TB, p.Tq) - 1;
+  int M = __ldg(p.mem_len + b);
+  if (M < 0 || M > p.Mmax) {
+    if (threadIdx.x == 0 && qb == 0 && g == 0) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
+    M = M < 0 ? 0 : p.Mmax;
+  }
+  const int NM = (M + kKeys - 1) / kKeys;                       // memory tiles
+  const int pos_last = p.Lloc - p.Tq + tlast;
+  const int T = NM + (pos_last + kKeys) / kKeys;                 // + local tiles up to pos_last
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS0 = tmem, tO = tmem + 2 * kKeys;
+  bool timed_out = false;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      mbar_arrive_expect_tx(q_full, L::kQ);
+      for (int hh = 0; hh < p.G; ++hh)
+#pragma unroll
+        for (int dc = 0; dc < L::kBoxes; ++dc)
+          tma_load_2d(Qs + dc * (kRows * 128) + hh * p.TB * 128, &tmQ, (g * p.G + hh) * DH + dc * 64,
+                      b * p.Tq + t0, q_full);
+      int j = 0;
+      for (; j < T; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1, kWaitPolls)) {
+          timed_out = true;
+          break;
+        }
+        uint8_t* Kd = KV + st * L::kStage;
+        uint8_t* Vd = Kd + L::kK;
+        mbar_arrive_expect_tx(&kv_full[st], L::kStage);
+        const bool mem = j < NM;
+        const CUtensorMap* mk = mem ? &tmKm : &tmKl;
+        const CUtensorMap* mv = mem ? &tmVm : &tmVl;
+        const int y = mem ? b * p.Mmax + j * kKeys : b * p.Lloc + (j - NM) * kKeys;
+#pragma unroll
+        for (int dc = 0; dc < L::kBoxes; ++dc) {
+          tma_load_2d(Kd + dc * (kKeys * 128), mk, g * DH + dc * 64, y, &kv_full[st]);
+          tma_load_2d(Vd + dc * (kKeys * 128), mv, g * DH + dc * 64, y, &kv_full[st]);
+        }
+      }
+      // drain the copies this thread issued
+      if (!mbar_wait(q_full, 0, kWaitPolls)) timed_out = true;
+      for (int st = 0; st < 2 && st < j; ++st) {
+        const int last = (j - 1 - st) / 2 * 2 + st;
+        if (!mbar_wait(&kv_full[st], (last >> 1) & 1, kWaitPolls)) timed_out = true;
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kRows, kKeys);
+      constexpr uint32_t idO = idesc_bf16_f32(kRows, DH, /*b_mn_major=*/true);
+      const uint32_t q0 = smem_u32(Qs), p0 = smem_u32(Ps);
+      auto issue_S = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(&kv_full[st], (j >> 1) & 1, kWaitPolls)) return false;
+        if (!mbar_wait(&s_free[st], ((j >> 1) & 1) ^ 1, kWaitPolls)) return false;
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(KV + st * L::kStage);
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const int box = k >> 2, kk = k & 3;
+          mma_bf16_ss(tS0 + st * kKeys, desc_k_sw128(q0 + box * kRows * 128 + kk * 32),
+                      desc_k_sw128(k0 + box * kKeys * 128 + kk * 32), idS, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[st]);
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, kWaitPolls) && issue_S(0);
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T && !issue_S(j + 1)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(p_full, j & 1, kWaitPolls)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(KV + (j & 1) * L::kStage + L::kK);
+#pragma unroll
+        for (int k = 0; k < kKeys / 16; ++k) {
+          const int box = k >> 2, kk = k & 3;
+          mma_bf16_ss(tO, desc_k_sw128(p0 + box * kRows * 128 + kk * 32),
+                      desc_mn_sw128(v0 + k * 16 * 128, kKeys * 128), idO, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(o_done);
+        mma_commit(&kv_empty[j & 1]);
+      }
+      if (!ok) timed_out = true;
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0, kWaitPolls)) timed_out = true;
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax
+    const int q = warp & 3;
+    const int r = q * 32 + lane;                      // this thread's row (TMEM lane)
+    const int hh = r / p.TB, tl = r - hh * p.TB;
+    const int t = t0 + tl;
+    const int pos = p.Lloc - p.Tq + t;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    float m_run = -INFINITY, l_run = 0.f;
+    uint8_t* prow = Ps + r * 128;
+    const int sw = r & 7;
+    for (int j = 0; j < T; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(&s_full[st], (j >> 1) & 1, kWaitPolls)) {
+        timed_out = true;
+        break;
+      }
+      tc_fence_after();
+      float s[kKeys];
+#pragma unroll
+      for (int c = 0; c < kKeys; c += 16) tmem_ld16(tmem + lane_off + st * kKeys + c, *reinterpret_cast<float(*)[16]>(&s[c]));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s_free[st]);
+      // mask and row max (log2 domain)
+      const bool memt = j < NM;
+      const int base = memt ? j * kKeys : (j - NM) * kKeys;
+      const int lim = memt ? M - base : pos - base + 1;  // keys [0, lim) of this tile are visible
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kKeys; ++c) {
+        s[c] = c < lim ? s[c] * p.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, s[c]);
+      }
+      // move the max (and rescale O) only when it grows by more than 2^8
+      const bool first = m_run == -INFINITY;
+      const bool grow = mt > m_run + kRescaleLog2;
+      float corr = 1.f;
+      if (grow) {
+        corr = first ? 0.f : fast_exp2(m_run - mt);
+        m_run = mt;
+      }
+      // P_{j-1}'s PV must be done before P_j overwrites the buffer (and before O is touched)
+      if (j > 0 && !mbar_wait(o_done, (j - 1) & 1, kWaitPolls)) {
+        timed_out = true;
+        break;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < DH; c += 16) {
+          float o[16];
+          tmem_ld16(tmem + lane_off + tO - tmem + c, o);
+          tmem_ld_wait();
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(o[i] * corr);
+          tmem_st16(tmem + lane_off + tO - tmem + c, w);
+        }
+        tmem_st_wait();
+      }
+      l_run *= corr;
+      float ls = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < kKeys; c0 += 8) {
+        float e[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          e[i] = fast_exp2(s[c0 + i] - m_run);
+          ls += e[i];
+        }
+        uint4 pk = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
+                              pack_bf16x2(e[6], e[7]));
+        const int box = c0 >> 6, chunk = (c0 & 63) >> 3;
+        *reinterpret_cast<uint4*>(prow + box * (kRows * 128) + ((chunk ^ sw) << 4)) = pk;
+      }
+      l_run += ls;
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // output: O / l, lse = (m + log2 l) ln 2
+    if (!timed_out && mbar_wait(o_done, (T - 1) & 1, kWaitPolls)) {
+      tc_fence_after();
+      const float inv = 1.f / l_run;
+      const bool rvalid = t < p.Tq;
+      __nv_bfloat16* orow = p.O + (((int64_t)b * p.Tq + t) * p.Hq + g * p.G + hh) * DH;
+#pragma unroll
+      for (int c = 0; c < DH; c += 16) {
+        float o[16];
+        tmem_ld16(tO + lane_off + c, o);
+        tmem_ld_wait();
+        if (rvalid) {
+          uint4 w0 = make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
+                                pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
+          uint4 w1 = make_uint4(pack_bf16x2(o[8] * inv, o[9] * inv), pack_bf16x2(o[10] * inv, o[11] * inv),
+                                pack_bf16x2(o[12] * inv, o[13] * inv), pack_bf16x2(o[14] * inv, o[15] * inv));
+          *reinterpret_cast<uint4*>(orow + c) = w0;
+          *reinterpret_cast<uint4*>(orow + c + 8) = w1;
+        }
+      }
+      if (rvalid && p.lse)
+        p.lse[((int64_t)b * p.Hq + g * p.G + hh) * p.Tq + t] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    } else {
+      timed_out = true;
+    }
+  }
+
+  if (timed_out) raise_flag(p.err_flag, MSA_FLAG_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+template <int DH>
+cudaError_t launch_dh(const AttnArgs& a, cudaStream_t s) {
+  using L = ALayout<DH>;
+  const int G = a.Hq / a.Hkv, TB = kRows / G;
+  CUtensorMap tq, tkm, tvm, tkl, tvl;
+  const uint64_t rowkv = (uint64_t)a.Hkv * DH * 2;
+  const int64_t mrows = a.B * (int64_t)(a.Mmax > 0 ? a.Mmax : 1);
+  if (!make_tmap_2d_bf16(&tq, a.Q, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB) ||
+      !make_tmap_2d_bf16(&tkm, a.Mmax > 0 ? a.Kmem : a.Kloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, kKeys) ||
+      !make_tmap_2d_bf16(&tvm, a.Mmax > 0 ? a.Vmem : a.Vloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, kKeys) ||
+      !make_tmap_2d_bf16(&tkl, a.Kloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKeys) ||
+      !make_tmap_2d_bf16(&tvl, a.Vloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKeys))
+    return cudaErrorInvalidValue;
+  AttnTcParams p;
+  p.mem_len = a.mem_len;
+  p.err_flag = a.err_flag;
+  p.O = reinterpret_cast<__nv_bfloat16*>(a.O);
+  p.lse = a.lse;
+  p.Tq = a.Tq;
+  p.Lloc = a.Lloc;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.Mmax = a.Mmax;
+  p.G = G;
+  p.TB = TB;
+  p.n_qblk = (a.Tq + TB - 1) / TB;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)p.n_qblk, (unsigned)a.Hkv, (unsigned)a.B);
+  count_launch();
+  attn_tc_kernel<DH><<<grid, kThreads, L::kSmem, s>>>(tq, tkm, tvm, tkl, tvl, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
 
 size_t attn_tc_workspace_size(msa_dtype, int64_t, int, int, int, int, int, int) { return 0; }
 
+// Shapes the tensor-core kernel takes: bf16, d = 128, dense memory rows, a GQA
+// group that divides the 128 rows into blocks of at least 8 tokens, and enough
+// query tokens to fill most of a block.
 cudaError_t launch_attn_tc(msa_dtype dt, const AttnArgs& a, cudaStream_t s, bool* handled) {
-  (void)dt;
-  (void)a;
-  (void)s;
   *handled = false;
-  return cudaSuccess;
+  if (dt != MSA_BF16 || a.d != 128) return cudaSuccess;
+  const int G = a.Hq / a.Hkv;
+  if (G < 1 || 128 % G != 0 || 128 / G < 8) return cudaSuccess;
+  if (a.Tq < 128 / G / 2 && a.Tq < 16) return cudaSuccess;
+  if (a.B > 65535 || a.Hkv > 65535) return cudaSuccess;
+  *handled = true;
+  return launch_dh<128>(a, s);
 }
 
 }  // namespace msa

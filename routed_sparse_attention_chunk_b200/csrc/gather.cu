@@ -34,17 +34,16 @@ __device__ __forceinline__ Sel selected(const int32_t* __restrict__ idx, const i
 }
 
 // grid (k, B): one CTA copies one selected document
-template <bool COPY>
-__global__ void gather_kernel(GatherArgs a, int row_vecs, int32_t* __restrict__ row_map) {
+__global__ void gather_kernel(GatherArgs a, int row_vecs) {
   const int64_t b = blockIdx.y;
   const int r = blockIdx.x;
   bool bad = false;
   int64_t start = 0;
   for (int q = 0; q < r; ++q) start += selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, a.k, q, &bad).n;
-  bool dummy = false;
-  const Sel me = selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, a.k, r, &dummy);
+  bool mine_bad = false;
+  const Sel me = selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, a.k, r, &mine_bad);
   if (threadIdx.x == 0) {
-    if (dummy) raise_flag(a.err_flag, MSA_FLAG_INDEX_OOB);
+    if (mine_bad) raise_flag(a.err_flag, MSA_FLAG_INDEX_OOB);
     if (r == a.k - 1) {
       const int64_t total = start + me.n;
       if (total > a.Mmax) raise_flag(a.err_flag, MSA_FLAG_OVERFLOW);
@@ -53,11 +52,6 @@ __global__ void gather_kernel(GatherArgs a, int row_vecs, int32_t* __restrict__ 
   }
   const int64_t n = min(me.n, max((int64_t)0, (int64_t)a.Mmax - start));
   if (n <= 0) return;
-  if (!COPY) {
-    for (int64_t i = threadIdx.x; i < n; i += blockDim.x)
-      row_map[b * a.Mmax + start + i] = (int32_t)(me.cs + i);
-    return;
-  }
   const uint4* Ks = reinterpret_cast<const uint4*>(a.Kbar) + me.cs * row_vecs;
   const uint4* Vs = reinterpret_cast<const uint4*>(a.Vbar) + me.cs * row_vecs;
   uint4* Kd = reinterpret_cast<uint4*>(a.Kmem) + (b * a.Mmax + start) * row_vecs;
@@ -76,26 +70,7 @@ cudaError_t launch_gather(msa_dtype dt, const GatherArgs& a, cudaStream_t s) {
   const int esz = dt == MSA_F32 ? 4 : 2;
   const int row_vecs = a.Hkv * a.d * esz / 16;
   count_launch();
-  gather_kernel<true><<<dim3(a.k, (unsigned)a.B), 256, 0, s>>>(a, row_vecs, nullptr);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_row_map(const int32_t* topk_idx, int64_t B, int k, const int64_t* doc_chunk_off,
-                           int64_t D, int64_t C, int Mmax, int32_t* row_map, int32_t* mem_len,
-                           int32_t* err_flag, cudaStream_t s) {
-  if (B <= 0) return cudaSuccess;
-  GatherArgs a{};
-  a.topk_idx = topk_idx;
-  a.B = B;
-  a.k = k;
-  a.doc_chunk_off = doc_chunk_off;
-  a.D = D;
-  a.C = C;
-  a.Mmax = Mmax;
-  a.mem_len = mem_len;
-  a.err_flag = err_flag;
-  count_launch();
-  gather_kernel<false><<<dim3(k, (unsigned)B), 128, 0, s>>>(a, 0, row_map);
+  gather_kernel<<<dim3(a.k, (unsigned)a.B), 256, 0, s>>>(a, row_vecs);
   return cudaGetLastError();
 }
 

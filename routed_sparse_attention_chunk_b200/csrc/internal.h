@@ -37,6 +37,7 @@ struct RouteArgs {
   const int64_t* doc_chunk_off;
   int64_t D, C;
   uint32_t* doc_key;  // [B, D] ordered keys, zeroed by the launcher
+  float* rq;          // workspace [B * Tq, Hr]: 1 / ||Qr|| per row and head
   int32_t* err_flag;
 };
 cudaError_t launch_route(msa_dtype dt, const RouteArgs& a, cudaStream_t s);
@@ -70,14 +71,12 @@ struct GatherArgs {
 };
 cudaError_t launch_gather(msa_dtype dt, const GatherArgs& a, cudaStream_t s);
 
-// Memory rows come either from dense [B, Mmax, Hkv, d] tensors (Kmem/Vmem) or,
-// when row_map is set, from bank rows row_map[b, m] of Kbank/Vbank [C, Hkv, d].
+// Memory rows are dense [B, Mmax, Hkv, d] tensors (Kmem/Vmem), rows [0, mem_len[b]) used.
 struct AttnArgs {
   const void *Q, *Kloc, *Vloc;
   int64_t B;
   int Tq, Lloc, Hq, Hkv, d;
-  const void *Kmem, *Vmem;  // dense memory rows, or the bank when row_map != null
-  const int32_t* row_map;   // [B, Mmax] bank chunk per memory row, or null
+  const void *Kmem, *Vmem;
   const int32_t* mem_len;   // [B]
   int Mmax;
   float scale;
@@ -89,11 +88,5 @@ struct AttnArgs {
 };
 size_t attn_workspace_size(msa_dtype dt, int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Mmax);
 cudaError_t launch_attn(msa_dtype dt, const AttnArgs& a, cudaStream_t s);
-
-// Bank chunk index of every memory row of the selected documents (the index
-// form of msa_gather, used by the fused layer).
-cudaError_t launch_row_map(const int32_t* topk_idx, int64_t B, int k, const int64_t* doc_chunk_off,
-                           int64_t D, int64_t C, int Mmax, int32_t* row_map, int32_t* mem_len,
-                           int32_t* err_flag, cudaStream_t s);
 
 }  // namespace msa

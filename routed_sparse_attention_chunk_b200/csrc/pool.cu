@@ -244,12 +244,11 @@ cudaError_t launch_bank_rnorm(msa_dtype dt, const void* Krbar, int64_t C, int Hr
   if (warps <= 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (warps * 32 + threads - 1) / threads;
+  count_launch();
   if (dt == MSA_F32)
-    count_launch();
     bank_rnorm_kernel<float><<<(unsigned)blocks, threads, 0, s>>>(
         reinterpret_cast<const float*>(Krbar), C, Hr, dr, kr_rnorm);
   else
-    count_launch();
     bank_rnorm_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, s>>>(
         reinterpret_cast<const __nv_bfloat16*>(Krbar), C, Hr, dr, kr_rnorm);
   return cudaGetLastError();

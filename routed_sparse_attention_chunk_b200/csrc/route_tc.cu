@@ -1,15 +1,335 @@
-// Tensor-core (tcgen05) routing scan for bf16 banks: not built yet; every
-// shape goes to the CUDA-core kernel in route.cu.
+// Step 2 of the MSA memory path on the 5th-generation tensor cores: the
+// routing scan of a bf16 bank.
+//
+// "MSA: Memory Sparse Attention" README, "Architecture": relevance is the
+// cosine similarity of Q_r with the chunk-pooled K̄_r, mean-pooled over router
+// heads, then the token-wise max; a document scores the max over its chunks.
+//
+//   S[c, r] = sum_h rk[c, h] rq[r, h] <K̄r[c, h], Qr[r, h]>        r = (b, t)
+//   doc_key[b, doc(c)] = max over t, c of S[c, (b, t)] / Hr
+//
+// Design.  One work item is a tile of 128 chunks (the MMA's M, one TMEM lane
+// per chunk) against a block of N query rows (the MMA's N).  For every router
+// head h the tile's K̄r[., h, :] and the block's Qr[., h, :] arrive by TMA
+// (128-byte swizzle), one tcgen05.mma chain (K = dr) writes the fp32 dot
+// products of that head into one of two TMEM accumulators, and the epilogue
+// warps fold rk * rq * dot into a register running sum while the tensor core
+// already works on the next head.  The per-head cosine weights are why the
+// heads cannot share one accumulator: the products stay exact (bf16 x bf16 in
+// fp32) and every scale is applied in fp32 afterwards.  After the last head the
+// epilogue takes the max over the block's tokens in registers, a segmented max
+// over the warp's chunks of one document, and one atomicMax per document
+// segment on an order-preserving key.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over work items):
+//   warp 0 lane 0  TMA producer (smem ring of STAGES head-slices)
+//   warp 1         TMEM allocator; lane 0 issues the MMAs
+//   warps 2..5     epilogue, one TMEM lane quarter each
+// Every mbarrier wait is bounded; on expiry the kernel raises MSA_FLAG_TIMEOUT,
+// drains its own copies and MMAs, frees TMEM and returns.
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
+#include "tma_host.h"
 
 namespace msa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileM = 128;
+constexpr int kThreads = 192;
+constexpr uint32_t kWaitPolls = 1u << 24;
+
+struct RouteTcParams {
+  const float* kr_rnorm;
+  const float* rq;  // [rows, Hr]
+  const int64_t* doc_chunk_off;
+  uint32_t* doc_key;
+  int32_t* err_flag;
+  int64_t D, C;
+  int rows, Tq, Hr;
+  int n_tiles, n_rb;
+  int64_t items;
+};
+
+template <int DR, int N>
+struct Layout {
+  static constexpr int kBoxes = DR / 64;                  // 64-element (128-byte) K boxes per head
+  static constexpr int kA = kTileM * DR * 2;              // K̄r slice of one head
+  static constexpr int kB = N * DR * 2;                   // Qr slice of one head
+  static constexpr int kStage = kA + kB;
+  static constexpr int kStages = (200 * 1024) / kStage > 6 ? 6 : (200 * 1024) / kStage;
+  static constexpr int kRq = 4 * 8 * N * 4;               // per epilogue warp: rq of the row block, Hr <= 8
+  static constexpr int kBar = 8 * (2 * kStages + 5) + 16;
+  static constexpr int kSmem = 1024 + kStages * kStage + kRq + kBar;
+  static constexpr uint32_t kTmemCols = 2 * N;            // two accumulators of N fp32 columns
+};
+
+// Segmented max over the warp's lanes (consecutive chunks) grouped by document,
+// then one atomicMax per document segment.
+__device__ __forceinline__ void doc_max_atomic(float v, int doc, int lane, uint32_t* keys) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float vo = __shfl_down_sync(0xffffffffu, v, o);
+    const int jo = __shfl_down_sync(0xffffffffu, doc, o);
+    if (lane + o < 32 && jo == doc) v = fmaxf(v, vo);
+  }
+  const int jp = __shfl_up_sync(0xffffffffu, doc, 1);
+  if (doc >= 0 && (lane == 0 || jp != doc)) atomicMax(keys + doc, float_to_key(v));
+}
+
+template <int DR, int N>
+__global__ void __launch_bounds__(kThreads, 1)
+route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                RouteTcParams p) {
+  using L = Layout<DR, N>;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  float* rq_s = reinterpret_cast<float*>(smem + S * L::kStage);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * L::kStage + L::kRq);
+  uint64_t* full = bars;              // [S]   TMA -> MMA
+  uint64_t* empty = bars + S;         // [S]   MMA -> TMA
+  uint64_t* accf = bars + 2 * S;      // [2]   MMA -> epilogue
+  uint64_t* acce = bars + 2 * S + 2;  // [2]   epilogue -> MMA
+  uint64_t* drain = bars + 2 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Hr = p.Hr;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accf[i], 1);
+      mbar_init(&acce[i], 128);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool timed_out = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmQ);
+      uint32_t it = 0;  // stage-fill counter
+      for (int64_t item = blockIdx.x; item < p.items && !timed_out; item += gridDim.x) {
+        const int tile = (int)(item / p.n_rb), rb = (int)(item % p.n_rb);
+        for (int h = 0; h < Hr; ++h, ++it) {
+          const uint32_t s = it % S, round = it / S;
+          if (!mbar_wait(&empty[s], (round & 1) ^ 1, kWaitPolls)) {
+            timed_out = true;
+            break;
+          }
+          uint8_t* A = stage_base + s * L::kStage;
+          uint8_t* Bq = A + L::kA;
+          mbar_arrive_expect_tx(&full[s], L::kStage);
+#pragma unroll
+          for (int j = 0; j < L::kBoxes; ++j) {
+            tma_load_2d(A + j * kTileM * 128, &tmK, h * DR + j * 64, tile * kTileM, &full[s]);
+            tma_load_2d(Bq + j * N * 128, &tmQ, h * DR + j * 64, rb * N, &full[s]);
+          }
+        }
+      }
+      // drain: every stage's last fill must have landed before the CTA leaves
+      const uint32_t fills = it;
+      for (uint32_t s = 0; s < (uint32_t)S && s < fills; ++s) {
+        const uint32_t last = (fills - 1 - s) / S * S + s;  // last fill index of stage s
+        if (!mbar_wait(&full[s], (last / S) & 1, kWaitPolls)) timed_out = true;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTileM, N);
+      uint32_t it = 0;
+      for (int64_t item = blockIdx.x; item < p.items && !timed_out; item += gridDim.x) {
+        for (int h = 0; h < Hr; ++h, ++it) {
+          const uint32_t s = it % S, round = it / S;
+          const uint32_t buf = it & 1, use = it >> 1;
+          if (!mbar_wait(&full[s], round & 1, kWaitPolls) || !mbar_wait(&acce[buf], (use & 1) ^ 1, kWaitPolls)) {
+            timed_out = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(stage_base + s * L::kStage);
+          const uint32_t b0 = a0 + L::kA;
+          const uint32_t d = tmem + buf * N;
+#pragma unroll
+          for (int k = 0; k < DR / 16; ++k) {
+            const int box = k >> 2, kk = k & 3;  // 4 K-steps of 16 per 128-byte row
+            const uint64_t ad = desc_k_sw128(a0 + box * kTileM * 128 + kk * 32);
+            const uint64_t bd = desc_k_sw128(b0 + box * N * 128 + kk * 32);
+            mma_bf16_ss(d, ad, bd, idesc, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&accf[buf]);
+        }
+      }
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0, kWaitPolls)) timed_out = true;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lanes [32q, 32q + 32) belong to this warp
+    float* rq_w = rq_s + q * 8 * N;  // this warp's private copy (no cross-warp barrier)
+    const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
+    const float invHr = 1.0f / (float)Hr;
+    uint32_t it = 0;
+    for (int64_t item = blockIdx.x; item < p.items && !timed_out; item += gridDim.x) {
+      const int tile = (int)(item / p.n_rb), rb = (int)(item % p.n_rb);
+      const int64_t c = (int64_t)tile * kTileM + q * 32 + lane;
+      const bool valid = c < p.C;
+      const int r0 = rb * N;
+      const int nvalid = min(N, p.rows - r0);
+      __syncwarp();
+      for (int i = lane; i < Hr * N; i += 32) {
+        const int h = i / N, col = i - h * N, r = r0 + col;
+        rq_w[i] = r < p.rows ? __ldg(p.rq + (int64_t)r * Hr + h) : 0.f;
+      }
+      __syncwarp();
+      const int doc = valid ? (int)owner_doc(p.doc_chunk_off, p.D, c) : -1;
+      float S_[N];
+#pragma unroll
+      for (int j = 0; j < N; ++j) S_[j] = 0.f;
+      for (int h = 0; h < Hr; ++h, ++it) {
+        const uint32_t buf = it & 1, use = it >> 1;
+        const float rk = valid ? __ldg(p.kr_rnorm + c * Hr + h) : 0.f;
+        if (!mbar_wait(&accf[buf], use & 1, kWaitPolls)) {
+          timed_out = true;
+          break;
+        }
+        tc_fence_after();
+        const float* rqh = rq_w + h * N;
+#pragma unroll
+        for (int j0 = 0; j0 < N; j0 += 32) {
+          float v0[16], v1[16];
+          tmem_ld16(lane_addr + buf * N + j0, v0);
+          tmem_ld16(lane_addr + buf * N + j0 + 16, v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            S_[j0 + i] = fmaf(v0[i], rk * rqh[j0 + i], S_[j0 + i]);
+            S_[j0 + 16 + i] = fmaf(v1[i], rk * rqh[j0 + 16 + i], S_[j0 + 16 + i]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&acce[buf]);
+      }
+      if (timed_out) break;
+      const int b_first = r0 / p.Tq, b_last = (r0 + nvalid - 1) / p.Tq;
+      if (b_first == b_last) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < N; ++j)
+          if (j < nvalid) m = fmaxf(m, S_[j]);
+        doc_max_atomic(m * invHr, doc, lane, p.doc_key + (int64_t)b_first * p.D);
+      } else {
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          if (j < nvalid) {
+            const int b = (r0 + j) / p.Tq;
+            doc_max_atomic(S_[j] * invHr, doc, lane, p.doc_key + (int64_t)b * p.D);
+          }
+        }
+      }
+    }
+  }
+
+  if (timed_out) raise_flag(p.err_flag, MSA_FLAG_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// rq[r, h] = 1 / max(||Qr[r, h]||, 1e-12): one warp per (row, head)
+template <int DR>
+__global__ void qnorm_kernel(const __nv_bfloat16* __restrict__ Qr, int64_t n, float* __restrict__ rq) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= n) return;
+  const __nv_bfloat16* x = Qr + w * DR;
+  float ss = 0.f;
+#pragma unroll
+  for (int i = lane; i < DR; i += 32) {
+    const float v = __bfloat162float(x[i]);
+    ss += v * v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) rq[w] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
+}
+
+template <int DR, int N>
+cudaError_t launch_t(const RouteArgs& a, cudaStream_t s) {
+  using L = Layout<DR, N>;
+  const int rows = (int)(a.B * a.Tq);
+  CUtensorMap tmK, tmQ;
+  if (!make_tmap_2d_bf16(&tmK, a.Krbar, (uint64_t)a.Hr * DR, (uint64_t)a.C, (uint64_t)a.Hr * DR * 2, 64, kTileM) ||
+      !make_tmap_2d_bf16(&tmQ, a.Qr, (uint64_t)a.Hr * DR, (uint64_t)rows, (uint64_t)a.Hr * DR * 2, 64, N))
+    return cudaErrorInvalidValue;
+  {
+    const int64_t n = (int64_t)rows * a.Hr;
+    const int64_t blocks = (n * 32 + 255) / 256;
+    count_launch();
+    qnorm_kernel<DR><<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(a.Qr), n, a.rq);
+  }
+  RouteTcParams p;
+  p.kr_rnorm = a.kr_rnorm;
+  p.rq = a.rq;
+  p.doc_chunk_off = a.doc_chunk_off;
+  p.doc_key = a.doc_key;
+  p.err_flag = a.err_flag;
+  p.D = a.D;
+  p.C = a.C;
+  p.rows = rows;
+  p.Tq = a.Tq;
+  p.Hr = a.Hr;
+  p.n_tiles = (int)((a.C + kTileM - 1) / kTileM);
+  p.n_rb = (rows + N - 1) / N;
+  p.items = (int64_t)p.n_tiles * p.n_rb;
+  if (p.items == 0) return cudaGetLastError();
+  cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<DR, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = p.items < sm_count() ? p.items : sm_count();
+  count_launch();
+  route_tc_kernel<DR, N><<<(unsigned)grid, kThreads, L::kSmem, s>>>(tmK, tmQ, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
 
 cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s, bool* handled) {
-  (void)a;
-  (void)s;
   *handled = false;
-  return cudaSuccess;
+  if (a.Hr < 1 || a.Hr > 8 || (a.dr != 64 && a.dr != 128) || a.C < 1) return cudaSuccess;
+  if (a.C > 0x7fffffffLL - kTileM || a.B * a.Tq > 0x7fffffffLL) return cudaSuccess;
+  // the TMA maps need 16-byte aligned bases (checked by the entry point)
+  const int64_t rows = a.B * a.Tq;
+  cudaError_t e;
+  if (a.dr == 128)
+    e = rows <= 64 ? launch_t<128, 64>(a, s) : launch_t<128, 128>(a, s);
+  else
+    e = rows <= 64 ? launch_t<64, 64>(a, s) : launch_t<64, 128>(a, s);
+  *handled = true;
+  return e;
 }
 
 }  // namespace msa
