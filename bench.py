@@ -144,6 +144,13 @@ def traffic_record(kernel_file: str):
     return r
 
 
+def workload_config(args) -> synth.Config:
+    cfg = synth.get_config(args.workload)
+    if args.docs:
+        cfg = cfg.scaled(D=args.docs, last_len=None, docs_per_slab=0)
+    return cfg
+
+
 # ----------------------------------------------------------------------------- GPU arm
 class MSAWorkload:
     """Device buffers of one workload and its step (pool + every layer's fused forward)."""
@@ -252,7 +259,7 @@ def run_gpu(args, rank, local_rank, world):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     import routed_sparse_attention_chunk_b200 as msa
-    cfg = synth.get_config(args.workload)
+    cfg = workload_config(args)
     peaks, peak_kind = load_peaks()
     counts = workload_counts(cfg)
     w = MSAWorkload(cfg, device, seed=1000 * rank)
@@ -416,7 +423,7 @@ def run_reference(args, rank, world):
     """The oracle arm: --steps K timed steps of a bounded sample, rank 0 only."""
     if rank != 0:
         return None
-    cfg = synth.get_config(args.workload)
+    cfg = workload_config(args)
     per_step = max(0.2, min(10.0, args.ref_budget / max(1, args.steps + args.warmup)))
     docs, tokens = 2, 4
     _, _, wall = oracle_step_sample(cfg, docs, tokens)          # calibration (counts as warm-up)
@@ -450,6 +457,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="1m", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--docs", type=int, default=0, help="use only this many documents (smaller profiling case)")
     ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")

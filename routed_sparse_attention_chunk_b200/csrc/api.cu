@@ -134,7 +134,7 @@ msa_status msa_pool(msa_dtype dt, const void* K, const void* V, const void* Kr, 
     return MSA_ERR_INVALID_ARG;
   // one CTA thread per 16-byte column vector must fit in a block
   const int vn = dt == MSA_F32 ? 4 : 8;
-  if (Hkv * (d / 2) / vn + Hkv * d / vn + Hr * dr / vn > 1024) return MSA_ERR_UNSUPPORTED;
+  if (Hkv * (d / 2) / vn + Hkv * d / vn + Hr * dr / vn > 480) return MSA_ERR_UNSUPPORTED;
   PoolArgs a{K, V, Kr, doc_tok_off, doc_chunk_off, D, Ntok, C, Hkv, d, Hr, dr, P, rope_cs, max_len,
              Kbar, Vbar, Krbar, kr_rnorm, err_flag};
   return cuda_status(launch_pool(dt, a, reinterpret_cast<cudaStream_t>(stream)));

@@ -237,7 +237,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int sw = r & 7;
     for (int j = 0; j < T; ++j) {
       const int st = j & 1;
-      if (!mbar_wait(&s_full[st], (j >> 1) & 1, kWaitPolls)) {
+      // waits are decided warp-wide so the warp-collective tcgen05 ops are never split
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1, kWaitPolls))) {
         timed_out = true;
         break;
       }
@@ -267,7 +268,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         m_run = mt;
       }
       // P_{j-1}'s PV must be done before P_j overwrites the buffer (and before O is touched)
-      if (j > 0 && !mbar_wait(o_done, (j - 1) & 1, kWaitPolls)) {
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, kWaitPolls))) {
         timed_out = true;
         break;
       }
@@ -276,12 +277,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int c = 0; c < DH; c += 16) {
           float o[16];
-          tmem_ld16(tmem + lane_off + tO - tmem + c, o);
+          tmem_ld16(tO + lane_off + c, o);
           tmem_ld_wait();
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(o[i] * corr);
-          tmem_st16(tmem + lane_off + tO - tmem + c, w);
+          tmem_st16(tO + lane_off + c, w);
         }
         tmem_st_wait();
       }
@@ -306,7 +307,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_arrive(p_full);
     }
     // output: O / l, lse = (m + log2 l) ln 2
-    if (!timed_out && mbar_wait(o_done, (T - 1) & 1, kWaitPolls)) {
+    if (!timed_out && __all_sync(0xffffffffu, mbar_wait(o_done, (T - 1) & 1, kWaitPolls))) {
       tc_fence_after();
       const float inv = 1.f / l_run;
       const bool rvalid = t < p.Tq;

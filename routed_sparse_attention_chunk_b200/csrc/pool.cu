@@ -5,191 +5,222 @@
 // K / V / K_r are chunk-mean pooled) and "Inference Pipeline" stage 1 (cache the
 // chunk-pooled K̄, V̄, K̄_r); Figure 2 caption (document-wise RoPE).
 //
-// The work is a pure HBM stream: every raw token is read once (16-byte vector
-// loads with the streaming cache hint), and 1/P of that volume is written.
-// One CTA pools one chunk; thread w owns one 16-byte column vector of the
-// token row (for K: one vector of the first half and its RoPE partner in the
-// second half) and, when the CTA has several token groups, every TS-th token.
+// The work is a pure HBM stream: every raw token is read once and 1/P of that
+// volume is written.  Persistent CTAs (one per SM) walk their chunks in order.
+// One producer thread copies the token rows of K, V and Kr into a ring of
+// shared-memory stages with bulk asynchronous copies (cp.async.bulk, completion
+// counted on an mbarrier), running ahead across chunk boundaries; the consumer
+// threads each own one 16-byte column vector of the token row (a K vector of
+// the first half together with its RoPE partner in the second half, or one V /
+// Kr vector), sum it over the chunk's tokens in fp32 from shared memory, and at
+// the chunk's end store the mean rounded to the storage type.  The Kr threads
+// also reduce the squared norm of the stored (rounded) values per head with
+// warp shuffles, so kr_rnorm describes exactly the bank that routing reads.
+// Every wait is bounded: on expiry the kernel raises MSA_FLAG_TIMEOUT and leaves.
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
+#include "tma_host.h"
 
 namespace msa {
 namespace {
 
-constexpr int kPoolMaxThreads = 512;
-constexpr int kPoolUnroll = 4;
+using namespace sm100;
 
-template <typename T>
-__device__ __forceinline__ uint4 ld_stream(const T* p) {
-  return __ldcs(reinterpret_cast<const uint4*>(p));
+constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr int kRingBytes = 192 * 1024;
+
+struct PoolGeom {
+  int nK, nV, nR, W;      // consumer items: Kr vectors, K pairs, V vectors
+  int TOK, NS;            // tokens per stage, stages in the ring
+  int rowK, rowR;         // bytes of one token's K (or V) row and Kr row
+  int stage;              // bytes per stage
+};
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+struct ChunkSpan {
+  int64_t s, e, ts;  // token range [s, e) and the document's first token
+  int flag;          // 0: pool it; otherwise the flag bit to raise and skip
+};
+
+__device__ __forceinline__ ChunkSpan chunk_span(const PoolArgs& a, int64_t c) {
+  const int64_t j = owner_doc(a.doc_chunk_off, a.D, c);
+  const int64_t cs = __ldg(a.doc_chunk_off + j), ce = __ldg(a.doc_chunk_off + j + 1);
+  const int64_t ts = __ldg(a.doc_tok_off + j), te = __ldg(a.doc_tok_off + j + 1);
+  const int64_t L = te - ts;
+  ChunkSpan r{0, 0, ts, 0};
+  const bool ok = c >= cs && c < ce && ts >= 0 && L >= 0 && te <= a.Ntok && (ce - cs) == (L + a.P - 1) / a.P;
+  if (!ok) {
+    r.flag = MSA_FLAG_OFFSETS;
+  } else if (L > a.max_len) {
+    r.flag = MSA_FLAG_INDEX_OOB;
+  } else {
+    r.s = ts + (c - cs) * a.P;
+    r.e = min(r.s + (int64_t)a.P, te);
+  }
+  return r;
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kPoolMaxThreads)
-pool_kernel(PoolArgs a, int nK, int nV, int nR, int TS) {
+__global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
   constexpr int VN = Vec<T>::N;
-  extern __shared__ float smem[];
-  const int W = nK + nV + nR;
-  const int tid = threadIdx.x;
-  const int grp = tid / W;
-  const int item = tid - grp * W;
-  const bool active = grp < TS;
-  const int halfv = a.d / 2 / VN;
-  const int64_t rowK = (int64_t)a.Hkv * a.d, rowR = (int64_t)a.Hr * a.dr;
-  float* part = smem;                                      // [TS-1][W][2*VN]
-  float* npart = smem + (size_t)(TS - 1) * W * 2 * VN;     // [nR]
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + (size_t)g.NS * g.stage);
+  uint64_t* empty = full + g.NS;
+  const int nconsumer_warps = (g.W + 31) / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (blockIdx.x == 0 && tid == 0) {
-    if (__ldg(a.doc_chunk_off) != 0 || __ldg(a.doc_tok_off) != 0 ||
-        __ldg(a.doc_chunk_off + a.D) != a.C || __ldg(a.doc_tok_off + a.D) > a.Ntok)
-      raise_flag(a.err_flag, MSA_FLAG_OFFSETS);
-  }
-
-  for (int64_t c = blockIdx.x; c < a.C; c += gridDim.x) {
-    const int64_t j = owner_doc(a.doc_chunk_off, a.D, c);
-    const int64_t cs = __ldg(a.doc_chunk_off + j), ce = __ldg(a.doc_chunk_off + j + 1);
-    const int64_t ts = __ldg(a.doc_tok_off + j), te = __ldg(a.doc_tok_off + j + 1);
-    const int64_t L = te - ts;
-    const bool ok = c >= cs && c < ce && ts >= 0 && L >= 0 && te <= a.Ntok &&
-                    (ce - cs) == (L + a.P - 1) / a.P;
-    if (!ok || L > a.max_len) {  // block-uniform: depends on c only
-      if (tid == 0) raise_flag(a.err_flag, ok ? MSA_FLAG_INDEX_OOB : MSA_FLAG_OFFSETS);
-      continue;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < g.NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], nconsumer_warps);
     }
-    const int64_t s = ts + (c - cs) * a.P;
-    const int64_t e = min(s + (int64_t)a.P, te);
-    const int n = (int)(e - s);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  bool timed_out = false;
 
-    float acc[2 * VN];
-#pragma unroll
-    for (int i = 0; i < 2 * VN; ++i) acc[i] = 0.f;
-
-    if (active) {
-      if (item < nK) {
-        // K: vector i0.. of the first half of head h and its partner in the second half
-        const int h = item / halfv, i0 = (item - h * halfv) * VN;
-        const T* base = reinterpret_cast<const T*>(a.K) + h * a.d + i0;
-        const int half = a.d / 2;
-        for (int64_t t0 = s + grp; t0 < e; t0 += (int64_t)TS * kPoolUnroll) {
-          uint4 lo[kPoolUnroll], hi[kPoolUnroll];
-#pragma unroll
-          for (int u = 0; u < kPoolUnroll; ++u) {
-            const int64_t t = t0 + (int64_t)u * TS;
-            if (t < e) {
-              lo[u] = ld_stream(base + t * rowK);
-              hi[u] = ld_stream(base + t * rowK + half);
-            } else {
-              lo[u] = hi[u] = make_uint4(0, 0, 0, 0);
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < kPoolUnroll; ++u) {
-            const int64_t t = t0 + (int64_t)u * TS;
-            if (t < e) {
-              const int p = (int)(t - ts);  // position inside the document
-              const float4* cs4 =
-                  reinterpret_cast<const float4*>(a.rope_cs + ((size_t)p * half + i0) * 2);
-              float xl[VN], xh[VN];
-              unpack(lo[u], xl);
-              unpack(hi[u], xh);
-#pragma unroll
-              for (int q = 0; q < VN / 2; ++q) {
-                const float4 w = __ldg(cs4 + q);  // (cos, sin) of pairs 2q and 2q+1
-                const float c0 = w.x, s0 = w.y, c1 = w.z, s1 = w.w;
-                acc[2 * q] += xl[2 * q] * c0 - xh[2 * q] * s0;
-                acc[VN + 2 * q] += xh[2 * q] * c0 + xl[2 * q] * s0;
-                acc[2 * q + 1] += xl[2 * q + 1] * c1 - xh[2 * q + 1] * s1;
-                acc[VN + 2 * q + 1] += xh[2 * q + 1] * c1 + xl[2 * q + 1] * s1;
-              }
-            }
-          }
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      if (blockIdx.x == 0 && (__ldg(a.doc_chunk_off) != 0 || __ldg(a.doc_tok_off) != 0 ||
+                              __ldg(a.doc_chunk_off + a.D) != a.C || __ldg(a.doc_tok_off + a.D) > a.Ntok))
+        raise_flag(a.err_flag, MSA_FLAG_OFFSETS);
+      const uint8_t* K = reinterpret_cast<const uint8_t*>(a.K);
+      const uint8_t* V = reinterpret_cast<const uint8_t*>(a.V);
+      const uint8_t* R = reinterpret_cast<const uint8_t*>(a.Kr);
+      uint32_t it = 0;
+      for (int64_t c = blockIdx.x; c < a.C && !timed_out; c += gridDim.x) {
+        const ChunkSpan sp = chunk_span(a, c);
+        if (sp.flag) {
+          raise_flag(a.err_flag, sp.flag);
+          continue;
         }
-      } else {
-        // V or Kr: plain mean of one column vector
-        const bool isV = item < nK + nV;
-        const int w = isV ? item - nK : item - nK - nV;
-        const T* base = isV ? reinterpret_cast<const T*>(a.V) + (size_t)w * VN
-                            : reinterpret_cast<const T*>(a.Kr) + (size_t)w * VN;
-        const int64_t row = isV ? rowK : rowR;
-        for (int64_t t0 = s + grp; t0 < e; t0 += (int64_t)TS * kPoolUnroll) {
-          uint4 v[kPoolUnroll];
-#pragma unroll
-          for (int u = 0; u < kPoolUnroll; ++u) {
-            const int64_t t = t0 + (int64_t)u * TS;
-            v[u] = t < e ? ld_stream(base + t * row) : make_uint4(0, 0, 0, 0);
+        for (int64_t t0 = sp.s; t0 < sp.e; t0 += g.TOK, ++it) {
+          const uint32_t st = it % g.NS, round = it / g.NS;
+          if (!mbar_wait(&empty[st], (round & 1) ^ 1, kWaitPolls)) {
+            timed_out = true;
+            break;
           }
+          const int nt = (int)min((int64_t)g.TOK, sp.e - t0);
+          uint8_t* dst = ring + (size_t)st * g.stage;
+          const uint32_t bK = (uint32_t)nt * g.rowK, bR = (uint32_t)nt * g.rowR;
+          mbar_arrive_expect_tx(&full[st], 2 * bK + bR);
+          bulk_load(dst, K + t0 * g.rowK, bK, &full[st]);
+          bulk_load(dst + (size_t)g.TOK * g.rowK, V + t0 * g.rowK, bK, &full[st]);
+          bulk_load(dst + (size_t)2 * g.TOK * g.rowK, R + t0 * g.rowR, bR, &full[st]);
+        }
+      }
+      // every copy issued must have landed before the CTA leaves
+      const uint32_t fills = it;
+      for (uint32_t st = 0; st < (uint32_t)g.NS && st < fills; ++st) {
+        const uint32_t last = (fills - 1 - st) / g.NS * g.NS + st;
+        if (!mbar_wait(&full[st], (last / g.NS) & 1, kWaitPolls)) timed_out = true;
+      }
+    }
+  } else if (warp <= nconsumer_warps) {
+    // ---------------------------------------------------------------- consumers
+    const int item = threadIdx.x - 32;  // [0, nR) Kr, [nR, nR+nK) K pairs, then V; >= W idle
+    const int kind = item < g.nR ? 0 : (item < g.nR + g.nK ? 1 : (item < g.W ? 2 : 3));
+    const int half = a.d / 2, halfv = half / VN;
+    int off_lo = 0, off_hi = 0, region = 0, h = 0, i0 = 0;
+    if (kind == 0) {
+      region = 2 * g.TOK * g.rowK;
+      off_lo = item * 16;
+    } else if (kind == 1) {
+      const int w = item - g.nR;
+      h = w / halfv;
+      i0 = (w - h * halfv) * VN;
+      off_lo = (h * a.d + i0) * (int)sizeof(T);
+      off_hi = off_lo + half * (int)sizeof(T);
+    } else if (kind == 2) {
+      region = g.TOK * g.rowK;
+      off_lo = (item - g.nR - g.nK) * 16;
+    }
+    const int rstride = kind == 0 ? g.rowR : g.rowK;
+    const int G = a.dr / VN;  // Kr lanes per router head (a power of two <= 32)
+    uint32_t it = 0;
+    for (int64_t c = blockIdx.x; c < a.C && !timed_out; c += gridDim.x) {
+      const ChunkSpan sp = chunk_span(a, c);
+      if (sp.flag) continue;
+      float acc[2 * VN];
 #pragma unroll
-          for (int u = 0; u < kPoolUnroll; ++u) {
+      for (int i = 0; i < 2 * VN; ++i) acc[i] = 0.f;
+      for (int64_t t0 = sp.s; t0 < sp.e; t0 += g.TOK, ++it) {
+        const uint32_t st = it % g.NS, round = it / g.NS;
+        // the whole warp leaves together, so no warp-collective op below is split
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[st], round & 1, kWaitPolls))) {
+          timed_out = true;
+          break;
+        }
+        const int nt = (int)min((int64_t)g.TOK, sp.e - t0);
+        const uint8_t* base = ring + (size_t)st * g.stage + region;
+        if (kind == 1) {
+          for (int u = 0; u < nt; ++u) {
+            float xl[VN], xh[VN];
+            unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_lo), xl);
+            unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_hi), xh);
+            const int p = (int)(t0 + u - sp.ts);  // position inside the document
+            const float4* cs4 = reinterpret_cast<const float4*>(a.rope_cs + ((size_t)p * half + i0) * 2);
+#pragma unroll
+            for (int q = 0; q < VN / 2; ++q) {
+              const float4 w = __ldg(cs4 + q);  // (cos, sin) of pairs i0+2q and i0+2q+1
+              acc[2 * q] += xl[2 * q] * w.x - xh[2 * q] * w.y;
+              acc[VN + 2 * q] += xh[2 * q] * w.x + xl[2 * q] * w.y;
+              acc[2 * q + 1] += xl[2 * q + 1] * w.z - xh[2 * q + 1] * w.w;
+              acc[VN + 2 * q + 1] += xh[2 * q + 1] * w.z + xl[2 * q + 1] * w.w;
+            }
+          }
+        } else if (kind != 3) {
+          for (int u = 0; u < nt; ++u) {
             float x[VN];
-            unpack(v[u], x);
+            unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_lo), x);
 #pragma unroll
             for (int i = 0; i < VN; ++i) acc[i] += x[i];
           }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
       }
-    }
-
-    // combine the token groups
-    if (TS > 1) {
-      if (active && grp > 0) {
-        float* dst = part + ((size_t)(grp - 1) * W + item) * 2 * VN;
-#pragma unroll
-        for (int i = 0; i < 2 * VN; ++i) dst[i] = acc[i];
-      }
-      __syncthreads();
-      if (grp == 0) {
-        for (int g = 1; g < TS; ++g) {
-          const float* src = part + ((size_t)(g - 1) * W + item) * 2 * VN;
-#pragma unroll
-          for (int i = 0; i < 2 * VN; ++i) acc[i] += src[i];
-        }
-      }
-    }
-
-    // mean, round to the storage type, store; Kr threads keep their squared norm part
-    if (grp == 0) {
-      const float fn = (float)n;
-      float m[VN];
-      if (item < nK) {
-        const int h = item / halfv, i0 = (item - h * halfv) * VN;
-        T* dst = reinterpret_cast<T*>(a.Kbar) + c * rowK + h * a.d + i0;
-#pragma unroll
-        for (int i = 0; i < VN; ++i) m[i] = acc[i] / fn;
-        *reinterpret_cast<uint4*>(dst) = pack(m);
-#pragma unroll
-        for (int i = 0; i < VN; ++i) m[i] = acc[VN + i] / fn;
-        *reinterpret_cast<uint4*>(dst + a.d / 2) = pack(m);
-      } else if (item < nK + nV) {
-        T* dst = reinterpret_cast<T*>(a.Vbar) + c * rowK + (size_t)(item - nK) * VN;
-#pragma unroll
-        for (int i = 0; i < VN; ++i) m[i] = acc[i] / fn;
-        *reinterpret_cast<uint4*>(dst) = pack(m);
-      } else {
-        const int w = item - nK - nV;
-        T* dst = reinterpret_cast<T*>(a.Krbar) + c * rowR + (size_t)w * VN;
+      if (timed_out) break;
+      // mean, round to the storage type, store
+      const float fn = (float)(sp.e - sp.s);
+      float m[VN], ss = 0.f;
+      if (kind == 0) {
 #pragma unroll
         for (int i = 0; i < VN; ++i) m[i] = acc[i] / fn;
         const uint4 pk = pack(m);
-        *reinterpret_cast<uint4*>(dst) = pk;
-        float r[VN];
-        unpack(pk, r);  // the stored (rounded) values
-        float ss = 0.f;
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.Krbar) + c * g.rowR + off_lo) = pk;
+        unpack(pk, m);  // the stored values
 #pragma unroll
-        for (int i = 0; i < VN; ++i) ss += r[i] * r[i];
-        npart[w] = ss;
+        for (int i = 0; i < VN; ++i) ss += m[i] * m[i];
+      } else if (kind == 1) {
+        uint8_t* dst = reinterpret_cast<uint8_t*>(a.Kbar) + c * g.rowK;
+#pragma unroll
+        for (int i = 0; i < VN; ++i) m[i] = acc[i] / fn;
+        *reinterpret_cast<uint4*>(dst + off_lo) = pack(m);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) m[i] = acc[VN + i] / fn;
+        *reinterpret_cast<uint4*>(dst + off_hi) = pack(m);
+      } else if (kind == 2) {
+#pragma unroll
+        for (int i = 0; i < VN; ++i) m[i] = acc[i] / fn;
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.Vbar) + c * g.rowK + off_lo) = pack(m);
       }
+      // per-head squared norm of the stored Kr: groups of G lanes (every lane
+      // of the warp runs the shuffles; only Kr lanes use the result)
+      for (int o = G >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (kind == 0 && a.kr_rnorm && (item % G) == 0)
+        a.kr_rnorm[c * a.Hr + item / G] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
     }
-    if (a.kr_rnorm) {
-      __syncthreads();
-      const int per = a.dr / VN;
-      if (tid < a.Hr) {
-        float ss = 0.f;
-        for (int i = 0; i < per; ++i) ss += npart[tid * per + i];
-        a.kr_rnorm[c * a.Hr + tid] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-      }
-    }
-    __syncthreads();
   }
+  if (timed_out) raise_flag(a.err_flag, MSA_FLAG_TIMEOUT);
 }
 
 template <typename T>
@@ -213,22 +244,30 @@ __global__ void bank_rnorm_kernel(const T* __restrict__ Kb, int64_t C, int Hr, i
 template <typename T>
 cudaError_t pool_t(const PoolArgs& a, cudaStream_t s) {
   constexpr int VN = Vec<T>::N;
-  const int nK = a.Hkv * (a.d / 2) / VN, nV = a.Hkv * a.d / VN, nR = a.Hr * a.dr / VN;
-  const int W = nK + nV + nR;
-  int TS = kPoolMaxThreads / W;
-  TS = TS < 1 ? 1 : (TS > 4 ? 4 : TS);
-  if (TS > a.P) TS = a.P;
-  const int threads = ((W * TS + 31) / 32) * 32;
-  const size_t sm = ((size_t)(TS - 1) * W * 2 * VN + nR) * sizeof(float);
-  if (sm > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(pool_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sm);
-    if (e != cudaSuccess) return e;
-  }
+  PoolGeom g;
+  g.nK = a.Hkv * (a.d / 2) / VN;
+  g.nV = a.Hkv * a.d / VN;
+  g.nR = a.Hr * a.dr / VN;
+  g.W = g.nK + g.nV + g.nR;
+  g.rowK = a.Hkv * a.d * (int)sizeof(T);
+  g.rowR = a.Hr * a.dr * (int)sizeof(T);
+  const int row = 2 * g.rowK + g.rowR;
+  g.TOK = 8;
+  while (g.TOK > 1 && 2 * g.TOK * row > kRingBytes) g.TOK >>= 1;
+  if (g.TOK > a.P) g.TOK = a.P;
+  g.stage = ((g.TOK * row + 127) / 128) * 128;
+  g.NS = kRingBytes / g.stage;
+  if (g.NS > 16) g.NS = 16;
+  if (g.NS < 2) return cudaErrorInvalidValue;
+  const int threads = 32 + ((g.W + 31) / 32) * 32;
+  if (threads > 512) return cudaErrorInvalidValue;
+  const size_t sm = 128 + (size_t)g.NS * g.stage + 16 * (size_t)g.NS;
+  cudaError_t e = cudaFuncSetAttribute(pool_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
   if (a.C <= 0) return cudaSuccess;
-  const int64_t grid = a.C < 0x7fffffff ? a.C : 0x7fffffff;
+  const int64_t grid = a.C < sm_count() ? a.C : sm_count();
   count_launch();
-  pool_kernel<T><<<(unsigned)grid, threads, sm, s>>>(a, nK, nV, nR, TS);
+  pool_kernel<T><<<(unsigned)grid, threads, sm, s>>>(a, g);
   return cudaGetLastError();
 }
 

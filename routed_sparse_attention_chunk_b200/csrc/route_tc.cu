@@ -210,7 +210,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       for (int h = 0; h < Hr; ++h, ++it) {
         const uint32_t buf = it & 1, use = it >> 1;
         const float rk = valid ? __ldg(p.kr_rnorm + c * Hr + h) : 0.f;
-        if (!mbar_wait(&accf[buf], use & 1, kWaitPolls)) {
+        // the whole warp leaves together, so tcgen05.ld and the shuffles are never split
+        if (!__all_sync(0xffffffffu, mbar_wait(&accf[buf], use & 1, kWaitPolls))) {
           timed_out = true;
           break;
         }

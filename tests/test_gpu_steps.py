@@ -235,6 +235,22 @@ def test_attention_bf16(B, Tq, Lloc, Hq, Hkv, d, Mmax, mem_lens):
     close_abs(to64(lse), olse, 2e-3, "lse")
 
 
+@pytest.mark.parametrize("B,Tq,Lloc,Hq,Hkv,Mmax,mem_lens", [
+    (3, 100, 260, 32, 8, 160, [128, 0, 77]),      # G=4: ragged memory tiles, one row without memory
+    (1, 300, 300, 8, 8, 128, [128]),              # G=1 (MHA): 128 tokens per block
+    (2, 50, 400, 64, 8, 256, [256, 200]),         # G=8: 16 tokens per block, two memory tiles
+    (1, 1030, 1030, 32, 8, 128, [128]),           # many local tiles, a partial last block
+])
+def test_attention_bf16_tensor_core_tiling(B, Tq, Lloc, Hq, Hkv, Mmax, mem_lens):
+    Q, Kl, Vl, Km, Vm, ml = _attn_inputs(B, Tq, Lloc, Hq, Hkv, 128, Mmax, mem_lens, torch.bfloat16, 4)
+    Og, lse, flag = attn_on_gpu(Q, Kl, Vl, Km, Vm, ml)
+    Oo, olse = O.attention(to64(Q), to64(Kl), to64(Vl), to64(Km), to64(Vm), mem_lens)
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    close_abs(to64(Og), Oo, TOL_BF16_ABS, "O")
+    close_abs(to64(lse), olse, 2e-3, "lse")
+
+
 def test_attention_bad_mem_len_is_flagged_not_faulted():
     Q, Kl, Vl, Km, Vm, ml = _attn_inputs(1, 4, 4, 2, 1, 64, 8, [9999], torch.bfloat16, 3)
     Og, lse, flag = attn_on_gpu(Q, Kl, Vl, Km, Vm, ml)
