@@ -61,6 +61,7 @@ typedef enum {
   MSA_ERR_UNSUPPORTED = -2, /* a shape or dtype this build has no kernel for */
   MSA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than *_workspace_size */
   MSA_ERR_CUDA = -4,        /* a CUDA launch or runtime call failed */
+  MSA_ERR_TOO_LARGE = -5,   /* the problem needs more scratch than msa_route_topk_noalloc holds */
 } msa_status;
 
 /* Bits of the device-side error flag. */
@@ -165,6 +166,35 @@ msa_status msa_route_topk(msa_dtype dt, const void* Qr, int64_t B, int Tq, int H
                           const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
                           float* doc_scores, int32_t* topk_idx, float* topk_score,
                           void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * msa_route_topk without a caller workspace.  The pages have no counterpart
+ * to this entry point: it exists for callers that cannot allocate device
+ * memory when they call the library, such as a plugin whose host framework
+ * owns every byte of device memory, or a serving loop that must not allocate
+ * after start-up because an allocation can stall on the device or fail under
+ * memory pressure.
+ * It computes exactly what msa_route_topk computes (same arguments, minus
+ * ws / ws_bytes) and allocates nothing: its scratch is a fixed array of
+ * MSA_NOALLOC_SCRATCH_BYTES in the library's own device memory, which every
+ * GPU that loads the library holds until the process exits.
+ *   - Problems whose msa_route_topk_workspace_size() exceeds
+ *     MSA_NOALLOC_SCRATCH_BYTES return MSA_ERR_TOO_LARGE before any work is
+ *     queued (for Hr = 8 and Tq <= 64 that is roughly B * D <= 4 million).
+ *   - The first call on each device looks the array's device address up (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array, which keeps the previous call's
+ *     contents (the routine clears what must start at zero itself).  Calls
+ *     that overlap on the GPU, e.g. on two streams at once, race on the array
+ *     and must not be issued.
+ * ---------------------------------------------------------------------- */
+#define MSA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+msa_status msa_route_topk_noalloc(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr,
+                                  const void* Krbar, const float* kr_rnorm,
+                                  const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
+                                  float* doc_scores, int32_t* topk_idx, float* topk_score,
+                                  int32_t* err_flag, msa_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Step 4: context assembly ("Inference Pipeline" stage 2: load only the

@@ -108,6 +108,23 @@ def route_topk(Qr, Krbar, kr_rnorm, doc_chunk_off, k, topk_idx, ws, topk_score=N
           _p(ws), ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))
 
 
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024  # MSA_NOALLOC_SCRATCH_BYTES in msa.h
+
+
+def route_topk_noalloc(Qr, Krbar, kr_rnorm, doc_chunk_off, k, topk_idx, topk_score=None, doc_scores=None,
+                       err_flag=None, stream=None):
+    """msa_route_topk_noalloc: route_topk with the library's fixed scratch instead of a workspace.
+
+    For callers that cannot allocate device memory at call time.  Overlapping
+    calls on the GPU race on the shared scratch; see include/msa.h.
+    """
+    B, Tq, Hr, dr = Qr.shape
+    _call("msa_route_topk_noalloc", _dt(Qr), _p(Qr), B, Tq, Hr, dr, _p(Krbar, Qr.dtype),
+          _p(kr_rnorm, torch.float32), _p(doc_chunk_off, torch.int64), doc_chunk_off.numel() - 1,
+          Krbar.shape[0], k, _p(doc_scores, torch.float32), _p(topk_idx, torch.int32),
+          _p(topk_score, torch.float32), _p(err_flag, torch.int32), _s(stream))
+
+
 def gather(topk_idx, doc_chunk_off, Kbar, Vbar, Kmem, Vmem, mem_len, err_flag=None, stream=None):
     """Step 4: copy the selected documents' chunks (msa_gather).  Kmem [B, Mmax, Hkv, d]."""
     B, k = topk_idx.shape

@@ -26,6 +26,8 @@ SIGNATURES = {
     "msa_route_topk_workspace_size": (SZ, [I64, C.c_int, C.c_int, I64, C.c_int]),
     "msa_route_topk": (C.c_int, [C.c_int, P, I64, C.c_int, C.c_int, C.c_int, P, P, P, I64, I64, C.c_int,
                                  P, P, P, P, SZ, P, P]),
+    "msa_route_topk_noalloc": (C.c_int, [C.c_int, P, I64, C.c_int, C.c_int, C.c_int, P, P, P, I64, I64,
+                                         C.c_int, P, P, P, P, P]),
     "msa_gather": (C.c_int, [C.c_int, P, I64, C.c_int, P, I64, I64, P, P, C.c_int, C.c_int, C.c_int,
                              P, P, P, P, P]),
     "msa_sparse_attn_workspace_size": (SZ, [I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]),

@@ -86,6 +86,7 @@ const char* msa_status_string(int status) {
     case MSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case MSA_ERR_WORKSPACE: return "workspace missing or too small";
     case MSA_ERR_CUDA: return "CUDA launch or runtime error";
+    case MSA_ERR_TOO_LARGE: return "problem larger than the no-allocation entry point's fixed scratch";
     default: return "unknown status";
   }
 }
