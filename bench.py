@@ -20,7 +20,6 @@ import argparse
 import hashlib
 import json
 import os
-import subprocess
 import sys
 import time
 
@@ -89,57 +88,67 @@ def workload_counts(cfg: synth.Config) -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """SM clock and throttle-reason samples (NVML, every ~2 ms) while the timed region runs."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, device: torch.device):
-        self.proc = None
+        import threading
+        self.samples, self.max_mhz, self.err = [], None, None
+        self._stop = threading.Event()
         try:
+            import pynvml as nv
+            nv.nvmlInit()
             uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+            self._h = nv.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+            self._nv = nv
+        except Exception as e:  # no NVML: report that instead of clocks
+            self._nv, self.err = None, f"nvml unavailable: {type(e).__name__}"
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)))
+            except Exception:
+                pass
+            self._stop.wait(0.002)
+
+    def start(self):
+        if self._nv is not None:
+            self._t.start()
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        self.proc.terminate()
-        out, _ = self.proc.communicate(timeout=10)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 8:
-                continue
-            try:
-                sm.append(float(f[0]))
-                mx.append(float(f[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err], "samples": 0}
+        self._stop.set()
+        self._t.join(timeout=5)
+        mhz = [m for m, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        return {"sm_mhz": float(np.median(mhz)) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if bits & b], "samples": len(mhz)}
 
 
-def traffic_record(kernel_file: str):
-    """Per-launch DRAM bytes of the dominant kernel from a committed ncu summary,
-    or None when the kernel source changed since the counters were taken."""
+def traffic_record(kernel_file: str, workload: str):
+    """Per-launch DRAM bytes (read + write) of a kernel on a workload from the
+    committed ncu summary profiles/traffic.json, or None when the record is
+    missing or the kernel's source changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f)
+    r = rec.get(f"{kernel_file}:{workload}")
     src = os.path.join(ROOT, "routed_sparse_attention_chunk_b200", "csrc", kernel_file)
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    r = rec.get(kernel_file)
-    if not r or r.get("source_sha256_16") != h:
+    if not r or not os.path.exists(src):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != r.get("source_sha256_16"):
         return None
     return r
 
@@ -147,22 +156,31 @@ def traffic_record(kernel_file: str):
 def workload_config(args) -> synth.Config:
     cfg = synth.get_config(args.workload)
     if args.docs:
-        cfg = cfg.scaled(D=args.docs, last_len=None, docs_per_slab=0)
+        cfg = cfg.scaled(D=args.docs, last_len=None)
     return cfg
 
 
 # ----------------------------------------------------------------------------- GPU arm
 class MSAWorkload:
-    """Device buffers of one workload and its step (pool + every layer's fused forward)."""
+    """Device buffers of one workload and its step.
 
-    def __init__(self, cfg: synth.Config, device, seed: int):
+    step "full": msa_pool of every raw token (resident in HBM), then for every
+    layer msa_route_topk -> msa_gather -> msa_sparse_attn (the calls
+    msa_layer_forward makes).  step "query": the bank is pooled once at set-up,
+    slab by slab (a 100M-token corpus cannot be resident), and the step is the
+    per-layer query path only.
+    """
+
+    STAGES = ("pool", "route_topk", "gather", "sparse_attn")
+
+    def __init__(self, cfg: synth.Config, device, seed: int, step_kind: str):
         import routed_sparse_attention_chunk_b200 as msa
-        self.msa, self.cfg, self.dev = msa, cfg, device
+        self.msa, self.cfg, self.dev, self.kind = msa, cfg, device, step_kind
         dt = cfg.torch_dtype
         self.layers = [synth.gen_query(cfg, l, device, seed) for l in range(cfg.layers)]
-        self.K, self.V, self.Kr = synth.gen_raw_slab(cfg, 0, cfg.D, device, seed, Qr0=self.layers[0]["Qr"][0])
         tok = synth.doc_tok_offsets(cfg)
         coff = msa.chunk_offsets(tok, cfg.P)
+        self.tok, self.coff = tok, coff
         self.D, self.C = cfg.D, int(coff[-1])
         self.tok_d = torch.from_numpy(tok).to(device)
         self.coff_d = torch.from_numpy(coff).to(device)
@@ -172,14 +190,36 @@ class MSAWorkload:
         self.Krb = torch.empty((self.C, cfg.Hr, cfg.dr), dtype=dt, device=device)
         self.rn = torch.empty((self.C, cfg.Hr), dtype=torch.float32, device=device)
         self.flag = torch.zeros(1, dtype=torch.int32, device=device)
-        B = cfg.B
+        self.raw = None
+        if step_kind == "full":
+            self.raw = synth.gen_raw_slab(cfg, 0, cfg.D, device, seed, Qr0=self.layers[0]["Qr"][0])
+        else:
+            self._pool_slabs(seed)
+        B, c = cfg.B, cfg
         self.O = [torch.empty_like(L["Q"]) for L in self.layers]
-        self.idx = [torch.empty((B, cfg.k), dtype=torch.int32, device=device) for _ in self.layers]
-        nws = msa.layer_forward_workspace_size(B, cfg.Tq, cfg.Lloc, cfg.Hq, cfg.Hkv, cfg.d, cfg.Hr, self.D, cfg.k, cfg.Mmax)
-        self.ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=device)
+        self.idx = [torch.empty((B, c.k), dtype=torch.int32, device=device) for _ in self.layers]
+        self.rws = torch.empty(msa.route_topk_workspace_size(B, c.Tq, c.Hr, self.D, self.C, c.k), dtype=torch.uint8,
+                               device=device)
+        self.Km = torch.zeros((B, c.Mmax, c.Hkv, c.d), dtype=dt, device=device)
+        self.Vm = torch.zeros_like(self.Km)
+        self.ml = torch.zeros(B, dtype=torch.int32, device=device)
+        n = msa.sparse_attn_workspace_size(B, c.Tq, c.Lloc, c.Hq, c.Hkv, c.d, c.Mmax)
+        self.aws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+    def _pool_slabs(self, seed):
+        c, msa = self.cfg, self.msa
+        for lo, hi in synth.slab_bounds(c):
+            K, V, Kr = synth.gen_raw_slab(c, lo, hi, self.dev, seed, Qr0=self.layers[0]["Qr"][0])
+            t = torch.from_numpy(self.tok[lo:hi + 1] - self.tok[lo]).to(self.dev)
+            cs, ce = int(self.coff[lo]), int(self.coff[hi])
+            ch = torch.from_numpy(self.coff[lo:hi + 1] - self.coff[lo]).to(self.dev)
+            msa.pool(K, V, Kr, t, ch, c.P, self.rope, self.Kb[cs:ce], self.Vb[cs:ce], self.Krb[cs:ce],
+                     self.rn[cs:ce], self.flag)
+            del K, V, Kr
+        torch.cuda.synchronize()
 
     def input_tensors(self):
-        ts = [self.K, self.V, self.Kr]
+        ts = list(self.raw) if self.raw is not None else []
         for L in self.layers:
             ts += [L["Qr"], L["Q"], L["Kloc"], L["Vloc"]]
         return ts
@@ -187,68 +227,72 @@ class MSAWorkload:
     def output_tensors(self):
         return self.O + self.idx
 
+    # the stages of one step
     def pool(self):
         c = self.cfg
-        self.msa.pool(self.K, self.V, self.Kr, self.tok_d, self.coff_d, c.P, self.rope, self.Kb, self.Vb,
-                      self.Krb, self.rn, self.flag)
+        K, V, Kr = self.raw
+        self.msa.pool(K, V, Kr, self.tok_d, self.coff_d, c.P, self.rope, self.Kb, self.Vb, self.Krb, self.rn,
+                      self.flag)
 
-    def layers_forward(self):
-        c = self.cfg
-        for l, L in enumerate(self.layers):
-            self.msa.layer_forward(L["Qr"], self.Krb, self.rn, self.coff_d, c.k, L["Q"], L["Kloc"], L["Vloc"],
-                                   self.Kb, self.Vb, c.Mmax, self.O[l], self.idx[l], self.ws, err_flag=self.flag)
+    def route_topk(self, l):
+        self.msa.route_topk(self.layers[l]["Qr"], self.Krb, self.rn, self.coff_d, self.cfg.k, self.idx[l], self.rws,
+                            err_flag=self.flag)
 
-    def step(self):
-        self.pool()
-        self.layers_forward()
+    def gather(self, l):
+        self.msa.gather(self.idx[l], self.coff_d, self.Kb, self.Vb, self.Km, self.Vm, self.ml, self.flag)
+
+    def sparse_attn(self, l):
+        L = self.layers[l]
+        self.msa.sparse_attn(L["Q"], L["Kloc"], L["Vloc"], self.Km, self.Vm, self.ml, self.O[l], ws=self.aws,
+                             err_flag=self.flag)
+
+    def step(self, rec=None):
+        """One step; rec(stage) records an event after each stage when given."""
+        if self.kind == "full":
+            self.pool()
+            rec and rec("pool")
+        for l in range(self.cfg.layers):
+            self.route_topk(l)
+            rec and rec("route_topk")
+            self.gather(l)
+            rec and rec("gather")
+            self.sparse_attn(l)
+            rec and rec("sparse_attn")
 
 
-def breakdown(w: MSAWorkload, counts: dict, peaks: dict, reps: int = 10) -> dict:
-    """Per-step-kind times from the unfused entry points (outside the timed region)."""
-    msa, c, dev = w.msa, w.cfg, w.dev
-    L = w.layers[0]
-    B = c.B
-    ws = torch.empty(msa.route_topk_workspace_size(B, c.Tq, c.Hr, w.D, c.k), dtype=torch.uint8, device=dev)
-    idx = torch.empty((B, c.k), dtype=torch.int32, device=dev)
-    Km = torch.zeros((B, c.Mmax, c.Hkv, c.d), dtype=c.torch_dtype, device=dev)
-    Vm = torch.zeros_like(Km)
-    ml = torch.zeros(B, dtype=torch.int32, device=dev)
-    O = torch.empty_like(L["Q"])
-    aws_n = msa.sparse_attn_workspace_size(B, c.Tq, c.Lloc, c.Hq, c.Hkv, c.d, c.Mmax)
-    aws = torch.empty(max(aws_n, 256), dtype=torch.uint8, device=dev)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    fns = {
-        "pool": w.pool,
-        "route_topk": lambda: msa.route_topk(L["Qr"], w.Krb, w.rn, w.coff_d, c.k, idx, ws),
-        "gather": lambda: msa.gather(idx, w.coff_d, w.Kb, w.Vb, Km, Vm, ml),
-        "sparse_attn": lambda: msa.sparse_attn(L["Q"], L["Kloc"], L["Vloc"], Km, Vm, ml, O, ws=aws),
-    }
-    out = {}
-    for name, fn in fns.items():
-        fn()
-        ts = []
-        for _ in range(reps):
-            flush.fill_(1.0)  # cold L2 for every timed call
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1))
-        out[name] = {"ms": float(np.median(ts))}
+def stage_roofline(name: str, ms: float, cfg: synth.Config, counts: dict, peaks: dict, peak_kind: str,
+                   long_region: bool) -> dict:
+    """Roofline object of one stage from its live per-launch time."""
+    tfl = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    tfl_name = "bf16_tflops_sustained" if long_region else "bf16_tflops"
     hbm = peaks["hbm_gbs"]
-    tfl = peaks["bf16_tflops"]
-    out["pool"].update(gbs=counts["pool_bytes"] / out["pool"]["ms"] / 1e6)
-    out["pool"]["frac_hbm"] = out["pool"]["gbs"] / hbm
-    r = out["route_topk"]
-    r.update(scan_gbs=counts["route_bytes"] / r["ms"] / 1e6, tflops=counts["route_flops"] / r["ms"] / 1e9)
-    r["frac_hbm"] = r["scan_gbs"] / hbm
-    r["frac_tensor"] = r["tflops"] / tfl
-    a = out["sparse_attn"]
-    a.update(tflops=counts["attn_flops"] / c.layers / a["ms"] / 1e9)
-    a["frac_tensor"] = a["tflops"] / tfl
-    out["note"] = "unfused calls of layer 0, median of %d, L2 flushed before each" % reps
-    return out
+    esz = 4 if cfg.dtype == "f32" else 2
+    if name == "pool":
+        return {"bound": "hbm", "achieved": counts["pool_bytes"] / ms / 1e6, "peak": hbm, "unit": "GB/s",
+                "kernel": "pool_kernel (msa_pool)", "alg_bytes_per_launch": counts["pool_bytes"],
+                "peak_source": f"{peak_kind} hbm_gbs"}
+    if name == "route_topk":
+        inten = counts["route_flops"] / counts["route_bytes"]
+        if inten < tfl * 1e3 / hbm:
+            return {"bound": "hbm", "achieved": counts["route_bytes"] / ms / 1e6, "peak": hbm, "unit": "GB/s",
+                    "kernel": "msa_route_topk (query norms + tcgen05 scan + top-k)",
+                    "alg_bytes_per_launch": counts["route_bytes"], "peak_source": f"{peak_kind} hbm_gbs"}
+        return {"bound": "tensor", "achieved": counts["route_flops"] / ms / 1e9, "peak": tfl, "unit": "TFLOP/s",
+                "kernel": "msa_route_topk (query norms + tcgen05 scan + top-k)",
+                "alg_flops_per_launch": counts["route_flops"], "peak_source": f"{peak_kind} {tfl_name}"}
+    if name == "sparse_attn":
+        fl = counts["attn_flops"] / cfg.layers
+        if cfg.Tq == 1:  # decode: the local and memory KV stream
+            by = cfg.B * (cfg.Lloc + cfg.Mmax) * cfg.Hkv * cfg.d * esz * 2
+            return {"bound": "hbm", "achieved": by / ms / 1e6, "peak": hbm, "unit": "GB/s",
+                    "kernel": "msa_sparse_attn (decode)", "alg_bytes_per_launch": by,
+                    "peak_source": f"{peak_kind} hbm_gbs"}
+        return {"bound": "tensor", "achieved": fl / ms / 1e9, "peak": tfl, "unit": "TFLOP/s",
+                "kernel": "attn_tc_kernel (msa_sparse_attn)", "alg_flops_per_launch": fl,
+                "peak_source": f"{peak_kind} {tfl_name}"}
+    by = 2 * 2 * cfg.B * cfg.Mmax * cfg.Hkv * cfg.d * esz
+    return {"bound": "hbm", "achieved": by / ms / 1e6, "peak": hbm, "unit": "GB/s", "kernel": "gather_kernel",
+            "alg_bytes_per_launch": by, "peak_source": f"{peak_kind} hbm_gbs"}
 
 
 def run_gpu(args, rank, local_rank, world):
@@ -260,56 +304,76 @@ def run_gpu(args, rank, local_rank, world):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     import routed_sparse_attention_chunk_b200 as msa
     cfg = workload_config(args)
+    step_kind = args.step or ("query" if cfg.docs_per_slab else "full")
     peaks, peak_kind = load_peaks()
     counts = workload_counts(cfg)
-    w = MSAWorkload(cfg, device, seed=1000 * rank)
+    w = MSAWorkload(cfg, device, seed=1000 * rank, step_kind=step_kind)
     in_bytes = sum(t.numel() * t.element_size() for t in w.input_tensors())
+    if step_kind == "query":
+        in_bytes += w.Krb.numel() * w.Krb.element_size()  # the scan reads the whole bank every step
     flush = None if in_bytes > L2_BYTES else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
 
-    # ---- warm-up, then exactly K timed steps
+    # ---- warm-up, then exactly K timed steps, an event after every stage
     stream = torch.cuda.current_stream()
     sampler = ClockSampler(device)
     for _ in range(args.warmup):
         w.step()
     torch.cuda.synchronize()
     barrier(world, device)
+    sampler.start()
     n0 = msa.kernel_launch_count()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    marks = []  # (stage, event) in launch order
+
+    def rec(stage):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        marks.append((stage, e))
+
+    starts = []
     t_all0, t_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     t_all0.record(stream)
     for i in range(args.steps):
         if flush is not None:
             flush.fill_(1.0)
-        ev[i][0].record(stream)
-        w.pool()
-        ev[i][1].record(stream)
-        w.layers_forward()
-        ev[i][2].record(stream)
+        rec("start")
+        w.step(rec)
     t_all1.record(stream)
     torch.cuda.synchronize()
     launches = msa.kernel_launch_count() - n0
     clocks = sampler.stop()
-    pool_ms = [a.elapsed_time(b) for a, b, _ in ev]
-    layer_ms = [b.elapsed_time(c) for _, b, c in ev]
-    step_ms_local = float(np.sum(pool_ms) + np.sum(layer_ms)) if flush is not None else t_all0.elapsed_time(t_all1)
+    stage_ms = {s: [] for s in MSAWorkload.STAGES}
+    for (s0, e0), (s1, e1) in zip(marks[:-1], marks[1:]):
+        if s1 != "start":
+            stage_ms[s1].append(e0.elapsed_time(e1))
+    timed_ms = t_all0.elapsed_time(t_all1)
+    step_sum = sum(sum(v) for v in stage_ms.values())
+    step_ms_local = step_sum if flush is not None else timed_ms
     flag = int(w.flag.item())
     barrier(world, device)
     total_ms = max_over_ranks(step_ms_local, world, device)
     ms_per_step = total_ms / args.steps
-    tokens_per_step = cfg.B * cfg.Tq * world
+    tokens_per_step = cfg.B * cfg.Tq * cfg.layers * world if step_kind == "query" and cfg.layers > 1 \
+        else cfg.B * cfg.Tq * world
     value = tokens_per_step / (ms_per_step / 1e3)
 
-    # ---- dominant kernel roofline (pool: HBM stream)
-    pool_avg = float(np.mean(pool_ms))
-    achieved = counts["pool_bytes"] / (pool_avg / 1e3) / 1e9
-    tr = traffic_record("pool.cu")
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": tr["dram_bytes_per_launch"] * (counts["pool_bytes"] / tr["alg_bytes_per_launch"]) if tr else None,
-                "kernel": "pool_kernel (msa_pool)", "alg_bytes_per_launch": counts["pool_bytes"],
-                "avg_launch_ms": round(pool_avg, 4), "peak_source": f"{peak_kind} hbm_gbs (copy test)"}
+    # ---- roofline of the dominant stage (live per-launch times from the timed region)
+    per_launch = {s: float(np.mean(v)) for s, v in stage_ms.items() if v}
+    totals = {s: float(np.sum(v)) for s, v in stage_ms.items() if v}
+    dom = max(totals, key=totals.get)
+    long_region = timed_ms > 2000.0
+    roofline = stage_roofline(dom, per_launch[dom], cfg, counts, peaks, peak_kind, long_region)
+    roofline["achieved"] = round(roofline["achieved"], 2)
+    roofline["frac"] = round(roofline["achieved"] / roofline["peak"], 4)
+    roofline["avg_launch_ms"] = round(per_launch[dom], 4)
+    tr = traffic_record({"pool": "pool.cu", "route_topk": "route_tc.cu", "sparse_attn": "attn_tc.cu",
+                         "gather": "gather.cu"}[dom], cfg.name)
+    roofline["traffic"] = tr["dram_bytes_per_launch"] if tr else None
+    stages = {s: {"ms_per_launch": round(per_launch[s], 4), "share": round(totals[s] / step_sum, 4),
+                  **{k: (round(v, 2) if isinstance(v, float) else v)
+                     for k, v in stage_roofline(s, per_launch[s], cfg, counts, peaks, peak_kind, long_region).items()
+                     if k in ("bound", "achieved", "unit")}}
+              for s in per_launch}
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -336,7 +400,7 @@ def run_gpu(args, rank, local_rank, world):
         e2e = {"value": round(tokens_per_step / (e2e_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "steps": n_e2e}
 
-    bd = breakdown(w, counts, peaks) if (rank == 0 and not args.no_breakdown) else None
+    route_ms = per_launch.get("route_topk")
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -344,16 +408,18 @@ def run_gpu(args, rank, local_rank, world):
         "config": {"workload": f"{cfg.name}: {cfg.D} docs, {cfg.ntok} memory tokens, {cfg.C} chunks (P={cfg.P}), "
                                f"B={cfg.B} x Tq={cfg.Tq}, Lloc={cfg.Lloc}, Hq/Hkv/Hr={cfg.Hq}/{cfg.Hkv}/{cfg.Hr}, "
                                f"d={cfg.d}, k={cfg.k}, layers={cfg.layers}",
-                   "step": "msa_pool of every raw token + msa_layer_forward per layer",
+                   "step": ("msa_pool of every raw token, then per layer msa_route_topk, msa_gather, msa_sparse_attn"
+                            if step_kind == "full" else
+                            "per layer msa_route_topk, msa_gather, msa_sparse_attn over a bank pooled before timing"),
                    "l2": "inputs larger than L2" if flush is None else "L2 flushed between steps (not timed)",
-                   "parallelism": f"{world} independent replica(s)" if world > 1 else "single GPU"},
-        "route_scan_gbs": round(counts["route_bytes"] / (float(bd["route_topk"]["ms"]) / 1e3) / 1e9, 1) if bd else None,
+                   "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+        "route_scan_gbs": round(counts["route_bytes"] / (route_ms / 1e3) / 1e9, 1) if route_ms else None,
         "roofline": roofline,
+        "stages": stages,
         "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clocks,
         "err_flag": flag,
-        "breakdown": bd,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_budget)
@@ -454,14 +520,15 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="1m", choices=sorted(synth.CONFIGS))
     ap.add_argument("--docs", type=int, default=0, help="use only this many documents (smaller profiling case)")
     ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--step", choices=["full", "query"], default=None,
+                    help="full: pool + query path per step; query: bank pooled before timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)

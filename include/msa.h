@@ -160,7 +160,7 @@ msa_status msa_bank_rnorm(msa_dtype dt, const void* Krbar, int64_t C, int Hr, in
  * Supported: dr in {64, 128}, Hr in [1, 8], 1 <= k <= min(D, 256).
  * Device flags: MSA_FLAG_OFFSETS for decreasing offsets or doc_chunk_off[D] != C.
  * ---------------------------------------------------------------------- */
-size_t msa_route_topk_workspace_size(int64_t B, int Tq, int Hr, int64_t D, int k);
+size_t msa_route_topk_workspace_size(int64_t B, int Tq, int Hr, int64_t D, int64_t C, int k);
 msa_status msa_route_topk(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr,
                           const void* Krbar, const float* kr_rnorm,
                           const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
@@ -245,7 +245,7 @@ msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const 
  * computed for fp32 storage and so also covers bf16.
  * ---------------------------------------------------------------------- */
 size_t msa_layer_forward_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d,
-                                        int Hr, int64_t D, int k, int Mmax);
+                                        int Hr, int64_t D, int64_t C, int k, int Mmax);
 msa_status msa_layer_forward(msa_dtype dt,
                              const void* Qr, int Hr, int dr,
                              const void* Krbar, const float* kr_rnorm,

@@ -94,8 +94,8 @@ def bank_rnorm(Krbar, kr_rnorm, stream=None):
           _p(kr_rnorm, torch.float32), _s(stream))
 
 
-def route_topk_workspace_size(B: int, Tq: int, Hr: int, D: int, k: int) -> int:
-    return _lib.load().msa_route_topk_workspace_size(B, Tq, Hr, D, k)
+def route_topk_workspace_size(B: int, Tq: int, Hr: int, D: int, C: int, k: int) -> int:
+    return _lib.load().msa_route_topk_workspace_size(B, Tq, Hr, D, C, k)
 
 
 def route_topk(Qr, Krbar, kr_rnorm, doc_chunk_off, k, topk_idx, ws, topk_score=None, doc_scores=None,
@@ -148,8 +148,8 @@ def sparse_attn(Q, Kloc, Vloc, Kmem, Vmem, mem_len, O, lse=None, scale=0.0, ws=N
           0 if ws is None else ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))
 
 
-def layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, k, Mmax) -> int:
-    return _lib.load().msa_layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, k, Mmax)
+def layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax) -> int:
+    return _lib.load().msa_layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax)
 
 
 def layer_forward(Qr, Krbar, kr_rnorm, doc_chunk_off, k, Q, Kloc, Vloc, Kbar, Vbar, Mmax, O, topk_idx, ws,

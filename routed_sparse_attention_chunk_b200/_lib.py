@@ -23,7 +23,7 @@ SIGNATURES = {
     "msa_pool": (C.c_int, [C.c_int, P, P, P, P, P, I64, I64, I64, C.c_int, C.c_int, C.c_int, C.c_int,
                            C.c_int, P, C.c_int, P, P, P, P, P, P]),
     "msa_bank_rnorm": (C.c_int, [C.c_int, P, I64, C.c_int, C.c_int, P, P]),
-    "msa_route_topk_workspace_size": (SZ, [I64, C.c_int, C.c_int, I64, C.c_int]),
+    "msa_route_topk_workspace_size": (SZ, [I64, C.c_int, C.c_int, I64, I64, C.c_int]),
     "msa_route_topk": (C.c_int, [C.c_int, P, I64, C.c_int, C.c_int, C.c_int, P, P, P, I64, I64, C.c_int,
                                  P, P, P, P, SZ, P, P]),
     "msa_route_topk_noalloc": (C.c_int, [C.c_int, P, I64, C.c_int, C.c_int, C.c_int, P, P, P, I64, I64,
@@ -34,7 +34,7 @@ SIGNATURES = {
     "msa_sparse_attn": (C.c_int, [C.c_int, P, P, P, I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                   P, P, P, C.c_int, F32, P, P, P, SZ, P, P]),
     "msa_layer_forward_workspace_size": (SZ, [I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
-                                              I64, C.c_int, C.c_int]),
+                                              I64, I64, C.c_int, C.c_int]),
     "msa_layer_forward": (C.c_int, [C.c_int, P, C.c_int, C.c_int, P, P, P, I64, I64, C.c_int,
                                     P, P, P, I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                     P, P, C.c_int, F32, P, P, P, P, P, P, SZ, P, P]),

@@ -31,21 +31,24 @@ struct RouteWs {
   uint32_t* doc_key;
   uint64_t* cand;
   float* rq;
+  int32_t* chunk_doc;
   int nslice;
   size_t bytes;
 };
 
-RouteWs route_ws_layout(void* base, int64_t B, int Tq, int Hr, int64_t D, int k) {
+RouteWs route_ws_layout(void* base, int64_t B, int Tq, int Hr, int64_t D, int64_t C, int k) {
   RouteWs w{};
   w.nslice = topk_num_slices(D, k);
   const size_t keys = round_up(sizeof(uint32_t) * (size_t)B * (size_t)D, 256);
   const size_t cand = w.nslice > 1 ? round_up(sizeof(uint64_t) * (size_t)B * w.nslice * k, 256) : 0;
   const size_t rq = round_up(sizeof(float) * (size_t)B * (size_t)Tq * (size_t)Hr, 256);
-  w.bytes = keys + cand + rq;
+  const size_t cdoc = round_up(sizeof(int32_t) * (size_t)(C > 0 ? C : 1), 256);
+  w.bytes = keys + cand + rq + cdoc;
   if (base) {
     w.doc_key = reinterpret_cast<uint32_t*>(base);
     w.cand = cand ? reinterpret_cast<uint64_t*>(static_cast<char*>(base) + keys) : nullptr;
     w.rq = reinterpret_cast<float*>(static_cast<char*>(base) + keys + cand);
+    w.chunk_doc = reinterpret_cast<int32_t*>(static_cast<char*>(base) + keys + cand + rq);
   }
   return w;
 }
@@ -150,9 +153,9 @@ msa_status msa_bank_rnorm(msa_dtype dt, const void* Krbar, int64_t C, int Hr, in
   return cuda_status(launch_bank_rnorm(dt, Krbar, C, Hr, dr, kr_rnorm, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-size_t msa_route_topk_workspace_size(int64_t B, int Tq, int Hr, int64_t D, int k) {
-  if (B < 0 || Tq < 1 || Hr < 1 || D < 1 || k < 1) return 0;
-  return route_ws_layout(nullptr, B, Tq, Hr, D, k).bytes;
+size_t msa_route_topk_workspace_size(int64_t B, int Tq, int Hr, int64_t D, int64_t C, int k) {
+  if (B < 0 || Tq < 1 || Hr < 1 || D < 1 || C < 0 || k < 1) return 0;
+  return route_ws_layout(nullptr, B, Tq, Hr, D, C, k).bytes;
 }
 
 msa_status msa_route_topk(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr, const void* Krbar,
@@ -162,10 +165,10 @@ msa_status msa_route_topk(msa_dtype dt, const void* Qr, int64_t B, int Tq, int H
   msa_status st = check_route(dt, Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, k, topk_idx);
   if (st != MSA_OK) return st;
   if (B == 0) return MSA_OK;
-  RouteWs w = route_ws_layout(ws, B, Tq, Hr, D, k);
+  RouteWs w = route_ws_layout(ws, B, Tq, Hr, D, C, k);
   if (!ws || ws_bytes < w.bytes || !aligned16(ws)) return MSA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  RouteArgs ra{Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, w.doc_key, w.rq, err_flag};
+  RouteArgs ra{Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, w.doc_key, w.rq, w.chunk_doc, err_flag};
   cudaError_t e = launch_route(dt, ra, s);
   if (e != cudaSuccess) return MSA_ERR_CUDA;
   TopkArgs ta{w.doc_key, B, D, k, w.cand, w.nslice, topk_idx, topk_score, doc_scores};
@@ -207,9 +210,9 @@ msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const 
 }
 
 size_t msa_layer_forward_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Hr, int64_t D,
-                                        int k, int Mmax) {
-  if (B < 0 || Tq < 1 || Hr < 1 || D < 1 || k < 1 || Mmax < 0) return 0;
-  size_t n = route_ws_layout(nullptr, B, Tq, Hr, D, k).bytes;
+                                        int64_t C, int k, int Mmax) {
+  if (B < 0 || Tq < 1 || Hr < 1 || D < 1 || C < 0 || k < 1 || Mmax < 0) return 0;
+  size_t n = route_ws_layout(nullptr, B, Tq, Hr, D, C, k).bytes;
   // gathered memory rows (sized for fp32 storage, the larger type) and their counts
   n += 2 * round_up(sizeof(float) * (size_t)B * (size_t)Mmax * (size_t)Hkv * (size_t)d, 256);
   n += round_up(sizeof(int32_t) * (size_t)B, 256);
@@ -229,10 +232,10 @@ msa_status msa_layer_forward(msa_dtype dt, const void* Qr, int Hr, int dr, const
   if (st != MSA_OK) return st;
   if (B == 0) return MSA_OK;
   if (!O || !Kbar || !Vbar || !aligned16(O) || !aligned16(Kbar) || !aligned16(Vbar)) return MSA_ERR_INVALID_ARG;
-  const size_t need = msa_layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, k, Mmax);
+  const size_t need = msa_layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  RouteWs w = route_ws_layout(ws, B, Tq, Hr, D, k);
+  RouteWs w = route_ws_layout(ws, B, Tq, Hr, D, C, k);
   char* p = static_cast<char*>(ws) + w.bytes;
   const size_t mem_bytes = round_up(sizeof(float) * (size_t)B * (size_t)Mmax * (size_t)Hkv * (size_t)d, 256);
   void* Kmem = p;
@@ -243,7 +246,7 @@ msa_status msa_layer_forward(msa_dtype dt, const void* Qr, int Hr, int dr, const
   void* attn_ws = p;
   const size_t attn_ws_bytes = ws_bytes - (size_t)(p - static_cast<char*>(ws));
 
-  RouteArgs ra{Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, w.doc_key, w.rq, err_flag};
+  RouteArgs ra{Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, w.doc_key, w.rq, w.chunk_doc, err_flag};
   if (launch_route(dt, ra, s) != cudaSuccess) return MSA_ERR_CUDA;
   TopkArgs ta{w.doc_key, B, D, k, w.cand, w.nslice, topk_idx, topk_score, doc_scores};
   if (launch_topk(ta, s) != cudaSuccess) return MSA_ERR_CUDA;

@@ -83,4 +83,46 @@ __device__ __forceinline__ int64_t owner_doc(const int64_t* __restrict__ off, in
   return lo;
 }
 
+// owner_doc for a whole warp at once, with 32-way probes: every round each lane
+// tests one of 32 evenly spaced offsets and a ballot keeps the last range that
+// can still hold c, so ~log32(D) dependent loads instead of log2(D).  All 32
+// lanes must call it with the same c; all get the same answer.  Requires
+// off[0] <= c.
+__device__ __forceinline__ int64_t warp_owner_doc(const int64_t* __restrict__ off, int64_t D, int64_t c,
+                                                  int lane) {
+  int64_t lo = 0, hi = D;  // answer in [lo, hi), off[lo] <= c
+  while (hi - lo > 1) {
+    const int64_t step = (hi - lo + 31) / 32;
+    const int64_t pos = lo + (int64_t)lane * step;
+    const bool le = pos < hi && __ldg(off + pos) <= c;
+    const unsigned m = __ballot_sync(0xffffffffu, le);
+    const int last = 31 - __clz(m);
+    lo += (int64_t)last * step;
+    hi = min(hi, lo + step);
+  }
+  return lo;
+}
+
+// Owning document of chunk c0 + lane for the 32 consecutive chunks of a warp
+// (-1 for chunks >= C).  One warp-wide search for c0, then each lane counts the
+// document boundaries at or below its chunk among the next 32 (documents with no
+// chunks are boundaries too); falls back to a per-lane search when 32
+// boundaries do not cover the warp's chunks.  All 32 lanes must call it.
+__device__ __forceinline__ int warp_chunk_docs(const int64_t* __restrict__ off, int64_t D, int64_t C, int64_t c0,
+                                               int lane) {
+  if (c0 >= C) return -1;
+  const int64_t j0 = warp_owner_doc(off, D, c0, lane);
+  const int64_t c = c0 + lane;
+  const int64_t bidx = j0 + 1 + lane;
+  const int64_t b = __ldg(off + (bidx < D ? bidx : D));
+  int cnt = 0;
+#pragma unroll
+  for (int l = 0; l < 32; ++l) cnt += __shfl_sync(0xffffffffu, b, l) <= c ? 1 : 0;
+  const int64_t b31 = __shfl_sync(0xffffffffu, b, 31);
+  const bool covered = b31 > c0 + 31 || j0 + 32 >= D;
+  if (c >= C) return -1;
+  if (covered) return (int)(j0 + cnt);
+  return (int)owner_doc(off, D, c);
+}
+
 }  // namespace msa

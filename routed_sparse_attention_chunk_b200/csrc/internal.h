@@ -38,6 +38,7 @@ struct RouteArgs {
   int64_t D, C;
   uint32_t* doc_key;  // [B, D] ordered keys, zeroed by the launcher
   float* rq;          // workspace [B * Tq, Hr]: 1 / ||Qr|| per row and head
+  int32_t* chunk_doc; // workspace [C]: owning document of every chunk
   int32_t* err_flag;
 };
 cudaError_t launch_route(msa_dtype dt, const RouteArgs& a, cudaStream_t s);

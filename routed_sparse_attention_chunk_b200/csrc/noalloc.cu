@@ -53,9 +53,9 @@ extern "C" msa_status msa_route_topk_noalloc(msa_dtype dt, const void* Qr, int64
                                              const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
                                              float* doc_scores, int32_t* topk_idx, float* topk_score,
                                              int32_t* err_flag, msa_stream_t stream) {
-  if (B < 0 || Tq < 1 || Hr < 1 || D < 1 || k < 1) return MSA_ERR_INVALID_ARG;
+  if (B < 0 || Tq < 1 || Hr < 1 || D < 1 || C < 0 || k < 1) return MSA_ERR_INVALID_ARG;
   if (B == 0) return MSA_OK;
-  const size_t need = msa_route_topk_workspace_size(B, Tq, Hr, D, k);
+  const size_t need = msa_route_topk_workspace_size(B, Tq, Hr, D, C, k);
   if (need == 0 || need > kScratchBytes) return MSA_ERR_TOO_LARGE;
   void* ws = nullptr;
   const msa_status st = scratch_address(&ws);

@@ -6,13 +6,16 @@
 // chunk-pooled K̄, V̄, K̄_r); Figure 2 caption (document-wise RoPE).
 //
 // The work is a pure HBM stream: every raw token is read once and 1/P of that
-// volume is written.  Persistent CTAs (one per SM) walk their chunks in order.
-// One producer thread copies the token rows of K, V and Kr into a ring of
-// shared-memory stages with bulk asynchronous copies (cp.async.bulk, completion
-// counted on an mbarrier), running ahead across chunk boundaries; the consumer
+// volume is written.  Persistent CTAs (one per SM) each own a contiguous range
+// of chunks.  One producer thread follows the owning document incrementally
+// and copies the token rows of K, V and Kr into a ring of shared-memory stages
+// with bulk asynchronous copies (cp.async.bulk, completion counted on an
+// mbarrier), running ahead across chunk boundaries; a small per-stage record
+// tells the consumers which chunk the stage belongs to.  The consumer
 // threads each own one 16-byte column vector of the token row (a K vector of
 // the first half together with its RoPE partner in the second half, or one V /
-// Kr vector), sum it over the chunk's tokens in fp32 from shared memory, and at
+// Kr vector), sum it over the chunk's tokens in fp32 from shared memory (the
+// stage also carries the RoPE (cos, sin) rows of its token positions), and at
 // the chunk's end store the mean rounded to the storage type.  The Kr threads
 // also reduce the squared norm of the stored (rounded) values per head with
 // warp shuffles, so kr_rnorm describes exactly the bank that routing reads.
@@ -33,7 +36,7 @@ constexpr int kRingBytes = 192 * 1024;
 struct PoolGeom {
   int nK, nV, nR, W;      // consumer items: Kr vectors, K pairs, V vectors
   int TOK, NS;            // tokens per stage, stages in the ring
-  int rowK, rowR;         // bytes of one token's K (or V) row and Kr row
+  int rowK, rowR, rowP;   // bytes of one token's K (or V) row, Kr row, and RoPE (cos, sin) row
   int stage;              // bytes per stage
 };
 
@@ -43,28 +46,14 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
-struct ChunkSpan {
-  int64_t s, e, ts;  // token range [s, e) and the document's first token
-  int flag;          // 0: pool it; otherwise the flag bit to raise and skip
+// What the consumers need to know about one stage of the ring.
+struct StageMeta {
+  int64_t c;   // chunk the stage's tokens belong to
+  int nt;      // tokens in this stage
+  int n;       // tokens in the whole chunk
+  int flags;   // kFirst: first stage of the chunk; kLast: its last stage; kEnd: no more work
 };
-
-__device__ __forceinline__ ChunkSpan chunk_span(const PoolArgs& a, int64_t c) {
-  const int64_t j = owner_doc(a.doc_chunk_off, a.D, c);
-  const int64_t cs = __ldg(a.doc_chunk_off + j), ce = __ldg(a.doc_chunk_off + j + 1);
-  const int64_t ts = __ldg(a.doc_tok_off + j), te = __ldg(a.doc_tok_off + j + 1);
-  const int64_t L = te - ts;
-  ChunkSpan r{0, 0, ts, 0};
-  const bool ok = c >= cs && c < ce && ts >= 0 && L >= 0 && te <= a.Ntok && (ce - cs) == (L + a.P - 1) / a.P;
-  if (!ok) {
-    r.flag = MSA_FLAG_OFFSETS;
-  } else if (L > a.max_len) {
-    r.flag = MSA_FLAG_INDEX_OOB;
-  } else {
-    r.s = ts + (c - cs) * a.P;
-    r.e = min(r.s + (int64_t)a.P, te);
-  }
-  return r;
-}
+constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
 template <typename T>
 __global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
@@ -73,6 +62,7 @@ __global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + (size_t)g.NS * g.stage);
   uint64_t* empty = full + g.NS;
+  StageMeta* meta = reinterpret_cast<StageMeta*>(empty + g.NS);
   const int nconsumer_warps = (g.W + 31) / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -88,33 +78,61 @@ __global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
+    // This CTA owns the contiguous chunks [c_begin, c_end); the owning document
+    // is found once by a warp-wide search and then advanced incrementally.
+    const int64_t per = (a.C + gridDim.x - 1) / gridDim.x;
+    const int64_t c_begin = (int64_t)blockIdx.x * per, c_end = min(a.C, c_begin + per);
+    const bool off_ok = __ldg(a.doc_chunk_off) == 0 && __ldg(a.doc_tok_off) == 0 &&
+                        __ldg(a.doc_chunk_off + a.D) == a.C && __ldg(a.doc_tok_off + a.D) <= a.Ntok;
+    int64_t j = (c_begin < c_end && off_ok) ? warp_owner_doc(a.doc_chunk_off, a.D, c_begin, lane) : 0;
     if (lane == 0) {
-      if (blockIdx.x == 0 && (__ldg(a.doc_chunk_off) != 0 || __ldg(a.doc_tok_off) != 0 ||
-                              __ldg(a.doc_chunk_off + a.D) != a.C || __ldg(a.doc_tok_off + a.D) > a.Ntok))
-        raise_flag(a.err_flag, MSA_FLAG_OFFSETS);
+      if (!off_ok && blockIdx.x == 0) raise_flag(a.err_flag, MSA_FLAG_OFFSETS);
       const uint8_t* K = reinterpret_cast<const uint8_t*>(a.K);
       const uint8_t* V = reinterpret_cast<const uint8_t*>(a.V);
       const uint8_t* R = reinterpret_cast<const uint8_t*>(a.Kr);
+      const uint8_t* P = reinterpret_cast<const uint8_t*>(a.rope_cs);
       uint32_t it = 0;
-      for (int64_t c = blockIdx.x; c < a.C && !timed_out; c += gridDim.x) {
-        const ChunkSpan sp = chunk_span(a, c);
-        if (sp.flag) {
-          raise_flag(a.err_flag, sp.flag);
+      for (int64_t c = off_ok ? c_begin : c_end; c < c_end && !timed_out; ++c) {
+        while (j + 1 < a.D && __ldg(a.doc_chunk_off + j + 1) <= c) ++j;
+        const int64_t cs = __ldg(a.doc_chunk_off + j), ce = __ldg(a.doc_chunk_off + j + 1);
+        const int64_t ts = __ldg(a.doc_tok_off + j), te = __ldg(a.doc_tok_off + j + 1);
+        const int64_t L = te - ts;
+        if (!(c >= cs && c < ce && ts >= 0 && L >= 0 && te <= a.Ntok && (ce - cs) == (L + a.P - 1) / a.P)) {
+          raise_flag(a.err_flag, MSA_FLAG_OFFSETS);
           continue;
         }
-        for (int64_t t0 = sp.s; t0 < sp.e; t0 += g.TOK, ++it) {
+        if (L > a.max_len) {
+          raise_flag(a.err_flag, MSA_FLAG_INDEX_OOB);
+          continue;
+        }
+        const int64_t s0 = ts + (c - cs) * a.P, e0 = min(s0 + (int64_t)a.P, te);
+        for (int64_t t0 = s0; t0 < e0; t0 += g.TOK, ++it) {
           const uint32_t st = it % g.NS, round = it / g.NS;
           if (!mbar_wait(&empty[st], (round & 1) ^ 1, kWaitPolls)) {
             timed_out = true;
             break;
           }
-          const int nt = (int)min((int64_t)g.TOK, sp.e - t0);
+          const int nt = (int)min((int64_t)g.TOK, e0 - t0);
+          meta[st] = StageMeta{c, nt, (int)(e0 - s0), (t0 == s0 ? kFirst : 0) | (t0 + nt >= e0 ? kLast : 0)};
           uint8_t* dst = ring + (size_t)st * g.stage;
-          const uint32_t bK = (uint32_t)nt * g.rowK, bR = (uint32_t)nt * g.rowR;
-          mbar_arrive_expect_tx(&full[st], 2 * bK + bR);
+          const uint32_t bK = (uint32_t)nt * g.rowK, bR = (uint32_t)nt * g.rowR, bP = (uint32_t)nt * g.rowP;
+          mbar_arrive_expect_tx(&full[st], 2 * bK + bR + bP);
           bulk_load(dst, K + t0 * g.rowK, bK, &full[st]);
           bulk_load(dst + (size_t)g.TOK * g.rowK, V + t0 * g.rowK, bK, &full[st]);
           bulk_load(dst + (size_t)2 * g.TOK * g.rowK, R + t0 * g.rowR, bR, &full[st]);
+          // (cos, sin) rows of the stage's positions inside the document
+          bulk_load(dst + (size_t)g.TOK * (2 * g.rowK + g.rowR), P + (t0 - ts) * g.rowP, bP, &full[st]);
+        }
+      }
+      // the end marker: a stage with no data
+      if (!timed_out) {
+        const uint32_t st = it % g.NS, round = it / g.NS;
+        if (mbar_wait(&empty[st], (round & 1) ^ 1, kWaitPolls)) {
+          meta[st] = StageMeta{-1, 0, 0, kEnd};
+          mbar_arrive_expect_tx(&full[st], 0);
+          ++it;
+        } else {
+          timed_out = true;
         }
       }
       // every copy issued must have landed before the CTA leaves
@@ -128,7 +146,7 @@ __global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
     // ---------------------------------------------------------------- consumers
     const int item = threadIdx.x - 32;  // [0, nR) Kr, [nR, nR+nK) K pairs, then V; >= W idle
     const int kind = item < g.nR ? 0 : (item < g.nR + g.nK ? 1 : (item < g.W ? 2 : 3));
-    const int half = a.d / 2, halfv = half / VN;
+    const int halfv = a.d / 2 / VN;
     int off_lo = 0, off_hi = 0, region = 0, h = 0, i0 = 0;
     if (kind == 0) {
       region = 2 * g.TOK * g.rowK;
@@ -138,59 +156,63 @@ __global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
       h = w / halfv;
       i0 = (w - h * halfv) * VN;
       off_lo = (h * a.d + i0) * (int)sizeof(T);
-      off_hi = off_lo + half * (int)sizeof(T);
+      off_hi = off_lo + (a.d / 2) * (int)sizeof(T);
     } else if (kind == 2) {
       region = g.TOK * g.rowK;
       off_lo = (item - g.nR - g.nK) * 16;
     }
     const int rstride = kind == 0 ? g.rowR : g.rowK;
     const int G = a.dr / VN;  // Kr lanes per router head (a power of two <= 32)
-    uint32_t it = 0;
-    for (int64_t c = blockIdx.x; c < a.C && !timed_out; c += gridDim.x) {
-      const ChunkSpan sp = chunk_span(a, c);
-      if (sp.flag) continue;
-      float acc[2 * VN];
+    float acc[2 * VN];
 #pragma unroll
-      for (int i = 0; i < 2 * VN; ++i) acc[i] = 0.f;
-      for (int64_t t0 = sp.s; t0 < sp.e; t0 += g.TOK, ++it) {
-        const uint32_t st = it % g.NS, round = it / g.NS;
-        // the whole warp leaves together, so no warp-collective op below is split
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[st], round & 1, kWaitPolls))) {
-          timed_out = true;
-          break;
-        }
-        const int nt = (int)min((int64_t)g.TOK, sp.e - t0);
-        const uint8_t* base = ring + (size_t)st * g.stage + region;
-        if (kind == 1) {
-          for (int u = 0; u < nt; ++u) {
-            float xl[VN], xh[VN];
-            unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_lo), xl);
-            unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_hi), xh);
-            const int p = (int)(t0 + u - sp.ts);  // position inside the document
-            const float4* cs4 = reinterpret_cast<const float4*>(a.rope_cs + ((size_t)p * half + i0) * 2);
-#pragma unroll
-            for (int q = 0; q < VN / 2; ++q) {
-              const float4 w = __ldg(cs4 + q);  // (cos, sin) of pairs i0+2q and i0+2q+1
-              acc[2 * q] += xl[2 * q] * w.x - xh[2 * q] * w.y;
-              acc[VN + 2 * q] += xh[2 * q] * w.x + xl[2 * q] * w.y;
-              acc[2 * q + 1] += xl[2 * q + 1] * w.z - xh[2 * q + 1] * w.w;
-              acc[VN + 2 * q + 1] += xh[2 * q + 1] * w.z + xl[2 * q + 1] * w.w;
-            }
-          }
-        } else if (kind != 3) {
-          for (int u = 0; u < nt; ++u) {
-            float x[VN];
-            unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_lo), x);
-#pragma unroll
-            for (int i = 0; i < VN; ++i) acc[i] += x[i];
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+    for (int i = 0; i < 2 * VN; ++i) acc[i] = 0.f;
+    for (uint32_t it = 0;; ++it) {
+      const uint32_t st = it % g.NS, round = it / g.NS;
+      // the whole warp leaves together, so no warp-collective op below is split
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[st], round & 1, kWaitPolls))) {
+        timed_out = true;
+        break;
       }
-      if (timed_out) break;
-      // mean, round to the storage type, store
-      const float fn = (float)(sp.e - sp.s);
+      const StageMeta md = meta[st];
+      if (md.flags & kEnd) break;
+      if (md.flags & kFirst) {
+#pragma unroll
+        for (int i = 0; i < 2 * VN; ++i) acc[i] = 0.f;
+      }
+      const int nt = md.nt;
+      const uint8_t* base = ring + (size_t)st * g.stage + region;
+      if (kind == 1) {
+        const uint8_t* rope = ring + (size_t)st * g.stage + (size_t)g.TOK * (2 * g.rowK + g.rowR) + i0 * 8;
+#pragma unroll 4
+        for (int u = 0; u < nt; ++u) {
+          float xl[VN], xh[VN];
+          unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_lo), xl);
+          unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_hi), xh);
+          const float4* cs4 = reinterpret_cast<const float4*>(rope + u * g.rowP);
+#pragma unroll
+          for (int q = 0; q < VN / 2; ++q) {
+            const float4 w = cs4[q];  // (cos, sin) of pairs i0+2q and i0+2q+1
+            acc[2 * q] += xl[2 * q] * w.x - xh[2 * q] * w.y;
+            acc[VN + 2 * q] += xh[2 * q] * w.x + xl[2 * q] * w.y;
+            acc[2 * q + 1] += xl[2 * q + 1] * w.z - xh[2 * q + 1] * w.w;
+            acc[VN + 2 * q + 1] += xh[2 * q + 1] * w.z + xl[2 * q + 1] * w.w;
+          }
+        }
+      } else if (kind != 3) {
+#pragma unroll 4
+        for (int u = 0; u < nt; ++u) {
+          float x[VN];
+          unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_lo), x);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[i] += x[i];
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      if (!(md.flags & kLast)) continue;
+      // chunk complete: mean, round to the storage type, store
+      const int64_t c = md.c;
+      const float fn = (float)md.n;
       float m[VN], ss = 0.f;
       if (kind == 0) {
 #pragma unroll
@@ -251,7 +273,8 @@ cudaError_t pool_t(const PoolArgs& a, cudaStream_t s) {
   g.W = g.nK + g.nV + g.nR;
   g.rowK = a.Hkv * a.d * (int)sizeof(T);
   g.rowR = a.Hr * a.dr * (int)sizeof(T);
-  const int row = 2 * g.rowK + g.rowR;
+  g.rowP = a.d * (int)sizeof(float);
+  const int row = 2 * g.rowK + g.rowR + g.rowP;
   g.TOK = 8;
   while (g.TOK > 1 && 2 * g.TOK * row > kRingBytes) g.TOK >>= 1;
   if (g.TOK > a.P) g.TOK = a.P;
@@ -261,7 +284,7 @@ cudaError_t pool_t(const PoolArgs& a, cudaStream_t s) {
   if (g.NS < 2) return cudaErrorInvalidValue;
   const int threads = 32 + ((g.W + 31) / 32) * 32;
   if (threads > 512) return cudaErrorInvalidValue;
-  const size_t sm = 128 + (size_t)g.NS * g.stage + 16 * (size_t)g.NS;
+  const size_t sm = 128 + (size_t)g.NS * g.stage + 16 * (size_t)g.NS + sizeof(StageMeta) * g.NS;
   cudaError_t e = cudaFuncSetAttribute(pool_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   if (a.C <= 0) return cudaSuccess;

@@ -40,9 +40,6 @@ route_generic_kernel(RouteArgs a) {
   const int64_t c = (int64_t)blockIdx.x * 32 + lane;
   const bool cvalid = c < a.C;
 
-  if (blockIdx.x == 0 && threadIdx.x == 0 && __ldg(a.doc_chunk_off + a.D) != a.C)
-    raise_flag(a.err_flag, MSA_FLAG_OFFSETS);
-
   // this lane's chunk key for head h, in registers
   float kr[DR];
   float rk = 0.f;
@@ -59,7 +56,7 @@ route_generic_kernel(RouteArgs a) {
     }
     if (cvalid) rk = __ldg(a.kr_rnorm + c * Hr + h);
   }
-  const int doc = cvalid ? (int)owner_doc(a.doc_chunk_off, a.D, c) : -1;
+  const int doc = cvalid ? __ldg(a.chunk_doc + c) : -1;
   const float invHr = 1.0f / (float)Hr;
 
   for (int64_t b = 0; b < a.B; ++b) {
@@ -138,9 +135,32 @@ cudaError_t route_generic_t(const RouteArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+// chunk_doc[c] = the document that owns chunk c, one warp per 32 chunks; also
+// flags offsets whose last entry is not C.
+__global__ void chunk_doc_kernel(const int64_t* __restrict__ off, int64_t D, int64_t C, int32_t* __restrict__ out,
+                                 int32_t* err_flag) {
+  const int lane = threadIdx.x & 31;
+  const int64_t c0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && (__ldg(off) != 0 || __ldg(off + D) != C))
+    raise_flag(err_flag, MSA_FLAG_OFFSETS);
+  if (c0 >= C) return;  // whole warp
+  int doc = warp_chunk_docs(off, D, C, c0, lane);
+  if (doc >= D) {  // only reachable with offsets that do not end at C: never index past D
+    raise_flag(err_flag, MSA_FLAG_OFFSETS);
+    doc = -1;
+  }
+  if (c0 + lane < C) out[c0 + lane] = doc;
+}
+
 cudaError_t launch_route(msa_dtype dt, const RouteArgs& a, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(a.doc_key, 0, sizeof(uint32_t) * a.B * a.D, s);
   if (e != cudaSuccess) return e;
+  if (a.C > 0) {
+    const int64_t blocks = (a.C + 255) / 256;
+    count_launch();
+    chunk_doc_kernel<<<(unsigned)blocks, 256, 0, s>>>(a.doc_chunk_off, a.D, a.C, a.chunk_doc, a.err_flag);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   if (dt == MSA_BF16) {
     bool handled = false;
     e = launch_route_tc(a, s, &handled);

@@ -21,10 +21,11 @@
 // over the warp's chunks of one document, and one atomicMax per document
 // segment on an order-preserving key.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work items):
+// Warp roles (320 threads, one CTA per SM, persistent over work items):
 //   warp 0 lane 0  TMA producer (smem ring of STAGES head-slices)
 //   warp 1         TMEM allocator; lane 0 issues the MMAs
-//   warps 2..5     epilogue, one TMEM lane quarter each
+//   warps 2..9     epilogue: two warpgroups, each reading half of the N columns
+//                  of every TMEM lane quarter with one wait per head
 // Every mbarrier wait is bounded; on expiry the kernel raises MSA_FLAG_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include "common.cuh"
@@ -38,13 +39,13 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer warp, MMA warp, 2 epilogue warpgroups
 constexpr uint32_t kWaitPolls = 1u << 24;
 
 struct RouteTcParams {
   const float* kr_rnorm;
   const float* rq;  // [rows, Hr]
-  const int64_t* doc_chunk_off;
+  const int32_t* chunk_doc;  // [C] owning document of every chunk
   uint32_t* doc_key;
   int32_t* err_flag;
   int64_t D, C;
@@ -60,7 +61,7 @@ struct Layout {
   static constexpr int kB = N * DR * 2;                   // Qr slice of one head
   static constexpr int kStage = kA + kB;
   static constexpr int kStages = (200 * 1024) / kStage > 6 ? 6 : (200 * 1024) / kStage;
-  static constexpr int kRq = 4 * 8 * N * 4;               // per epilogue warp: rq of the row block, Hr <= 8
+  static constexpr int kRq = 8 * 8 * (N / 2) * 4;         // per epilogue warp: rq of its columns, Hr <= 8
   static constexpr int kBar = 8 * (2 * kStages + 5) + 16;
   static constexpr int kSmem = 1024 + kStages * kStage + kRq + kBar;
   static constexpr uint32_t kTmemCols = 2 * N;            // two accumulators of N fp32 columns
@@ -107,7 +108,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accf[i], 1);
-      mbar_init(&acce[i], 128);
+      mbar_init(&acce[i], 256);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -186,63 +187,67 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lanes [32q, 32q + 32) belong to this warp
-    float* rq_w = rq_s + q * 8 * N;  // this warp's private copy (no cross-warp barrier)
-    const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
+    // two warpgroups; each covers all 128 TMEM lanes and half of the N columns
+    constexpr int NH = N / 2;
+    const int q = warp & 3;                 // TMEM lanes [32q, 32q + 32) belong to this warp
+    const int wg = (warp - 2) >> 2;         // column half of this warpgroup
+    const int col0 = wg * NH;
+    float* rq_w = rq_s + (warp - 2) * 8 * NH;  // this warp's private copy (no cross-warp barrier)
+    const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16) + col0;
     const float invHr = 1.0f / (float)Hr;
     uint32_t it = 0;
     for (int64_t item = blockIdx.x; item < p.items && !timed_out; item += gridDim.x) {
       const int tile = (int)(item / p.n_rb), rb = (int)(item % p.n_rb);
       const int64_t c = (int64_t)tile * kTileM + q * 32 + lane;
       const bool valid = c < p.C;
-      const int r0 = rb * N;
-      const int nvalid = min(N, p.rows - r0);
+      const int r0 = rb * N + col0;                 // first query row of this warp's columns
+      const int nvalid = max(0, min(NH, p.rows - r0));
       __syncwarp();
-      for (int i = lane; i < Hr * N; i += 32) {
-        const int h = i / N, col = i - h * N, r = r0 + col;
+      for (int i = lane; i < Hr * NH; i += 32) {
+        const int h = i / NH, col = i - h * NH, r = r0 + col;
         rq_w[i] = r < p.rows ? __ldg(p.rq + (int64_t)r * Hr + h) : 0.f;
       }
       __syncwarp();
-      const int doc = valid ? (int)owner_doc(p.doc_chunk_off, p.D, c) : -1;
-      float S_[N];
+      const int doc = valid ? __ldg(p.chunk_doc + c) : -1;
+      float rkv[8];  // this chunk's 1/||K̄r|| for every head, loaded together
 #pragma unroll
-      for (int j = 0; j < N; ++j) S_[j] = 0.f;
+      for (int h = 0; h < 8; ++h) rkv[h] = (valid && h < Hr) ? __ldg(p.kr_rnorm + c * Hr + h) : 0.f;
+      float S_[NH];
+#pragma unroll
+      for (int j = 0; j < NH; ++j) S_[j] = 0.f;
       for (int h = 0; h < Hr; ++h, ++it) {
         const uint32_t buf = it & 1, use = it >> 1;
-        const float rk = valid ? __ldg(p.kr_rnorm + c * Hr + h) : 0.f;
+        float rk = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rk = i == h ? rkv[i] : rk;
         // the whole warp leaves together, so tcgen05.ld and the shuffles are never split
         if (!__all_sync(0xffffffffu, mbar_wait(&accf[buf], use & 1, kWaitPolls))) {
           timed_out = true;
           break;
         }
         tc_fence_after();
-        const float* rqh = rq_w + h * N;
+        float v[NH];
 #pragma unroll
-        for (int j0 = 0; j0 < N; j0 += 32) {
-          float v0[16], v1[16];
-          tmem_ld16(lane_addr + buf * N + j0, v0);
-          tmem_ld16(lane_addr + buf * N + j0 + 16, v1);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            S_[j0 + i] = fmaf(v0[i], rk * rqh[j0 + i], S_[j0 + i]);
-            S_[j0 + 16 + i] = fmaf(v1[i], rk * rqh[j0 + 16 + i], S_[j0 + 16 + i]);
-          }
-        }
+        for (int j0 = 0; j0 < NH; j0 += 16) tmem_ld16(lane_addr + buf * N + j0, *reinterpret_cast<float(*)[16]>(&v[j0]));
+        tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(&acce[buf]);
+        mbar_arrive(&acce[buf]);  // the accumulator is in registers: the MMA may reuse it
+        const float* rqh = rq_w + h * NH;
+#pragma unroll
+        for (int j = 0; j < NH; ++j) S_[j] = fmaf(v[j], rk * rqh[j], S_[j]);
       }
       if (timed_out) break;
+      if (nvalid == 0) continue;
       const int b_first = r0 / p.Tq, b_last = (r0 + nvalid - 1) / p.Tq;
       if (b_first == b_last) {
         float m = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < N; ++j)
+        for (int j = 0; j < NH; ++j)
           if (j < nvalid) m = fmaxf(m, S_[j]);
         doc_max_atomic(m * invHr, doc, lane, p.doc_key + (int64_t)b_first * p.D);
       } else {
 #pragma unroll
-        for (int j = 0; j < N; ++j) {
+        for (int j = 0; j < NH; ++j) {
           if (j < nvalid) {
             const int b = (r0 + j) / p.Tq;
             doc_max_atomic(S_[j] * invHr, doc, lane, p.doc_key + (int64_t)b * p.D);
@@ -296,7 +301,7 @@ cudaError_t launch_t(const RouteArgs& a, cudaStream_t s) {
   RouteTcParams p;
   p.kr_rnorm = a.kr_rnorm;
   p.rq = a.rq;
-  p.doc_chunk_off = a.doc_chunk_off;
+  p.chunk_doc = a.chunk_doc;
   p.doc_key = a.doc_key;
   p.err_flag = a.err_flag;
   p.D = a.D;

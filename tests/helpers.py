@@ -92,7 +92,8 @@ def route_on_gpu(Qr, Krb, rn, coff: np.ndarray, k: int):
     dev = Qr.device
     B = Qr.shape[0]
     D = len(coff) - 1
-    ws = torch.empty(msa.route_topk_workspace_size(B, Qr.shape[1], Qr.shape[2], D, k), dtype=torch.uint8, device=dev)
+    ws = torch.empty(msa.route_topk_workspace_size(B, Qr.shape[1], Qr.shape[2], D, Krb.shape[0], k), dtype=torch.uint8,
+                     device=dev)
     idx = torch.empty((B, k), dtype=torch.int32, device=dev)
     sc = torch.empty((B, k), dtype=torch.float32, device=dev)
     ds = torch.empty((B, D), dtype=torch.float32, device=dev)

@@ -99,7 +99,7 @@ def test_route_rejects_bad_arguments():
     assert _route(idx=None) == INVALID
     assert _route(Qr=FAKE + 2) == INVALID
     assert _route(ws=None) == WORKSPACE
-    need = _lib.load().msa_route_topk_workspace_size(1, 4, 8, 10, 3)
+    need = _lib.load().msa_route_topk_workspace_size(1, 4, 8, 10, 20, 3)
     assert need > 0 and _route(wsb=need - 1) == WORKSPACE
     assert _route(B=0) == OK
 
@@ -129,8 +129,8 @@ def test_gather_and_layer_reject_bad_arguments():
     assert lib.msa_gather(*dict(g, d=100).values(), None) == UNSUPPORTED
     assert lib.msa_gather(*dict(g, ml=None).values(), None) == INVALID
     assert lib.msa_gather(*dict(g, Km=FAKE + 1).values(), None) == INVALID
-    need = lib.msa_layer_forward_workspace_size(1, 8, 8, 32, 8, 128, 8, 10, 3, 24)
-    assert need > lib.msa_route_topk_workspace_size(1, 8, 8, 10, 3)
+    need = lib.msa_layer_forward_workspace_size(1, 8, 8, 32, 8, 128, 8, 10, 20, 3, 24)
+    assert need > lib.msa_route_topk_workspace_size(1, 8, 8, 10, 20, 3)
     L = dict(dt=1, Qr=FAKE, Hr=8, dr=128, Krb=FAKE, rn=FAKE, chk=FAKE, D=10, C=20, k=3, Q=FAKE, Kl=FAKE,
              Vl=FAKE, B=1, Tq=8, Lloc=8, Hq=32, Hkv=8, d=128, Kb=FAKE, Vb=FAKE, Mmax=24, scale=0.0, O=FAKE,
              lse=None, idx=FAKE, sc=None, ds=None, ws=FAKE, wsb=need, flag=None)

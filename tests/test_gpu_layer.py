@@ -20,7 +20,8 @@ def _layer_gpu(cfg, q, Kb, Vb, Krb, rn, coff):
     B, Tq = cfg.B, cfg.Tq
     D = len(coff) - 1
     Mmax = cfg.Mmax
-    ws = torch.empty(msa.layer_forward_workspace_size(B, Tq, cfg.Lloc, cfg.Hq, cfg.Hkv, cfg.d, cfg.Hr, D, cfg.k, Mmax),
+    ws = torch.empty(msa.layer_forward_workspace_size(B, Tq, cfg.Lloc, cfg.Hq, cfg.Hkv, cfg.d, cfg.Hr, D, Krb.shape[0],
+                                                      cfg.k, Mmax),
                      dtype=torch.uint8, device=DEV)
     O_ = torch.empty_like(q["Q"])
     lse = torch.empty((B, cfg.Hq, Tq), dtype=torch.float32, device=DEV)

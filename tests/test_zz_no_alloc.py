@@ -60,7 +60,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
 def test_noalloc_rejects_a_problem_larger_than_its_scratch():
     lib = _lib.load()
     B, Tq, Hr, D, k = 64, 1, 8, 1 << 17, 16          # 64 x 131072 document keys alone are 32 MiB
-    need = lib.msa_route_topk_workspace_size(B, Tq, Hr, D, k)
+    need = lib.msa_route_topk_workspace_size(B, Tq, Hr, D, 4 * D, k)
     assert need > msa.NOALLOC_SCRATCH_BYTES
     # the size check comes before any use of the (never dereferenced) pointers
     fake = 0x10000
