@@ -192,7 +192,7 @@ class MSAWorkload:
         self.flag = torch.zeros(1, dtype=torch.int32, device=device)
         self.raw = None
         if step_kind == "full":
-            self.raw = synth.gen_raw_slab(cfg, 0, cfg.D, device, seed, Qr0=self.layers[0]["Qr"][0])
+            self._fill_raw(seed)
         else:
             self._pool_slabs(seed)
         B, c = cfg.B, cfg
@@ -205,6 +205,19 @@ class MSAWorkload:
         self.ml = torch.zeros(B, dtype=torch.int32, device=device)
         n = msa.sparse_attn_workspace_size(B, c.Tq, c.Lloc, c.Hq, c.Hkv, c.d, c.Mmax)
         self.aws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+    def _fill_raw(self, seed):
+        """Resident raw K / V / Kr for the whole corpus, drawn slab by slab."""
+        c, n = self.cfg, int(self.tok[-1])
+        dt = c.torch_dtype
+        self.raw = (torch.empty((n, c.Hkv, c.d), dtype=dt, device=self.dev),
+                    torch.empty((n, c.Hkv, c.d), dtype=dt, device=self.dev),
+                    torch.empty((n, c.Hr, c.dr), dtype=dt, device=self.dev))
+        for lo, hi in synth.slab_bounds(c):
+            t0, t1 = int(self.tok[lo]), int(self.tok[hi])
+            for dst, src in zip(self.raw, synth.gen_raw_slab(c, lo, hi, self.dev, seed, Qr0=self.layers[0]["Qr"][0])):
+                dst[t0:t1].copy_(src)
+        torch.cuda.synchronize()
 
     def _pool_slabs(self, seed):
         c, msa = self.cfg, self.msa
@@ -304,7 +317,8 @@ def run_gpu(args, rank, local_rank, world):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     import routed_sparse_attention_chunk_b200 as msa
     cfg = workload_config(args)
-    step_kind = args.step or ("query" if cfg.docs_per_slab else "full")
+    raw_bytes = cfg.ntok * (2 * cfg.Hkv * cfg.d + cfg.Hr * cfg.dr) * (4 if cfg.dtype == "f32" else 2)
+    step_kind = args.step or ("query" if raw_bytes > 80e9 else "full")
     peaks, peak_kind = load_peaks()
     counts = workload_counts(cfg)
     w = MSAWorkload(cfg, device, seed=1000 * rank, step_kind=step_kind)
@@ -353,8 +367,7 @@ def run_gpu(args, rank, local_rank, world):
     barrier(world, device)
     total_ms = max_over_ranks(step_ms_local, world, device)
     ms_per_step = total_ms / args.steps
-    tokens_per_step = cfg.B * cfg.Tq * cfg.layers * world if step_kind == "query" and cfg.layers > 1 \
-        else cfg.B * cfg.Tq * world
+    tokens_per_step = cfg.B * cfg.Tq * world  # query tokens through the whole layer stack
     value = tokens_per_step / (ms_per_step / 1e3)
 
     # ---- roofline of the dominant stage (live per-launch times from the timed region)

@@ -20,7 +20,9 @@
 namespace msa {
 
 cudaError_t launch_attn_tc(msa_dtype dt, const AttnArgs& a, cudaStream_t s, bool* handled);
-size_t attn_tc_workspace_size(msa_dtype dt, int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Mmax);
+bool decode_applies(msa_dtype dt, const AttnArgs& a);
+size_t decode_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int Mmax);
+cudaError_t launch_attn_decode(const AttnArgs& a, cudaStream_t s);
 
 namespace {
 
@@ -153,11 +155,21 @@ cudaError_t attn_generic_t(const AttnArgs& a, cudaStream_t s) {
 }  // namespace
 
 size_t attn_workspace_size(msa_dtype dt, int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Mmax) {
-  return attn_tc_workspace_size(dt, B, Tq, Lloc, Hq, Hkv, d, Mmax);
+  AttnArgs a{};
+  a.B = B;
+  a.Tq = Tq;
+  a.Lloc = Lloc;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = d;
+  a.Mmax = Mmax;
+  if (Hkv > 0 && decode_applies(dt, a)) return decode_workspace_size(B, Tq, Lloc, Hq, Hkv, Mmax);
+  return 0;
 }
 
 cudaError_t launch_attn(msa_dtype dt, const AttnArgs& a, cudaStream_t s) {
   if (a.B <= 0) return cudaSuccess;
+  if (decode_applies(dt, a)) return launch_attn_decode(a, s);
   bool handled = false;
   cudaError_t e = launch_attn_tc(dt, a, s, &handled);
   if (e != cudaSuccess || handled) return e;

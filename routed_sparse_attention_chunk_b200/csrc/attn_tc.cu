@@ -379,8 +379,6 @@ cudaError_t launch_dh(const AttnArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-size_t attn_tc_workspace_size(msa_dtype, int64_t, int, int, int, int, int, int) { return 0; }
-
 // Shapes the tensor-core kernel takes: bf16, d = 128, dense memory rows, a GQA
 // group that divides the 128 rows into blocks of at least 8 tokens, and enough
 // query tokens to fill most of a block.

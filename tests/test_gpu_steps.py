@@ -251,6 +251,22 @@ def test_attention_bf16_tensor_core_tiling(B, Tq, Lloc, Hq, Hkv, Mmax, mem_lens)
     close_abs(to64(lse), olse, 2e-3, "lse")
 
 
+@pytest.mark.parametrize("B,Tq,Lloc,Hq,Hkv,Mmax,mem_lens", [
+    (5, 1, 4096, 32, 8, 128, [128, 0, 77, 1, 128]),   # the batched-decode shape, ragged memory
+    (2, 4, 700, 32, 8, 200, [200, 13]),               # 4 tokens x G=4: 16 rows, causal inside the block
+    (3, 2, 300, 64, 8, 128, [5, 128, 64]),             # G=8, 2 tokens: 16 rows
+    (2, 3, 129, 8, 8, 0, [0, 0]),                      # MHA, no memory at all
+])
+def test_attention_bf16_decode_shapes(B, Tq, Lloc, Hq, Hkv, Mmax, mem_lens):
+    Q, Kl, Vl, Km, Vm, ml = _attn_inputs(B, Tq, Lloc, Hq, Hkv, 128, Mmax, mem_lens, torch.bfloat16, 5)
+    Og, lse, flag = attn_on_gpu(Q, Kl, Vl, Km, Vm, ml)
+    Oo, olse = O.attention(to64(Q), to64(Kl), to64(Vl), to64(Km), to64(Vm), mem_lens)
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    close_abs(to64(Og), Oo, TOL_BF16_ABS, "O")
+    close_abs(to64(lse), olse, 2e-3, "lse")
+
+
 def test_attention_bad_mem_len_is_flagged_not_faulted():
     Q, Kl, Vl, Km, Vm, ml = _attn_inputs(1, 4, 4, 2, 1, 64, 8, [9999], torch.bfloat16, 3)
     Og, lse, flag = attn_on_gpu(Q, Kl, Vl, Km, Vm, ml)
