@@ -39,7 +39,7 @@ struct RouteWs {
 RouteWs route_ws_layout(void* base, int64_t B, int Tq, int Hr, int64_t D, int64_t C, int k) {
   RouteWs w{};
   w.nslice = topk_num_slices(D, k);
-  const size_t keys = round_up(sizeof(uint32_t) * (size_t)B * (size_t)D, 256);
+  const size_t keys = round_up(sizeof(uint32_t) * ((size_t)B * (size_t)D + (size_t)B), 256);  // + counters
   const size_t cand = w.nslice > 1 ? round_up(sizeof(uint64_t) * (size_t)B * w.nslice * k, 256) : 0;
   const size_t rq = round_up(sizeof(float) * (size_t)B * (size_t)Tq * (size_t)Hr, 256);
   const size_t cdoc = round_up(sizeof(int32_t) * (size_t)(C > 0 ? C : 1), 256);
@@ -171,7 +171,7 @@ msa_status msa_route_topk(msa_dtype dt, const void* Qr, int64_t B, int Tq, int H
   RouteArgs ra{Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, w.doc_key, w.rq, w.chunk_doc, err_flag};
   cudaError_t e = launch_route(dt, ra, s);
   if (e != cudaSuccess) return MSA_ERR_CUDA;
-  TopkArgs ta{w.doc_key, B, D, k, w.cand, w.nslice, topk_idx, topk_score, doc_scores};
+  TopkArgs ta{w.doc_key, B, D, k, w.cand, w.doc_key + B * D, w.nslice, topk_idx, topk_score, doc_scores};
   return cuda_status(launch_topk(ta, s));
 }
 
@@ -248,7 +248,7 @@ msa_status msa_layer_forward(msa_dtype dt, const void* Qr, int Hr, int dr, const
 
   RouteArgs ra{Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, w.doc_key, w.rq, w.chunk_doc, err_flag};
   if (launch_route(dt, ra, s) != cudaSuccess) return MSA_ERR_CUDA;
-  TopkArgs ta{w.doc_key, B, D, k, w.cand, w.nslice, topk_idx, topk_score, doc_scores};
+  TopkArgs ta{w.doc_key, B, D, k, w.cand, w.doc_key + B * D, w.nslice, topk_idx, topk_score, doc_scores};
   if (launch_topk(ta, s) != cudaSuccess) return MSA_ERR_CUDA;
   GatherArgs ga{topk_idx, B, k, doc_chunk_off, D, C, Kbar, Vbar, Hkv, d, Mmax, Kmem, Vmem, mem_len, err_flag};
   if (launch_gather(dt, ga, s) != cudaSuccess) return MSA_ERR_CUDA;

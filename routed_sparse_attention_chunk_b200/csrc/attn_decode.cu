@@ -3,23 +3,25 @@
 // ("MSA x Qwen3.5" model card, "Architecture summary"; "MSA: Memory Sparse
 // Attention" README, "Inference Pipeline" stage 3, sparse generation).
 //
-// The work is an HBM stream of K and V: with the GQA group packed as rows
-// (R = G * Tq <= 16 rows per KV head) every key costs 2 R d multiply-adds, far
-// below what the memory system delivers per SM, so this runs on CUDA cores and
-// is shaped for bandwidth:
-//   * persistent CTAs (one per SM) walk work units = (batch row, KV head,
-//     key split); every split but the last holds the same number of 128-key
-//     tiles;
-//   * a producer thread streams K and V tiles with 2D TMA (128-byte swizzle)
-//     into a ring of shared-memory stages;
-//   * four compute warps: for Q K^T a lane owns one key of the tile and reads
-//     its swizzled K row against the Q rows (fp32, pre-scaled, in shared
-//     memory); the tile's row maxima and exp2 weights go through shared memory;
-//     for P V a thread owns two output dimensions and half of the tile's keys;
-//   * each unit leaves (max, sum, unnormalised O) per row in the workspace and a
-//     second kernel merges the splits of every (batch row, KV head).
-// Every wait is bounded; after the first expired wait the CTA stops waiting,
-// finishes its loops without data, and raises MSA_FLAG_TIMEOUT.
+// Decoding reads every K and V row once and does little arithmetic per row, so
+// the kernel is shaped for HBM bandwidth; the contractions still run on the
+// tensor cores, with the roles of prefill swapped so that the 128 keys of a
+// tile are the MMA's M (one TMEM lane each) and the R = G * Tq <= 16 query
+// rows of one KV head are its N = 16:
+//   S^T[key, row] = K_tile (TMA, 128-byte swizzle) x Q^T        (tcgen05.mma)
+//   O^T[d, row]  += V_tile^T (MN-major, straight from the tile) x P^T
+// with S^T double-buffered in TMEM so the tensor core computes the next tile
+// while the softmax warps work on this one.  Each softmax thread owns one TMEM
+// lane: a key of S^T and a dimension of O^T.  Column (row) maxima are reduced
+// across the 128 lanes with shuffles and shared memory; the running max moves
+// only when it grows by more than 2^8 (then O^T is rescaled in TMEM).
+// Persistent CTAs (one per SM) walk work units = (batch row, KV head, key
+// split); each unit leaves (max, sum, unnormalised O) per row in the workspace
+// and a second kernel merges the splits.
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..5 softmax / output.  Every wait is bounded; after the first
+// expired wait the CTA stops waiting, runs its loops out without data and
+// raises MSA_FLAG_TIMEOUT.
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -31,12 +33,12 @@ namespace {
 using namespace sm100;
 
 constexpr int kDH = 128;
-constexpr int kKeys = 128;              // keys per tile
-constexpr int kMaxRows = 16;            // R = G * Tq
+constexpr int kKeys = 128;              // keys per tile (the MMA's M)
+constexpr int kMaxRows = 16;            // R = G * Tq (the MMA's N, padded to 16)
 constexpr int kStages = 3;
-constexpr int kCompute = 128;           // compute threads (4 warps)
-constexpr int kThreads = kCompute + 32; // + producer warp
+constexpr int kThreads = 192;
 constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr float kRescaleLog2 = 8.0f;
 
 struct DecParams {
   const __nv_bfloat16* Q;
@@ -53,10 +55,12 @@ struct DecParams {
 };
 
 struct DLayout {
-  static constexpr int kTile = kKeys * kDH * 2;      // one K (or V) tile
+  static constexpr int kTile = kKeys * kDH * 2;       // one K (or V) tile, two 64-wide boxes
   static constexpr int kStage = 2 * kTile;
-  static constexpr int kSmem = 1024 + kStages * kStage + kMaxRows * kDH * 4 + kKeys * kMaxRows * 4 +
-                               4 * kMaxRows * 4 + 2 * 64 * kMaxRows * 2 * 4 + 8 * (2 * kStages) + 64;
+  static constexpr int kQ = kMaxRows * kDH * 2;       // Q rows, K-major, 128-byte swizzle
+  static constexpr int kP = kMaxRows * kKeys * 2;     // P^T rows (query rows x keys)
+  static constexpr int kSmem = 1024 + kStages * kStage + kQ + kP + 4 * kMaxRows * 4 + 8 * 16 + 16;
+  static constexpr uint32_t kTmemCols = 64;           // S0, S1, O (16 columns each)
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -64,7 +68,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Byte offset of element (row, col) in a K-major, 128-byte-swizzled tile whose
+// rows hold 64 elements per box and `rows` rows per box.
+__device__ __forceinline__ int sw128_off(int row, int col, int rows) {
+  const int box = col >> 6, c = col & 63;
+  return box * (rows * 128) + row * 128 + ((((c >> 3) ^ (row & 7))) << 4) + (c & 7) * 2;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_constant__ CUtensorMap tmVm,
@@ -72,33 +84,53 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  float* q_s = reinterpret_cast<float*>(ring + kStages * DLayout::kStage);  // [R][kDH]
-  float* p_s = q_s + kMaxRows * kDH;                                        // [kKeys][R]
-  float* red_s = p_s + kKeys * kMaxRows;                                    // [4 warps][R]
-  float* o_s = red_s + 4 * kMaxRows;                                        // [64 pairs][R][2]
-  float* l_s = o_s + 64 * kMaxRows * 2;                                     // [64][R] (sums of the upper key half)
-  uint64_t* full = reinterpret_cast<uint64_t*>(l_s + 64 * kMaxRows);
-  uint64_t* empty = full + kStages;
-  volatile int* abort_s = reinterpret_cast<volatile int*>(empty + kStages);
+  uint8_t* Qs = ring + kStages * DLayout::kStage;
+  uint8_t* Ps = Qs + DLayout::kQ;
+  float* red_s = reinterpret_cast<float*>(Ps + DLayout::kP);  // [4 warps][16]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red_s + 4 * kMaxRows);
+  uint64_t* kv_full = bars;            // [3]
+  uint64_t* kv_empty = bars + 3;       // [3]
+  uint64_t* s_full = bars + 6;         // [2]
+  uint64_t* s_free = bars + 8;         // [2]
+  uint64_t* q_ready = bars + 10;
+  uint64_t* p_full = bars + 11;
+  uint64_t* o_done = bars + 12;
+  uint64_t* drain = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_s = reinterpret_cast<volatile int*>(bars + 15);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int R = p.R;
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 4);  // one arrival per compute warp
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    mbar_init(q_ready, 128);
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
     *abort_s = 0;
     fence_mbar_init();
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, DLayout::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tO = tmem + 32;
 
-  if (warp == 4) {
+  if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       uint32_t it = 0;
-      bool ok = true;
-      for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      for (int64_t u = blockIdx.x; u < p.units && !*abort_s; u += gridDim.x) {
         const int s = (int)(u % p.S);
         const int64_t bg = u / p.S;
         const int g = (int)(bg % p.Hkv);
@@ -106,196 +138,227 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
         const int t_end = min((s + 1) * p.tps, p.NM + p.NL);
         for (int t = s * p.tps; t < t_end; ++t, ++it) {
           const uint32_t st = it % kStages, round = it / kStages;
-          if (!mbar_wait(&empty[st], (round & 1) ^ 1, kWaitPolls)) {
-            ok = false;
+          if (!mbar_wait(&kv_empty[st], (round & 1) ^ 1, kWaitPolls)) {
             *abort_s = 1;
             break;
           }
           uint8_t* Kd = ring + st * DLayout::kStage;
           uint8_t* Vd = Kd + DLayout::kTile;
-          mbar_arrive_expect_tx(&full[st], DLayout::kStage);
+          mbar_arrive_expect_tx(&kv_full[st], DLayout::kStage);
           const bool mem = t < p.NM;
           const CUtensorMap* mk = mem ? &tmKm : &tmKl;
           const CUtensorMap* mv = mem ? &tmVm : &tmVl;
           const int y = mem ? (int)(b * p.Mmax + t * kKeys) : (int)(b * p.Lloc + (t - p.NM) * kKeys);
           for (int dc = 0; dc < 2; ++dc) {
-            tma_load_2d(Kd + dc * (kKeys * 128), mk, g * kDH + dc * 64, y, &full[st]);
-            tma_load_2d(Vd + dc * (kKeys * 128), mv, g * kDH + dc * 64, y, &full[st]);
+            tma_load_2d(Kd + dc * (kKeys * 128), mk, g * kDH + dc * 64, y, &kv_full[st]);
+            tma_load_2d(Vd + dc * (kKeys * 128), mv, g * kDH + dc * 64, y, &kv_full[st]);
           }
         }
       }
       const uint32_t fills = it;
       for (uint32_t st = 0; st < (uint32_t)kStages && st < fills; ++st) {
         const uint32_t last = (fills - 1 - st) / kStages * kStages + st;
-        if (!mbar_wait(&full[st], (last / kStages) & 1, kWaitPolls)) *abort_s = 1;
+        if (!mbar_wait(&kv_full[st], (last / kStages) & 1, kWaitPolls)) *abort_s = 1;
       }
     }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kKeys, kMaxRows);                              // K x Q^T
+      constexpr uint32_t idO = idesc_bf16_f32(kDH, kMaxRows, /*b_mn=*/false, /*a_mn=*/true);  // V^T x P^T
+      const uint32_t q0 = smem_u32(Qs), p0 = smem_u32(Ps);
+      uint32_t it = 0, js = 0;  // it: K/V tiles; js: S buffers used
+      int64_t nunit = 0;
+      for (int64_t u = blockIdx.x; u < p.units; u += gridDim.x, ++nunit) {
+        const int s = (int)(u % p.S);
+        const int t0 = s * p.tps, t_end = min((s + 1) * p.tps, p.NM + p.NL);
+        const int T = t_end - t0;
+        if (!*abort_s && !mbar_wait(q_ready, (uint32_t)(nunit & 1), kWaitPolls)) *abort_s = 1;
+        auto issue_S = [&](int j) {
+          const uint32_t st = (it + j) % kStages, round = (it + j) / kStages;
+          const uint32_t sb = (js + j) & 1, use = (js + j) >> 1;
+          if (!*abort_s && (!mbar_wait(&kv_full[st], round & 1, kWaitPolls) ||
+                            !mbar_wait(&s_free[sb], (use & 1) ^ 1, kWaitPolls)))
+            *abort_s = 1;
+          tc_fence_after();
+          const uint32_t k0 = smem_u32(ring + st * DLayout::kStage);
+#pragma unroll
+          for (int k = 0; k < kDH / 16; ++k) {
+            const int box = k >> 2, kk = k & 3;
+            mma_bf16_ss(tS + sb * 16, desc_k_sw128(k0 + box * (kKeys * 128) + kk * 32),
+                        desc_k_sw128(q0 + box * (kMaxRows * 128) + kk * 32), idS, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&s_full[sb]);
+        };
+        if (T > 0) issue_S(0);
+        for (int j = 0; j < T; ++j) {
+          if (j + 1 < T) issue_S(j + 1);
+          const uint32_t st = (it + j) % kStages;
+          if (!*abort_s && !mbar_wait(p_full, (uint32_t)((it + j) & 1), kWaitPolls)) *abort_s = 1;
+          tc_fence_after();
+          const uint32_t v0 = smem_u32(ring + st * DLayout::kStage + DLayout::kTile);
+#pragma unroll
+          for (int k = 0; k < kKeys / 16; ++k) {
+            const int box = k >> 2, kk = k & 3;
+            mma_bf16_ss(tO, desc_mn_sw128(v0 + k * 16 * 128, kKeys * 128),
+                        desc_k_sw128(p0 + box * (kMaxRows * 128) + kk * 32), idO, (j > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(o_done);
+          mma_commit(&kv_empty[st]);
+        }
+        it += T;
+        js += T;
+      }
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0, kWaitPolls)) *abort_s = 1;
+    }
   } else {
-    // ---------------------------------------------------------------- compute
-    uint32_t it = 0;
-    const int dp = tid & 63, kh = tid >> 6;  // P V: output pair dp (dims 2dp, 2dp+1), key half kh
+    // ---------------------------------------------------------------- softmax / output
+    const int q = warp & 3;
+    const int r_lane = q * 32 + lane;               // this thread's TMEM lane: key of S^T, dim of O^T
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const int et = tid - 64;                        // 0..127
+    uint32_t it = 0, js = 0;
     for (int64_t u = blockIdx.x; u < p.units; u += gridDim.x) {
       const int s = (int)(u % p.S);
       const int64_t bg = u / p.S;
       const int g = (int)(bg % p.Hkv);
       const int64_t b = bg / p.Hkv;
+      const int t0 = s * p.tps, t_end = min((s + 1) * p.tps, p.NM + p.NL);
+      const int T = t_end - t0;
       int M = __ldg(p.mem_len + b);
       if (M < 0 || M > p.Mmax) {
-        if (tid == 0 && s == 0 && g == 0) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
+        if (et == 0 && s == 0 && g == 0) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
         M = M < 0 ? 0 : p.Mmax;
       }
-      // Q rows (row r = token r / G, head g * G + r % G), fp32, scaled into the log2 domain
-      bar_compute();
-      for (int i = tid; i < R * kDH; i += kCompute) {
-        const int r = i / kDH, col = i - r * kDH;
-        const int t = r / p.G, h = g * p.G + r % p.G;
-        q_s[i] = __bfloat162float(p.Q[((b * p.Tq + t) * p.Hq + h) * (int64_t)kDH + col]) * p.scale_log2;
+      // Q rows into the swizzled K-major tile (rows past R are zero): row r = token r / G, head g*G + r % G
+      for (int i = et; i < kMaxRows * (kDH / 8); i += 128) {
+        const int r = i / (kDH / 8), c8 = (i % (kDH / 8)) * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < p.R) {
+          const int t = r / p.G, h = g * p.G + r % p.G;
+          v = __ldg(reinterpret_cast<const uint4*>(p.Q + ((b * p.Tq + t) * p.Hq + h) * (int64_t)kDH + c8));
+        }
+        *reinterpret_cast<uint4*>(Qs + sw128_off(r, c8, kMaxRows)) = v;
       }
-      bar_compute();
-      float m_run[kMaxRows], l_run[kMaxRows], o0[kMaxRows], o1[kMaxRows];
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(q_ready);
+      float m_run[kMaxRows], l_run[kMaxRows];
 #pragma unroll
       for (int r = 0; r < kMaxRows; ++r) {
         m_run[r] = -INFINITY;
         l_run[r] = 0.f;
-        o0[r] = o1[r] = 0.f;
       }
-      const int t_end = min((s + 1) * p.tps, p.NM + p.NL);
-      for (int t = s * p.tps; t < t_end; ++t, ++it) {
-        const uint32_t st = it % kStages, round = it / kStages;
-        if (!*abort_s) {
-          const bool got = __all_sync(0xffffffffu, mbar_wait(&full[st], round & 1, kWaitPolls));
-          if (!got) *abort_s = 1;
-        }
-        const uint8_t* Kt = ring + st * DLayout::kStage;
-        const uint8_t* Vt = Kt + DLayout::kTile;
-        // -------- Q K^T: lane owns key kr = 32 * warp + lane
-        const int kr = 32 * warp + lane;
-        const bool mem = t < p.NM;
-        const int key_base = mem ? t * kKeys : (t - p.NM) * kKeys;
+      for (int j = 0; j < T; ++j) {
+        const int t = t0 + j;
+        const uint32_t sb = (js + j) & 1, use = (js + j) >> 1;
+        if (!*abort_s && !__all_sync(0xffffffffu, mbar_wait(&s_full[sb], use & 1, kWaitPolls))) *abort_s = 1;
+        tc_fence_after();
         float sc[kMaxRows];
-#pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) sc[r] = 0.f;
-#pragma unroll 4
-        for (int ch = 0; ch < kDH / 8; ++ch) {
-          const int box = ch >> 3, c16 = ch & 7;
-          const uint4 kv = *reinterpret_cast<const uint4*>(Kt + box * (kKeys * 128) + kr * 128 +
-                                                           ((c16 ^ (kr & 7)) << 4));
-          float k8[8];
-          unpack(kv, k8);
-#pragma unroll
-          for (int r = 0; r < kMaxRows; ++r) {
-            if (r < R) {
-              const float4 qa = *reinterpret_cast<const float4*>(q_s + r * kDH + ch * 8);
-              const float4 qb = *reinterpret_cast<const float4*>(q_s + r * kDH + ch * 8 + 4);
-              sc[r] += qa.x * k8[0] + qa.y * k8[1] + qa.z * k8[2] + qa.w * k8[3] + qb.x * k8[4] + qb.y * k8[5] +
-                       qb.z * k8[6] + qb.w * k8[7];
-            }
-          }
-        }
-        // mask: memory rows past mem_len, local rows past each row's causal position
-        const int key = key_base + kr;
+        tmem_ld16(tS + sb * 16 + lane_off, sc);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s_free[sb]);
+        // mask; scale into the log2 domain
+        const bool mem = t < p.NM;
+        const int key = (mem ? t : t - p.NM) * kKeys + r_lane;
 #pragma unroll
         for (int r = 0; r < kMaxRows; ++r) {
-          const int pos = p.Lloc - p.Tq + r / p.G;
-          const bool vis = r < R && (mem ? key < M : key <= pos);
-          sc[r] = vis ? sc[r] : -INFINITY;
+          const bool vis = r < p.R && (mem ? key < M : key <= p.Lloc - p.Tq + r / p.G);
+          sc[r] = vis ? sc[r] * p.scale_log2 : -INFINITY;
         }
-        // tile max per row: warp reduce, then across the 4 warps through shared memory
+        // column maxima over the tile's 128 keys
+        float mx[kMaxRows];
 #pragma unroll
         for (int r = 0; r < kMaxRows; ++r) {
           float v = sc[r];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0 && r < R) red_s[warp * kMaxRows + r] = v;
+          mx[r] = v;
         }
-        bar_compute();
+        if (lane == 0) {
+#pragma unroll
+          for (int r = 0; r < kMaxRows; r += 4)
+            *reinterpret_cast<float4*>(red_s + q * kMaxRows + r) = make_float4(mx[r], mx[r + 1], mx[r + 2], mx[r + 3]);
+        }
+        bar_softmax();
+        bool grow = false;
         float corr[kMaxRows];
 #pragma unroll
         for (int r = 0; r < kMaxRows; ++r) {
-          if (r < R) {
-            const float mt = fmaxf(fmaxf(red_s[r], red_s[kMaxRows + r]), fmaxf(red_s[2 * kMaxRows + r], red_s[3 * kMaxRows + r]));
-            const float mn = fmaxf(m_run[r], mt);
-            corr[r] = mn == -INFINITY ? 1.f : fast_exp2(m_run[r] - mn);
-            m_run[r] = mn;
-            const float pv = mn == -INFINITY ? 0.f : fast_exp2(sc[r] - mn);
-            p_s[kr * kMaxRows + r] = pv;
-            l_run[r] = l_run[r] * corr[r] + pv;  // this thread's keys only; summed at the end
-          } else {
-            corr[r] = 1.f;
+          const float mt = fmaxf(fmaxf(red_s[r], red_s[kMaxRows + r]), fmaxf(red_s[2 * kMaxRows + r], red_s[3 * kMaxRows + r]));
+          corr[r] = 1.f;
+          if (mt > m_run[r] + kRescaleLog2) {  // same decision in every thread
+            corr[r] = m_run[r] == -INFINITY ? 0.f : fast_exp2(m_run[r] - mt);
+            m_run[r] = mt;
+            grow = true;
           }
         }
-        bar_compute();
-        // -------- P V: thread owns dims (2dp, 2dp+1) over keys [64 kh, 64 kh + 64)
-        const int box = dp >> 5, c16 = (dp & 31) >> 2, w2 = dp & 3;  // 16-byte chunk and 32-bit word
+        bar_softmax();  // red_s is rewritten next tile
+        float pr[kMaxRows];
 #pragma unroll
         for (int r = 0; r < kMaxRows; ++r) {
-          o0[r] *= corr[r];
-          o1[r] *= corr[r];
+          pr[r] = sc[r] == -INFINITY ? 0.f : fast_exp2(sc[r] - m_run[r]);
+          l_run[r] = l_run[r] * corr[r] + pr[r];
         }
-#pragma unroll 4
-        for (int j = 0; j < 64; ++j) {
-          const int kk = kh * 64 + j;
-          const uint32_t vw = *reinterpret_cast<const uint32_t*>(Vt + box * (kKeys * 128) + kk * 128 +
-                                                                 ((c16 ^ (kk & 7)) << 4) + w2 * 4);
-          const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xffff0000u);
+        // P V of the previous tile must be done before P is overwritten or O rescaled
+        if (j > 0 && !*abort_s && !__all_sync(0xffffffffu, mbar_wait(o_done, (it + j - 1) & 1, kWaitPolls)))
+          *abort_s = 1;
+        if (j > 0 && grow) {
+          tc_fence_after();
+          float o[16];
+          tmem_ld16(tO + lane_off, o);
+          tmem_ld_wait();
+          uint32_t w[16];
 #pragma unroll
-          for (int r4 = 0; r4 < kMaxRows; r4 += 4) {
-            if (r4 < R) {
-              const float4 pp = *reinterpret_cast<const float4*>(p_s + kk * kMaxRows + r4);
-              o0[r4] += pp.x * v0;
-              o1[r4] += pp.x * v1;
-              o0[r4 + 1] += pp.y * v0;
-              o1[r4 + 1] += pp.y * v1;
-              o0[r4 + 2] += pp.z * v0;
-              o1[r4 + 2] += pp.z * v1;
-              o0[r4 + 3] += pp.w * v0;
-              o1[r4 + 3] += pp.w * v1;
-            }
-          }
+          for (int r = 0; r < 16; ++r) w[r] = __float_as_uint(o[r] * corr[r]);
+          tmem_st16(tO + lane_off, w);
+          tmem_st_wait();
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r)
+          *reinterpret_cast<__nv_bfloat16*>(Ps + sw128_off(r, r_lane, kMaxRows)) = __float2bfloat16_rn(pr[r]);
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
       }
-      // -------- unit result: l summed over all threads, O over the two key halves
+      // unit result: O^T[d = r_lane][row], the row maxima and the summed weights
+      if (T > 0 && !*abort_s && !__all_sync(0xffffffffu, mbar_wait(o_done, (it + T - 1) & 1, kWaitPolls)))
+        *abort_s = 1;
+      tc_fence_after();
+      float o[16];
+      tmem_ld16(tO + lane_off, o);
+      tmem_ld_wait();
+      float* out = p.part + (size_t)u * p.R * (kDH + 2);
 #pragma unroll
       for (int r = 0; r < kMaxRows; ++r) {
         float v = l_run[r];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0 && r < R) red_s[warp * kMaxRows + r] = v;
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) red_s[q * kMaxRows + r] = v;
+        if (r < p.R) out[r * (kDH + 2) + 2 + r_lane] = T > 0 ? o[r] : 0.f;
       }
-      if (kh == 1) {
-#pragma unroll
-        for (int r = 0; r < kMaxRows; ++r)
-          if (r < R) {
-            o_s[(dp * kMaxRows + r) * 2] = o0[r];
-            o_s[(dp * kMaxRows + r) * 2 + 1] = o1[r];
-          }
-      }
-      bar_compute();
-      float* out = p.part + (size_t)u * R * (kDH + 2);
-      if (kh == 0) {
-#pragma unroll
-        for (int r = 0; r < kMaxRows; ++r)
-          if (r < R) {
-            float2 w;
-            w.x = o0[r] + o_s[(dp * kMaxRows + r) * 2];
-            w.y = o1[r] + o_s[(dp * kMaxRows + r) * 2 + 1];
-            *reinterpret_cast<float2*>(out + r * (kDH + 2) + 2 + 2 * dp) = w;
-          }
-      }
-      if (tid < R) {
-        // every thread holds the same running max per row
+      bar_softmax();
+      if (et < p.R) {
         float m = -INFINITY;
 #pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) m = r == tid ? m_run[r] : m;
-        out[tid * (kDH + 2)] = m;
-        out[tid * (kDH + 2) + 1] =
-            red_s[tid] + red_s[kMaxRows + tid] + red_s[2 * kMaxRows + tid] + red_s[3 * kMaxRows + tid];
+        for (int r = 0; r < kMaxRows; ++r) m = r == et ? m_run[r] : m;
+        out[et * (kDH + 2)] = m;
+        out[et * (kDH + 2) + 1] = red_s[et] + red_s[kMaxRows + et] + red_s[2 * kMaxRows + et] + red_s[3 * kMaxRows + et];
       }
+      bar_softmax();
+      tc_fence_before();
+      it += T;
+      js += T;
     }
   }
+  tc_fence_before();
   __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, DLayout::kTmemCols);
+  }
   if (tid == 0 && *abort_s) raise_flag(p.err_flag, MSA_FLAG_TIMEOUT);
 }
 

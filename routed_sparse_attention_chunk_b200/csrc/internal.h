@@ -36,7 +36,7 @@ struct RouteArgs {
   const float* kr_rnorm;
   const int64_t* doc_chunk_off;
   int64_t D, C;
-  uint32_t* doc_key;  // [B, D] ordered keys, zeroed by the launcher
+  uint32_t* doc_key;  // [B, D] ordered keys followed by [B] top-k counters, zeroed by the launcher
   float* rq;          // workspace [B * Tq, Hr]: 1 / ||Qr|| per row and head
   int32_t* chunk_doc; // workspace [C]: owning document of every chunk
   int32_t* err_flag;
@@ -49,7 +49,8 @@ struct TopkArgs {
   const uint32_t* doc_key;
   int64_t B, D;
   int k;
-  uint64_t* cand;  // workspace [B, nslice, k]
+  uint64_t* cand;      // workspace [B, nslice, k]
+  uint32_t* counters;  // workspace [B], zero on entry (the routing launcher clears it); left zero
   int nslice;
   int32_t* topk_idx;
   float* topk_score;

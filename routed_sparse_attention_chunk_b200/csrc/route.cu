@@ -153,7 +153,8 @@ __global__ void chunk_doc_kernel(const int64_t* __restrict__ off, int64_t D, int
 }
 
 cudaError_t launch_route(msa_dtype dt, const RouteArgs& a, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(a.doc_key, 0, sizeof(uint32_t) * a.B * a.D, s);
+  // document keys and the top-k counters that follow them start at zero
+  cudaError_t e = cudaMemsetAsync(a.doc_key, 0, sizeof(uint32_t) * (a.B * a.D + a.B), s);
   if (e != cudaSuccess) return e;
   if (a.C > 0) {
     const int64_t blocks = (a.C + 255) / 256;

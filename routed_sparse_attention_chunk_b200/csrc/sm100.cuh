@@ -152,9 +152,22 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t smem_addr) {
 // K-major, shape M x N: D format in bits 4-5 (1 = f32), A format 7-9 and B
 // format 10-12 (1 = bf16), transpose bits 15 / 16 (0 = K-major), N >> 3 in
 // 17-22, M >> 4 in 24-28.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major = false) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major = false, bool a_mn_major = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor for an MN-major operand in 128-byte swizzle:
+// rows of 128 bytes along M (or N), consecutive K rows 128 bytes apart, groups
+// of 8 K rows 1024 bytes apart, and 64-element M/N blocks `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3fffu);
+  d |= (uint64_t)((lbo >> 4) & 0x3fffu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
 }
 
 }  // namespace sm100

@@ -7,12 +7,13 @@
 // so that one unsigned comparison orders by score descending and, for equal
 // scores, by lower document index first; padding is key 0, below every real key.
 //
-// Two passes of the same block routine: pass 1 splits each row into slices and
-// keeps each slice's top-k; pass 2 merges the slices' candidates.  The block
-// routine streams its input through shared memory in blocks of kSortN keys,
-// keeping the running top-k at the front, and sorts each block with a bitonic
-// network.  The top-k of a union is contained in the union of the parts'
-// top-k, so the result is exact.
+// One launch, grid (slices, B).  Every CTA streams its slice of the row through
+// shared memory in blocks, keeping the running top-k at the front and sorting
+// each block with a bitonic network sized to the block.  The slice's top-k goes
+// to the workspace; the last CTA of the row to finish (an atomic counter, no
+// waiting) merges the slices' candidates the same way and writes the result.
+// The top-k of a union is contained in the union of the parts' top-k, so the
+// result is exact.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,10 +23,17 @@ namespace {
 constexpr int kSortN = 2048;
 constexpr int kSortThreads = 1024;
 
-__device__ __forceinline__ void bitonic_desc(uint64_t* s) {
-  for (int size = 2; size <= kSortN; size <<= 1) {
+__device__ __forceinline__ int next_pow2(int x) {
+  int n = 1;
+  while (n < x) n <<= 1;
+  return n;
+}
+
+// Sort s[0, n) descending (n a power of two <= kSortN).
+__device__ void bitonic_desc(uint64_t* s, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < kSortN / 2; i += blockDim.x) {
+      for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
         const int pos = 2 * i - (i & (stride - 1));
         const int par = pos + stride;
         const bool desc = (pos & size) == 0;
@@ -40,49 +48,55 @@ __device__ __forceinline__ void bitonic_desc(uint64_t* s) {
   }
 }
 
-// FROM_DOC: the input is the [B, D] document key array (pass 1); otherwise the
-// [B, nin] candidate keys of pass 1 (pass 2).
-template <bool FROM_DOC>
-__global__ void __launch_bounds__(kSortThreads)
-topk_kernel(const uint32_t* __restrict__ doc_key, const uint64_t* __restrict__ cand_in,
-            int64_t nin, int k, int nslice, uint64_t* __restrict__ cand_out,
-            int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
-  __shared__ uint64_t s[kSortN];
-  const int64_t b = blockIdx.y;
-  const int slice = blockIdx.x;
-  const int64_t per = (nin + nslice - 1) / nslice;
-  const int64_t lo = (int64_t)slice * per;
-  const int64_t hi = min(nin, lo + per);
-
+// Top-k of n keys produced by load(i), i < n, left sorted in s[0, k).
+template <typename Load>
+__device__ void block_topk(uint64_t* s, int64_t n, int k, Load load) {
   for (int i = threadIdx.x; i < k; i += blockDim.x) s[i] = 0ull;
-  const int fresh = kSortN - k;
-  for (int64_t base = lo; base < hi || base == lo; base += fresh) {
+  const int fresh_max = kSortN - k;
+  for (int64_t base = 0; base < n || base == 0; base += fresh_max) {
+    const int fresh = (int)min((int64_t)fresh_max, max((int64_t)0, n - base));
+    const int m = next_pow2(max(k + fresh, 2));
     __syncthreads();
-    for (int i = threadIdx.x; i < fresh; i += blockDim.x) {
-      const int64_t x = base + i;
-      uint64_t key = 0ull;
-      if (x < hi) {
-        if (FROM_DOC)
-          key = ((uint64_t)__ldg(doc_key + b * nin + x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)x);
-        else
-          key = __ldg(cand_in + b * nin + x);
-      }
-      s[k + i] = key;
-    }
+    for (int i = threadIdx.x; i < m - k; i += blockDim.x) s[k + i] = i < fresh ? load(base + i) : 0ull;
     __syncthreads();
-    bitonic_desc(s);
-    if (base >= hi) break;
+    bitonic_desc(s, m);
+    if (base + fresh >= n) break;
   }
   __syncthreads();
-  if (cand_out) {
-    for (int i = threadIdx.x; i < k; i += blockDim.x)
-      cand_out[(b * nslice + slice) * k + i] = s[i];
-  } else {
-    for (int i = threadIdx.x; i < k; i += blockDim.x) {
-      const uint64_t key = s[i];
-      out_idx[b * k + i] = (int32_t)(0xffffffffu - (uint32_t)(key & 0xffffffffu));
-      if (out_score) out_score[b * k + i] = key_to_float((uint32_t)(key >> 32));
-    }
+}
+
+__global__ void __launch_bounds__(kSortThreads)
+topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, uint64_t* cand,
+            uint32_t* counters, int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
+  __shared__ uint64_t s[kSortN];
+  __shared__ int last;
+  const int64_t b = blockIdx.y;
+  const int slice = blockIdx.x;
+  const int64_t per = (D + nslice - 1) / nslice;
+  const int64_t lo = (int64_t)slice * per;
+  const int64_t n = max((int64_t)0, min(D, lo + per) - lo);
+  const uint32_t* row = doc_key + b * D;
+  block_topk(s, n, k, [&](int64_t i) -> uint64_t {
+    const int64_t x = lo + i;
+    return ((uint64_t)__ldg(row + x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)x);
+  });
+  if (nslice > 1) {
+    // publish this slice's candidates; the last CTA of the row merges them
+    for (int i = threadIdx.x; i < k; i += blockDim.x) cand[(b * nslice + slice) * k + i] = s[i];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(counters + b, 1u) == (unsigned)(nslice - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const uint64_t* c = cand + b * nslice * k;
+    block_topk(s, (int64_t)nslice * k, k, [&](int64_t i) -> uint64_t { return __ldcg(c + i); });
+    if (threadIdx.x == 0) counters[b] = 0u;  // ready for the next call on this workspace
+  }
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    const uint64_t key = s[i];
+    out_idx[b * k + i] = (int32_t)(0xffffffffu - (uint32_t)(key & 0xffffffffu));
+    if (out_score) out_score[b * k + i] = key_to_float((uint32_t)(key >> 32));
   }
 }
 
@@ -94,6 +108,7 @@ __global__ void decode_scores_kernel(const uint32_t* __restrict__ key, int64_t n
 }  // namespace
 
 int topk_num_slices(int64_t D, int k) {
+  // slices of at most one sort block; capped so the merge stays a few blocks
   const int64_t fresh = kSortN - k;
   int64_t n = (D + fresh - 1) / fresh;
   if (n < 1) n = 1;
@@ -109,18 +124,9 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
     count_launch();
     decode_scores_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, s>>>(a.doc_key, n, a.doc_scores);
   }
-  if (a.nslice == 1) {
-    count_launch();
-    topk_kernel<true><<<dim3(1, (unsigned)a.B), kSortThreads, 0, s>>>(
-        a.doc_key, nullptr, a.D, a.k, 1, nullptr, a.topk_idx, a.topk_score);
-    return cudaGetLastError();
-  }
   count_launch();
-  topk_kernel<true><<<dim3(a.nslice, (unsigned)a.B), kSortThreads, 0, s>>>(
-      a.doc_key, nullptr, a.D, a.k, a.nslice, a.cand, nullptr, nullptr);
-  count_launch();
-  topk_kernel<false><<<dim3(1, (unsigned)a.B), kSortThreads, 0, s>>>(
-      nullptr, a.cand, (int64_t)a.nslice * a.k, a.k, 1, nullptr, a.topk_idx, a.topk_score);
+  topk_kernel<<<dim3(a.nslice, (unsigned)a.B), kSortThreads, 0, s>>>(a.doc_key, a.D, a.k, a.nslice, a.cand,
+                                                                      a.counters, a.topk_idx, a.topk_score);
   return cudaGetLastError();
 }
 
