@@ -62,8 +62,10 @@ struct Layout {
   static constexpr int kStage = kA + kB;
   static constexpr int kStages = (200 * 1024) / kStage > 6 ? 6 : (200 * 1024) / kStage;
   static constexpr int kRq = 8 * 8 * (N / 2) * 4;         // per epilogue warp: rq of its columns, Hr <= 8
+  static constexpr int kTr = 8 * 32 * 17 * 4;              // per epilogue warp: 32 chunks x 16 columns (+1 pad)
   static constexpr int kBar = 8 * (2 * kStages + 5) + 16;
-  static constexpr int kSmem = 1024 + kStages * kStage + kRq + kBar;
+  static constexpr int kSmem = 1024 + kStages * kStage + kRq + kTr + kBar;
+  static_assert(kSmem <= 232448, "shared memory of one CTA");
   static constexpr uint32_t kTmemCols = 2 * N;            // two accumulators of N fp32 columns
 };
 
@@ -90,7 +92,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
   float* rq_s = reinterpret_cast<float*>(smem + S * L::kStage);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * L::kStage + L::kRq);
+  float* tr_s = reinterpret_cast<float*>(smem + S * L::kStage + L::kRq);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * L::kStage + L::kRq + L::kTr);
   uint64_t* full = bars;              // [S]   TMA -> MMA
   uint64_t* empty = bars + S;         // [S]   MMA -> TMA
   uint64_t* accf = bars + 2 * S;      // [2]   MMA -> epilogue
@@ -246,11 +249,36 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           if (j < nvalid) m = fmaxf(m, S_[j]);
         doc_max_atomic(m * invHr, doc, lane, p.doc_key + (int64_t)b_first * p.D);
       } else {
+        // The columns belong to several queries (e.g. one token per query in
+        // decode).  Transpose 16 columns at a time through shared memory so
+        // that lane (16 * half + j) owns column j for the chunks of its half of
+        // the warp, then walk those chunks in order: the document boundaries are
+        // the same for every lane, so the walk is warp-uniform and a document
+        // segment ends in one atomicMax per column.  A document that straddles
+        // the two halves gets two atomics, which max-combine.
+        float* tr = tr_s + (warp - 2) * 32 * 17;
+        const int hf = lane >> 4, jl = lane & 15;
 #pragma unroll
-        for (int j = 0; j < NH; ++j) {
-          if (j < nvalid) {
-            const int b = (r0 + j) / p.Tq;
-            doc_max_atomic(S_[j] * invHr, doc, lane, p.doc_key + (int64_t)b * p.D);
+        for (int h0 = 0; h0 < NH; h0 += 16) {
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) tr[lane * 17 + j] = S_[h0 + j];
+          __syncwarp();
+          const bool colv = h0 + jl < nvalid;
+          const int b = colv ? (r0 + h0 + jl) / p.Tq : 0;
+          uint32_t* keys = p.doc_key + (int64_t)b * p.D;
+          int cur = __shfl_sync(0xffffffffu, doc, 16 * hf);
+          float m = -INFINITY;
+#pragma unroll
+          for (int ii = 0; ii < 16; ++ii) {
+            const int i = 16 * hf + ii;
+            m = fmaxf(m, tr[i * 17 + jl]);
+            const int nd = ii + 1 < 16 ? __shfl_sync(0xffffffffu, doc, i + 1) : -2;
+            if (nd != cur) {
+              if (colv && cur >= 0) atomicMax(keys + cur, float_to_key(m * invHr));
+              m = -INFINITY;
+              cur = nd;
+            }
           }
         }
       }
