@@ -11,8 +11,11 @@
 //     position (bottom-right aligned: token i sits at Lloc - Tq + i);
 //   * S = Q K^T by tcgen05.mma into one of two TMEM buffers (the tensor core
 //     computes S_{j+1} while the softmax warps work on S_j), P = exp2(S - m) in
-//     bf16 written to shared memory in the swizzled K-major layout, and
-//     O += P V with V read MN-major straight from its TMA tile;
+//     bf16 written to one of two shared-memory buffers in the swizzled K-major
+//     layout, and O += P V with V read MN-major straight from its TMA tile;
+//   * K and V tiles have separate two-deep stages: K_j is released when S_j is
+//     done and V_j when PV_j is, so the next K load never waits behind a PV,
+//     and with two P buffers the softmax of tile j+1 does not wait for PV_j;
 //   * the running max is only moved (and O rescaled in TMEM) when it grows by
 //     more than 2^8, so most tiles skip the rescale; the final 1/l and the
 //     log-sum-exp use the same max, which keeps the result exact.
@@ -48,12 +51,12 @@ template <int DH>
 struct ALayout {
   static constexpr int kBoxes = DH / 64;
   static constexpr int kQ = kRows * DH * 2;
-  static constexpr int kK = kKeys * DH * 2;
-  static constexpr int kStage = 2 * kK;  // K then V
+  static constexpr int kK = kKeys * DH * 2;  // one K (or V) tile
   static constexpr int kP = kRows * kKeys * 2;
-  static constexpr int kBar = 8 * 16;
-  static constexpr int kSmem = 1024 + kQ + 2 * kStage + kP + kBar;
+  static constexpr int kBar = 8 * 24;
+  static constexpr int kSmem = 1024 + kQ + 4 * kK + 2 * kP + kBar;  // Q, K[2], V[2], P[2]
   static constexpr uint32_t kTmemCols = 512;  // S0, S1 (128 each), O (DH)
+  static_assert(kSmem <= 232448, "shared memory of one CTA");
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -75,18 +78,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Qs = smem;
-  uint8_t* KV = Qs + L::kQ;                  // [2 stages][K, V]
-  uint8_t* Ps = KV + 2 * L::kStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Ps + L::kP);
+  uint8_t* Ks = Qs + L::kQ;        // [2] K tiles
+  uint8_t* Vs = Ks + 2 * L::kK;    // [2] V tiles
+  uint8_t* Ps = Vs + 2 * L::kK;    // [2] P tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Ps + 2 * L::kP);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* o_done = bars + 10;
-  uint64_t* drain = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* k_full = bars + 1;    // [2] TMA -> MMA
+  uint64_t* k_empty = bars + 3;   // [2] S MMA done -> TMA
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2] PV MMA done -> TMA
+  uint64_t* s_full = bars + 9;    // [2] S MMA done -> softmax
+  uint64_t* s_free = bars + 11;   // [2] S in registers -> MMA
+  uint64_t* p_full = bars + 13;   // [2] P written -> MMA
+  uint64_t* p_free = bars + 15;   // [2] PV MMA done -> softmax (P buffer free, O up to date)
+  uint64_t* drain = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // longest blocks first: block index 0 takes the last query block
@@ -107,13 +113,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&p_free[i], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -130,6 +138,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
+    // K and V tiles have their own stages: K_j is free once S_j is done, V_j
+    // once PV_j is, and the tensor core runs S_{j+1} before PV_j, so the loads
+    // go K0, K1, V0, K2, V1, K3, ... in the order their stages free up.
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       mbar_arrive_expect_tx(q_full, L::kQ);
@@ -138,31 +149,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int dc = 0; dc < L::kBoxes; ++dc)
           tma_load_2d(Qs + dc * (kRows * 128) + hh * p.TB * 128, &tmQ, (g * p.G + hh) * DH + dc * 64,
                       b * p.Tq + t0, q_full);
-      int j = 0;
-      for (; j < T; ++j) {
+      auto load = [&](int j, bool is_v) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1, kWaitPolls)) {
-          timed_out = true;
-          break;
-        }
-        uint8_t* Kd = KV + st * L::kStage;
-        uint8_t* Vd = Kd + L::kK;
-        mbar_arrive_expect_tx(&kv_full[st], L::kStage);
+        uint64_t* empty = is_v ? &v_empty[st] : &k_empty[st];
+        uint64_t* full = is_v ? &v_full[st] : &k_full[st];
+        if (!mbar_wait(empty, ((j >> 1) & 1) ^ 1, kWaitPolls)) return false;
+        uint8_t* dst = (is_v ? Vs : Ks) + st * L::kK;
+        mbar_arrive_expect_tx(full, L::kK);
         const bool mem = j < NM;
-        const CUtensorMap* mk = mem ? &tmKm : &tmKl;
-        const CUtensorMap* mv = mem ? &tmVm : &tmVl;
+        const CUtensorMap* map = is_v ? (mem ? &tmVm : &tmVl) : (mem ? &tmKm : &tmKl);
         const int y = mem ? b * p.Mmax + j * kKeys : b * p.Lloc + (j - NM) * kKeys;
 #pragma unroll
-        for (int dc = 0; dc < L::kBoxes; ++dc) {
-          tma_load_2d(Kd + dc * (kKeys * 128), mk, g * DH + dc * 64, y, &kv_full[st]);
-          tma_load_2d(Vd + dc * (kKeys * 128), mv, g * DH + dc * 64, y, &kv_full[st]);
+        for (int dc = 0; dc < L::kBoxes; ++dc) tma_load_2d(dst + dc * (kKeys * 128), map, g * DH + dc * 64, y, full);
+        return true;
+      };
+      int nk = 0, nv = 0;
+      bool ok = true;
+      while (ok && nk < 2 && nk < T) {
+        if (!(ok = load(nk, false))) break;
+        ++nk;
+      }
+      for (int j = 0; ok && j < T; ++j) {
+        if (!(ok = load(j, true))) break;
+        ++nv;
+        if (nk < T) {
+          if (!(ok = load(nk, false))) break;
+          ++nk;
         }
       }
+      if (!ok) timed_out = true;
       // drain the copies this thread issued
       if (!mbar_wait(q_full, 0, kWaitPolls)) timed_out = true;
-      for (int st = 0; st < 2 && st < j; ++st) {
-        const int last = (j - 1 - st) / 2 * 2 + st;
-        if (!mbar_wait(&kv_full[st], (last >> 1) & 1, kWaitPolls)) timed_out = true;
+      for (int st = 0; st < 2; ++st) {
+        if (st < nk && !mbar_wait(&k_full[st], (((nk - 1 - st) / 2 * 2 + st) >> 1) & 1, kWaitPolls)) timed_out = true;
+        if (st < nv && !mbar_wait(&v_full[st], (((nv - 1 - st) / 2 * 2 + st) >> 1) & 1, kWaitPolls)) timed_out = true;
       }
     }
   } else if (warp == 1) {
@@ -170,13 +190,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(kRows, kKeys);
       constexpr uint32_t idO = idesc_bf16_f32(kRows, DH, /*b_mn_major=*/true);
-      const uint32_t q0 = smem_u32(Qs), p0 = smem_u32(Ps);
+      const uint32_t q0 = smem_u32(Qs);
       auto issue_S = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(&kv_full[st], (j >> 1) & 1, kWaitPolls)) return false;
+        if (!mbar_wait(&k_full[st], (j >> 1) & 1, kWaitPolls)) return false;
         if (!mbar_wait(&s_free[st], ((j >> 1) & 1) ^ 1, kWaitPolls)) return false;
         tc_fence_after();
-        const uint32_t k0 = smem_u32(KV + st * L::kStage);
+        const uint32_t k0 = smem_u32(Ks + st * L::kK);
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
           const int box = k >> 2, kk = k & 3;
@@ -184,28 +204,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                       desc_k_sw128(k0 + box * kKeys * 128 + kk * 32), idS, k > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[st]);
+        mma_commit(&k_empty[st]);
         return true;
       };
       bool ok = mbar_wait(q_full, 0, kWaitPolls) && issue_S(0);
       for (int j = 0; ok && j < T; ++j) {
+        const int st = j & 1;
         if (j + 1 < T && !issue_S(j + 1)) {
           ok = false;
           break;
         }
-        if (!mbar_wait(p_full, j & 1, kWaitPolls)) {
+        if (!mbar_wait(&p_full[st], (j >> 1) & 1, kWaitPolls) || !mbar_wait(&v_full[st], (j >> 1) & 1, kWaitPolls)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t v0 = smem_u32(KV + (j & 1) * L::kStage + L::kK);
+        const uint32_t p0 = smem_u32(Ps + st * L::kP);
+        const uint32_t v0 = smem_u32(Vs + st * L::kK);
 #pragma unroll
         for (int k = 0; k < kKeys / 16; ++k) {
           const int box = k >> 2, kk = k & 3;
           mma_bf16_ss(tO, desc_k_sw128(p0 + box * kRows * 128 + kk * 32),
                       desc_mn_sw128(v0 + k * 16 * 128, kKeys * 128), idO, (j > 0 || k > 0) ? 1u : 0u);
         }
-        mma_commit(o_done);
-        mma_commit(&kv_empty[j & 1]);
+        mma_commit(&p_free[st]);
+        mma_commit(&v_empty[st]);
       }
       if (!ok) timed_out = true;
       mma_commit(drain);
@@ -219,8 +242,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int t = t0 + tl;
     const int pos = p.Lloc - p.Tq + t;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    float m_run = -INFINITY, l_run = 0.f;
-    uint8_t* prow = Ps + r * 128;
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;  // running max in the scaled log2 domain
     const int sw = r & 7;
     for (int j = 0; j < T; ++j) {
       const int st = j & 1;
@@ -236,17 +259,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&s_free[st]);
-      // mask and row max (log2 domain)
+      // keys [0, lim) of this tile are visible to this row; most tiles are whole
       const bool memt = j < NM;
       const int base = memt ? j * kKeys : (j - NM) * kKeys;
-      const int lim = memt ? M - base : pos - base + 1;  // keys [0, lim) of this tile are visible
-      float mt = -INFINITY;
+      const int lim = memt ? M - base : pos - base + 1;
+      float mx = -INFINITY;
+      if (__all_sync(0xffffffffu, lim >= kKeys)) {
 #pragma unroll
-      for (int c = 0; c < kKeys; ++c) {
-        s[c] = c < lim ? s[c] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[c]);
+        for (int c = 0; c < kKeys; ++c) mx = fmaxf(mx, s[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kKeys; ++c) {
+          s[c] = c < lim ? s[c] : -INFINITY;
+          mx = fmaxf(mx, s[c]);
+        }
       }
       // move the max (and rescale O) only when it grows by more than 2^8
+      const float mt = mx * sl2;
       const bool first = m_run == -INFINITY;
       const bool grow = mt > m_run + kRescaleLog2;
       float corr = 1.f;
@@ -254,12 +283,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         corr = first ? 0.f : fast_exp2(m_run - mt);
         m_run = mt;
       }
-      // P_{j-1}'s PV must be done before P_j overwrites the buffer (and before O is touched)
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, kWaitPolls))) {
-        timed_out = true;
-        break;
-      }
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O must hold every earlier PV before it is rescaled
+        const int jp = j - 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&p_free[jp & 1], (jp >> 1) & 1, kWaitPolls))) {
+          timed_out = true;
+          break;
+        }
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < DH; c += 16) {
@@ -273,14 +303,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         tmem_st_wait();
       }
+      // P buffer st was read by PV_{j-2}
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_free[st], ((j >> 1) & 1) ^ 1, kWaitPolls))) {
+        timed_out = true;
+        break;
+      }
       l_run *= corr;
+      const float nm = -m_run;
+      uint8_t* prow = Ps + st * L::kP + r * 128;
       float ls = 0.f;
 #pragma unroll
       for (int c0 = 0; c0 < kKeys; c0 += 8) {
         float e[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          e[i] = fast_exp2(s[c0 + i] - m_run);
+          e[i] = fast_exp2(fmaf(s[c0 + i], sl2, nm));
           ls += e[i];
         }
         uint4 pk = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
@@ -291,10 +328,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       l_run += ls;
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[st]);
     }
     // output: O / l, lse = (m + log2 l) ln 2
-    if (!timed_out && __all_sync(0xffffffffu, mbar_wait(o_done, (T - 1) & 1, kWaitPolls))) {
+    const int jl = T - 1;
+    if (!timed_out && __all_sync(0xffffffffu, mbar_wait(&p_free[jl & 1], (jl >> 1) & 1, kWaitPolls))) {
       tc_fence_after();
       const float inv = 1.f / l_run;
       const bool rvalid = t < p.Tq;
