@@ -7,10 +7,15 @@
 // so that one unsigned comparison orders by score descending and, for equal
 // scores, by lower document index first; padding is key 0, below every real key.
 //
-// One launch, grid (slices, B).  Every CTA streams its slice of the row through
-// shared memory in blocks, keeping the running top-k at the front and sorting
-// each block with a bitonic network sized to the block.  The slice's top-k goes
-// to the workspace; the last CTA of the row to finish (an atomic counter, no
+// One launch, grid (slices, B).  A slice of up to 32768 documents is read
+// twice, 32 keys per thread.  The k-th largest of the per-thread maxima, tau,
+// is found with a bitonic sort of those 1024 maxima; the k largest keys of the
+// slice are all >= tau (k distinct thread maxima already are), and at most k
+// threads hold a key >= tau, so at most 32 k keys survive the filter.  The
+// survivors are sorted in shared memory and the slice's top-k goes to the
+// workspace (when more than 2048 survive, which needs k > 64, the slice is
+// instead streamed through shared memory in blocks, keeping the running top-k
+// at the front).  The last CTA of the row to finish (an atomic counter, no
 // waiting) merges the slices' candidates the same way and writes the result.
 // The top-k of a union is contained in the union of the parts' top-k, so the
 // result is exact.
@@ -22,6 +27,8 @@ namespace {
 
 constexpr int kSortN = 2048;
 constexpr int kSortThreads = 1024;
+constexpr int kPer = 32;                         // keys per thread in the filter
+constexpr int kSlice = kSortThreads * kPer;      // documents per slice
 
 __device__ __forceinline__ int next_pow2(int x) {
   int n = 1;
@@ -65,21 +72,67 @@ __device__ void block_topk(uint64_t* s, int64_t n, int k, Load load) {
   __syncthreads();
 }
 
+__device__ __forceinline__ uint64_t doc_key64(uint32_t score_key, int64_t doc) {
+  return ((uint64_t)score_key << 32) | (uint64_t)(0xffffffffu - (uint32_t)doc);
+}
+
+// Top-k of keys row[lo, lo + n), n <= kSlice, left sorted in s[0, k); false
+// when more than kSortN keys pass the filter (s is then clobbered).
+__device__ bool slice_topk_filter(uint64_t* s, int* cnt, const uint32_t* row, int64_t lo, int64_t n, int k) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint64_t mx = 0ull;
+#pragma unroll 8
+  for (int m = 0; m < kPer; ++m) {
+    const int64_t i = tid + (int64_t)m * kSortThreads;
+    if (i < n) mx = max(mx, doc_key64(__ldg(row + lo + i), lo + i));
+  }
+  s[tid] = mx;
+  if (tid == 0) *cnt = 0;
+  __syncthreads();
+  bitonic_desc(s, kSortThreads);
+  const uint64_t tau = s[k - 1];
+  __syncthreads();
+  // second pass over the slice (now in L1/L2)
+#pragma unroll 4
+  for (int m = 0; m < kPer; ++m) {
+    const int64_t i = tid + (int64_t)m * kSortThreads;
+    const uint64_t key = i < n ? doc_key64(__ldg(row + lo + i), lo + i) : 0ull;
+    const bool pass = i < n && key >= tau;
+    const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+    if (bal) {
+      int base = 0;
+      if (lane == 0) base = atomicAdd(cnt, __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const int pos = base + __popc(bal & ((1u << lane) - 1u));
+      if (pass && pos < kSortN) s[pos] = key;
+    }
+  }
+  __syncthreads();
+  const int total = *cnt;
+  if (total > kSortN) return false;
+  const int m2 = next_pow2(max(total, max(k, 2)));
+  for (int i = total + tid; i < m2; i += kSortThreads) s[i] = 0ull;
+  __syncthreads();
+  bitonic_desc(s, m2);
+  return true;
+}
+
 __global__ void __launch_bounds__(kSortThreads)
 topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, uint64_t* cand,
             uint32_t* counters, int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
   __shared__ uint64_t s[kSortN];
-  __shared__ int last;
+  __shared__ int last, cnt;
   const int64_t b = blockIdx.y;
   const int slice = blockIdx.x;
   const int64_t per = (D + nslice - 1) / nslice;
   const int64_t lo = (int64_t)slice * per;
   const int64_t n = max((int64_t)0, min(D, lo + per) - lo);
   const uint32_t* row = doc_key + b * D;
-  block_topk(s, n, k, [&](int64_t i) -> uint64_t {
-    const int64_t x = lo + i;
-    return ((uint64_t)__ldg(row + x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)x);
-  });
+  // (the branch is uniform over the CTA)
+  if (n > kSlice || !slice_topk_filter(s, &cnt, row, lo, n, k)) {
+    __syncthreads();
+    block_topk(s, n, k, [&](int64_t i) -> uint64_t { return doc_key64(__ldg(row + lo + i), lo + i); });
+  }
   if (nslice > 1) {
     // publish this slice's candidates; the last CTA of the row merges them
     for (int i = threadIdx.x; i < k; i += blockDim.x) cand[(b * nslice + slice) * k + i] = s[i];
@@ -108,9 +161,9 @@ __global__ void decode_scores_kernel(const uint32_t* __restrict__ key, int64_t n
 }  // namespace
 
 int topk_num_slices(int64_t D, int k) {
-  // slices of at most one sort block; capped so the merge stays a few blocks
-  const int64_t fresh = kSortN - k;
-  int64_t n = (D + fresh - 1) / fresh;
+  // slices the filter takes whole; capped so the merge stays a few blocks
+  (void)k;
+  int64_t n = (D + kSlice - 1) / kSlice;
   if (n < 1) n = 1;
   if (n > 1024) n = 1024;
   return (int)n;

@@ -160,6 +160,54 @@ def test_topk_exact_ties_prefer_lower_index():
     assert np.array_equal(idx.cpu().numpy(), oi)   # exact: equal scores resolved by index
 
 
+def test_topk_many_slices_merge():
+    # three slices of the per-row filter plus the last-CTA merge, two query rows
+    Krb, rn, coff = _bank_case(70000, 2, 64, seed=21)
+    g = torch.Generator(device=DEV).manual_seed(12)
+    Qr = torch.randn((2, 3, 2, 64), generator=g, device=DEV).bfloat16()
+    idx, sc, ds, flag = route_on_gpu(Qr, Krb, rn, coff, 16)
+    ods = O.route(to64(Qr), to64(Krb), coff)
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    check_topk(idx.cpu().numpy(), to64(sc), ods, 16, TOL_SCORE_ABS)
+
+
+def test_topk_filter_overflow_takes_streaming_path():
+    # k = 100 over one slice of 32768 one-chunk documents.  The documents held
+    # by the first 100 threads of the filter (index mod 1024 < 100) all score
+    # high and rise with (thread, item), so several thousand keys pass the
+    # threshold and the slice falls back to the streamed block sort.
+    D, k, dr = 32768, 100, 64
+    idx_all = np.arange(D)
+    t, m = idx_all % 1024, idx_all // 1024
+    heavy = t < k
+    a = np.where(heavy, 1.0 + (t * 32 + m) / 4096.0, -1.0)
+    bank = np.zeros((D, 1, dr), dtype=np.float32)
+    bank[:, 0, 0] = a
+    bank[:, 0, 1] = 1.0
+    Krb = torch.from_numpy(bank).to(DEV).bfloat16()
+    rn = torch.empty((D, 1), dtype=torch.float32, device=DEV)
+    msa.bank_rnorm(Krb, rn)
+    coff = np.arange(D + 1, dtype=np.int64)
+    qr = np.zeros((1, 1, 1, dr), dtype=np.float32)
+    qr[..., 0] = 1.0
+    Qr = torch.from_numpy(qr).to(DEV).bfloat16()
+    idx, sc, ds, flag = route_on_gpu(Qr, Krb, rn, coff, k)
+    ods = O.route(to64(Qr), to64(Krb), coff)
+    oi, _ = O.topk(ods, k)
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    # the filter's survivor count, from the oracle's scores: keys >= the k-th
+    # largest per-thread maximum, keys ordered by (score, lower index)
+    order = np.lexsort((idx_all, -ods[0]))             # rank 0 = largest key
+    rank = np.empty(D, dtype=np.int64)
+    rank[order] = np.arange(D)
+    thread_best = np.array([rank[t == i].min() for i in range(1024)])
+    tau_rank = np.sort(thread_best)[k - 1]
+    assert int((rank <= tau_rank).sum()) > 2048
+    assert np.array_equal(idx.cpu().numpy(), oi)
+
+
 # ---------------------------------------------------------------- step 4: gather
 def test_gather_bitexact_and_flags():
     rng = np.random.default_rng(5)
