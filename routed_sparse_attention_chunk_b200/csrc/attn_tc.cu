@@ -10,12 +10,15 @@
 //     mem_len are masked), then the local rows up to the block's last causal
 //     position (bottom-right aligned: token i sits at Lloc - Tq + i);
 //   * S = Q K^T by tcgen05.mma into one of two TMEM buffers (the tensor core
-//     computes S_{j+1} while the softmax warps work on S_j), P = exp2(S - m) in
-//     bf16 written to one of two shared-memory buffers in the swizzled K-major
-//     layout, and O += P V with V read MN-major straight from its TMA tile;
-//   * K and V tiles have separate two-deep stages: K_j is released when S_j is
-//     done and V_j when PV_j is, so the next K load never waits behind a PV,
-//     and with two P buffers the softmax of tile j+1 does not wait for PV_j;
+//     computes S_{j+1} while the softmax warps work on S_j); P = exp2(S - m)
+//     is rounded to bf16 and written back over its own S tile in TMEM (two
+//     values per 32-bit column, one row per lane), and O += P V takes P as the
+//     MMA's A operand straight from tensor memory and V MN-major from its TMA
+//     tile.  The tensor core runs its MMAs in issue order, so S_{j+2} (issued
+//     after PV_j) never overwrites P_j before PV_j has read it;
+//   * K and V tiles have separate three-deep stages: K_j is released when S_j
+//     is done and V_j when PV_j is, which keeps three loads in flight against
+//     the latency of a TMA tile;
 //   * the running max is only moved (and O rescaled in TMEM) when it grows by
 //     more than 2^8, so most tiles skip the rescale; the final 1/l and the
 //     log-sum-exp use the same max, which keeps the result exact.
@@ -37,6 +40,7 @@ constexpr int kKeys = 128;   // keys per tile
 constexpr int kThreads = 192;
 constexpr uint32_t kWaitPolls = 1u << 24;
 constexpr float kRescaleLog2 = 8.0f;  // move the running max only when it grows by more than this
+constexpr int kKV = 3;                // K and V stages
 
 struct AttnTcParams {
   const int32_t* mem_len;
@@ -52,9 +56,8 @@ struct ALayout {
   static constexpr int kBoxes = DH / 64;
   static constexpr int kQ = kRows * DH * 2;
   static constexpr int kK = kKeys * DH * 2;  // one K (or V) tile
-  static constexpr int kP = kRows * kKeys * 2;
   static constexpr int kBar = 8 * 24;
-  static constexpr int kSmem = 1024 + kQ + 4 * kK + 2 * kP + kBar;  // Q, K[2], V[2], P[2]
+  static constexpr int kSmem = 1024 + kQ + 2 * kKV * kK + kBar;  // Q, K[kKV], V[kKV]
   static constexpr uint32_t kTmemCols = 512;  // S0, S1 (128 each), O (DH)
   static_assert(kSmem <= 232448, "shared memory of one CTA");
 };
@@ -63,10 +66,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 template <int DH>
@@ -78,21 +77,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Qs = smem;
-  uint8_t* Ks = Qs + L::kQ;        // [2] K tiles
-  uint8_t* Vs = Ks + 2 * L::kK;    // [2] V tiles
-  uint8_t* Ps = Vs + 2 * L::kK;    // [2] P tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Ps + 2 * L::kP);
+  uint8_t* Ks = Qs + L::kQ;          // [kKV] K tiles
+  uint8_t* Vs = Ks + kKV * L::kK;    // [kKV] V tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Vs + kKV * L::kK);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2] TMA -> MMA
-  uint64_t* k_empty = bars + 3;   // [2] S MMA done -> TMA
-  uint64_t* v_full = bars + 5;    // [2]
-  uint64_t* v_empty = bars + 7;   // [2] PV MMA done -> TMA
-  uint64_t* s_full = bars + 9;    // [2] S MMA done -> softmax
-  uint64_t* s_free = bars + 11;   // [2] S in registers -> MMA
-  uint64_t* p_full = bars + 13;   // [2] P written -> MMA
-  uint64_t* p_free = bars + 15;   // [2] PV MMA done -> softmax (P buffer free, O up to date)
-  uint64_t* drain = bars + 17;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* k_full = bars + 1;             // [kKV] TMA -> MMA
+  uint64_t* k_empty = k_full + kKV;        // [kKV] S MMA done -> TMA
+  uint64_t* v_full = k_empty + kKV;        // [kKV]
+  uint64_t* v_empty = v_full + kKV;        // [kKV] PV MMA done -> TMA
+  uint64_t* s_full = v_empty + kKV;        // [2] S MMA done -> softmax
+  uint64_t* p_full = s_full + 2;           // [2] P written over S -> MMA
+  uint64_t* p_free = p_full + 2;           // [2] PV MMA done -> softmax (O up to date)
+  uint64_t* drain = p_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // longest blocks first: block index 0 takes the last query block
@@ -112,13 +109,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kKV; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
       mbar_init(&p_full[i], 128);
       mbar_init(&p_free[i], 1);
     }
@@ -140,7 +138,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ---------------------------------------------------------------- producer
     // K and V tiles have their own stages: K_j is free once S_j is done, V_j
     // once PV_j is, and the tensor core runs S_{j+1} before PV_j, so the loads
-    // go K0, K1, V0, K2, V1, K3, ... in the order their stages free up.
+    // go K0, K1, K2, V0, K3, V1, K4, ... in the order their stages free up.
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       mbar_arrive_expect_tx(q_full, L::kQ);
@@ -150,10 +148,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tma_load_2d(Qs + dc * (kRows * 128) + hh * p.TB * 128, &tmQ, (g * p.G + hh) * DH + dc * 64,
                       b * p.Tq + t0, q_full);
       auto load = [&](int j, bool is_v) -> bool {
-        const int st = j & 1;
+        const int st = j % kKV;
         uint64_t* empty = is_v ? &v_empty[st] : &k_empty[st];
         uint64_t* full = is_v ? &v_full[st] : &k_full[st];
-        if (!mbar_wait(empty, ((j >> 1) & 1) ^ 1, kWaitPolls)) return false;
+        if (!mbar_wait(empty, ((j / kKV) & 1) ^ 1, kWaitPolls)) return false;
         uint8_t* dst = (is_v ? Vs : Ks) + st * L::kK;
         mbar_arrive_expect_tx(full, L::kK);
         const bool mem = j < NM;
@@ -165,7 +163,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       };
       int nk = 0, nv = 0;
       bool ok = true;
-      while (ok && nk < 2 && nk < T) {
+      while (ok && nk < kKV && nk < T) {
         if (!(ok = load(nk, false))) break;
         ++nk;
       }
@@ -180,9 +178,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (!ok) timed_out = true;
       // drain the copies this thread issued
       if (!mbar_wait(q_full, 0, kWaitPolls)) timed_out = true;
-      for (int st = 0; st < 2; ++st) {
-        if (st < nk && !mbar_wait(&k_full[st], (((nk - 1 - st) / 2 * 2 + st) >> 1) & 1, kWaitPolls)) timed_out = true;
-        if (st < nv && !mbar_wait(&v_full[st], (((nv - 1 - st) / 2 * 2 + st) >> 1) & 1, kWaitPolls)) timed_out = true;
+      for (int st = 0; st < kKV; ++st) {
+        // the last fill of stage st is fill (n - 1 - st) / kKV of it
+        if (st < nk && !mbar_wait(&k_full[st], ((nk - 1 - st) / kKV) & 1, kWaitPolls)) timed_out = true;
+        if (st < nv && !mbar_wait(&v_full[st], ((nv - 1 - st) / kKV) & 1, kWaitPolls)) timed_out = true;
       }
     }
   } else if (warp == 1) {
@@ -191,44 +190,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t idS = idesc_bf16_f32(kRows, kKeys);
       constexpr uint32_t idO = idesc_bf16_f32(kRows, DH, /*b_mn_major=*/true);
       const uint32_t q0 = smem_u32(Qs);
+      // S_j goes to TMEM buffer j & 1, which holds P_{j-2} until PV_{j-2} has
+      // read it; PV_{j-2} was issued earlier, and the MMAs run in issue order.
       auto issue_S = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&k_full[st], (j >> 1) & 1, kWaitPolls)) return false;
-        if (!mbar_wait(&s_free[st], ((j >> 1) & 1) ^ 1, kWaitPolls)) return false;
+        const int ks = j % kKV;
+        if (!mbar_wait(&k_full[ks], (j / kKV) & 1, kWaitPolls)) return false;
         tc_fence_after();
-        const uint32_t k0 = smem_u32(Ks + st * L::kK);
+        const uint32_t k0 = smem_u32(Ks + ks * L::kK);
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
           const int box = k >> 2, kk = k & 3;
-          mma_bf16_ss(tS0 + st * kKeys, desc_k_sw128(q0 + box * kRows * 128 + kk * 32),
+          mma_bf16_ss(tS0 + (j & 1) * kKeys, desc_k_sw128(q0 + box * kRows * 128 + kk * 32),
                       desc_k_sw128(k0 + box * kKeys * 128 + kk * 32), idS, k > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[st]);
-        mma_commit(&k_empty[st]);
+        mma_commit(&s_full[j & 1]);
+        mma_commit(&k_empty[ks]);
         return true;
       };
       bool ok = mbar_wait(q_full, 0, kWaitPolls) && issue_S(0);
       for (int j = 0; ok && j < T; ++j) {
-        const int st = j & 1;
+        const int st = j & 1, vs = j % kKV;
         if (j + 1 < T && !issue_S(j + 1)) {
           ok = false;
           break;
         }
-        if (!mbar_wait(&p_full[st], (j >> 1) & 1, kWaitPolls) || !mbar_wait(&v_full[st], (j >> 1) & 1, kWaitPolls)) {
+        if (!mbar_wait(&p_full[st], (j >> 1) & 1, kWaitPolls) || !mbar_wait(&v_full[vs], (j / kKV) & 1, kWaitPolls)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t p0 = smem_u32(Ps + st * L::kP);
-        const uint32_t v0 = smem_u32(Vs + st * L::kK);
+        const uint32_t v0 = smem_u32(Vs + vs * L::kK);
+        // A = P_j from TMEM: 16 keys of bf16 per step are 8 columns
 #pragma unroll
-        for (int k = 0; k < kKeys / 16; ++k) {
-          const int box = k >> 2, kk = k & 3;
-          mma_bf16_ss(tO, desc_k_sw128(p0 + box * kRows * 128 + kk * 32),
-                      desc_mn_sw128(v0 + k * 16 * 128, kKeys * 128), idO, (j > 0 || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < kKeys / 16; ++k)
+          mma_bf16_ts(tO, tS0 + st * kKeys + k * 8, desc_mn_sw128(v0 + k * 16 * 128, kKeys * 128), idO,
+                      (j > 0 || k > 0) ? 1u : 0u);
         mma_commit(&p_free[st]);
-        mma_commit(&v_empty[st]);
+        mma_commit(&v_empty[vs]);
       }
       if (!ok) timed_out = true;
       mma_commit(drain);
@@ -244,7 +242,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;  // running max in the scaled log2 domain
-    const int sw = r & 7;
     for (int j = 0; j < T; ++j) {
       const int st = j & 1;
       // waits are decided warp-wide so the warp-collective tcgen05 ops are never split
@@ -257,8 +254,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int c = 0; c < kKeys; c += 16) tmem_ld16(tmem + lane_off + st * kKeys + c, *reinterpret_cast<float(*)[16]>(&s[c]));
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s_free[st]);
       // keys [0, lim) of this tile are visible to this row; most tiles are whole
       const bool memt = j < NM;
       const int base = memt ? j * kKeys : (j - NM) * kKeys;
@@ -303,30 +298,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         tmem_st_wait();
       }
-      // P buffer st was read by PV_{j-2}
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_free[st], ((j >> 1) & 1) ^ 1, kWaitPolls))) {
-        timed_out = true;
-        break;
-      }
       l_run *= corr;
       const float nm = -m_run;
-      uint8_t* prow = Ps + st * L::kP + r * 128;
-      float ls = 0.f;
+      // P_j over S_j: 32 keys (16 columns of bf16 pairs) per store
+      float lsa[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c0 = 0; c0 < kKeys; c0 += 8) {
-        float e[8];
+      for (int c0 = 0; c0 < kKeys; c0 += 32) {
+        uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          e[i] = fast_exp2(fmaf(s[c0 + i], sl2, nm));
-          ls += e[i];
+        for (int i = 0; i < 16; ++i) {
+          const float e0 = fast_exp2(fmaf(s[c0 + 2 * i], sl2, nm));
+          const float e1 = fast_exp2(fmaf(s[c0 + 2 * i + 1], sl2, nm));
+          lsa[i & 3] += e0 + e1;
+          w[i] = pack_bf16x2(e0, e1);
         }
-        uint4 pk = make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
-                              pack_bf16x2(e[6], e[7]));
-        const int box = c0 >> 6, chunk = (c0 & 63) >> 3;
-        *reinterpret_cast<uint4*>(prow + box * (kRows * 128) + ((chunk ^ sw) << 4)) = pk;
+        tmem_st16(tmem + lane_off + st * kKeys + c0 / 2, w);
       }
-      l_run += ls;
-      fence_async_smem();
+      l_run += (lsa[0] + lsa[1]) + (lsa[2] + lsa[3]);
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[st]);
     }
