@@ -20,7 +20,8 @@
 
 namespace msa {
 
-cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s, bool* handled);
+bool route_tc_applies(const RouteArgs& a);
+cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s);
 
 namespace {
 
@@ -135,38 +136,66 @@ cudaError_t route_generic_t(const RouteArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-// chunk_doc[c] = the document that owns chunk c, one warp per 32 chunks; also
-// flags offsets whose last entry is not C.
-__global__ void chunk_doc_kernel(const int64_t* __restrict__ off, int64_t D, int64_t C, int32_t* __restrict__ out,
-                                 int32_t* err_flag) {
-  const int lane = threadIdx.x & 31;
-  const int64_t c0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32;
-  if (blockIdx.x == 0 && threadIdx.x == 0 && (__ldg(off) != 0 || __ldg(off + D) != C))
-    raise_flag(err_flag, MSA_FLAG_OFFSETS);
-  if (c0 >= C) return;  // whole warp
-  int doc = warp_chunk_docs(off, D, C, c0, lane);
-  if (doc >= D) {  // only reachable with offsets that do not end at C: never index past D
-    raise_flag(err_flag, MSA_FLAG_OFFSETS);
-    doc = -1;
+// One launch ahead of the scan: zero the document keys and the top-k counters
+// that follow them, map every chunk to its owning document (one warp per 32
+// chunks; offsets whose ends are not 0 and C are flagged), and for the
+// tensor-core scan the inverse norms rq[r, h] = 1 / max(||Qr[r, h]||, 1e-12)
+// of the bf16 query rows (one warp per row and head).  Blocks
+// [0, nb_zero) zero, [nb_zero, nb_zero + nb_map) map, the rest take norms.
+__global__ void __launch_bounds__(256)
+route_prelude_kernel(uint32_t* __restrict__ keys, int64_t nkeys, int nb_zero, const int64_t* __restrict__ off,
+                     int64_t D, int64_t C, int32_t* __restrict__ chunk_doc, int nb_map,
+                     const __nv_bfloat16* __restrict__ Qr, int64_t nq, int dr, float* __restrict__ rq,
+                     int32_t* err_flag) {
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int blk = blockIdx.x;
+  if (blk < nb_zero) {
+    const int64_t per = (nkeys + nb_zero - 1) / nb_zero;
+    const int64_t lo = (int64_t)blk * per, hi = min(nkeys, lo + per);
+    for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) keys[i] = 0u;
+    return;
   }
-  if (c0 + lane < C) out[c0 + lane] = doc;
+  if (blk < nb_zero + nb_map) {
+    const int64_t c0 = ((int64_t)(blk - nb_zero) * 8 + wib) * 32;
+    if (blk == nb_zero && threadIdx.x == 0 && (__ldg(off) != 0 || __ldg(off + D) != C))
+      raise_flag(err_flag, MSA_FLAG_OFFSETS);
+    if (c0 >= C) return;  // whole warp
+    int doc = warp_chunk_docs(off, D, C, c0, lane);
+    if (doc >= D) {  // only reachable with offsets that do not end at C: never index past D
+      raise_flag(err_flag, MSA_FLAG_OFFSETS);
+      doc = -1;
+    }
+    if (c0 + lane < C) chunk_doc[c0 + lane] = doc;
+    return;
+  }
+  const int64_t w = (int64_t)(blk - nb_zero - nb_map) * 8 + wib;
+  if (w >= nq) return;
+  const __nv_bfloat16* x = Qr + w * dr;
+  float ss = 0.f;
+  for (int i = lane; i < dr; i += 32) {
+    const float v = __bfloat162float(x[i]);
+    ss += v * v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) rq[w] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
 }
 
 cudaError_t launch_route(msa_dtype dt, const RouteArgs& a, cudaStream_t s) {
-  // document keys and the top-k counters that follow them start at zero
-  cudaError_t e = cudaMemsetAsync(a.doc_key, 0, sizeof(uint32_t) * (a.B * a.D + a.B), s);
+  const bool tc = dt == MSA_BF16 && route_tc_applies(a);
+  const int64_t nkeys = a.B * a.D + a.B;  // document keys, then the top-k counters
+  const int64_t zb = (nkeys + 8191) / 8192;
+  const int nb_zero = (int)(zb < 1 ? 1 : (zb > 1024 ? 1024 : zb));
+  const int nb_map = (int)((a.C + 255) / 256);
+  const int64_t nq = tc ? a.B * a.Tq * a.Hr : 0;
+  const int64_t nb_q = (nq + 7) / 8;
+  count_launch();
+  route_prelude_kernel<<<(unsigned)(nb_zero + nb_map + nb_q), 256, 0, s>>>(
+      a.doc_key, nkeys, nb_zero, a.doc_chunk_off, a.D, a.C, a.chunk_doc, nb_map,
+      reinterpret_cast<const __nv_bfloat16*>(a.Qr), nq, a.dr, a.rq, a.err_flag);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (a.C > 0) {
-    const int64_t blocks = (a.C + 255) / 256;
-    count_launch();
-    chunk_doc_kernel<<<(unsigned)blocks, 256, 0, s>>>(a.doc_chunk_off, a.D, a.C, a.chunk_doc, a.err_flag);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  if (dt == MSA_BF16) {
-    bool handled = false;
-    e = launch_route_tc(a, s, &handled);
-    if (e != cudaSuccess || handled) return e;
-  }
+  if (tc) return launch_route_tc(a, s);
   if (dt == MSA_F32)
     return a.dr == 64 ? route_generic_t<float, 64>(a, s) : route_generic_t<float, 128>(a, s);
   return a.dr == 64 ? route_generic_t<__nv_bfloat16, 64>(a, s) : route_generic_t<__nv_bfloat16, 128>(a, s);

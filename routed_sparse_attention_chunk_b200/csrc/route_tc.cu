@@ -294,24 +294,6 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   }
 }
 
-// rq[r, h] = 1 / max(||Qr[r, h]||, 1e-12): one warp per (row, head)
-template <int DR>
-__global__ void qnorm_kernel(const __nv_bfloat16* __restrict__ Qr, int64_t n, float* __restrict__ rq) {
-  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= n) return;
-  const __nv_bfloat16* x = Qr + w * DR;
-  float ss = 0.f;
-#pragma unroll
-  for (int i = lane; i < DR; i += 32) {
-    const float v = __bfloat162float(x[i]);
-    ss += v * v;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) rq[w] = 1.0f / fmaxf(sqrtf(ss), 1e-12f);
-}
-
 template <int DR, int N>
 cudaError_t launch_t(const RouteArgs& a, cudaStream_t s) {
   using L = Layout<DR, N>;
@@ -320,12 +302,6 @@ cudaError_t launch_t(const RouteArgs& a, cudaStream_t s) {
   if (!make_tmap_2d_bf16(&tmK, a.Krbar, (uint64_t)a.Hr * DR, (uint64_t)a.C, (uint64_t)a.Hr * DR * 2, 64, kTileM) ||
       !make_tmap_2d_bf16(&tmQ, a.Qr, (uint64_t)a.Hr * DR, (uint64_t)rows, (uint64_t)a.Hr * DR * 2, 64, N))
     return cudaErrorInvalidValue;
-  {
-    const int64_t n = (int64_t)rows * a.Hr;
-    const int64_t blocks = (n * 32 + 255) / 256;
-    count_launch();
-    qnorm_kernel<DR><<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(a.Qr), n, a.rq);
-  }
   RouteTcParams p;
   p.kr_rnorm = a.kr_rnorm;
   p.rq = a.rq;
@@ -351,19 +327,18 @@ cudaError_t launch_t(const RouteArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s, bool* handled) {
-  *handled = false;
-  if (a.Hr < 1 || a.Hr > 8 || (a.dr != 64 && a.dr != 128) || a.C < 1) return cudaSuccess;
-  if (a.C > 0x7fffffffLL - kTileM || a.B * a.Tq > 0x7fffffffLL) return cudaSuccess;
-  // the TMA maps need 16-byte aligned bases (checked by the entry point)
+bool route_tc_applies(const RouteArgs& a) {
+  if (a.Hr < 1 || a.Hr > 8 || (a.dr != 64 && a.dr != 128) || a.C < 1) return false;
+  return a.C <= 0x7fffffffLL - kTileM && a.B * a.Tq <= 0x7fffffffLL;
+}
+
+// The caller has zeroed the keys, built chunk_doc and the query norms rq (the
+// routing prelude); the TMA maps need 16-byte aligned bases (checked by the
+// entry point).
+cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s) {
   const int64_t rows = a.B * a.Tq;
-  cudaError_t e;
-  if (a.dr == 128)
-    e = rows <= 64 ? launch_t<128, 64>(a, s) : launch_t<128, 128>(a, s);
-  else
-    e = rows <= 64 ? launch_t<64, 64>(a, s) : launch_t<64, 128>(a, s);
-  *handled = true;
-  return e;
+  if (a.dr == 128) return rows <= 64 ? launch_t<128, 64>(a, s) : launch_t<128, 128>(a, s);
+  return rows <= 64 ? launch_t<64, 64>(a, s) : launch_t<64, 128>(a, s);
 }
 
 }  // namespace msa

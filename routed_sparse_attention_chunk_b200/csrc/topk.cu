@@ -7,9 +7,9 @@
 // so that one unsigned comparison orders by score descending and, for equal
 // scores, by lower document index first; padding is key 0, below every real key.
 //
-// One launch, grid (slices, B).  A slice of up to 32768 documents is read
+// One launch, grid (slices, B).  A slice of up to 8192 documents is read
 // twice, 32 keys per thread.  The k-th largest of the per-thread maxima, tau,
-// is found with a bitonic sort of those 1024 maxima; the k largest keys of the
+// is found with a bitonic sort of those 256 maxima; the k largest keys of the
 // slice are all >= tau (k distinct thread maxima already are), and at most k
 // threads hold a key >= tau, so at most 32 k keys survive the filter.  The
 // survivors are sorted in shared memory and the slice's top-k goes to the
@@ -26,7 +26,7 @@ namespace msa {
 namespace {
 
 constexpr int kSortN = 2048;
-constexpr int kSortThreads = 1024;
+constexpr int kSortThreads = 256;
 constexpr int kPer = 32;                         // keys per thread in the filter
 constexpr int kSlice = kSortThreads * kPer;      // documents per slice
 
