@@ -288,6 +288,10 @@ def test_attention_bf16(B, Tq, Lloc, Hq, Hkv, d, Mmax, mem_lens):
     (1, 300, 300, 8, 8, 128, [128]),              # G=1 (MHA): 128 tokens per block
     (2, 50, 400, 64, 8, 256, [256, 200]),         # G=8: 16 tokens per block, two memory tiles
     (1, 1030, 1030, 32, 8, 128, [128]),           # many local tiles, a partial last block
+    (4, 480, 480, 32, 8, 128, [128, 0, 100, 128]),  # odd block count, ragged memory across the batch
+    (2, 1100, 1300, 32, 8, 256, [256, 37]),       # local history longer than the query, partial last block
+    (1, 600, 600, 64, 8, 128, [128]),             # G=8: 16 tokens per tile, many tiles
+    (2, 512, 512, 40, 40, 64, [64, 30]),          # G=1 with 40 heads: 128 tokens per tile
 ])
 def test_attention_bf16_tensor_core_tiling(B, Tq, Lloc, Hq, Hkv, Mmax, mem_lens):
     Q, Kl, Vl, Km, Vm, ml = _attn_inputs(B, Tq, Lloc, Hq, Hkv, 128, Mmax, mem_lens, torch.bfloat16, 4)
