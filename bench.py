@@ -379,7 +379,8 @@ def run_gpu(args, rank, local_rank, world):
     roofline["achieved"] = round(roofline["achieved"], 2)
     roofline["frac"] = round(roofline["achieved"] / roofline["peak"], 4)
     roofline["avg_launch_ms"] = round(per_launch[dom], 4)
-    tr = traffic_record({"pool": "pool.cu", "route_topk": "route_tc.cu", "sparse_attn": "attn_tc.cu",
+    tr = traffic_record({"pool": "pool.cu", "route_topk": "route_tc.cu",
+                         "sparse_attn": "attn_decode.cu" if cfg.Tq == 1 else "attn_tc.cu",
                          "gather": "gather.cu"}[dom], cfg.name)
     roofline["traffic"] = tr["dram_bytes_per_launch"] if tr else None
     stages = {s: {"ms_per_launch": round(per_launch[s], 4), "share": round(totals[s] / step_sum, 4),

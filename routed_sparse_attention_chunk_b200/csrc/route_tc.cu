@@ -198,23 +198,38 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     float* rq_w = rq_s + (warp - 2) * 8 * NH;  // this warp's private copy (no cross-warp barrier)
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16) + col0;
     const float invHr = 1.0f / (float)Hr;
+    // This lane's chunk of the next item: its document and its 1/||K̄r|| per
+    // head are loaded one item ahead, so their latency overlaps the current
+    // item's document walk instead of stalling the accumulator hand-off.
+    int doc_n = -1;
+    float rkv_n[8];
+    auto prefetch = [&](int64_t item) {
+      const int64_t cn = (item / p.n_rb) * kTileM + q * 32 + lane;
+      const bool vn = item < p.items && cn < p.C;
+      doc_n = vn ? __ldg(p.chunk_doc + cn) : -1;
+#pragma unroll
+      for (int h = 0; h < 8; ++h) rkv_n[h] = (vn && h < Hr) ? __ldg(p.kr_rnorm + cn * Hr + h) : 0.f;
+    };
+    prefetch(blockIdx.x);
+    int rb_loaded = -1;  // query rows whose norms rq_w holds
     uint32_t it = 0;
     for (int64_t item = blockIdx.x; item < p.items && !timed_out; item += gridDim.x) {
-      const int tile = (int)(item / p.n_rb), rb = (int)(item % p.n_rb);
-      const int64_t c = (int64_t)tile * kTileM + q * 32 + lane;
-      const bool valid = c < p.C;
+      const int rb = (int)(item % p.n_rb);
       const int r0 = rb * N + col0;                 // first query row of this warp's columns
       const int nvalid = max(0, min(NH, p.rows - r0));
-      __syncwarp();
-      for (int i = lane; i < Hr * NH; i += 32) {
-        const int h = i / NH, col = i - h * NH, r = r0 + col;
-        rq_w[i] = r < p.rows ? __ldg(p.rq + (int64_t)r * Hr + h) : 0.f;
+      if (rb != rb_loaded) {  // every item when the rows span several blocks, once otherwise
+        __syncwarp();
+        for (int i = lane; i < Hr * NH; i += 32) {
+          const int h = i / NH, col = i - h * NH, r = r0 + col;
+          rq_w[i] = r < p.rows ? __ldg(p.rq + (int64_t)r * Hr + h) : 0.f;
+        }
+        __syncwarp();
+        rb_loaded = rb;
       }
-      __syncwarp();
-      const int doc = valid ? __ldg(p.chunk_doc + c) : -1;
-      float rkv[8];  // this chunk's 1/||K̄r|| for every head, loaded together
+      const int doc = doc_n;
+      float rkv[8];  // this chunk's 1/||K̄r|| for every head
 #pragma unroll
-      for (int h = 0; h < 8; ++h) rkv[h] = (valid && h < Hr) ? __ldg(p.kr_rnorm + c * Hr + h) : 0.f;
+      for (int h = 0; h < 8; ++h) rkv[h] = rkv_n[h];
       float S_[NH];
 #pragma unroll
       for (int j = 0; j < NH; ++j) S_[j] = 0.f;
@@ -240,6 +255,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         for (int j = 0; j < NH; ++j) S_[j] = fmaf(v[j], rk * rqh[j], S_[j]);
       }
       if (timed_out) break;
+      prefetch(item + gridDim.x);
       if (nvalid == 0) continue;
       const int b_first = r0 / p.Tq, b_last = (r0 + nvalid - 1) / p.Tq;
       if (b_first == b_last) {
