@@ -12,9 +12,10 @@
 // per chunk) against a block of N query rows (the MMA's N).  For every router
 // head h the tile's K̄r[., h, :] and the block's Qr[., h, :] arrive by TMA
 // (128-byte swizzle), one tcgen05.mma chain (K = dr) writes the fp32 dot
-// products of that head into one of two TMEM accumulators, and the epilogue
-// warps fold rk * rq * dot into a register running sum while the tensor core
-// already works on the next head.  The per-head cosine weights are why the
+// products of that head into the next of the TMEM accumulators (all 512
+// columns: 8 of N = 64 or 4 of N = 128, so the tensor core can run a whole
+// item ahead of the epilogue), and the epilogue warps fold rk * rq * dot into
+// a register running sum.  The per-head cosine weights are why the
 // heads cannot share one accumulator: the products stay exact (bf16 x bf16 in
 // fp32) and every scale is applied in fp32 afterwards.  After the last head the
 // epilogue takes the max over the block's tokens in registers, a segmented max
@@ -63,10 +64,11 @@ struct Layout {
   static constexpr int kStages = (200 * 1024) / kStage > 6 ? 6 : (200 * 1024) / kStage;
   static constexpr int kRq = 8 * 8 * (N / 2) * 4;         // per epilogue warp: rq of its columns, Hr <= 8
   static constexpr int kTr = 8 * 32 * 17 * 4;              // per epilogue warp: 32 chunks x 16 columns (+1 pad)
-  static constexpr int kBar = 8 * (2 * kStages + 5) + 16;
+  static constexpr int kAcc = 512 / N;                      // fp32 accumulators of N columns in TMEM
+  static constexpr int kBar = 8 * (2 * kStages + 2 * kAcc + 1) + 16;
   static constexpr int kSmem = 1024 + kStages * kStage + kRq + kTr + kBar;
   static_assert(kSmem <= 232448, "shared memory of one CTA");
-  static constexpr uint32_t kTmemCols = 2 * N;            // two accumulators of N fp32 columns
+  static constexpr uint32_t kTmemCols = 512;              // all of TMEM: kAcc accumulators
 };
 
 // Segmented max over the warp's lanes (consecutive chunks) grouped by document,
@@ -96,10 +98,11 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * L::kStage + L::kRq + L::kTr);
   uint64_t* full = bars;              // [S]   TMA -> MMA
   uint64_t* empty = bars + S;         // [S]   MMA -> TMA
-  uint64_t* accf = bars + 2 * S;      // [2]   MMA -> epilogue
-  uint64_t* acce = bars + 2 * S + 2;  // [2]   epilogue -> MMA
-  uint64_t* drain = bars + 2 * S + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  constexpr int NA = L::kAcc;
+  uint64_t* accf = bars + 2 * S;      // [NA]  MMA -> epilogue
+  uint64_t* acce = accf + NA;         // [NA]  epilogue -> MMA
+  uint64_t* drain = acce + NA;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hr = p.Hr;
@@ -109,7 +112,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NA; ++i) {
       mbar_init(&accf[i], 1);
       mbar_init(&acce[i], 256);
     }
@@ -165,7 +168,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       for (int64_t item = blockIdx.x; item < p.items && !timed_out; item += gridDim.x) {
         for (int h = 0; h < Hr; ++h, ++it) {
           const uint32_t s = it % S, round = it / S;
-          const uint32_t buf = it & 1, use = it >> 1;
+          const uint32_t buf = it % NA, use = it / NA;
           if (!mbar_wait(&full[s], round & 1, kWaitPolls) || !mbar_wait(&acce[buf], (use & 1) ^ 1, kWaitPolls)) {
             timed_out = true;
             break;
@@ -234,7 +237,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 #pragma unroll
       for (int j = 0; j < NH; ++j) S_[j] = 0.f;
       for (int h = 0; h < Hr; ++h, ++it) {
-        const uint32_t buf = it & 1, use = it >> 1;
+        const uint32_t buf = it % NA, use = it / NA;
         float rk = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) rk = i == h ? rkv[i] : rk;
