@@ -150,9 +150,18 @@ route_prelude_kernel(uint32_t* __restrict__ keys, int64_t nkeys, int nb_zero, co
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int blk = blockIdx.x;
   if (blk < nb_zero) {
+    // 16-byte stores over the aligned body of this block's range
     const int64_t per = (nkeys + nb_zero - 1) / nb_zero;
     const int64_t lo = (int64_t)blk * per, hi = min(nkeys, lo + per);
-    for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x) keys[i] = 0u;
+    if (lo >= hi) return;
+    uint32_t* k0 = keys + lo;
+    const int64_t n = hi - lo;
+    const int64_t pre = min(n, (int64_t)(((16u - (reinterpret_cast<uintptr_t>(k0) & 15u)) & 15u) >> 2));
+    const int64_t nv = (n - pre) >> 2;
+    for (int64_t i = threadIdx.x; i < pre; i += blockDim.x) k0[i] = 0u;
+    uint4* v = reinterpret_cast<uint4*>(k0 + pre);
+    for (int64_t i = threadIdx.x; i < nv; i += blockDim.x) v[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t i = pre + 4 * nv + threadIdx.x; i < n; i += blockDim.x) k0[i] = 0u;
     return;
   }
   if (blk < nb_zero + nb_map) {

@@ -7,16 +7,18 @@
 // so that one unsigned comparison orders by score descending and, for equal
 // scores, by lower document index first; padding is key 0, below every real key.
 //
-// One launch, grid (slices, B).  A slice of up to 8192 documents is read
-// twice, 32 keys per thread.  The k-th largest of the per-thread maxima, tau,
-// is found with a bitonic sort of those 256 maxima; the k largest keys of the
-// slice are all >= tau (k distinct thread maxima already are), and at most k
-// threads hold a key >= tau, so at most 32 k keys survive the filter.  The
-// survivors are sorted in shared memory and the slice's top-k goes to the
-// workspace (when more than 2048 survive, which needs k > 64, the slice is
-// instead streamed through shared memory in blocks, keeping the running top-k
-// at the front).  The last CTA of the row to finish (an atomic counter, no
-// waiting) merges the slices' candidates the same way and writes the result.
+// One launch, grid (slices, B).  A slice of up to 8192 documents is held in
+// registers, 32 keys per thread.  The threshold tau is the k-th largest of the
+// 256 per-thread maxima: the k largest keys of the slice are all >= tau (k
+// distinct thread maxima already are), and only the k threads whose maximum
+// passes hold keys >= tau, so at most 32 k keys survive.  For k <= 32 the work
+// stays in warps: each warp sorts its 32 maxima across lanes with shuffles,
+// warp 0 merges the eight sorted lists (bitonic top-32 merges) to find tau, and
+// up to 32 survivors are sorted in one warp's registers; larger k or more
+// survivors take shared-memory bitonic sorts (and more than 2048 survivors,
+// which needs k > 64, a block sort streamed over the slice).  The slice's
+// top-k goes to the workspace; the last CTA of the row to finish (an atomic
+// counter, no waiting) merges the slices' sorted lists and writes the result.
 // The top-k of a union is contained in the union of the parts' top-k, so the
 // result is exact.
 #include "common.cuh"
@@ -76,27 +78,80 @@ __device__ __forceinline__ uint64_t doc_key64(uint32_t score_key, int64_t doc) {
   return ((uint64_t)score_key << 32) | (uint64_t)(0xffffffffu - (uint32_t)doc);
 }
 
+// 32 keys, one per lane, sorted descending across the warp (a bitonic network
+// over lanes: no shared memory, no block barrier).
+__device__ __forceinline__ uint64_t warp_sort_desc(uint64_t x, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, x, stride);
+      const bool desc = (lane & size) == 0 || size == 32;
+      x = (((lane & stride) == 0) == desc) ? max(x, o) : min(x, o);
+    }
+  }
+  return x;
+}
+
+// The 32 largest of two descending lane-lists, descending: a[i] against
+// b[31 - i] keeps the top 32 as a bitonic sequence, which five compare-exchange
+// steps sort.
+__device__ __forceinline__ uint64_t warp_merge_top(uint64_t a, uint64_t b, int lane) {
+  uint64_t x = max(a, __shfl_sync(0xffffffffu, b, 31 - lane));
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, x, stride);
+    x = (lane & stride) == 0 ? max(x, o) : min(x, o);
+  }
+  return x;
+}
+
 // Top-k of keys row[lo, lo + n), n <= kSlice, left sorted in s[0, k); false
 // when more than kSortN keys pass the filter (s is then clobbered).
-__device__ bool slice_topk_filter(uint64_t* s, int* cnt, const uint32_t* row, int64_t lo, int64_t n, int k) {
-  const int tid = threadIdx.x, lane = tid & 31;
-  uint64_t mx = 0ull;
-#pragma unroll 8
+__device__ bool slice_topk_filter(uint64_t* s, int* cnt, uint64_t* tau_s, const uint32_t* row, int64_t lo,
+                                  int64_t n, int k) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // all 32 keys of this thread in registers from one round of loads
+  uint32_t v[kPer];
+#pragma unroll
   for (int m = 0; m < kPer; ++m) {
     const int64_t i = tid + (int64_t)m * kSortThreads;
-    if (i < n) mx = max(mx, doc_key64(__ldg(row + lo + i), lo + i));
+    v[m] = i < n ? __ldg(row + lo + i) : 0u;
   }
-  s[tid] = mx;
-  if (tid == 0) *cnt = 0;
-  __syncthreads();
-  bitonic_desc(s, kSortThreads);
-  const uint64_t tau = s[k - 1];
-  __syncthreads();
-  // second pass over the slice (now in L1/L2)
-#pragma unroll 4
+  uint64_t mx = 0ull;
+#pragma unroll
   for (int m = 0; m < kPer; ++m) {
     const int64_t i = tid + (int64_t)m * kSortThreads;
-    const uint64_t key = i < n ? doc_key64(__ldg(row + lo + i), lo + i) : 0ull;
+    if (i < n) mx = max(mx, doc_key64(v[m], lo + i));
+  }
+  // tau = the k-th largest of the 256 thread maxima
+  uint64_t tau;
+  if (k <= 32) {
+    // each warp sorts its maxima; warp 0 merges the eight sorted lists
+    s[tid] = warp_sort_desc(mx, lane);
+    if (tid == 0) *cnt = 0;
+    __syncthreads();
+    if (warp == 0) {
+      uint64_t m = s[lane];
+      for (int w = 1; w < kSortThreads / 32; ++w) m = warp_merge_top(m, s[w * 32 + lane], lane);
+      const uint64_t t = __shfl_sync(0xffffffffu, m, k - 1);
+      if (lane == 0) *tau_s = t;
+    }
+    __syncthreads();
+    tau = *tau_s;
+  } else {
+    s[tid] = mx;
+    if (tid == 0) *cnt = 0;
+    __syncthreads();
+    bitonic_desc(s, kSortThreads);
+    tau = s[k - 1];
+    __syncthreads();
+  }
+  // keep the keys >= tau (the k thread maxima and what else their threads hold)
+#pragma unroll
+  for (int m = 0; m < kPer; ++m) {
+    const int64_t i = tid + (int64_t)m * kSortThreads;
+    const uint64_t key = i < n ? doc_key64(v[m], lo + i) : 0ull;
     const bool pass = i < n && key >= tau;
     const uint32_t bal = __ballot_sync(0xffffffffu, pass);
     if (bal) {
@@ -110,6 +165,14 @@ __device__ bool slice_topk_filter(uint64_t* s, int* cnt, const uint32_t* row, in
   __syncthreads();
   const int total = *cnt;
   if (total > kSortN) return false;
+  if (total <= 32) {  // one warp sorts the survivors in registers
+    if (warp == 0) {
+      const uint64_t x = warp_sort_desc(lane < total ? s[lane] : 0ull, lane);
+      s[lane] = x;
+    }
+    __syncthreads();
+    return true;
+  }
   const int m2 = next_pow2(max(total, max(k, 2)));
   for (int i = total + tid; i < m2; i += kSortThreads) s[i] = 0ull;
   __syncthreads();
@@ -121,6 +184,7 @@ __global__ void __launch_bounds__(kSortThreads)
 topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, uint64_t* cand,
             uint32_t* counters, int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
   __shared__ uint64_t s[kSortN];
+  __shared__ uint64_t tau_s;
   __shared__ int last, cnt;
   const int64_t b = blockIdx.y;
   const int slice = blockIdx.x;
@@ -129,7 +193,7 @@ topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, 
   const int64_t n = max((int64_t)0, min(D, lo + per) - lo);
   const uint32_t* row = doc_key + b * D;
   // (the branch is uniform over the CTA)
-  if (n > kSlice || !slice_topk_filter(s, &cnt, row, lo, n, k)) {
+  if (n > kSlice || !slice_topk_filter(s, &cnt, &tau_s, row, lo, n, k)) {
     __syncthreads();
     block_topk(s, n, k, [&](int64_t i) -> uint64_t { return doc_key64(__ldg(row + lo + i), lo + i); });
   }
@@ -143,7 +207,18 @@ topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, 
     if (!last) return;
     __threadfence();
     const uint64_t* c = cand + b * nslice * k;
-    block_topk(s, (int64_t)nslice * k, k, [&](int64_t i) -> uint64_t { return __ldcg(c + i); });
+    if (k <= 32) {
+      // every slice's list is sorted: warp 0 merges them pairwise in registers
+      if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        uint64_t m = lane < k ? __ldcg(c + lane) : 0ull;
+        for (int sl = 1; sl < nslice; ++sl) m = warp_merge_top(m, lane < k ? __ldcg(c + sl * k + lane) : 0ull, lane);
+        s[lane] = m;
+      }
+      __syncthreads();
+    } else {
+      block_topk(s, (int64_t)nslice * k, k, [&](int64_t i) -> uint64_t { return __ldcg(c + i); });
+    }
     if (threadIdx.x == 0) counters[b] = 0u;  // ready for the next call on this workspace
   }
   for (int i = threadIdx.x; i < k; i += blockDim.x) {
