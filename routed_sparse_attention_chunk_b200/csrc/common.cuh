@@ -74,6 +74,11 @@ __device__ __forceinline__ void raise_flag(int32_t* flag, int bits) {
 
 // Index of the document owning chunk c: the j with off[j] <= c < off[j+1]
 // (largest j with off[j] <= c); off is non-decreasing, length D+1.
+// Programmatic dependent launch: wait for the previous kernel on the stream to
+// finish (and its writes to be visible); let the next kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ int64_t owner_doc(const int64_t* __restrict__ off, int64_t D, int64_t c) {
   int64_t lo = 0, hi = D;  // answer in [lo, hi)
   while (hi - lo > 1) {

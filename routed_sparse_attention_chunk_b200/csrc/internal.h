@@ -13,6 +13,26 @@ namespace msa {
 // Counts every kernel launch of the library (read by msa_kernel_launch_count).
 void count_launch(int n = 1);
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel on the stream is still running (once that kernel
+// triggers its dependents, or exits), and must execute griddepcontrol.wait
+// before it touches anything the previous kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 struct PoolArgs {
   const void *K, *V, *Kr;
   const int64_t *doc_tok_off, *doc_chunk_off;

@@ -147,6 +147,9 @@ route_prelude_kernel(uint32_t* __restrict__ keys, int64_t nkeys, int nb_zero, co
                      int64_t D, int64_t C, int32_t* __restrict__ chunk_doc, int nb_map,
                      const __nv_bfloat16* __restrict__ Qr, int64_t nq, int dr, float* __restrict__ rq,
                      int32_t* err_flag) {
+  // the scan may launch now: its TMA and MMA warps need nothing written here,
+  // and its epilogue waits for this grid before reading any of it
+  pdl_trigger();
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int blk = blockIdx.x;
   if (blk < nb_zero) {

@@ -213,6 +213,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 #pragma unroll
       for (int h = 0; h < 8; ++h) rkv_n[h] = (vn && h < Hr) ? __ldg(p.kr_rnorm + cn * Hr + h) : 0.f;
     };
+    // the routing prelude (keys zeroed, chunk map, query norms) must be done
+    pdl_wait();
     prefetch(blockIdx.x);
     int rb_loaded = -1;  // query rows whose norms rq_w holds
     uint32_t it = 0;
@@ -340,8 +342,7 @@ cudaError_t launch_t(const RouteArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int64_t grid = p.items < sm_count() ? p.items : sm_count();
   count_launch();
-  route_tc_kernel<DR, N><<<(unsigned)grid, kThreads, L::kSmem, s>>>(tmK, tmQ, p);
-  return cudaGetLastError();
+  return launch_pdl(route_tc_kernel<DR, N>, dim3((unsigned)grid), dim3(kThreads), (size_t)L::kSmem, s, tmK, tmQ, p);
 }
 
 }  // namespace

@@ -186,6 +186,7 @@ topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, 
   __shared__ uint64_t s[kSortN];
   __shared__ uint64_t tau_s;
   __shared__ int last, cnt;
+  pdl_wait();  // the scan's keys (launched as a programmatic dependent of it)
   const int64_t b = blockIdx.y;
   const int slice = blockIdx.x;
   const int64_t per = (D + nslice - 1) / nslice;
@@ -253,9 +254,8 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
     decode_scores_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, s>>>(a.doc_key, n, a.doc_scores);
   }
   count_launch();
-  topk_kernel<<<dim3(a.nslice, (unsigned)a.B), kSortThreads, 0, s>>>(a.doc_key, a.D, a.k, a.nslice, a.cand,
-                                                                      a.counters, a.topk_idx, a.topk_score);
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel, dim3(a.nslice, (unsigned)a.B), dim3(kSortThreads), 0, s, a.doc_key, a.D, a.k,
+                    a.nslice, a.cand, a.counters, a.topk_idx, a.topk_score);
 }
 
 }  // namespace msa
