@@ -59,7 +59,8 @@ struct DLayout {
   static constexpr int kStage = 2 * kTile;
   static constexpr int kQ = kMaxRows * kDH * 2;       // Q rows, K-major, 128-byte swizzle
   static constexpr int kP = kMaxRows * kKeys * 2;     // P^T rows (query rows x keys)
-  static constexpr int kSmem = 1024 + kStages * kStage + kQ + kP + 4 * kMaxRows * 4 + 8 * 16 + 16;
+  static constexpr int kRed = 3 * kMaxRows * 4 * 4;    // [2 tile parities + unit end][rows][4 warps]
+  static constexpr int kSmem = 1024 + kStages * kStage + kQ + kP + kRed + 8 * 16 + 16;
   static constexpr uint32_t kTmemCols = 64;           // S0, S1, O (16 columns each)
 };
 
@@ -69,6 +70,12 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 __device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Maximum of v over the 32 lanes, in every lane (one instruction on sm_100a).
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Byte offset of element (row, col) in a K-major, 128-byte-swizzled tile whose
@@ -86,8 +93,8 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
   uint8_t* ring = smem;
   uint8_t* Qs = ring + kStages * DLayout::kStage;
   uint8_t* Ps = Qs + DLayout::kQ;
-  float* red_s = reinterpret_cast<float*>(Ps + DLayout::kP);  // [4 warps][16]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red_s + 4 * kMaxRows);
+  float* red_s = reinterpret_cast<float*>(Ps + DLayout::kP);  // [3][16 rows][4 warps]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red_s) + DLayout::kRed);
   uint64_t* kv_full = bars;            // [3]
   uint64_t* kv_empty = bars + 3;       // [3]
   uint64_t* s_full = bars + 6;         // [2]
@@ -268,26 +275,26 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
           const bool vis = r < p.R && (mem ? key < M : key <= p.Lloc - p.Tq + r / p.G);
           sc[r] = vis ? sc[r] * p.scale_log2 : -INFINITY;
         }
-        // column maxima over the tile's 128 keys
-        float mx[kMaxRows];
+        // column maxima over the tile's 128 keys: a warp reduction per column,
+        // then the four warps' maxima through shared memory.  The exchange
+        // buffer alternates with the tile's parity, so one barrier per tile
+        // suffices (a buffer is rewritten two tiles later, after every thread
+        // has passed the barrier of the tile in between).
+        float* red = red_s + ((it + j) & 1) * (kMaxRows * 4);
+        float mine = -INFINITY;  // lane r < 16 keeps this warp's maximum of column r
 #pragma unroll
         for (int r = 0; r < kMaxRows; ++r) {
-          float v = sc[r];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          mx[r] = v;
+          const float v = warp_max(sc[r]);
+          mine = lane == r ? v : mine;
         }
-        if (lane == 0) {
-#pragma unroll
-          for (int r = 0; r < kMaxRows; r += 4)
-            *reinterpret_cast<float4*>(red_s + q * kMaxRows + r) = make_float4(mx[r], mx[r + 1], mx[r + 2], mx[r + 3]);
-        }
+        if (lane < kMaxRows) red[lane * 4 + q] = mine;
         bar_softmax();
         bool grow = false;
         float corr[kMaxRows];
 #pragma unroll
         for (int r = 0; r < kMaxRows; ++r) {
-          const float mt = fmaxf(fmaxf(red_s[r], red_s[kMaxRows + r]), fmaxf(red_s[2 * kMaxRows + r], red_s[3 * kMaxRows + r]));
+          const float4 w = *reinterpret_cast<const float4*>(red + r * 4);
+          const float mt = fmaxf(fmaxf(w.x, w.y), fmaxf(w.z, w.w));
           corr[r] = 1.f;
           if (mt > m_run[r] + kRescaleLog2) {  // same decision in every thread
             corr[r] = m_run[r] == -INFINITY ? 0.f : fast_exp2(m_run[r] - mt);
@@ -295,7 +302,6 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
             grow = true;
           }
         }
-        bar_softmax();  // red_s is rewritten next tile
         float pr[kMaxRows];
 #pragma unroll
         for (int r = 0; r < kMaxRows; ++r) {
@@ -331,12 +337,13 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
       tmem_ld16(tO + lane_off, o);
       tmem_ld_wait();
       float* out = p.part + (size_t)u * p.R * (kDH + 2);
+      float* red_l = red_s + 2 * (kMaxRows * 4);  // the unit's row sums, apart from the tile buffers
 #pragma unroll
       for (int r = 0; r < kMaxRows; ++r) {
         float v = l_run[r];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == 0) red_s[q * kMaxRows + r] = v;
+        if (lane == 0) red_l[r * 4 + q] = v;
         if (r < p.R) out[r * (kDH + 2) + 2 + r_lane] = T > 0 ? o[r] : 0.f;
       }
       bar_softmax();
@@ -345,7 +352,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
 #pragma unroll
         for (int r = 0; r < kMaxRows; ++r) m = r == et ? m_run[r] : m;
         out[et * (kDH + 2)] = m;
-        out[et * (kDH + 2) + 1] = red_s[et] + red_s[kMaxRows + et] + red_s[2 * kMaxRows + et] + red_s[3 * kMaxRows + et];
+        out[et * (kDH + 2) + 1] = red_l[et * 4] + red_l[et * 4 + 1] + red_l[et * 4 + 2] + red_l[et * 4 + 3];
       }
       bar_softmax();
       tc_fence_before();
