@@ -153,6 +153,24 @@ def traffic_record(kernel_file: str, workload: str):
     return r
 
 
+def workload_label(cfg: synth.Config) -> str:
+    return (f"{cfg.name}: {cfg.D} docs, {cfg.ntok} memory tokens, {cfg.C} chunks (P={cfg.P}), "
+            f"B={cfg.B} x Tq={cfg.Tq}, Lloc={cfg.Lloc}, Hq/Hkv/Hr={cfg.Hq}/{cfg.Hkv}/{cfg.Hr}, "
+            f"d={cfg.d}, k={cfg.k}, layers={cfg.layers}")
+
+
+def step_label(step_kind: str) -> str:
+    return ("msa_pool of every raw token, then per layer msa_route_topk, msa_gather, msa_sparse_attn"
+            if step_kind == "full" else
+            "per layer msa_route_topk, msa_gather, msa_sparse_attn over a bank pooled before timing")
+
+
+def step_kind_for(cfg: synth.Config, args) -> str:
+    """'full' (pool + layers) unless the raw corpus does not fit the device next to the bank."""
+    raw_bytes = cfg.ntok * (2 * cfg.Hkv * cfg.d + cfg.Hr * cfg.dr) * (4 if cfg.dtype == "f32" else 2)
+    return args.step or ("query" if raw_bytes > 80e9 else "full")
+
+
 def workload_config(args) -> synth.Config:
     cfg = synth.get_config(args.workload)
     if args.docs:
@@ -317,8 +335,7 @@ def run_gpu(args, rank, local_rank, world):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     import routed_sparse_attention_chunk_b200 as msa
     cfg = workload_config(args)
-    raw_bytes = cfg.ntok * (2 * cfg.Hkv * cfg.d + cfg.Hr * cfg.dr) * (4 if cfg.dtype == "f32" else 2)
-    step_kind = args.step or ("query" if raw_bytes > 80e9 else "full")
+    step_kind = step_kind_for(cfg, args)
     peaks, peak_kind = load_peaks()
     counts = workload_counts(cfg)
     w = MSAWorkload(cfg, device, seed=1000 * rank, step_kind=step_kind)
@@ -419,12 +436,8 @@ def run_gpu(args, rank, local_rank, world):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded generators; see workloads/synth.py)",
-        "config": {"workload": f"{cfg.name}: {cfg.D} docs, {cfg.ntok} memory tokens, {cfg.C} chunks (P={cfg.P}), "
-                               f"B={cfg.B} x Tq={cfg.Tq}, Lloc={cfg.Lloc}, Hq/Hkv/Hr={cfg.Hq}/{cfg.Hkv}/{cfg.Hr}, "
-                               f"d={cfg.d}, k={cfg.k}, layers={cfg.layers}",
-                   "step": ("msa_pool of every raw token, then per layer msa_route_topk, msa_gather, msa_sparse_attn"
-                            if step_kind == "full" else
-                            "per layer msa_route_topk, msa_gather, msa_sparse_attn over a bank pooled before timing"),
+        "config": {"workload": workload_label(cfg),
+                   "step": step_label(step_kind),
                    "l2": "inputs larger than L2" if flush is None else "L2 flushed between steps (not timed)",
                    "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
         "route_scan_gbs": round(counts["route_bytes"] / (route_ms / 1e3) / 1e9, 1) if route_ms else None,
@@ -436,7 +449,7 @@ def run_gpu(args, rank, local_rank, world):
         "err_flag": flag,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_budget)
+        result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_budget, with_pool=step_kind == "full")
     if world > 1:
         import torch.distributed as dist
         barrier(world, device)
@@ -445,7 +458,7 @@ def run_gpu(args, rank, local_rank, world):
 
 
 # ----------------------------------------------------------------------------- CPU oracle arm
-def oracle_step_sample(cfg: synth.Config, docs: int, tokens: int, seed: int = 0):
+def oracle_step_sample(cfg: synth.Config, docs: int, tokens: int, seed: int = 0, with_pool: bool = True):
     """Time the oracle on a bounded sample of one step; returns (estimated full-step seconds, sample text).
 
     Pool: `docs` documents' raw tokens (time scaled by D / docs).  Query path of
@@ -460,8 +473,9 @@ def oracle_step_sample(cfg: synth.Config, docs: int, tokens: int, seed: int = 0)
     K, V, Kr = synth.gen_raw_slab(sub, 0, docs, "cpu", seed)
     off = synth.doc_tok_offsets(sub)
     t0 = time.perf_counter()
-    O.pool(K.double().numpy(), V.double().numpy(), Kr.double().numpy(), off, cfg.P, cfg.theta,
-           out_bf16=cfg.dtype == "bf16")
+    if with_pool:
+        O.pool(K.double().numpy(), V.double().numpy(), Kr.double().numpy(), off, cfg.P, cfg.theta,
+               out_bf16=cfg.dtype == "bf16")
     t_pool = (time.perf_counter() - t0) * cfg.D / docs
     # full-size bank for the query path (drawn, not pooled: only the time is used)
     rng = np.random.default_rng(seed)
@@ -475,7 +489,8 @@ def oracle_step_sample(cfg: synth.Config, docs: int, tokens: int, seed: int = 0)
     Km, Vm, ml = O.gather(idx, coff, Kb, Kb, cfg.Mmax)
     O.attention(q["Q"].double().numpy(), q["Kloc"].double().numpy(), q["Vloc"].double().numpy(), Km, Vm, ml)
     t_query = (time.perf_counter() - t0) * cfg.Tq / tokens * cfg.layers
-    text = (f"oracle (numpy fp64) pool of {docs} of {cfg.D} documents scaled x{cfg.D / docs:.0f}; route over all "
+    text = ((f"oracle (numpy fp64) pool of {docs} of {cfg.D} documents scaled x{cfg.D / docs:.0f}; " if with_pool
+             else "oracle (numpy fp64), bank pooled outside the step; ") + f"route over all "
             f"{cfg.C} chunks + top-k + gather + attention for {tokens} of {cfg.Tq} query tokens scaled "
             f"x{cfg.Tq / tokens:.0f}" + (f" and x{cfg.layers} layers" if cfg.layers > 1 else ""))
     return t_pool + t_query, text, time.perf_counter() - wall0
@@ -490,11 +505,11 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(cfg: synth.Config, budget_s: float = 20.0) -> dict:
+def cpu_baseline(cfg: synth.Config, budget_s: float = 20.0, with_pool: bool = True) -> dict:
     docs, tokens = 8, 16
-    _, _, wall = oracle_step_sample(cfg, docs, tokens)           # calibration run
+    _, _, wall = oracle_step_sample(cfg, docs, tokens, with_pool=with_pool)           # calibration run
     grow = max(1.0, min(16.0, budget_s / max(wall, 1e-3)))
-    est, text, wall = oracle_step_sample(cfg, int(docs * grow), int(tokens * grow))
+    est, text, wall = oracle_step_sample(cfg, int(docs * grow), int(tokens * grow), with_pool=with_pool)
     return {"value": round(cfg.B * cfg.Tq / est, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": text + f"; sample wall {wall:.1f} s; host {os.cpu_count()} logical CPUs"}
 
@@ -504,17 +519,19 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     cfg = workload_config(args)
+    kind = step_kind_for(cfg, args)
+    wp = kind == "full"
     per_step = max(0.2, min(10.0, args.ref_budget / max(1, args.steps + args.warmup)))
     docs, tokens = 2, 4
-    _, _, wall = oracle_step_sample(cfg, docs, tokens)          # calibration (counts as warm-up)
+    _, _, wall = oracle_step_sample(cfg, docs, tokens, with_pool=wp)   # calibration (counts as warm-up)
     grow = max(1.0, min(32.0, per_step / max(wall, 1e-3)))
     docs, tokens = int(docs * grow), int(tokens * grow)
     for _ in range(max(0, args.warmup - 1)):
-        oracle_step_sample(cfg, docs, tokens)
+        oracle_step_sample(cfg, docs, tokens, with_pool=wp)
     ests, texts = [], None
     wall0 = time.perf_counter()
     for _ in range(args.steps):
-        e, texts, _ = oracle_step_sample(cfg, docs, tokens)
+        e, texts, _ = oracle_step_sample(cfg, docs, tokens, with_pool=wp)
         ests.append(e)
     wall = time.perf_counter() - wall0
     est = float(np.mean(ests))
@@ -524,7 +541,7 @@ def run_reference(args, rank, world):
         "warmup": args.warmup, "ms_per_step": round(est * 1e3, 2), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generators; see workloads/synth.py)",
         "impl": "reference",
-        "config": {"workload": cfg.name, "parallelism": "host cores"},
+        "config": {"workload": workload_label(cfg), "step": step_label(kind), "parallelism": "host cores"},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": texts + f"; {args.steps} steps in {wall:.1f} s wall (target {per_step:.1f} s/step)"},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
