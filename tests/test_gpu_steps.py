@@ -129,6 +129,10 @@ def _bank_case(C_docs, Hr, dr, seed):
     (1, 64, 8, 128, 1500, 16),    # 100M workload's query shape
     (3, 37, 4, 64, 257, 5),       # odd sizes, dr = 64
     (2, 9, 1, 128, 40, 40),       # one router head, k = D
+    (4, 2, 8, 128, 20000, 32),    # largest k of the warp-level top-k, three slices merged
+    (3, 3, 8, 128, 17000, 33),    # smallest k of the block-level top-k, three slices
+    (2, 5, 2, 64, 9000, 1),       # k = 1 over two slices
+    (1, 4, 2, 64, 20, 20),        # fewer documents than a warp, k = D
 ])
 def test_route_topk_bf16(B, Tq, Hr, dr, D, k):
     Krb, rn, coff = _bank_case(D, Hr, dr, seed=B * 1000 + Tq)
