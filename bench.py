@@ -166,7 +166,10 @@ def step_label(step_kind: str) -> str:
 
 
 def step_kind_for(cfg: synth.Config, args) -> str:
-    """'full' (pool + layers) unless the raw corpus does not fit the device next to the bank."""
+    """'full' (pool + layers) unless the raw corpus does not fit the device next to the bank, or the
+    bank's K̄ / V̄ live in host memory (the pool writes them on the device first)."""
+    if getattr(args, "bank_kv", "device") == "host":
+        return "query"
     raw_bytes = cfg.ntok * (2 * cfg.Hkv * cfg.d + cfg.Hr * cfg.dr) * (4 if cfg.dtype == "f32" else 2)
     return args.step or ("query" if raw_bytes > 80e9 else "full")
 
@@ -191,7 +194,7 @@ class MSAWorkload:
 
     STAGES = ("pool", "route_topk", "gather", "sparse_attn")
 
-    def __init__(self, cfg: synth.Config, device, seed: int, step_kind: str):
+    def __init__(self, cfg: synth.Config, device, seed: int, step_kind: str, bank_kv: str = "device"):
         import routed_sparse_attention_chunk_b200 as msa
         self.msa, self.cfg, self.dev, self.kind = msa, cfg, device, step_kind
         dt = cfg.torch_dtype
@@ -213,6 +216,11 @@ class MSAWorkload:
             self._fill_raw(seed)
         else:
             self._pool_slabs(seed)
+        if bank_kv == "host":
+            # host tier: K̄ / V̄ in page-locked host memory, read in place by the gather
+            self.Kb = self.Kb.cpu().pin_memory()
+            self.Vb = self.Vb.cpu().pin_memory()
+            torch.cuda.empty_cache()
         B, c = cfg.B, cfg
         self.O = [torch.empty_like(L["Q"]) for L in self.layers]
         self.idx = [torch.empty((B, c.k), dtype=torch.int32, device=device) for _ in self.layers]
@@ -338,7 +346,7 @@ def run_gpu(args, rank, local_rank, world):
     step_kind = step_kind_for(cfg, args)
     peaks, peak_kind = load_peaks()
     counts = workload_counts(cfg)
-    w = MSAWorkload(cfg, device, seed=1000 * rank, step_kind=step_kind)
+    w = MSAWorkload(cfg, device, seed=1000 * rank, step_kind=step_kind, bank_kv=args.bank_kv)
     in_bytes = sum(t.numel() * t.element_size() for t in w.input_tensors())
     if step_kind == "query":
         in_bytes += w.Krb.numel() * w.Krb.element_size()  # the scan reads the whole bank every step
@@ -438,6 +446,7 @@ def run_gpu(args, rank, local_rank, world):
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded generators; see workloads/synth.py)",
         "config": {"workload": workload_label(cfg),
                    "step": step_label(step_kind),
+                   **({"bank_kv": "pinned host memory, read in place by msa_gather"} if args.bank_kv == "host" else {}),
                    "l2": "inputs larger than L2" if flush is None else "L2 flushed between steps (not timed)",
                    "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
         "route_scan_gbs": round(counts["route_bytes"] / (route_ms / 1e3) / 1e9, 1) if route_ms else None,
@@ -561,6 +570,8 @@ def main():
     ap.add_argument("--step", choices=["full", "query"], default=None,
                     help="full: pool + query path per step; query: bank pooled before timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bank-kv", choices=["device", "host"], default="device",
+                    help="where the pooled K̄ / V̄ live (host: page-locked host memory, the query path only)")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)
     args = ap.parse_args()

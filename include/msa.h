@@ -203,6 +203,12 @@ msa_status msa_route_topk_noalloc(msa_dtype dt, const void* Qr, int64_t B, int T
  * rows [0, mem_len[b]) of Kmem / Vmem; rows past mem_len[b] are left untouched.
  *   topk_idx int32 [B, k];  doc_chunk_off int64 [D+1]
  *   Kbar, Vbar [C, Hkv, d] dtype dt;  Kmem, Vmem [B, Mmax, Hkv, d];  mem_len int32 [B]
+ * Host tier ("Inference Pipeline": the pooled K̄ / V̄ may stay in host memory
+ * while K̄r stays on the GPU): Kbar and Vbar may be page-locked host memory
+ * that the device addresses directly (cudaHostAlloc, or cudaHostRegister with
+ * cudaHostRegisterMapped, under unified addressing); only the selected rows
+ * then cross the host link.  Pageable host memory returns
+ * MSA_ERR_INVALID_ARG.  The same holds for Kbar / Vbar of msa_layer_forward.
  * Device flags: MSA_FLAG_INDEX_OOB for a document index outside [0, D) or a
  * chunk outside [0, C) (that document is skipped), MSA_FLAG_OVERFLOW when the
  * selected chunks exceed Mmax (the rows that do not fit are dropped).

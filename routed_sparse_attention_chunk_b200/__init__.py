@@ -29,12 +29,13 @@ def _dt(t: torch.Tensor) -> int:
     return DTYPES[t.dtype]
 
 
-def _p(t, dtype=None):
-    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+def _p(t, dtype=None, host_ok=False):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL).  With host_ok, a
+    page-locked CPU tensor is accepted too (the device reads it in place)."""
     if t is None:
         return None
-    if not t.is_cuda:
-        raise ValueError("the MSA library takes CUDA tensors")
+    if not t.is_cuda and not (host_ok and t.is_pinned()):
+        raise ValueError("the MSA library takes CUDA tensors" + (" or pinned CPU tensors" if host_ok else ""))
     if not t.is_contiguous():
         raise ValueError("the MSA library takes contiguous tensors")
     if dtype is not None and t.dtype != dtype:
@@ -129,7 +130,8 @@ def gather(topk_idx, doc_chunk_off, Kbar, Vbar, Kmem, Vmem, mem_len, err_flag=No
     """Step 4: copy the selected documents' chunks (msa_gather).  Kmem [B, Mmax, Hkv, d]."""
     B, k = topk_idx.shape
     _call("msa_gather", _dt(Kbar), _p(topk_idx, torch.int32), B, k, _p(doc_chunk_off, torch.int64),
-          doc_chunk_off.numel() - 1, Kbar.shape[0], _p(Kbar), _p(Vbar, Kbar.dtype), Kbar.shape[1],
+          doc_chunk_off.numel() - 1, Kbar.shape[0], _p(Kbar, host_ok=True), _p(Vbar, Kbar.dtype, host_ok=True),
+          Kbar.shape[1],
           Kbar.shape[2], Kmem.shape[1], _p(Kmem, Kbar.dtype), _p(Vmem, Kbar.dtype),
           _p(mem_len, torch.int32), _p(err_flag, torch.int32), _s(stream))
 
@@ -160,6 +162,7 @@ def layer_forward(Qr, Krbar, kr_rnorm, doc_chunk_off, k, Q, Kloc, Vloc, Kbar, Vb
     _call("msa_layer_forward", _dt(Qr), _p(Qr), Hr, dr, _p(Krbar, Qr.dtype), _p(kr_rnorm, torch.float32),
           _p(doc_chunk_off, torch.int64), doc_chunk_off.numel() - 1, Krbar.shape[0], k,
           _p(Q, Qr.dtype), _p(Kloc, Qr.dtype), _p(Vloc, Qr.dtype), B, Tq, Kloc.shape[1], Hq, Kloc.shape[2], d,
-          _p(Kbar, Qr.dtype), _p(Vbar, Qr.dtype), Mmax, float(scale), _p(O, Qr.dtype), _p(lse, torch.float32),
+          _p(Kbar, Qr.dtype, host_ok=True), _p(Vbar, Qr.dtype, host_ok=True), Mmax, float(scale), _p(O, Qr.dtype),
+          _p(lse, torch.float32),
           _p(topk_idx, torch.int32), _p(topk_score, torch.float32), _p(doc_scores, torch.float32),
           _p(ws), ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))

@@ -19,6 +19,20 @@ void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_r
 namespace {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// True when kernels may dereference p as it is: device or managed memory, or
+// page-locked host memory mapped at the same address (unified addressing).
+// Pageable host memory (and anything the runtime does not know) is refused, so
+// a misplaced host pointer is an argument error, not a device fault.
+bool device_readable(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return true;
+  return at.type == cudaMemoryTypeHost && at.devicePointer == p;
+}
 inline bool head_dim_ok(int d) { return d == 64 || d == 128; }
 inline bool dtype_ok(msa_dtype dt) { return dt == MSA_F32 || dt == MSA_BF16; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -184,6 +198,7 @@ msa_status msa_gather(msa_dtype dt, const int32_t* topk_idx, int64_t B, int k, c
   if (!topk_idx || !doc_chunk_off || !Kbar || !Vbar || !mem_len || (Mmax > 0 && (!Kmem || !Vmem)))
     return MSA_ERR_INVALID_ARG;
   if (!aligned16(Kbar) || !aligned16(Vbar) || !aligned16(Kmem) || !aligned16(Vmem)) return MSA_ERR_INVALID_ARG;
+  if (!device_readable(Kbar) || !device_readable(Vbar)) return MSA_ERR_INVALID_ARG;
   GatherArgs a{topk_idx, B, k, doc_chunk_off, D, C, Kbar, Vbar, Hkv, d, Mmax, Kmem, Vmem, mem_len, err_flag};
   return cuda_status(launch_gather(dt, a, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -234,6 +249,7 @@ msa_status msa_layer_forward(msa_dtype dt, const void* Qr, int Hr, int dr, const
   if (!O || !Kbar || !Vbar || !aligned16(O) || !aligned16(Kbar) || !aligned16(Vbar)) return MSA_ERR_INVALID_ARG;
   const size_t need = msa_layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  if (!device_readable(Kbar) || !device_readable(Vbar)) return MSA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   RouteWs w = route_ws_layout(ws, B, Tq, Hr, D, C, k);
   char* p = static_cast<char*>(ws) + w.bytes;
