@@ -37,6 +37,10 @@ the plainest reading and says so at the function (the list of readings):
      bottom-right aligned: query token i sits at local position Lloc - Tq + i];
      q-head h reads KV head floor(h / (Hq / Hkv)); the scale is 1/sqrt(d).
   R7 Stored bf16 values are the fp64 result rounded to nearest, ties to even.
+  R14 The backward of the query path (the pages train MSA end to end through the
+     sparse attention but print no gradient) is the exact derivative of R6's
+     attention, and the gather's adjoint adds each gathered row's gradient back
+     into its chunk; the top-k choice itself carries no gradient.
 
 Layouts are row-major with the innermost dimension last:
   K, V [Ntok, Hkv, d]; Kr [Ntok, Hr, dr]; doc_tok_off int64 [D+1]
@@ -320,6 +324,82 @@ def attention(Q, Kloc, Vloc, Kmem, Vmem, mem_len, scale=None):
             O[b, :, h] = (w / den) @ vals
             lse[b, h] = (mx + np.log(den))[:, 0]
     return O, lse
+
+
+# ----------------------------------------------------------------------------
+# backward of steps 5 and 4 (the differentiable part of the query path)
+# ----------------------------------------------------------------------------
+def attention_backward(Q, Kloc, Vloc, Kmem, Vmem, mem_len, dO, scale=None):
+    """Gradient of attention()'s output O for an upstream gradient dO (reading R14).
+
+    MSA is trained end to end through its sparse attention ("MSA: Memory Sparse
+    Attention" README, Figure 2 caption and "Architecture": top-k selection is
+    fused with sparse attention so the layer stays differentiable).  With
+    s = scale q·kᵀ over the same visible keys as the forward, p = softmax(s),
+    o = p v:
+        dv_j = sum_i p_ij do_i          dp_ij = do_i · v_j
+        ds_ij = p_ij (dp_ij - sum_l p_il dp_il)
+        dq_i = scale sum_j ds_ij k_j    dk_j = scale sum_i ds_ij q_i
+    summed over the q-heads of a GQA group for the shared K/V.  Returns
+    (dQ, dKloc, dVloc, dKmem, dVmem) in fp64; memory rows past mem_len[b] get 0.
+    Pins: central finite differences of sum(dO * O) on a small case; the
+    gradients of keys no query sees are zero.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    Kl, Vl = np.asarray(Kloc, dtype=np.float64), np.asarray(Vloc, dtype=np.float64)
+    Km, Vm = np.asarray(Kmem, dtype=np.float64), np.asarray(Vmem, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    B, Tq, Hq, d = Q.shape
+    Lloc, Hkv = Kl.shape[1], Kl.shape[2]
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    group = Hq // Hkv
+    dQ = np.zeros_like(Q)
+    dKl, dVl = np.zeros_like(Kl), np.zeros_like(Vl)
+    dKm, dVm = np.zeros_like(Km), np.zeros_like(Vm)
+    for b in range(B):
+        M = int(mem_len[b])
+        for h in range(Hq):
+            g = h // group
+            keys = np.concatenate([Km[b, :M, g], Kl[b, :, g]], axis=0)
+            vals = np.concatenate([Vm[b, :M, g], Vl[b, :, g]], axis=0)
+            logits = scale * (Q[b, :, h] @ keys.T)
+            pos = Lloc - Tq + np.arange(Tq)
+            visible = np.concatenate(
+                [np.ones((Tq, M), bool), np.arange(Lloc)[None, :] <= pos[:, None]], axis=1)
+            logits = np.where(visible, logits, -np.inf)
+            w = np.exp(logits - logits.max(axis=1, keepdims=True))
+            P = w / w.sum(axis=1, keepdims=True)                   # [Tq, M + Lloc]
+            dP = dO[b, :, h] @ vals.T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            dQ[b, :, h] = scale * (dS @ keys)
+            dkeys = scale * (dS.T @ Q[b, :, h])
+            dvals = P.T @ dO[b, :, h]
+            dKm[b, :M, g] += dkeys[:M]
+            dVm[b, :M, g] += dvals[:M]
+            dKl[b, :, g] += dkeys[M:]
+            dVl[b, :, g] += dvals[M:]
+    return dQ, dKl, dVl, dKm, dVm
+
+
+def gather_backward(topk_idx, doc_chunk_off, dKmem, dVmem, mem_len, C: int):
+    """Adjoint of gather(): add every gathered row's gradient back into its chunk.
+
+    A chunk selected by several queries accumulates all their gradients.
+    Returns (dKbar, dVbar) [C, Hkv, d] in fp64.  Pin: the adjoint identity
+    <gather(x), y> = <x, gather_backward(y)> for random x and y.
+    """
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    off = np.asarray(doc_chunk_off, dtype=np.int64)
+    dKm, dVm = np.asarray(dKmem, dtype=np.float64), np.asarray(dVmem, dtype=np.float64)
+    dKb = np.zeros((C,) + dKm.shape[2:])
+    dVb = np.zeros((C,) + dVm.shape[2:])
+    for b in range(idx.shape[0]):
+        rows = [c for j in idx[b] for c in range(off[j], off[j + 1])][:int(mem_len[b])]
+        for r, c in enumerate(rows):
+            dKb[c] += dKm[b, r]
+            dVb[c] += dVm[b, r]
+    return dKb, dVb
 
 
 # ----------------------------------------------------------------------------

@@ -41,6 +41,14 @@ MUTANTS = [
      "test_attention_matches_sdpa", (5, 11, 0, 2, 2)),
     ("attention", "[np.ones((Tq, M), bool),", "[np.arange(M)[None, :] <= np.arange(Tq)[:, None],",
      "test_attention_matches_sdpa", (6, 9, 13, 8, 2)),
+    ("attention_backward", "dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))", "dS = P * dP",
+     "test_attention_backward_matches_central_differences", ()),
+    ("attention_backward", "dvals = P.T @ dO[b, :, h]", "dvals = P.T @ dO[b, :, g]",
+     "test_attention_backward_matches_central_differences", ()),
+    ("attention_backward", "dkeys = scale * (dS.T @ Q[b, :, h])", "dkeys = dS.T @ Q[b, :, h]",
+     "test_attention_backward_matches_central_differences", ()),
+    ("gather_backward", "dKb[c] += dKm[b, r]", "dKb[c] = dKm[b, r]",
+     "test_gather_backward_is_the_adjoint_of_gather", ()),
 ]
 
 

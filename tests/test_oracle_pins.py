@@ -328,3 +328,67 @@ def test_layer_with_all_documents_is_dense_attention_over_bank():
     Od, _ = O.attention(q["Q"].numpy(), q["Kloc"].numpy(), q["Vloc"].numpy(), Kb[None], Vb[None],
                         [int(coff[-1])])
     np.testing.assert_allclose(r["O"], Od, atol=1e-12)
+
+
+# ---------------------------------------------------------------- backward of steps 5 and 4
+def _fd_case(seed=0):
+    rng = np.random.default_rng(seed)
+    B, Tq, Lloc, Hq, Hkv, d, Mmax = 2, 3, 5, 4, 2, 4, 3
+    Q = rng.standard_normal((B, Tq, Hq, d))
+    Kl, Vl = rng.standard_normal((B, Lloc, Hkv, d)), rng.standard_normal((B, Lloc, Hkv, d))
+    Km, Vm = rng.standard_normal((B, Mmax, Hkv, d)), rng.standard_normal((B, Mmax, Hkv, d))
+    ml = np.array([3, 1])
+    dO = rng.standard_normal((B, Tq, Hq, d))
+    return [Q, Kl, Vl, Km, Vm], ml, dO
+
+
+def test_attention_backward_matches_central_differences():
+    """Every input element: d<dO, O>/dx by central differences of the forward oracle."""
+    xs, ml, dO = _fd_case()
+    grads = O.attention_backward(*xs, ml, dO)
+
+    def loss(ys):
+        return float((O.attention(*ys, ml)[0] * dO).sum())
+
+    eps = 1e-6
+    for which, (x, gx) in enumerate(zip(xs, grads)):
+        num = np.zeros_like(x)
+        for i in np.ndindex(x.shape):
+            keep = x[i]
+            x[i] = keep + eps
+            up = loss(xs)
+            x[i] = keep - eps
+            dn = loss(xs)
+            x[i] = keep
+            num[i] = (up - dn) / (2 * eps)
+        assert np.allclose(gx, num, atol=1e-7, rtol=1e-6), which
+
+
+def test_attention_backward_unseen_keys_get_no_gradient():
+    xs, ml, dO = _fd_case(1)
+    dQ, dKl, dVl, dKm, dVm = O.attention_backward(*xs, ml, dO)
+    # memory rows past mem_len and, with Lloc - Tq = 2, local rows 3 and 4 only
+    # for later tokens: row 4 is seen by the last token alone
+    assert not dKm[1, 1:].any() and not dVm[1, 1:].any()
+    xs[0][:, -1] = 0.0
+    dO[:, -1] = 0.0   # the last token contributes nothing, so local row 4 gets nothing
+    _, dKl, dVl, _, _ = O.attention_backward(*xs, ml, dO)
+    assert not dKl[:, 4].any() and not dVl[:, 4].any()
+
+
+def test_gather_backward_is_the_adjoint_of_gather():
+    rng = np.random.default_rng(7)
+    off = np.array([0, 2, 2, 5, 6, 9])          # documents of 2, 0, 3, 1, 3 chunks
+    C, Hkv, d, Mmax = 9, 2, 3, 8
+    idx = np.array([[2, 0, 4], [4, 3, 2], [1, 0, 3]])
+    Kb, Vb = rng.standard_normal((C, Hkv, d)), rng.standard_normal((C, Hkv, d))
+    Km, Vm, ml = O.gather(idx, off, Kb, Vb, Mmax)
+    yK, yV = rng.standard_normal(Km.shape), rng.standard_normal(Vm.shape)
+    for b in range(3):
+        yK[b, ml[b]:] = 0.0
+        yV[b, ml[b]:] = 0.0
+    gK, gV = O.gather_backward(idx, off, yK, yV, ml, C)
+    assert math.isclose((Km * yK).sum(), (Kb * gK).sum(), rel_tol=1e-12)
+    assert math.isclose((Vm * yV).sum(), (Vb * gV).sum(), rel_tol=1e-12)
+    # chunk 6..8 (document 4) is selected by queries 0 and 1: both gradients land
+    assert np.allclose(gK[6], yK[0, 5] + yK[1, 0])
