@@ -334,6 +334,103 @@ def stage_roofline(name: str, ms: float, cfg: synth.Config, counts: dict, peaks:
             "alg_bytes_per_launch": by, "peak_source": f"{peak_kind} hbm_gbs"}
 
 
+def run_backward(args, rank, local_rank, world):
+    """Backward of the query path: per layer msa_sparse_attn_backward + msa_gather_backward, the
+    forward outputs (O, lse, the gathered rows) computed once before timing."""
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    import routed_sparse_attention_chunk_b200 as msa
+    cfg = workload_config(args)
+    counts = workload_counts(cfg)
+    w = MSAWorkload(cfg, device, seed=1000 * rank, step_kind="query")
+    B, c = cfg.B, cfg
+    f32 = dict(dtype=torch.float32, device=device)
+    dt = cfg.torch_dtype
+    layers = []
+    for l in range(cfg.layers):
+        L = w.layers[l]
+        w.route_topk(l)
+        Km = torch.zeros((B, c.Mmax, c.Hkv, c.d), dtype=dt, device=device)
+        Vm = torch.zeros_like(Km)
+        ml = torch.zeros(B, dtype=torch.int32, device=device)
+        msa.gather(w.idx[l], w.coff_d, w.Kb, w.Vb, Km, Vm, ml, w.flag)
+        lse = torch.empty((B, c.Hq, c.Tq), **f32)
+        msa.sparse_attn(L["Q"], L["Kloc"], L["Vloc"], Km, Vm, ml, w.O[l], lse, ws=w.aws, err_flag=w.flag)
+        g = torch.Generator(device=device).manual_seed(7 + l)
+        dO = (0.5 * torch.randn(L["Q"].shape, generator=g, device=device)).to(dt)
+        layers.append((L, Km, Vm, ml, lse, dO))
+    dQ = torch.empty((B, c.Tq, c.Hq, c.d), **f32)
+    dKl, dVl = torch.empty((B, c.Lloc, c.Hkv, c.d), **f32), torch.empty((B, c.Lloc, c.Hkv, c.d), **f32)
+    dKm, dVm = torch.empty((B, c.Mmax, c.Hkv, c.d), **f32), torch.empty((B, c.Mmax, c.Hkv, c.d), **f32)
+    dKb, dVb = torch.zeros((w.C, c.Hkv, c.d), **f32), torch.zeros((w.C, c.Hkv, c.d), **f32)
+    bws = torch.empty(max(256, msa.sparse_attn_backward_workspace_size(B, c.Tq, c.Hq)), dtype=torch.uint8,
+                      device=device)
+    stream = torch.cuda.current_stream()
+    marks = []
+
+    def rec(stage):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        marks.append((stage, e))
+
+    def step(r=None):
+        for l, (L, Km, Vm, ml, lse, dO) in enumerate(layers):
+            msa.sparse_attn_backward(L["Q"], L["Kloc"], L["Vloc"], Km, Vm, ml, w.O[l], lse, dO, dQ, dKl, dVl, dKm,
+                                     dVm, bws, err_flag=w.flag)
+            r and r("attn_backward")
+            msa.gather_backward(w.idx[l], w.coff_d, dKm, dVm, ml, dKb, dVb, w.flag)
+            r and r("gather_backward")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    sampler = ClockSampler(device)
+    sampler.start()
+    n0 = msa.kernel_launch_count()
+    for _ in range(args.steps):
+        rec("start")
+        step(rec)
+    torch.cuda.synchronize()
+    launches = msa.kernel_launch_count() - n0
+    clocks = sampler.stop()
+    stage_ms = {"attn_backward": [], "gather_backward": []}
+    for (s0, e0), (s1, e1) in zip(marks[:-1], marks[1:]):
+        if s1 != "start":
+            stage_ms[s1].append(e0.elapsed_time(e1))
+    step_sum = sum(sum(v) for v in stage_ms.values())
+    flag = int(w.flag.item())
+    barrier(world, device)
+    total_ms = max_over_ranks(step_sum, world, device)
+    ms_per_step = total_ms / args.steps
+    value = B * c.Tq * world / (ms_per_step / 1e3)
+    # CUDA-core fp32 peak from the unit counts and the maximum SM clock: 148 SMs x 128 FMA lanes x 2 flops
+    mhz = clocks.get("sm_max_mhz") or 1965
+    peak = torch.cuda.get_device_properties(device).multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
+    per = float(np.mean(stage_ms["attn_backward"]))
+    flops = 2.5 * counts["attn_flops"] / cfg.layers  # 10 d flops per visible (row, key) pair: s, dp, dq, dk, dv
+    achieved = flops / per / 1e9
+    gper = float(np.mean(stage_ms["gather_backward"]))
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (gradients; inputs " + cfg.dtype + ")", "data": "synthetic",
+        "config": {"workload": workload_label(cfg), "step": "backward: per layer msa_sparse_attn_backward + "
+                   "msa_gather_backward (forward outputs computed before timing)", "parallelism": "single GPU"},
+        "roofline": {"bound": "alu", "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "kernel": "bwd_dq_kernel + bwd_dkv_kernel (CUDA cores, fp32)", "alg_flops_per_launch": flops,
+                     "peak_source": "derived: SMs x 128 fp32 lanes x 2 x max SM clock", "frac": round(achieved / peak, 4),
+                     "avg_launch_ms": round(per, 4), "traffic": None},
+        "stages": {"attn_backward": {"ms_per_launch": round(per, 4)},
+                   "gather_backward": {"ms_per_launch": round(gper, 4)}},
+        "gpu_launches": launches, "clocks": clocks, "err_flag": flag,
+    }
+
+
 def run_gpu(args, rank, local_rank, world):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -570,6 +667,8 @@ def main():
     ap.add_argument("--step", choices=["full", "query"], default=None,
                     help="full: pool + query path per step; query: bank pooled before timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="which_pass", choices=["forward", "backward"], default="forward",
+                    help="backward: time the backward of the query path instead of the forward step")
     ap.add_argument("--bank-kv", choices=["device", "host"], default="device",
                     help="where the pooled K̄ / V̄ live (host: page-locked host memory, the query path only)")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
@@ -580,6 +679,8 @@ def main():
     rank, local_rank, world = dist_env()
     if args.impl == "reference":
         res = run_reference(args, rank, world)
+    elif args.which_pass == "backward":
+        res = run_backward(args, rank, local_rank, world)
     else:
         res = run_gpu(args, rank, local_rank, world)
     if rank == 0 and res is not None:

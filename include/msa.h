@@ -242,6 +242,44 @@ msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const 
                            void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Backward of step 5.  MSA is trained end to end through its sparse attention
+ * ("MSA: Memory Sparse Attention" README, "Architecture"; Figure 2 caption);
+ * the pages print no gradient, so this is the exact derivative of
+ * msa_sparse_attn for an upstream gradient dO:
+ *   p_ij = exp(scale q_i.k_j - lse_i),  D_i = sum dO_i * O_i
+ *   ds_ij = p_ij (dO_i.v_j - D_i)
+ *   dQ_i = scale sum_j ds_ij k_j;  dK_j = scale sum_i ds_ij q_i;  dV_j = sum_i p_ij dO_i
+ * the sums over i running over the q-heads of the GQA group and the tokens that
+ * see key j.  Inputs as in msa_sparse_attn plus the forward's O (dtype dt) and
+ * lse (fp32 [B, Hq, Tq], required) and dO (dtype dt, [B, Tq, Hq, d]).  Outputs
+ * are fp32 and fully written: dQ [B, Tq, Hq, d]; dKloc, dVloc [B, Lloc, Hkv, d];
+ * dKmem, dVmem [B, Mmax, Hkv, d] (rows past mem_len[b] are zero).  The
+ * workspace holds D (msa_sparse_attn_backward_workspace_size bytes).  CUDA-core
+ * kernels, fp32 arithmetic.  Device flags as in msa_sparse_attn.
+ * ---------------------------------------------------------------------- */
+size_t msa_sparse_attn_backward_workspace_size(int64_t B, int Tq, int Hq);
+msa_status msa_sparse_attn_backward(msa_dtype dt, const void* Q, const void* Kloc, const void* Vloc,
+                                    int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d,
+                                    const void* Kmem, const void* Vmem, const int32_t* mem_len, int Mmax,
+                                    float scale, const void* O, const float* lse, const void* dO,
+                                    float* dQ, float* dKloc, float* dVloc, float* dKmem, float* dVmem,
+                                    void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Backward of step 4: the adjoint of msa_gather.  Every gathered row's
+ * gradient (dKmem / dVmem fp32 [B, Mmax, Hkv, d], rows [0, mem_len[b])) is
+ * ADDED into its chunk of dKbar / dVbar (fp32 [C, Hkv, d]; the caller zeroes
+ * them, or passes earlier gradients to accumulate); a chunk selected by
+ * several queries receives the sum.  topk_idx, doc_chunk_off and mem_len are
+ * the ones the forward gather used.  Device flags: MSA_FLAG_INDEX_OOB for a
+ * document index or chunk range out of range (that document is skipped).
+ * ---------------------------------------------------------------------- */
+msa_status msa_gather_backward(const int32_t* topk_idx, int64_t B, int k, const int64_t* doc_chunk_off,
+                               int64_t D, int64_t C, const float* dKmem, const float* dVmem,
+                               const int32_t* mem_len, int Hkv, int d, int Mmax, float* dKbar, float* dVbar,
+                               int32_t* err_flag, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Steps 2-5 for one layer in one call: route + top-k, the selected chunks
  * copied into the workspace (the msa_gather kernel), then attention over them
  * and the local KV.  Arguments as in msa_route_topk and msa_sparse_attn; Mmax

@@ -150,6 +150,31 @@ def sparse_attn(Q, Kloc, Vloc, Kmem, Vmem, mem_len, O, lse=None, scale=0.0, ws=N
           0 if ws is None else ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))
 
 
+def sparse_attn_backward_workspace_size(B, Tq, Hq) -> int:
+    return _lib.load().msa_sparse_attn_backward_workspace_size(B, Tq, Hq)
+
+
+def sparse_attn_backward(Q, Kloc, Vloc, Kmem, Vmem, mem_len, O, lse, dO, dQ, dKloc, dVloc, dKmem, dVmem, ws,
+                         scale=0.0, err_flag=None, stream=None):
+    """Backward of step 5 (msa_sparse_attn_backward): fp32 gradients of Q, Kloc, Vloc, Kmem, Vmem."""
+    B, Tq, Hq, d = Q.shape
+    f = torch.float32
+    _call("msa_sparse_attn_backward", _dt(Q), _p(Q), _p(Kloc, Q.dtype), _p(Vloc, Q.dtype), B, Tq, Kloc.shape[1], Hq,
+          Kloc.shape[2], d, _p(Kmem, Q.dtype), _p(Vmem, Q.dtype), _p(mem_len, torch.int32), Kmem.shape[1],
+          float(scale), _p(O, Q.dtype), _p(lse, f), _p(dO, Q.dtype), _p(dQ, f), _p(dKloc, f), _p(dVloc, f),
+          _p(dKmem, f), _p(dVmem, f), _p(ws), ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))
+
+
+def gather_backward(topk_idx, doc_chunk_off, dKmem, dVmem, mem_len, dKbar, dVbar, err_flag=None, stream=None):
+    """Backward of step 4 (msa_gather_backward): adds the gathered rows' gradients into dKbar / dVbar."""
+    B, k = topk_idx.shape
+    f = torch.float32
+    _call("msa_gather_backward", _p(topk_idx, torch.int32), B, k, _p(doc_chunk_off, torch.int64),
+          doc_chunk_off.numel() - 1, dKbar.shape[0], _p(dKmem, f), _p(dVmem, f), _p(mem_len, torch.int32),
+          dKbar.shape[1], dKbar.shape[2], dKmem.shape[1], _p(dKbar, f), _p(dVbar, f), _p(err_flag, torch.int32),
+          _s(stream))
+
+
 def layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax) -> int:
     return _lib.load().msa_layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax)
 

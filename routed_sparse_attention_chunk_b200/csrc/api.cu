@@ -203,6 +203,43 @@ msa_status msa_gather(msa_dtype dt, const int32_t* topk_idx, int64_t B, int k, c
   return cuda_status(launch_gather(dt, a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t msa_sparse_attn_backward_workspace_size(int64_t B, int Tq, int Hq) {
+  if (B < 0 || Tq < 1 || Hq < 1) return 0;
+  return attn_bwd_workspace_size(B, Tq, Hq);
+}
+
+msa_status msa_sparse_attn_backward(msa_dtype dt, const void* Q, const void* Kloc, const void* Vloc, int64_t B,
+                                    int Tq, int Lloc, int Hq, int Hkv, int d, const void* Kmem, const void* Vmem,
+                                    const int32_t* mem_len, int Mmax, float scale, const void* O, const float* lse,
+                                    const void* dO, float* dQ, float* dKloc, float* dVloc, float* dKmem,
+                                    float* dVmem, void* ws, size_t ws_bytes, int32_t* err_flag,
+                                    msa_stream_t stream) {
+  msa_status st = check_attn(dt, Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, Mmax);
+  if (st != MSA_OK) return st;
+  if (B == 0) return MSA_OK;
+  if (!mem_len || !O || !lse || !dO || !dQ || !dKloc || !dVloc) return MSA_ERR_INVALID_ARG;
+  if (Mmax > 0 && (!Kmem || !Vmem || !dKmem || !dVmem)) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(O) || !aligned16(dO) || !aligned16(Kmem) || !aligned16(Vmem)) return MSA_ERR_INVALID_ARG;
+  const size_t need = attn_bwd_workspace_size(B, Tq, Hq);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  AttnBwdArgs a{Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, Kmem, Vmem, mem_len, Mmax,
+                scale > 0.f ? scale : 1.0f / sqrtf((float)d), O, dO, lse, dQ, dKloc, dVloc, dKmem, dVmem,
+                static_cast<float*>(ws), err_flag};
+  return cuda_status(launch_attn_bwd(dt, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_gather_backward(const int32_t* topk_idx, int64_t B, int k, const int64_t* doc_chunk_off, int64_t D,
+                               int64_t C, const float* dKmem, const float* dVmem, const int32_t* mem_len, int Hkv,
+                               int d, int Mmax, float* dKbar, float* dVbar, int32_t* err_flag,
+                               msa_stream_t stream) {
+  if (B < 0 || k < 1 || D < 1 || C < 0 || Hkv < 1 || Mmax < 0) return MSA_ERR_INVALID_ARG;
+  if (!head_dim_ok(d) || B > 65535 || k > 65535) return MSA_ERR_UNSUPPORTED;
+  if (B == 0 || Mmax == 0) return MSA_OK;
+  if (!topk_idx || !doc_chunk_off || !dKmem || !dVmem || !mem_len || !dKbar || !dVbar) return MSA_ERR_INVALID_ARG;
+  GatherBwdArgs a{topk_idx, B, k, doc_chunk_off, D, C, dKmem, dVmem, mem_len, Hkv, d, Mmax, dKbar, dVbar, err_flag};
+  return cuda_status(launch_gather_bwd(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t msa_sparse_attn_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Mmax) {
   return attn_workspace_size(MSA_BF16, B, Tq, Lloc, Hq, Hkv, d, Mmax);
 }

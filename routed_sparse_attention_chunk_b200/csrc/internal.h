@@ -63,6 +63,40 @@ struct RouteArgs {
 };
 cudaError_t launch_route(msa_dtype dt, const RouteArgs& a, cudaStream_t s);
 
+// Backward of the sparse attention (gradients in fp32; Drow is a workspace of
+// [B, Hq, Tq] fp32 row dot products of dO and O).
+struct AttnBwdArgs {
+  const void *Q, *Kloc, *Vloc;
+  int64_t B;
+  int Tq, Lloc, Hq, Hkv, d;
+  const void *Kmem, *Vmem;
+  const int32_t* mem_len;
+  int Mmax;
+  float scale;
+  const void *O, *dO;
+  const float* lse;
+  float *dQ, *dKloc, *dVloc, *dKmem, *dVmem;
+  float* Drow;
+  int32_t* err_flag;
+};
+size_t attn_bwd_workspace_size(int64_t B, int Tq, int Hq);
+cudaError_t launch_attn_bwd(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s);
+
+// Adjoint of the gather: dKbar / dVbar [C, Hkv, d] fp32 += the gathered rows' gradients.
+struct GatherBwdArgs {
+  const int32_t* topk_idx;
+  int64_t B;
+  int k;
+  const int64_t* doc_chunk_off;
+  int64_t D, C;
+  const float *dKmem, *dVmem;
+  const int32_t* mem_len;
+  int Hkv, d, Mmax;
+  float *dKbar, *dVbar;
+  int32_t* err_flag;
+};
+cudaError_t launch_gather_bwd(const GatherBwdArgs& a, cudaStream_t s);
+
 // Top-k over ordered document keys [B, D]: writes idx / score (score may be null)
 // and optionally decodes every document score into doc_scores.
 struct TopkArgs {

@@ -146,3 +146,26 @@ def test_binding_rejects_host_and_strided_tensors():
         msa.bank_rnorm(x, torch.zeros((4, 8)))
     with pytest.raises(TypeError):
         msa._dt(torch.zeros(2, dtype=torch.float16))
+
+
+def test_backward_entry_points_reject_bad_arguments():
+    lib = _lib.load()
+    bw = dict(dt=1, Q=FAKE, Kl=FAKE, Vl=FAKE, B=1, Tq=8, Lloc=8, Hq=32, Hkv=8, d=128, Km=FAKE, Vm=FAKE, ml=FAKE,
+              Mmax=16, scale=0.0, O=FAKE, lse=FAKE, dO=FAKE, dQ=FAKE, dKl=FAKE, dVl=FAKE, dKm=FAKE, dVm=FAKE,
+              ws=FAKE, wsb=lib.msa_sparse_attn_backward_workspace_size(1, 8, 32), flag=None)
+    call = lambda **kw: lib.msa_sparse_attn_backward(*dict(bw, **kw).values(), None)
+    assert call(d=96) == UNSUPPORTED
+    assert call(Lloc=4) == INVALID            # Lloc < Tq
+    assert call(lse=None) == INVALID          # the forward's lse is required
+    assert call(dKm=None) == INVALID          # memory gradients required when Mmax > 0
+    assert call(dO=FAKE + 4) == INVALID       # misaligned
+    assert call(wsb=3) == WORKSPACE
+    assert call(B=0) == OK
+    assert lib.msa_sparse_attn_backward_workspace_size(2, 5, 4) >= 2 * 5 * 4 * 4
+    gb = dict(idx=FAKE, B=2, k=4, chk=FAKE, D=10, C=30, dKm=FAKE, dVm=FAKE, ml=FAKE, Hkv=8, d=128, Mmax=32,
+              dKb=FAKE, dVb=FAKE, flag=None)
+    gcall = lambda **kw: lib.msa_gather_backward(*dict(gb, **kw).values(), None)
+    assert gcall(d=100) == UNSUPPORTED
+    assert gcall(dKb=None) == INVALID
+    assert gcall(k=0) == INVALID
+    assert gcall(B=0) == OK
