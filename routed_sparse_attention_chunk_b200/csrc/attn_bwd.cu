@@ -13,19 +13,27 @@
 // with the sums over i running over the q-heads of a GQA group and the tokens
 // that see key j.  CUDA-core kernels, fp32 arithmetic, fp32 gradients:
 //   * bwd_rowdot_kernel: D_i, one warp per (token, q-head) row;
-//   * bwd_dq_kernel: 16 rows of one KV head's group per CTA, key tiles of 16
-//     through shared memory (the forward's row layout);
-//   * bwd_dkv_kernel: 16 keys of one KV head per CTA, the rows that see them
+//   * dQ: on the tensor cores for the forward's tensor-core shapes
+//     (attn_bwd_tc.cu), else bwd_dq_kernel: 16 rows of one KV head's group per
+//     CTA, key tiles of 16 through shared memory (the forward's row layout);
+//   * dK / dV: on the tensor cores for those shapes too, else bwd_dkv_kernel:
+//     16 keys of one KV head per CTA, the rows that see them
 //     in blocks of 16 through shared memory; every dK / dV row is written by
 //     exactly one CTA (rows of memory past mem_len get zeros);
 //   * gather_bwd_kernel: one CTA per selected document, fp32 atomic adds into
 //     the chunk gradients (documents chosen by several queries accumulate).
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace msa {
+
+cudaError_t launch_attn_dq_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s, bool* handled);
+cudaError_t launch_attn_dkv_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s, bool* handled);
+
 namespace {
 
 constexpr int kRB = 16, kKT = 16, kNT = 128;  // rows, keys per tile (static smem <= 48 KB at d = 128)
@@ -265,9 +273,18 @@ cudaError_t bwd_t(const AttnBwdArgs& a, cudaStream_t s) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int group = a.Hq / a.Hkv;
-  count_launch();
-  bwd_dq_kernel<T, DH><<<dim3((unsigned)((a.Tq * group + kRB - 1) / kRB), (unsigned)a.Hkv, (unsigned)a.B), kNT, 0, s>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bool handled = false;
+  if ((e = launch_attn_dq_tc(std::is_same<T, float>::value ? MSA_F32 : MSA_BF16, a, s, &handled)) != cudaSuccess)
+    return e;
+  if (!handled) {
+    count_launch();
+    bwd_dq_kernel<T, DH><<<dim3((unsigned)((a.Tq * group + kRB - 1) / kRB), (unsigned)a.Hkv, (unsigned)a.B), kNT, 0,
+                           s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = launch_attn_dkv_tc(std::is_same<T, float>::value ? MSA_F32 : MSA_BF16, a, s, &handled)) != cudaSuccess)
+    return e;
+  if (handled) return cudaSuccess;
   const int tiles = (a.Mmax + kKT - 1) / kKT + (a.Lloc + kKT - 1) / kKT;
   count_launch();
   bwd_dkv_kernel<T, DH><<<dim3((unsigned)tiles, (unsigned)a.Hkv, (unsigned)a.B), kNT, 0, s>>>(a);

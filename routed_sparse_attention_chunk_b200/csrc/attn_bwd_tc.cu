@@ -1,0 +1,685 @@
+// Backward of step 5 on the 5th-generation tensor cores: dQ of the sparse
+// attention over [selected memory rows ++ causal local rows] (the exact
+// derivative of the forward; "MSA: Memory Sparse Attention" README,
+// "Architecture": the layer is trained end to end through its sparse
+// attention).  For a 128-row query tile (the GQA group's G q-heads x 128/G
+// tokens, as in the forward) and every key tile j of 128 keys:
+//   S = Q K_j^T and dP = dO V_j^T        (tcgen05.mma into TMEM, fp32)
+//   P = exp(scale S - lse),  dS = P (dP - D)   (softmax warps, one row per
+//        thread, 32 columns at a time: the forward's log-sum-exp makes a row
+//        max unnecessary); dS is rounded to bf16 and written back over S
+//   dQ += dS K_j                          (dS as the MMA's A operand from TMEM,
+//                                          K_j MN-major from its TMA tile)
+// and dQ * scale is written in fp32 at the end.  The MMAs run in issue order,
+// so S_{j+1} (issued after dQ_j) never overwrites dS_j before it is read.
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..5 softmax.  Every wait is bounded and ends the CTA with
+// MSA_FLAG_TIMEOUT on expiry.
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+#include "tma_host.h"
+
+namespace msa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kRows = 128;   // MMA M: query rows per tile
+constexpr int kKeys = 128;   // keys per tile
+constexpr int kThreads = 192;
+constexpr uint32_t kWaitPolls = 1u << 24;
+
+struct DqParams {
+  const int32_t* mem_len;
+  int32_t* err_flag;
+  const float* lse;   // [B, Hq, Tq] natural log
+  const float* Drow;  // [B, Hq, Tq]
+  float* dQ;          // [B, Tq, Hq, d] fp32
+  int Tq, Lloc, Hq, Hkv, Mmax, G, TB, n_qblk;
+  float scale, scale_log2;
+};
+
+template <int DH>
+struct DqLayout {
+  static constexpr int kBoxes = DH / 64;
+  static constexpr int kQ = kRows * DH * 2;
+  static constexpr int kK = kKeys * DH * 2;
+  static constexpr int kBar = 8 * 16;
+  static constexpr int kSmem = 1024 + 2 * kQ + 4 * kK + kBar;  // Q, dO, K[2], V[2]
+  static constexpr uint32_t kTmemCols = 512;                   // S, dP, dQ (128 each)
+  static_assert(kSmem <= 232448, "shared memory of one CTA");
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                  const __grid_constant__ CUtensorMap tmKm, const __grid_constant__ CUtensorMap tmVm,
+                  const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVl, DqParams p) {
+  using L = DqLayout<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Qs = smem;
+  uint8_t* dOs = Qs + L::kQ;
+  uint8_t* Ks = dOs + L::kQ;        // [2]
+  uint8_t* Vs = Ks + 2 * L::kK;     // [2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Vs + 2 * L::kK);
+  uint64_t* q_full = bars + 0;      // Q and dO landed
+  uint64_t* k_full = bars + 1;      // [2]
+  uint64_t* k_empty = bars + 3;     // [2] dQ MMA of the tile done
+  uint64_t* v_full = bars + 5;      // [2]
+  uint64_t* v_empty = bars + 7;     // [2] dP MMA of the tile done
+  uint64_t* sp_full = bars + 9;     // S and dP in TMEM
+  uint64_t* ds_full = bars + 10;    // dS written over S (128 arrivals)
+  uint64_t* dq_done = bars + 11;    // last dQ MMA done
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = p.n_qblk - 1 - (int)blockIdx.x;  // longest blocks first
+  const int g = blockIdx.y;
+  const int b = blockIdx.z;
+  const int t0 = qb * p.TB;
+  const int tlast = min(t0 + p.TB, p.Tq) - 1;
+  int M = __ldg(p.mem_len + b);
+  if (M < 0 || M > p.Mmax) {
+    if (threadIdx.x == 0 && qb == 0 && g == 0) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
+    M = M < 0 ? 0 : p.Mmax;
+  }
+  const int NM = (M + kKeys - 1) / kKeys;
+  const int T = NM + (p.Lloc - p.Tq + tlast + kKeys) / kKeys;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    mbar_init(sp_full, 1);
+    mbar_init(ds_full, 128);
+    mbar_init(dq_done, 1);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tP = tmem + kKeys, tQ = tmem + 2 * kKeys;
+  bool timed_out = false;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * L::kQ);
+      for (int hh = 0; hh < p.G; ++hh)
+#pragma unroll
+        for (int dc = 0; dc < L::kBoxes; ++dc) {
+          const int x = (g * p.G + hh) * DH + dc * 64, y = b * p.Tq + t0;
+          tma_load_2d(Qs + dc * (kRows * 128) + hh * p.TB * 128, &tmQ, x, y, q_full);
+          tma_load_2d(dOs + dc * (kRows * 128) + hh * p.TB * 128, &tmdO, x, y, q_full);
+        }
+      int j = 0;
+      for (; j < T; ++j) {
+        const int st = j & 1, ph = ((j >> 1) & 1) ^ 1;
+        const bool mem = j < NM;
+        const int y = mem ? b * p.Mmax + j * kKeys : b * p.Lloc + (j - NM) * kKeys;
+        if (!mbar_wait(&k_empty[st], ph, kWaitPolls)) {
+          timed_out = true;
+          break;
+        }
+        mbar_arrive_expect_tx(&k_full[st], L::kK);
+#pragma unroll
+        for (int dc = 0; dc < L::kBoxes; ++dc)
+          tma_load_2d(Ks + st * L::kK + dc * (kKeys * 128), mem ? &tmKm : &tmKl, g * DH + dc * 64, y, &k_full[st]);
+        if (!mbar_wait(&v_empty[st], ph, kWaitPolls)) {
+          timed_out = true;
+          ++j;  // K_j was issued
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[st], L::kK);
+#pragma unroll
+        for (int dc = 0; dc < L::kBoxes; ++dc)
+          tma_load_2d(Vs + st * L::kK + dc * (kKeys * 128), mem ? &tmVm : &tmVl, g * DH + dc * 64, y, &v_full[st]);
+      }
+      // drain: every copy issued must land before the CTA leaves
+      if (!mbar_wait(q_full, 0, kWaitPolls)) timed_out = true;
+      for (int st = 0; st < 2 && st < j; ++st) {
+        const int last = (j - 1 - st) / 2 * 2 + st;
+        if (!mbar_wait(&k_full[st], (last >> 1) & 1, kWaitPolls)) timed_out = true;
+        if (!mbar_wait(&v_full[st], (last >> 1) & 1, kWaitPolls)) timed_out = true;
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kRows, kKeys);
+      constexpr uint32_t idQ = idesc_bf16_f32(kRows, DH, /*b_mn_major=*/true);
+      const uint32_t q0 = smem_u32(Qs), o0 = smem_u32(dOs);
+      // dQ += dS_j K_j: A = dS_j from TMEM (16 keys of bf16 = 8 columns per step)
+      auto issue_dq = [&](int j) {
+        const uint32_t k0 = smem_u32(Ks + (j & 1) * L::kK);
+#pragma unroll
+        for (int k = 0; k < kKeys / 16; ++k)
+          mma_bf16_ts(tQ, tS + k * 8, desc_mn_sw128(k0 + k * 16 * 128, kKeys * 128), idQ, (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&k_empty[j & 1]);
+      };
+      bool ok = mbar_wait(q_full, 0, kWaitPolls);
+      for (int j = 0; ok && j < T; ++j) {
+        const int st = j & 1, ph = (j >> 1) & 1;
+        if (!mbar_wait(&k_full[st], ph, kWaitPolls) || !mbar_wait(&v_full[st], ph, kWaitPolls)) {
+          ok = false;
+          break;
+        }
+        if (j > 0) {
+          if (!mbar_wait(ds_full, (j - 1) & 1, kWaitPolls)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_dq(j - 1);
+        }
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(Ks + st * L::kK), v0 = smem_u32(Vs + st * L::kK);
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const int box = k >> 2, kk = k & 3;
+          mma_bf16_ss(tS, desc_k_sw128(q0 + box * kRows * 128 + kk * 32), desc_k_sw128(k0 + box * kKeys * 128 + kk * 32),
+                      idS, k > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const int box = k >> 2, kk = k & 3;
+          mma_bf16_ss(tP, desc_k_sw128(o0 + box * kRows * 128 + kk * 32), desc_k_sw128(v0 + box * kKeys * 128 + kk * 32),
+                      idS, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&v_empty[st]);
+        mma_commit(sp_full);
+      }
+      if (ok && mbar_wait(ds_full, (T - 1) & 1, kWaitPolls)) {
+        tc_fence_after();
+        issue_dq(T - 1);
+        mma_commit(dq_done);
+      } else {
+        ok = false;
+      }
+      if (!ok) timed_out = true;
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0, kWaitPolls)) timed_out = true;
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int hh = r / p.TB, t = t0 + r - hh * p.TB;
+    const int h = g * p.G + hh;
+    const bool rvalid = t < p.Tq;
+    const int pos = p.Lloc - p.Tq + t;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const float nl = rvalid ? -__ldg(p.lse + ((int64_t)b * p.Hq + h) * p.Tq + t) * 1.4426950408889634f : 0.f;
+    const float Dr = rvalid ? __ldg(p.Drow + ((int64_t)b * p.Hq + h) * p.Tq + t) : 0.f;
+    for (int j = 0; j < T; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(sp_full, j & 1, kWaitPolls))) {
+        timed_out = true;
+        break;
+      }
+      tc_fence_after();
+      const bool memt = j < NM;
+      const int base = memt ? j * kKeys : (j - NM) * kKeys;
+      const int lim = rvalid ? (memt ? M - base : pos - base + 1) : 0;  // keys [0, lim) are visible
+#pragma unroll
+      for (int c0 = 0; c0 < kKeys; c0 += 32) {
+        float s[32], dp[32];
+        tmem_ld16(tS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
+        tmem_ld16(tS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+        tmem_ld16(tP + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
+        tmem_ld16(tP + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = c0 + 2 * i;
+          const float p0 = c < lim ? fast_exp2(fmaf(s[2 * i], p.scale_log2, nl)) : 0.f;
+          const float p1 = c + 1 < lim ? fast_exp2(fmaf(s[2 * i + 1], p.scale_log2, nl)) : 0.f;
+          w[i] = pack_bf16x2(p0 * (dp[2 * i] - Dr), p1 * (dp[2 * i + 1] - Dr));
+        }
+        tmem_st16(tS + lane_off + c0 / 2, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    if (!timed_out && __all_sync(0xffffffffu, mbar_wait(dq_done, 0, kWaitPolls))) {
+      tc_fence_after();
+      float* out = p.dQ + (((int64_t)b * p.Tq + t) * p.Hq + h) * DH;
+#pragma unroll
+      for (int c = 0; c < DH; c += 16) {
+        float o[16];
+        tmem_ld16(tQ + lane_off + c, o);
+        tmem_ld_wait();
+        if (rvalid) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(out + c + i) =
+                make_float4(o[i] * p.scale, o[i + 1] * p.scale, o[i + 2] * p.scale, o[i + 3] * p.scale);
+        }
+      }
+    } else {
+      timed_out = true;
+    }
+  }
+
+  if (timed_out) raise_flag(p.err_flag, MSA_FLAG_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK and dV.  One CTA per 128-key tile of one (KV head, batch row); for every
+// 128-row query tile that sees the keys:
+//   S^T = K Q^T, dP^T = V dO^T          (keys are the MMA's M, one TMEM lane each)
+//   P^T = exp(scale S^T - lse), dS^T = P^T (dP^T - D)   (softmax warps, one key per
+//        thread, the rows' lse and D staged in shared memory); both rounded to
+//        bf16 and written back over S^T and dP^T
+//   dV += P^T dO,  dK += dS^T Q          (A from TMEM, dO / Q MN-major from TMA)
+// dK * scale and dV are written in fp32 at the end; rows of the tile that are
+// not keys (memory rows past mem_len) get zeros.  Query tiles are double
+// buffered; the MMAs of tile i+1's S^T / dP^T follow tile i's dV / dK in issue
+// order, so they never overwrite P^T / dS^T before those are read.
+struct DkvParams {
+  const int32_t* mem_len;
+  int32_t* err_flag;
+  const float* lse;
+  const float* Drow;
+  float *dKm, *dVm, *dKl, *dVl;  // fp32 outputs
+  int Tq, Lloc, Hq, Hkv, Mmax, G, TB, n_qblk, n_mem_tiles;
+  float scale, scale_log2;
+};
+
+template <int DH>
+struct DkvLayout {
+  static constexpr int kBoxes = DH / 64;
+  static constexpr int kT = 128 * DH * 2;  // one 128-row bf16 tile
+  static constexpr int kRed = 2 * 2 * 128 * 4;  // [2 buffers][lse, D][128 rows]
+  static constexpr int kBar = 8 * 16;
+  static constexpr int kSmem = 1024 + 2 * kT + 4 * kT + kRed + kBar;  // K, V, Q[2], dO[2]
+  static constexpr uint32_t kTmemCols = 512;  // S^T, dP^T, dK, dV
+  static_assert(kSmem <= 232448, "shared memory of one CTA");
+};
+
+// Barrier of the 128 softmax threads that also ANDs a predicate over them, so
+// that a failed wait ends the loop for every softmax warp at once.
+__device__ __forceinline__ bool bar_soft_and(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.b32 pi, %1, 0;\n bar.red.and.pred po, 1, 128, pi;\n"
+      " selp.u32 %0, 1, 0, po;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                   const __grid_constant__ CUtensorMap tmKm, const __grid_constant__ CUtensorMap tmVm,
+                   const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVl, DkvParams p) {
+  using L = DkvLayout<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Ks = smem;
+  uint8_t* Vs = Ks + L::kT;
+  uint8_t* Qs = Vs + L::kT;          // [2]
+  uint8_t* dOs = Qs + 2 * L::kT;     // [2]
+  float* red = reinterpret_cast<float*>(dOs + 2 * L::kT);  // [2][2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + L::kRed);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;       // [2]
+  uint64_t* q_empty = bars + 3;      // [2] dV / dK MMAs of the query tile done
+  uint64_t* sp_full = bars + 5;      // S^T, dP^T in TMEM
+  uint64_t* pd_full = bars + 6;      // P^T, dS^T written (128 arrivals)
+  uint64_t* acc_done = bars + 7;
+  uint64_t* drain = bars + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.y;
+  const int b = blockIdx.z;
+  int M = __ldg(p.mem_len + b);
+  if (M < 0 || M > p.Mmax) M = M < 0 ? 0 : p.Mmax;  // flagged by the dQ kernel
+  const bool memt = (int)blockIdx.x < p.n_mem_tiles;
+  const int base = memt ? blockIdx.x * 128 : ((int)blockIdx.x - p.n_mem_tiles) * 128;
+  const int nk = memt ? min(128, p.Mmax - base) : min(128, p.Lloc - base);   // rows of the tile
+  const int nlive = memt ? max(0, min(128, M - base)) : nk;                  // rows that are keys
+  // query tiles that see the keys: all for memory keys; local key l is seen from
+  // token l - (Lloc - Tq) on
+  const int tfirst = memt ? 0 : max(0, base - (p.Lloc - p.Tq));
+  const int i0 = tfirst / p.TB;
+  const int NQ = nlive > 0 ? p.n_qblk - i0 : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    mbar_init(sp_full, 1);
+    mbar_init(pd_full, 128);
+    mbar_init(acc_done, 1);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tP = tmem + 128, tK = tmem + 256, tV = tmem + 384;
+  bool timed_out = false;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0 && NQ > 0) {
+      const int y = memt ? b * p.Mmax + base : b * p.Lloc + base;
+      mbar_arrive_expect_tx(kv_full, 2 * L::kT);
+#pragma unroll
+      for (int dc = 0; dc < L::kBoxes; ++dc) {
+        tma_load_2d(Ks + dc * (128 * 128), memt ? &tmKm : &tmKl, g * DH + dc * 64, y, kv_full);
+        tma_load_2d(Vs + dc * (128 * 128), memt ? &tmVm : &tmVl, g * DH + dc * 64, y, kv_full);
+      }
+      int n = 0;
+      for (; n < NQ; ++n) {
+        const int st = n & 1;
+        if (!mbar_wait(&q_empty[st], ((n >> 1) & 1) ^ 1, kWaitPolls)) {
+          timed_out = true;
+          break;
+        }
+        const int t0 = (i0 + n) * p.TB;
+        mbar_arrive_expect_tx(&q_full[st], 2 * L::kT);
+        for (int hh = 0; hh < p.G; ++hh)
+#pragma unroll
+          for (int dc = 0; dc < L::kBoxes; ++dc) {
+            const int x = (g * p.G + hh) * DH + dc * 64, yq = b * p.Tq + t0;
+            tma_load_2d(Qs + st * L::kT + dc * (128 * 128) + hh * p.TB * 128, &tmQ, x, yq, &q_full[st]);
+            tma_load_2d(dOs + st * L::kT + dc * (128 * 128) + hh * p.TB * 128, &tmdO, x, yq, &q_full[st]);
+          }
+      }
+      if (!mbar_wait(kv_full, 0, kWaitPolls)) timed_out = true;
+      for (int st = 0; st < 2 && st < n; ++st) {
+        const int last = (n - 1 - st) / 2 * 2 + st;
+        if (!mbar_wait(&q_full[st], (last >> 1) & 1, kWaitPolls)) timed_out = true;
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && NQ > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128);
+      constexpr uint32_t idA = idesc_bf16_f32(128, DH, /*b_mn_major=*/true);
+      const uint32_t k0 = smem_u32(Ks), v0 = smem_u32(Vs);
+      // dV += P^T dO, dK += dS^T Q for query tile n (A from TMEM: 16 rows of bf16 = 8 columns)
+      auto issue_acc = [&](int n) {
+        const uint32_t q0 = smem_u32(Qs + (n & 1) * L::kT), o0 = smem_u32(dOs + (n & 1) * L::kT);
+#pragma unroll
+        for (int k = 0; k < 128 / 16; ++k) {
+          mma_bf16_ts(tV, tS + k * 8, desc_mn_sw128(o0 + k * 16 * 128, 128 * 128), idA, (n > 0 || k > 0) ? 1u : 0u);
+          mma_bf16_ts(tK, tP + k * 8, desc_mn_sw128(q0 + k * 16 * 128, 128 * 128), idA, (n > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&q_empty[n & 1]);
+      };
+      bool ok = mbar_wait(kv_full, 0, kWaitPolls);
+      for (int n = 0; ok && n < NQ; ++n) {
+        if (!mbar_wait(&q_full[n & 1], (n >> 1) & 1, kWaitPolls)) {
+          ok = false;
+          break;
+        }
+        if (n > 0) {
+          if (!mbar_wait(pd_full, (n - 1) & 1, kWaitPolls)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_acc(n - 1);
+        }
+        tc_fence_after();
+        const uint32_t q0 = smem_u32(Qs + (n & 1) * L::kT), o0 = smem_u32(dOs + (n & 1) * L::kT);
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const int box = k >> 2, kk = k & 3;
+          mma_bf16_ss(tS, desc_k_sw128(k0 + box * 128 * 128 + kk * 32), desc_k_sw128(q0 + box * 128 * 128 + kk * 32), idS,
+                      k > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const int box = k >> 2, kk = k & 3;
+          mma_bf16_ss(tP, desc_k_sw128(v0 + box * 128 * 128 + kk * 32), desc_k_sw128(o0 + box * 128 * 128 + kk * 32), idS,
+                      k > 0 ? 1u : 0u);
+        }
+        mma_commit(sp_full);
+      }
+      if (ok && mbar_wait(pd_full, (NQ - 1) & 1, kWaitPolls)) {
+        tc_fence_after();
+        issue_acc(NQ - 1);
+        mma_commit(acc_done);
+      } else {
+        ok = false;
+      }
+      if (!ok) timed_out = true;
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0, kWaitPolls)) timed_out = true;
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax (one key per thread)
+    const int q = warp & 3;
+    const int kr = q * 32 + lane;  // this thread's key row of the tile (TMEM lane)
+    const int tid = threadIdx.x - 64;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool key_live = kr < nlive;
+    for (int n = 0; n < NQ; ++n) {
+      // the rows' -lse * log2(e) and D of this query tile, in the buffer of its parity
+      float* rl = red + (n & 1) * 256;
+      {
+        const int hh = tid / p.TB, t = (i0 + n) * p.TB + tid - hh * p.TB;
+        const int64_t li = ((int64_t)b * p.Hq + g * p.G + hh) * p.Tq + t;
+        rl[tid] = t < p.Tq ? -__ldg(p.lse + li) * 1.4426950408889634f : 0.f;
+        rl[128 + tid] = t < p.Tq ? __ldg(p.Drow + li) : 0.f;
+      }
+      // the staging barrier doubles as a vote on the wait, so the warps leave together
+      const bool okw = __all_sync(0xffffffffu, mbar_wait(sp_full, n & 1, kWaitPolls));
+      if (!bar_soft_and(okw)) {
+        timed_out = true;
+        break;
+      }
+      tc_fence_after();
+      const int t0 = (i0 + n) * p.TB;
+      const int key = base + kr;  // local row index for local tiles
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        float s[32], dp[32];
+        tmem_ld16(tS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
+        tmem_ld16(tS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+        tmem_ld16(tP + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
+        tmem_ld16(tP + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
+        tmem_ld_wait();
+        uint32_t wp[16], wd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float pr[2], ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int r = c0 + 2 * i + u;
+            const int t = t0 + (r & (p.TB - 1));
+            const bool vis = key_live && t < p.Tq && (memt || key <= p.Lloc - p.Tq + t);
+            pr[u] = vis ? fast_exp2(fmaf(s[2 * i + u], p.scale_log2, rl[r])) : 0.f;
+            ds[u] = pr[u] * (dp[2 * i + u] - rl[128 + r]);
+          }
+          wp[i] = pack_bf16x2(pr[0], pr[1]);
+          wd[i] = pack_bf16x2(ds[0], ds[1]);
+        }
+        tmem_st16(tS + lane_off + c0 / 2, wp);
+        tmem_st16(tP + lane_off + c0 / 2, wd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(pd_full);
+    }
+    // outputs: dK * scale, dV (fp32); rows that are not keys get zeros
+    const bool got = NQ > 0 && !timed_out && __all_sync(0xffffffffu, mbar_wait(acc_done, 0, kWaitPolls));
+    if (NQ > 0 && !got) timed_out = true;
+    if (kr < nk || NQ > 0) {
+      float* dKo = (memt ? p.dKm : p.dKl) + (((int64_t)b * (memt ? p.Mmax : p.Lloc) + base + kr) * p.Hkv + g) * DH;
+      float* dVo = (memt ? p.dVm : p.dVl) + (((int64_t)b * (memt ? p.Mmax : p.Lloc) + base + kr) * p.Hkv + g) * DH;
+      if (got) tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < DH; c += 16) {
+        float ok_[16], ov[16];
+        if (got) {
+          tmem_ld16(tK + lane_off + c, ok_);
+          tmem_ld16(tV + lane_off + c, ov);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ok_[i] = ov[i] = 0.f;
+        }
+        if (kr < nk) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float m = key_live ? 1.f : 0.f;
+            *reinterpret_cast<float4*>(dKo + c + i) =
+                make_float4(ok_[i] * p.scale * m, ok_[i + 1] * p.scale * m, ok_[i + 2] * p.scale * m, ok_[i + 3] * p.scale * m);
+            *reinterpret_cast<float4*>(dVo + c + i) = make_float4(ov[i] * m, ov[i + 1] * m, ov[i + 2] * m, ov[i + 3] * m);
+          }
+        }
+      }
+    }
+  }
+
+  if (timed_out) raise_flag(p.err_flag, MSA_FLAG_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace
+
+// dK / dV on the tensor cores (same shapes as the dQ kernel).
+cudaError_t launch_attn_dkv_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s, bool* handled) {
+  *handled = false;
+  if (dt != MSA_BF16 || a.d != 128) return cudaSuccess;
+  const int G = a.Hq / a.Hkv;
+  if (G < 1 || 128 % G != 0 || 128 / G < 8 || a.B > 65535 || a.Hkv > 65535) return cudaSuccess;
+  constexpr int DH = 128;
+  using L = DkvLayout<DH>;
+  const int TB = 128 / G;
+  CUtensorMap tq, tdo, tkm, tvm, tkl, tvl;
+  const uint64_t rowkv = (uint64_t)a.Hkv * DH * 2;
+  const int64_t mrows = a.B * (int64_t)(a.Mmax > 0 ? a.Mmax : 1);
+  if (!make_tmap_2d_bf16(&tq, a.Q, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB) ||
+      !make_tmap_2d_bf16(&tdo, a.dO, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB) ||
+      !make_tmap_2d_bf16(&tkm, a.Mmax > 0 ? a.Kmem : a.Kloc, (uint64_t)a.Hkv * DH,
+                         (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, 128) ||
+      !make_tmap_2d_bf16(&tvm, a.Mmax > 0 ? a.Vmem : a.Vloc, (uint64_t)a.Hkv * DH,
+                         (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, 128) ||
+      !make_tmap_2d_bf16(&tkl, a.Kloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, 128) ||
+      !make_tmap_2d_bf16(&tvl, a.Vloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, 128))
+    return cudaErrorInvalidValue;
+  DkvParams p;
+  p.mem_len = a.mem_len;
+  p.err_flag = a.err_flag;
+  p.lse = a.lse;
+  p.Drow = a.Drow;
+  p.dKm = a.dKmem;
+  p.dVm = a.dVmem;
+  p.dKl = a.dKloc;
+  p.dVl = a.dVloc;
+  p.Tq = a.Tq;
+  p.Lloc = a.Lloc;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.Mmax = a.Mmax;
+  p.G = G;
+  p.TB = TB;
+  p.n_qblk = (a.Tq + TB - 1) / TB;
+  p.n_mem_tiles = (a.Mmax + 127) / 128;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  cudaError_t e = cudaFuncSetAttribute(attn_dkv_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+  if (e != cudaSuccess) return e;
+  const int tiles = p.n_mem_tiles + (a.Lloc + 127) / 128;
+  *handled = true;
+  count_launch();
+  attn_dkv_tc_kernel<DH><<<dim3((unsigned)tiles, (unsigned)a.Hkv, (unsigned)a.B), kThreads, L::kSmem, s>>>(
+      tq, tdo, tkm, tvm, tkl, tvl, p);
+  return cudaGetLastError();
+}
+
+// dQ on the tensor cores for the shapes the forward's tensor-core kernel takes
+// (bf16, d = 128, a GQA group dividing 128 rows into blocks of >= 8 tokens).
+cudaError_t launch_attn_dq_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s, bool* handled) {
+  *handled = false;
+  if (dt != MSA_BF16 || a.d != 128) return cudaSuccess;
+  const int G = a.Hq / a.Hkv;
+  if (G < 1 || 128 % G != 0 || 128 / G < 8 || a.B > 65535 || a.Hkv > 65535) return cudaSuccess;
+  constexpr int DH = 128;
+  using L = DqLayout<DH>;
+  const int TB = kRows / G;
+  CUtensorMap tq, tdo, tkm, tvm, tkl, tvl;
+  const uint64_t rowkv = (uint64_t)a.Hkv * DH * 2;
+  const int64_t mrows = a.B * (int64_t)(a.Mmax > 0 ? a.Mmax : 1);
+  if (!make_tmap_2d_bf16(&tq, a.Q, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB) ||
+      !make_tmap_2d_bf16(&tdo, a.dO, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB) ||
+      !make_tmap_2d_bf16(&tkm, a.Mmax > 0 ? a.Kmem : a.Kloc, (uint64_t)a.Hkv * DH,
+                         (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, kKeys) ||
+      !make_tmap_2d_bf16(&tvm, a.Mmax > 0 ? a.Vmem : a.Vloc, (uint64_t)a.Hkv * DH,
+                         (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, kKeys) ||
+      !make_tmap_2d_bf16(&tkl, a.Kloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKeys) ||
+      !make_tmap_2d_bf16(&tvl, a.Vloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKeys))
+    return cudaErrorInvalidValue;
+  DqParams p;
+  p.mem_len = a.mem_len;
+  p.err_flag = a.err_flag;
+  p.lse = a.lse;
+  p.Drow = a.Drow;
+  p.dQ = a.dQ;
+  p.Tq = a.Tq;
+  p.Lloc = a.Lloc;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.Mmax = a.Mmax;
+  p.G = G;
+  p.TB = TB;
+  p.n_qblk = (a.Tq + TB - 1) / TB;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  cudaError_t e = cudaFuncSetAttribute(attn_dq_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+  if (e != cudaSuccess) return e;
+  *handled = true;
+  count_launch();
+  attn_dq_tc_kernel<DH><<<dim3((unsigned)p.n_qblk, (unsigned)a.Hkv, (unsigned)a.B), kThreads, L::kSmem, s>>>(
+      tq, tdo, tkm, tvm, tkl, tvl, p);
+  return cudaGetLastError();
+}
+
+}  // namespace msa
