@@ -408,22 +408,32 @@ def run_backward(args, rank, local_rank, world):
     total_ms = max_over_ranks(step_sum, world, device)
     ms_per_step = total_ms / args.steps
     value = B * c.Tq * world / (ms_per_step / 1e3)
-    # CUDA-core fp32 peak from the unit counts and the maximum SM clock: 148 SMs x 128 FMA lanes x 2 flops
-    mhz = clocks.get("sm_max_mhz") or 1965
-    peak = torch.cuda.get_device_properties(device).multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
     per = float(np.mean(stage_ms["attn_backward"]))
     flops = 2.5 * counts["attn_flops"] / cfg.layers  # 10 d flops per visible (row, key) pair: s, dp, dq, dk, dv
     achieved = flops / per / 1e9
     gper = float(np.mean(stage_ms["gather_backward"]))
+    G = c.Hq // c.Hkv
+    tensor = cfg.dtype == "bf16" and c.d == 128 and 128 % G == 0 and 128 // G >= 8
+    if tensor:  # the tcgen05 dQ and dK / dV kernels: the bf16 tensor peak
+        peaks, peak_kind = load_peaks()
+        long_region = step_sum > 2000.0
+        pname = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+        peak = peaks.get(pname, FALLBACK_PEAKS["bf16_tflops"])
+        bound, kname, psrc = "tensor", "attn_dq_tc_kernel + attn_dkv_tc_kernel (tcgen05)", f"{peak_kind} {pname}"
+    else:  # CUDA-core fp32 peak from the unit counts and the maximum SM clock: SMs x 128 FMA lanes x 2 flops
+        mhz = clocks.get("sm_max_mhz") or 1965
+        peak = torch.cuda.get_device_properties(device).multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
+        bound, kname = "alu", "bwd_dq_kernel + bwd_dkv_kernel (CUDA cores, fp32)"
+        psrc = "derived: SMs x 128 fp32 lanes x 2 x max SM clock"
     return {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 (gradients; inputs " + cfg.dtype + ")", "data": "synthetic",
         "config": {"workload": workload_label(cfg), "step": "backward: per layer msa_sparse_attn_backward + "
                    "msa_gather_backward (forward outputs computed before timing)", "parallelism": "single GPU"},
-        "roofline": {"bound": "alu", "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
-                     "kernel": "bwd_dq_kernel + bwd_dkv_kernel (CUDA cores, fp32)", "alg_flops_per_launch": flops,
-                     "peak_source": "derived: SMs x 128 fp32 lanes x 2 x max SM clock", "frac": round(achieved / peak, 4),
+        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "kernel": kname, "alg_flops_per_launch": flops,
+                     "peak_source": psrc, "frac": round(achieved / peak, 4),
                      "avg_launch_ms": round(per, 4), "traffic": None},
         "stages": {"attn_backward": {"ms_per_launch": round(per, 4)},
                    "gather_backward": {"ms_per_launch": round(gper, 4)}},
