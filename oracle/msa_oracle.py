@@ -41,6 +41,11 @@ the plainest reading and says so at the function (the list of readings):
      sparse attention but print no gradient) is the exact derivative of R6's
      attention, and the gather's adjoint adds each gathered row's gradient back
      into its chunk; the top-k choice itself carries no gradient.
+  R15 The routing score's gradient (the model card names an auxiliary routing
+     loss but does not define it) is taken for an upstream gradient of the
+     selected documents' scores: the max passes it to its argmax (token, chunk),
+     first in (chunk, token) order on ties, and the cosine's derivative spreads it
+     over that token's Qr and that chunk's K̄r.
 
 Layouts are row-major with the innermost dimension last:
   K, V [Ntok, Hkv, d]; Kr [Ntok, Hr, dr]; doc_tok_off int64 [D+1]
@@ -400,6 +405,47 @@ def gather_backward(topk_idx, doc_chunk_off, dKmem, dVmem, mem_len, C: int):
             dKb[c] += dKm[b, r]
             dVb[c] += dVm[b, r]
     return dKb, dVb
+
+
+def route_backward(Qr, Krbar, doc_chunk_off, topk_idx, d_score):
+    """Gradient of the selected documents' scores (reading R15).
+
+    score(b, j) = max over chunks c of j and tokens t of s[b, t, c] with
+    s = (1/Hr) sum_h cos(Qr[b, t, h], K̄r[c, h]) (route()).  Given d_score[b, r],
+    the upstream gradient of score(b, topk_idx[b, r]) (e.g. from an auxiliary
+    routing loss), the max passes it to its argmax (the first pair in (chunk,
+    token) order on ties) and the cosine's derivative
+        d cos(q, k) / dq = k / (|q| |k|) - cos(q, k) q / |q|^2
+    distributes it to that token's Qr and that chunk's K̄r, per head, with 1/Hr.
+    Returns (dQr [B, Tq, Hr, dr], dKrbar [C, Hr, dr]) in fp64.  Documents with
+    no chunks get no gradient.  Pin: central finite differences of
+    sum_r d_score[b, r] * score(b, topk_idx[b, r]) on a case with distinct maxima.
+    """
+    Qr = np.asarray(Qr, dtype=np.float64)
+    Kb = np.asarray(Krbar, dtype=np.float64)
+    off = np.asarray(doc_chunk_off, dtype=np.int64)
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    g = np.asarray(d_score, dtype=np.float64)
+    B, Tq, Hr, dr = Qr.shape
+    dQ = np.zeros_like(Qr)
+    dK = np.zeros_like(Kb)
+    s = cosine_scores(Qr, Kb)                                   # [B, Tq, C]
+    for b in range(B):
+        for r, j in enumerate(idx[b]):
+            a, e = int(off[j]), int(off[j + 1])
+            if e <= a:
+                continue
+            sc = s[b, :, a:e].T                                 # [chunks, Tq]: chunk-major order
+            c_rel, t = np.unravel_index(int(np.argmax(sc)), sc.shape)
+            c = a + int(c_rel)
+            for h in range(Hr):
+                q, k = Qr[b, t, h], Kb[c, h]
+                nq, nk = max(np.linalg.norm(q), NORM_EPS), max(np.linalg.norm(k), NORM_EPS)
+                cos = float(q @ k) / (nq * nk)
+                w = g[b, r] / Hr
+                dQ[b, t, h] += w * (k / (nq * nk) - cos * q / nq ** 2)
+                dK[c, h] += w * (q / (nq * nk) - cos * k / nk ** 2)
+    return dQ, dK
 
 
 # ----------------------------------------------------------------------------

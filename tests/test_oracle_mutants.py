@@ -49,6 +49,10 @@ MUTANTS = [
      "test_attention_backward_matches_central_differences", ()),
     ("gather_backward", "dKb[c] += dKm[b, r]", "dKb[c] = dKm[b, r]",
      "test_gather_backward_is_the_adjoint_of_gather", ()),
+    ("route_backward", "dQ[b, t, h] += w * (k / (nq * nk) - cos * q / nq ** 2)", "dQ[b, t, h] += w * k / (nq * nk)",
+     "test_route_backward_matches_central_differences", ()),
+    ("route_backward", "sc = s[b, :, a:e].T", "sc = s[b, :, a:e]",
+     "test_route_backward_matches_central_differences", ()),
 ]
 
 

@@ -392,3 +392,35 @@ def test_gather_backward_is_the_adjoint_of_gather():
     assert math.isclose((Vm * yV).sum(), (Vb * gV).sum(), rel_tol=1e-12)
     # chunk 6..8 (document 4) is selected by queries 0 and 1: both gradients land
     assert np.allclose(gK[6], yK[0, 5] + yK[1, 0])
+
+
+def test_route_backward_matches_central_differences():
+    """d/dx of sum_r g[b, r] * score(b, topk[b, r]) by central differences (distinct maxima)."""
+    rng = np.random.default_rng(11)
+    B, Tq, Hr, dr = 2, 3, 2, 4
+    off = np.array([0, 2, 3, 6, 6, 8])                 # documents of 2, 1, 3, 0, 2 chunks
+    C = int(off[-1])
+    Qr = rng.standard_normal((B, Tq, Hr, dr))
+    Kb = rng.standard_normal((C, Hr, dr))
+    idx = np.array([[2, 0, 3], [4, 1, 2]])            # document 3 is empty: no gradient from it
+    g = rng.standard_normal((B, 3))
+    dQ, dK = O.route_backward(Qr, Kb, off, idx, g)
+
+    def loss(q, k):
+        sc = O.route(q, k, off)
+        return float(sum(g[b, r] * sc[b, j] for b in range(B) for r, j in enumerate(idx[b]) if np.isfinite(sc[b, j])))
+
+    eps = 1e-6
+    for x, gx, args in ((Qr, dQ, 0), (Kb, dK, 1)):
+        num = np.zeros_like(x)
+        for i in np.ndindex(x.shape):
+            keep = x[i]
+            x[i] = keep + eps
+            up = loss(Qr, Kb)
+            x[i] = keep - eps
+            dn = loss(Qr, Kb)
+            x[i] = keep
+            num[i] = (up - dn) / (2 * eps)
+        assert np.allclose(gx, num, atol=1e-7, rtol=1e-6), args
+    # only the argmax token of each selected document is touched
+    assert np.count_nonzero(np.abs(dQ).sum(axis=(2, 3))) <= 2 * 2
