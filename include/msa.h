@@ -280,6 +280,38 @@ msa_status msa_gather_backward(const int32_t* topk_idx, int64_t B, int k, const 
                                int32_t* err_flag, msa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Backward of step 2 for the selected documents.  A document's routing score
+ * is the max over its chunks c and the query's tokens t of the head-mean
+ * cosine s(t, c) = (1/Hr) sum_h cos(Qr[b, t, h], Krbar[c, h]) ("MSA: Memory
+ * Sparse Attention" README, "Architecture"); the model card's auxiliary
+ * routing loss is not defined on the pages, so its gradient with respect to
+ * each selected document's score, d_score (fp32 [B, k], host layout as
+ * topk_idx), is the input.  The max passes it to its argmax pair (t*, c*),
+ * the first in (chunk, token) order on exact ties, with s computed as
+ * msa_route_topk computes it (kr_rnorm for the key norms); then for every
+ * router head h, with q = Qr[b, t*, h], k = Krbar[c*, h]:
+ *   dQr[b, t*, h]  += d_score / Hr * (k / (|q| |k|) - cos(q, k) q / |q|^2)
+ *   dKrbar[c*, h]  += d_score / Hr * (q / (|q| |k|) - cos(q, k) k / |k|^2)
+ * (norms floored at 1e-12).  Qr, Krbar, kr_rnorm, doc_chunk_off and topk_idx
+ * are the ones the forward routing used (dtype dt; fp32 / int64 / int32).
+ * dQr (fp32 [B, Tq, Hr, dr]) and dKrbar (fp32 [C, Hr, dr]) are ADDED to: the
+ * caller zeroes them or passes earlier gradients; a token or chunk that wins
+ * for several documents or queries receives the sum (fp32 atomics, so the
+ * summation order is not fixed).  A document with no chunks gets no
+ * gradient.  The workspace holds msa_route_backward_workspace_size(B, k)
+ * bytes.  Errors as msa_route_topk; device flags: MSA_FLAG_INDEX_OOB for a
+ * document index or chunk range out of range, or a document with more than
+ * 2^31 - 1 (chunk, token) pairs (that document is skipped).
+ * ---------------------------------------------------------------------- */
+size_t msa_route_backward_workspace_size(int64_t B, int k);
+msa_status msa_route_backward(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr,
+                              const void* Krbar, const float* kr_rnorm,
+                              const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
+                              const int32_t* topk_idx, const float* d_score,
+                              float* dQr, float* dKrbar,
+                              void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Steps 2-5 for one layer in one call: route + top-k, the selected chunks
  * copied into the workspace (the msa_gather kernel), then attention over them
  * and the local KV.  Arguments as in msa_route_topk and msa_sparse_attn; Mmax

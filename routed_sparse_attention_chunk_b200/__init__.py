@@ -175,6 +175,23 @@ def gather_backward(topk_idx, doc_chunk_off, dKmem, dVmem, mem_len, dKbar, dVbar
           _s(stream))
 
 
+def route_backward_workspace_size(B, k) -> int:
+    return _lib.load().msa_route_backward_workspace_size(B, k)
+
+
+def route_backward(Qr, Krbar, kr_rnorm, doc_chunk_off, topk_idx, d_score, dQr, dKrbar, ws, err_flag=None,
+                   stream=None):
+    """Backward of step 2 (msa_route_backward): adds the selected documents' routing-score gradients
+    d_score [B, k] into dQr [B, Tq, Hr, dr] and dKrbar [C, Hr, dr] (fp32)."""
+    B, Tq, Hr, dr = Qr.shape
+    k = topk_idx.shape[1]
+    f = torch.float32
+    _call("msa_route_backward", _dt(Qr), _p(Qr), B, Tq, Hr, dr, _p(Krbar, Qr.dtype), _p(kr_rnorm, f),
+          _p(doc_chunk_off, torch.int64), doc_chunk_off.numel() - 1, Krbar.shape[0], k,
+          _p(topk_idx, torch.int32), _p(d_score, f), _p(dQr, f), _p(dKrbar, f), _p(ws),
+          ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))
+
+
 def layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax) -> int:
     return _lib.load().msa_layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax)
 

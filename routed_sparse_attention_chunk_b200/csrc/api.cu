@@ -240,6 +240,27 @@ msa_status msa_gather_backward(const int32_t* topk_idx, int64_t B, int k, const 
   return cuda_status(launch_gather_bwd(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t msa_route_backward_workspace_size(int64_t B, int k) {
+  if (B < 0 || k < 1) return 0;
+  return route_bwd_workspace_size(B, k);
+}
+
+msa_status msa_route_backward(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr, const void* Krbar,
+                              const float* kr_rnorm, const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
+                              const int32_t* topk_idx, const float* d_score, float* dQr, float* dKrbar, void* ws,
+                              size_t ws_bytes, int32_t* err_flag, msa_stream_t stream) {
+  msa_status st = check_route(dt, Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, k, topk_idx);
+  if (st != MSA_OK) return st;
+  if (B > 65535 || k > 65535) return MSA_ERR_UNSUPPORTED;
+  if (B == 0) return MSA_OK;
+  if (!d_score || !dQr || !dKrbar) return MSA_ERR_INVALID_ARG;
+  const size_t need = route_bwd_workspace_size(B, k);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  RouteBwdArgs a{Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, k, topk_idx, d_score,
+                 dQr, dKrbar, ws, err_flag};
+  return cuda_status(launch_route_bwd(dt, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t msa_sparse_attn_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Mmax) {
   return attn_workspace_size(MSA_BF16, B, Tq, Lloc, Hq, Hkv, d, Mmax);
 }

@@ -97,6 +97,25 @@ struct GatherBwdArgs {
 };
 cudaError_t launch_gather_bwd(const GatherBwdArgs& a, cudaStream_t s);
 
+// Backward of the routing score of the selected documents (route_bwd.cu).
+struct RouteBwdArgs {
+  const void* Qr;
+  int64_t B;
+  int Tq, Hr, dr;
+  const void* Krbar;
+  const float* kr_rnorm;
+  const int64_t* doc_chunk_off;
+  int64_t D, C;
+  int k;
+  const int32_t* topk_idx;
+  const float* d_score;
+  float *dQr, *dKrbar;
+  void* ws;  // route_bwd_workspace_size bytes
+  int32_t* err_flag;
+};
+size_t route_bwd_workspace_size(int64_t B, int k);
+cudaError_t launch_route_bwd(msa_dtype dt, const RouteBwdArgs& a, cudaStream_t s);
+
 // Top-k over ordered document keys [B, D]: writes idx / score (score may be null)
 // and optionally decodes every document score into doc_scores.
 struct TopkArgs {

@@ -16,7 +16,7 @@ import routed_sparse_attention_chunk_b200 as msa
 from oracle import msa_oracle as O
 from workloads import synth
 
-from .helpers import attn_on_gpu, to64
+from .helpers import attn_on_gpu, pool_on_gpu, route_on_gpu, to64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -126,3 +126,90 @@ def test_layer_backward_chain_matches_oracle_chain():
     r = O.attention_backward(to64(q["Q"]), to64(q["Kloc"]), to64(q["Vloc"]), oKm, oVm, oml, to64(dO))
     oKb, oVb = O.gather_backward(idx, coff, r[3], r[4], oml, C)
     _check((dQ, dKb, dVb), (r[0], oKb, oVb), TOL_BWD_BF16, names=("dQ", "dKbar", "dVbar"))
+
+
+def _route_bwd_case(B, Tq, Hr, dr, lengths, k, dtype, seed, idx=None):
+    """Random Qr / K̄r and a selection; documents whose best (chunk, token) pair is within 1e-4 of
+    the runner-up get d_score 0, so the argmax both sides take is unique wherever it matters."""
+    rng = np.random.default_rng(seed)
+    coff = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    C, D = int(coff[-1]), len(lengths)
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    Qr = torch.randn((B, Tq, Hr, dr), generator=g, device=DEV).to(dtype)
+    Krb = torch.randn((max(C, 1), Hr, dr), generator=g, device=DEV).to(dtype)[:C].contiguous()
+    rn = torch.empty((C, Hr), dtype=torch.float32, device=DEV)
+    msa.bank_rnorm(Krb, rn)
+    if idx is None:
+        idx = np.stack([rng.choice(D, size=k, replace=False) for _ in range(B)]).astype(np.int32)
+    s = O.cosine_scores(to64(Qr), to64(Krb))                 # [B, Tq, C]
+    dsc = rng.standard_normal((B, k)).astype(np.float32)
+    for b in range(B):
+        for r, j in enumerate(idx[b]):
+            v = np.sort(s[b, :, coff[j]:coff[j + 1]].ravel())
+            if v.size > 1 and v[-1] - v[-2] < 1e-4:
+                dsc[b, r] = 0.0
+    return Qr, Krb, rn, coff, idx, dsc
+
+
+def _route_bwd_gpu(Qr, Krb, rn, coff, idx, dsc):
+    B, Tq, Hr, dr = Qr.shape
+    t = lambda a: torch.from_numpy(a).to(DEV)
+    dQr = torch.zeros((B, Tq, Hr, dr), dtype=torch.float32, device=DEV)
+    dKrb = torch.zeros((Krb.shape[0], Hr, dr), dtype=torch.float32, device=DEV)
+    ws = torch.empty(msa.route_backward_workspace_size(B, idx.shape[1]), dtype=torch.uint8, device=DEV)
+    flag = torch.zeros(1, dtype=torch.int32, device=DEV)
+    msa.route_backward(Qr, Krb, rn, t(coff), t(idx), t(dsc), dQr, dKrb, ws, flag)
+    torch.cuda.synchronize()
+    return dQr, dKrb, flag
+
+
+@pytest.mark.parametrize("B,Tq,Hr,dr,maxlen,D,k,dtype", [
+    (3, 5, 8, 128, 6, 30, 6, torch.float32),       # few pairs per document
+    (2, 64, 8, 128, 40, 24, 8, torch.bfloat16),    # thousands of pairs: every split busy, ragged tail
+    (4, 1, 4, 64, 9, 50, 16, torch.bfloat16),      # decode: one token, max over chunks only
+    (2, 33, 1, 64, 3, 12, 12, torch.float32),      # Hr = 1, every document selected
+])
+def test_route_backward_matches_oracle(B, Tq, Hr, dr, maxlen, D, k, dtype):
+    rng = np.random.default_rng(B * 1000 + Tq)
+    lengths = rng.integers(1, maxlen + 1, size=D)
+    lengths[D // 2] = 0                               # an empty document (no gradient if selected)
+    Qr, Krb, rn, coff, idx, dsc = _route_bwd_case(B, Tq, Hr, dr, lengths, k, dtype, seed=B + Tq)
+    dQr, dKrb, flag = _route_bwd_gpu(Qr, Krb, rn, coff, idx, dsc)
+    oQ, oK = O.route_backward(to64(Qr), to64(Krb), coff, idx, dsc)
+    assert flag.item() == 0
+    assert (dsc != 0).sum() >= idx.size // 2          # most documents have a unique argmax
+    _check((dQr, dKrb), (oQ, oK), TOL_BWD_F32, names=("dQr", "dKrbar"))
+
+
+def test_route_backward_accumulates_over_shared_documents_after_routing():
+    """Selection by the routing kernels themselves (so several queries pick the same documents);
+    the gradients are added onto what dQr / dK̄r already hold.  64 selections from 40 documents
+    must share some."""
+    cfg = synth.get_config("1m").scaled(D=40, B=4, Tq=16, Lloc=32)
+    q = synth.gen_query(cfg, 0, DEV)
+    K, V, Kr = synth.gen_raw_slab(cfg, 0, cfg.D, DEV, Qr0=q["Qr"][0])
+    Kb, Vb, Krb, coff, rn, flag = pool_on_gpu(cfg, K, V, Kr, synth.doc_tok_offsets(cfg))
+    idx, _, _, _ = route_on_gpu(q["Qr"], Krb, rn, coff, cfg.k)
+    idx = idx.cpu().numpy()
+    Qr = q["Qr"]
+    s = O.cosine_scores(to64(Qr), to64(Krb))
+    rng = np.random.default_rng(9)
+    dsc = rng.standard_normal(idx.shape).astype(np.float32)
+    for b in range(idx.shape[0]):
+        for r, j in enumerate(idx[b]):
+            v = np.sort(s[b, :, coff[j]:coff[j + 1]].ravel())
+            if v.size > 1 and v[-1] - v[-2] < 1e-4:
+                dsc[b, r] = 0.0
+    B, Tq, Hr, dr = Qr.shape
+    t = lambda a: torch.from_numpy(a).to(DEV)
+    base_q = torch.randn((B, Tq, Hr, dr), device=DEV)
+    base_k = torch.randn((Krb.shape[0], Hr, dr), device=DEV)
+    dQr, dKrb = base_q.clone(), base_k.clone()
+    ws = torch.empty(msa.route_backward_workspace_size(B, cfg.k), dtype=torch.uint8, device=DEV)
+    flag = torch.zeros(1, dtype=torch.int32, device=DEV)
+    msa.route_backward(Qr, Krb, rn, t(coff), t(idx), t(dsc), dQr, dKrb, ws, flag)
+    torch.cuda.synchronize()
+    oQ, oK = O.route_backward(to64(Qr), to64(Krb), coff, idx, dsc)
+    assert flag.item() == 0
+    assert len(np.unique(idx)) < idx.size
+    _check((dQr - base_q, dKrb - base_k), (oQ, oK), TOL_BWD_F32, names=("dQr", "dKrbar"))
