@@ -12,18 +12,21 @@
 //     dk_j = scale sum_i ds_ij q_i     dv_j = sum_i p_ij dO_i
 // with the sums over i running over the q-heads of a GQA group and the tokens
 // that see key j.  CUDA-core kernels, fp32 arithmetic, fp32 gradients:
-//   * bwd_rowdot_kernel: D_i, one warp per (token, q-head) row;
+//   * bwd_rowdot_kernel: D_i, 16 bytes of a row per lane (and, when the
+//     tensor-core dK / dV kernel splits key tiles, zeroes its outputs);
 //   * dQ: on the tensor cores for the forward's tensor-core shapes
 //     (attn_bwd_tc.cu), else bwd_dq_kernel: 16 rows of one KV head's group per
 //     CTA, key tiles of 16 through shared memory (the forward's row layout);
-//   * dK / dV: on the tensor cores for those shapes too, else bwd_dkv_kernel:
-//     16 keys of one KV head per CTA, the rows that see them
-//     in blocks of 16 through shared memory; every dK / dV row is written by
-//     exactly one CTA (rows of memory past mem_len get zeros);
+//   * dK / dV: on the tensor cores for bf16, d = 128 and GQA groups of <= 8
+//     heads (attn_bwd_tc.cu), else bwd_dkv_kernel: 16 keys of one KV head per
+//     CTA, the rows that see them in blocks of 16 through shared memory; every
+//     dK / dV row is written by exactly one CTA (rows of memory past mem_len
+//     get zeros);
 //   * gather_bwd_kernel: one CTA per selected document, fp32 atomic adds into
 //     the chunk gradients (documents chosen by several queries accumulate).
 #include <math.h>
 
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -32,24 +35,46 @@
 namespace msa {
 
 cudaError_t launch_attn_dq_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s, bool* handled);
-cudaError_t launch_attn_dkv_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s, bool* handled);
 
 namespace {
 
 constexpr int kRB = 16, kKT = 16, kNT = 128;  // rows, keys per tile (static smem <= 48 KB at d = 128)
 
-template <typename T>
-__global__ void bwd_rowdot_kernel(const T* __restrict__ O, const T* __restrict__ dO, int64_t rows, int d,
-                                  float* __restrict__ Drow, int Tq, int Hq) {
-  // row w = (b, t, h) in O's layout; D is stored [B, Hq, Tq] like the lse
-  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= rows) return;
-  float s = 0.f;
-  for (int i = lane; i < d; i += 32) s += to_f32(O[w * d + i]) * to_f32(dO[w * d + i]);
+// Buffers the row-dot launch zeroes (fp32, counted in float4).
+struct ZeroList {
+  float4* p[4];
+  int64_t n[4];
+};
+
+// D_i = <dO_i, O_i> with LPR lanes per row, 16 bytes each; blocks past
+// row_blocks zero the buffers of z instead.
+template <typename T, int LPR>
+__global__ void bwd_rowdot_kernel(const T* __restrict__ O, const T* __restrict__ dO, int64_t rows,
+                                  float* __restrict__ Drow, int Tq, int Hq, int64_t row_blocks, ZeroList z) {
+  if ((int64_t)blockIdx.x >= row_blocks) {
+    const int64_t i0 = ((int64_t)blockIdx.x - row_blocks) * blockDim.x + threadIdx.x;
+    const int64_t stride = ((int64_t)gridDim.x - row_blocks) * blockDim.x;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) {
+    for (int k = 0; k < 4; ++k)
+      for (int64_t i = i0; i < z.n[k]; i += stride) z.p[k][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  constexpr int VN = Vec<T>::N;
+  constexpr int d = LPR * VN;
+  // row w = (b, t, h) in O's layout; D is stored [B, Hq, Tq] like the lse
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / LPR;
+  const int sub = threadIdx.x % LPR;
+  float s = 0.f;
+  if (w < rows) {
+    float x[VN], y[VN];
+    unpack(__ldg(reinterpret_cast<const uint4*>(O + w * d) + sub), x);
+    unpack(__ldg(reinterpret_cast<const uint4*>(dO + w * d) + sub), y);
+#pragma unroll
+    for (int i = 0; i < VN; ++i) s = fmaf(x[i], y[i], s);
+  }
+#pragma unroll
+  for (int o = LPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (sub == 0 && w < rows) {
     const int64_t h = w % Hq, t = (w / Hq) % Tq, b = w / ((int64_t)Hq * Tq);
     Drow[(b * Hq + h) * Tq + t] = s;
   }
@@ -266,25 +291,36 @@ __global__ void __launch_bounds__(kNT) bwd_dkv_kernel(AttnBwdArgs a) {
 
 template <typename T, int DH>
 cudaError_t bwd_t(const AttnBwdArgs& a, cudaStream_t s) {
+  const msa_dtype dt = std::is_same<T, float>::value ? MSA_F32 : MSA_BF16;
+  const DkvPlan pl = attn_dkv_tc_plan(dt, a);
+  // split dK / dV tiles accumulate with atomics: zero the outputs in the row-dot launch
+  ZeroList z{};
+  int64_t zero_blocks = 0;
+  if (pl.applies && pl.max_chunks > 1) {
+    const int64_t nl = a.B * (int64_t)a.Lloc * a.Hkv * DH / 4, nm = a.B * (int64_t)a.Mmax * a.Hkv * DH / 4;
+    z = ZeroList{{reinterpret_cast<float4*>(a.dKloc), reinterpret_cast<float4*>(a.dVloc),
+                  reinterpret_cast<float4*>(a.dKmem), reinterpret_cast<float4*>(a.dVmem)},
+                 {nl, nl, nm, nm}};
+    zero_blocks = std::min<int64_t>(4 * 148, (2 * (nl + nm) + 255) / 256);
+  }
+  constexpr int LPR = DH / Vec<T>::N;
   const int64_t rows = a.B * a.Tq * a.Hq;
+  const int64_t row_blocks = (rows * LPR + 255) / 256;
   count_launch();
-  bwd_rowdot_kernel<T><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, s>>>(
-      reinterpret_cast<const T*>(a.O), reinterpret_cast<const T*>(a.dO), rows, DH, a.Drow, a.Tq, a.Hq);
+  bwd_rowdot_kernel<T, LPR><<<(unsigned)(row_blocks + zero_blocks), 256, 0, s>>>(
+      reinterpret_cast<const T*>(a.O), reinterpret_cast<const T*>(a.dO), rows, a.Drow, a.Tq, a.Hq, row_blocks, z);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int group = a.Hq / a.Hkv;
   bool handled = false;
-  if ((e = launch_attn_dq_tc(std::is_same<T, float>::value ? MSA_F32 : MSA_BF16, a, s, &handled)) != cudaSuccess)
-    return e;
+  if ((e = launch_attn_dq_tc(dt, a, s, &handled)) != cudaSuccess) return e;
   if (!handled) {
     count_launch();
     bwd_dq_kernel<T, DH><<<dim3((unsigned)((a.Tq * group + kRB - 1) / kRB), (unsigned)a.Hkv, (unsigned)a.B), kNT, 0,
                            s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if ((e = launch_attn_dkv_tc(std::is_same<T, float>::value ? MSA_F32 : MSA_BF16, a, s, &handled)) != cudaSuccess)
-    return e;
-  if (handled) return cudaSuccess;
+  if (pl.applies) return launch_attn_dkv_tc(dt, a, pl, s);
   const int tiles = (a.Mmax + kKT - 1) / kKT + (a.Lloc + kKT - 1) / kKT;
   count_launch();
   bwd_dkv_kernel<T, DH><<<dim3((unsigned)tiles, (unsigned)a.Hkv, (unsigned)a.B), kNT, 0, s>>>(a);

@@ -15,6 +15,9 @@
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warps 2..5 softmax.  Every wait is bounded and ends the CTA with
 // MSA_FLAG_TIMEOUT on expiry.
+#include <algorithm>
+#include <climits>
+
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -291,35 +294,44 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 }
 
 // ---------------------------------------------------------------------------
-// dK and dV.  One CTA per 128-key tile of one (KV head, batch row); for every
-// 128-row query tile that sees the keys:
+// dK and dV.  One CTA per 128-key tile of one (KV head, batch row) and one
+// chunk of the query steps that see the keys (a long range is split so that
+// every SM gets a similar share); per step of 64 query rows (the GQA group's G
+// heads x 64/G tokens):
 //   S^T = K Q^T, dP^T = V dO^T          (keys are the MMA's M, one TMEM lane each)
 //   P^T = exp(scale S^T - lse), dS^T = P^T (dP^T - D)   (softmax warps, one key per
 //        thread, the rows' lse and D staged in shared memory); both rounded to
 //        bf16 and written back over S^T and dP^T
 //   dV += P^T dO,  dK += dS^T Q          (A from TMEM, dO / Q MN-major from TMA)
-// dK * scale and dV are written in fp32 at the end; rows of the tile that are
-// not keys (memory rows past mem_len) get zeros.  Query tiles are double
-// buffered; the MMAs of tile i+1's S^T / dP^T follow tile i's dV / dK in issue
-// order, so they never overwrite P^T / dS^T before those are read.
+// S^T and dP^T have two TMEM buffers each, so the tensor cores compute step
+// n+1 while the softmax warps work on step n; the MMAs of step n+1 are issued
+// after step n-1's dV / dK, which read the same buffer, and the MMAs run in
+// issue order.  Q / dO come through a 4-deep TMA ring.  dK * scale and dV are
+// written in fp32 at the end: stored when the tile's query range is one chunk
+// (rows that are not keys, memory rows past mem_len, get zeros), else added
+// with fp32 atomics onto outputs the row-dot kernel zeroed first.
+constexpr int kQS = 64;       // query rows per step (N of S^T / dP^T, K of dV / dK)
+constexpr int kQStages = 4;   // Q / dO ring
+
 struct DkvParams {
   const int32_t* mem_len;
   int32_t* err_flag;
   const float* lse;
   const float* Drow;
   float *dKm, *dVm, *dKl, *dVl;  // fp32 outputs
-  int Tq, Lloc, Hq, Hkv, Mmax, G, TB, n_qblk, n_mem_tiles;
+  int Tq, Lloc, Hq, Hkv, Mmax, G, TB2, n_qstep, n_mem_tiles, chunk, max_chunks;
   float scale, scale_log2;
 };
 
 template <int DH>
 struct DkvLayout {
   static constexpr int kBoxes = DH / 64;
-  static constexpr int kT = 128 * DH * 2;  // one 128-row bf16 tile
-  static constexpr int kRed = 2 * 2 * 128 * 4;  // [2 buffers][lse, D][128 rows]
-  static constexpr int kBar = 8 * 16;
-  static constexpr int kSmem = 1024 + 2 * kT + 4 * kT + kRed + kBar;  // K, V, Q[2], dO[2]
-  static constexpr uint32_t kTmemCols = 512;  // S^T, dP^T, dK, dV
+  static constexpr int kT = 128 * DH * 2;   // one 128-row bf16 tile (K or V)
+  static constexpr int kQ = kQS * DH * 2;   // one 64-row step of Q or dO
+  static constexpr int kRed = 2 * 2 * kQS * 4;  // [2 buffers][lse, D][64 rows]
+  static constexpr int kBar = 16 * 8;
+  static constexpr int kSmem = 1024 + 2 * kT + 2 * kQStages * kQ + kRed + kBar;  // K, V, Q[4], dO[4]
+  static constexpr uint32_t kTmemCols = 512;  // S^T[2], dP^T[2] (64 each), dK, dV (128 each)
   static_assert(kSmem <= 232448, "shared memory of one CTA");
 };
 
@@ -342,46 +354,54 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                    const __grid_constant__ CUtensorMap tmKm, const __grid_constant__ CUtensorMap tmVm,
                    const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVl, DkvParams p) {
   using L = DkvLayout<DH>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* Ks = smem;
-  uint8_t* Vs = Ks + L::kT;
-  uint8_t* Qs = Vs + L::kT;          // [2]
-  uint8_t* dOs = Qs + 2 * L::kT;     // [2]
-  float* red = reinterpret_cast<float*>(dOs + 2 * L::kT);  // [2][2][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + L::kRed);
-  uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;       // [2]
-  uint64_t* q_empty = bars + 3;      // [2] dV / dK MMAs of the query tile done
-  uint64_t* sp_full = bars + 5;      // S^T, dP^T in TMEM
-  uint64_t* pd_full = bars + 6;      // P^T, dS^T written (128 arrivals)
-  uint64_t* acc_done = bars + 7;
-  uint64_t* drain = bars + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = (int)blockIdx.x / p.max_chunks, ck = (int)blockIdx.x % p.max_chunks;
   const int g = blockIdx.y;
   const int b = blockIdx.z;
   int M = __ldg(p.mem_len + b);
   if (M < 0 || M > p.Mmax) M = M < 0 ? 0 : p.Mmax;  // flagged by the dQ kernel
-  const bool memt = (int)blockIdx.x < p.n_mem_tiles;
-  const int base = memt ? blockIdx.x * 128 : ((int)blockIdx.x - p.n_mem_tiles) * 128;
+  const bool memt = tile < p.n_mem_tiles;
+  const int base = memt ? tile * 128 : (tile - p.n_mem_tiles) * 128;
   const int nk = memt ? min(128, p.Mmax - base) : min(128, p.Lloc - base);   // rows of the tile
   const int nlive = memt ? max(0, min(128, M - base)) : nk;                  // rows that are keys
-  // query tiles that see the keys: all for memory keys; local key l is seen from
+  // query steps that see the keys: all for memory keys; local key l is seen from
   // token l - (Lloc - Tq) on
   const int tfirst = memt ? 0 : max(0, base - (p.Lloc - p.Tq));
-  const int i0 = tfirst / p.TB;
-  const int NQ = nlive > 0 ? p.n_qblk - i0 : 0;
+  const int s0 = tfirst / p.TB2;
+  const int ns_all = nlive > 0 ? p.n_qstep - s0 : 0;
+  const int nchunks = (ns_all + p.chunk - 1) / p.chunk;
+  if (ck >= max(nchunks, 1)) return;  // uniform over the CTA, before any barrier or TMEM
+  const bool split = nchunks > 1;
+  const int sA = s0 + ck * p.chunk;
+  const int NS = ns_all > 0 ? min(p.chunk, ns_all - ck * p.chunk) : 0;
 
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Ks = smem;
+  uint8_t* Vs = Ks + L::kT;
+  uint8_t* Qs = Vs + L::kT;                 // [kQStages]
+  uint8_t* dOs = Qs + kQStages * L::kQ;     // [kQStages]
+  float* red = reinterpret_cast<float*>(dOs + kQStages * L::kQ);  // [2][lse, D][64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + L::kRed);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;               // [kQStages]
+  uint64_t* q_empty = bars + 1 + kQStages;   // [kQStages] dV / dK MMAs of the step done
+  uint64_t* sp_full = bars + 1 + 2 * kQStages;  // [2] S^T, dP^T of the buffer in TMEM
+  uint64_t* pd_full = sp_full + 2;           // [2] P^T, dS^T written (128 arrivals)
+  uint64_t* acc_done = pd_full + 2;
+  uint64_t* drain = acc_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kQStages; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
-    mbar_init(sp_full, 1);
-    mbar_init(pd_full, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sp_full[i], 1);
+      mbar_init(&pd_full[i], 128);
+    }
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -394,12 +414,12 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + 128, tK = tmem + 256, tV = tmem + 384;
+  const uint32_t tS = tmem, tP = tmem + 2 * kQS, tK = tmem + 4 * kQS, tV = tmem + 4 * kQS + 128;
   bool timed_out = false;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0 && NQ > 0) {
+    if (lane == 0 && NS > 0) {
       const int y = memt ? b * p.Mmax + base : b * p.Lloc + base;
       mbar_arrive_expect_tx(kv_full, 2 * L::kT);
 #pragma unroll
@@ -408,81 +428,83 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tma_load_2d(Vs + dc * (128 * 128), memt ? &tmVm : &tmVl, g * DH + dc * 64, y, kv_full);
       }
       int n = 0;
-      for (; n < NQ; ++n) {
-        const int st = n & 1;
-        if (!mbar_wait(&q_empty[st], ((n >> 1) & 1) ^ 1, kWaitPolls)) {
+      for (; n < NS; ++n) {
+        const int st = n % kQStages;
+        if (!mbar_wait(&q_empty[st], ((n / kQStages) & 1) ^ 1, kWaitPolls)) {
           timed_out = true;
           break;
         }
-        const int t0 = (i0 + n) * p.TB;
-        mbar_arrive_expect_tx(&q_full[st], 2 * L::kT);
+        const int t0 = (sA + n) * p.TB2;
+        mbar_arrive_expect_tx(&q_full[st], 2 * L::kQ);
         for (int hh = 0; hh < p.G; ++hh)
 #pragma unroll
           for (int dc = 0; dc < L::kBoxes; ++dc) {
             const int x = (g * p.G + hh) * DH + dc * 64, yq = b * p.Tq + t0;
-            tma_load_2d(Qs + st * L::kT + dc * (128 * 128) + hh * p.TB * 128, &tmQ, x, yq, &q_full[st]);
-            tma_load_2d(dOs + st * L::kT + dc * (128 * 128) + hh * p.TB * 128, &tmdO, x, yq, &q_full[st]);
+            tma_load_2d(Qs + st * L::kQ + dc * (kQS * 128) + hh * p.TB2 * 128, &tmQ, x, yq, &q_full[st]);
+            tma_load_2d(dOs + st * L::kQ + dc * (kQS * 128) + hh * p.TB2 * 128, &tmdO, x, yq, &q_full[st]);
           }
       }
+      // drain: every copy issued must land before the CTA leaves
       if (!mbar_wait(kv_full, 0, kWaitPolls)) timed_out = true;
-      for (int st = 0; st < 2 && st < n; ++st) {
-        const int last = (n - 1 - st) / 2 * 2 + st;
-        if (!mbar_wait(&q_full[st], (last >> 1) & 1, kWaitPolls)) timed_out = true;
+      for (int st = 0; st < kQStages && st < n; ++st) {
+        const int last = (n - 1 - st) / kQStages * kQStages + st;
+        if (!mbar_wait(&q_full[st], (last / kQStages) & 1, kWaitPolls)) timed_out = true;
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && NQ > 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(128, 128);
+    if (lane == 0 && NS > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, kQS);
       constexpr uint32_t idA = idesc_bf16_f32(128, DH, /*b_mn_major=*/true);
       const uint32_t k0 = smem_u32(Ks), v0 = smem_u32(Vs);
-      // dV += P^T dO, dK += dS^T Q for query tile n (A from TMEM: 16 rows of bf16 = 8 columns)
-      auto issue_acc = [&](int n) {
-        const uint32_t q0 = smem_u32(Qs + (n & 1) * L::kT), o0 = smem_u32(dOs + (n & 1) * L::kT);
+      // S^T, dP^T of step n into buffer n & 1
+      auto issue_sp = [&](int n) -> bool {
+        const int st = n % kQStages, buf = n & 1;
+        if (!mbar_wait(&q_full[st], (n / kQStages) & 1, kWaitPolls)) return false;
+        tc_fence_after();
+        const uint32_t q0 = smem_u32(Qs + st * L::kQ), o0 = smem_u32(dOs + st * L::kQ);
 #pragma unroll
-        for (int k = 0; k < 128 / 16; ++k) {
-          mma_bf16_ts(tV, tS + k * 8, desc_mn_sw128(o0 + k * 16 * 128, 128 * 128), idA, (n > 0 || k > 0) ? 1u : 0u);
-          mma_bf16_ts(tK, tP + k * 8, desc_mn_sw128(q0 + k * 16 * 128, 128 * 128), idA, (n > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < DH / 16; ++k) {
+          const int box = k >> 2, kk = k & 3;
+          mma_bf16_ss(tS + buf * kQS, desc_k_sw128(k0 + box * 128 * 128 + kk * 32),
+                      desc_k_sw128(q0 + box * kQS * 128 + kk * 32), idS, k > 0 ? 1u : 0u);
         }
-        mma_commit(&q_empty[n & 1]);
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const int box = k >> 2, kk = k & 3;
+          mma_bf16_ss(tP + buf * kQS, desc_k_sw128(v0 + box * 128 * 128 + kk * 32),
+                      desc_k_sw128(o0 + box * kQS * 128 + kk * 32), idS, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&sp_full[buf]);
+        return true;
       };
-      bool ok = mbar_wait(kv_full, 0, kWaitPolls);
-      for (int n = 0; ok && n < NQ; ++n) {
-        if (!mbar_wait(&q_full[n & 1], (n >> 1) & 1, kWaitPolls)) {
+      // dV += P^T dO, dK += dS^T Q for step n (A from TMEM: 16 query rows of bf16 = 8 columns)
+      auto issue_acc = [&](int n) {
+        const int st = n % kQStages, buf = n & 1;
+        const uint32_t q0 = smem_u32(Qs + st * L::kQ), o0 = smem_u32(dOs + st * L::kQ);
+#pragma unroll
+        for (int k = 0; k < kQS / 16; ++k) {
+          mma_bf16_ts(tV, tS + buf * kQS + k * 8, desc_mn_sw128(o0 + k * 16 * 128, kQS * 128), idA,
+                      (n > 0 || k > 0) ? 1u : 0u);
+          mma_bf16_ts(tK, tP + buf * kQS + k * 8, desc_mn_sw128(q0 + k * 16 * 128, kQS * 128), idA,
+                      (n > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&q_empty[st]);
+      };
+      bool ok = mbar_wait(kv_full, 0, kWaitPolls) && issue_sp(0);
+      for (int n = 0; ok && n < NS; ++n) {
+        if (n + 1 < NS && !issue_sp(n + 1)) {
           ok = false;
           break;
         }
-        if (n > 0) {
-          if (!mbar_wait(pd_full, (n - 1) & 1, kWaitPolls)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_acc(n - 1);
+        if (!mbar_wait(&pd_full[n & 1], (n >> 1) & 1, kWaitPolls)) {
+          ok = false;
+          break;
         }
         tc_fence_after();
-        const uint32_t q0 = smem_u32(Qs + (n & 1) * L::kT), o0 = smem_u32(dOs + (n & 1) * L::kT);
-#pragma unroll
-        for (int k = 0; k < DH / 16; ++k) {
-          const int box = k >> 2, kk = k & 3;
-          mma_bf16_ss(tS, desc_k_sw128(k0 + box * 128 * 128 + kk * 32), desc_k_sw128(q0 + box * 128 * 128 + kk * 32), idS,
-                      k > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < DH / 16; ++k) {
-          const int box = k >> 2, kk = k & 3;
-          mma_bf16_ss(tP, desc_k_sw128(v0 + box * 128 * 128 + kk * 32), desc_k_sw128(o0 + box * 128 * 128 + kk * 32), idS,
-                      k > 0 ? 1u : 0u);
-        }
-        mma_commit(sp_full);
+        issue_acc(n);
       }
-      if (ok && mbar_wait(pd_full, (NQ - 1) & 1, kWaitPolls)) {
-        tc_fence_after();
-        issue_acc(NQ - 1);
-        mma_commit(acc_done);
-      } else {
-        ok = false;
-      }
+      if (ok) mma_commit(acc_done);
       if (!ok) timed_out = true;
       mma_commit(drain);
       if (!mbar_wait(drain, 0, kWaitPolls)) timed_out = true;
@@ -494,79 +516,103 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int tid = threadIdx.x - 64;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const bool key_live = kr < nlive;
-    for (int n = 0; n < NQ; ++n) {
-      // the rows' -lse * log2(e) and D of this query tile, in the buffer of its parity
-      float* rl = red + (n & 1) * 256;
+    const int key = base + kr;
+    const int tmin = memt ? INT_MIN : key - (p.Lloc - p.Tq);  // first token that sees the key
+    // the tile's last key is seen from this token on (every key of the tile visible)
+    const int tall = memt ? 0 : base + 127 - (p.Lloc - p.Tq);
+    for (int n = 0; n < NS; ++n) {
+      const int buf = n & 1;
+      const int t0 = (sA + n) * p.TB2;
+      // the rows' -lse * log2(e) (threads 0..63) and D (64..127) of this step
+      float* rl = red + buf * (2 * kQS);
       {
-        const int hh = tid / p.TB, t = (i0 + n) * p.TB + tid - hh * p.TB;
+        const int r = tid & (kQS - 1);
+        const int hh = r / p.TB2, t = t0 + r - hh * p.TB2;
         const int64_t li = ((int64_t)b * p.Hq + g * p.G + hh) * p.Tq + t;
-        rl[tid] = t < p.Tq ? -__ldg(p.lse + li) * 1.4426950408889634f : 0.f;
-        rl[128 + tid] = t < p.Tq ? __ldg(p.Drow + li) : 0.f;
+        if (tid < kQS)
+          rl[r] = t < p.Tq ? -__ldg(p.lse + li) * 1.4426950408889634f : 0.f;
+        else
+          rl[kQS + r] = t < p.Tq ? __ldg(p.Drow + li) : 0.f;
       }
       // the staging barrier doubles as a vote on the wait, so the warps leave together
-      const bool okw = __all_sync(0xffffffffu, mbar_wait(sp_full, n & 1, kWaitPolls));
+      const bool okw = __all_sync(0xffffffffu, mbar_wait(&sp_full[buf], (n >> 1) & 1, kWaitPolls));
       if (!bar_soft_and(okw)) {
         timed_out = true;
         break;
       }
       tc_fence_after();
-      const int t0 = (i0 + n) * p.TB;
-      const int key = base + kr;  // local row index for local tiles
+      const bool full = nlive == 128 && t0 + p.TB2 <= p.Tq && tall <= t0;
+      const float4* rl4 = reinterpret_cast<const float4*>(rl);
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < kQS; c0 += 32) {
         float s[32], dp[32];
-        tmem_ld16(tS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
-        tmem_ld16(tS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
-        tmem_ld16(tP + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
-        tmem_ld16(tP + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
+        tmem_ld16(tS + buf * kQS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
+        tmem_ld16(tS + buf * kQS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+        tmem_ld16(tP + buf * kQS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
+        tmem_ld16(tP + buf * kQS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
         tmem_ld_wait();
         uint32_t wp[16], wd[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float pr[2], ds[2];
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 l4 = rl4[(c0 >> 2) + i4], d4 = rl4[(kQS >> 2) + (c0 >> 2) + i4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pr[4], ds[4];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int r = c0 + 2 * i + u;
-            const int t = t0 + (r & (p.TB - 1));
-            const bool vis = key_live && t < p.Tq && (memt || key <= p.Lloc - p.Tq + t);
-            pr[u] = vis ? fast_exp2(fmaf(s[2 * i + u], p.scale_log2, rl[r])) : 0.f;
-            ds[u] = pr[u] * (dp[2 * i + u] - rl[128 + r]);
+          for (int u = 0; u < 4; ++u) {
+            const int c = 4 * i4 + u;
+            float e = fast_exp2(fmaf(s[c], p.scale_log2, lv[u]));
+            if (!full) {
+              const int t = t0 + ((c0 + c) & (p.TB2 - 1));
+              e = (key_live && t < p.Tq && t >= tmin) ? e : 0.f;
+            }
+            pr[u] = e;
+            ds[u] = e * (dp[c] - dv[u]);
           }
-          wp[i] = pack_bf16x2(pr[0], pr[1]);
-          wd[i] = pack_bf16x2(ds[0], ds[1]);
+          wp[2 * i4] = pack_bf16x2(pr[0], pr[1]);
+          wp[2 * i4 + 1] = pack_bf16x2(pr[2], pr[3]);
+          wd[2 * i4] = pack_bf16x2(ds[0], ds[1]);
+          wd[2 * i4 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        tmem_st16(tS + lane_off + c0 / 2, wp);
-        tmem_st16(tP + lane_off + c0 / 2, wd);
+        tmem_st16(tS + buf * kQS + lane_off + c0 / 2, wp);
+        tmem_st16(tP + buf * kQS + lane_off + c0 / 2, wd);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(pd_full);
+      mbar_arrive(&pd_full[buf]);
     }
-    // outputs: dK * scale, dV (fp32); rows that are not keys get zeros
-    const bool got = NQ > 0 && !timed_out && __all_sync(0xffffffffu, mbar_wait(acc_done, 0, kWaitPolls));
-    if (NQ > 0 && !got) timed_out = true;
-    if (kr < nk || NQ > 0) {
-      float* dKo = (memt ? p.dKm : p.dKl) + (((int64_t)b * (memt ? p.Mmax : p.Lloc) + base + kr) * p.Hkv + g) * DH;
-      float* dVo = (memt ? p.dVm : p.dVl) + (((int64_t)b * (memt ? p.Mmax : p.Lloc) + base + kr) * p.Hkv + g) * DH;
-      if (got) tc_fence_after();
+    // outputs: dK * scale, dV (fp32)
+    const bool got = NS > 0 && !timed_out && __all_sync(0xffffffffu, mbar_wait(acc_done, 0, kWaitPolls));
+    if (NS > 0 && !got) timed_out = true;
+    // the TMEM loads are warp-collective (got is uniform); only the stores depend on the lane.
+    // A split tile adds onto zeroed outputs, so its non-key rows and a timed-out CTA add nothing.
+    const bool write = kr < nk && (!split || (got && key_live));
+    float* dKo = (memt ? p.dKm : p.dKl) + (((int64_t)b * (memt ? p.Mmax : p.Lloc) + key) * p.Hkv + g) * DH;
+    float* dVo = (memt ? p.dVm : p.dVl) + (((int64_t)b * (memt ? p.Mmax : p.Lloc) + key) * p.Hkv + g) * DH;
+    if (got) tc_fence_after();
+    const float m = key_live ? 1.f : 0.f;
 #pragma unroll
-      for (int c = 0; c < DH; c += 16) {
-        float ok_[16], ov[16];
-        if (got) {
-          tmem_ld16(tK + lane_off + c, ok_);
-          tmem_ld16(tV + lane_off + c, ov);
-          tmem_ld_wait();
-        } else {
+    for (int c = 0; c < DH; c += 16) {
+      float ok_[16], ov[16];
+      if (got) {
+        tmem_ld16(tK + lane_off + c, ok_);
+        tmem_ld16(tV + lane_off + c, ov);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) ok_[i] = ov[i] = 0.f;
-        }
-        if (kr < nk) {
+        for (int i = 0; i < 16; ++i) ok_[i] = ov[i] = 0.f;
+      }
+      if (write) {
 #pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float m = key_live ? 1.f : 0.f;
-            *reinterpret_cast<float4*>(dKo + c + i) =
-                make_float4(ok_[i] * p.scale * m, ok_[i + 1] * p.scale * m, ok_[i + 2] * p.scale * m, ok_[i + 3] * p.scale * m);
-            *reinterpret_cast<float4*>(dVo + c + i) = make_float4(ov[i] * m, ov[i + 1] * m, ov[i + 2] * m, ov[i + 3] * m);
+        for (int i = 0; i < 16; i += 4) {
+          const float4 vk = make_float4(ok_[i] * p.scale * m, ok_[i + 1] * p.scale * m, ok_[i + 2] * p.scale * m,
+                                        ok_[i + 3] * p.scale * m);
+          const float4 vv = make_float4(ov[i] * m, ov[i + 1] * m, ov[i + 2] * m, ov[i + 3] * m);
+          if (split) {
+            atomicAdd(reinterpret_cast<float4*>(dKo + c + i), vk);
+            atomicAdd(reinterpret_cast<float4*>(dVo + c + i), vv);
+          } else {
+            *reinterpret_cast<float4*>(dKo + c + i) = vk;
+            *reinterpret_cast<float4*>(dVo + c + i) = vv;
           }
         }
       }
@@ -584,20 +630,42 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
 }  // namespace
 
-// dK / dV on the tensor cores (same shapes as the dQ kernel).
-cudaError_t launch_attn_dkv_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s, bool* handled) {
-  *handled = false;
-  if (dt != MSA_BF16 || a.d != 128) return cudaSuccess;
+// Work split of the tensor-core dK / dV kernel: 64-row query steps per CTA
+// ("chunk") and the most chunks any key tile has.  Shapes: bf16, d = 128, a
+// GQA group of G <= 8 heads dividing 64 rows into blocks of >= 8 tokens.
+DkvPlan attn_dkv_tc_plan(msa_dtype dt, const AttnBwdArgs& a) {
+  DkvPlan pl{false, 0, 0};
+  if (dt != MSA_BF16 || a.d != 128 || a.Hkv < 1) return pl;
   const int G = a.Hq / a.Hkv;
-  if (G < 1 || 128 % G != 0 || 128 / G < 8 || a.B > 65535 || a.Hkv > 65535) return cudaSuccess;
+  if (G < 1 || kQS % G != 0 || kQS / G < 8 || a.B > 65535 || a.Hkv > 65535) return pl;
+  const int TB2 = kQS / G;
+  const int n_qstep = (a.Tq + TB2 - 1) / TB2;
+  // 64-row steps of all key tiles of one (head, batch row): memory tiles see every
+  // step; local tile i from the token that sees its first key on
+  int64_t steps = (int64_t)((a.Mmax + 127) / 128) * n_qstep;
+  for (int base = 0; base < a.Lloc; base += 128) steps += n_qstep - std::max(0, base - (a.Lloc - a.Tq)) / TB2;
+  steps *= (int64_t)a.Hkv * a.B;
+  // about six CTAs' worth per SM, no chunk under 8 steps
+  const int64_t target = (steps + 6 * 148 - 1) / (6 * 148);
+  pl.chunk = (int)std::min<int64_t>(n_qstep, std::max<int64_t>(8, target));
+  pl.max_chunks = (n_qstep + pl.chunk - 1) / pl.chunk;
+  const int tiles = (a.Mmax + 127) / 128 + (a.Lloc + 127) / 128;
+  if ((int64_t)tiles * pl.max_chunks > 0x7fffffff) return pl;
+  pl.applies = true;
+  return pl;
+}
+
+cudaError_t launch_attn_dkv_tc(msa_dtype dt, const AttnBwdArgs& a, const DkvPlan& pl, cudaStream_t s) {
+  if (!pl.applies) return cudaErrorInvalidValue;
   constexpr int DH = 128;
   using L = DkvLayout<DH>;
-  const int TB = 128 / G;
+  const int G = a.Hq / a.Hkv;
+  const int TB2 = kQS / G;
   CUtensorMap tq, tdo, tkm, tvm, tkl, tvl;
   const uint64_t rowkv = (uint64_t)a.Hkv * DH * 2;
   const int64_t mrows = a.B * (int64_t)(a.Mmax > 0 ? a.Mmax : 1);
-  if (!make_tmap_2d_bf16(&tq, a.Q, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB) ||
-      !make_tmap_2d_bf16(&tdo, a.dO, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB) ||
+  if (!make_tmap_2d_bf16(&tq, a.Q, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB2) ||
+      !make_tmap_2d_bf16(&tdo, a.dO, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB2) ||
       !make_tmap_2d_bf16(&tkm, a.Mmax > 0 ? a.Kmem : a.Kloc, (uint64_t)a.Hkv * DH,
                          (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, 128) ||
       !make_tmap_2d_bf16(&tvm, a.Mmax > 0 ? a.Vmem : a.Vloc, (uint64_t)a.Hkv * DH,
@@ -620,18 +688,19 @@ cudaError_t launch_attn_dkv_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t 
   p.Hkv = a.Hkv;
   p.Mmax = a.Mmax;
   p.G = G;
-  p.TB = TB;
-  p.n_qblk = (a.Tq + TB - 1) / TB;
+  p.TB2 = TB2;
+  p.n_qstep = (a.Tq + TB2 - 1) / TB2;
   p.n_mem_tiles = (a.Mmax + 127) / 128;
+  p.chunk = pl.chunk;
+  p.max_chunks = pl.max_chunks;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   cudaError_t e = cudaFuncSetAttribute(attn_dkv_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
   const int tiles = p.n_mem_tiles + (a.Lloc + 127) / 128;
-  *handled = true;
   count_launch();
-  attn_dkv_tc_kernel<DH><<<dim3((unsigned)tiles, (unsigned)a.Hkv, (unsigned)a.B), kThreads, L::kSmem, s>>>(
-      tq, tdo, tkm, tvm, tkl, tvl, p);
+  attn_dkv_tc_kernel<DH><<<dim3((unsigned)(tiles * pl.max_chunks), (unsigned)a.Hkv, (unsigned)a.B), kThreads,
+                           L::kSmem, s>>>(tq, tdo, tkm, tvm, tkl, tvl, p);
   return cudaGetLastError();
 }
 

@@ -80,6 +80,15 @@ struct AttnBwdArgs {
   int32_t* err_flag;
 };
 size_t attn_bwd_workspace_size(int64_t B, int Tq, int Hq);
+// Work split of the tensor-core dK / dV kernel (attn_bwd_tc.cu).  When a key
+// tile's query steps span several chunks (max_chunks > 1) the kernel adds its
+// partial dK / dV with atomics, so the outputs must be zeroed before it runs.
+struct DkvPlan {
+  bool applies;
+  int chunk, max_chunks;
+};
+DkvPlan attn_dkv_tc_plan(msa_dtype dt, const AttnBwdArgs& a);
+cudaError_t launch_attn_dkv_tc(msa_dtype dt, const AttnBwdArgs& a, const DkvPlan& pl, cudaStream_t s);
 cudaError_t launch_attn_bwd(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s);
 
 // Adjoint of the gather: dKbar / dVbar [C, Hkv, d] fp32 += the gathered rows' gradients.

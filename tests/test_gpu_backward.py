@@ -61,6 +61,8 @@ def _check(gpu, ora, tol, names=("dQ", "dKloc", "dVloc", "dKmem", "dVmem")):
     (3, 40, 70, 32, 8, 128, 48, [48, 0, 17], torch.bfloat16, TOL_BWD_BF16),      # Qwen heads, ragged memory
     (1, 100, 130, 64, 8, 128, 40, [33], torch.bfloat16, TOL_BWD_BF16),           # G = 8, many tiles, odd sizes
     (2, 33, 33, 8, 8, 64, 16, [16, 5], torch.float32, TOL_BWD_F32),              # MHA, Tq = Lloc
+    (2, 300, 420, 32, 8, 128, 200, [200, 77], torch.bfloat16, TOL_BWD_BF16),     # key tiles split over query chunks
+    (1, 160, 160, 16, 16, 128, 0, [0], torch.bfloat16, TOL_BWD_BF16),            # MHA on the tensor cores, no memory
 ])
 def test_attention_backward_matches_oracle(B, Tq, Lloc, Hq, Hkv, d, Mmax, mem_lens, dtype, tol):
     Q, Kl, Vl, Km, Vm, ml, dO = _inputs(B, Tq, Lloc, Hq, Hkv, d, Mmax, mem_lens, dtype, seed=B * 100 + Tq)
