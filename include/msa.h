@@ -200,7 +200,7 @@ msa_status msa_route_topk_noalloc(msa_dtype dt, const void* Qr, int64_t B, int T
  * Step 4: context assembly ("Inference Pipeline" stage 2: load only the
  * selected K̄ / V̄).  For query b, the chunks of documents topk_idx[b, 0..k-1]
  * are copied in rank order (each document's chunks in ascending order) into
- * rows [0, mem_len[b]) of Kmem / Vmem; rows past mem_len[b] are left untouched.
+ * rows [0, mem_len[b]) of Kmem / Vmem; rows [mem_len[b], Mmax) are set to zero.
  *   topk_idx int32 [B, k];  doc_chunk_off int64 [D+1]
  *   Kbar, Vbar [C, Hkv, d] dtype dt;  Kmem, Vmem [B, Mmax, Hkv, d];  mem_len int32 [B]
  * Host tier ("Inference Pipeline": the pooled K̄ / V̄ may stay in host memory
@@ -230,7 +230,10 @@ msa_status msa_gather(msa_dtype dt, const int32_t* topk_idx, int64_t B, int k,
  *   Q [B, Tq, Hq, d];  Kloc, Vloc [B, Lloc, Hkv, d];  Kmem, Vmem [B, Mmax, Hkv, d]
  *   mem_len int32 [B] (each in [0, Mmax]);  O [B, Tq, Hq, d];  lse fp32 [B, Hq, Tq] or NULL
  *   scale <= 0 means 1/sqrt(d).
- * Requires Lloc >= Tq >= 1, Hq % Hkv == 0, d in {64, 128}.
+ * Requires Lloc >= Tq >= 1, Hq % Hkv == 0, d in {64, 128}.  Memory rows
+ * [mem_len[b], Mmax) are masked out but must hold finite values: the
+ * tensor-core kernels multiply them by zero weights and 0 x NaN is NaN
+ * (msa_gather leaves zeros there).
  * Device flags: MSA_FLAG_INDEX_OOB when a mem_len is outside [0, Mmax] (that
  * batch row is computed with mem_len clamped into range).
  * ---------------------------------------------------------------------- */

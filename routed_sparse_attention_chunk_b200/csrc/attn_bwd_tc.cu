@@ -256,7 +256,7 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           const int c = c0 + 2 * i;
           const float p0 = c < lim ? fast_exp2(fmaf(s[2 * i], p.scale_log2, nl)) : 0.f;
           const float p1 = c + 1 < lim ? fast_exp2(fmaf(s[2 * i + 1], p.scale_log2, nl)) : 0.f;
-          w[i] = pack_bf16x2(p0 * (dp[2 * i] - Dr), p1 * (dp[2 * i + 1] - Dr));
+          w[i] = pack_bf16x2(c < lim ? p0 * (dp[2 * i] - Dr) : 0.f, c + 1 < lim ? p1 * (dp[2 * i + 1] - Dr) : 0.f);
         }
         tmem_st16(tS + lane_off + c0 / 2, w);
       }
@@ -312,6 +312,7 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 // with fp32 atomics onto outputs the row-dot kernel zeroed first.
 constexpr int kQS = 64;       // query rows per step (N of S^T / dP^T, K of dV / dK)
 constexpr int kQStages = 4;   // Q / dO ring
+constexpr int kDkvThreads = 320;  // producer, MMA issuer, two softmax warpgroups
 
 struct DkvParams {
   const int32_t* mem_len;
@@ -335,12 +336,12 @@ struct DkvLayout {
   static_assert(kSmem <= 232448, "shared memory of one CTA");
 };
 
-// Barrier of the 128 softmax threads that also ANDs a predicate over them, so
+// Barrier of the 256 softmax threads that also ANDs a predicate over them, so
 // that a failed wait ends the loop for every softmax warp at once.
 __device__ __forceinline__ bool bar_soft_and(bool pred) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred pi, po;\n setp.ne.b32 pi, %1, 0;\n bar.red.and.pred po, 1, 128, pi;\n"
+      "{\n .reg .pred pi, po;\n setp.ne.b32 pi, %1, 0;\n bar.red.and.pred po, 1, 256, pi;\n"
       " selp.u32 %0, 1, 0, po;\n}"
       : "=r"(r)
       : "r"((uint32_t)pred)
@@ -349,7 +350,7 @@ __device__ __forceinline__ bool bar_soft_and(bool pred) {
 }
 
 template <int DH>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kDkvThreads, 1)
 attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                    const __grid_constant__ CUtensorMap tmKm, const __grid_constant__ CUtensorMap tmVm,
                    const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVl, DkvParams p) {
@@ -386,7 +387,7 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   uint64_t* q_full = bars + 1;               // [kQStages]
   uint64_t* q_empty = bars + 1 + kQStages;   // [kQStages] dV / dK MMAs of the step done
   uint64_t* sp_full = bars + 1 + 2 * kQStages;  // [2] S^T, dP^T of the buffer in TMEM
-  uint64_t* pd_full = sp_full + 2;           // [2] P^T, dS^T written (128 arrivals)
+  uint64_t* pd_full = sp_full + 2;           // [2] P^T, dS^T written (256 arrivals)
   uint64_t* acc_done = pd_full + 2;
   uint64_t* drain = acc_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -400,7 +401,7 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sp_full[i], 1);
-      mbar_init(&pd_full[i], 128);
+      mbar_init(&pd_full[i], 256);
     }
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
@@ -511,7 +512,10 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
   } else {
     // ---------------------------------------------------------------- softmax (one key per thread)
+    // Two warpgroups: warp w reaches TMEM lanes 32 (w % 4) ..; warpgroup `half`
+    // takes query columns [32 half, 32 half + 32) of every step.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int kr = q * 32 + lane;  // this thread's key row of the tile (TMEM lane)
     const int tid = threadIdx.x - 64;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
@@ -520,20 +524,24 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int tmin = memt ? INT_MIN : key - (p.Lloc - p.Tq);  // first token that sees the key
     // the tile's last key is seen from this token on (every key of the tile visible)
     const int tall = memt ? 0 : base + 127 - (p.Lloc - p.Tq);
+    // threads 0..63 stage -lse * log2(e) of the step's rows, 64..127 their D; the
+    // value of step n+1 is loaded while step n is processed
+    const int sr = tid & (kQS - 1);
+    const int shh = sr / p.TB2;
+    const int64_t srow = ((int64_t)b * p.Hq + g * p.G + shh) * p.Tq;
+    auto stage_load = [&](int n) -> float {
+      const int t = (sA + n) * p.TB2 + sr - shh * p.TB2;
+      if (tid >= 2 * kQS || t >= p.Tq) return 0.f;
+      return tid < kQS ? -__ldg(p.lse + srow + t) * 1.4426950408889634f : __ldg(p.Drow + srow + t);
+    };
+    float staged = NS > 0 ? stage_load(0) : 0.f;
+    const int c0 = half * 32;
     for (int n = 0; n < NS; ++n) {
       const int buf = n & 1;
       const int t0 = (sA + n) * p.TB2;
-      // the rows' -lse * log2(e) (threads 0..63) and D (64..127) of this step
       float* rl = red + buf * (2 * kQS);
-      {
-        const int r = tid & (kQS - 1);
-        const int hh = r / p.TB2, t = t0 + r - hh * p.TB2;
-        const int64_t li = ((int64_t)b * p.Hq + g * p.G + hh) * p.Tq + t;
-        if (tid < kQS)
-          rl[r] = t < p.Tq ? -__ldg(p.lse + li) * 1.4426950408889634f : 0.f;
-        else
-          rl[kQS + r] = t < p.Tq ? __ldg(p.Drow + li) : 0.f;
-      }
+      if (tid < 2 * kQS) rl[tid] = staged;  // [lse(64), D(64)]
+      if (n + 1 < NS) staged = stage_load(n + 1);
       // the staging barrier doubles as a vote on the wait, so the warps leave together
       const bool okw = __all_sync(0xffffffffu, mbar_wait(&sp_full[buf], (n >> 1) & 1, kWaitPolls));
       if (!bar_soft_and(okw)) {
@@ -543,77 +551,76 @@ attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_after();
       const bool full = nlive == 128 && t0 + p.TB2 <= p.Tq && tall <= t0;
       const float4* rl4 = reinterpret_cast<const float4*>(rl);
+      float s[32], dp[32];
+      tmem_ld16(tS + buf * kQS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
+      tmem_ld16(tS + buf * kQS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+      tmem_ld16(tP + buf * kQS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
+      tmem_ld16(tP + buf * kQS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
+      tmem_ld_wait();
+      if (!full) {  // masked step: the diagonal, a ragged end, memory rows past mem_len
 #pragma unroll
-      for (int c0 = 0; c0 < kQS; c0 += 32) {
-        float s[32], dp[32];
-        tmem_ld16(tS + buf * kQS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
-        tmem_ld16(tS + buf * kQS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
-        tmem_ld16(tP + buf * kQS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
-        tmem_ld16(tP + buf * kQS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
-        tmem_ld_wait();
-        uint32_t wp[16], wd[16];
-#pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 l4 = rl4[(c0 >> 2) + i4], d4 = rl4[(kQS >> 2) + (c0 >> 2) + i4];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pr[4], ds[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = 4 * i4 + u;
-            float e = fast_exp2(fmaf(s[c], p.scale_log2, lv[u]));
-            if (!full) {
-              const int t = t0 + ((c0 + c) & (p.TB2 - 1));
-              e = (key_live && t < p.Tq && t >= tmin) ? e : 0.f;
-            }
-            pr[u] = e;
-            ds[u] = e * (dp[c] - dv[u]);
+        for (int c = 0; c < 32; ++c) {
+          const int t = t0 + ((c0 + c) & (p.TB2 - 1));
+          if (!(key_live && t < p.Tq && t >= tmin)) {
+            s[c] = -INFINITY;  // p = 0
+            dp[c] = 0.f;       // and dS = 0 even where the masked row's dP is not finite
           }
-          wp[2 * i4] = pack_bf16x2(pr[0], pr[1]);
-          wp[2 * i4 + 1] = pack_bf16x2(pr[2], pr[3]);
-          wd[2 * i4] = pack_bf16x2(ds[0], ds[1]);
-          wd[2 * i4 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        tmem_st16(tS + buf * kQS + lane_off + c0 / 2, wp);
-        tmem_st16(tP + buf * kQS + lane_off + c0 / 2, wd);
       }
+      uint32_t wp[16], wd[16];
+#pragma unroll
+      for (int i4 = 0; i4 < 8; ++i4) {
+        const float4 l4 = rl4[(c0 >> 2) + i4], d4 = rl4[(kQS >> 2) + (c0 >> 2) + i4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float pr[4], ds[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = 4 * i4 + u;
+          pr[u] = fast_exp2(fmaf(s[c], p.scale_log2, lv[u]));
+          ds[u] = pr[u] * (dp[c] - dv[u]);
+        }
+        wp[2 * i4] = pack_bf16x2(pr[0], pr[1]);
+        wp[2 * i4 + 1] = pack_bf16x2(pr[2], pr[3]);
+        wd[2 * i4] = pack_bf16x2(ds[0], ds[1]);
+        wd[2 * i4 + 1] = pack_bf16x2(ds[2], ds[3]);
+      }
+      tmem_st16(tS + buf * kQS + lane_off + c0 / 2, wp);
+      tmem_st16(tP + buf * kQS + lane_off + c0 / 2, wd);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&pd_full[buf]);
     }
-    // outputs: dK * scale, dV (fp32)
+    // outputs: dK * scale (warpgroup 0), dV (warpgroup 1), fp32
     const bool got = NS > 0 && !timed_out && __all_sync(0xffffffffu, mbar_wait(acc_done, 0, kWaitPolls));
     if (NS > 0 && !got) timed_out = true;
     // the TMEM loads are warp-collective (got is uniform); only the stores depend on the lane.
     // A split tile adds onto zeroed outputs, so its non-key rows and a timed-out CTA add nothing.
     const bool write = kr < nk && (!split || (got && key_live));
-    float* dKo = (memt ? p.dKm : p.dKl) + (((int64_t)b * (memt ? p.Mmax : p.Lloc) + key) * p.Hkv + g) * DH;
-    float* dVo = (memt ? p.dVm : p.dVl) + (((int64_t)b * (memt ? p.Mmax : p.Lloc) + key) * p.Hkv + g) * DH;
+    float* out = (half == 0 ? (memt ? p.dKm : p.dKl) : (memt ? p.dVm : p.dVl)) +
+                 (((int64_t)b * (memt ? p.Mmax : p.Lloc) + key) * p.Hkv + g) * DH;
+    const uint32_t tacc = half == 0 ? tK : tV;
     if (got) tc_fence_after();
-    const float m = key_live ? 1.f : 0.f;
+    const float m = half == 0 ? p.scale : 1.f;
 #pragma unroll
-    for (int c = 0; c < DH; c += 16) {
-      float ok_[16], ov[16];
+    for (int c = 0; c < DH; c += 32) {
+      float o[32];
       if (got) {
-        tmem_ld16(tK + lane_off + c, ok_);
-        tmem_ld16(tV + lane_off + c, ov);
+        tmem_ld16(tacc + lane_off + c, *reinterpret_cast<float(*)[16]>(&o[0]));
+        tmem_ld16(tacc + lane_off + c + 16, *reinterpret_cast<float(*)[16]>(&o[16]));
         tmem_ld_wait();
       } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) ok_[i] = ov[i] = 0.f;
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
       }
       if (write) {
 #pragma unroll
-        for (int i = 0; i < 16; i += 4) {
-          const float4 vk = make_float4(ok_[i] * p.scale * m, ok_[i + 1] * p.scale * m, ok_[i + 2] * p.scale * m,
-                                        ok_[i + 3] * p.scale * m);
-          const float4 vv = make_float4(ov[i] * m, ov[i + 1] * m, ov[i + 2] * m, ov[i + 3] * m);
-          if (split) {
-            atomicAdd(reinterpret_cast<float4*>(dKo + c + i), vk);
-            atomicAdd(reinterpret_cast<float4*>(dVo + c + i), vv);
-          } else {
-            *reinterpret_cast<float4*>(dKo + c + i) = vk;
-            *reinterpret_cast<float4*>(dVo + c + i) = vv;
-          }
+        for (int i = 0; i < 32; i += 4) {
+          const float4 v = key_live ? make_float4(o[i] * m, o[i + 1] * m, o[i + 2] * m, o[i + 3] * m)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+          if (split)
+            atomicAdd(reinterpret_cast<float4*>(out + c + i), v);
+          else
+            *reinterpret_cast<float4*>(out + c + i) = v;
         }
       }
     }
@@ -699,7 +706,7 @@ cudaError_t launch_attn_dkv_tc(msa_dtype dt, const AttnBwdArgs& a, const DkvPlan
   if (e != cudaSuccess) return e;
   const int tiles = p.n_mem_tiles + (a.Lloc + 127) / 128;
   count_launch();
-  attn_dkv_tc_kernel<DH><<<dim3((unsigned)(tiles * pl.max_chunks), (unsigned)a.Hkv, (unsigned)a.B), kThreads,
+  attn_dkv_tc_kernel<DH><<<dim3((unsigned)(tiles * pl.max_chunks), (unsigned)a.Hkv, (unsigned)a.B), kDkvThreads,
                            L::kSmem, s>>>(tq, tdo, tkm, tvm, tkl, tvl, p);
   return cudaGetLastError();
 }

@@ -50,6 +50,18 @@ __global__ void gather_kernel(GatherArgs a, int row_vecs) {
       a.mem_len[b] = (int32_t)(total < a.Mmax ? total : a.Mmax);
     }
   }
+  if (r == a.k - 1) {
+    // rows past the selection are zeroed: the attention kernels mask them, but a
+    // masked weight of 0 times a non-finite value would still be NaN
+    const int64_t total = min(start + me.n, (int64_t)a.Mmax);
+    uint4* Kz = reinterpret_cast<uint4*>(a.Kmem) + (b * a.Mmax + total) * row_vecs;
+    uint4* Vz = reinterpret_cast<uint4*>(a.Vmem) + (b * a.Mmax + total) * row_vecs;
+    const int64_t nz = ((int64_t)a.Mmax - total) * row_vecs;
+    for (int64_t i = threadIdx.x; i < nz; i += blockDim.x) {
+      Kz[i] = make_uint4(0u, 0u, 0u, 0u);
+      Vz[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   const int64_t n = min(me.n, max((int64_t)0, (int64_t)a.Mmax - start));
   if (n <= 0) return;
   const uint4* Ks = reinterpret_cast<const uint4*>(a.Kbar) + me.cs * row_vecs;

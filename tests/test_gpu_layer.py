@@ -97,3 +97,35 @@ def test_fused_layer_equals_unfused_calls():
     torch.cuda.synchronize()
     assert torch.equal(idx1, idx2) and torch.equal(sc1, sc2) and torch.equal(ds1, ds2)
     assert torch.equal(O1, O2) and torch.equal(lse1, lse2)
+
+
+@pytest.mark.parametrize("name,scale", [("1m", dict(D=96, Tq=40, Lloc=70)),
+                                        ("decode16m", dict(D=200, B=5, Lloc=256, docs_per_slab=0))])
+def test_layer_ignores_stale_workspace_bytes(name, scale):
+    """The gathered rows live in the caller's workspace; rows past a query's selection are masked,
+    and the gather zeroes them, so a workspace full of NaN bit patterns (0xFF bytes) gives the same
+    output as a zeroed one.  Mmax is larger than any selection, so every query has such rows."""
+    cfg = synth.get_config(name).scaled(**scale)
+    q = synth.gen_query(cfg, 0, DEV)
+    K, V, Kr = synth.gen_raw_slab(cfg, 0, cfg.D, DEV, Qr0=q["Qr"][0])
+    Kb, Vb, Krb, coff, rn, _ = pool_on_gpu(cfg, K, V, Kr, synth.doc_tok_offsets(cfg))
+    D, Mmax = len(coff) - 1, cfg.Mmax + 200
+
+    def run(fill):
+        ws = torch.full((msa.layer_forward_workspace_size(cfg.B, cfg.Tq, cfg.Lloc, cfg.Hq, cfg.Hkv, cfg.d, cfg.Hr, D,
+                                                          Krb.shape[0], cfg.k, Mmax),), fill, dtype=torch.uint8,
+                        device=DEV)
+        O_ = torch.empty_like(q["Q"])
+        lse = torch.empty((cfg.B, cfg.Hq, cfg.Tq), dtype=torch.float32, device=DEV)
+        idx = torch.empty((cfg.B, cfg.k), dtype=torch.int32, device=DEV)
+        flag = torch.zeros(1, dtype=torch.int32, device=DEV)
+        msa.layer_forward(q["Qr"], Krb, rn, torch.from_numpy(coff).to(DEV), cfg.k, q["Q"], q["Kloc"], q["Vloc"],
+                          Kb, Vb, Mmax, O_, idx, ws, lse, None, None, 0.0, flag)
+        torch.cuda.synchronize()
+        return O_, lse, idx, flag
+
+    O0, lse0, idx0, f0 = run(0)
+    O1, lse1, idx1, f1 = run(255)
+    assert f0.item() == 0 and f1.item() == 0
+    assert torch.isfinite(O1.float()).all()
+    assert torch.equal(idx0, idx1) and torch.equal(O0, O1) and torch.equal(lse0, lse1)

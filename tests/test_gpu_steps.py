@@ -251,6 +251,40 @@ def test_gather_bitexact_and_flags():
     assert ml.max().item() <= 3
 
 
+def test_gather_zeroes_rows_past_the_selection():
+    """Rows [mem_len, Mmax) of the output are set to zero (they start as NaN here), so the
+    attention kernels, which multiply masked rows by zero weights, stay finite."""
+    rng = np.random.default_rng(8)
+    D = 40
+    n = rng.integers(1, 5, size=D)
+    coff = _ragged_offsets(n)
+    C = int(coff[-1])
+    Kb = synth.gen_bank_bf16(C, 8, 128, DEV, 2, "K")
+    Vb = synth.gen_bank_bf16(C, 8, 128, DEV, 2, "V")
+    B, k, Mmax = 3, 5, 150
+    sel = np.stack([rng.choice(D, k, replace=False) for _ in range(B)]).astype(np.int32)
+    Km = torch.full((B, Mmax, 8, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
+    Vm = torch.full_like(Km, float("nan"))
+    ml = torch.zeros(B, dtype=torch.int32, device=DEV)
+    msa.gather(torch.from_numpy(sel).to(DEV), torch.from_numpy(coff).to(DEV), Kb, Vb, Km, Vm, ml)
+    torch.cuda.synchronize()
+    for b in range(B):
+        m = int(ml[b])
+        assert 0 < m < Mmax
+        assert not Km[b, m:].float().abs().sum() and not Vm[b, m:].float().abs().sum()
+    oKm, oVm, oml = O.gather(sel, coff, to64(Kb), to64(Vb), Mmax)
+    for Tq, Lloc in ((1, 300), (100, 150)):      # decode and prefill kernels
+        g = torch.Generator(device=DEV).manual_seed(Tq)
+        Q = (0.5 * torch.randn((B, Tq, 32, 128), generator=g, device=DEV)).bfloat16()
+        Kl = (0.5 * torch.randn((B, Lloc, 8, 128), generator=g, device=DEV)).bfloat16()
+        Vl = (0.5 * torch.randn((B, Lloc, 8, 128), generator=g, device=DEV)).bfloat16()
+        Og, lse, flag = attn_on_gpu(Q, Kl, Vl, Km, Vm, ml)
+        Oo, _ = O.attention(to64(Q), to64(Kl), to64(Vl), oKm, oVm, oml)
+        torch.cuda.synchronize()
+        assert flag.item() == 0
+        close_abs(to64(Og), Oo, TOL_BF16_ABS, f"O (Tq={Tq})")
+
+
 # ---------------------------------------------------------------- step 5: attention
 def _attn_inputs(B, Tq, Lloc, Hq, Hkv, d, Mmax, mem_lens, dtype, seed):
     g = torch.Generator(device=DEV).manual_seed(seed)
