@@ -1,20 +1,22 @@
-// Backward of step 5 on the 5th-generation tensor cores: dQ of the sparse
-// attention over [selected memory rows ++ causal local rows] (the exact
+// Backward of step 5 on the 5th-generation tensor cores: dQ, dK and dV of the
+// sparse attention over [selected memory rows ++ causal local rows] (the exact
 // derivative of the forward; "MSA: Memory Sparse Attention" README,
 // "Architecture": the layer is trained end to end through its sparse
-// attention).  For a 128-row query tile (the GQA group's G q-heads x 128/G
-// tokens, as in the forward) and every key tile j of 128 keys:
+// attention).  dQ: for a 128-row query tile (the GQA group's G q-heads x 128/G
+// tokens, as in the forward) and every step j of 64 keys:
 //   S = Q K_j^T and dP = dO V_j^T        (tcgen05.mma into TMEM, fp32)
 //   P = exp(scale S - lse),  dS = P (dP - D)   (softmax warps, one row per
-//        thread, 32 columns at a time: the forward's log-sum-exp makes a row
-//        max unnecessary); dS is rounded to bf16 and written back over S
+//        thread: the forward's log-sum-exp makes a row max unnecessary); dS
+//        is rounded to bf16 and written back over S
 //   dQ += dS K_j                          (dS as the MMA's A operand from TMEM,
 //                                          K_j MN-major from its TMA tile)
-// and dQ * scale is written in fp32 at the end.  The MMAs run in issue order,
-// so S_{j+1} (issued after dQ_j) never overwrites dS_j before it is read.
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2..5 softmax.  Every wait is bounded and ends the CTA with
-// MSA_FLAG_TIMEOUT on expiry.
+// and dQ * scale is written in fp32 at the end.  S and dP have two TMEM
+// buffers, so the tensor cores compute step j+1 while the softmax warps work
+// on step j; the MMAs run in issue order, so S_{j+1} (issued after dQ_{j-1},
+// which reads the same buffer) never overwrites dS_{j-1} before it is read.
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..9 softmax in two warpgroups of 32 key columns each.  Every
+// wait is bounded and ends the CTA with MSA_FLAG_TIMEOUT on expiry.
 #include <algorithm>
 #include <climits>
 
@@ -29,8 +31,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kRows = 128;   // MMA M: query rows per tile
-constexpr int kKeys = 128;   // keys per tile
-constexpr int kThreads = 192;
+constexpr int kKS = 64;      // keys per dQ step (N of S / dP, K of dQ)
+constexpr int kKVStages = 4; // K / V ring of the dQ kernel
+constexpr int kDqThreads = 320;
 constexpr uint32_t kWaitPolls = 1u << 24;
 
 struct DqParams {
@@ -47,10 +50,10 @@ template <int DH>
 struct DqLayout {
   static constexpr int kBoxes = DH / 64;
   static constexpr int kQ = kRows * DH * 2;
-  static constexpr int kK = kKeys * DH * 2;
-  static constexpr int kBar = 8 * 16;
-  static constexpr int kSmem = 1024 + 2 * kQ + 4 * kK + kBar;  // Q, dO, K[2], V[2]
-  static constexpr uint32_t kTmemCols = 512;                   // S, dP, dQ (128 each)
+  static constexpr int kK = kKS * DH * 2;   // one 64-key step of K or V
+  static constexpr int kBar = 16 * 8;
+  static constexpr int kSmem = 1024 + 2 * kQ + 2 * kKVStages * kK + kBar;  // Q, dO, K[4], V[4]
+  static constexpr uint32_t kTmemCols = 512;  // S[2], dP[2] (64 each), dQ (128)
   static_assert(kSmem <= 232448, "shared memory of one CTA");
 };
 
@@ -60,8 +63,21 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Barrier of the 256 softmax threads that also ANDs a predicate over them, so
+// that a failed wait ends the loop for every softmax warp at once.
+__device__ __forceinline__ bool bar_soft_and(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.b32 pi, %1, 0;\n bar.red.and.pred po, 1, 256, pi;\n"
+      " selp.u32 %0, 1, 0, po;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
 template <int DH>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
 attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmKm, const __grid_constant__ CUtensorMap tmVm,
                   const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVl, DqParams p) {
@@ -70,19 +86,17 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Qs = smem;
   uint8_t* dOs = Qs + L::kQ;
-  uint8_t* Ks = dOs + L::kQ;        // [2]
-  uint8_t* Vs = Ks + 2 * L::kK;     // [2]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Vs + 2 * L::kK);
-  uint64_t* q_full = bars + 0;      // Q and dO landed
-  uint64_t* k_full = bars + 1;      // [2]
-  uint64_t* k_empty = bars + 3;     // [2] dQ MMA of the tile done
-  uint64_t* v_full = bars + 5;      // [2]
-  uint64_t* v_empty = bars + 7;     // [2] dP MMA of the tile done
-  uint64_t* sp_full = bars + 9;     // S and dP in TMEM
-  uint64_t* ds_full = bars + 10;    // dS written over S (128 arrivals)
-  uint64_t* dq_done = bars + 11;    // last dQ MMA done
-  uint64_t* drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint8_t* Ks = dOs + L::kQ;                 // [kKVStages]
+  uint8_t* Vs = Ks + kKVStages * L::kK;      // [kKVStages]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Vs + kKVStages * L::kK);
+  uint64_t* q_full = bars + 0;               // Q and dO landed
+  uint64_t* kv_full = bars + 1;              // [kKVStages]
+  uint64_t* kv_empty = bars + 1 + kKVStages; // [kKVStages] dQ MMA of the step done
+  uint64_t* sp_full = bars + 1 + 2 * kKVStages;  // [2] S and dP of the buffer in TMEM
+  uint64_t* ds_full = sp_full + 2;           // [2] dS written over S (256 arrivals)
+  uint64_t* dq_done = ds_full + 2;           // last dQ MMA done
+  uint64_t* drain = dq_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = p.n_qblk - 1 - (int)blockIdx.x;  // longest blocks first
@@ -95,19 +109,19 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     if (threadIdx.x == 0 && qb == 0 && g == 0) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
     M = M < 0 ? 0 : p.Mmax;
   }
-  const int NM = (M + kKeys - 1) / kKeys;
-  const int T = NM + (p.Lloc - p.Tq + tlast + kKeys) / kKeys;
+  const int NM = (M + kKS - 1) / kKS;                           // memory steps
+  const int T = NM + (p.Lloc - p.Tq + tlast + kKS) / kKS;       // + local steps up to the last causal key
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
+    for (int i = 0; i < kKVStages; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(sp_full, 1);
-    mbar_init(ds_full, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sp_full[i], 1);
+      mbar_init(&ds_full[i], 256);
+    }
     mbar_init(dq_done, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -120,7 +134,7 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + kKeys, tQ = tmem + 2 * kKeys;
+  const uint32_t tS = tmem, tP = tmem + 2 * kKS, tQ = tmem + 4 * kKS;
   bool timed_out = false;
 
   if (warp == 0) {
@@ -136,95 +150,89 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
       int j = 0;
       for (; j < T; ++j) {
-        const int st = j & 1, ph = ((j >> 1) & 1) ^ 1;
+        const int st = j % kKVStages;
         const bool mem = j < NM;
-        const int y = mem ? b * p.Mmax + j * kKeys : b * p.Lloc + (j - NM) * kKeys;
-        if (!mbar_wait(&k_empty[st], ph, kWaitPolls)) {
+        const int y = mem ? b * p.Mmax + j * kKS : b * p.Lloc + (j - NM) * kKS;
+        if (!mbar_wait(&kv_empty[st], ((j / kKVStages) & 1) ^ 1, kWaitPolls)) {
           timed_out = true;
           break;
         }
-        mbar_arrive_expect_tx(&k_full[st], L::kK);
+        mbar_arrive_expect_tx(&kv_full[st], 2 * L::kK);
 #pragma unroll
-        for (int dc = 0; dc < L::kBoxes; ++dc)
-          tma_load_2d(Ks + st * L::kK + dc * (kKeys * 128), mem ? &tmKm : &tmKl, g * DH + dc * 64, y, &k_full[st]);
-        if (!mbar_wait(&v_empty[st], ph, kWaitPolls)) {
-          timed_out = true;
-          ++j;  // K_j was issued
-          break;
+        for (int dc = 0; dc < L::kBoxes; ++dc) {
+          tma_load_2d(Ks + st * L::kK + dc * (kKS * 128), mem ? &tmKm : &tmKl, g * DH + dc * 64, y, &kv_full[st]);
+          tma_load_2d(Vs + st * L::kK + dc * (kKS * 128), mem ? &tmVm : &tmVl, g * DH + dc * 64, y, &kv_full[st]);
         }
-        mbar_arrive_expect_tx(&v_full[st], L::kK);
-#pragma unroll
-        for (int dc = 0; dc < L::kBoxes; ++dc)
-          tma_load_2d(Vs + st * L::kK + dc * (kKeys * 128), mem ? &tmVm : &tmVl, g * DH + dc * 64, y, &v_full[st]);
       }
       // drain: every copy issued must land before the CTA leaves
       if (!mbar_wait(q_full, 0, kWaitPolls)) timed_out = true;
-      for (int st = 0; st < 2 && st < j; ++st) {
-        const int last = (j - 1 - st) / 2 * 2 + st;
-        if (!mbar_wait(&k_full[st], (last >> 1) & 1, kWaitPolls)) timed_out = true;
-        if (!mbar_wait(&v_full[st], (last >> 1) & 1, kWaitPolls)) timed_out = true;
+      for (int st = 0; st < kKVStages && st < j; ++st) {
+        const int last = (j - 1 - st) / kKVStages * kKVStages + st;
+        if (!mbar_wait(&kv_full[st], (last / kKVStages) & 1, kWaitPolls)) timed_out = true;
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(kRows, kKeys);
+      constexpr uint32_t idS = idesc_bf16_f32(kRows, kKS);
       constexpr uint32_t idQ = idesc_bf16_f32(kRows, DH, /*b_mn_major=*/true);
       const uint32_t q0 = smem_u32(Qs), o0 = smem_u32(dOs);
-      // dQ += dS_j K_j: A = dS_j from TMEM (16 keys of bf16 = 8 columns per step)
-      auto issue_dq = [&](int j) {
-        const uint32_t k0 = smem_u32(Ks + (j & 1) * L::kK);
-#pragma unroll
-        for (int k = 0; k < kKeys / 16; ++k)
-          mma_bf16_ts(tQ, tS + k * 8, desc_mn_sw128(k0 + k * 16 * 128, kKeys * 128), idQ, (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(&k_empty[j & 1]);
-      };
-      bool ok = mbar_wait(q_full, 0, kWaitPolls);
-      for (int j = 0; ok && j < T; ++j) {
-        const int st = j & 1, ph = (j >> 1) & 1;
-        if (!mbar_wait(&k_full[st], ph, kWaitPolls) || !mbar_wait(&v_full[st], ph, kWaitPolls)) {
-          ok = false;
-          break;
-        }
-        if (j > 0) {
-          if (!mbar_wait(ds_full, (j - 1) & 1, kWaitPolls)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_dq(j - 1);
-        }
+      // S, dP of step j into buffer j & 1
+      auto issue_sp = [&](int j) -> bool {
+        const int st = j % kKVStages, buf = j & 1;
+        if (!mbar_wait(&kv_full[st], (j / kKVStages) & 1, kWaitPolls)) return false;
         tc_fence_after();
         const uint32_t k0 = smem_u32(Ks + st * L::kK), v0 = smem_u32(Vs + st * L::kK);
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
           const int box = k >> 2, kk = k & 3;
-          mma_bf16_ss(tS, desc_k_sw128(q0 + box * kRows * 128 + kk * 32), desc_k_sw128(k0 + box * kKeys * 128 + kk * 32),
-                      idS, k > 0 ? 1u : 0u);
+          mma_bf16_ss(tS + buf * kKS, desc_k_sw128(q0 + box * kRows * 128 + kk * 32),
+                      desc_k_sw128(k0 + box * kKS * 128 + kk * 32), idS, k > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
           const int box = k >> 2, kk = k & 3;
-          mma_bf16_ss(tP, desc_k_sw128(o0 + box * kRows * 128 + kk * 32), desc_k_sw128(v0 + box * kKeys * 128 + kk * 32),
-                      idS, k > 0 ? 1u : 0u);
+          mma_bf16_ss(tP + buf * kKS, desc_k_sw128(o0 + box * kRows * 128 + kk * 32),
+                      desc_k_sw128(v0 + box * kKS * 128 + kk * 32), idS, k > 0 ? 1u : 0u);
         }
-        mma_commit(&v_empty[st]);
-        mma_commit(sp_full);
-      }
-      if (ok && mbar_wait(ds_full, (T - 1) & 1, kWaitPolls)) {
+        mma_commit(&sp_full[buf]);
+        return true;
+      };
+      // dQ += dS_j K_j: A = dS_j from TMEM (16 keys of bf16 = 8 columns per MMA)
+      auto issue_dq = [&](int j) {
+        const int st = j % kKVStages, buf = j & 1;
+        const uint32_t k0 = smem_u32(Ks + st * L::kK);
+#pragma unroll
+        for (int k = 0; k < kKS / 16; ++k)
+          mma_bf16_ts(tQ, tS + buf * kKS + k * 8, desc_mn_sw128(k0 + k * 16 * 128, kKS * 128), idQ,
+                      (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&kv_empty[st]);
+      };
+      bool ok = mbar_wait(q_full, 0, kWaitPolls) && issue_sp(0);
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T && !issue_sp(j + 1)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&ds_full[j & 1], (j >> 1) & 1, kWaitPolls)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        issue_dq(T - 1);
-        mma_commit(dq_done);
-      } else {
-        ok = false;
+        issue_dq(j);
       }
+      if (ok) mma_commit(dq_done);
       if (!ok) timed_out = true;
       mma_commit(drain);
       if (!mbar_wait(drain, 0, kWaitPolls)) timed_out = true;
     }
   } else {
     // ---------------------------------------------------------------- softmax
+    // Two warpgroups: warp w reaches TMEM lanes 32 (w % 4) ..; warpgroup `half`
+    // takes key columns [32 half, 32 half + 32) of every step.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int c0 = half * 32;
     const int r = q * 32 + lane;
     const int hh = r / p.TB, t = t0 + r - hh * p.TB;
     const int h = g * p.G + hh;
@@ -234,47 +242,55 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const float nl = rvalid ? -__ldg(p.lse + ((int64_t)b * p.Hq + h) * p.Tq + t) * 1.4426950408889634f : 0.f;
     const float Dr = rvalid ? __ldg(p.Drow + ((int64_t)b * p.Hq + h) * p.Tq + t) : 0.f;
     for (int j = 0; j < T; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(sp_full, j & 1, kWaitPolls))) {
+      const int buf = j & 1;
+      const bool okw = __all_sync(0xffffffffu, mbar_wait(&sp_full[buf], (j >> 1) & 1, kWaitPolls));
+      if (!bar_soft_and(okw)) {
         timed_out = true;
         break;
       }
       tc_fence_after();
       const bool memt = j < NM;
-      const int base = memt ? j * kKeys : (j - NM) * kKeys;
-      const int lim = rvalid ? (memt ? M - base : pos - base + 1) : 0;  // keys [0, lim) are visible
+      const int base = (memt ? j * kKS : (j - NM) * kKS) + c0;
+      const int lim = rvalid ? (memt ? M - base : pos - base + 1) : 0;  // columns [0, lim) are visible
+      float s[32], dp[32];
+      tmem_ld16(tS + buf * kKS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
+      tmem_ld16(tS + buf * kKS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+      tmem_ld16(tP + buf * kKS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
+      tmem_ld16(tP + buf * kKS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
+      tmem_ld_wait();
+      if (!__all_sync(0xffffffffu, lim >= 32)) {  // masked columns: p = 0 and dS = 0
 #pragma unroll
-      for (int c0 = 0; c0 < kKeys; c0 += 32) {
-        float s[32], dp[32];
-        tmem_ld16(tS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
-        tmem_ld16(tS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
-        tmem_ld16(tP + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
-        tmem_ld16(tP + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
-        tmem_ld_wait();
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = c0 + 2 * i;
-          const float p0 = c < lim ? fast_exp2(fmaf(s[2 * i], p.scale_log2, nl)) : 0.f;
-          const float p1 = c + 1 < lim ? fast_exp2(fmaf(s[2 * i + 1], p.scale_log2, nl)) : 0.f;
-          w[i] = pack_bf16x2(c < lim ? p0 * (dp[2 * i] - Dr) : 0.f, c + 1 < lim ? p1 * (dp[2 * i + 1] - Dr) : 0.f);
-        }
-        tmem_st16(tS + lane_off + c0 / 2, w);
+        for (int c = 0; c < 32; ++c)
+          if (c >= lim) {
+            s[c] = -INFINITY;
+            dp[c] = Dr;
+          }
       }
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float p0 = fast_exp2(fmaf(s[2 * i], p.scale_log2, nl));
+        const float p1 = fast_exp2(fmaf(s[2 * i + 1], p.scale_log2, nl));
+        w[i] = pack_bf16x2(p0 * (dp[2 * i] - Dr), p1 * (dp[2 * i + 1] - Dr));
+      }
+      tmem_st16(tS + buf * kKS + lane_off + c0 / 2, w);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(ds_full);
+      mbar_arrive(&ds_full[buf]);
     }
+    // dQ * scale: warpgroup `half` writes columns [64 half, 64 half + 64) of its rows
     if (!timed_out && __all_sync(0xffffffffu, mbar_wait(dq_done, 0, kWaitPolls))) {
       tc_fence_after();
-      float* out = p.dQ + (((int64_t)b * p.Tq + t) * p.Hq + h) * DH;
+      float* out = p.dQ + (((int64_t)b * p.Tq + t) * p.Hq + h) * DH + half * (DH / 2);
 #pragma unroll
-      for (int c = 0; c < DH; c += 16) {
-        float o[16];
-        tmem_ld16(tQ + lane_off + c, o);
+      for (int c = 0; c < DH / 2; c += 32) {
+        float o[32];
+        tmem_ld16(tQ + lane_off + half * (DH / 2) + c, *reinterpret_cast<float(*)[16]>(&o[0]));
+        tmem_ld16(tQ + lane_off + half * (DH / 2) + c + 16, *reinterpret_cast<float(*)[16]>(&o[16]));
         tmem_ld_wait();
         if (rvalid) {
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
+          for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4*>(out + c + i) =
                 make_float4(o[i] * p.scale, o[i + 1] * p.scale, o[i + 2] * p.scale, o[i + 3] * p.scale);
         }
@@ -335,19 +351,6 @@ struct DkvLayout {
   static constexpr uint32_t kTmemCols = 512;  // S^T[2], dP^T[2] (64 each), dK, dV (128 each)
   static_assert(kSmem <= 232448, "shared memory of one CTA");
 };
-
-// Barrier of the 256 softmax threads that also ANDs a predicate over them, so
-// that a failed wait ends the loop for every softmax warp at once.
-__device__ __forceinline__ bool bar_soft_and(bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred pi, po;\n setp.ne.b32 pi, %1, 0;\n bar.red.and.pred po, 1, 256, pi;\n"
-      " selp.u32 %0, 1, 0, po;\n}"
-      : "=r"(r)
-      : "r"((uint32_t)pred)
-      : "memory");
-  return r != 0;
-}
 
 template <int DH>
 __global__ void __launch_bounds__(kDkvThreads, 1)
@@ -727,11 +730,11 @@ cudaError_t launch_attn_dq_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s
   if (!make_tmap_2d_bf16(&tq, a.Q, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB) ||
       !make_tmap_2d_bf16(&tdo, a.dO, (uint64_t)a.Hq * DH, (uint64_t)(a.B * a.Tq), (uint64_t)a.Hq * DH * 2, 64, TB) ||
       !make_tmap_2d_bf16(&tkm, a.Mmax > 0 ? a.Kmem : a.Kloc, (uint64_t)a.Hkv * DH,
-                         (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, kKeys) ||
+                         (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, kKS) ||
       !make_tmap_2d_bf16(&tvm, a.Mmax > 0 ? a.Vmem : a.Vloc, (uint64_t)a.Hkv * DH,
-                         (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, kKeys) ||
-      !make_tmap_2d_bf16(&tkl, a.Kloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKeys) ||
-      !make_tmap_2d_bf16(&tvl, a.Vloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKeys))
+                         (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc), rowkv, 64, kKS) ||
+      !make_tmap_2d_bf16(&tkl, a.Kloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKS) ||
+      !make_tmap_2d_bf16(&tvl, a.Vloc, (uint64_t)a.Hkv * DH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKS))
     return cudaErrorInvalidValue;
   DqParams p;
   p.mem_len = a.mem_len;
@@ -753,7 +756,7 @@ cudaError_t launch_attn_dq_tc(msa_dtype dt, const AttnBwdArgs& a, cudaStream_t s
   if (e != cudaSuccess) return e;
   *handled = true;
   count_launch();
-  attn_dq_tc_kernel<DH><<<dim3((unsigned)p.n_qblk, (unsigned)a.Hkv, (unsigned)a.B), kThreads, L::kSmem, s>>>(
+  attn_dq_tc_kernel<DH><<<dim3((unsigned)p.n_qblk, (unsigned)a.Hkv, (unsigned)a.B), kDqThreads, L::kSmem, s>>>(
       tq, tdo, tkm, tvm, tkl, tvl, p);
   return cudaGetLastError();
 }
