@@ -10,13 +10,14 @@
 //        is rounded to bf16 and written back over S
 //   dQ += dS K_j                          (dS as the MMA's A operand from TMEM,
 //                                          K_j MN-major from its TMA tile)
-// and dQ * scale is written in fp32 at the end.  S and dP have two TMEM
-// buffers, so the tensor cores compute step j+1 while the softmax warps work
-// on step j; the MMAs run in issue order, so S_{j+1} (issued after dQ_{j-1},
-// which reads the same buffer) never overwrites dS_{j-1} before it is read.
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2..9 softmax in two warpgroups of 32 key columns each.  Every
-// wait is bounded and ends the CTA with MSA_FLAG_TIMEOUT on expiry.
+// and dQ * scale is written in fp32 at the end.  S and dP have three TMEM
+// buffers and two softmax warpgroups take alternate steps, so two steps are in
+// the softmax while the tensor cores compute the next; the MMAs run in issue
+// order, so S_{j+2} (issued after dQ_{j-1}, which reads the same buffer) never
+// overwrites dS_{j-1} before it is read.  Warp roles (320 threads): warp 0 TMA
+// producer, warp 1 TMEM owner + MMA issuer, warps 2..9 softmax (warpgroup 0
+// even steps, 1 odd).  Every wait is bounded and ends the CTA with
+// MSA_FLAG_TIMEOUT on expiry.
 #include <algorithm>
 #include <climits>
 
@@ -51,9 +52,9 @@ struct DqLayout {
   static constexpr int kBoxes = DH / 64;
   static constexpr int kQ = kRows * DH * 2;
   static constexpr int kK = kKS * DH * 2;   // one 64-key step of K or V
-  static constexpr int kBar = 16 * 8;
+  static constexpr int kBar = 24 * 8;        // 17 barriers and the TMEM address
   static constexpr int kSmem = 1024 + 2 * kQ + 2 * kKVStages * kK + kBar;  // Q, dO, K[4], V[4]
-  static constexpr uint32_t kTmemCols = 512;  // S[2], dP[2] (64 each), dQ (128)
+  static constexpr uint32_t kTmemCols = 512;  // S[3], dP[3] (64 each), dQ (128)
   static_assert(kSmem <= 232448, "shared memory of one CTA");
 };
 
@@ -92,9 +93,9 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   uint64_t* q_full = bars + 0;               // Q and dO landed
   uint64_t* kv_full = bars + 1;              // [kKVStages]
   uint64_t* kv_empty = bars + 1 + kKVStages; // [kKVStages] dQ MMA of the step done
-  uint64_t* sp_full = bars + 1 + 2 * kKVStages;  // [2] S and dP of the buffer in TMEM
-  uint64_t* ds_full = sp_full + 2;           // [2] dS written over S (256 arrivals)
-  uint64_t* dq_done = ds_full + 2;           // last dQ MMA done
+  uint64_t* sp_full = bars + 1 + 2 * kKVStages;  // [3] S and dP of the buffer in TMEM
+  uint64_t* ds_full = sp_full + 3;           // [3] dS written over S (128 arrivals: one warpgroup)
+  uint64_t* dq_done = ds_full + 3;           // last dQ MMA done
   uint64_t* drain = dq_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
@@ -118,9 +119,9 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&sp_full[i], 1);
-      mbar_init(&ds_full[i], 256);
+      mbar_init(&ds_full[i], 128);
     }
     mbar_init(dq_done, 1);
     mbar_init(drain, 1);
@@ -134,7 +135,7 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + 2 * kKS, tQ = tmem + 4 * kKS;
+  const uint32_t tS = tmem, tP = tmem + 3 * kKS, tQ = tmem + 6 * kKS;
   bool timed_out = false;
 
   if (warp == 0) {
@@ -177,9 +178,9 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       constexpr uint32_t idS = idesc_bf16_f32(kRows, kKS);
       constexpr uint32_t idQ = idesc_bf16_f32(kRows, DH, /*b_mn_major=*/true);
       const uint32_t q0 = smem_u32(Qs), o0 = smem_u32(dOs);
-      // S, dP of step j into buffer j & 1
+      // S, dP of step j into buffer j % 3
       auto issue_sp = [&](int j) -> bool {
-        const int st = j % kKVStages, buf = j & 1;
+        const int st = j % kKVStages, buf = j % 3;
         if (!mbar_wait(&kv_full[st], (j / kKVStages) & 1, kWaitPolls)) return false;
         tc_fence_after();
         const uint32_t k0 = smem_u32(Ks + st * L::kK), v0 = smem_u32(Vs + st * L::kK);
@@ -200,7 +201,7 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       };
       // dQ += dS_j K_j: A = dS_j from TMEM (16 keys of bf16 = 8 columns per MMA)
       auto issue_dq = [&](int j) {
-        const int st = j % kKVStages, buf = j & 1;
+        const int st = j % kKVStages, buf = j % 3;
         const uint32_t k0 = smem_u32(Ks + st * L::kK);
 #pragma unroll
         for (int k = 0; k < kKS / 16; ++k)
@@ -208,13 +209,13 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                       (j > 0 || k > 0) ? 1u : 0u);
         mma_commit(&kv_empty[st]);
       };
-      bool ok = mbar_wait(q_full, 0, kWaitPolls) && issue_sp(0);
+      bool ok = mbar_wait(q_full, 0, kWaitPolls) && issue_sp(0) && (T < 2 || issue_sp(1));
       for (int j = 0; ok && j < T; ++j) {
-        if (j + 1 < T && !issue_sp(j + 1)) {
+        if (j + 2 < T && !issue_sp(j + 2)) {
           ok = false;
           break;
         }
-        if (!mbar_wait(&ds_full[j & 1], (j >> 1) & 1, kWaitPolls)) {
+        if (!mbar_wait(&ds_full[j % 3], (j / 3) & 1, kWaitPolls)) {
           ok = false;
           break;
         }
@@ -229,10 +230,9 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   } else {
     // ---------------------------------------------------------------- softmax
     // Two warpgroups: warp w reaches TMEM lanes 32 (w % 4) ..; warpgroup `half`
-    // takes key columns [32 half, 32 half + 32) of every step.
+    // takes steps j = half, half + 2, ... (all 64 key columns of each).
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
-    const int c0 = half * 32;
     const int r = q * 32 + lane;
     const int hh = r / p.TB, t = t0 + r - hh * p.TB;
     const int h = g * p.G + hh;
@@ -241,39 +241,42 @@ attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float nl = rvalid ? -__ldg(p.lse + ((int64_t)b * p.Hq + h) * p.Tq + t) * 1.4426950408889634f : 0.f;
     const float Dr = rvalid ? __ldg(p.Drow + ((int64_t)b * p.Hq + h) * p.Tq + t) : 0.f;
-    for (int j = 0; j < T; ++j) {
-      const int buf = j & 1;
-      const bool okw = __all_sync(0xffffffffu, mbar_wait(&sp_full[buf], (j >> 1) & 1, kWaitPolls));
-      if (!bar_soft_and(okw)) {
+    for (int j = half; j < T; j += 2) {
+      const int buf = j % 3;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sp_full[buf], (j / 3) & 1, kWaitPolls))) {
         timed_out = true;
         break;
       }
       tc_fence_after();
       const bool memt = j < NM;
-      const int base = (memt ? j * kKS : (j - NM) * kKS) + c0;
+      const int base = memt ? j * kKS : (j - NM) * kKS;
       const int lim = rvalid ? (memt ? M - base : pos - base + 1) : 0;  // columns [0, lim) are visible
-      float s[32], dp[32];
-      tmem_ld16(tS + buf * kKS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
-      tmem_ld16(tS + buf * kKS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
-      tmem_ld16(tP + buf * kKS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
-      tmem_ld16(tP + buf * kKS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
-      tmem_ld_wait();
-      if (!__all_sync(0xffffffffu, lim >= 32)) {  // masked columns: p = 0 and dS = 0
+      const bool whole = __all_sync(0xffffffffu, lim >= kKS);
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (c >= lim) {
-            s[c] = -INFINITY;
-            dp[c] = Dr;
-          }
-      }
-      uint32_t w[16];
+      for (int c0 = 0; c0 < kKS; c0 += 32) {
+        float s[32], dp[32];
+        tmem_ld16(tS + buf * kKS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&s[0]));
+        tmem_ld16(tS + buf * kKS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&s[16]));
+        tmem_ld16(tP + buf * kKS + lane_off + c0, *reinterpret_cast<float(*)[16]>(&dp[0]));
+        tmem_ld16(tP + buf * kKS + lane_off + c0 + 16, *reinterpret_cast<float(*)[16]>(&dp[16]));
+        tmem_ld_wait();
+        if (!whole) {  // masked columns: p = 0 and dS = 0
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float p0 = fast_exp2(fmaf(s[2 * i], p.scale_log2, nl));
-        const float p1 = fast_exp2(fmaf(s[2 * i + 1], p.scale_log2, nl));
-        w[i] = pack_bf16x2(p0 * (dp[2 * i] - Dr), p1 * (dp[2 * i + 1] - Dr));
+          for (int c = 0; c < 32; ++c)
+            if (c0 + c >= lim) {
+              s[c] = -INFINITY;
+              dp[c] = Dr;
+            }
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(s[2 * i], p.scale_log2, nl));
+          const float p1 = fast_exp2(fmaf(s[2 * i + 1], p.scale_log2, nl));
+          w[i] = pack_bf16x2(p0 * (dp[2 * i] - Dr), p1 * (dp[2 * i + 1] - Dr));
+        }
+        tmem_st16(tS + buf * kKS + lane_off + c0 / 2, w);
       }
-      tmem_st16(tS + buf * kKS + lane_off + c0 / 2, w);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ds_full[buf]);
