@@ -335,8 +335,8 @@ def stage_roofline(name: str, ms: float, cfg: synth.Config, counts: dict, peaks:
 
 
 def run_backward(args, rank, local_rank, world):
-    """Backward of the query path: per layer msa_sparse_attn_backward + msa_gather_backward, the
-    forward outputs (O, lse, the gathered rows) computed once before timing."""
+    """Backward of the query path: per layer msa_sparse_attn_backward + msa_gather_backward +
+    msa_route_backward, the forward outputs (O, lse, the gathered rows) computed once before timing."""
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     if world > 1:
@@ -369,6 +369,13 @@ def run_backward(args, rank, local_rank, world):
     dKb, dVb = torch.zeros((w.C, c.Hkv, c.d), **f32), torch.zeros((w.C, c.Hkv, c.d), **f32)
     bws = torch.empty(max(256, msa.sparse_attn_backward_workspace_size(B, c.Tq, c.Hq)), dtype=torch.uint8,
                       device=device)
+    # routing-score backward: the routing loss is not given, so its gradient per selected document is a
+    # seeded synthetic input; dQr / dK̄r accumulate over the layers like dK̄ / dV̄
+    d_score = [torch.randn((B, c.k), generator=torch.Generator(device=device).manual_seed(11 + l), device=device)
+               for l in range(cfg.layers)]
+    dQr = torch.zeros((B, c.Tq, c.Hr, c.dr), **f32)
+    dKrb = torch.zeros((w.C, c.Hr, c.dr), **f32)
+    rbws = torch.empty(max(256, msa.route_backward_workspace_size(B, c.Tq, c.k)), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
     marks = []
 
@@ -384,6 +391,8 @@ def run_backward(args, rank, local_rank, world):
             r and r("attn_backward")
             msa.gather_backward(w.idx[l], w.coff_d, dKm, dVm, ml, dKb, dVb, w.flag)
             r and r("gather_backward")
+            msa.route_backward(L["Qr"], w.Krb, w.rn, w.coff_d, w.idx[l], d_score[l], dQr, dKrb, rbws, w.flag)
+            r and r("route_backward")
 
     for _ in range(args.warmup):
         step()
@@ -398,7 +407,7 @@ def run_backward(args, rank, local_rank, world):
     torch.cuda.synchronize()
     launches = msa.kernel_launch_count() - n0
     clocks = sampler.stop()
-    stage_ms = {"attn_backward": [], "gather_backward": []}
+    stage_ms = {"attn_backward": [], "gather_backward": [], "route_backward": []}
     for (s0, e0), (s1, e1) in zip(marks[:-1], marks[1:]):
         if s1 != "start":
             stage_ms[s1].append(e0.elapsed_time(e1))
@@ -412,6 +421,7 @@ def run_backward(args, rank, local_rank, world):
     flops = 2.5 * counts["attn_flops"] / cfg.layers  # 10 d flops per visible (row, key) pair: s, dp, dq, dk, dv
     achieved = flops / per / 1e9
     gper = float(np.mean(stage_ms["gather_backward"]))
+    rper = float(np.mean(stage_ms["route_backward"]))
     G = c.Hq // c.Hkv
     tensor = cfg.dtype == "bf16" and c.d == 128 and 128 % G == 0 and 128 // G >= 8
     if tensor:  # the tcgen05 dQ and dK / dV kernels: the bf16 tensor peak
@@ -430,13 +440,15 @@ def run_backward(args, rank, local_rank, world):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 (gradients; inputs " + cfg.dtype + ")", "data": "synthetic",
         "config": {"workload": workload_label(cfg), "step": "backward: per layer msa_sparse_attn_backward + "
-                   "msa_gather_backward (forward outputs computed before timing)", "parallelism": "single GPU"},
+                   "msa_gather_backward + msa_route_backward (forward outputs computed before timing; the routing "
+                   "loss's gradient per selected document is a seeded synthetic input)", "parallelism": "single GPU"},
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
                      "kernel": kname, "alg_flops_per_launch": flops,
                      "peak_source": psrc, "frac": round(achieved / peak, 4),
                      "avg_launch_ms": round(per, 4), "traffic": None},
         "stages": {"attn_backward": {"ms_per_launch": round(per, 4)},
-                   "gather_backward": {"ms_per_launch": round(gper, 4)}},
+                   "gather_backward": {"ms_per_launch": round(gper, 4)},
+                   "route_backward": {"ms_per_launch": round(rper, 4)}},
         "gpu_launches": launches, "clocks": clocks, "err_flag": flag,
     }
 

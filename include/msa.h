@@ -301,12 +301,12 @@ msa_status msa_gather_backward(const int32_t* topk_idx, int64_t B, int k, const 
  * caller zeroes them or passes earlier gradients; a token or chunk that wins
  * for several documents or queries receives the sum (fp32 atomics, so the
  * summation order is not fixed).  A document with no chunks gets no
- * gradient.  The workspace holds msa_route_backward_workspace_size(B, k)
+ * gradient.  The workspace holds msa_route_backward_workspace_size(B, Tq, k)
  * bytes.  Errors as msa_route_topk; device flags: MSA_FLAG_INDEX_OOB for a
  * document index or chunk range out of range, or a document with more than
  * 2^31 - 1 (chunk, token) pairs (that document is skipped).
  * ---------------------------------------------------------------------- */
-size_t msa_route_backward_workspace_size(int64_t B, int k);
+size_t msa_route_backward_workspace_size(int64_t B, int Tq, int k);
 msa_status msa_route_backward(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr,
                               const void* Krbar, const float* kr_rnorm,
                               const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,

@@ -175,8 +175,8 @@ def gather_backward(topk_idx, doc_chunk_off, dKmem, dVmem, mem_len, dKbar, dVbar
           _s(stream))
 
 
-def route_backward_workspace_size(B, k) -> int:
-    return _lib.load().msa_route_backward_workspace_size(B, k)
+def route_backward_workspace_size(B, Tq, k) -> int:
+    return _lib.load().msa_route_backward_workspace_size(B, Tq, k)
 
 
 def route_backward(Qr, Krbar, kr_rnorm, doc_chunk_off, topk_idx, d_score, dQr, dKrbar, ws, err_flag=None,

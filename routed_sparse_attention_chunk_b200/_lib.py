@@ -38,7 +38,7 @@ SIGNATURES = {
                                            P, P, P, C.c_int, F32, P, P, P, P, P, P, P, P, P, SZ, P, P]),
     "msa_gather_backward": (C.c_int, [P, I64, C.c_int, P, I64, I64, P, P, P, C.c_int, C.c_int, C.c_int,
                                       P, P, P, P]),
-    "msa_route_backward_workspace_size": (SZ, [I64, C.c_int]),
+    "msa_route_backward_workspace_size": (SZ, [I64, C.c_int, C.c_int]),
     "msa_route_backward": (C.c_int, [C.c_int, P, I64, C.c_int, C.c_int, C.c_int, P, P, P, I64, I64, C.c_int,
                                      P, P, P, P, P, SZ, P, P]),
     "msa_layer_forward_workspace_size": (SZ, [I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,

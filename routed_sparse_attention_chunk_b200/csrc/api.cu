@@ -240,9 +240,9 @@ msa_status msa_gather_backward(const int32_t* topk_idx, int64_t B, int k, const 
   return cuda_status(launch_gather_bwd(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-size_t msa_route_backward_workspace_size(int64_t B, int k) {
-  if (B < 0 || k < 1) return 0;
-  return route_bwd_workspace_size(B, k);
+size_t msa_route_backward_workspace_size(int64_t B, int Tq, int k) {
+  if (B < 0 || Tq < 1 || k < 1) return 0;
+  return route_bwd_workspace_size(B, Tq, k);
 }
 
 msa_status msa_route_backward(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr, const void* Krbar,
@@ -254,7 +254,7 @@ msa_status msa_route_backward(msa_dtype dt, const void* Qr, int64_t B, int Tq, i
   if (B > 65535 || k > 65535) return MSA_ERR_UNSUPPORTED;
   if (B == 0) return MSA_OK;
   if (!d_score || !dQr || !dKrbar) return MSA_ERR_INVALID_ARG;
-  const size_t need = route_bwd_workspace_size(B, k);
+  const size_t need = route_bwd_workspace_size(B, Tq, k);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
   RouteBwdArgs a{Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, k, topk_idx, d_score,
                  dQr, dKrbar, ws, err_flag};

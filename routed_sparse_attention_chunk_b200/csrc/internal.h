@@ -122,7 +122,7 @@ struct RouteBwdArgs {
   void* ws;  // route_bwd_workspace_size bytes
   int32_t* err_flag;
 };
-size_t route_bwd_workspace_size(int64_t B, int k);
+size_t route_bwd_workspace_size(int64_t B, int Tq, int k);
 cudaError_t launch_route_bwd(msa_dtype dt, const RouteBwdArgs& a, cudaStream_t s);
 
 // Top-k over ordered document keys [B, D]: writes idx / score (score may be null)

@@ -8,12 +8,14 @@
 // derivative spreads it over that token's Qr and that chunk's K̄r:
 //   dQr[t*, h] += g/Hr (k / (|q| |k|) - cos q / |q|^2)
 //   dK̄r[c*, h] += g/Hr (q / (|q| |k|) - cos k / |k|^2)
-// Two launches: route_bwd_scan_kernel, grid (splits, k, B), recomputes s for
-// its share of the document's (chunk, token) pairs (one pair per thread, fp32)
-// and leaves its best pair in the workspace; route_bwd_grad_kernel, grid
-// (k, B), one warp per router head, picks the best pair over the splits and
-// adds the gradient with fp32 atomics (a token or chunk shared by several
-// documents or queries accumulates).
+// Two launches: route_bwd_scan_kernel, grid (ceil(Tq / 64), k, B), recomputes
+// s for the document's chunks and 64 of the query's tokens (four threads per
+// token, a quarter of the router heads each, the Qr row read once per group of
+// 8 chunks whose normalised K̄r rows sit in shared memory; fp32) and leaves its
+// best pair in the workspace;
+// route_bwd_grad_kernel, grid (k, B), one warp per router head, picks the best
+// pair over the splits and adds the gradient with fp32 atomics (a token or
+// chunk shared by several documents or queries accumulates).
 #include <math.h>
 
 #include "common.cuh"
@@ -22,7 +24,7 @@
 namespace msa {
 namespace {
 
-constexpr int kSplits = 16;
+constexpr int kTokPerBlock = 64;  // tokens per scan block (4 threads each)
 constexpr int kScanThreads = 256;
 
 struct Cand {
@@ -34,10 +36,16 @@ __device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
   return a.pair >= 0 && (b.pair < 0 || a.s > b.s || (a.s == b.s && a.pair < b.pair));
 }
 
+constexpr int kCG = 8;        // chunks per shared-memory group
+constexpr int kPad = 4;       // floats after each head's row: the 4 threads of a token read
+                              // 4 heads at once, and rows 528 bytes apart fall in different banks
+constexpr int kMaxHD = 8 * (128 + kPad);  // Hr * (dr + kPad) at most
+
 template <typename T>
 __global__ void __launch_bounds__(kScanThreads) route_bwd_scan_kernel(RouteBwdArgs a, Cand* __restrict__ ws) {
   const int split = blockIdx.x, r = blockIdx.y;
   const int64_t b = blockIdx.z;
+  __shared__ __align__(16) float khat[kCG][kMaxHD];  // K̄r[c, h, :] / |K̄r[c, h]|, head rows dr + kPad apart
   __shared__ Cand red[kScanThreads / 32];
   Cand best{-INFINITY, -1};
   const int32_t j = __ldg(a.topk_idx + b * a.k + r);
@@ -47,38 +55,83 @@ __global__ void __launch_bounds__(kScanThreads) route_bwd_scan_kernel(RouteBwdAr
     const int64_t ce = __ldg(a.doc_chunk_off + j + 1);
     if (cs >= 0 && ce <= a.C && ce >= cs) n = ce - cs;
   }
-  int64_t pairs = n * a.Tq;
-  if (pairs > 0x7fffffffLL) {  // the pair index is int32: such a document is skipped
+  if (n * a.Tq > 0x7fffffffLL) {  // the pair index is int32: such a document is skipped
     if (split == 0 && threadIdx.x == 0) raise_flag(a.err_flag, MSA_FLAG_INDEX_OOB);
-    pairs = 0;
+    n = 0;
   }
-  const int64_t per = (pairs + kSplits - 1) / kSplits;
-  const int64_t p0 = split * per, p1 = min(pairs, p0 + per);
-  const T* Q = reinterpret_cast<const T*>(a.Qr);
+  const int HD = a.Hr * a.dr;
+  const int ta = split * kTokPerBlock, tb = min(a.Tq, ta + kTokPerBlock);
+  const int sub = threadIdx.x & 3, tl = threadIdx.x >> 2;
   const T* K = reinterpret_cast<const T*>(a.Krbar);
   constexpr int VN = Vec<T>::N;
-  for (int64_t p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
-    const int64_t c = cs + p / a.Tq;
-    const int t = (int)(p % a.Tq);
-    float s = 0.f;
-    for (int h = 0; h < a.Hr; ++h) {
-      const uint4* qv = reinterpret_cast<const uint4*>(Q + ((b * a.Tq + t) * a.Hr + h) * (int64_t)a.dr);
-      const uint4* kv = reinterpret_cast<const uint4*>(K + (c * a.Hr + h) * (int64_t)a.dr);
-      float dot = 0.f, nq = 0.f;
-      for (int v = 0; v < a.dr / VN; ++v) {
-        float x[VN], y[VN];
-        unpack(__ldg(qv + v), x);
-        unpack(__ldg(kv + v), y);
+  for (int64_t g0 = 0; g0 < n; g0 += kCG) {
+    const int ng = (int)min((int64_t)kCG, n - g0);
+    __syncthreads();  // the previous group's rows are no longer read
+    // 16-byte vectors: (chunk, head) row rh, vector v of the row
+    const int nv = a.dr / VN;
+    for (int i = threadIdx.x; i < ng * a.Hr * nv; i += blockDim.x) {
+      const int rh = i / nv, v = i - rh * nv;
+      const int cc = rh / a.Hr, h = rh - cc * a.Hr;
+      const int64_t c = cs + g0 + cc;
+      float x[VN];
+      unpack(__ldg(reinterpret_cast<const uint4*>(K + c * HD + h * a.dr) + v), x);
+      const float rk = __ldg(a.kr_rnorm + c * a.Hr + h);
+      float* dst = &khat[cc][h * (a.dr + kPad) + v * VN];
 #pragma unroll
-        for (int i = 0; i < VN; ++i) {
-          dot = fmaf(x[i], y[i], dot);
-          nq = fmaf(x[i], x[i], nq);
+      for (int u = 0; u < VN; u += 4)
+        *reinterpret_cast<float4*>(dst + u) = make_float4(x[u] * rk, x[u + 1] * rk, x[u + 2] * rk, x[u + 3] * rk);
+    }
+    __syncthreads();
+    for (int t0 = ta; t0 < tb; t0 += kScanThreads / 4) {  // uniform over the block
+      const int t = t0 + tl;
+      const bool tv = t < tb;
+      float sc[kCG];
+#pragma unroll
+      for (int cc = 0; cc < kCG; ++cc) sc[cc] = 0.f;
+      if (tv) {
+        const uint4* qv = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.Qr) + (b * a.Tq + t) * HD);
+        for (int h = sub; h < a.Hr; h += 4) {
+          float dot[kCG], nq = 0.f;
+#pragma unroll
+          for (int cc = 0; cc < kCG; ++cc) dot[cc] = 0.f;
+          for (int v = 0; v < a.dr / VN; ++v) {
+            float x[VN];
+            unpack(__ldg(qv + (h * a.dr) / VN + v), x);
+            const int e0 = h * (a.dr + kPad) + v * VN;
+#pragma unroll
+            for (int i = 0; i < VN; ++i) nq = fmaf(x[i], x[i], nq);
+#pragma unroll
+            for (int cc = 0; cc < kCG; ++cc) {
+              if (cc < ng) {
+#pragma unroll
+                for (int i = 0; i < VN; i += 4) {
+                  const float4 k4 = *reinterpret_cast<const float4*>(&khat[cc][e0 + i]);
+                  dot[cc] = fmaf(x[i], k4.x, fmaf(x[i + 1], k4.y, fmaf(x[i + 2], k4.z, fmaf(x[i + 3], k4.w, dot[cc]))));
+                }
+              }
+            }
+          }
+          const float rq = 1.f / fmaxf(sqrtf(nq), 1e-12f);
+#pragma unroll
+          for (int cc = 0; cc < kCG; ++cc) sc[cc] += dot[cc] * rq;
         }
       }
-      s += dot / fmaxf(sqrtf(nq), 1e-12f) * __ldg(a.kr_rnorm + c * a.Hr + h);
+      // the four threads of a token hold the sums over their heads
+#pragma unroll
+      for (int cc = 0; cc < kCG; ++cc) {
+        sc[cc] += __shfl_xor_sync(0xffffffffu, sc[cc], 1);
+        sc[cc] += __shfl_xor_sync(0xffffffffu, sc[cc], 2);
+      }
+      if (tv && sub == 0) {
+#pragma unroll
+        for (int cc = 0; cc < kCG; ++cc) {
+          if (cc < ng) {
+            const Cand cand{sc[cc] / (float)a.Hr, (int32_t)((g0 + cc) * a.Tq + t)};
+            if (better(cand, best)) best = cand;
+          }
+        }
+      }
     }
-    const Cand cand{s / (float)a.Hr, (int32_t)p};
-    if (better(cand, best)) best = cand;
   }
   // block argmax (ties to the lower pair index)
 #pragma unroll
@@ -91,7 +144,7 @@ __global__ void __launch_bounds__(kScanThreads) route_bwd_scan_kernel(RouteBwdAr
   if (threadIdx.x == 0) {
     for (int w = 1; w < kScanThreads / 32; ++w)
       if (better(red[w], best)) best = red[w];
-    ws[(b * a.k + r) * kSplits + split] = best;
+    ws[(b * a.k + r) * gridDim.x + split] = best;
   }
 }
 
@@ -111,8 +164,9 @@ __global__ void route_bwd_grad_kernel(RouteBwdArgs a, const Cand* __restrict__ w
     return;
   }
   Cand best{-INFINITY, -1};
-  for (int sp = 0; sp < kSplits; ++sp) {
-    const Cand c = ws[(b * a.k + r) * kSplits + sp];
+  const int nsplit = (a.Tq + kTokPerBlock - 1) / kTokPerBlock;
+  for (int sp = 0; sp < nsplit; ++sp) {
+    const Cand c = ws[(b * a.k + r) * nsplit + sp];
     if (better(c, best)) best = c;
   }
   if (best.pair < 0 || h >= a.Hr) return;  // a document with no chunks
@@ -149,7 +203,8 @@ template <typename T>
 cudaError_t route_bwd_t(const RouteBwdArgs& a, cudaStream_t s) {
   Cand* ws = static_cast<Cand*>(a.ws);
   count_launch();
-  route_bwd_scan_kernel<T><<<dim3(kSplits, (unsigned)a.k, (unsigned)a.B), kScanThreads, 0, s>>>(a, ws);
+  const unsigned nsplit = (unsigned)((a.Tq + kTokPerBlock - 1) / kTokPerBlock);
+  route_bwd_scan_kernel<T><<<dim3(nsplit, (unsigned)a.k, (unsigned)a.B), kScanThreads, 0, s>>>(a, ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   count_launch();
@@ -159,8 +214,9 @@ cudaError_t route_bwd_t(const RouteBwdArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-size_t route_bwd_workspace_size(int64_t B, int k) {
-  return ((sizeof(Cand) * (size_t)B * (size_t)k * kSplits) + 255) / 256 * 256;
+size_t route_bwd_workspace_size(int64_t B, int Tq, int k) {
+  const size_t nsplit = (size_t)((Tq + kTokPerBlock - 1) / kTokPerBlock);
+  return ((sizeof(Cand) * (size_t)B * (size_t)k * nsplit) + 255) / 256 * 256;
 }
 
 cudaError_t launch_route_bwd(msa_dtype dt, const RouteBwdArgs& a, cudaStream_t s) {

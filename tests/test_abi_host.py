@@ -170,7 +170,7 @@ def test_backward_entry_points_reject_bad_arguments():
     assert gcall(k=0) == INVALID
     assert gcall(B=0) == OK
     rb = dict(dt=1, Qr=FAKE, B=2, Tq=4, Hr=8, dr=128, Krb=FAKE, rn=FAKE, chk=FAKE, D=10, C=30, k=4, idx=FAKE,
-              dsc=FAKE, dQr=FAKE, dKrb=FAKE, ws=FAKE, wsb=lib.msa_route_backward_workspace_size(2, 4), flag=None)
+              dsc=FAKE, dQr=FAKE, dKrb=FAKE, ws=FAKE, wsb=lib.msa_route_backward_workspace_size(2, 4, 4), flag=None)
     rcall = lambda **kw: lib.msa_route_backward(*dict(rb, **kw).values(), None)
     assert rcall(dr=96) == UNSUPPORTED
     assert rcall(Hr=9) == UNSUPPORTED
@@ -180,4 +180,5 @@ def test_backward_entry_points_reject_bad_arguments():
     assert rcall(Qr=FAKE + 4) == INVALID      # misaligned
     assert rcall(wsb=0) == WORKSPACE
     assert rcall(B=0) == OK
-    assert lib.msa_route_backward_workspace_size(2, 4) >= 2 * 4 * 8
+    assert lib.msa_route_backward_workspace_size(2, 4, 4) >= 2 * 4 * 8
+    assert lib.msa_route_backward_workspace_size(2, 130, 4) >= 2 * 4 * 8 * 3   # a candidate per 64 tokens

@@ -158,7 +158,7 @@ def _route_bwd_gpu(Qr, Krb, rn, coff, idx, dsc):
     t = lambda a: torch.from_numpy(a).to(DEV)
     dQr = torch.zeros((B, Tq, Hr, dr), dtype=torch.float32, device=DEV)
     dKrb = torch.zeros((Krb.shape[0], Hr, dr), dtype=torch.float32, device=DEV)
-    ws = torch.empty(msa.route_backward_workspace_size(B, idx.shape[1]), dtype=torch.uint8, device=DEV)
+    ws = torch.empty(msa.route_backward_workspace_size(B, Tq, idx.shape[1]), dtype=torch.uint8, device=DEV)
     flag = torch.zeros(1, dtype=torch.int32, device=DEV)
     msa.route_backward(Qr, Krb, rn, t(coff), t(idx), t(dsc), dQr, dKrb, ws, flag)
     torch.cuda.synchronize()
@@ -170,6 +170,8 @@ def _route_bwd_gpu(Qr, Krb, rn, coff, idx, dsc):
     (2, 64, 8, 128, 40, 24, 8, torch.bfloat16),    # thousands of pairs: every split busy, ragged tail
     (4, 1, 4, 64, 9, 50, 16, torch.bfloat16),      # decode: one token, max over chunks only
     (2, 33, 1, 64, 3, 12, 12, torch.float32),      # Hr = 1, every document selected
+    (2, 150, 3, 64, 5, 20, 6, torch.bfloat16),     # three token blocks (ragged), Hr not a multiple of 4
+    (1, 200, 8, 128, 19, 10, 4, torch.float32),    # documents of more than 8 chunks: several chunk groups
 ])
 def test_route_backward_matches_oracle(B, Tq, Hr, dr, maxlen, D, k, dtype):
     rng = np.random.default_rng(B * 1000 + Tq)
@@ -207,7 +209,7 @@ def test_route_backward_accumulates_over_shared_documents_after_routing():
     base_q = torch.randn((B, Tq, Hr, dr), device=DEV)
     base_k = torch.randn((Krb.shape[0], Hr, dr), device=DEV)
     dQr, dKrb = base_q.clone(), base_k.clone()
-    ws = torch.empty(msa.route_backward_workspace_size(B, cfg.k), dtype=torch.uint8, device=DEV)
+    ws = torch.empty(msa.route_backward_workspace_size(B, Tq, cfg.k), dtype=torch.uint8, device=DEV)
     flag = torch.zeros(1, dtype=torch.int32, device=DEV)
     msa.route_backward(Qr, Krb, rn, t(coff), t(idx), t(dsc), dQr, dKrb, ws, flag)
     torch.cuda.synchronize()
