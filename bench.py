@@ -231,6 +231,28 @@ class MSAWorkload:
         self.ml = torch.zeros(B, dtype=torch.int32, device=device)
         n = msa.sparse_attn_workspace_size(B, c.Tq, c.Lloc, c.Hq, c.Hkv, c.d, c.Mmax)
         self.aws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+        self.pipe = None
+
+    def enable_pipeline(self):
+        """Run the query path through the three-stream schedule (route of batch i+1, gather of batch
+        i and attention of batch i-1 overlapped); a second topk_idx per layer lets route and gather of
+        consecutive batches overlap."""
+        from routed_sparse_attention_chunk_b200.pipeline import QueryPipeline
+        c = self.cfg
+        bank = dict(Krbar=self.Krb, kr_rnorm=self.rn, doc_chunk_off=self.coff_d, Kbar=self.Kb, Vbar=self.Vb)
+        self.pipe = QueryPipeline(bank, c.k, c.Mmax, c.B, c.Tq, c.Lloc, c.Hq, c.Hkv, c.d, c.Hr, c.torch_dtype,
+                                  self.dev, err_flag=self.flag)
+        self.idx2 = [torch.empty_like(t) for t in self.idx]
+
+    def pipelined_steps(self, n, marks=None):
+        """n steps (every layer of each) enqueued through the schedule in one call, so consecutive steps
+        overlap too; the caller's stream waits for all of it."""
+        runs = []
+        for i in range(n):
+            for l, L in enumerate(self.layers):
+                runs.append(dict(L, O=self.O[l], topk_idx=(self.idx[l] if (i * len(self.layers) + l) % 2 == 0
+                                                            else self.idx2[l])))
+        self.pipe.run(runs, marks)
 
     def _fill_raw(self, seed):
         """Resident raw K / V / Kr for the whole corpus, drawn slab by slab."""
@@ -471,6 +493,12 @@ def run_gpu(args, rank, local_rank, world):
         in_bytes += w.Krb.numel() * w.Krb.element_size()  # the scan reads the whole bank every step
     flush = None if in_bytes > L2_BYTES else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
 
+    if args.pipeline:
+        if step_kind != "query":
+            raise SystemExit("--pipeline runs the query path over a bank pooled before timing (--step query)")
+        w.enable_pipeline()
+        return run_pipelined(args, rank, world, device, w, cfg, counts, peaks, peak_kind, flush)
+
     # ---- warm-up, then exactly K timed steps, an event after every stage
     stream = torch.cuda.current_stream()
     sampler = ClockSampler(device)
@@ -578,6 +606,124 @@ def run_gpu(args, rank, local_rank, world):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_budget, with_pool=step_kind == "full")
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world, device)
+        dist.destroy_process_group()
+    return result
+
+
+def host_link_gbs(device, mib: int = 256) -> float:
+    """Page-locked host -> device copy bandwidth (copy engine, best of 5): the host link's measured peak."""
+    h = torch.empty(mib << 20, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(mib << 20, dtype=torch.uint8, device=device)
+    best = float("inf")
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        d.copy_(h, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    return (mib << 20) / (best / 1e3) / 1e9
+
+
+def run_pipelined(args, rank, world, device, w, cfg, counts, peaks, peak_kind, flush):
+    """Timed region: the K steps enqueued through the three-stream schedule in one call; per-stage
+    launch times from events recorded on each stage's own stream."""
+    import routed_sparse_attention_chunk_b200 as msa
+    stream = torch.cuda.current_stream()
+    link = host_link_gbs(device) if args.bank_kv == "host" else None
+    sampler = ClockSampler(device)
+    w.pipelined_steps(args.warmup)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    sampler.start()
+    n0 = msa.kernel_launch_count()
+    marks = []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    w.pipelined_steps(args.steps, marks)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = msa.kernel_launch_count() - n0
+    clocks = sampler.stop()
+    timed_ms = t0.elapsed_time(t1)
+    flag = int(w.flag.item())
+    barrier(world, device)
+    ms_per_step = max_over_ranks(timed_ms, world, device) / args.steps
+    tokens_per_step = cfg.B * cfg.Tq * world
+    value = tokens_per_step / (ms_per_step / 1e3)
+    stage_ms = {}
+    for stage, e0, e1 in marks:
+        stage_ms.setdefault(stage, []).append(e0.elapsed_time(e1))
+    per_launch = {st: float(np.mean(v)) for st, v in stage_ms.items()}
+    totals = {st: float(np.sum(v)) for st, v in stage_ms.items()}
+    dom = max(totals, key=totals.get)
+    long_region = timed_ms > 2000.0
+    if dom == "gather" and link is not None:
+        esz = 4 if cfg.dtype == "f32" else 2
+        rows = int(w.pipe.ml[(w.pipe.n - 1) % 2].sum())  # rows the last batch selected (every batch alike)
+        by = 2 * rows * cfg.Hkv * cfg.d * esz  # K̄ and V̄ rows crossing the host link
+        roofline = {"bound": "host_link", "achieved": by / per_launch[dom] / 1e6, "peak": round(link, 1),
+                    "unit": "GB/s", "kernel": "gather_kernel (msa_gather, K̄ / V̄ in page-locked host memory)",
+                    "alg_bytes_per_launch": by,
+                    "peak_source": "measured in this run: page-locked host to device copy, 256 MiB, best of 5"}
+    else:
+        roofline = stage_roofline(dom, per_launch[dom], cfg, counts, peaks, peak_kind, long_region)
+    roofline["achieved"] = round(roofline["achieved"], 2)
+    roofline["frac"] = round(roofline["achieved"] / roofline["peak"], 4)
+    roofline["avg_launch_ms"] = round(per_launch[dom], 4)
+    roofline["traffic"] = None
+    stages = {st: {"ms_per_launch": round(per_launch[st], 4),
+                   "busy_per_step": round(totals[st] / args.steps / ms_per_step, 4)} for st in per_launch}
+
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t.detach().cpu().pin_memory() for t in w.input_tensors()]
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in w.output_tensors()]
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+        dev_in, dev_out = w.input_tensors(), w.output_tensors()
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+        barrier(world, device)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            for d, h in zip(dev_in, host_in):
+                d.copy_(h, non_blocking=True)
+            w.pipelined_steps(1)
+            for h, d in zip(host_out, dev_out):
+                h.copy_(d, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / n_e2e
+        e2e = {"value": round(tokens_per_step / (e2e_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "steps": n_e2e,
+               "note": "inputs copied in and outputs read back every step, so steps do not overlap"}
+    route_ms = per_launch.get("route_topk")
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded generators; see workloads/synth.py)",
+        "config": {"workload": workload_label(cfg),
+                   "step": step_label("query") + "; three-stream schedule: route of batch i+1, gather of batch i "
+                   "and attention of batch i-1 overlap",
+                   **({"bank_kv": "pinned host memory, read in place by msa_gather"} if args.bank_kv == "host" else {}),
+                   "l2": "inputs larger than L2" if flush is None else "L2 not flushed: steps overlap by design",
+                   "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+        "route_scan_gbs": round(counts["route_bytes"] / (route_ms / 1e3) / 1e9, 1) if route_ms else None,
+        "roofline": roofline,
+        "stages": stages,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "err_flag": flag,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_budget, with_pool=False)
     if world > 1:
         import torch.distributed as dist
         barrier(world, device)
@@ -693,6 +839,8 @@ def main():
                     help="backward: time the backward of the query path instead of the forward step")
     ap.add_argument("--bank-kv", choices=["device", "host"], default="device",
                     help="where the pooled K̄ / V̄ live (host: page-locked host memory, the query path only)")
+    ap.add_argument("--pipeline", action="store_true",
+                    help="query path through the three-stream schedule (route i+1 | gather i | attention i-1)")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)
     args = ap.parse_args()

@@ -33,6 +33,15 @@ bool device_readable(const void* p) {
   if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return true;
   return at.type == cudaMemoryTypeHost && at.devicePointer == p;
 }
+// Page-locked host memory the device reads in place (the host tier of K̄ / V̄).
+bool host_resident(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeHost;
+}
 inline bool head_dim_ok(int d) { return d == 64 || d == 128; }
 inline bool dtype_ok(msa_dtype dt) { return dt == MSA_F32 || dt == MSA_BF16; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -199,7 +208,8 @@ msa_status msa_gather(msa_dtype dt, const int32_t* topk_idx, int64_t B, int k, c
     return MSA_ERR_INVALID_ARG;
   if (!aligned16(Kbar) || !aligned16(Vbar) || !aligned16(Kmem) || !aligned16(Vmem)) return MSA_ERR_INVALID_ARG;
   if (!device_readable(Kbar) || !device_readable(Vbar)) return MSA_ERR_INVALID_ARG;
-  GatherArgs a{topk_idx, B, k, doc_chunk_off, D, C, Kbar, Vbar, Hkv, d, Mmax, Kmem, Vmem, mem_len, err_flag};
+  GatherArgs a{topk_idx, B, k, doc_chunk_off, D, C, Kbar, Vbar, Hkv, d, Mmax, Kmem, Vmem, mem_len, err_flag,
+               host_resident(Kbar)};
   return cuda_status(launch_gather(dt, a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -324,7 +334,8 @@ msa_status msa_layer_forward(msa_dtype dt, const void* Qr, int Hr, int dr, const
   if (launch_route(dt, ra, s) != cudaSuccess) return MSA_ERR_CUDA;
   TopkArgs ta{w.doc_key, B, D, k, w.cand, w.doc_key + B * D, w.nslice, topk_idx, topk_score, doc_scores};
   if (launch_topk(ta, s) != cudaSuccess) return MSA_ERR_CUDA;
-  GatherArgs ga{topk_idx, B, k, doc_chunk_off, D, C, Kbar, Vbar, Hkv, d, Mmax, Kmem, Vmem, mem_len, err_flag};
+  GatherArgs ga{topk_idx, B, k, doc_chunk_off, D, C, Kbar, Vbar, Hkv, d, Mmax, Kmem, Vmem, mem_len, err_flag,
+                host_resident(Kbar)};
   if (launch_gather(dt, ga, s) != cudaSuccess) return MSA_ERR_CUDA;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d);
   AttnArgs a{Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, Kmem, Vmem, mem_len, Mmax, scale, O, lse,

@@ -8,6 +8,8 @@
 // Every index is checked before it is used: a document outside [0, D) or a
 // chunk range outside [0, C) is skipped and raises MSA_FLAG_INDEX_OOB; rows that
 // do not fit in Mmax are dropped and raise MSA_FLAG_OVERFLOW.  Nothing traps.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,45 +35,71 @@ __device__ __forceinline__ Sel selected(const int32_t* __restrict__ idx, const i
   return {cs, ce - cs};
 }
 
-// grid (k, B): one CTA copies one selected document
-__global__ void gather_kernel(GatherArgs a, int row_vecs) {
-  const int64_t b = blockIdx.y;
-  const int r = blockIdx.x;
-  bool bad = false;
-  int64_t start = 0;
-  for (int q = 0; q < r; ++q) start += selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, a.k, q, &bad).n;
-  bool mine_bad = false;
-  const Sel me = selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, a.k, r, &mine_bad);
-  if (threadIdx.x == 0) {
-    if (mine_bad) raise_flag(a.err_flag, MSA_FLAG_INDEX_OOB);
+// One item per selected document (b, r).  Device banks: grid B * k, one item
+// per CTA.  Host banks: a few CTAs loop over the items with 8 loads of 16
+// bytes in flight per thread; that keeps the host link busy (it needs about
+// 100 KB in flight) while leaving the SMs to the routing and attention of
+// neighbouring batches, which would otherwise wait behind CTAs that spend
+// their time on host-link latency.
+constexpr int kHostCtas = 16;
+
+template <int kUnroll>  // 16-byte loads in flight per thread and tensor
+__global__ void __launch_bounds__(256) gather_kernel(GatherArgs a, int row_vecs) {
+  const int64_t items = a.B * a.k;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const int64_t b = item / a.k;
+    const int r = (int)(item - b * a.k);
+    bool bad = false;
+    int64_t start = 0;
+    for (int q = 0; q < r; ++q) start += selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, a.k, q, &bad).n;
+    bool mine_bad = false;
+    const Sel me = selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, a.k, r, &mine_bad);
+    if (threadIdx.x == 0) {
+      if (mine_bad) raise_flag(a.err_flag, MSA_FLAG_INDEX_OOB);
+      if (r == a.k - 1) {
+        const int64_t total = start + me.n;
+        if (total > a.Mmax) raise_flag(a.err_flag, MSA_FLAG_OVERFLOW);
+        a.mem_len[b] = (int32_t)(total < a.Mmax ? total : a.Mmax);
+      }
+    }
     if (r == a.k - 1) {
-      const int64_t total = start + me.n;
-      if (total > a.Mmax) raise_flag(a.err_flag, MSA_FLAG_OVERFLOW);
-      a.mem_len[b] = (int32_t)(total < a.Mmax ? total : a.Mmax);
+      // rows past the selection are zeroed: the attention kernels mask them, but a
+      // masked weight of 0 times a non-finite value would still be NaN
+      const int64_t total = min(start + me.n, (int64_t)a.Mmax);
+      uint4* Kz = reinterpret_cast<uint4*>(a.Kmem) + (b * a.Mmax + total) * row_vecs;
+      uint4* Vz = reinterpret_cast<uint4*>(a.Vmem) + (b * a.Mmax + total) * row_vecs;
+      const int64_t nz = ((int64_t)a.Mmax - total) * row_vecs;
+      for (int64_t i = threadIdx.x; i < nz; i += blockDim.x) {
+        Kz[i] = make_uint4(0u, 0u, 0u, 0u);
+        Vz[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
-  }
-  if (r == a.k - 1) {
-    // rows past the selection are zeroed: the attention kernels mask them, but a
-    // masked weight of 0 times a non-finite value would still be NaN
-    const int64_t total = min(start + me.n, (int64_t)a.Mmax);
-    uint4* Kz = reinterpret_cast<uint4*>(a.Kmem) + (b * a.Mmax + total) * row_vecs;
-    uint4* Vz = reinterpret_cast<uint4*>(a.Vmem) + (b * a.Mmax + total) * row_vecs;
-    const int64_t nz = ((int64_t)a.Mmax - total) * row_vecs;
-    for (int64_t i = threadIdx.x; i < nz; i += blockDim.x) {
-      Kz[i] = make_uint4(0u, 0u, 0u, 0u);
-      Vz[i] = make_uint4(0u, 0u, 0u, 0u);
+    const int64_t n = min(me.n, max((int64_t)0, (int64_t)a.Mmax - start));
+    if (n <= 0) continue;
+    const uint4* Ks = reinterpret_cast<const uint4*>(a.Kbar) + me.cs * row_vecs;
+    const uint4* Vs = reinterpret_cast<const uint4*>(a.Vbar) + me.cs * row_vecs;
+    uint4* Kd = reinterpret_cast<uint4*>(a.Kmem) + (b * a.Mmax + start) * row_vecs;
+    uint4* Vd = reinterpret_cast<uint4*>(a.Vmem) + (b * a.Mmax + start) * row_vecs;
+    const int64_t nv = n * row_vecs;
+    for (int64_t i0 = threadIdx.x; i0 < nv; i0 += (int64_t)blockDim.x * kUnroll) {
+      uint4 kb[kUnroll], vb[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = i0 + (int64_t)u * blockDim.x;
+        if (i < nv) {
+          kb[u] = __ldg(Ks + i);
+          vb[u] = __ldg(Vs + i);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = i0 + (int64_t)u * blockDim.x;
+        if (i < nv) {
+          Kd[i] = kb[u];
+          Vd[i] = vb[u];
+        }
+      }
     }
-  }
-  const int64_t n = min(me.n, max((int64_t)0, (int64_t)a.Mmax - start));
-  if (n <= 0) return;
-  const uint4* Ks = reinterpret_cast<const uint4*>(a.Kbar) + me.cs * row_vecs;
-  const uint4* Vs = reinterpret_cast<const uint4*>(a.Vbar) + me.cs * row_vecs;
-  uint4* Kd = reinterpret_cast<uint4*>(a.Kmem) + (b * a.Mmax + start) * row_vecs;
-  uint4* Vd = reinterpret_cast<uint4*>(a.Vmem) + (b * a.Mmax + start) * row_vecs;
-  const int64_t nv = n * row_vecs;
-  for (int64_t i = threadIdx.x; i < nv; i += blockDim.x) {
-    Kd[i] = __ldg(Ks + i);
-    Vd[i] = __ldg(Vs + i);
   }
 }
 
@@ -81,8 +109,13 @@ cudaError_t launch_gather(msa_dtype dt, const GatherArgs& a, cudaStream_t s) {
   if (a.B <= 0) return cudaSuccess;
   const int esz = dt == MSA_F32 ? 4 : 2;
   const int row_vecs = a.Hkv * a.d * esz / 16;
+  const int64_t items = a.B * a.k;
+  const unsigned grid = (unsigned)(a.host_src ? std::min<int64_t>(items, kHostCtas) : items);
   count_launch();
-  gather_kernel<<<dim3(a.k, (unsigned)a.B), 256, 0, s>>>(a, row_vecs);
+  if (a.host_src)
+    gather_kernel<8><<<grid, 256, 0, s>>>(a, row_vecs);
+  else
+    gather_kernel<2><<<grid, 256, 0, s>>>(a, row_vecs);
   return cudaGetLastError();
 }
 

@@ -152,6 +152,7 @@ struct GatherArgs {
   void *Kmem, *Vmem;
   int32_t* mem_len;
   int32_t* err_flag;
+  bool host_src;  // Kbar / Vbar in page-locked host memory: few CTAs, many loads in flight each
 };
 cudaError_t launch_gather(msa_dtype dt, const GatherArgs& a, cudaStream_t s);
 

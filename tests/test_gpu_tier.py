@@ -104,3 +104,43 @@ def test_pageable_host_bank_is_refused_before_any_launch():
                                 ml.data_ptr(), None, None)
     assert st == -1                      # MSA_ERR_INVALID_ARG, nothing launched
     torch.cuda.synchronize()
+
+
+def test_pipelined_host_tier_equals_sequential_calls():
+    """The three-stream schedule (route of batch i+1, host gather of batch i and attention of
+    batch i-1 overlapped) gives the outputs of the sequential calls, bit for bit, for a run of
+    distinct batches, also when the caller reuses two topk_idx tensors in turn."""
+    from routed_sparse_attention_chunk_b200.pipeline import QueryPipeline
+    cfg = synth.get_config("decode16m").scaled(D=200, B=5, Lloc=256, docs_per_slab=0)
+    q, Kb, Vb, Krb, coff, rn = _bank(cfg)
+    coff_d = torch.from_numpy(coff).to(DEV)
+    batches = [synth.gen_query(cfg, 0, DEV, seed) for seed in range(6)]
+    ref = []
+    for bt in batches:
+        idx, _, _, _ = route_on_gpu(bt["Qr"], Krb, rn, coff, cfg.k)
+        Km, Vm, ml, _ = _gather(idx, coff, Kb, Vb, cfg)
+        O_ = torch.empty_like(bt["Q"])
+        ws = torch.empty(max(256, msa.sparse_attn_workspace_size(cfg.B, cfg.Tq, cfg.Lloc, cfg.Hq, cfg.Hkv, cfg.d,
+                                                                 cfg.Mmax)), dtype=torch.uint8, device=DEV)
+        msa.sparse_attn(bt["Q"], bt["Kloc"], bt["Vloc"], Km, Vm, ml, O_, ws=ws)
+        torch.cuda.synchronize()
+        ref.append((idx.clone(), O_))
+    Kh, Vh = Kb.cpu().pin_memory(), Vb.cpu().pin_memory()
+    bank = dict(Krbar=Krb, kr_rnorm=rn, doc_chunk_off=coff_d, Kbar=Kh, Vbar=Vh)
+    for reuse in (False, True):
+        pipe = QueryPipeline(bank, cfg.k, cfg.Mmax, cfg.B, cfg.Tq, cfg.Lloc, cfg.Hq, cfg.Hkv, cfg.d, cfg.Hr,
+                             Kb.dtype, DEV)
+        ring = [torch.empty((cfg.B, cfg.k), dtype=torch.int32, device=DEV) for _ in range(2)]
+        runs = [dict(bt, O=torch.empty_like(bt["Q"]),
+                     topk_idx=ring[i % 2] if reuse else torch.empty((cfg.B, cfg.k), dtype=torch.int32, device=DEV))
+                for i, bt in enumerate(batches)]
+        marks = []
+        pipe.run(runs[:2], marks)
+        pipe.run(runs[2:], marks)         # the event rings continue across calls
+        torch.cuda.synchronize()
+        assert pipe.flag.item() == 0
+        assert len(marks) == 3 * len(runs)
+        for i, (r, (idx, O_)) in enumerate(zip(runs, ref)):
+            assert torch.equal(r["O"], O_), f"batch {i} (reuse={reuse})"
+            if not reuse:
+                assert torch.equal(r["topk_idx"], idx)
