@@ -21,7 +21,10 @@
 //     the latency of a TMA tile;
 //   * the running max is only moved (and O rescaled in TMEM) when it grows by
 //     more than 2^8, so most tiles skip the rescale; the final 1/l and the
-//     log-sum-exp use the same max, which keeps the result exact.
+//     log-sum-exp use the same max, which keeps the result exact;
+//   * the softmax warps are the critical path (one warp per SM sub-partition,
+//     bound by instruction issue): the row max runs as eight independent
+//     chains, and the scaled arguments and row sums use packed f32x2 math.
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warps 2..5 softmax / correction / output (one row per thread).
 // Every wait is bounded and ends the CTA with MSA_FLAG_TIMEOUT on expiry.
@@ -66,6 +69,26 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction for two values).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
 template <int DH>
@@ -258,17 +281,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const bool memt = j < NM;
       const int base = memt ? j * kKeys : (j - NM) * kKeys;
       const int lim = memt ? M - base : pos - base + 1;
-      float mx = -INFINITY;
-      if (__all_sync(0xffffffffu, lim >= kKeys)) {
+      const bool whole = __all_sync(0xffffffffu, lim >= kKeys);
+      if (!whole) {
 #pragma unroll
-        for (int c = 0; c < kKeys; ++c) mx = fmaxf(mx, s[c]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < kKeys; ++c) {
-          s[c] = c < lim ? s[c] : -INFINITY;
-          mx = fmaxf(mx, s[c]);
-        }
+        for (int c = 0; c < kKeys; ++c) s[c] = c < lim ? s[c] : -INFINITY;
       }
+      // eight independent chains (max is exact in any order)
+      float m8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < kKeys; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       // move the max (and rescale O) only when it grows by more than 2^8
       const float mt = mx * sl2;
       const bool first = m_run == -INFINITY;
@@ -300,20 +325,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
       l_run *= corr;
       const float nm = -m_run;
-      // P_j over S_j: 32 keys (16 columns of bf16 pairs) per store
-      float lsa[4] = {0.f, 0.f, 0.f, 0.f};
+      // P_j over S_j: 32 keys (16 columns of bf16 pairs) per store; the scaled arguments and the row
+      // sums in packed pairs (one f32x2 instruction for two keys)
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), nmx2 = f2_pack(nm, nm);
+      uint64_t lsa2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
       for (int c0 = 0; c0 < kKeys; c0 += 32) {
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float e0 = fast_exp2(fmaf(s[c0 + 2 * i], sl2, nm));
-          const float e1 = fast_exp2(fmaf(s[c0 + 2 * i + 1], sl2, nm));
-          lsa[i & 3] += e0 + e1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[c0 + 2 * i], s[c0 + 2 * i + 1]), sl2x2, nmx2), x0, x1);
+          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+          lsa2[i & 1] = f2_add(lsa2[i & 1], f2_pack(e0, e1));
           w[i] = pack_bf16x2(e0, e1);
         }
         tmem_st16(tmem + lane_off + st * kKeys + c0 / 2, w);
       }
+      float lsa[4];
+      f2_unpack(lsa2[0], lsa[0], lsa[1]);
+      f2_unpack(lsa2[1], lsa[2], lsa[3]);
       l_run += (lsa[0] + lsa[1]) + (lsa[2] + lsa[3]);
       tmem_st_wait();
       tc_fence_before();
