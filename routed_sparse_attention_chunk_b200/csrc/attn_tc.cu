@@ -23,8 +23,10 @@
 //     more than 2^8, so most tiles skip the rescale; the final 1/l and the
 //     log-sum-exp use the same max, which keeps the result exact;
 //   * the softmax warps are the critical path (one warp per SM sub-partition,
-//     bound by instruction issue): the row max runs as eight independent
-//     chains, and the scaled arguments and row sums use packed f32x2 math.
+//     bound by instruction issue; the two that share a sub-partition with the
+//     TMA and MMA warps finish last): the row max runs as eight independent
+//     chains of three-input maxima, the scaled arguments and row sums use
+//     packed f32x2 math, and the MMA warp reuses its operand descriptors.
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warps 2..5 softmax / correction / output (one row per thread).
 // Every wait is bounded and ends the CTA with MSA_FLAG_TIMEOUT on expiry.
@@ -84,6 +86,12 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
+}
+// max of three (exact, like any max; no NaN reaches it)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
@@ -212,19 +220,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(kRows, kKeys);
       constexpr uint32_t idO = idesc_bf16_f32(kRows, DH, /*b_mn_major=*/true);
-      const uint32_t q0 = smem_u32(Qs);
+      // descriptors of the operand bases; a k-step adds its byte offset / 16 to
+      // the 14-bit start-address field (shared addresses stay below 256 KB, so
+      // the field never carries)
+      const uint64_t dq = desc_k_sw128(smem_u32(Qs));
+      const uint64_t dk0 = desc_k_sw128(smem_u32(Ks)), dv0 = desc_mn_sw128(smem_u32(Vs), kKeys * 128);
       // S_j goes to TMEM buffer j & 1, which holds P_{j-2} until PV_{j-2} has
       // read it; PV_{j-2} was issued earlier, and the MMAs run in issue order.
       auto issue_S = [&](int j) -> bool {
         const int ks = j % kKV;
         if (!mbar_wait(&k_full[ks], (j / kKV) & 1, kWaitPolls)) return false;
         tc_fence_after();
-        const uint32_t k0 = smem_u32(Ks + ks * L::kK);
+        const uint64_t dk = dk0 + (uint64_t)((ks * L::kK) >> 4);
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
           const int box = k >> 2, kk = k & 3;
-          mma_bf16_ss(tS0 + (j & 1) * kKeys, desc_k_sw128(q0 + box * kRows * 128 + kk * 32),
-                      desc_k_sw128(k0 + box * kKeys * 128 + kk * 32), idS, k > 0 ? 1u : 0u);
+          mma_bf16_ss(tS0 + (j & 1) * kKeys, dq + (uint64_t)((box * kRows * 128 + kk * 32) >> 4),
+                      dk + (uint64_t)((box * kKeys * 128 + kk * 32) >> 4), idS, k > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[j & 1]);
         mma_commit(&k_empty[ks]);
@@ -242,11 +254,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           break;
         }
         tc_fence_after();
-        const uint32_t v0 = smem_u32(Vs + vs * L::kK);
+        const uint64_t dv = dv0 + (uint64_t)((vs * L::kK) >> 4);
         // A = P_j from TMEM: 16 keys of bf16 per step are 8 columns
 #pragma unroll
         for (int k = 0; k < kKeys / 16; ++k)
-          mma_bf16_ts(tO, tS0 + st * kKeys + k * 8, desc_mn_sw128(v0 + k * 16 * 128, kKeys * 128), idO,
+          mma_bf16_ts(tO, tS0 + st * kKeys + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idO,
                       (j > 0 || k > 0) ? 1u : 0u);
         mma_commit(&p_free[st]);
         mma_commit(&v_empty[vs]);
@@ -286,14 +298,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int c = 0; c < kKeys; ++c) s[c] = c < lim ? s[c] : -INFINITY;
       }
-      // eight independent chains (max is exact in any order)
+      // eight independent chains of three-input maxima (max is exact in any order)
+      static_assert(kKeys == 128, "the chains cover 128 keys");
       float m8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m8[i] = s[i];
+      for (int i = 0; i < 8; ++i) m8[i] = fmax3(s[i], s[i + 8], s[i + 16]);
 #pragma unroll
-      for (int c = 8; c < kKeys; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      for (int c = 24; c < 120; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[120 + i]);
+      const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
       // move the max (and rescale O) only when it grows by more than 2^8
       const float mt = mx * sl2;
       const bool first = m_run == -INFINITY;

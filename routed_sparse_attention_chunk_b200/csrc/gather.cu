@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tma_host.h"
 
 namespace msa {
 namespace {
@@ -36,11 +37,13 @@ __device__ __forceinline__ Sel selected(const int32_t* __restrict__ idx, const i
 }
 
 // One item per selected document (b, r).  Device banks: grid B * k, one item
-// per CTA.  Host banks: a few CTAs loop over the items with 8 loads of 16
-// bytes in flight per thread; that keeps the host link busy (it needs about
-// 100 KB in flight) while leaving the SMs to the routing and attention of
-// neighbouring batches, which would otherwise wait behind CTAs that spend
-// their time on host-link latency.
+// per CTA, with 8 loads of 16 bytes in flight per thread when there are fewer
+// than two CTAs per SM (a single query's k documents: the copy is latency-bound)
+// and 2 otherwise.  Host banks: a few CTAs loop over the items with 8 loads in
+// flight per thread; that keeps the host link busy (it needs about 100 KB in
+// flight) while leaving the SMs to the routing and attention of neighbouring
+// batches, which would otherwise wait behind CTAs that spend their time on
+// host-link latency.
 constexpr int kHostCtas = 16;
 
 template <int kUnroll>  // 16-byte loads in flight per thread and tensor
@@ -112,7 +115,7 @@ cudaError_t launch_gather(msa_dtype dt, const GatherArgs& a, cudaStream_t s) {
   const int64_t items = a.B * a.k;
   const unsigned grid = (unsigned)(a.host_src ? std::min<int64_t>(items, kHostCtas) : items);
   count_launch();
-  if (a.host_src)
+  if (a.host_src || items < 2 * (int64_t)sm_count())
     gather_kernel<8><<<grid, 256, 0, s>>>(a, row_vecs);
   else
     gather_kernel<2><<<grid, 256, 0, s>>>(a, row_vecs);
