@@ -133,6 +133,9 @@ def _bank_case(C_docs, Hr, dr, seed):
     (3, 3, 8, 128, 17000, 33),    # smallest k of the block-level top-k, three slices
     (2, 5, 2, 64, 9000, 1),       # k = 1 over two slices
     (1, 4, 2, 64, 20, 20),        # fewer documents than a warp, k = D
+    (1, 512, 8, 128, 9000, 16),   # ~40K chunks, 4 blocks of 128 query rows
+    (2, 300, 1, 128, 9000, 16),   # blocks that span two queries, ragged last block
+    (1, 600, 2, 64, 9000, 16),    # dr = 64, ragged last block
 ])
 def test_route_topk_bf16(B, Tq, Hr, dr, D, k):
     Krb, rn, coff = _bank_case(D, Hr, dr, seed=B * 1000 + Tq)
