@@ -15,9 +15,13 @@
 // lane: a key of S^T and a dimension of O^T.  Column (row) maxima are reduced
 // across the 128 lanes with shuffles and shared memory; the running max moves
 // only when it grows by more than 2^8 (then O^T is rescaled in TMEM).
-// Persistent CTAs (one per SM) walk work units = (batch row, KV head, key
-// split); each unit leaves (max, sum, unnormalised O) per row in the workspace
-// and a second kernel merges the splits.
+// One CTA per SM streams an equal, contiguous share of all (batch row, KV
+// head, key tile) triples; each stretch of that share inside one (batch row,
+// KV head) is a segment, which leaves (max, sum, unnormalised O) per row in the
+// workspace, and a second kernel merges the segments.  The softmax threads
+// handle only the R real query rows (rounded up to 4, 8 or 16), and load the
+// next segment's Q rows while the current one streams, into the other of two
+// Q buffers.
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warps 2..5 softmax / output.  Every wait is bounded; after the first
 // expired wait the CTA stops waiting, runs its loops out without data and
@@ -44,25 +48,43 @@ struct DecParams {
   const __nv_bfloat16* Q;
   const int32_t* mem_len;
   int32_t* err_flag;
-  float* part;  // [units][R][kDH + 2]: m, l, O
+  float* part;  // [B * Hkv][Smax][R][kDH + 2]: m, l, O of one segment
   int64_t B;
   int Tq, Lloc, Hq, Hkv, Mmax, G, R;
   int NM;       // memory tiles (ceil(Mmax / kKeys)); rows past mem_len are masked
   int NL;       // local tiles (ceil(Lloc / kKeys))
-  int S, tps;   // splits per (b, g) and tiles per split
-  int64_t units;
+  int T;        // tiles per (b, g): NM + NL
+  int Smax;     // partial slots per (b, g)
+  int64_t Ttot, per;  // all tiles (B * Hkv * T) and tiles per CTA
   float scale_log2;
 };
 
 struct DLayout {
   static constexpr int kTile = kKeys * kDH * 2;       // one K (or V) tile, two 64-wide boxes
   static constexpr int kStage = 2 * kTile;
-  static constexpr int kQ = kMaxRows * kDH * 2;       // Q rows, K-major, 128-byte swizzle
+  static constexpr int kQ = kMaxRows * kDH * 2;       // Q rows, K-major, 128-byte swizzle (two buffers)
   static constexpr int kP = kMaxRows * kKeys * 2;     // P^T rows (query rows x keys)
-  static constexpr int kRed = 3 * kMaxRows * 4 * 4;    // [2 tile parities + unit end][rows][4 warps]
-  static constexpr int kSmem = 1024 + kStages * kStage + kQ + kP + kRed + 8 * 16 + 16;
+  static constexpr int kRed = 3 * kMaxRows * 4 * 4;    // [2 tile parities + segment end][rows][4 warps]
+  static constexpr int kSmem = 1024 + kStages * kStage + 2 * kQ + kP + kRed + 8 * 16 + 16;
   static constexpr uint32_t kTmemCols = 64;           // S0, S1, O (16 columns each)
 };
+
+// One CTA's share of the work is the contiguous range [f0, f1) of the flattened
+// tile index f = (b * Hkv + g) * T + t, so every CTA streams the same number of
+// tiles; a segment is the part of that range that lies in one (b, g).  The
+// segment's partial result goes to slot (CTA - first CTA touching (b, g)).
+struct Seg {
+  int64_t bg;
+  int t0, t1, slot;
+};
+__device__ __forceinline__ Seg seg_at(const DecParams& p, int64_t f, int64_t f1) {
+  Seg s;
+  s.bg = f / p.T;
+  s.t0 = (int)(f - s.bg * p.T);
+  s.t1 = (int)min((int64_t)p.T, (int64_t)s.t0 + (f1 - f));
+  s.slot = (int)((int64_t)blockIdx.x - (s.bg * p.T) / p.per);
+  return s;
+}
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -85,14 +107,17 @@ __device__ __forceinline__ int sw128_off(int row, int col, int rows) {
   return box * (rows * 128) + row * 128 + ((((c >> 3) ^ (row & 7))) << 4) + (c & 7) * 2;
 }
 
+// kR >= R is the number of query rows the softmax threads handle (4, 8 or 16);
+// the MMA's N stays 16 and the columns past kR are never read.
+template <int kR>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_constant__ CUtensorMap tmVm,
                    const __grid_constant__ CUtensorMap tmKl, const __grid_constant__ CUtensorMap tmVl, DecParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint8_t* Qs = ring + kStages * DLayout::kStage;
-  uint8_t* Ps = Qs + DLayout::kQ;
+  uint8_t* Qs = ring + kStages * DLayout::kStage;  // two buffers, alternating by segment
+  uint8_t* Ps = Qs + 2 * DLayout::kQ;
   float* red_s = reinterpret_cast<float*>(Ps + DLayout::kP);  // [3][16 rows][4 warps]
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red_s) + DLayout::kRed);
   uint64_t* kv_full = bars;            // [3]
@@ -107,6 +132,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
   volatile int* abort_s = reinterpret_cast<volatile int*>(bars + 15);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t f0 = (int64_t)blockIdx.x * p.per, f1 = min(f0 + p.per, p.Ttot);
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&kv_full[i], 1);
@@ -137,13 +163,11 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int64_t u = blockIdx.x; u < p.units && !*abort_s; u += gridDim.x) {
-        const int s = (int)(u % p.S);
-        const int64_t bg = u / p.S;
-        const int g = (int)(bg % p.Hkv);
-        const int64_t b = bg / p.Hkv;
-        const int t_end = min((s + 1) * p.tps, p.NM + p.NL);
-        for (int t = s * p.tps; t < t_end; ++t, ++it) {
+      for (int64_t f = f0; f < f1 && !*abort_s;) {
+        const Seg sg = seg_at(p, f, f1);
+        const int g = (int)(sg.bg % p.Hkv);
+        const int64_t b = sg.bg / p.Hkv;
+        for (int t = sg.t0; t < sg.t1; ++t, ++it) {
           const uint32_t st = it % kStages, round = it / kStages;
           if (!mbar_wait(&kv_empty[st], (round & 1) ^ 1, kWaitPolls)) {
             *abort_s = 1;
@@ -161,6 +185,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
             tma_load_2d(Vd + dc * (kKeys * 128), mv, g * kDH + dc * 64, y, &kv_full[st]);
           }
         }
+        f += sg.t1 - sg.t0;
       }
       const uint32_t fills = it;
       for (uint32_t st = 0; st < (uint32_t)kStages && st < fills; ++st) {
@@ -173,14 +198,13 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(kKeys, kMaxRows);                              // K x Q^T
       constexpr uint32_t idO = idesc_bf16_f32(kDH, kMaxRows, /*b_mn=*/false, /*a_mn=*/true);  // V^T x P^T
-      const uint32_t q0 = smem_u32(Qs), p0 = smem_u32(Ps);
-      uint32_t it = 0, js = 0;  // it: K/V tiles; js: S buffers used
-      int64_t nunit = 0;
-      for (int64_t u = blockIdx.x; u < p.units; u += gridDim.x, ++nunit) {
-        const int s = (int)(u % p.S);
-        const int t0 = s * p.tps, t_end = min((s + 1) * p.tps, p.NM + p.NL);
-        const int T = t_end - t0;
-        if (!*abort_s && !mbar_wait(q_ready, (uint32_t)(nunit & 1), kWaitPolls)) *abort_s = 1;
+      const uint32_t p0 = smem_u32(Ps);
+      uint32_t it = 0, js = 0, nseg = 0;  // it: K/V tiles; js: S buffers used; nseg: segments
+      for (int64_t f = f0; f < f1; ++nseg) {
+        const Seg sg = seg_at(p, f, f1);
+        const int T = sg.t1 - sg.t0;
+        const uint32_t q0 = smem_u32(Qs + (nseg & 1) * DLayout::kQ);
+        if (!*abort_s && !mbar_wait(q_ready, nseg & 1, kWaitPolls)) *abort_s = 1;
         auto issue_S = [&](int j) {
           const uint32_t st = (it + j) % kStages, round = (it + j) / kStages;
           const uint32_t sb = (js + j) & 1, use = (js + j) >> 1;
@@ -197,7 +221,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
           }
           mma_commit(&s_full[sb]);
         };
-        if (T > 0) issue_S(0);
+        issue_S(0);
         for (int j = 0; j < T; ++j) {
           if (j + 1 < T) issue_S(j + 1);
           const uint32_t st = (it + j) % kStages;
@@ -215,6 +239,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
         }
         it += T;
         js += T;
+        f += T;
       }
       mma_commit(drain);
       if (!mbar_wait(drain, 0, kWaitPolls)) *abort_s = 1;
@@ -225,35 +250,60 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
     const int r_lane = q * 32 + lane;               // this thread's TMEM lane: key of S^T, dim of O^T
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const int et = tid - 64;                        // 0..127
-    uint32_t it = 0, js = 0;
-    for (int64_t u = blockIdx.x; u < p.units; u += gridDim.x) {
-      const int s = (int)(u % p.S);
-      const int64_t bg = u / p.S;
-      const int g = (int)(bg % p.Hkv);
-      const int64_t b = bg / p.Hkv;
-      const int t0 = s * p.tps, t_end = min((s + 1) * p.tps, p.NM + p.NL);
-      const int T = t_end - t0;
-      int M = __ldg(p.mem_len + b);
-      if (M < 0 || M > p.Mmax) {
-        if (et == 0 && s == 0 && g == 0) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
-        M = M < 0 ? 0 : p.Mmax;
-      }
-      // Q rows into the swizzled K-major tile (rows past R are zero): row r = token r / G, head g*G + r % G
-      for (int i = et; i < kMaxRows * (kDH / 8); i += 128) {
-        const int r = i / (kDH / 8), c8 = (i % (kDH / 8)) * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
+    // Q rows of a segment into a swizzled K-major buffer: element i of R * 16
+    // 16-byte pieces is row r = i / 16 (token r / G, head g * G + r % G).
+    auto load_q = [&](const Seg& sg, uint4 (&v)[2]) {
+      const int g = (int)(sg.bg % p.Hkv);
+      const int64_t b = sg.bg / p.Hkv;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int i = et + 128 * k, r = i >> 4, c8 = (i & 15) * 8;
+        v[k] = make_uint4(0, 0, 0, 0);
         if (r < p.R) {
           const int t = r / p.G, h = g * p.G + r % p.G;
-          v = __ldg(reinterpret_cast<const uint4*>(p.Q + ((b * p.Tq + t) * p.Hq + h) * (int64_t)kDH + c8));
+          v[k] = __ldg(reinterpret_cast<const uint4*>(p.Q + ((b * p.Tq + t) * p.Hq + h) * (int64_t)kDH + c8));
         }
-        *reinterpret_cast<uint4*>(Qs + sw128_off(r, c8, kMaxRows)) = v;
       }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(q_ready);
-      float m_run[kMaxRows], l_run[kMaxRows];
+    };
+    auto store_q = [&](uint8_t* buf, const uint4 (&v)[2]) {
 #pragma unroll
-      for (int r = 0; r < kMaxRows; ++r) {
+      for (int k = 0; k < 2; ++k) {
+        const int i = et + 128 * k, r = i >> 4, c8 = (i & 15) * 8;
+        if (r < p.R) *reinterpret_cast<uint4*>(buf + sw128_off(r, c8, kMaxRows)) = v[k];
+      }
+    };
+    // rows past R stay zero in both buffers; segment 0's rows go to buffer 0
+    for (int i = et; i < 2 * kMaxRows * (kDH / 8); i += 128) {
+      const int bsel = i / (kMaxRows * (kDH / 8)), r = (i >> 4) % kMaxRows, c8 = (i & 15) * 8;
+      if (r >= p.R) *reinterpret_cast<uint4*>(Qs + bsel * DLayout::kQ + sw128_off(r, c8, kMaxRows)) = make_uint4(0, 0, 0, 0);
+    }
+    {
+      uint4 v[2];
+      load_q(seg_at(p, f0, f1), v);
+      store_q(Qs, v);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    mbar_arrive(q_ready);
+
+    uint32_t it = 0, js = 0, nseg = 0;
+    for (int64_t f = f0; f < f1; ++nseg) {
+      const Seg sg = seg_at(p, f, f1);
+      const int64_t b = sg.bg / p.Hkv;
+      const int t0 = sg.t0;
+      const int T = sg.t1 - sg.t0;
+      const int64_t fn = f + T;
+      // the next segment's Q rows, loaded now and stored after this segment's first tile
+      uint4 qn[2];
+      if (fn < f1) load_q(seg_at(p, fn, f1), qn);
+      int M = __ldg(p.mem_len + b);
+      if (M < 0 || M > p.Mmax) {
+        if (et == 0 && sg.t0 == 0 && sg.bg % p.Hkv == 0) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
+        M = M < 0 ? 0 : p.Mmax;
+      }
+      float m_run[kR], l_run[kR];
+#pragma unroll
+      for (int r = 0; r < kR; ++r) {
         m_run[r] = -INFINITY;
         l_run[r] = 0.f;
       }
@@ -262,8 +312,8 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
         const uint32_t sb = (js + j) & 1, use = (js + j) >> 1;
         if (!*abort_s && !__all_sync(0xffffffffu, mbar_wait(&s_full[sb], use & 1, kWaitPolls))) *abort_s = 1;
         tc_fence_after();
-        float sc[kMaxRows];
-        tmem_ld16(tS + sb * 16 + lane_off, sc);
+        float sc[kR];
+        tmem_ld_cols<kR>(tS + sb * 16 + lane_off, sc);
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&s_free[sb]);
@@ -271,7 +321,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
         const bool mem = t < p.NM;
         const int key = (mem ? t : t - p.NM) * kKeys + r_lane;
 #pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) {
+        for (int r = 0; r < kR; ++r) {
           const bool vis = r < p.R && (mem ? key < M : key <= p.Lloc - p.Tq + r / p.G);
           sc[r] = vis ? sc[r] * p.scale_log2 : -INFINITY;
         }
@@ -281,18 +331,18 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
         // suffices (a buffer is rewritten two tiles later, after every thread
         // has passed the barrier of the tile in between).
         float* red = red_s + ((it + j) & 1) * (kMaxRows * 4);
-        float mine = -INFINITY;  // lane r < 16 keeps this warp's maximum of column r
+        float mine = -INFINITY;  // lane r < kR keeps this warp's maximum of column r
 #pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) {
+        for (int r = 0; r < kR; ++r) {
           const float v = warp_max(sc[r]);
           mine = lane == r ? v : mine;
         }
-        if (lane < kMaxRows) red[lane * 4 + q] = mine;
+        if (lane < kR) red[lane * 4 + q] = mine;
         bar_softmax();
         bool grow = false;
-        float corr[kMaxRows];
+        float corr[kR];
 #pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) {
+        for (int r = 0; r < kR; ++r) {
           const float4 w = *reinterpret_cast<const float4*>(red + r * 4);
           const float mt = fmaxf(fmaxf(w.x, w.y), fmaxf(w.z, w.w));
           corr[r] = 1.f;
@@ -302,9 +352,9 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
             grow = true;
           }
         }
-        float pr[kMaxRows];
+        float pr[kR];
 #pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) {
+        for (int r = 0; r < kR; ++r) {
           pr[r] = sc[r] == -INFINITY ? 0.f : fast_exp2(sc[r] - m_run[r]);
           l_run[r] = l_run[r] * corr[r] + pr[r];
         }
@@ -313,44 +363,47 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
           *abort_s = 1;
         if (j > 0 && grow) {
           tc_fence_after();
-          float o[16];
-          tmem_ld16(tO + lane_off, o);
+          float o[kR];
+          tmem_ld_cols<kR>(tO + lane_off, o);
           tmem_ld_wait();
-          uint32_t w[16];
+          uint32_t w[kR];
 #pragma unroll
-          for (int r = 0; r < 16; ++r) w[r] = __float_as_uint(o[r] * corr[r]);
-          tmem_st16(tO + lane_off, w);
+          for (int r = 0; r < kR; ++r) w[r] = __float_as_uint(o[r] * corr[r]);
+          tmem_st_cols<kR>(tO + lane_off, w);
           tmem_st_wait();
         }
 #pragma unroll
-        for (int r = 0; r < kMaxRows; ++r)
+        for (int r = 0; r < kR; ++r)
           *reinterpret_cast<__nv_bfloat16*>(Ps + sw128_off(r, r_lane, kMaxRows)) = __float2bfloat16_rn(pr[r]);
+        // The other Q buffer was last read by the previous segment's S MMAs,
+        // all complete before that segment's last o_done.
+        if (j == 0 && fn < f1) store_q(Qs + ((nseg + 1) & 1) * DLayout::kQ, qn);
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(p_full);
+        if (j == 0 && fn < f1) mbar_arrive(q_ready);
       }
-      // unit result: O^T[d = r_lane][row], the row maxima and the summed weights
-      if (T > 0 && !*abort_s && !__all_sync(0xffffffffu, mbar_wait(o_done, (it + T - 1) & 1, kWaitPolls)))
-        *abort_s = 1;
+      // segment result: O^T[d = r_lane][row], the row maxima and the summed weights
+      if (!*abort_s && !__all_sync(0xffffffffu, mbar_wait(o_done, (it + T - 1) & 1, kWaitPolls))) *abort_s = 1;
       tc_fence_after();
-      float o[16];
-      tmem_ld16(tO + lane_off, o);
+      float o[kR];
+      tmem_ld_cols<kR>(tO + lane_off, o);
       tmem_ld_wait();
-      float* out = p.part + (size_t)u * p.R * (kDH + 2);
-      float* red_l = red_s + 2 * (kMaxRows * 4);  // the unit's row sums, apart from the tile buffers
+      float* out = p.part + (size_t)(sg.bg * p.Smax + sg.slot) * p.R * (kDH + 2);
+      float* red_l = red_s + 2 * (kMaxRows * 4);  // the segment's row sums, apart from the tile buffers
 #pragma unroll
-      for (int r = 0; r < kMaxRows; ++r) {
+      for (int r = 0; r < kR; ++r) {
         float v = l_run[r];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
         if (lane == 0) red_l[r * 4 + q] = v;
-        if (r < p.R) out[r * (kDH + 2) + 2 + r_lane] = T > 0 ? o[r] : 0.f;
+        if (r < p.R) out[r * (kDH + 2) + 2 + r_lane] = o[r];
       }
       bar_softmax();
       if (et < p.R) {
         float m = -INFINITY;
 #pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) m = r == et ? m_run[r] : m;
+        for (int r = 0; r < kR; ++r) m = r == et ? m_run[r] : m;
         out[et * (kDH + 2)] = m;
         out[et * (kDH + 2) + 1] = red_l[et * 4] + red_l[et * 4 + 1] + red_l[et * 4 + 2] + red_l[et * 4 + 3];
       }
@@ -358,6 +411,7 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
       tc_fence_before();
       it += T;
       js += T;
+      f = fn;
     }
   }
   tc_fence_before();
@@ -369,18 +423,21 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
   if (tid == 0 && *abort_s) raise_flag(p.err_flag, MSA_FLAG_TIMEOUT);
 }
 
-// Merge the S splits of every (b, g) row: O = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
+// Merge the segments of every (b, g) row: O = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
+// The segments of (b, g) are those of the CTAs whose tile ranges meet its tiles.
 __global__ void decode_combine_kernel(DecParams p, __nv_bfloat16* __restrict__ O, float* __restrict__ lse) {
   const int64_t bg = blockIdx.x;  // one CTA per (b, g), one warp per row
   const int g = (int)(bg % p.Hkv);
   const int64_t b = bg / p.Hkv;
   const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (r >= p.R) return;
+  const int ns = (int)((bg * p.T + p.T - 1) / p.per - (bg * p.T) / p.per + 1);
+  const float* base = p.part + (size_t)bg * p.Smax * p.R * (kDH + 2);
   float m = -INFINITY;
-  for (int s = 0; s < p.S; ++s) m = fmaxf(m, p.part[((bg * p.S + s) * p.R + r) * (kDH + 2)]);
+  for (int s = 0; s < ns; ++s) m = fmaxf(m, base[((size_t)s * p.R + r) * (kDH + 2)]);
   float l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < p.S; ++s) {
-    const float* src = p.part + ((bg * p.S + s) * p.R + r) * (kDH + 2);
+  for (int s = 0; s < ns; ++s) {
+    const float* src = base + ((size_t)s * p.R + r) * (kDH + 2);
     const float ms = src[0];
     const float w = ms == -INFINITY ? 0.f : fast_exp2(ms - m);
     l += w * src[1];
@@ -395,8 +452,8 @@ __global__ void decode_combine_kernel(DecParams p, __nv_bfloat16* __restrict__ O
 }
 
 struct DecodePlan {
-  int R, NM, NL, S, tps;
-  int64_t units;
+  int R, NM, NL, T, Smax;
+  int64_t bgs, Ttot, per, grid;
 };
 
 DecodePlan plan(const AttnArgs& a) {
@@ -404,14 +461,17 @@ DecodePlan plan(const AttnArgs& a) {
   d.R = (a.Hq / a.Hkv) * a.Tq;
   d.NM = (a.Mmax + kKeys - 1) / kKeys;
   d.NL = (a.Lloc + kKeys - 1) / kKeys;
-  const int T = d.NM + d.NL;
-  const int64_t bg = a.B * a.Hkv;
-  // enough equal units for ~8 per SM, each at least one tile; every split holds tps tiles
-  int S = (int)((8LL * sm_count() + bg - 1) / bg);
-  S = S < 1 ? 1 : (S > T ? T : S);
-  d.tps = (T + S - 1) / S;
-  d.S = (T + d.tps - 1) / d.tps;
-  d.units = bg * d.S;
+  d.T = d.NM + d.NL;
+  d.bgs = a.B * a.Hkv;
+  d.Ttot = d.bgs * d.T;
+  if (d.Ttot <= 0) return d;
+  // one CTA per SM, each streaming an equal contiguous share of all tiles
+  const int64_t g0 = d.Ttot < sm_count() ? d.Ttot : sm_count();
+  d.per = (d.Ttot + g0 - 1) / g0;
+  d.grid = (d.Ttot + d.per - 1) / d.per;
+  // a (b, g) of T tiles meets at most (T - 1) / per + 2 consecutive ranges
+  int64_t smax = (d.T - 1) / d.per + 2;
+  d.Smax = (int)(smax < d.grid ? smax : d.grid);
   return d;
 }
 
@@ -432,12 +492,13 @@ size_t decode_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int M
   a.Hkv = Hkv;
   a.Mmax = Mmax;
   const DecodePlan d = plan(a);
-  return sizeof(float) * (size_t)d.units * d.R * (kDH + 2);
+  return sizeof(float) * (size_t)d.bgs * d.Smax * d.R * (kDH + 2);
 }
 
 cudaError_t launch_attn_decode(const AttnArgs& a, cudaStream_t s) {
   const DecodePlan d = plan(a);
-  const size_t need = sizeof(float) * (size_t)d.units * d.R * (kDH + 2);
+  if (d.Ttot <= 0) return cudaSuccess;
+  const size_t need = sizeof(float) * (size_t)d.bgs * d.Smax * d.R * (kDH + 2);
   if (!a.ws || a.ws_bytes < need) return cudaErrorInvalidValue;
   CUtensorMap tkm, tvm, tkl, tvl;
   const uint64_t rowkv = (uint64_t)a.Hkv * kDH * 2;
@@ -465,15 +526,16 @@ cudaError_t launch_attn_decode(const AttnArgs& a, cudaStream_t s) {
   p.R = d.R;
   p.NM = d.NM;
   p.NL = d.NL;
-  p.S = d.S;
-  p.tps = d.tps;
-  p.units = d.units;
+  p.T = d.T;
+  p.Smax = d.Smax;
+  p.Ttot = d.Ttot;
+  p.per = d.per;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DLayout::kSmem);
+  auto kern = d.R <= 4 ? attn_decode_kernel<4> : (d.R <= 8 ? attn_decode_kernel<8> : attn_decode_kernel<16>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DLayout::kSmem);
   if (e != cudaSuccess) return e;
-  const int64_t grid = d.units < sm_count() ? d.units : sm_count();
   count_launch();
-  attn_decode_kernel<<<(unsigned)grid, kThreads, DLayout::kSmem, s>>>(tkm, tvm, tkl, tvl, p);
+  kern<<<(unsigned)d.grid, kThreads, DLayout::kSmem, s>>>(tkm, tvm, tkl, tvl, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   count_launch();
   decode_combine_kernel<<<(unsigned)(a.B * a.Hkv), 32 * d.R, 0, s>>>(p, reinterpret_cast<__nv_bfloat16*>(a.O), a.lse);
