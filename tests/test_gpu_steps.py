@@ -136,6 +136,11 @@ def _bank_case(C_docs, Hr, dr, seed):
     (1, 512, 8, 128, 9000, 16),   # ~40K chunks, 4 blocks of 128 query rows
     (2, 300, 1, 128, 9000, 16),   # blocks that span two queries, ragged last block
     (1, 600, 2, 64, 9000, 16),    # dr = 64, ragged last block
+    # CTA-pair scan (blocks of 256 rows inside one query)
+    (3, 512, 8, 128, 1500, 16),   # several queries, Tq a multiple of 256
+    (1, 4096, 8, 128, 300, 16),   # the 16-layer workload's query length: 16 row blocks
+    (1, 256, 3, 128, 1001, 7),    # one row block, three router heads
+    (1, 300, 8, 128, 20, 4),      # under 128 chunks: the pair's second CTA holds none
 ])
 def test_route_topk_bf16(B, Tq, Hr, dr, D, k):
     Krb, rn, coff = _bank_case(D, Hr, dr, seed=B * 1000 + Tq)
