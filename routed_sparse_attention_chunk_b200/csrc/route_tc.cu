@@ -385,11 +385,6 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
 
 template <int DR>
 struct PairLayout {
@@ -416,14 +411,15 @@ constexpr int kPairThreads = 384;
 constexpr uint32_t kRegsControl = 40, kRegsEpilogue = 232;
 constexpr uint32_t kPairRegsNeeded = 128 * kRegsControl + 256 * kRegsEpilogue;
 
-// Item at position L of the work order: (tile pair, row block).
-__device__ __forceinline__ void pair_item(int64_t L, const RouteTcParams& p, int& tile, int& rb) {
-  const int64_t per_group = (int64_t)kGroup * p.n_rb;
-  const int g = (int)(L / per_group);
-  const int w = (int)(L - (int64_t)g * per_group);
-  const int tg = min(kGroup, p.n_tiles - g * kGroup);
-  rb = w / tg;
-  tile = g * kGroup + (w - rb * tg);
+// Item at position L of the work order: (tile pair, row block).  The host
+// keeps the item count below 2^31, so 32-bit arithmetic suffices.
+__device__ __forceinline__ void pair_item(uint32_t L, const RouteTcParams& p, int& tile, int& rb) {
+  const uint32_t per_group = (uint32_t)kGroup * (uint32_t)p.n_rb;
+  const uint32_t g = L / per_group;
+  const uint32_t w = L - g * per_group;
+  const uint32_t tg = (uint32_t)min(kGroup, p.n_tiles - (int)g * kGroup);
+  rb = (int)(w / tg);
+  tile = (int)(g * kGroup + (w - (uint32_t)rb * tg));
 }
 
 template <int DR>
@@ -589,9 +585,9 @@ route_tc_pair_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       const bool cvalid = cn < p.C;
       const int doc = cvalid ? __ldg(p.chunk_doc + cn) : -1;
       const float* rkp = p.kr_rnorm + (cvalid ? cn : 0) * Hr;
-      uint64_t S2[NH / 2];  // running sums of column pairs (packed fp32)
+      float S_[NH];
 #pragma unroll
-      for (int j = 0; j < NH / 2; ++j) S2[j] = 0;
+      for (int j = 0; j < NH; ++j) S_[j] = 0.f;
       for (int h = 0; h < Hr; ++h, ++it) {
         const uint32_t buf = it & 1, use = it >> 1;
         const float rk = cvalid ? __ldg(rkp + h) : 0.f;  // issued before the wait, used after it
@@ -615,9 +611,14 @@ route_tc_pair_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
 #pragma unroll
           for (int j4 = 0; j4 < 64; j4 += 4) {
             const float4 w = *reinterpret_cast<const float4*>(rqh + j0 + j4);
-            const int i2 = (j0 + j4) / 2;
-            S2[i2] = f2_fma(f2_mul(f2_pack(v[j4], v[j4 + 1]), rk2), f2_pack(w.x, w.y), S2[i2]);
-            S2[i2 + 1] = f2_fma(f2_mul(f2_pack(v[j4 + 2], v[j4 + 3]), rk2), f2_pack(w.z, w.w), S2[i2 + 1]);
+            // rk * rq for four columns in two packed multiplies, then one fma per column
+            float k0, k1, k2, k3;
+            f2_unpack(f2_mul(f2_pack(w.x, w.y), rk2), k0, k1);
+            f2_unpack(f2_mul(f2_pack(w.z, w.w), rk2), k2, k3);
+            S_[j0 + j4] = fmaf(v[j4], k0, S_[j0 + j4]);
+            S_[j0 + j4 + 1] = fmaf(v[j4 + 1], k1, S_[j0 + j4 + 1]);
+            S_[j0 + j4 + 2] = fmaf(v[j4 + 2], k2, S_[j0 + j4 + 2]);
+            S_[j0 + j4 + 3] = fmaf(v[j4 + 3], k3, S_[j0 + j4 + 3]);
           }
         }
         tc_fence_before();
@@ -627,12 +628,16 @@ route_tc_pair_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
       if (timed_out) break;
       if (nvalid == 0) continue;
       float m = -INFINITY;
+      if (nvalid == NH) {  // the usual case: a tree of maxima over all columns
 #pragma unroll
-      for (int j = 0; j < NH / 2; ++j) {
-        float x0, x1;
-        f2_unpack(S2[j], x0, x1);
-        if (2 * j < nvalid) m = fmaxf(m, x0);
-        if (2 * j + 1 < nvalid) m = fmaxf(m, x1);
+        for (int w = NH / 2; w >= 1; w /= 2)
+#pragma unroll
+          for (int j = 0; j < w; ++j) S_[j] = fmaxf(S_[j], S_[j + w]);
+        m = S_[0];
+      } else {
+#pragma unroll
+        for (int j = 0; j < NH; ++j)
+          if (j < nvalid) m = fmaxf(m, S_[j]);
       }
       doc_max_atomic(m * invHr, doc, lane, p.doc_key + (int64_t)(r0 / p.Tq) * p.D);
     }
@@ -667,6 +672,7 @@ cudaError_t launch_pair_t(const RouteArgs& a, cudaStream_t s) {
   p.n_rb = (rows + L::kN - 1) / L::kN;
   p.items = (int64_t)p.n_tiles * p.n_rb;
   if (p.items == 0) return cudaGetLastError();
+  if (p.items > 0x7fffffffLL) return launch_t<DR, 128>(a, s);  // the work order is 32-bit
   auto kern = route_tc_pair_kernel<DR>;
   // The register split may only hand out what the launch allocated; a build
   // that gives the kernel fewer registers per thread takes the one-CTA scan.
