@@ -12,9 +12,10 @@
 // with bulk asynchronous copies (cp.async.bulk, completion counted on an
 // mbarrier), running ahead across chunk boundaries; a small per-stage record
 // tells the consumers which chunk the stage belongs to.  The consumer
-// threads each own one 16-byte column vector of the token row (a K vector of
-// the first half together with its RoPE partner in the second half, or one V /
-// Kr vector), sum it over the chunk's tokens in fp32 from shared memory (the
+// threads each own one column vector of the token row (8 bytes of K from the
+// first half of a head together with their RoPE partners in the second half,
+// or one 16-byte V / Kr vector), sum it over the chunk's tokens in fp32 from
+// shared memory (the
 // stage also carries the RoPE (cos, sin) rows of its token positions), and at
 // the chunk's end store the mean rounded to the storage type.  The Kr threads
 // also reduce the squared norm of the stored (rounded) values per head with
@@ -44,6 +45,26 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
+}
+
+// 8-byte vectors: the RoPE threads each own half a 16-byte vector of the low
+// and of the high half of a head, so that four warps (one per SM sub-partition)
+// share the rotation arithmetic, which sets the pace of a stage's consumers.
+__device__ __forceinline__ void unpack8(const uint2& u, float (&f)[2]) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+}
+__device__ __forceinline__ void unpack8(const uint2& u, float (&f)[4]) {
+  f[0] = __uint_as_float(u.x << 16);  // bf16 -> fp32 is exact
+  f[1] = __uint_as_float(u.x & 0xffff0000u);
+  f[2] = __uint_as_float(u.y << 16);
+  f[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+__device__ __forceinline__ uint2 pack8(const float (&f)[2]) {
+  return make_uint2(__float_as_uint(f[0]), __float_as_uint(f[1]));
+}
+__device__ __forceinline__ uint2 pack8(const float (&f)[4]) {
+  return make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
 }
 
 // What the consumers need to know about one stage of the ring.
@@ -144,9 +165,10 @@ __global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
     }
   } else if (warp <= nconsumer_warps) {
     // ---------------------------------------------------------------- consumers
+    constexpr int KN = VN / 2;          // elements of each half a RoPE thread owns
     const int item = threadIdx.x - 32;  // [0, nR) Kr, [nR, nR+nK) K pairs, then V; >= W idle
     const int kind = item < g.nR ? 0 : (item < g.nR + g.nK ? 1 : (item < g.W ? 2 : 3));
-    const int halfv = a.d / 2 / VN;
+    const int halfv = a.d / 2 / KN;
     int off_lo = 0, off_hi = 0, region = 0, h = 0, i0 = 0;
     if (kind == 0) {
       region = 2 * g.TOK * g.rowK;
@@ -154,7 +176,7 @@ __global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
     } else if (kind == 1) {
       const int w = item - g.nR;
       h = w / halfv;
-      i0 = (w - h * halfv) * VN;
+      i0 = (w - h * halfv) * KN;
       off_lo = (h * a.d + i0) * (int)sizeof(T);
       off_hi = off_lo + (a.d / 2) * (int)sizeof(T);
     } else if (kind == 2) {
@@ -185,17 +207,17 @@ __global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
         const uint8_t* rope = ring + (size_t)st * g.stage + (size_t)g.TOK * (2 * g.rowK + g.rowR) + i0 * 8;
 #pragma unroll 4
         for (int u = 0; u < nt; ++u) {
-          float xl[VN], xh[VN];
-          unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_lo), xl);
-          unpack(*reinterpret_cast<const uint4*>(base + u * rstride + off_hi), xh);
+          float xl[KN], xh[KN];
+          unpack8(*reinterpret_cast<const uint2*>(base + u * rstride + off_lo), xl);
+          unpack8(*reinterpret_cast<const uint2*>(base + u * rstride + off_hi), xh);
           const float4* cs4 = reinterpret_cast<const float4*>(rope + u * g.rowP);
 #pragma unroll
-          for (int q = 0; q < VN / 2; ++q) {
+          for (int q = 0; q < KN / 2; ++q) {
             const float4 w = cs4[q];  // (cos, sin) of pairs i0+2q and i0+2q+1
             acc[2 * q] += xl[2 * q] * w.x - xh[2 * q] * w.y;
-            acc[VN + 2 * q] += xh[2 * q] * w.x + xl[2 * q] * w.y;
+            acc[KN + 2 * q] += xh[2 * q] * w.x + xl[2 * q] * w.y;
             acc[2 * q + 1] += xl[2 * q + 1] * w.z - xh[2 * q + 1] * w.w;
-            acc[VN + 2 * q + 1] += xh[2 * q + 1] * w.z + xl[2 * q + 1] * w.w;
+            acc[KN + 2 * q + 1] += xh[2 * q + 1] * w.z + xl[2 * q + 1] * w.w;
           }
         }
       } else if (kind != 3) {
@@ -224,12 +246,13 @@ __global__ void __launch_bounds__(512, 1) pool_kernel(PoolArgs a, PoolGeom g) {
         for (int i = 0; i < VN; ++i) ss += m[i] * m[i];
       } else if (kind == 1) {
         uint8_t* dst = reinterpret_cast<uint8_t*>(a.Kbar) + c * g.rowK;
+        float mk[KN];
 #pragma unroll
-        for (int i = 0; i < VN; ++i) m[i] = acc[i] / fn;
-        *reinterpret_cast<uint4*>(dst + off_lo) = pack(m);
+        for (int i = 0; i < KN; ++i) mk[i] = acc[i] / fn;
+        *reinterpret_cast<uint2*>(dst + off_lo) = pack8(mk);
 #pragma unroll
-        for (int i = 0; i < VN; ++i) m[i] = acc[VN + i] / fn;
-        *reinterpret_cast<uint4*>(dst + off_hi) = pack(m);
+        for (int i = 0; i < KN; ++i) mk[i] = acc[KN + i] / fn;
+        *reinterpret_cast<uint2*>(dst + off_hi) = pack8(mk);
       } else if (kind == 2) {
 #pragma unroll
         for (int i = 0; i < VN; ++i) m[i] = acc[i] / fn;
@@ -267,7 +290,7 @@ template <typename T>
 cudaError_t pool_t(const PoolArgs& a, cudaStream_t s) {
   constexpr int VN = Vec<T>::N;
   PoolGeom g;
-  g.nK = a.Hkv * (a.d / 2) / VN;
+  g.nK = a.Hkv * (a.d / 2) / (VN / 2);
   g.nV = a.Hkv * a.d / VN;
   g.nR = a.Hr * a.dr / VN;
   g.W = g.nK + g.nV + g.nR;
