@@ -10,8 +10,10 @@
 // rows of one KV head are its N = 16:
 //   S^T[key, row] = K_tile (TMA, 128-byte swizzle) x Q^T        (tcgen05.mma)
 //   O^T[d, row]  += V_tile^T (MN-major, straight from the tile) x P^T
-// with S^T double-buffered in TMEM so the tensor core computes the next tile
-// while the softmax warps work on this one.  Each softmax thread owns one TMEM
+// with S^T double-buffered in TMEM and P^T in shared memory, so the tensor
+// core computes the next tile while the softmax warps work on this one; the
+// MMA thread polls its barriers without blocking and issues each tile's S and
+// P V as soon as their inputs are ready.  Each softmax thread owns one TMEM
 // lane: a key of S^T and a dimension of O^T.  Column (row) maxima are reduced
 // across the 128 lanes with shuffles and shared memory; the running max moves
 // only when it grows by more than 2^8 (then O^T is rescaled in TMEM).
@@ -42,6 +44,7 @@ constexpr int kMaxRows = 16;            // R = G * Tq (the MMA's N, padded to 16
 constexpr int kStages = 3;
 constexpr int kThreads = 192;
 constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr uint32_t kSpinLimit = 1u << 28;  // non-blocking polls of the MMA issuer without progress
 constexpr float kRescaleLog2 = 8.0f;
 
 struct DecParams {
@@ -63,9 +66,9 @@ struct DLayout {
   static constexpr int kTile = kKeys * kDH * 2;       // one K (or V) tile, two 64-wide boxes
   static constexpr int kStage = 2 * kTile;
   static constexpr int kQ = kMaxRows * kDH * 2;       // Q rows, K-major, 128-byte swizzle (two buffers)
-  static constexpr int kP = kMaxRows * kKeys * 2;     // P^T rows (query rows x keys)
+  static constexpr int kP = kMaxRows * kKeys * 2;     // P^T rows (query rows x keys); two buffers
   static constexpr int kRed = 3 * kMaxRows * 4 * 4;    // [2 tile parities + segment end][rows][4 warps]
-  static constexpr int kSmem = 1024 + kStages * kStage + 2 * kQ + kP + kRed + 8 * 16 + 16;
+  static constexpr int kSmem = 1024 + kStages * kStage + 2 * kQ + 2 * kP + kRed + 8 * 18 + 16;
   static constexpr uint32_t kTmemCols = 64;           // S0, S1, O (16 columns each)
 };
 
@@ -118,18 +121,18 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
   uint8_t* ring = smem;
   uint8_t* Qs = ring + kStages * DLayout::kStage;  // two buffers, alternating by segment
   uint8_t* Ps = Qs + 2 * DLayout::kQ;
-  float* red_s = reinterpret_cast<float*>(Ps + DLayout::kP);  // [3][16 rows][4 warps]
+  float* red_s = reinterpret_cast<float*>(Ps + 2 * DLayout::kP);  // [3][16 rows][4 warps]
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red_s) + DLayout::kRed);
   uint64_t* kv_full = bars;            // [3]
   uint64_t* kv_empty = bars + 3;       // [3]
   uint64_t* s_full = bars + 6;         // [2]
   uint64_t* s_free = bars + 8;         // [2]
   uint64_t* q_ready = bars + 10;
-  uint64_t* p_full = bars + 11;
-  uint64_t* o_done = bars + 12;
-  uint64_t* drain = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
-  volatile int* abort_s = reinterpret_cast<volatile int*>(bars + 15);
+  uint64_t* p_full = bars + 11;        // [2] per P buffer
+  uint64_t* o_done = bars + 13;        // [2] per P buffer: its P V has completed
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_s = reinterpret_cast<volatile int*>(bars + 17);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t f0 = (int64_t)blockIdx.x * p.per, f1 = min(f0 + p.per, p.Ttot);
@@ -143,8 +146,10 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
       mbar_init(&s_free[i], 128);
     }
     mbar_init(q_ready, 128);
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_done[i], 1);
+    }
     mbar_init(drain, 1);
     *abort_s = 0;
     fence_mbar_init();
@@ -205,37 +210,52 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
         const int T = sg.t1 - sg.t0;
         const uint32_t q0 = smem_u32(Qs + (nseg & 1) * DLayout::kQ);
         if (!*abort_s && !mbar_wait(q_ready, nseg & 1, kWaitPolls)) *abort_s = 1;
-        auto issue_S = [&](int j) {
-          const uint32_t st = (it + j) % kStages, round = (it + j) / kStages;
-          const uint32_t sb = (js + j) & 1, use = (js + j) >> 1;
-          if (!*abort_s && (!mbar_wait(&kv_full[st], round & 1, kWaitPolls) ||
-                            !mbar_wait(&s_free[sb], (use & 1) ^ 1, kWaitPolls)))
-            *abort_s = 1;
-          tc_fence_after();
-          const uint32_t k0 = smem_u32(ring + st * DLayout::kStage);
+        // Issue S = K Q^T of a tile as soon as its K/V stage and an S buffer are
+        // ready, and O += V^T P^T of a tile as soon as its P is: one thread polls
+        // both (test_wait does not block), so a tile's P V is never held back by
+        // the next tile's copy.  Tile g = it + j (over the CTA's whole range)
+        // uses P buffer g & 1, phase g >> 1.
+        int nS = 0, nP = 0;
+        uint32_t spins = 0;
+        while (nP < T && !*abort_s) {
+          bool prog = false;
+          if (nS < T) {
+            const uint32_t g = it + nS, st = g % kStages, round = g / kStages;
+            const uint32_t sb = (js + nS) & 1, use = (js + nS) >> 1;
+            if (mbar_test(&kv_full[st], round & 1) && mbar_test(&s_free[sb], (use & 1) ^ 1)) {
+              tc_fence_after();
+              const uint32_t k0 = smem_u32(ring + st * DLayout::kStage);
 #pragma unroll
-          for (int k = 0; k < kDH / 16; ++k) {
-            const int box = k >> 2, kk = k & 3;
-            mma_bf16_ss(tS + sb * 16, desc_k_sw128(k0 + box * (kKeys * 128) + kk * 32),
-                        desc_k_sw128(q0 + box * (kMaxRows * 128) + kk * 32), idS, k > 0 ? 1u : 0u);
+              for (int k = 0; k < kDH / 16; ++k) {
+                const int box = k >> 2, kk = k & 3;
+                mma_bf16_ss(tS + sb * 16, desc_k_sw128(k0 + box * (kKeys * 128) + kk * 32),
+                            desc_k_sw128(q0 + box * (kMaxRows * 128) + kk * 32), idS, k > 0 ? 1u : 0u);
+              }
+              mma_commit(&s_full[sb]);
+              ++nS;
+              prog = true;
+            }
           }
-          mma_commit(&s_full[sb]);
-        };
-        issue_S(0);
-        for (int j = 0; j < T; ++j) {
-          if (j + 1 < T) issue_S(j + 1);
-          const uint32_t st = (it + j) % kStages;
-          if (!*abort_s && !mbar_wait(p_full, (uint32_t)((it + j) & 1), kWaitPolls)) *abort_s = 1;
-          tc_fence_after();
-          const uint32_t v0 = smem_u32(ring + st * DLayout::kStage + DLayout::kTile);
+          if (nP < nS) {
+            const uint32_t g = it + nP, st = g % kStages, pb = g & 1;
+            if (mbar_test(&p_full[pb], (g >> 1) & 1)) {
+              tc_fence_after();
+              const uint32_t v0 = smem_u32(ring + st * DLayout::kStage + DLayout::kTile);
+              const uint32_t pp = p0 + pb * DLayout::kP;
 #pragma unroll
-          for (int k = 0; k < kKeys / 16; ++k) {
-            const int box = k >> 2, kk = k & 3;
-            mma_bf16_ss(tO, desc_mn_sw128(v0 + k * 16 * 128, kKeys * 128),
-                        desc_k_sw128(p0 + box * (kMaxRows * 128) + kk * 32), idO, (j > 0 || k > 0) ? 1u : 0u);
+              for (int k = 0; k < kKeys / 16; ++k) {
+                const int box = k >> 2, kk = k & 3;
+                mma_bf16_ss(tO, desc_mn_sw128(v0 + k * 16 * 128, kKeys * 128),
+                            desc_k_sw128(pp + box * (kMaxRows * 128) + kk * 32), idO, (nP > 0 || k > 0) ? 1u : 0u);
+              }
+              mma_commit(&o_done[pb]);
+              mma_commit(&kv_empty[st]);
+              ++nP;
+              prog = true;
+            }
           }
-          mma_commit(o_done);
-          mma_commit(&kv_empty[st]);
+          if (prog) spins = 0;
+          else if (++spins > kSpinLimit) *abort_s = 1;
         }
         it += T;
         js += T;
@@ -358,8 +378,14 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
           pr[r] = sc[r] == -INFINITY ? 0.f : fast_exp2(sc[r] - m_run[r]);
           l_run[r] = l_run[r] * corr[r] + pr[r];
         }
-        // P V of the previous tile must be done before P is overwritten or O rescaled
-        if (j > 0 && !*abort_s && !__all_sync(0xffffffffu, mbar_wait(o_done, (it + j - 1) & 1, kWaitPolls)))
+        // P buffer g & 1 was last read by the P V of tile g - 2; O is rescaled
+        // only after the P V of tile g - 1
+        const uint32_t g = it + j;
+        if (g >= 2 && !*abort_s &&
+            !__all_sync(0xffffffffu, mbar_wait(&o_done[g & 1], ((g - 2) >> 1) & 1, kWaitPolls)))
+          *abort_s = 1;
+        if (j > 0 && grow && !*abort_s &&
+            !__all_sync(0xffffffffu, mbar_wait(&o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, kWaitPolls)))
           *abort_s = 1;
         if (j > 0 && grow) {
           tc_fence_after();
@@ -374,17 +400,22 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
         }
 #pragma unroll
         for (int r = 0; r < kR; ++r)
-          *reinterpret_cast<__nv_bfloat16*>(Ps + sw128_off(r, r_lane, kMaxRows)) = __float2bfloat16_rn(pr[r]);
+          *reinterpret_cast<__nv_bfloat16*>(Ps + (g & 1) * DLayout::kP + sw128_off(r, r_lane, kMaxRows)) =
+              __float2bfloat16_rn(pr[r]);
         // The other Q buffer was last read by the previous segment's S MMAs,
-        // all complete before that segment's last o_done.
+        // all complete before that segment's last P V.
         if (j == 0 && fn < f1) store_q(Qs + ((nseg + 1) & 1) * DLayout::kQ, qn);
         fence_async_smem();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(&p_full[g & 1]);
         if (j == 0 && fn < f1) mbar_arrive(q_ready);
       }
       // segment result: O^T[d = r_lane][row], the row maxima and the summed weights
-      if (!*abort_s && !__all_sync(0xffffffffu, mbar_wait(o_done, (it + T - 1) & 1, kWaitPolls))) *abort_s = 1;
+      {
+        const uint32_t g = it + T - 1;  // the segment's last tile
+        if (!*abort_s && !__all_sync(0xffffffffu, mbar_wait(&o_done[g & 1], (g >> 1) & 1, kWaitPolls)))
+          *abort_s = 1;
+      }
       tc_fence_after();
       float o[kR];
       tmem_ld_cols<kR>(tO + lane_off, o);
