@@ -46,6 +46,12 @@ the plainest reading and says so at the function (the list of readings):
      selected documents' scores: the max passes it to its argmax (token, chunk),
      first in (chunk, token) order on ties, and the cosine's derivative spreads it
      over that token's Qr and that chunk's K̄r.
+  R16 The linear (DGA) layers' memory injection ("MSA x Qwen3.5" model card,
+     "Architecture summary": the top-k documents' recurrent states are summed
+     into S_ext, the initial state of the query path's gated delta rule) sums
+     each query's selected documents' states elementwise; how a document's state
+     is produced, and the delta rule that consumes S_ext, are defined outside
+     the pages and are not part of this module.
 
 Layouts are row-major with the innermost dimension last:
   K, V [Ntok, Hkv, d]; Kr [Ntok, Hr, dr]; doc_tok_off int64 [D+1]
@@ -286,6 +292,28 @@ def gather(topk_idx, doc_chunk_off, Kbar, Vbar, Mmax: int):
         Km[b, :n], Vm[b, :n] = Kb[rows], Vb[rows]
         mem_len[b] = n
     return Km, Vm, mem_len
+
+
+def state_gather_sum(states, topk_idx):
+    """Reading R16: S_ext[b] = sum over the query's selected documents j of states[j].
+
+    states [D, ...] (one recurrent state per document, any trailing shape),
+    topk_idx int [B, k] -> S_ext [B, ...] in fp64.  Every selected index must lie
+    in [0, D); a document selected twice counts twice.
+    Pins: one selected document gives its state back exactly; one-hot states
+    count how often each document is selected; the sum is invariant under the
+    order of the selection and linear in the states; selecting every document
+    once gives numpy's sum over all documents.
+    """
+    st = np.asarray(states, dtype=np.float64)
+    idx = np.asarray(topk_idx, dtype=np.int64)
+    if idx.size and (idx.min() < 0 or idx.max() >= st.shape[0]):
+        raise ValueError("selected document index out of range")
+    out = np.zeros((idx.shape[0],) + st.shape[1:], dtype=np.float64)
+    for b in range(idx.shape[0]):
+        for j in idx[b]:
+            out[b] += st[j]
+    return out
 
 
 # ----------------------------------------------------------------------------

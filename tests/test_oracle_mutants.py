@@ -53,6 +53,10 @@ MUTANTS = [
      "test_route_backward_matches_central_differences", ()),
     ("route_backward", "sc = s[b, :, a:e].T", "sc = s[b, :, a:e]",
      "test_route_backward_matches_central_differences", ()),
+    ("state_gather_sum", "out[b] += st[j]", "out[b] = st[j]",
+     "test_state_gather_sum_one_hot_states_count_selections", ()),
+    ("state_gather_sum", "for j in idx[b]:", "for j in sorted(set(idx[b].tolist())):",
+     "test_state_gather_sum_one_hot_states_count_selections", ()),
 ]
 
 

@@ -424,3 +424,34 @@ def test_route_backward_matches_central_differences():
         assert np.allclose(gx, num, atol=1e-7, rtol=1e-6), args
     # only the argmax token of each selected document is touched
     assert np.count_nonzero(np.abs(dQ).sum(axis=(2, 3))) <= 2 * 2
+
+
+# ---------------------------------------------------------------- DGA state injection (reading R16)
+def test_state_gather_sum_single_selection_returns_the_state():
+    rng = np.random.default_rng(21)
+    st = rng.standard_normal((7, 2, 3, 4))
+    out = O.state_gather_sum(st, np.array([[5], [0], [6]]))
+    assert np.array_equal(out[0], st[5]) and np.array_equal(out[1], st[0]) and np.array_equal(out[2], st[6])
+
+
+def test_state_gather_sum_one_hot_states_count_selections():
+    D = 6
+    st = np.eye(D).reshape(D, D)                   # document j's state is the unit vector e_j
+    idx = np.array([[3, 1, 3, 5], [0, 0, 0, 2]])     # repeats count twice / three times
+    out = O.state_gather_sum(st, idx)
+    assert np.array_equal(out[0], [0, 1, 0, 2, 0, 1])
+    assert np.array_equal(out[1], [3, 0, 1, 0, 0, 0])
+
+
+def test_state_gather_sum_order_invariant_linear_and_total():
+    rng = np.random.default_rng(22)
+    D = 9
+    st = rng.standard_normal((D, 5, 3))
+    idx = np.array([[4, 2, 7], [1, 8, 0]])
+    a = O.state_gather_sum(st, idx)
+    assert np.allclose(a, O.state_gather_sum(st, idx[:, ::-1]), rtol=0, atol=1e-12)
+    assert np.allclose(O.state_gather_sum(2.5 * st, idx), 2.5 * a, rtol=1e-14, atol=0)
+    every = O.state_gather_sum(st, np.arange(D)[None, :])
+    assert np.allclose(every[0], np.sum(st, axis=0), rtol=1e-14, atol=1e-14)
+    with pytest.raises(ValueError):
+        O.state_gather_sum(st, np.array([[D]]))
