@@ -482,6 +482,81 @@ def run_backward(args, rank, local_rank, world):
     }
 
 
+STATE_SHAPE = (32, 128, 128)  # a linear (DGA) layer's recurrent state: value heads x key dim x value dim
+
+
+def run_state(args, rank, local_rank, world):
+    """The linear (DGA) layers' memory injection: per query, the sum of its k
+    selected documents' recurrent states (msa_state_gather_sum).  The states are a
+    seeded synthetic bank of min(D, 8192) documents (the routing that picks them is
+    timed by the forward pass); each step draws a fresh selection of k distinct
+    documents per query, and L2 is flushed before every launch."""
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    import routed_sparse_attention_chunk_b200 as msa
+    cfg = workload_config(args)
+    dt = cfg.torch_dtype
+    Dst = min(cfg.D, 8192)
+    S = int(np.prod(STATE_SHAPE))
+    g = torch.Generator(device=device).manual_seed(17 + 1000 * rank)
+    states = torch.empty((Dst,) + STATE_SHAPE, dtype=dt, device=device)
+    for i in range(0, Dst, 256):  # in slices, so no fp32 copy of the whole bank exists at once
+        states[i:i + 256] = torch.randn((min(256, Dst - i),) + STATE_SHAPE, generator=g, device=device).to(dt)
+    n_sel = args.warmup + args.steps
+    sel = torch.stack([torch.stack([torch.randperm(Dst, generator=g, device=device)[:cfg.k] for _ in range(cfg.B)])
+                       for _ in range(n_sel)]).to(torch.int32)
+    out = torch.empty((cfg.B,) + STATE_SHAPE, dtype=torch.float32, device=device)
+    flag = torch.zeros(1, dtype=torch.int32, device=device)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)  # 256 MB, twice the L2
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        flush.fill_(1.0)
+        msa.state_gather_sum(states, sel[i], out, err_flag=flag)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    sampler = ClockSampler(device)
+    sampler.start()
+    n0 = msa.kernel_launch_count()
+    ev = []
+    for i in range(args.steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        msa.state_gather_sum(states, sel[args.warmup + i], out, err_flag=flag)
+        e1.record(stream)
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    launches = msa.kernel_launch_count() - n0
+    clocks = sampler.stop()
+    step_sum = sum(e0.elapsed_time(e1) for e0, e1 in ev)
+    barrier(world, device)
+    total_ms = max_over_ranks(step_sum, world, device)
+    ms_per_step = total_ms / args.steps
+    esz = states.element_size()
+    by = cfg.B * cfg.k * S * esz + cfg.B * S * 4  # the selected states read once, one fp32 state written
+    peaks, peak_kind = load_peaks()
+    achieved = by / (step_sum / args.steps) / 1e6
+    value = cfg.B * cfg.Tq * world / (ms_per_step / 1e3)
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype + " states, f32 sums", "data": "synthetic",
+        "config": {"workload": workload_label(cfg),
+                   "step": f"msa_state_gather_sum: per query the sum of {cfg.k} selected documents' recurrent "
+                           f"states of {STATE_SHAPE[0]} x {STATE_SHAPE[1]} x {STATE_SHAPE[2]} from a bank of {Dst}",
+                   "l2": "flushed before every launch", "parallelism": "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "kernel": "state_sum_kernel (msa_state_gather_sum)", "alg_bytes_per_launch": by,
+                     "peak_source": f"{peak_kind} hbm_gbs", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "avg_launch_ms": round(step_sum / args.steps, 4), "traffic": None},
+        "gpu_launches": launches, "clocks": clocks, "err_flag": int(flag.item()),
+    }
+
+
 def run_gpu(args, rank, local_rank, world):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -842,8 +917,9 @@ def main():
     ap.add_argument("--step", choices=["full", "query"], default=None,
                     help="full: pool + query path per step; query: bank pooled before timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which_pass", choices=["forward", "backward"], default="forward",
-                    help="backward: time the backward of the query path instead of the forward step")
+    ap.add_argument("--pass", dest="which_pass", choices=["forward", "backward", "state"], default="forward",
+                    help="backward: time the backward of the query path instead of the forward step; "
+                         "state: the linear layers' memory injection (sum of the selected documents' states)")
     ap.add_argument("--bank-kv", choices=["device", "host"], default="device",
                     help="where the pooled K̄ / V̄ live (host: page-locked host memory, the query path only)")
     ap.add_argument("--pipeline", action="store_true",
@@ -858,6 +934,8 @@ def main():
         res = run_reference(args, rank, world)
     elif args.which_pass == "backward":
         res = run_backward(args, rank, local_rank, world)
+    elif args.which_pass == "state":
+        res = run_state(args, rank, local_rank, world)
     else:
         res = run_gpu(args, rank, local_rank, world)
     if rank == 0 and res is not None:

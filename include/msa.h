@@ -336,6 +336,25 @@ msa_status msa_layer_forward(msa_dtype dt,
                              float* doc_scores,
                              void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Memory injection of the linear (DGA) layers ("MSA x Qwen3.5" model card,
+ * "Architecture summary": the top-k documents' recurrent states are summed
+ * into S_ext, the initial state of the query path's gated delta rule).  For
+ * query b:
+ *   S_ext[b, :] = sum over r < k of states[topk_idx[b, r], :]
+ * summed in fp32 in rank order; a document selected twice counts twice.
+ *   states [D, S] dtype dt (one recurrent state of S elements per document,
+ *   e.g. heads x key dim x value dim);  topk_idx int32 [B, k];  S_ext fp32 [B, S]
+ * S must make a state a whole number of 16-byte vectors (S % 8 == 0 for bf16,
+ * S % 4 == 0 for fp32), else MSA_ERR_UNSUPPORTED; B <= 65535.  How the states
+ * are produced, and the delta rule that consumes S_ext, are not part of this
+ * library.  Device flag: MSA_FLAG_INDEX_OOB for an index outside [0, D); that
+ * selection adds nothing.
+ * ---------------------------------------------------------------------- */
+msa_status msa_state_gather_sum(msa_dtype dt, const void* states, int64_t D, int64_t S,
+                                const int32_t* topk_idx, int64_t B, int k, float* S_ext,
+                                int32_t* err_flag, msa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

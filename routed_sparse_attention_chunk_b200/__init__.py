@@ -136,6 +136,19 @@ def gather(topk_idx, doc_chunk_off, Kbar, Vbar, Kmem, Vmem, mem_len, err_flag=No
           _p(mem_len, torch.int32), _p(err_flag, torch.int32), _s(stream))
 
 
+def state_gather_sum(states, topk_idx, S_ext, err_flag=None, stream=None):
+    """Linear (DGA) layers' memory injection (msa_state_gather_sum): S_ext[b] = sum of
+    the selected documents' recurrent states.  states [D, ...] bf16 or fp32;
+    topk_idx int32 [B, k]; S_ext fp32 [B, ...] with the states' trailing shape."""
+    D = states.shape[0]
+    S = states.numel() // D if D else 0
+    B, k = topk_idx.shape
+    if S_ext.numel() != B * S:
+        raise ValueError("S_ext must hold one state per query")
+    _call("msa_state_gather_sum", _dt(states), _p(states), D, S, _p(topk_idx, torch.int32), B, k,
+          _p(S_ext, torch.float32), _p(err_flag, torch.int32), _s(stream))
+
+
 def sparse_attn_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Mmax) -> int:
     return _lib.load().msa_sparse_attn_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Mmax)
 

@@ -46,6 +46,7 @@ SIGNATURES = {
     "msa_layer_forward": (C.c_int, [C.c_int, P, C.c_int, C.c_int, P, P, P, I64, I64, C.c_int,
                                     P, P, P, I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                     P, P, C.c_int, F32, P, P, P, P, P, P, SZ, P, P]),
+    "msa_state_gather_sum": (C.c_int, [C.c_int, P, I64, I64, P, I64, C.c_int, P, P, P]),
 }
 
 _lib = None

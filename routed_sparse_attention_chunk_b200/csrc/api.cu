@@ -343,4 +343,15 @@ msa_status msa_layer_forward(msa_dtype dt, const void* Qr, int Hr, int dr, const
   return cuda_status(launch_attn(dt, a, s));
 }
 
+msa_status msa_state_gather_sum(msa_dtype dt, const void* states, int64_t D, int64_t S, const int32_t* topk_idx,
+                                int64_t B, int k, float* S_ext, int32_t* err_flag, msa_stream_t stream) {
+  if (!dtype_ok(dt) || D < 1 || S < 1 || B < 0 || k < 1) return MSA_ERR_INVALID_ARG;
+  if (S % (dt == MSA_F32 ? 4 : 8) != 0 || B > 65535) return MSA_ERR_UNSUPPORTED;  // 16-byte vectors
+  if (B == 0) return MSA_OK;
+  if (!states || !topk_idx || !S_ext) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(states) || !aligned16(S_ext) || !device_readable(states)) return MSA_ERR_INVALID_ARG;
+  return cuda_status(launch_state_sum(dt, states, D, S, topk_idx, B, k, S_ext, err_flag,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

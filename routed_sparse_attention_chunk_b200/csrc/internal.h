@@ -63,6 +63,11 @@ struct RouteArgs {
 };
 cudaError_t launch_route(msa_dtype dt, const RouteArgs& a, cudaStream_t s);
 
+// Sum of each query's selected documents' recurrent states (the DGA layers'
+// injected initial state): out[b] = sum_r states[idx[b, r]] in fp32.
+cudaError_t launch_state_sum(msa_dtype dt, const void* states, int64_t D, int64_t S, const int32_t* idx,
+                             int64_t B, int k, float* out, int32_t* err_flag, cudaStream_t s);
+
 // Backward of the sparse attention (gradients in fp32; Drow is a workspace of
 // [B, Hq, Tq] fp32 row dot products of dO and O).
 struct AttnBwdArgs {

@@ -182,3 +182,17 @@ def test_backward_entry_points_reject_bad_arguments():
     assert rcall(B=0) == OK
     assert lib.msa_route_backward_workspace_size(2, 4, 4) >= 2 * 4 * 8
     assert lib.msa_route_backward_workspace_size(2, 130, 4) >= 2 * 4 * 8 * 3   # a candidate per 64 tokens
+
+
+def test_state_gather_sum_rejects_bad_arguments():
+    lib = _lib.load()
+    a = dict(dt=1, st=FAKE, D=10, S=64, idx=FAKE, B=2, k=3, out=FAKE, flag=None)
+    assert lib.msa_state_gather_sum(*dict(a, S=60).values(), None) == UNSUPPORTED     # bf16: S % 8
+    assert lib.msa_state_gather_sum(*dict(a, dt=0, S=62).values(), None) == UNSUPPORTED  # fp32: S % 4
+    assert lib.msa_state_gather_sum(*dict(a, B=70000).values(), None) == UNSUPPORTED
+    assert lib.msa_state_gather_sum(*dict(a, dt=7).values(), None) == INVALID
+    assert lib.msa_state_gather_sum(*dict(a, k=0).values(), None) == INVALID
+    assert lib.msa_state_gather_sum(*dict(a, D=0).values(), None) == INVALID
+    assert lib.msa_state_gather_sum(*dict(a, out=None).values(), None) == INVALID
+    assert lib.msa_state_gather_sum(*dict(a, out=FAKE + 4).values(), None) == INVALID
+    assert lib.msa_state_gather_sum(*dict(a, B=0).values(), None) == OK              # nothing to do
