@@ -108,6 +108,26 @@ __device__ __forceinline__ int64_t warp_owner_doc(const int64_t* __restrict__ of
   return lo;
 }
 
+// warp_owner_doc that first looks at the 32 documents around the proportional
+// guess c * D / C (one coalesced load; right whenever the documents' chunk
+// counts are close to uniform) and searches only if the owner is not among
+// them.  All 32 lanes must call it with the same c; all get the same answer,
+// a document in [0, D) whatever the offsets hold.
+__device__ __forceinline__ int64_t warp_owner_doc_near(const int64_t* __restrict__ off, int64_t D, int64_t C,
+                                                       int64_t c, int lane) {
+  int64_t g = (C > 0 ? (int64_t)((double)c * (double)D / (double)C) : 0) - 16;
+  if (g > D - 32) g = D - 32;
+  if (g < 0) g = 0;
+  const int64_t j = g + lane;
+  const unsigned m = __ballot_sync(0xffffffffu, j < D && __ldg(off + j) <= c);
+  if (m != 0) {
+    const int last = 31 - __clz(m);
+    // the window's next document starts after c (or there is none): it is the owner
+    if (last < 31 || g + 32 >= D) return g + last;
+  }
+  return warp_owner_doc(off, D, c, lane);
+}
+
 // Owning document of chunk c0 + lane for the 32 consecutive chunks of a warp
 // (-1 for chunks >= C).  One warp-wide search for c0, then each lane counts the
 // document boundaries at or below its chunk among the next 32 (documents with no
@@ -116,7 +136,7 @@ __device__ __forceinline__ int64_t warp_owner_doc(const int64_t* __restrict__ of
 __device__ __forceinline__ int warp_chunk_docs(const int64_t* __restrict__ off, int64_t D, int64_t C, int64_t c0,
                                                int lane) {
   if (c0 >= C) return -1;
-  const int64_t j0 = warp_owner_doc(off, D, c0, lane);
+  const int64_t j0 = warp_owner_doc_near(off, D, C, c0, lane);
   const int64_t c = c0 + lane;
   const int64_t bidx = j0 + 1 + lane;
   const int64_t b = __ldg(off + (bidx < D ? bidx : D));
