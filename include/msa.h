@@ -15,6 +15,12 @@
  *                         [selected memory rows ++ causal local KV].
  *   msa_layer_forward   - steps 2-5 in one call, with the gathered chunks kept
  *                         in the caller's workspace.
+ * Beyond the forward path: the backward of steps 5, 4 and 2
+ * (msa_sparse_attn_backward, msa_gather_backward, msa_route_backward), the sum
+ * of the selected documents' recurrent states that the linear (DGA) layers
+ * take as their initial state (msa_state_gather_sum, from the "MSA x Qwen3.5"
+ * model card), and a routing entry point that allocates nothing
+ * (msa_route_topk_noalloc).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
