@@ -242,6 +242,11 @@ msa_status msa_gather(msa_dtype dt, const int32_t* topk_idx, int64_t B, int k,
  * (msa_gather leaves zeros there).
  * Device flags: MSA_FLAG_INDEX_OOB when a mem_len is outside [0, Mmax] (that
  * batch row is computed with mem_len clamped into range).
+ * Workspace: msa_sparse_attn_workspace_size bytes, 16-byte aligned; for decode
+ * shapes (a few query rows per KV head) the size depends on the current
+ * device's SM count, so query it with the device that runs the call current
+ * (a workspace that is too small returns MSA_ERR_WORKSPACE and launches
+ * nothing).
  * ---------------------------------------------------------------------- */
 size_t msa_sparse_attn_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Mmax);
 msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const void* Vloc,
