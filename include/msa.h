@@ -184,9 +184,16 @@ msa_status msa_route_topk(msa_dtype dt, const void* Qr, int64_t B, int Tq, int H
  * ws / ws_bytes) and allocates nothing: its scratch is a fixed array of
  * MSA_NOALLOC_SCRATCH_BYTES in the library's own device memory, which every
  * GPU that loads the library holds until the process exits.
- *   - Problems whose msa_route_topk_workspace_size() exceeds
- *     MSA_NOALLOC_SCRATCH_BYTES return MSA_ERR_TOO_LARGE before any work is
- *     queued (for Hr = 8 and Tq <= 64 that is roughly B * D <= 4 million).
+ *   - Arguments are checked first, exactly as msa_route_topk checks them (a
+ *     bad argument returns its own error).  Then problems whose
+ *     msa_route_topk_workspace_size() exceeds MSA_NOALLOC_SCRATCH_BYTES return
+ *     MSA_ERR_TOO_LARGE.  Either way nothing is queued.  That size is, up to
+ *     256-byte rounding of each part, 4 (B D + B) + 4 C + 4 B Tq Hr bytes, plus
+ *     8 B k ceil(D / 8192) when D > 8192: the per-document keys and counters,
+ *     the chunk -> document map, the query norms and the top-k candidates.
+ *     So one query over documents of 8 chunks fits up to 465,768 documents
+ *     (3.7 million chunks; Hr = 8, Tq = 64, k = 16), and 64 one-token queries
+ *     up to 58,018 documents.
  *   - The first call on each device looks the array's device address up (with
  *     that device current) and caches it; make that first call before any
  *     stream capture.

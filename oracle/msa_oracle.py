@@ -223,18 +223,6 @@ def route(Qr, Krbar, doc_chunk_off) -> np.ndarray:
     return out
 
 
-def route_docs(Qr, Krbar, doc_chunk_off, docs) -> np.ndarray:
-    """route() restricted to the listed documents: [B, len(docs)] (for sampled full-size checks)."""
-    off = np.asarray(doc_chunk_off, dtype=np.int64)
-    Kb = np.asarray(Krbar)
-    out = np.full((np.asarray(Qr).shape[0], len(docs)), -np.inf)
-    for n, j in enumerate(docs):
-        a, b = int(off[j]), int(off[j + 1])
-        if b > a:
-            out[:, n] = cosine_scores(Qr, Kb[a:b]).max(axis=(1, 2))
-    return out
-
-
 # ----------------------------------------------------------------------------
 # step 3: top-k documents
 # ----------------------------------------------------------------------------

@@ -103,6 +103,14 @@ msa_status check_attn(msa_dtype dt, const void* Q, const void* Kloc, const void*
 
 }  // namespace
 
+namespace msa {
+msa_status route_topk_args_status(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr,
+                                  const void* Krbar, const float* kr_rnorm, const int64_t* doc_chunk_off,
+                                  int64_t D, int64_t C, int k, const int32_t* topk_idx) {
+  return check_route(dt, Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, k, topk_idx);
+}
+}  // namespace msa
+
 extern "C" {
 
 const char* msa_status_string(int status) {

@@ -62,6 +62,11 @@ struct RouteArgs {
   int32_t* err_flag;
 };
 cudaError_t launch_route(msa_dtype dt, const RouteArgs& a, cudaStream_t s);
+// The argument checks msa_route_topk runs before it looks at its workspace (no launch, no
+// pointer dereferenced): MSA_OK or the error msa_route_topk would return for these arguments.
+msa_status route_topk_args_status(msa_dtype dt, const void* Qr, int64_t B, int Tq, int Hr, int dr,
+                                  const void* Krbar, const float* kr_rnorm, const int64_t* doc_chunk_off,
+                                  int64_t D, int64_t C, int k, const int32_t* topk_idx);
 
 // Sum of each query's selected documents' recurrent states (the DGA layers'
 // injected initial state): out[b] = sum_r states[idx[b, r]] in fp32.

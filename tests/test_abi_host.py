@@ -196,3 +196,17 @@ def test_state_gather_sum_rejects_bad_arguments():
     assert lib.msa_state_gather_sum(*dict(a, out=None).values(), None) == INVALID
     assert lib.msa_state_gather_sum(*dict(a, out=FAKE + 4).values(), None) == INVALID
     assert lib.msa_state_gather_sum(*dict(a, B=0).values(), None) == OK              # nothing to do
+
+
+def test_noalloc_checks_arguments_before_its_size():
+    # msa_route_topk_noalloc runs msa_route_topk's argument checks first, so an
+    # invalid argument reports its own error even when the problem is also too
+    # large for the fixed scratch; a valid oversize problem reports TOO_LARGE
+    lib = _lib.load()
+    B, Tq, Hr, D, k = 64, 1, 8, 1 << 17, 16
+    call = lambda qr, dr, kk: lib.msa_route_topk_noalloc(1, qr, B, Tq, Hr, dr, FAKE, FAKE, FAKE, D, 4 * D, kk,
+                                                         None, FAKE, None, None, None)
+    assert call(FAKE, 96, k) == UNSUPPORTED      # dr = 96
+    assert call(None, 128, k) == INVALID         # no Qr
+    assert call(FAKE, 128, D + 1) == INVALID     # k > D
+    assert call(FAKE, 128, k) == -5              # MSA_ERR_TOO_LARGE
