@@ -52,6 +52,15 @@ the plainest reading and says so at the function (the list of readings):
      each query's selected documents' states elementwise; how a document's state
      is produced, and the delta rule that consumes S_ext, are defined outside
      the pages and are not part of this module.
+  R17 Memory Interleave (README, Figure 3 caption: an optional multi-round
+     interleave for multi-hop questions; FAQ "What is Memory Interleave?":
+     multi-round reasoning that jumps across scattered memory segments) is read
+     as R rounds of the memory path: round r routes its router query over the
+     bank, selects the k best documents not selected in an earlier round, and
+     attends over every round's documents so far (round order, then rank
+     order); the next round's router query is a given linear map W of this
+     round's attention output (the pages produce it with the model, which is not
+     available; W stands in for it).
 
 Layouts are row-major with the innermost dimension last:
   K, V [Ntok, Hkv, d]; Kr [Ntok, Hr, dr]; doc_tok_off int64 [D+1]
@@ -462,6 +471,72 @@ def route_backward(Qr, Krbar, doc_chunk_off, topk_idx, d_score):
                 dQ[b, t, h] += w * (k / (nq * nk) - cos * q / nq ** 2)
                 dK[c, h] += w * (q / (nq * nk) - cos * k / nk ** 2)
     return dQ, dK
+
+
+# ----------------------------------------------------------------------------
+# Memory Interleave (reading R17)
+# ----------------------------------------------------------------------------
+def exclude_selected(doc_scores, selected):
+    """Scores with each query's already-selected documents set to -inf (R17: a round
+    selects documents no earlier round selected).  selected: per query, a list of
+    document indices.  Pin: with every other score equal, top-k then returns the
+    lowest-index documents outside the excluded set."""
+    out = np.array(doc_scores, dtype=np.float64, copy=True)
+    for b, docs in enumerate(selected):
+        if len(docs):
+            out[b, np.asarray(docs, dtype=np.int64)] = -np.inf
+    return out
+
+
+def round_query(O_prev, W, Hr: int, dr: int):
+    """Next round's router query (R17): Qr[b, t] = O_prev[b, t] (as one Hq*d vector) times W [Hq*d, Hr*dr],
+    reshaped to [B, Tq, Hr, dr].  Pins: a one-hot W copies one output component to one
+    router component; the map is linear."""
+    O_prev = np.asarray(O_prev, dtype=np.float64)
+    B, Tq = O_prev.shape[:2]
+    flat = O_prev.reshape(B * Tq, -1)
+    return (flat @ np.asarray(W, dtype=np.float64)).reshape(B, Tq, Hr, dr)
+
+
+def interleave(Qr0, Krbar, doc_chunk_off, k: int, rounds: int, W, Q, Kloc, Vloc, Kbar, Vbar, Mmax: int,
+               scale=None, O_feed=None, qr_store=None):
+    """Memory Interleave over R = rounds rounds (reading R17), in the README's pipeline order per round.
+
+    Returns a dict with topk_idx / topk_score [B, rounds * k] (round r in columns
+    [r k, (r + 1) k)), O / lse of the last round, O_rounds (every round's output)
+    and Qr_rounds (every round's router query).  O_feed (list of arrays) supplies
+    the round outputs the next router queries are computed from instead of this
+    function's own (for step-by-step comparison with a device that stores them in
+    bf16); qr_store (a function) rounds each computed router query the way the
+    device stores it.  Pins: one round is layer_forward; the rounds' selections
+    are disjoint; with W = 0 every later round selects the lowest-index documents
+    not yet selected; brute force over the k-subsets outside the excluded set.
+    """
+    Qr = np.asarray(Qr0, dtype=np.float64)
+    B = Qr.shape[0]
+    Hr, dr = Qr.shape[2], Qr.shape[3]
+    chosen = [[] for _ in range(B)]
+    idx_all = np.zeros((B, rounds * k), dtype=np.int64)
+    sc_all = np.zeros((B, rounds * k))
+    outs, lses, qrs = [], [], []
+    for r in range(rounds):
+        qrs.append(Qr)
+        ds = exclude_selected(route(Qr, Krbar, doc_chunk_off), chosen)
+        ti, ts = topk(ds, k)
+        idx_all[:, r * k:(r + 1) * k] = ti
+        sc_all[:, r * k:(r + 1) * k] = ts
+        for b in range(B):
+            chosen[b] += [int(j) for j in ti[b]]
+        Km, Vm, ml = gather(np.array(chosen, dtype=np.int64), doc_chunk_off, Kbar, Vbar, Mmax)
+        O_r, lse_r = attention(Q, Kloc, Vloc, Km, Vm, ml, scale)
+        outs.append(O_r)
+        lses.append(lse_r)
+        if r + 1 < rounds:
+            src = O_feed[r] if O_feed is not None else O_r
+            Qr = round_query(src, W, Hr, dr)
+            if qr_store is not None:
+                Qr = qr_store(Qr)
+    return dict(topk_idx=idx_all, topk_score=sc_all, O=outs[-1], lse=lses[-1], O_rounds=outs, Qr_rounds=qrs)
 
 
 # ----------------------------------------------------------------------------

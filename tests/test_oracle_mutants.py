@@ -57,6 +57,13 @@ MUTANTS = [
      "test_state_gather_sum_one_hot_states_count_selections", ()),
     ("state_gather_sum", "for j in idx[b]:", "for j in sorted(set(idx[b].tolist())):",
      "test_state_gather_sum_one_hot_states_count_selections", ()),
+    ("interleave", "ds = exclude_selected(route(Qr, Krbar, doc_chunk_off), chosen)",
+     "ds = route(Qr, Krbar, doc_chunk_off)", "test_interleave_rounds_match_bruteforce_over_free_documents", ()),
+    ("interleave", "chosen[b] += [int(j) for j in ti[b]]", "chosen[b] = [int(j) for j in ti[b]]",
+     "test_interleave_attends_over_the_union_of_rounds", ()),
+    ("exclude_selected", "= -np.inf", "= 0.0", "test_interleave_zero_map_selects_lowest_free_documents", ()),
+    ("round_query", "flat = O_prev.reshape(B * Tq, -1)", "flat = O_prev.transpose(0, 2, 1, 3).reshape(B * Tq, -1)",
+     "test_round_query_one_hot_map_and_linearity", ()),
 ]
 
 

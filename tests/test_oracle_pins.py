@@ -455,3 +455,103 @@ def test_state_gather_sum_order_invariant_linear_and_total():
     assert np.allclose(every[0], np.sum(st, axis=0), rtol=1e-14, atol=1e-14)
     with pytest.raises(ValueError):
         O.state_gather_sum(st, np.array([[D]]))
+
+
+# ------------------------------------------------------------------ Memory Interleave (reading R17)
+def _interleave_case(seed, D=12, Tq=3, Lloc=5, Hq=4, Hkv=2, d=8, Hr=2, dr=8):
+    r = np.random.default_rng(seed)
+    n = r.integers(1, 4, size=D)
+    coff = np.concatenate([[0], np.cumsum(n)]).astype(np.int64)
+    C = int(coff[-1])
+    return dict(
+        Qr0=r.standard_normal((1, Tq, Hr, dr)), Krbar=r.standard_normal((C, Hr, dr)), coff=coff,
+        Q=r.standard_normal((1, Tq, Hq, d)), Kloc=r.standard_normal((1, Lloc, Hkv, d)),
+        Vloc=r.standard_normal((1, Lloc, Hkv, d)), Kbar=r.standard_normal((C, Hkv, d)),
+        Vbar=r.standard_normal((C, Hkv, d)), W=r.standard_normal((Hq * d, Hr * dr)), n=n)
+
+
+def _run_interleave(c, k, rounds, W=None, Mmax=None):
+    return O.interleave(c["Qr0"], c["Krbar"], c["coff"], k, rounds, c["W"] if W is None else W, c["Q"], c["Kloc"],
+                        c["Vloc"], c["Kbar"], c["Vbar"], Mmax or int(c["n"].sum()))
+
+
+def test_interleave_one_round_is_the_layer():
+    c = _interleave_case(1)
+    a = _run_interleave(c, 3, 1)
+    b = O.layer_forward(c["Qr0"], c["Krbar"], c["coff"], 3, c["Q"], c["Kloc"], c["Vloc"], c["Kbar"], c["Vbar"],
+                        int(c["n"].sum()))
+    assert np.array_equal(a["topk_idx"], b["topk_idx"])
+    assert np.array_equal(a["O"], b["O"]) and np.array_equal(a["lse"], b["lse"])
+
+
+def test_interleave_zero_map_selects_lowest_free_documents():
+    # with W = 0 every later router query is zero, every cosine is 0 (norm floor), all
+    # documents tie and the tie rule takes the lowest-index documents not yet selected
+    c = _interleave_case(2, D=14)
+    k, R = 3, 4
+    res = _run_interleave(c, k, R, W=np.zeros_like(c["W"]))
+    sel = res["topk_idx"][0]
+    taken = set(sel[:k].tolist())
+    for r in range(1, R):
+        free = [j for j in range(14) if j not in taken]
+        assert sel[r * k:(r + 1) * k].tolist() == free[:k]
+        taken |= set(free[:k])
+        assert np.all(res["topk_score"][0, r * k:(r + 1) * k] == 0.0)
+
+
+def test_interleave_rounds_match_bruteforce_over_free_documents():
+    # each round's selection is the best k-subset (largest score sum, then lower indices)
+    # among the documents no earlier round took, by enumeration
+    c = _interleave_case(3, D=9)
+    k, R = 2, 3
+    res = _run_interleave(c, k, R)
+    sel = res["topk_idx"][0]
+    assert len(set(sel.tolist())) == R * k, "rounds must select disjoint documents"
+    taken = []
+    for r in range(R):
+        sc = O.route(res["Qr_rounds"][r], c["Krbar"], c["coff"])[0]
+        free = [j for j in range(9) if j not in taken]
+        best = max(itertools.combinations(free, k), key=lambda sub: (sum(sc[j] for j in sub), [-j for j in sub]))
+        assert sorted(sel[r * k:(r + 1) * k].tolist()) == sorted(best)
+        taken += sel[r * k:(r + 1) * k].tolist()
+
+
+def test_round_query_one_hot_map_and_linearity():
+    r = np.random.default_rng(4)
+    B, Tq, Hq, d, Hr, dr = 2, 3, 2, 4, 3, 2
+    Op = r.standard_normal((B, Tq, Hq, d))
+    W = np.zeros((Hq * d, Hr * dr))
+    W[5, 3] = 1.0   # output component (head 1, dim 1) -> router component (head 1, dim 1)
+    W[2, 0] = 2.0   # (head 0, dim 2) -> twice into (head 0, dim 0)
+    q = O.round_query(Op, W, Hr, dr)
+    assert q.shape == (B, Tq, Hr, dr)
+    np.testing.assert_array_equal(q[:, :, 1, 1], Op[:, :, 1, 1])
+    np.testing.assert_array_equal(q[:, :, 0, 0], 2.0 * Op[:, :, 0, 2])
+    assert np.count_nonzero(q) == np.count_nonzero(Op[:, :, 1, 1]) + np.count_nonzero(Op[:, :, 0, 2])
+    W2 = r.standard_normal(W.shape)
+    np.testing.assert_allclose(O.round_query(Op, 3 * W - W2, Hr, dr),
+                               3 * O.round_query(Op, W, Hr, dr) - O.round_query(Op, W2, Hr, dr), atol=1e-12)
+
+
+def test_interleave_attends_over_the_union_of_rounds():
+    # Q = 0 makes every visible key weigh the same; each document's value rows are its
+    # one-hot id and the local values are zero, so round r's output counts the chunks of
+    # every document selected up to round r: n_j / (memory rows + visible local rows)
+    D, k, R, Tq, Lloc = 10, 2, 3, 2, 3
+    c = _interleave_case(5, D=D, Tq=Tq, Lloc=Lloc, Hq=2, Hkv=1, d=16)
+    c["Q"] = np.zeros_like(c["Q"])
+    c["Vloc"] = np.zeros_like(c["Vloc"])
+    doc_of_chunk = np.repeat(np.arange(D), c["n"])
+    c["Vbar"] = np.zeros_like(c["Vbar"])
+    c["Vbar"][np.arange(len(doc_of_chunk)), 0, doc_of_chunk] = 1.0
+    res = _run_interleave(c, k, R)
+    sel = res["topk_idx"][0]
+    for r in range(R):
+        union = sel[:(r + 1) * k]
+        M = int(c["n"][union].sum())
+        for t in range(Tq):
+            vis = M + (Lloc - Tq + t) + 1
+            want = np.zeros(16)
+            want[union] = c["n"][union] / vis
+            for h in range(2):
+                np.testing.assert_allclose(res["O_rounds"][r][0, t, h], want, atol=1e-12)
