@@ -61,6 +61,17 @@ the plainest reading and says so at the function (the list of readings):
      order); the next round's router query is a given linear map W of this
      round's attention output (the pages produce it with the model, which is not
      available; W stands in for it).
+  R18 The linear (DGA) layers' query path consumes S_ext as the initial state of
+     the gated delta rule (model card, "Architecture summary").  The pages do not
+     define that rule; it is the recurrence of Gated DeltaNet (Yang, Kautz and
+     Hatamizadeh, "Gated Delta Networks: Improving Mamba2 with Delta Rule", ICLR
+     2025), written here per value head with the state h (key dim x value dim, the
+     transpose of the paper's S):
+         h_t = exp(g_t) (I - beta_t k_t k_t^T) h_{t-1} + beta_t k_t v_t^T
+         o_t = h_t^T (scale q_t)
+     with h_0 = S_ext, log gates g_t <= 0 and write strengths beta_t given; a
+     value head h reads key head h / (Hv / Hk).  Keys are used as given (the
+     model normalises them before the rule).
 
 Layouts are row-major with the innermost dimension last:
   K, V [Ntok, Hkv, d]; Kr [Ntok, Hr, dr]; doc_tok_off int64 [D+1]
@@ -471,6 +482,86 @@ def route_backward(Qr, Krbar, doc_chunk_off, topk_idx, d_score):
                 dQ[b, t, h] += w * (k / (nq * nk) - cos * q / nq ** 2)
                 dK[c, h] += w * (q / (nq * nk) - cos * k / nk ** 2)
     return dQ, dK
+
+
+# ----------------------------------------------------------------------------
+# the linear (DGA) layers' query path: gated delta rule from S_ext (reading R18)
+# ----------------------------------------------------------------------------
+def gated_delta_rule(q, k, v, g, beta, h0=None, scale=1.0):
+    """The gated delta rule of reading R18, token by token (the definition).
+
+    q, k [B, T, Hk, dk]; v [B, T, Hv, dv]; g, beta [B, T, Hv]; h0 [B, Hv, dk, dv]
+    or None (zeros).  Returns (o [B, T, Hv, dv], h_T [B, Hv, dk, dv]) in fp64.
+    Pins: beta = 0 decays h0 by the cumulative gate; with unit gates, beta = 1 and
+    a unit key the state returns v at that key; orthonormal keys overwrite
+    exactly their rows of h0; the output is affine in h0; the chunked form below
+    agrees.
+    """
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    g, beta = np.asarray(g, dtype=np.float64), np.asarray(beta, dtype=np.float64)
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    grp = Hv // Hk
+    h = np.zeros((B, Hv, dk, dv)) if h0 is None else np.array(h0, dtype=np.float64, copy=True)
+    o = np.zeros((B, T, Hv, dv))
+    for b in range(B):
+        for hv in range(Hv):
+            hk = hv // grp
+            H = h[b, hv]
+            for t in range(T):
+                kt, qt, vt = k[b, t, hk], q[b, t, hk], v[b, t, hv]
+                a, bt = math.exp(g[b, t, hv]), beta[b, t, hv]
+                H = a * (H - bt * np.outer(kt, kt @ H)) + bt * np.outer(kt, vt)
+                o[b, t, hv] = H.T @ (scale * qt)
+            h[b, hv] = H
+    return o, h
+
+
+def gated_delta_rule_chunked(q, k, v, g, beta, h0=None, scale=1.0, chunk: int = 64):
+    """The same rule computed chunk by chunk (the form the GPU kernel uses), for cross-checking.
+
+    Within a chunk of C tokens, with G_i the cumulative log gate from the chunk's
+    start, the state after token i is exp(G_i) h0 + sum_{j <= i} exp(G_i - G_j) k_j u_j^T,
+    where the new-value rows u solve the unit lower-triangular system
+        u_i + beta_i sum_{j < i} exp(G_i - G_j) (k_i . k_j) u_j = beta_i (v_i - exp(G_i) h0^T k_i),
+    so o_i = scale (exp(G_i) h0^T q_i + sum_{j <= i} exp(G_i - G_j) (q_i . k_j) u_j) and the
+    chunk ends with h = exp(G_C) h0 + sum_j exp(G_C - G_j) k_j u_j^T.  (Derived from the
+    recurrence by induction over i; it is the chunkwise form of the Gated DeltaNet paper.)
+    Pin: equal to gated_delta_rule up to rounding.
+    """
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    g, beta = np.asarray(g, dtype=np.float64), np.asarray(beta, dtype=np.float64)
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    grp = Hv // Hk
+    h = np.zeros((B, Hv, dk, dv)) if h0 is None else np.array(h0, dtype=np.float64, copy=True)
+    o = np.zeros((B, T, Hv, dv))
+    for b in range(B):
+        for hv in range(Hv):
+            hk = hv // grp
+            H = h[b, hv]
+            for c0 in range(0, T, chunk):
+                c1 = min(c0 + chunk, T)
+                K, Q, V = k[b, c0:c1, hk], q[b, c0:c1, hk], v[b, c0:c1, hv]
+                G = np.cumsum(g[b, c0:c1, hv])
+                bt = beta[b, c0:c1, hv]
+                n = c1 - c0
+                decay = np.exp(np.minimum(G[:, None] - G[None, :], 0.0))  # exp(G_i - G_j) for j <= i
+                A = np.tril(np.ones((n, n)), -1) * decay * (K @ K.T)
+                rhs = bt[:, None] * (V - np.exp(G)[:, None] * (K @ H))
+                U = np.linalg.solve(np.eye(n) + bt[:, None] * A, rhs)
+                P = np.tril(np.ones((n, n))) * decay * (Q @ K.T)
+                o[b, c0:c1, hv] = scale * (np.exp(G)[:, None] * (Q @ H) + P @ U)
+                H = math.exp(G[-1]) * H + (np.exp(G[-1] - G)[:, None] * K).T @ U
+            h[b, hv] = H
+    return o, h
+
+
+def dga_query(states, topk_idx, q, k, v, g, beta, scale=1.0):
+    """The linear layers' memory path (model card, "Architecture summary"; readings R16, R18):
+    S_ext = state_gather_sum(states, topk_idx) is the initial state of the gated delta rule over
+    the query tokens.  states [D, Hv, dk, dv].  Returns (o, h_T)."""
+    return gated_delta_rule(q, k, v, g, beta, state_gather_sum(states, topk_idx), scale)
 
 
 # ----------------------------------------------------------------------------

@@ -64,6 +64,17 @@ MUTANTS = [
     ("exclude_selected", "= -np.inf", "= 0.0", "test_interleave_zero_map_selects_lowest_free_documents", ()),
     ("round_query", "flat = O_prev.reshape(B * Tq, -1)", "flat = O_prev.transpose(0, 2, 1, 3).reshape(B * Tq, -1)",
      "test_round_query_one_hot_map_and_linearity", ()),
+    ("gated_delta_rule", "H = a * (H - bt * np.outer(kt, kt @ H)) + bt * np.outer(kt, vt)",
+     "H = a * H + bt * np.outer(kt, vt)", "test_gdr_full_write_recalls_the_value_at_its_key", ()),
+    ("gated_delta_rule", "o[b, t, hv] = H.T @ (scale * qt)", "o[b, t, hv] = H @ (scale * qt)",
+     "test_gdr_zero_write_strength_decays_the_initial_state", ()),
+    ("gated_delta_rule", "hk = hv // grp", "hk = hv % Hk", "test_gdr_value_heads_share_their_key_head", ()),
+    ("gated_delta_rule", "a, bt = math.exp(g[b, t, hv]), beta[b, t, hv]", "a, bt = 1.0, beta[b, t, hv]",
+     "test_gdr_zero_write_strength_decays_the_initial_state", ()),
+    ("gated_delta_rule_chunked", "A = np.tril(np.ones((n, n)), -1) * decay * (K @ K.T)",
+     "A = np.tril(np.ones((n, n)), -1) * (K @ K.T)", "test_gdr_chunked_form_equals_the_recurrence", (37, 8)),
+    ("state_gather_sum", "out[b] += st[j]", "out[b] = st[j]", "test_dga_query_starts_from_the_selected_documents_states",
+     ()),
 ]
 
 

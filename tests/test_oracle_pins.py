@@ -555,3 +555,89 @@ def test_interleave_attends_over_the_union_of_rounds():
             want[union] = c["n"][union] / vis
             for h in range(2):
                 np.testing.assert_allclose(res["O_rounds"][r][0, t, h], want, atol=1e-12)
+
+
+# ------------------------------------------------------------------ gated delta rule (reading R18)
+def _gdr_case(seed, B=1, T=9, Hk=1, Hv=1, dk=6, dv=6, unit_keys=True):
+    r = np.random.default_rng(seed)
+    k = r.standard_normal((B, T, Hk, dk))
+    if unit_keys:
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    return dict(q=r.standard_normal((B, T, Hk, dk)), k=k, v=r.standard_normal((B, T, Hv, dv)),
+                g=-r.uniform(0.0, 0.3, (B, T, Hv)), beta=r.uniform(0.1, 1.0, (B, T, Hv)),
+                h0=r.standard_normal((B, Hv, dk, dv)))
+
+
+def test_gdr_zero_write_strength_decays_the_initial_state():
+    # beta = 0: nothing is written, h_t = exp(g_1 + ... + g_t) h0 and o_t = scale h_t^T q_t
+    c = _gdr_case(1, T=7)
+    o, h = O.gated_delta_rule(c["q"], c["k"], c["v"], c["g"], np.zeros_like(c["beta"]), c["h0"], scale=0.5)
+    G = np.cumsum(c["g"][0, :, 0])
+    for t in range(7):
+        np.testing.assert_allclose(o[0, t, 0], 0.5 * math.exp(G[t]) * c["h0"][0, 0].T @ c["q"][0, t, 0], atol=1e-12)
+    np.testing.assert_allclose(h[0, 0], math.exp(G[-1]) * c["h0"][0, 0], atol=1e-12)
+
+
+def test_gdr_full_write_recalls_the_value_at_its_key():
+    # unit gate, beta = 1, a unit key: (I - k k^T) erases what the state held at k, then k v^T
+    # writes v there, so h^T k = v exactly whatever h0 was; reading with q = k returns scale v
+    c = _gdr_case(2, T=1)
+    c["q"] = c["k"].copy()
+    o, h = O.gated_delta_rule(c["q"], c["k"], c["v"], np.zeros((1, 1, 1)), np.ones((1, 1, 1)), c["h0"], scale=2.0)
+    np.testing.assert_allclose(h[0, 0].T @ c["k"][0, 0, 0], c["v"][0, 0, 0], atol=1e-12)
+    np.testing.assert_allclose(o[0, 0, 0], 2.0 * c["v"][0, 0, 0], atol=1e-12)
+
+
+def test_gdr_orthonormal_keys_overwrite_exactly_their_rows():
+    # keys e_2, e_0, e_2: rows 0 and 2 end as the last value written at them, the rest are h0's
+    dk = dv = 5
+    c = _gdr_case(3, T=3, dk=dk, dv=dv)
+    k = np.zeros((1, 3, 1, dk))
+    for t, row in enumerate((2, 0, 2)):
+        k[0, t, 0, row] = 1.0
+    _, h = O.gated_delta_rule(c["q"], k, c["v"], np.zeros((1, 3, 1)), np.ones((1, 3, 1)), c["h0"])
+    want = c["h0"][0, 0].copy()
+    want[0] = c["v"][0, 1, 0]
+    want[2] = c["v"][0, 2, 0]
+    np.testing.assert_allclose(h[0, 0], want, atol=1e-12)
+
+
+def test_gdr_output_is_affine_in_the_initial_state():
+    c = _gdr_case(4, T=6)
+    run = lambda h0: O.gated_delta_rule(c["q"], c["k"], c["v"], c["g"], c["beta"], h0)[0]
+    base = run(np.zeros_like(c["h0"]))
+    np.testing.assert_allclose(run(3 * c["h0"]) - base, 3 * (run(c["h0"]) - base), atol=1e-10)
+
+
+def test_gdr_value_heads_share_their_key_head():
+    # two value heads on one key head with the same values, gates and strengths give the same output
+    c = _gdr_case(5, T=8, Hk=2, Hv=4)
+    for a, b in ((0, 1), (2, 3)):
+        for name in ("v", "g", "beta"):
+            c[name][:, :, b] = c[name][:, :, a]
+        c["h0"][:, b] = c["h0"][:, a]
+    o, _ = O.gated_delta_rule(c["q"], c["k"], c["v"], c["g"], c["beta"], c["h0"])
+    np.testing.assert_allclose(o[:, :, 1], o[:, :, 0], atol=1e-12)
+    np.testing.assert_allclose(o[:, :, 3], o[:, :, 2], atol=1e-12)
+    assert np.abs(o[:, :, 0] - o[:, :, 2]).max() > 1e-3
+
+
+@pytest.mark.parametrize("T,chunk", [(37, 8), (64, 64), (70, 16), (5, 64)])
+def test_gdr_chunked_form_equals_the_recurrence(T, chunk):
+    c = _gdr_case(6, B=2, T=T, Hk=2, Hv=4, dk=8, dv=6)
+    o1, h1 = O.gated_delta_rule(c["q"], c["k"], c["v"], c["g"], c["beta"], c["h0"], scale=0.7)
+    o2, h2 = O.gated_delta_rule_chunked(c["q"], c["k"], c["v"], c["g"], c["beta"], c["h0"], scale=0.7, chunk=chunk)
+    np.testing.assert_allclose(o2, o1, atol=1e-10)
+    np.testing.assert_allclose(h2, h1, atol=1e-10)
+
+
+def test_dga_query_starts_from_the_selected_documents_states():
+    r = np.random.default_rng(7)
+    c = _gdr_case(7, B=2, T=4, Hk=1, Hv=2)
+    states = r.standard_normal((5, 2, 6, 6))
+    idx = np.array([[1, 3], [4, 4]])
+    o, h = O.dga_query(states, idx, c["q"], c["k"], c["v"], c["g"], c["beta"])
+    h0 = np.stack([states[1] + states[3], 2 * states[4]])
+    o2, h2 = O.gated_delta_rule(c["q"], c["k"], c["v"], c["g"], c["beta"], h0)
+    np.testing.assert_allclose(o, o2, atol=1e-12)
+    np.testing.assert_allclose(h, h2, atol=1e-12)
