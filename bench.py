@@ -1,11 +1,18 @@
 #!/usr/bin/env python3
 """Throughput of the MSA memory path on B200 (one JSON line on rank 0).
 
-A step is one pass of the whole memory path over one batch of synthetic input:
-msa_pool of the raw per-token K / V / Kr of every document into the bank, then
-msa_layer_forward (route + top-k + index-driven gather + attention) for the
-query of each layer.  The default workload is the 1M-token memory of the
-Qwen3-4B-shaped layer (2048 documents x 512 tokens, Tq = 512 prefill tokens).
+A step is one pass of the query path of every layer over one batch of
+synthetic input, on a memory bank pooled (msa_pool) before the timed region:
+per layer msa_route_topk (cosine routing scan of the whole bank + top-k) and
+msa_sparse_attn_indexed (attention over the selected documents' chunks read
+in place from the bank by index, ++ the causal local KV) -- the two calls
+msa_layer_forward makes.  Pooling is the offline stage of the pages'
+inference pipeline; it is timed on its own and reported beside the step.
+The default workload is the 100M-token memory bank (195,313 documents,
+1,562,500 chunks, Tq = 64 query tokens, Qwen3-4B-shaped heads); on one GPU
+the same line also carries stage results of the 16M-token decode batch, the
+10M-token 16-layer prefill stack and the 1M-token layer, each with the SM
+clock it ran at.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl msa|reference]
 
@@ -166,19 +173,31 @@ def workload_label(cfg: synth.Config) -> str:
             f"d={cfg.d}, k={cfg.k}, layers={cfg.layers}")
 
 
-def step_label(step_kind: str) -> str:
-    return ("msa_pool of every raw token, then per layer msa_route_topk, msa_gather, msa_sparse_attn"
-            if step_kind == "full" else
-            "per layer msa_route_topk, msa_gather, msa_sparse_attn over a bank pooled before timing")
+def raw_bytes(cfg: synth.Config) -> int:
+    """Bytes of the raw per-token K, V and Kr of the whole corpus."""
+    return cfg.ntok * (2 * cfg.Hkv * cfg.d + cfg.Hr * cfg.dr) * (4 if cfg.dtype == "f32" else 2)
+
+
+RAW_RESIDENT_MAX = 80e9  # a corpus this large is pooled slab by slab instead of held resident
+
+
+def step_label(step_kind: str, unfused: bool = False) -> str:
+    q = ("per layer msa_route_topk, msa_gather, msa_sparse_attn" if unfused else
+         "per layer msa_route_topk + msa_sparse_attn_indexed (the calls of msa_layer_forward: routing scan + top-k, "
+         "then attention over the selected chunks read in place from the bank)")
+    return ("msa_pool of every raw token, then " + q) if step_kind == "full" else \
+        (q + " over a bank pooled before timing")
 
 
 def step_kind_for(cfg: synth.Config, args) -> str:
-    """'full' (pool + layers) unless the raw corpus does not fit the device next to the bank, or the
-    bank's K̄ / V̄ live in host memory (the pool writes them on the device first)."""
+    """'query' (the query path over a bank pooled before timing) unless --step full asks for the
+    offline pool inside the step too (only when the raw corpus fits the device next to the bank and
+    the bank's K̄ / V̄ stay on the device)."""
     if getattr(args, "bank_kv", "device") == "host":
         return "query"
-    raw_bytes = cfg.ntok * (2 * cfg.Hkv * cfg.d + cfg.Hr * cfg.dr) * (4 if cfg.dtype == "f32" else 2)
-    return args.step or ("query" if raw_bytes > 80e9 else "full")
+    if args.step == "full" and raw_bytes(cfg) <= RAW_RESIDENT_MAX:
+        return "full"
+    return "query"
 
 
 def workload_config(args) -> synth.Config:
@@ -192,18 +211,19 @@ def workload_config(args) -> synth.Config:
 class MSAWorkload:
     """Device buffers of one workload and its step.
 
-    step "full": msa_pool of every raw token (resident in HBM), then for every
-    layer msa_route_topk -> msa_gather -> msa_sparse_attn (the calls
-    msa_layer_forward makes).  step "query": the bank is pooled once at set-up,
-    slab by slab (a 100M-token corpus cannot be resident), and the step is the
-    per-layer query path only.
+    The bank (K̄, V̄, K̄r, 1/‖K̄r‖) is pooled at set-up: from a resident raw corpus
+    in one msa_pool call when the corpus fits the device (then the pool can be
+    timed on its own, or inside the step with step "full"), else slab by slab as
+    the raw tokens are drawn (a 100M-token corpus cannot be resident), with the
+    pool launches timed by events as they run.  The step per layer is
+    msa_route_topk then msa_sparse_attn_indexed (unfused: msa_gather then
+    msa_sparse_attn on the copied rows).
     """
 
-    STAGES = ("pool", "route_topk", "gather", "sparse_attn")
-
-    def __init__(self, cfg: synth.Config, device, seed: int, step_kind: str, bank_kv: str = "device"):
+    def __init__(self, cfg: synth.Config, device, seed: int, step_kind: str, bank_kv: str = "device",
+                 unfused: bool = False, keep_raw: bool = False):
         import routed_sparse_attention_chunk_b200 as msa
-        self.msa, self.cfg, self.dev, self.kind = msa, cfg, device, step_kind
+        self.msa, self.cfg, self.dev, self.kind, self.unfused = msa, cfg, device, step_kind, unfused
         dt = cfg.torch_dtype
         self.layers = [synth.gen_query(cfg, l, device, seed) for l in range(cfg.layers)]
         tok = synth.doc_tok_offsets(cfg)
@@ -219,8 +239,11 @@ class MSAWorkload:
         self.rn = torch.empty((self.C, cfg.Hr), dtype=torch.float32, device=device)
         self.flag = torch.zeros(1, dtype=torch.int32, device=device)
         self.raw = None
-        if step_kind == "full":
+        self.slab_pool_ms = None  # pool launches of the slab-by-slab set-up, timed by events
+        if (step_kind == "full" or keep_raw) and raw_bytes(cfg) <= RAW_RESIDENT_MAX:
             self._fill_raw(seed)
+            self.pool()
+            torch.cuda.synchronize()
         else:
             self._pool_slabs(seed)
         if bank_kv == "host":
@@ -233,12 +256,21 @@ class MSAWorkload:
         self.idx = [torch.empty((B, c.k), dtype=torch.int32, device=device) for _ in self.layers]
         self.rws = torch.empty(msa.route_topk_workspace_size(B, c.Tq, c.Hr, self.D, self.C, c.k), dtype=torch.uint8,
                                device=device)
-        self.Km = torch.zeros((B, c.Mmax, c.Hkv, c.d), dtype=dt, device=device)
-        self.Vm = torch.zeros_like(self.Km)
-        self.ml = torch.zeros(B, dtype=torch.int32, device=device)
+        self.iws = torch.empty(max(256, msa.sparse_attn_indexed_workspace_size(B, c.Tq, c.Lloc, c.Hq, c.Hkv, c.d, c.k,
+                                                                                c.Mmax)),
+                               dtype=torch.uint8, device=device)
         n = msa.sparse_attn_workspace_size(B, c.Tq, c.Lloc, c.Hq, c.Hkv, c.d, c.Mmax)
         self.aws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+        if unfused:
+            self.Km = torch.zeros((B, c.Mmax, c.Hkv, c.d), dtype=dt, device=device)
+            self.Vm = torch.zeros_like(self.Km)
+            self.ml = torch.zeros(B, dtype=torch.int32, device=device)
         self.pipe = None
+
+    @property
+    def stages(self):
+        q = ("route_topk", "gather", "sparse_attn") if self.unfused else ("route_topk", "sparse_attn")
+        return (("pool",) if self.kind == "full" else ()) + q
 
     def enable_pipeline(self):
         """Run the query path through the three-stream schedule (route of batch i+1, gather of batch
@@ -276,18 +308,25 @@ class MSAWorkload:
 
     def _pool_slabs(self, seed):
         c, msa = self.cfg, self.msa
+        stream = torch.cuda.current_stream()
+        evs = []
         for lo, hi in synth.slab_bounds(c):
             K, V, Kr = synth.gen_raw_slab(c, lo, hi, self.dev, seed, Qr0=self.layers[0]["Qr"][0])
             t = torch.from_numpy(self.tok[lo:hi + 1] - self.tok[lo]).to(self.dev)
             cs, ce = int(self.coff[lo]), int(self.coff[hi])
             ch = torch.from_numpy(self.coff[lo:hi + 1] - self.coff[lo]).to(self.dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
             msa.pool(K, V, Kr, t, ch, c.P, self.rope, self.Kb[cs:ce], self.Vb[cs:ce], self.Krb[cs:ce],
                      self.rn[cs:ce], self.flag)
+            e1.record(stream)
+            evs.append((e0, e1))
             del K, V, Kr
         torch.cuda.synchronize()
+        self.slab_pool_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
 
     def input_tensors(self):
-        ts = list(self.raw) if self.raw is not None else []
+        ts = list(self.raw) if (self.raw is not None and self.kind == "full") else []
         for L in self.layers:
             ts += [L["Qr"], L["Q"], L["Kloc"], L["Vloc"]]
         return ts
@@ -311,8 +350,12 @@ class MSAWorkload:
 
     def sparse_attn(self, l):
         L = self.layers[l]
-        self.msa.sparse_attn(L["Q"], L["Kloc"], L["Vloc"], self.Km, self.Vm, self.ml, self.O[l], ws=self.aws,
-                             err_flag=self.flag)
+        if self.unfused:
+            self.msa.sparse_attn(L["Q"], L["Kloc"], L["Vloc"], self.Km, self.Vm, self.ml, self.O[l], ws=self.aws,
+                                 err_flag=self.flag)
+        else:
+            self.msa.sparse_attn_indexed(L["Q"], L["Kloc"], L["Vloc"], self.idx[l], self.coff_d, self.Kb, self.Vb,
+                                         self.cfg.Mmax, self.O[l], self.iws, err_flag=self.flag)
 
     def step(self, rec=None):
         """One step; rec(stage) records an event after each stage when given."""
@@ -322,8 +365,9 @@ class MSAWorkload:
         for l in range(self.cfg.layers):
             self.route_topk(l)
             rec and rec("route_topk")
-            self.gather(l)
-            rec and rec("gather")
+            if self.unfused:
+                self.gather(l)
+                rec and rec("gather")
             self.sparse_attn(l)
             rec and rec("sparse_attn")
 
@@ -353,14 +397,146 @@ def stage_roofline(name: str, ms: float, cfg: synth.Config, counts: dict, peaks:
         if cfg.Tq == 1:  # decode: the local and memory KV stream
             by = cfg.B * (cfg.Lloc + cfg.Mmax) * cfg.Hkv * cfg.d * esz * 2
             return {"bound": "hbm", "achieved": by / ms / 1e6, "peak": hbm, "unit": "GB/s",
-                    "kernel": "msa_sparse_attn (decode)", "alg_bytes_per_launch": by,
-                    "peak_source": f"{peak_kind} hbm_gbs"}
+                    "kernel": "msa_sparse_attn_indexed (plan + attn_decode_kernel + combine)",
+                    "alg_bytes_per_launch": by, "peak_source": f"{peak_kind} hbm_gbs"}
         return {"bound": "tensor", "achieved": fl / ms / 1e9, "peak": tfl, "unit": "TFLOP/s",
-                "kernel": "attn_tc_kernel (msa_sparse_attn)", "alg_flops_per_launch": fl,
+                "kernel": "msa_sparse_attn_indexed (plan + attn_tc_kernel)", "alg_flops_per_launch": fl,
                 "peak_source": f"{peak_kind} {tfl_name}"}
     by = 2 * 2 * cfg.B * cfg.Mmax * cfg.Hkv * cfg.d * esz
     return {"bound": "hbm", "achieved": by / ms / 1e6, "peak": hbm, "unit": "GB/s", "kernel": "gather_kernel",
             "alg_bytes_per_launch": by, "peak_source": f"{peak_kind} hbm_gbs"}
+
+
+def timed_steps(w: MSAWorkload, steps: int, warmup: int, flush, world: int, device):
+    """W untimed steps, then exactly K steps with an event after every stage.  Returns per-stage
+    launch times (ms), the whole timed region (ms), NVML clocks during it and the launch count."""
+    msa = w.msa
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(device)
+    for _ in range(warmup):
+        w.step()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    sampler.start()
+    n0 = msa.kernel_launch_count()
+    marks = []  # (stage, event) in launch order
+
+    def rec(stage):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        marks.append((stage, e))
+
+    t_all0, t_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_all0.record(stream)
+    for _ in range(steps):
+        if flush is not None:
+            flush.fill_(1.0)
+        rec("start")
+        w.step(rec)
+    t_all1.record(stream)
+    torch.cuda.synchronize()
+    launches = msa.kernel_launch_count() - n0
+    clocks = sampler.stop()
+    stage_ms = {s: [] for s in w.stages}
+    for (s0, e0), (s1, e1) in zip(marks[:-1], marks[1:]):
+        if s1 != "start":
+            stage_ms[s1].append(e0.elapsed_time(e1))
+    return stage_ms, t_all0.elapsed_time(t_all1), clocks, launches
+
+
+def timed_pool(w: MSAWorkload, launches: int, warmup: int, device):
+    """msa_pool of the resident raw corpus on its own: per-launch times (ms) and clocks."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        w.pool()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device)
+    sampler.start()
+    ev = []
+    for _ in range(launches):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        w.pool()
+        e1.record(stream)
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in ev], sampler.stop()
+
+
+def read_stream_gbs(device, gib: int = 4) -> float:
+    """Read-only HBM stream measured live: a torch sum over a `gib` GiB bf16 tensor (best of 5)."""
+    x = torch.ones(gib * (1 << 29), dtype=torch.bfloat16, device=device)
+    nbytes = x.numel() * x.element_size()
+    best = float("inf")
+    for _ in range(6):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch.sum(x, dtype=torch.float32)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del x
+    torch.cuda.empty_cache()
+    return nbytes / (best / 1e3) / 1e9
+
+
+def stage_entry(name, times, cfg, counts, peaks, peak_kind, long_region, clocks, total=None) -> dict:
+    """Per-stage summary: time per launch, achieved work rate and its fraction of the peak, and
+    the launch's length in SM cycles at the median clock sampled while it ran."""
+    per = float(np.mean(times))
+    r = stage_roofline(name, per, cfg, counts, peaks, peak_kind, long_region)
+    mhz = clocks.get("sm_mhz")
+    out = {"ms_per_launch": round(per, 4), "launches": len(times), "bound": r["bound"],
+           "achieved": round(r["achieved"], 2), "unit": r["unit"], "peak": r["peak"],
+           "frac": round(r["achieved"] / r["peak"], 4), "peak_source": r["peak_source"],
+           "sm_mhz": mhz, "kcycles_per_launch": round(per * mhz, 1) if mhz else None}
+    if total:
+        out["share"] = round(float(np.sum(times)) / total, 4)
+    return out
+
+
+def workload_extra(name: str, device, seed: int, peaks: dict, peak_kind: str, steps: int, warmup: int) -> dict:
+    """Stage results of another workload, measured in the same run: the query-path step (W warm-up,
+    K timed), each stage's achieved rate against its roofline, and the offline pool on its own."""
+    cfg = synth.get_config(name)
+    counts = workload_counts(cfg)
+    keep_raw = raw_bytes(cfg) <= RAW_RESIDENT_MAX
+    w = MSAWorkload(cfg, device, seed=seed, step_kind="query", keep_raw=keep_raw)
+    in_bytes = w.Krb.numel() * w.Krb.element_size() + sum(t.numel() * t.element_size() for t in w.input_tensors())
+    flush = None if in_bytes > L2_BYTES else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    stage_ms, timed_ms, clocks, launches = timed_steps(w, steps, warmup, flush, 1, device)
+    step_sum = sum(sum(v) for v in stage_ms.values())
+    ms_per_step = (step_sum if flush is not None else timed_ms) / steps
+    long_region = sustained_region(timed_ms, clocks)
+    out = {"workload": workload_label(cfg), "step": step_label("query"), "steps": steps, "warmup": warmup,
+           "ms_per_step": round(ms_per_step, 4), "value": round(cfg.B * cfg.Tq / (ms_per_step / 1e3), 1),
+           "unit": UNIT, "clocks": clocks, "gpu_launches": int(launches),
+           "l2": "inputs larger than L2" if flush is None else "L2 flushed between steps (not timed)",
+           "stages": {s: stage_entry(s, v, cfg, counts, peaks, peak_kind, long_region, clocks, step_sum)
+                      for s, v in stage_ms.items() if v}}
+    if w.raw is not None:
+        n = 3 if raw_bytes(cfg) > 20e9 else 10
+        ptimes, pclocks = timed_pool(w, n, 2, device)
+        out["offline_pool"] = stage_entry("pool", ptimes, cfg, counts, peaks, peak_kind,
+                                          sustained_region(float(np.sum(ptimes)), pclocks), pclocks)
+        out["offline_pool"]["clocks"] = pclocks
+    elif w.slab_pool_ms:
+        out["offline_pool"] = slab_pool_entry(w, cfg, counts, peaks, peak_kind)
+    out["err_flag"] = int(w.flag.item())
+    del w
+    torch.cuda.empty_cache()
+    return out
+
+
+def slab_pool_entry(w: MSAWorkload, cfg, counts, peaks, peak_kind) -> dict:
+    """The bank built slab by slab at set-up: total pool time over every slab (one pass, events)."""
+    ms = float(np.sum(w.slab_pool_ms))
+    gbs = counts["pool_bytes"] / ms / 1e6
+    return {"ms_total": round(ms, 3), "slabs": len(w.slab_pool_ms), "achieved": round(gbs, 2), "unit": "GB/s",
+            "peak": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_kind} hbm_gbs",
+            "note": "one pass over the corpus while the bank is built (no warm-up); the slabs' raw tokens are drawn "
+                    "between launches"}
 
 
 def run_backward(args, rank, local_rank, world):
@@ -557,6 +733,108 @@ def run_state(args, rank, local_rank, world):
     }
 
 
+EXTRA_WORKLOADS = ("decode16m", "stack10m", "1m")
+EXTRA_STEPS = {"decode16m": 30, "stack10m": 8, "1m": 30}
+
+
+DGA_HEADS = (16, 32)  # key heads, value heads of the linear layers (d = 128); the pages give no head counts
+
+
+def run_dga(args, rank, local_rank, world):
+    """The linear (DGA) layers' memory path for the workload's queries: per step, the sum of each
+    query's k selected documents' recurrent states (msa_state_gather_sum, S_ext) and the gated delta
+    rule over the query tokens from S_ext (msa_gated_delta_rule).  States, selections and token
+    projections are seeded synthetic inputs; L2 is flushed before every step."""
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    import routed_sparse_attention_chunk_b200 as msa
+    cfg = workload_config(args)
+    dt = cfg.torch_dtype
+    Hk, Hv = DGA_HEADS
+    d = 128
+    B, T = cfg.B, cfg.Tq
+    Dst = min(cfg.D, 4096)
+    g = torch.Generator(device=device).manual_seed(23 + 1000 * rank)
+    states = torch.empty((Dst, Hv, d, d), dtype=dt, device=device)
+    for i in range(0, Dst, 256):
+        states[i:i + 256] = (0.1 * torch.randn((min(256, Dst - i), Hv, d, d), generator=g, device=device)).to(dt)
+    sel = torch.stack([torch.randperm(Dst, generator=g, device=device)[:cfg.k] for _ in range(B)]).to(torch.int32)
+    kk = torch.randn((B, T, Hk, d), generator=g, device=device)
+    kk = (kk / kk.norm(dim=-1, keepdim=True)).to(dt)
+    q = (torch.randn((B, T, Hk, d), generator=g, device=device) * 0.35).to(dt)
+    v = torch.randn((B, T, Hv, d), generator=g, device=device).to(dt)
+    lg = -0.3 * torch.rand((B, T, Hv), generator=g, device=device)
+    beta = torch.rand((B, T, Hv), generator=g, device=device)
+    S_ext = torch.empty((B, Hv, d, d), dtype=torch.float32, device=device)
+    o = torch.empty((B, T, Hv, d), dtype=dt, device=device)
+    flag = torch.zeros(1, dtype=torch.int32, device=device)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        msa.state_gather_sum(states, sel, S_ext, err_flag=flag)
+        if ev is not None:
+            ev.record(stream)
+        msa.gated_delta_rule(q, kk, v, lg, beta, o, S_ext)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    sampler = ClockSampler(device)
+    sampler.start()
+    n0 = msa.kernel_launch_count()
+    marks = []
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        step(e1)
+        e2.record(stream)
+        marks.append((e0, e1, e2))
+    torch.cuda.synchronize()
+    launches = msa.kernel_launch_count() - n0
+    clocks = sampler.stop()
+    sum_ms = [a.elapsed_time(b) for a, b, _ in marks]
+    gdr_ms = [b.elapsed_time(c) for _, b, c in marks]
+    step_local = sum(sum_ms) + sum(gdr_ms)
+    barrier(world, device)
+    ms_per_step = max_over_ranks(step_local, world, device) / args.steps
+    value = B * T * world / (ms_per_step / 1e3)
+    per = float(np.mean(gdr_ms))
+    flops = 6.0 * d * d * Hv * B * T  # per token and value head: k^T h, the rank-1 update and h^T q
+    mhz = clocks.get("sm_max_mhz") or 1965
+    peak = torch.cuda.get_device_properties(device).multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
+    S = Hv * d * d
+    sum_bytes = B * cfg.k * S * states.element_size() + B * S * 4
+    peaks, peak_kind = load_peaks()
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype + " inputs, f32 state", "data": "synthetic",
+        "config": {"workload": workload_label(cfg),
+                   "step": f"linear (DGA) layer memory path: msa_state_gather_sum of {cfg.k} selected documents' "
+                           f"states ({Hv} x {d} x {d}, from a bank of {Dst}) then msa_gated_delta_rule over {T} "
+                           f"query tokens x {B} queries ({Hk} key heads, {Hv} value heads, d = {d})",
+                   "l2": "flushed before every step", "parallelism": "single GPU"},
+        "roofline": {"bound": "alu", "achieved": round(flops / per / 1e9, 2), "peak": round(peak, 1),
+                     "unit": "TFLOP/s", "kernel": "gdr_chunk_kernel (msa_gated_delta_rule)",
+                     "alg_flops_per_launch": flops,
+                     "peak_source": "derived: SMs x 128 fp32 lanes x 2 x max SM clock",
+                     "frac": round(flops / per / 1e9 / peak, 4), "avg_launch_ms": round(per, 4), "traffic": None},
+        "stages": {"state_gather_sum": {"ms_per_launch": round(float(np.mean(sum_ms)), 4),
+                                        "achieved": round(sum_bytes / float(np.mean(sum_ms)) / 1e6, 2),
+                                        "unit": "GB/s", "peak": peaks["hbm_gbs"], "peak_source": f"{peak_kind} hbm_gbs"},
+                   "gated_delta_rule": {"ms_per_launch": round(per, 4)}},
+        "gpu_launches": launches, "clocks": clocks, "err_flag": int(flag.item()),
+    }
+
+
 def run_gpu(args, rank, local_rank, world):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -569,10 +847,10 @@ def run_gpu(args, rank, local_rank, world):
     step_kind = step_kind_for(cfg, args)
     peaks, peak_kind = load_peaks()
     counts = workload_counts(cfg)
-    w = MSAWorkload(cfg, device, seed=1000 * rank, step_kind=step_kind, bank_kv=args.bank_kv)
+    w = MSAWorkload(cfg, device, seed=1000 * rank, step_kind=step_kind, bank_kv=args.bank_kv,
+                    unfused=args.unfused or args.bank_kv == "host")
     in_bytes = sum(t.numel() * t.element_size() for t in w.input_tensors())
-    if step_kind == "query":
-        in_bytes += w.Krb.numel() * w.Krb.element_size()  # the scan reads the whole bank every step
+    in_bytes += w.Krb.numel() * w.Krb.element_size()  # the scan reads the whole bank every step
     flush = None if in_bytes > L2_BYTES else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
 
     if args.pipeline:
@@ -582,39 +860,7 @@ def run_gpu(args, rank, local_rank, world):
         return run_pipelined(args, rank, world, device, w, cfg, counts, peaks, peak_kind, flush)
 
     # ---- warm-up, then exactly K timed steps, an event after every stage
-    stream = torch.cuda.current_stream()
-    sampler = ClockSampler(device)
-    for _ in range(args.warmup):
-        w.step()
-    torch.cuda.synchronize()
-    barrier(world, device)
-    sampler.start()
-    n0 = msa.kernel_launch_count()
-    marks = []  # (stage, event) in launch order
-
-    def rec(stage):
-        e = torch.cuda.Event(enable_timing=True)
-        e.record(stream)
-        marks.append((stage, e))
-
-    starts = []
-    t_all0, t_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    t_all0.record(stream)
-    for i in range(args.steps):
-        if flush is not None:
-            flush.fill_(1.0)
-        rec("start")
-        w.step(rec)
-    t_all1.record(stream)
-    torch.cuda.synchronize()
-    launches = msa.kernel_launch_count() - n0
-    clocks = sampler.stop()
-    stage_ms = {s: [] for s in MSAWorkload.STAGES}
-    for (s0, e0), (s1, e1) in zip(marks[:-1], marks[1:]):
-        if s1 != "start":
-            stage_ms[s1].append(e0.elapsed_time(e1))
-    timed_ms = t_all0.elapsed_time(t_all1)
+    stage_ms, timed_ms, clocks, launches = timed_steps(w, args.steps, args.warmup, flush, world, device)
     step_sum = sum(sum(v) for v in stage_ms.values())
     step_ms_local = step_sum if flush is not None else timed_ms
     flag = int(w.flag.item())
@@ -637,11 +883,13 @@ def run_gpu(args, rank, local_rank, world):
                          "sparse_attn": "attn_decode.cu" if cfg.Tq == 1 else "attn_tc.cu",
                          "gather": "gather.cu"}[dom], cfg.name)
     roofline["traffic"] = tr["dram_bytes_per_launch"] if tr else None
-    stages = {s: {"ms_per_launch": round(per_launch[s], 4), "share": round(totals[s] / step_sum, 4),
-                  **{k: (round(v, 2) if isinstance(v, float) else v)
-                     for k, v in stage_roofline(s, per_launch[s], cfg, counts, peaks, peak_kind, long_region).items()
-                     if k in ("bound", "achieved", "unit")}}
-              for s in per_launch}
+    if roofline["bound"] == "hbm" and world == 1:
+        rs = read_stream_gbs(device)
+        roofline["read_stream_gbs"] = round(rs, 1)
+        roofline["frac_of_read_stream"] = round(roofline["achieved"] / rs, 4)
+        roofline["read_stream_source"] = "measured in this run: torch sum over a 4 GiB bf16 tensor, best of 5"
+    stages = {s: stage_entry(s, v, cfg, counts, peaks, peak_kind, long_region, clocks, step_sum)
+              for s, v in stage_ms.items() if v}
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -652,6 +900,7 @@ def run_gpu(args, rank, local_rank, world):
         d2h = sum(t.numel() * t.element_size() for t in host_out)
         dev_in, dev_out = w.input_tensors(), w.output_tensors()
         n_e2e = max(1, min(args.steps, args.e2e_steps))
+        stream = torch.cuda.current_stream()
         barrier(world, device)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -674,7 +923,7 @@ def run_gpu(args, rank, local_rank, world):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded generators; see workloads/synth.py)",
         "config": {"workload": workload_label(cfg),
-                   "step": step_label(step_kind),
+                   "step": step_label(step_kind, w.unfused),
                    **({"bank_kv": "pinned host memory, read in place by msa_gather"} if args.bank_kv == "host" else {}),
                    "l2": "inputs larger than L2" if flush is None else "L2 flushed between steps (not timed)",
                    "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
@@ -686,6 +935,20 @@ def run_gpu(args, rank, local_rank, world):
         "clocks": clocks,
         "err_flag": flag,
     }
+    if step_kind == "query" and w.slab_pool_ms:
+        result["offline_pool"] = slab_pool_entry(w, cfg, counts, peaks, peak_kind)
+    extra = [x for x in (args.extra.split(",") if args.extra not in (None, "", "none") else [])
+             if x and x != cfg.name]
+    for x in extra:
+        if x not in synth.CONFIGS:
+            raise SystemExit(f"--extra: unknown workload {x}")
+    if extra and world == 1 and args.bank_kv == "device" and not args.docs:
+        del w
+        torch.cuda.empty_cache()
+        result["workloads"] = {}
+        for name in extra:
+            result["workloads"][name] = workload_extra(name, device, 0, peaks, peak_kind,
+                                                       EXTRA_STEPS.get(name, 20), 3)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_budget, with_pool=step_kind == "full")
     if world > 1:
@@ -814,42 +1077,58 @@ def run_pipelined(args, rank, world, device, w, cfg, counts, peaks, peak_kind, f
 
 
 # ----------------------------------------------------------------------------- CPU oracle arm
-def oracle_step_sample(cfg: synth.Config, docs: int, tokens: int, seed: int = 0, with_pool: bool = True):
-    """Time the oracle on a bounded sample of one step; returns (estimated full-step seconds, sample text).
+def oracle_step_sample(cfg: synth.Config, docs: int, tokens: int, seed: int = 0, with_pool: bool = True,
+                       rdocs: int = 0):
+    """Time the oracle on a bounded sample of one step; returns (estimated full-step seconds, sample text,
+    sample wall seconds).
 
-    Pool: `docs` documents' raw tokens (time scaled by D / docs).  Query path of
-    layer 0 (route over the full-size bank, top-k, gather, attention) for
-    `tokens` query tokens (time scaled by Tq / tokens), times the layer count.
+    Pool (only when the step includes it): `docs` documents' raw tokens, time
+    scaled by D / docs.  Query path of layer 0 for `tokens` query tokens: the
+    route over the chunks of `rdocs` documents (time scaled by C / their chunks
+    and by Tq / tokens), the top-k over those documents' scores (scaled by
+    D / rdocs), then gather + attention (scaled by Tq / tokens); times the
+    layer count.
     """
     from oracle import msa_oracle as O
     wall0 = time.perf_counter()
     docs = max(1, min(docs, cfg.D))
     tokens = max(1, min(tokens, cfg.Tq))
-    sub = cfg.scaled(D=docs, last_len=None, docs_per_slab=0, planted_doc=-1)
-    K, V, Kr = synth.gen_raw_slab(sub, 0, docs, "cpu", seed)
-    off = synth.doc_tok_offsets(sub)
-    t0 = time.perf_counter()
+    rdocs = max(cfg.k, min(rdocs or cfg.D, cfg.D))
+    t_pool = 0.0
     if with_pool:
+        sub = cfg.scaled(D=docs, last_len=None, docs_per_slab=0, planted_doc=-1)
+        K, V, Kr = synth.gen_raw_slab(sub, 0, docs, "cpu", seed)
+        off = synth.doc_tok_offsets(sub)
+        t0 = time.perf_counter()
         O.pool(K.double().numpy(), V.double().numpy(), Kr.double().numpy(), off, cfg.P, cfg.theta,
                out_bf16=cfg.dtype == "bf16")
-    t_pool = (time.perf_counter() - t0) * cfg.D / docs
-    # full-size bank for the query path (drawn, not pooled: only the time is used)
-    rng = np.random.default_rng(seed)
-    Krb = rng.standard_normal((cfg.C, cfg.Hr, cfg.dr)).astype(np.float32).astype(np.float64)
+        t_pool = (time.perf_counter() - t0) * cfg.D / docs
+    # a bank of the first rdocs documents' chunks (drawn, not pooled: only the time is used)
     coff = O.chunk_offsets(synth.doc_tok_offsets(cfg), cfg.P)
+    scoff = coff[: rdocs + 1]
+    Cs = int(scoff[-1])
+    rng = np.random.default_rng(seed)
+    Krb = rng.standard_normal((Cs, cfg.Hr, cfg.dr)).astype(np.float32).astype(np.float64)
+    Kb = rng.standard_normal((Cs, cfg.Hkv, cfg.d)).astype(np.float32)
     q = synth.gen_query(cfg.scaled(Tq=tokens, Lloc=max(tokens, cfg.Lloc - cfg.Tq + tokens)), 0, "cpu", seed)
-    Kb = rng.standard_normal((cfg.C, cfg.Hkv, cfg.d)).astype(np.float32)
     t0 = time.perf_counter()
-    ds = O.route(q["Qr"].double().numpy(), Krb, coff)
+    ds = O.route(q["Qr"].double().numpy(), Krb, scoff)
+    t_route = (time.perf_counter() - t0) * (cfg.C / Cs) * (cfg.Tq / tokens)
+    t0 = time.perf_counter()
     idx, _ = O.topk(ds, cfg.k)
-    Km, Vm, ml = O.gather(idx, coff, Kb, Kb, cfg.Mmax)
+    t_topk = (time.perf_counter() - t0) * cfg.D / rdocs
+    t0 = time.perf_counter()
+    Km, Vm, ml = O.gather(idx, scoff, Kb, Kb, cfg.Mmax)
     O.attention(q["Q"].double().numpy(), q["Kloc"].double().numpy(), q["Vloc"].double().numpy(), Km, Vm, ml)
-    t_query = (time.perf_counter() - t0) * cfg.Tq / tokens * cfg.layers
+    t_attn = (time.perf_counter() - t0) * cfg.Tq / tokens
+    est = t_pool + (t_route + t_topk + t_attn) * cfg.layers
     text = ((f"oracle (numpy fp64) pool of {docs} of {cfg.D} documents scaled x{cfg.D / docs:.0f}; " if with_pool
-             else "oracle (numpy fp64), bank pooled outside the step; ") + f"route over all "
-            f"{cfg.C} chunks + top-k + gather + attention for {tokens} of {cfg.Tq} query tokens scaled "
-            f"x{cfg.Tq / tokens:.0f}" + (f" and x{cfg.layers} layers" if cfg.layers > 1 else ""))
-    return t_pool + t_query, text, time.perf_counter() - wall0
+             else "oracle (numpy fp64), bank pooled outside the step; ") +
+            f"route over {Cs} of {cfg.C} chunks ({rdocs} of {cfg.D} documents) for {tokens} of {cfg.Tq} query "
+            f"tokens scaled x{cfg.C / Cs:.1f} x{cfg.Tq / tokens:.0f}, top-k scaled x{cfg.D / rdocs:.1f}, gather + "
+            f"attention for {tokens} tokens scaled x{cfg.Tq / tokens:.0f}" +
+            (f", x{cfg.layers} layers" if cfg.layers > 1 else ""))
+    return est, text, time.perf_counter() - wall0
 
 
 def blas_threads() -> int:
@@ -862,10 +1141,11 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(cfg: synth.Config, budget_s: float = 20.0, with_pool: bool = True) -> dict:
-    docs, tokens = 8, 16
-    _, _, wall = oracle_step_sample(cfg, docs, tokens, with_pool=with_pool)           # calibration run
+    docs, tokens, rdocs = 8, 16, 512
+    _, _, wall = oracle_step_sample(cfg, docs, tokens, with_pool=with_pool, rdocs=rdocs)   # calibration run
     grow = max(1.0, min(16.0, budget_s / max(wall, 1e-3)))
-    est, text, wall = oracle_step_sample(cfg, int(docs * grow), int(tokens * grow), with_pool=with_pool)
+    est, text, wall = oracle_step_sample(cfg, int(docs * grow), int(tokens * grow), with_pool=with_pool,
+                                         rdocs=int(rdocs * grow))
     return {"value": round(cfg.B * cfg.Tq / est, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": text + f"; sample wall {wall:.1f} s; host {os.cpu_count()} logical CPUs"}
 
@@ -878,16 +1158,16 @@ def run_reference(args, rank, world):
     kind = step_kind_for(cfg, args)
     wp = kind == "full"
     per_step = max(0.2, min(10.0, args.ref_budget / max(1, args.steps + args.warmup)))
-    docs, tokens = 2, 4
-    _, _, wall = oracle_step_sample(cfg, docs, tokens, with_pool=wp)   # calibration (counts as warm-up)
+    docs, tokens, rdocs = 2, 4, 256
+    _, _, wall = oracle_step_sample(cfg, docs, tokens, with_pool=wp, rdocs=rdocs)   # calibration (a warm-up)
     grow = max(1.0, min(32.0, per_step / max(wall, 1e-3)))
-    docs, tokens = int(docs * grow), int(tokens * grow)
+    docs, tokens, rdocs = int(docs * grow), int(tokens * grow), int(rdocs * grow)
     for _ in range(max(0, args.warmup - 1)):
-        oracle_step_sample(cfg, docs, tokens, with_pool=wp)
+        oracle_step_sample(cfg, docs, tokens, with_pool=wp, rdocs=rdocs)
     ests, texts = [], None
     wall0 = time.perf_counter()
     for _ in range(args.steps):
-        e, texts, _ = oracle_step_sample(cfg, docs, tokens, with_pool=wp)
+        e, texts, _ = oracle_step_sample(cfg, docs, tokens, with_pool=wp, rdocs=rdocs)
         ests.append(e)
     wall = time.perf_counter() - wall0
     est = float(np.mean(ests))
@@ -909,15 +1189,20 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="1m", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--workload", default="100m", choices=sorted(synth.CONFIGS))
     ap.add_argument("--docs", type=int, default=0, help="use only this many documents (smaller profiling case)")
     ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time msa_gather and msa_sparse_attn (copied rows) instead of msa_sparse_attn_indexed")
+    ap.add_argument("--extra", default=None,
+                    help="comma-separated workloads whose stage results join the line (one GPU only), or none; "
+                         "default: " + ",".join(EXTRA_WORKLOADS) + " with the default 100m workload, none otherwise")
     ap.add_argument("--step", choices=["full", "query"], default=None,
                     help="full: pool + query path per step; query: bank pooled before timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which_pass", choices=["forward", "backward", "state"], default="forward",
+    ap.add_argument("--pass", dest="which_pass", choices=["forward", "backward", "state", "dga"], default="forward",
                     help="backward: time the backward of the query path instead of the forward step; "
                          "state: the linear layers' memory injection (sum of the selected documents' states)")
     ap.add_argument("--bank-kv", choices=["device", "host"], default="device",
@@ -927,6 +1212,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)
     args = ap.parse_args()
+    if args.extra is None:
+        args.extra = ",".join(EXTRA_WORKLOADS) if (args.workload == "100m" and not args.docs) else ""
     if args.warmup < 3 and args.impl == "msa":
         ap.error("--warmup must be >= 3")
     rank, local_rank, world = dist_env()
@@ -936,6 +1223,8 @@ def main():
         res = run_backward(args, rank, local_rank, world)
     elif args.which_pass == "state":
         res = run_state(args, rank, local_rank, world)
+    elif args.which_pass == "dga":
+        res = run_dga(args, rank, local_rank, world)
     else:
         res = run_gpu(args, rank, local_rank, world)
     if rank == 0 and res is not None:

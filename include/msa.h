@@ -13,13 +13,19 @@
  *   4. msa_gather       - copy the selected documents' pooled K/V chunks.
  *   5. msa_sparse_attn  - GQA softmax attention of the query tokens over
  *                         [selected memory rows ++ causal local KV].
- *   msa_layer_forward   - steps 2-5 in one call, with the gathered chunks kept
- *                         in the caller's workspace.
+ *   4.+5. msa_sparse_attn_indexed - the same attention with the selected
+ *                         chunks read in place from the bank by index (no
+ *                         gathered copy).
+ *   msa_layer_forward   - steps 2-5 in one call: msa_route_topk, then
+ *                         msa_sparse_attn_indexed.
+ * msa_interleave_forward runs several such rounds (the pages' Memory
+ * Interleave for multi-hop questions).
  * Beyond the forward path: the backward of steps 5, 4 and 2
  * (msa_sparse_attn_backward, msa_gather_backward, msa_route_backward), the sum
  * of the selected documents' recurrent states that the linear (DGA) layers
  * take as their initial state (msa_state_gather_sum, from the "MSA x Qwen3.5"
- * model card), and a routing entry point that allocates nothing
+ * model card) and the gated delta rule that starts from it
+ * (msa_gated_delta_rule), and a routing entry point that allocates nothing
  * (msa_route_topk_noalloc).
  *
  * Conventions shared by every entry point
@@ -90,6 +96,17 @@ const char* msa_version(void);
  * (memsets and copies are not kernels and are not counted).  For accounting:
  * the difference across a region is the number of library kernels it ran. */
 uint64_t msa_kernel_launch_count(void);
+
+/* For tests of the device-side error path only.  Sets how many times the
+ * bf16 prefill attention kernel (msa_sparse_attn and the index-driven
+ * attention on prefill shapes) polls each barrier wait that paces its
+ * pipeline; a negative value restores the default (2^24).  With 0 every such
+ * wait expires at once: the kernel then waits (with the default bound) for the
+ * copies and tensor-core operations it already issued, frees its tensor
+ * memory, raises MSA_FLAG_TIMEOUT in *err_flag and returns; the outputs of
+ * that call are undefined and the next call with the default is unaffected.
+ * Process-wide; set it only while no other thread launches the library. */
+void msa_testing_set_wait_polls(int64_t polls);
 
 /* ------------------------------------------------------------------------
  * RoPE table (host).  Fills host_out[max_len][d/2][2] with (cos, sin) of the
@@ -263,6 +280,47 @@ msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const 
                            void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Steps 4 and 5 fused: attention over the selected documents' chunks read in
+ * place from the bank ("Inference Pipeline" stage 2: load only the selected
+ * K̄ / V̄ and concatenate them with the local context; "MSA x Qwen3.5" card,
+ * "Architecture summary").  The result is that of msa_gather followed by
+ * msa_sparse_attn with the same Mmax: query b's memory rows are the chunks of
+ * documents topk_idx[b, 0..k) in rank order (each document's chunks in
+ * ascending order), at most Mmax of them (more raise MSA_FLAG_OVERFLOW and
+ * the rows past Mmax are dropped), followed by its causal local rows.
+ *   Q, Kloc, Vloc, O, lse, scale as in msa_sparse_attn;
+ *   topk_idx int32 [B, k];  doc_chunk_off int64 [D+1];
+ *   Kbar, Vbar [C, Hkv, d] dtype dt (device memory, or page-locked host memory
+ *   as for msa_gather).
+ * For bf16, d = 128 and the shapes the tensor-core kernels take (decode: up to
+ * 16 query rows per KV head; prefill: a GQA group that divides 128 rows), a
+ * small plan kernel cuts every query's selection into runs of at most 8
+ * consecutive chunk rows of one document, and the attention kernel loads those
+ * runs straight from the bank with TMA.  A run shorter than 8 rows is padded
+ * with masked rows, and decode shapes reserve memory tiles for such padding,
+ * so the floating-point summation order (not the keys, not the weights) can
+ * differ from msa_sparse_attn's; for prefill shapes and documents whose chunk
+ * counts are multiples of 8 the two agree bit for bit.  Other shapes, fp32,
+ * and banks in host memory gather the rows into the workspace first and run
+ * msa_sparse_attn's kernels.
+ * Workspace: msa_sparse_attn_indexed_workspace_size bytes, 16-byte aligned;
+ * like msa_sparse_attn's, it depends on the current device's SM count for
+ * decode shapes.  Its contents need no initialisation and are not kept.
+ * Errors as msa_sparse_attn plus MSA_ERR_INVALID_ARG for k < 1, D < 1, C < 0,
+ * missing index / offset / bank pointers, or pageable host banks;
+ * MSA_ERR_UNSUPPORTED for k > 65535.  Device flags: MSA_FLAG_INDEX_OOB for a
+ * document index outside [0, D) or a chunk range outside [0, C) (that
+ * document is skipped), MSA_FLAG_OVERFLOW as above.
+ * ---------------------------------------------------------------------- */
+size_t msa_sparse_attn_indexed_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int k, int Mmax);
+msa_status msa_sparse_attn_indexed(msa_dtype dt, const void* Q, const void* Kloc, const void* Vloc,
+                                   int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d,
+                                   const int32_t* topk_idx, int k, const int64_t* doc_chunk_off, int64_t D,
+                                   int64_t C, const void* Kbar, const void* Vbar, int Mmax, float scale,
+                                   void* O, float* lse, void* ws, size_t ws_bytes, int32_t* err_flag,
+                                   msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Backward of step 5.  MSA is trained end to end through its sparse attention
  * ("MSA: Memory Sparse Attention" README, "Architecture"; Figure 2 caption);
  * the pages print no gradient, so this is the exact derivative of
@@ -275,8 +333,11 @@ msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const 
  * lse (fp32 [B, Hq, Tq], required) and dO (dtype dt, [B, Tq, Hq, d]).  Outputs
  * are fp32 and fully written: dQ [B, Tq, Hq, d]; dKloc, dVloc [B, Lloc, Hkv, d];
  * dKmem, dVmem [B, Mmax, Hkv, d] (rows past mem_len[b] are zero).  The
- * workspace holds D (msa_sparse_attn_backward_workspace_size bytes).  CUDA-core
- * kernels, fp32 arithmetic.  Device flags as in msa_sparse_attn.
+ * workspace holds D (msa_sparse_attn_backward_workspace_size bytes).  bf16
+ * with d = 128 and the forward's tensor-core GQA shapes runs on tcgen05 kernels
+ * (S, dP, dQ, dK and dV contractions on the tensor cores, fp32 accumulators in
+ * TMEM); fp32 inputs, d = 64 and other shapes run on CUDA-core kernels with
+ * fp32 arithmetic.  Device flags as in msa_sparse_attn.
  * ---------------------------------------------------------------------- */
 size_t msa_sparse_attn_backward_workspace_size(int64_t B, int Tq, int Hq);
 msa_status msa_sparse_attn_backward(msa_dtype dt, const void* Q, const void* Kloc, const void* Vloc,
@@ -333,13 +394,15 @@ msa_status msa_route_backward(msa_dtype dt, const void* Qr, int64_t B, int Tq, i
                               void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * Steps 2-5 for one layer in one call: route + top-k, the selected chunks
- * copied into the workspace (the msa_gather kernel), then attention over them
- * and the local KV.  Arguments as in msa_route_topk and msa_sparse_attn; Mmax
- * bounds the memory rows per query (selected chunks past it are dropped and
- * flagged MSA_FLAG_OVERFLOW).  topk_idx is required (it is the layer's routing
- * output); doc_scores, topk_score and lse may be NULL.  The workspace size is
- * computed for fp32 storage and so also covers bf16.
+ * Steps 2-5 for one layer in one call ("Inference Pipeline" stage 2): route +
+ * top-k (msa_route_topk), then attention over the selected documents' chunks,
+ * read in place from the bank by index, and the local KV
+ * (msa_sparse_attn_indexed).  Arguments as in those two calls; Mmax bounds the
+ * memory rows per query (selected chunks past it are dropped and flagged
+ * MSA_FLAG_OVERFLOW).  topk_idx is required (it is the layer's routing
+ * output); doc_scores, topk_score and lse may be NULL.  The workspace is the
+ * two calls' workspaces side by side (sized for fp32 storage, so it also
+ * covers bf16).
  * ---------------------------------------------------------------------- */
 size_t msa_layer_forward_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d,
                                         int Hr, int64_t D, int64_t C, int k, int Mmax);
@@ -353,6 +416,49 @@ msa_status msa_layer_forward(msa_dtype dt,
                              void* O, float* lse, int32_t* topk_idx, float* topk_score,
                              float* doc_scores,
                              void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Memory Interleave ("MSA: Memory Sparse Attention" README, Figure 3 caption:
+ * an optional multi-round interleave after online routing, for multi-hop
+ * questions; FAQ "What is Memory Interleave?": multi-round reasoning that
+ * jumps across scattered memory segments).  The pages describe it in words
+ * only; this library reads it as R rounds of the layer's memory path in which
+ * each round retrieves k further documents and reasons over all of them:
+ *   round r = 0 .. R-1:
+ *     doc_score = routing of Qr_r over the bank (as msa_route_topk)
+ *     S_r       = the k best documents not selected in rounds 0 .. r-1
+ *                 (documents of earlier rounds score -inf; same order and ties
+ *                 as msa_route_topk)
+ *     O_r       = attention over the chunks of S_0 ++ S_1 ++ ... ++ S_r (round
+ *                 order, then rank order; at most Mmax rows, more raise
+ *                 MSA_FLAG_OVERFLOW) ++ the causal local KV
+ *                 (msa_sparse_attn_indexed)
+ *     Qr_{r+1}  = O_r [B * Tq, Hq * d] x W_route [Hq * d, Hr * dr]  (the
+ *                 caller's round-to-round map of the attention output to the
+ *                 next router query; fp32 accumulation, stored in dtype dt)
+ *   Qr0 [B, Tq, Hr, dr], W_route (required when rounds > 1) dtype dt.
+ *   O, lse: the last round's output and log-sum-exp (lse may be NULL).
+ *   O_rounds: NULL or [rounds - 1, B, Tq, Hq, d], the earlier rounds' outputs.
+ *   Qr_rounds: NULL or [rounds - 1, B, Tq, Hr, dr] (dtype dt), the router
+ *   queries of rounds 1 .. rounds-1 as the map stored them.
+ *   topk_idx int32 [B, rounds * k] (required): round r's selection in columns
+ *   [r k, (r + 1) k);  topk_score fp32 [B, rounds * k] or NULL.
+ * Requires rounds * k <= D and B * Tq <= 1,048,560; the rest as
+ * msa_layer_forward.  R = 1 is msa_layer_forward.  Workspace:
+ * msa_interleave_workspace_size bytes (its contents need no initialisation).
+ * ---------------------------------------------------------------------- */
+size_t msa_interleave_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Hr, int dr,
+                                     int64_t D, int64_t C, int k, int rounds, int Mmax);
+msa_status msa_interleave_forward(msa_dtype dt, const void* Qr0, int Hr, int dr,
+                                  const void* Krbar, const float* kr_rnorm,
+                                  const int64_t* doc_chunk_off, int64_t D, int64_t C, int k, int rounds,
+                                  const void* W_route,
+                                  const void* Q, const void* Kloc, const void* Vloc,
+                                  int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d,
+                                  const void* Kbar, const void* Vbar, int Mmax, float scale,
+                                  void* O, float* lse, void* O_rounds, void* Qr_rounds,
+                                  int32_t* topk_idx, float* topk_score,
+                                  void* ws, size_t ws_bytes, int32_t* err_flag, msa_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Memory injection of the linear (DGA) layers ("MSA x Qwen3.5" model card,
@@ -372,6 +478,30 @@ msa_status msa_layer_forward(msa_dtype dt,
 msa_status msa_state_gather_sum(msa_dtype dt, const void* states, int64_t D, int64_t S,
                                 const int32_t* topk_idx, int64_t B, int k, float* S_ext,
                                 int32_t* err_flag, msa_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The linear (DGA) layers' query path ("MSA x Qwen3.5" model card,
+ * "Architecture summary": the summed state S_ext of the selected documents is
+ * the initial state of the query path's chunked gated delta rule).  The pages
+ * do not define the rule; this is the recurrence of Gated DeltaNet (Yang,
+ * Kautz and Hatamizadeh, "Gated Delta Networks: Improving Mamba2 with Delta
+ * Rule", ICLR 2025), per value head with the state h (key dim x value dim):
+ *   h_t = exp(g_t) (I - beta_t k_t k_t^T) h_{t-1} + beta_t k_t v_t^T
+ *   o_t = h_t^T (scale q_t)          (scale <= 0 means 1/sqrt(dk))
+ * h_0 = h0 (S_ext from msa_state_gather_sum, whose states are laid out
+ * [Hv, dk, dv]; NULL means zeros).  Value head h reads key head h / (Hv / Hk).
+ *   q, k [B, T, Hk, dk];  v [B, T, Hv, dv];  o [B, T, Hv, dv]   dtype dt
+ *   g (log gates, <= 0), beta [B, T, Hv] fp32;  h0, hT fp32 [B, Hv, dk, dv]
+ *   (hT, the state after the last token, may be NULL).
+ * Keys are used as given (the model normalises them before the rule).
+ * Computed chunk by chunk (64 tokens) in fp32 on the CUDA cores, one CTA per
+ * (value head, query): the within-chunk products, a unit lower-triangular
+ * solve for the chunk's new values, then the state update.
+ * Supported: dk = dv = 128, Hv % Hk == 0, B <= 65535.  No workspace.
+ * ---------------------------------------------------------------------- */
+msa_status msa_gated_delta_rule(msa_dtype dt, const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, int64_t B, int T, int Hk, int Hv, int dk, int dv,
+                                const float* h0, float scale, void* o, float* hT, msa_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -63,6 +63,12 @@ def kernel_launch_count() -> int:
     return int(_lib.load().msa_kernel_launch_count())
 
 
+def testing_set_wait_polls(polls: int) -> None:
+    """Test hook (msa_testing_set_wait_polls): polls of the prefill attention kernel's pipeline
+    waits; 0 makes every such wait expire at once, a negative value restores the default."""
+    _lib.load().msa_testing_set_wait_polls(int(polls))
+
+
 def rope_table(theta: float, d: int, max_len: int) -> torch.Tensor:
     """Host fp32 [max_len, d/2, 2] table of (cos, sin) built in fp64 by the library."""
     out = torch.empty((max_len, d // 2, 2), dtype=torch.float32)
@@ -163,6 +169,23 @@ def sparse_attn(Q, Kloc, Vloc, Kmem, Vmem, mem_len, O, lse=None, scale=0.0, ws=N
           0 if ws is None else ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))
 
 
+def sparse_attn_indexed_workspace_size(B, Tq, Lloc, Hq, Hkv, d, k, Mmax) -> int:
+    return _lib.load().msa_sparse_attn_indexed_workspace_size(B, Tq, Lloc, Hq, Hkv, d, k, Mmax)
+
+
+def sparse_attn_indexed(Q, Kloc, Vloc, topk_idx, doc_chunk_off, Kbar, Vbar, Mmax, O, ws, lse=None, scale=0.0,
+                        err_flag=None, stream=None):
+    """Steps 4+5 fused (msa_sparse_attn_indexed): attention over the selected documents' chunks,
+    read in place from the bank K̄ / V̄ [C, Hkv, d] by index, and the causal local rows."""
+    B, Tq, Hq, d = Q.shape
+    k = topk_idx.shape[1]
+    _call("msa_sparse_attn_indexed", _dt(Q), _p(Q), _p(Kloc, Q.dtype), _p(Vloc, Q.dtype), B, Tq, Kloc.shape[1], Hq,
+          Kloc.shape[2], d, _p(topk_idx, torch.int32), k, _p(doc_chunk_off, torch.int64), doc_chunk_off.numel() - 1,
+          Kbar.shape[0], _p(Kbar, Q.dtype, host_ok=True), _p(Vbar, Q.dtype, host_ok=True), Mmax, float(scale),
+          _p(O, Q.dtype), _p(lse, torch.float32), _p(ws), ws.numel() * ws.element_size(),
+          _p(err_flag, torch.int32), _s(stream))
+
+
 def sparse_attn_backward_workspace_size(B, Tq, Hq) -> int:
     return _lib.load().msa_sparse_attn_backward_workspace_size(B, Tq, Hq)
 
@@ -211,7 +234,8 @@ def layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax) -> 
 
 def layer_forward(Qr, Krbar, kr_rnorm, doc_chunk_off, k, Q, Kloc, Vloc, Kbar, Vbar, Mmax, O, topk_idx, ws,
                   lse=None, topk_score=None, doc_scores=None, scale=0.0, err_flag=None, stream=None):
-    """Steps 2-5 fused (msa_layer_forward): memory rows read from the bank by index."""
+    """Steps 2-5 in one call (msa_layer_forward): route + top-k, then attention over the selected
+    documents' chunks read in place from the bank by index (msa_sparse_attn_indexed)."""
     B, Tq, Hr, dr = Qr.shape
     Hq, d = Q.shape[2], Q.shape[3]
     _call("msa_layer_forward", _dt(Qr), _p(Qr), Hr, dr, _p(Krbar, Qr.dtype), _p(kr_rnorm, torch.float32),
@@ -221,3 +245,35 @@ def layer_forward(Qr, Krbar, kr_rnorm, doc_chunk_off, k, Q, Kloc, Vloc, Kbar, Vb
           _p(lse, torch.float32),
           _p(topk_idx, torch.int32), _p(topk_score, torch.float32), _p(doc_scores, torch.float32),
           _p(ws), ws.numel() * ws.element_size(), _p(err_flag, torch.int32), _s(stream))
+
+
+def interleave_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, dr, D, C, k, rounds, Mmax) -> int:
+    return _lib.load().msa_interleave_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, dr, D, C, k, rounds, Mmax)
+
+
+def interleave_forward(Qr0, Krbar, kr_rnorm, doc_chunk_off, k, rounds, W_route, Q, Kloc, Vloc, Kbar, Vbar, Mmax, O,
+                       topk_idx, ws, lse=None, O_rounds=None, Qr_rounds=None, topk_score=None, scale=0.0,
+                       err_flag=None, stream=None):
+    """Memory Interleave (msa_interleave_forward): `rounds` rounds of route -> k new documents ->
+    attention over every round's documents; the next round's router query is O_r x W_route.
+    topk_idx int32 [B, rounds * k]; W_route [Hq * d, Hr * dr] (None when rounds == 1)."""
+    B, Tq, Hr, dr = Qr0.shape
+    Hq, d = Q.shape[2], Q.shape[3]
+    _call("msa_interleave_forward", _dt(Qr0), _p(Qr0), Hr, dr, _p(Krbar, Qr0.dtype), _p(kr_rnorm, torch.float32),
+          _p(doc_chunk_off, torch.int64), doc_chunk_off.numel() - 1, Krbar.shape[0], k, rounds,
+          _p(W_route, Qr0.dtype), _p(Q, Qr0.dtype), _p(Kloc, Qr0.dtype), _p(Vloc, Qr0.dtype), B, Tq, Kloc.shape[1],
+          Hq, Kloc.shape[2], d, _p(Kbar, Qr0.dtype, host_ok=True), _p(Vbar, Qr0.dtype, host_ok=True), Mmax,
+          float(scale), _p(O, Qr0.dtype), _p(lse, torch.float32), _p(O_rounds, Qr0.dtype), _p(Qr_rounds, Qr0.dtype),
+          _p(topk_idx, torch.int32), _p(topk_score, torch.float32), _p(ws), ws.numel() * ws.element_size(),
+          _p(err_flag, torch.int32), _s(stream))
+
+
+def gated_delta_rule(q, k, v, g, beta, o, h0=None, hT=None, scale=0.0, stream=None):
+    """The linear (DGA) layers' query path (msa_gated_delta_rule): the gated delta rule over the
+    query tokens from the initial state h0 (S_ext).  q, k [B, T, Hk, 128]; v, o [B, T, Hv, 128];
+    g, beta fp32 [B, T, Hv]; h0, hT fp32 [B, Hv, 128, 128] or None."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    f = torch.float32
+    _call("msa_gated_delta_rule", _dt(q), _p(q), _p(k, q.dtype), _p(v, q.dtype), _p(g, f), _p(beta, f), B, T, Hk, Hv,
+          dk, dv, _p(h0, f), float(scale), _p(o, q.dtype), _p(hT, f), _s(stream))

@@ -18,6 +18,7 @@ SIGNATURES = {
     "msa_status_string": (C.c_char_p, [C.c_int]),
     "msa_version": (C.c_char_p, []),
     "msa_kernel_launch_count": (C.c_uint64, []),
+    "msa_testing_set_wait_polls": (None, [I64]),
     "msa_rope_table_host": (C.c_int, [C.c_double, C.c_int, C.c_int, P]),
     "msa_chunk_offsets_host": (C.c_int, [P, I64, C.c_int, P]),
     "msa_pool": (C.c_int, [C.c_int, P, P, P, P, P, I64, I64, I64, C.c_int, C.c_int, C.c_int, C.c_int,
@@ -33,6 +34,10 @@ SIGNATURES = {
     "msa_sparse_attn_workspace_size": (SZ, [I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int]),
     "msa_sparse_attn": (C.c_int, [C.c_int, P, P, P, I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                   P, P, P, C.c_int, F32, P, P, P, SZ, P, P]),
+    "msa_sparse_attn_indexed_workspace_size": (SZ, [I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                                    C.c_int]),
+    "msa_sparse_attn_indexed": (C.c_int, [C.c_int, P, P, P, I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                          P, C.c_int, P, I64, I64, P, P, C.c_int, F32, P, P, P, SZ, P, P]),
     "msa_sparse_attn_backward_workspace_size": (SZ, [I64, C.c_int, C.c_int]),
     "msa_sparse_attn_backward": (C.c_int, [C.c_int, P, P, P, I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                            P, P, P, C.c_int, F32, P, P, P, P, P, P, P, P, P, SZ, P, P]),
@@ -46,7 +51,14 @@ SIGNATURES = {
     "msa_layer_forward": (C.c_int, [C.c_int, P, C.c_int, C.c_int, P, P, P, I64, I64, C.c_int,
                                     P, P, P, I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                     P, P, C.c_int, F32, P, P, P, P, P, P, SZ, P, P]),
+    "msa_interleave_workspace_size": (SZ, [I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                           I64, I64, C.c_int, C.c_int, C.c_int]),
+    "msa_interleave_forward": (C.c_int, [C.c_int, P, C.c_int, C.c_int, P, P, P, I64, I64, C.c_int, C.c_int, P,
+                                         P, P, P, I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                         P, P, C.c_int, F32, P, P, P, P, P, P, P, SZ, P, P]),
     "msa_state_gather_sum": (C.c_int, [C.c_int, P, I64, I64, P, I64, C.c_int, P, P, P]),
+    "msa_gated_delta_rule": (C.c_int, [C.c_int, P, P, P, P, P, I64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                       P, F32, P, P, P]),
 }
 
 _lib = None

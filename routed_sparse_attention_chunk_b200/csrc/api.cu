@@ -101,6 +101,89 @@ msa_status check_attn(msa_dtype dt, const void* Q, const void* Kloc, const void*
   return MSA_OK;
 }
 
+// Workspace of msa_sparse_attn_indexed: the segment plan, then either the
+// decode kernel's partial results (index-driven attention) or, for shapes and
+// banks the tensor-core kernels do not read in place, the gathered rows (sized
+// for fp32 storage) and the dense attention's workspace.
+struct IndexedWs {
+  int Smax;
+  int32_t *seg_row, *nseg, *mem_len;
+  uint8_t* seg_cnt;
+  void *attn_ws, *Kmem, *Vmem, *dense_ws;
+  size_t attn_ws_bytes, dense_ws_bytes, bytes;
+};
+
+IndexedWs indexed_ws_layout(void* base, int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int k, int Mmax) {
+  IndexedWs w{};
+  w.Smax = plan_smax(Mmax, k);
+  const size_t rows = round_up(sizeof(int32_t) * (size_t)B * w.Smax, 256);
+  const size_t cnts = round_up((size_t)B * w.Smax, 256);
+  const size_t per_b = round_up(sizeof(int32_t) * (size_t)B, 256);
+  const size_t plan = rows + cnts + 2 * per_b;
+  w.attn_ws_bytes = round_up(attn_indexed_workspace_size(B, Tq, Lloc, Hq, Hkv, w.Smax), 256);
+  const size_t mem = round_up(sizeof(float) * (size_t)B * (size_t)Mmax * (size_t)Hkv * (size_t)d, 256);
+  w.dense_ws_bytes = round_up(attn_workspace_size(MSA_BF16, B, Tq, Lloc, Hq, Hkv, d, Mmax), 256);
+  const size_t dense = 2 * mem + w.dense_ws_bytes;
+  w.bytes = plan + (w.attn_ws_bytes > dense ? w.attn_ws_bytes : dense);
+  if (base) {
+    char* p = static_cast<char*>(base);
+    w.seg_row = reinterpret_cast<int32_t*>(p);
+    w.seg_cnt = reinterpret_cast<uint8_t*>(p + rows);
+    w.nseg = reinterpret_cast<int32_t*>(p + rows + cnts);
+    w.mem_len = reinterpret_cast<int32_t*>(p + rows + cnts + per_b);
+    w.attn_ws = p + plan;
+    w.Kmem = p + plan;
+    w.Vmem = p + plan + mem;
+    w.dense_ws = p + plan + 2 * mem;
+  }
+  return w;
+}
+
+msa_status check_indexed(const int32_t* topk_idx, int k, const int64_t* doc_chunk_off, int64_t D, int64_t C,
+                         const void* Kbar, const void* Vbar) {
+  if (k < 1 || D < 1 || C < 0 || D > kMaxIndex || C > kMaxIndex) return MSA_ERR_INVALID_ARG;
+  if (k > 65535) return MSA_ERR_UNSUPPORTED;
+  if (!topk_idx || !doc_chunk_off || !Kbar || !Vbar) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(Kbar) || !aligned16(Vbar)) return MSA_ERR_INVALID_ARG;
+  return MSA_OK;
+}
+
+// Steps 4 + 5 once the arguments are checked: the index-driven attention when the
+// tensor-core kernels take the shape and the bank is in device memory, else the
+// gather into the workspace followed by the dense attention.
+msa_status run_indexed(msa_dtype dt, const void* Q, const void* Kloc, const void* Vloc, int64_t B, int Tq, int Lloc,
+                       int Hq, int Hkv, int d, const int32_t* topk_idx, int k, int idx_ld,
+                       const int64_t* doc_chunk_off, int64_t D, int64_t C, const void* Kbar, const void* Vbar,
+                       int Mmax, float scale, void* O, float* lse, const IndexedWs& w, int32_t* err_flag,
+                       cudaStream_t s) {
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d);
+  AttnArgs a{Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, nullptr, nullptr, w.mem_len, Mmax, scale, O, lse,
+             nullptr, 0, err_flag, nullptr, nullptr, nullptr, 0, C};
+  const bool on_device = !host_resident(Kbar) && !host_resident(Vbar);
+  if (on_device && C > 0 && attn_indexed_applies(dt, a)) {
+    PlanArgs pa{topk_idx, B, k, doc_chunk_off, D, C, Mmax, w.Smax, w.seg_row, w.seg_cnt, w.nseg, w.mem_len, err_flag,
+                idx_ld};
+    if (launch_plan(pa, s) != cudaSuccess) return MSA_ERR_CUDA;
+    a.Kmem = Kbar;
+    a.Vmem = Vbar;
+    a.seg_row = w.seg_row;
+    a.seg_cnt = w.seg_cnt;
+    a.nseg = w.nseg;
+    a.Smax = w.Smax;
+    a.ws = w.attn_ws;
+    a.ws_bytes = w.attn_ws_bytes;
+    return cuda_status(launch_attn(dt, a, s));
+  }
+  GatherArgs ga{topk_idx, B, k, doc_chunk_off, D, C, Kbar, Vbar, Hkv, d, Mmax, w.Kmem, w.Vmem, w.mem_len, err_flag,
+                host_resident(Kbar), idx_ld};
+  if (launch_gather(dt, ga, s) != cudaSuccess) return MSA_ERR_CUDA;
+  a.Kmem = w.Kmem;
+  a.Vmem = w.Vmem;
+  a.ws = w.dense_ws;
+  a.ws_bytes = w.dense_ws_bytes;
+  return cuda_status(launch_attn(dt, a, s));
+}
+
 }  // namespace
 
 namespace msa {
@@ -128,6 +211,8 @@ const char* msa_status_string(int status) {
 const char* msa_version(void) { return "0.1.0"; }
 
 uint64_t msa_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void msa_testing_set_wait_polls(int64_t polls) { attn_tc_set_test_polls(polls); }
 
 msa_status msa_rope_table_host(double theta, int d, int max_len, float* host_out) {
   if (!host_out || d < 2 || (d & 1) || max_len < 1 || !(theta > 0.0)) return MSA_ERR_INVALID_ARG;
@@ -300,15 +385,36 @@ msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const 
   return cuda_status(launch_attn(dt, a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t msa_sparse_attn_indexed_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int k,
+                                              int Mmax) {
+  if (B < 0 || Tq < 1 || Lloc < 1 || Hq < 1 || Hkv < 1 || d < 1 || k < 1 || Mmax < 0) return 0;
+  return indexed_ws_layout(nullptr, B, Tq, Lloc, Hq, Hkv, d, k, Mmax).bytes;
+}
+
+msa_status msa_sparse_attn_indexed(msa_dtype dt, const void* Q, const void* Kloc, const void* Vloc, int64_t B,
+                                   int Tq, int Lloc, int Hq, int Hkv, int d, const int32_t* topk_idx, int k,
+                                   const int64_t* doc_chunk_off, int64_t D, int64_t C, const void* Kbar,
+                                   const void* Vbar, int Mmax, float scale, void* O, float* lse, void* ws,
+                                   size_t ws_bytes, int32_t* err_flag, msa_stream_t stream) {
+  msa_status st = check_attn(dt, Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, Mmax);
+  if (st != MSA_OK) return st;
+  st = check_indexed(topk_idx, k, doc_chunk_off, D, C, Kbar, Vbar);
+  if (st != MSA_OK) return st;
+  if (B == 0) return MSA_OK;
+  if (!O || !aligned16(O)) return MSA_ERR_INVALID_ARG;
+  const IndexedWs w = indexed_ws_layout(ws, B, Tq, Lloc, Hq, Hkv, d, k, Mmax);
+  if (!ws || ws_bytes < w.bytes || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  if (!device_readable(Kbar) || !device_readable(Vbar)) return MSA_ERR_INVALID_ARG;
+  return run_indexed(dt, Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, topk_idx, k, k, doc_chunk_off, D, C, Kbar, Vbar,
+                     Mmax, scale, O, lse, w, err_flag, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t msa_layer_forward_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Hr, int64_t D,
                                         int64_t C, int k, int Mmax) {
-  if (B < 0 || Tq < 1 || Hr < 1 || D < 1 || C < 0 || k < 1 || Mmax < 0) return 0;
-  size_t n = route_ws_layout(nullptr, B, Tq, Hr, D, C, k).bytes;
-  // gathered memory rows (sized for fp32 storage, the larger type) and their counts
-  n += 2 * round_up(sizeof(float) * (size_t)B * (size_t)Mmax * (size_t)Hkv * (size_t)d, 256);
-  n += round_up(sizeof(int32_t) * (size_t)B, 256);
-  n += round_up(attn_workspace_size(MSA_BF16, B, Tq, Lloc, Hq, Hkv, d, Mmax), 256);
-  return n;
+  if (B < 0 || Tq < 1 || Lloc < 1 || Hq < 1 || Hkv < 1 || d < 1 || Hr < 1 || D < 1 || C < 0 || k < 1 || Mmax < 0)
+    return 0;
+  return route_ws_layout(nullptr, B, Tq, Hr, D, C, k).bytes +
+         indexed_ws_layout(nullptr, B, Tq, Lloc, Hq, Hkv, d, k, Mmax).bytes;
 }
 
 msa_status msa_layer_forward(msa_dtype dt, const void* Qr, int Hr, int dr, const void* Krbar,
@@ -321,34 +427,99 @@ msa_status msa_layer_forward(msa_dtype dt, const void* Qr, int Hr, int dr, const
   if (st != MSA_OK) return st;
   st = check_attn(dt, Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, Mmax);
   if (st != MSA_OK) return st;
+  st = check_indexed(topk_idx, k, doc_chunk_off, D, C, Kbar, Vbar);
+  if (st != MSA_OK) return st;
   if (B == 0) return MSA_OK;
-  if (!O || !Kbar || !Vbar || !aligned16(O) || !aligned16(Kbar) || !aligned16(Vbar)) return MSA_ERR_INVALID_ARG;
+  if (!O || !aligned16(O)) return MSA_ERR_INVALID_ARG;
   const size_t need = msa_layer_forward_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, D, C, k, Mmax);
   if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
   if (!device_readable(Kbar) || !device_readable(Vbar)) return MSA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   RouteWs w = route_ws_layout(ws, B, Tq, Hr, D, C, k);
-  char* p = static_cast<char*>(ws) + w.bytes;
-  const size_t mem_bytes = round_up(sizeof(float) * (size_t)B * (size_t)Mmax * (size_t)Hkv * (size_t)d, 256);
-  void* Kmem = p;
-  void* Vmem = p + mem_bytes;
-  p += 2 * mem_bytes;
-  int32_t* mem_len = reinterpret_cast<int32_t*>(p);
-  p += round_up(sizeof(int32_t) * (size_t)B, 256);
-  void* attn_ws = p;
-  const size_t attn_ws_bytes = ws_bytes - (size_t)(p - static_cast<char*>(ws));
-
+  const IndexedWs iw = indexed_ws_layout(static_cast<char*>(ws) + w.bytes, B, Tq, Lloc, Hq, Hkv, d, k, Mmax);
   RouteArgs ra{Qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, w.doc_key, w.rq, w.chunk_doc, err_flag};
   if (launch_route(dt, ra, s) != cudaSuccess) return MSA_ERR_CUDA;
   TopkArgs ta{w.doc_key, B, D, k, w.cand, w.doc_key + B * D, w.nslice, topk_idx, topk_score, doc_scores};
   if (launch_topk(ta, s) != cudaSuccess) return MSA_ERR_CUDA;
-  GatherArgs ga{topk_idx, B, k, doc_chunk_off, D, C, Kbar, Vbar, Hkv, d, Mmax, Kmem, Vmem, mem_len, err_flag,
-                host_resident(Kbar)};
-  if (launch_gather(dt, ga, s) != cudaSuccess) return MSA_ERR_CUDA;
-  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d);
-  AttnArgs a{Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, Kmem, Vmem, mem_len, Mmax, scale, O, lse,
-             attn_ws, attn_ws_bytes, err_flag};
-  return cuda_status(launch_attn(dt, a, s));
+  return run_indexed(dt, Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, topk_idx, k, k, doc_chunk_off, D, C, Kbar, Vbar,
+                     Mmax, scale, O, lse, iw, err_flag, s);
+}
+
+size_t msa_interleave_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Hr, int dr, int64_t D,
+                                     int64_t C, int k, int rounds, int Mmax) {
+  if (B < 0 || Tq < 1 || Lloc < 1 || Hq < 1 || Hkv < 1 || d < 1 || Hr < 1 || dr < 1 || D < 1 || C < 0 || k < 1 ||
+      rounds < 1 || Mmax < 0 || (int64_t)rounds * k > kMaxIndex)
+    return 0;
+  return route_ws_layout(nullptr, B, Tq, Hr, D, C, k).bytes +
+         indexed_ws_layout(nullptr, B, Tq, Lloc, Hq, Hkv, d, rounds * k, Mmax).bytes +
+         round_up(sizeof(float) * (size_t)B * (size_t)Tq * (size_t)Hr * (size_t)dr, 256);
+}
+
+msa_status msa_interleave_forward(msa_dtype dt, const void* Qr0, int Hr, int dr, const void* Krbar,
+                                  const float* kr_rnorm, const int64_t* doc_chunk_off, int64_t D, int64_t C, int k,
+                                  int rounds, const void* W_route, const void* Q, const void* Kloc, const void* Vloc,
+                                  int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, const void* Kbar,
+                                  const void* Vbar, int Mmax, float scale, void* O, float* lse, void* O_rounds,
+                                  void* Qr_rounds, int32_t* topk_idx, float* topk_score, void* ws, size_t ws_bytes,
+                                  int32_t* err_flag, msa_stream_t stream) {
+  if (rounds < 1 || k < 1 || (int64_t)rounds * k > D) return MSA_ERR_INVALID_ARG;
+  msa_status st = check_route(dt, Qr0, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, k, topk_idx);
+  if (st != MSA_OK) return st;
+  st = check_attn(dt, Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, Mmax);
+  if (st != MSA_OK) return st;
+  st = check_indexed(topk_idx, rounds * k, doc_chunk_off, D, C, Kbar, Vbar);
+  if (st != MSA_OK) return st;
+  if (rounds > 1 && !W_route) return MSA_ERR_INVALID_ARG;
+  if (B * (int64_t)Tq > 65535ll * 16) return MSA_ERR_UNSUPPORTED;  // rows of the round-to-round map's grid
+  if (B == 0) return MSA_OK;
+  if (!O || !aligned16(O) || !aligned16(O_rounds) || !aligned16(Qr_rounds)) return MSA_ERR_INVALID_ARG;
+  const size_t need = msa_interleave_workspace_size(B, Tq, Lloc, Hq, Hkv, d, Hr, dr, D, C, k, rounds, Mmax);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MSA_ERR_WORKSPACE;
+  if (!device_readable(Kbar) || !device_readable(Vbar)) return MSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const RouteWs w = route_ws_layout(ws, B, Tq, Hr, D, C, k);
+  char* p = static_cast<char*>(ws) + w.bytes;
+  const IndexedWs iw = indexed_ws_layout(p, B, Tq, Lloc, Hq, Hkv, d, rounds * k, Mmax);
+  void* qr_ws = p + iw.bytes;
+  const int ld = rounds * k;
+  const size_t esz = dt == MSA_F32 ? 4 : 2;
+  const size_t o_bytes = (size_t)B * Tq * Hq * d * esz;
+  const size_t qr_bytes = (size_t)B * Tq * Hr * dr * esz;
+  // round r >= 1 routes with the router query the map wrote: slot r - 1 of Qr_rounds, or the workspace
+  auto qr_slot = [&](int r) -> void* {
+    return Qr_rounds ? static_cast<char*>(Qr_rounds) + (size_t)(r - 1) * qr_bytes : qr_ws;
+  };
+  for (int r = 0; r < rounds; ++r) {
+    const void* qr = r == 0 ? Qr0 : qr_slot(r);
+    RouteArgs ra{qr, B, Tq, Hr, dr, Krbar, kr_rnorm, doc_chunk_off, D, C, w.doc_key, w.rq, w.chunk_doc, err_flag};
+    if (launch_route(dt, ra, s) != cudaSuccess) return MSA_ERR_CUDA;
+    // documents of the earlier rounds are passed over
+    if (launch_exclude(w.doc_key, B, D, topk_idx, ld, r * k, s) != cudaSuccess) return MSA_ERR_CUDA;
+    TopkArgs ta{w.doc_key, B, D, k, w.cand, w.doc_key + B * D, w.nslice, topk_idx + (size_t)r * k,
+                topk_score ? topk_score + (size_t)r * k : nullptr, nullptr, ld};
+    if (launch_topk(ta, s) != cudaSuccess) return MSA_ERR_CUDA;
+    const bool last = r == rounds - 1;
+    void* Or = (last || !O_rounds) ? O : static_cast<char*>(O_rounds) + (size_t)r * o_bytes;
+    st = run_indexed(dt, Q, Kloc, Vloc, B, Tq, Lloc, Hq, Hkv, d, topk_idx, (r + 1) * k, ld, doc_chunk_off, D, C,
+                     Kbar, Vbar, Mmax, scale, Or, last ? lse : nullptr, iw, err_flag, s);
+    if (st != MSA_OK) return st;
+    if (!last && launch_project(dt, Or, W_route, qr_slot(r + 1), B * (int64_t)Tq, Hq * d, Hr * dr, s) != cudaSuccess)
+      return MSA_ERR_CUDA;
+  }
+  return MSA_OK;
+}
+
+msa_status msa_gated_delta_rule(msa_dtype dt, const void* q, const void* k, const void* v, const float* g,
+                                const float* beta, int64_t B, int T, int Hk, int Hv, int dk, int dv, const float* h0,
+                                float scale, void* o, float* hT, msa_stream_t stream) {
+  if (!dtype_ok(dt) || B < 0 || T < 0 || Hk < 1 || Hv < 1 || Hv % Hk != 0) return MSA_ERR_INVALID_ARG;
+  if (dk != 128 || dv != 128 || B > 65535 || Hv > 65535) return MSA_ERR_UNSUPPORTED;
+  if (B == 0 || T == 0) return MSA_OK;
+  if (!q || !k || !v || !g || !beta || !o) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return MSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)dk);
+  return cuda_status(launch_gdr(dt, q, k, v, g, beta, B, T, Hk, Hv, dk, h0, scale, o, hT,
+                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
 msa_status msa_state_gather_sum(msa_dtype dt, const void* states, int64_t D, int64_t S, const int32_t* topk_idx,

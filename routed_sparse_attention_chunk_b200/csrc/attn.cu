@@ -20,8 +20,10 @@
 namespace msa {
 
 cudaError_t launch_attn_tc(msa_dtype dt, const AttnArgs& a, cudaStream_t s, bool* handled);
+bool attn_tc_applies(msa_dtype dt, const AttnArgs& a);
 bool decode_applies(msa_dtype dt, const AttnArgs& a);
 size_t decode_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int Mmax);
+size_t decode_workspace_size_smax(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int Smax);
 cudaError_t launch_attn_decode(const AttnArgs& a, cudaStream_t s);
 
 namespace {
@@ -167,8 +169,25 @@ size_t attn_workspace_size(msa_dtype dt, int64_t B, int Tq, int Lloc, int Hq, in
   return 0;
 }
 
+bool attn_indexed_applies(msa_dtype dt, const AttnArgs& a) {
+  return a.Hkv > 0 && a.Hq % a.Hkv == 0 && (decode_applies(dt, a) || attn_tc_applies(dt, a));
+}
+
+size_t attn_indexed_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int Smax) {
+  AttnArgs a{};
+  a.B = B;
+  a.Tq = Tq;
+  a.Lloc = Lloc;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.d = 128;
+  if (Hkv > 0 && decode_applies(MSA_BF16, a)) return decode_workspace_size_smax(B, Tq, Lloc, Hq, Hkv, Smax);
+  return 0;
+}
+
 cudaError_t launch_attn(msa_dtype dt, const AttnArgs& a, cudaStream_t s) {
   if (a.B <= 0) return cudaSuccess;
+  if (a.seg_row && !attn_indexed_applies(dt, a)) return cudaErrorInvalidValue;  // only the tensor-core kernels read a plan
   if (decode_applies(dt, a)) return launch_attn_decode(a, s);
   bool handled = false;
   cudaError_t e = launch_attn_tc(dt, a, s, &handled);

@@ -50,11 +50,17 @@ constexpr float kRescaleLog2 = 8.0f;
 struct DecParams {
   const __nv_bfloat16* Q;
   const int32_t* mem_len;
+  // index-driven memory rows (null seg_row: dense Kmem / Vmem): segment s of
+  // batch row b starts at bank row seg_row[b * plan_smax + s] and holds
+  // seg_cnt[...] rows; memory tile t holds segments [16 t, 16 t + 16)
+  const int32_t* seg_row;
+  const uint8_t* seg_cnt;
+  int plan_smax;
   int32_t* err_flag;
   float* part;  // [B * Hkv][Smax][R][kDH + 2]: m, l, O of one segment
   int64_t B;
   int Tq, Lloc, Hq, Hkv, Mmax, G, R;
-  int NM;       // memory tiles (ceil(Mmax / kKeys)); rows past mem_len are masked
+  int NM;       // memory tiles (ceil(Mmax / kKeys), or Smax / 16 from a plan); masked rows as above
   int NL;       // local tiles (ceil(Lloc / kKeys))
   int T;        // tiles per (b, g): NM + NL
   int Smax;     // partial slots per (b, g)
@@ -166,32 +172,54 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int64_t f = f0; f < f1 && !*abort_s;) {
-        const Seg sg = seg_at(p, f, f1);
-        const int g = (int)(sg.bg % p.Hkv);
-        const int64_t b = sg.bg / p.Hkv;
-        for (int t = sg.t0; t < sg.t1; ++t, ++it) {
-          const uint32_t st = it % kStages, round = it / kStages;
-          if (!mbar_wait(&kv_empty[st], (round & 1) ^ 1, kWaitPolls)) {
-            *abort_s = 1;
-            break;
+    // Lane 0 waits and arms the barriers; a memory tile read from the bank is 16
+    // boxes of kSegRows rows (one segment each), issued by lanes 0..15, each
+    // landing on a 1 KB swizzle atom so the tile's layout is that of one box.
+    const bool bank = p.seg_row != nullptr;
+    uint32_t it = 0;
+    bool stop = false;
+    for (int64_t f = f0; f < f1 && !stop;) {
+      const Seg sg = seg_at(p, f, f1);
+      const int g = (int)(sg.bg % p.Hkv);
+      const int64_t b = sg.bg / p.Hkv;
+      for (int t = sg.t0; t < sg.t1; ++t, ++it) {
+        const uint32_t st = it % kStages, round = it / kStages;
+        int ok = 1;
+        if (lane == 0) {
+          ok = !*abort_s && mbar_wait(&kv_empty[st], (round & 1) ^ 1, kWaitPolls);
+          if (!ok) *abort_s = 1;
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          stop = true;
+          break;
+        }
+        uint8_t* Kd = ring + st * DLayout::kStage;
+        uint8_t* Vd = Kd + DLayout::kTile;
+        if (lane == 0) mbar_arrive_expect_tx(&kv_full[st], DLayout::kStage);
+        __syncwarp();
+        const bool mem = t < p.NM;
+        const CUtensorMap* mk = mem ? &tmKm : &tmKl;
+        const CUtensorMap* mv = mem ? &tmVm : &tmVl;
+        if (mem && bank) {
+          if (lane < kKeys / kSegRows) {
+            const int y = __ldg(p.seg_row + b * p.plan_smax + t * (kKeys / kSegRows) + lane);
+            const int so = lane * (kSegRows * 128);
+            for (int dc = 0; dc < 2; ++dc) {
+              tma_load_2d(Kd + dc * (kKeys * 128) + so, mk, g * kDH + dc * 64, y, &kv_full[st]);
+              tma_load_2d(Vd + dc * (kKeys * 128) + so, mv, g * kDH + dc * 64, y, &kv_full[st]);
+            }
           }
-          uint8_t* Kd = ring + st * DLayout::kStage;
-          uint8_t* Vd = Kd + DLayout::kTile;
-          mbar_arrive_expect_tx(&kv_full[st], DLayout::kStage);
-          const bool mem = t < p.NM;
-          const CUtensorMap* mk = mem ? &tmKm : &tmKl;
-          const CUtensorMap* mv = mem ? &tmVm : &tmVl;
+        } else if (lane == 0) {
           const int y = mem ? (int)(b * p.Mmax + t * kKeys) : (int)(b * p.Lloc + (t - p.NM) * kKeys);
           for (int dc = 0; dc < 2; ++dc) {
             tma_load_2d(Kd + dc * (kKeys * 128), mk, g * kDH + dc * 64, y, &kv_full[st]);
             tma_load_2d(Vd + dc * (kKeys * 128), mv, g * kDH + dc * 64, y, &kv_full[st]);
           }
         }
-        f += sg.t1 - sg.t0;
       }
+      f += sg.t1 - sg.t0;
+    }
+    if (lane == 0) {
       const uint32_t fills = it;
       for (uint32_t st = 0; st < (uint32_t)kStages && st < fills; ++st) {
         const uint32_t last = (fills - 1 - st) / kStages * kStages + st;
@@ -316,7 +344,8 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
       // the next segment's Q rows, loaded now and stored after this segment's first tile
       uint4 qn[2];
       if (fn < f1) load_q(seg_at(p, fn, f1), qn);
-      int M = __ldg(p.mem_len + b);
+      const bool bank = p.seg_row != nullptr;
+      int M = bank ? 0 : __ldg(p.mem_len + b);
       if (M < 0 || M > p.Mmax) {
         if (et == 0 && sg.t0 == 0 && sg.bg % p.Hkv == 0) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
         M = M < 0 ? 0 : p.Mmax;
@@ -330,6 +359,9 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
       for (int j = 0; j < T; ++j) {
         const int t = t0 + j;
         const uint32_t sb = (js + j) & 1, use = (js + j) >> 1;
+        // a bank tile: this thread's key is row (r_lane % kSegRows) of segment 16 t + r_lane / kSegRows
+        int seg_n = 0;
+        if (bank && t < p.NM) seg_n = __ldg(p.seg_cnt + b * p.plan_smax + t * (kKeys / kSegRows) + (r_lane >> 3));
         if (!*abort_s && !__all_sync(0xffffffffu, mbar_wait(&s_full[sb], use & 1, kWaitPolls))) *abort_s = 1;
         tc_fence_after();
         float sc[kR];
@@ -340,9 +372,10 @@ attn_decode_kernel(const __grid_constant__ CUtensorMap tmKm, const __grid_consta
         // mask; scale into the log2 domain
         const bool mem = t < p.NM;
         const int key = (mem ? t : t - p.NM) * kKeys + r_lane;
+        const bool mem_vis = bank ? (r_lane & (kSegRows - 1)) < seg_n : key < M;
 #pragma unroll
         for (int r = 0; r < kR; ++r) {
-          const bool vis = r < p.R && (mem ? key < M : key <= p.Lloc - p.Tq + r / p.G);
+          const bool vis = r < p.R && (mem ? mem_vis : key <= p.Lloc - p.Tq + r / p.G);
           sc[r] = vis ? sc[r] * p.scale_log2 : -INFINITY;
         }
         // column maxima over the tile's 128 keys: a warp reduction per column,
@@ -490,7 +523,7 @@ struct DecodePlan {
 DecodePlan plan(const AttnArgs& a) {
   DecodePlan d{};
   d.R = (a.Hq / a.Hkv) * a.Tq;
-  d.NM = (a.Mmax + kKeys - 1) / kKeys;
+  d.NM = a.seg_row ? a.Smax / (kKeys / kSegRows) : (a.Mmax + kKeys - 1) / kKeys;
   d.NL = (a.Lloc + kKeys - 1) / kKeys;
   d.T = d.NM + d.NL;
   d.bgs = a.B * a.Hkv;
@@ -514,6 +547,19 @@ bool decode_applies(msa_dtype dt, const AttnArgs& a) {
   return R <= kMaxRows && a.Tq <= 4;
 }
 
+size_t decode_workspace_size_smax(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int Smax) {
+  AttnArgs a{};
+  a.B = B;
+  a.Tq = Tq;
+  a.Lloc = Lloc;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Smax = Smax;
+  a.seg_row = reinterpret_cast<const int32_t*>(16);  // marks the plan layout; never dereferenced
+  const DecodePlan d = plan(a);
+  return sizeof(float) * (size_t)d.bgs * d.Smax * d.R * (kDH + 2);
+}
+
 size_t decode_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int Mmax) {
   AttnArgs a{};
   a.B = B;
@@ -534,17 +580,23 @@ cudaError_t launch_attn_decode(const AttnArgs& a, cudaStream_t s) {
   CUtensorMap tkm, tvm, tkl, tvl;
   const uint64_t rowkv = (uint64_t)a.Hkv * kDH * 2;
   const int64_t mrows = a.B * (int64_t)(a.Mmax > 0 ? a.Mmax : 1);
-  const void* km = a.Mmax > 0 ? a.Kmem : a.Kloc;
-  const void* vm = a.Mmax > 0 ? a.Vmem : a.Vloc;
-  const uint64_t mr = (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc);
-  if (!make_tmap_2d_bf16(&tkm, km, (uint64_t)a.Hkv * kDH, mr, rowkv, 64, kKeys) ||
-      !make_tmap_2d_bf16(&tvm, vm, (uint64_t)a.Hkv * kDH, mr, rowkv, 64, kKeys) ||
+  const bool bank = a.seg_row != nullptr;
+  // memory maps: the bank [C, Hkv * d] in boxes of one segment, or the dense rows [B * Mmax, Hkv * d]
+  const void* km = bank || a.Mmax > 0 ? a.Kmem : a.Kloc;
+  const void* vm = bank || a.Mmax > 0 ? a.Vmem : a.Vloc;
+  const uint64_t mr = bank ? (uint64_t)(a.C > 0 ? a.C : 1) : (uint64_t)(a.Mmax > 0 ? mrows : a.B * a.Lloc);
+  const uint32_t mbox = bank ? kSegRows : kKeys;
+  if (!make_tmap_2d_bf16(&tkm, km, (uint64_t)a.Hkv * kDH, mr, rowkv, 64, mbox) ||
+      !make_tmap_2d_bf16(&tvm, vm, (uint64_t)a.Hkv * kDH, mr, rowkv, 64, mbox) ||
       !make_tmap_2d_bf16(&tkl, a.Kloc, (uint64_t)a.Hkv * kDH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKeys) ||
       !make_tmap_2d_bf16(&tvl, a.Vloc, (uint64_t)a.Hkv * kDH, (uint64_t)(a.B * a.Lloc), rowkv, 64, kKeys))
     return cudaErrorInvalidValue;
   DecParams p;
   p.Q = reinterpret_cast<const __nv_bfloat16*>(a.Q);
   p.mem_len = a.mem_len;
+  p.seg_row = a.seg_row;
+  p.seg_cnt = a.seg_cnt;
+  p.plan_smax = a.Smax;
   p.err_flag = a.err_flag;
   p.part = reinterpret_cast<float*>(a.ws);
   p.B = a.B;

@@ -21,9 +21,10 @@ struct Sel {
   int64_t cs, n;  // first chunk and chunk count of the selected document (n = 0: skipped)
 };
 
+// Rank r of query b in a selection list whose rows are ld entries apart.
 __device__ __forceinline__ Sel selected(const int32_t* __restrict__ idx, const int64_t* __restrict__ off,
-                                        int64_t D, int64_t C, int64_t b, int k, int r, bool* bad) {
-  const int32_t j = __ldg(idx + b * k + r);
+                                        int64_t D, int64_t C, int64_t b, int ld, int r, bool* bad) {
+  const int32_t j = __ldg(idx + b * ld + r);
   if (j < 0 || (int64_t)j >= D) {
     *bad = true;
     return {0, 0};
@@ -52,11 +53,12 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a, int row_vecs)
   for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
     const int64_t b = item / a.k;
     const int r = (int)(item - b * a.k);
+    const int ld = a.idx_ld > 0 ? a.idx_ld : a.k;
     bool bad = false;
     int64_t start = 0;
-    for (int q = 0; q < r; ++q) start += selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, a.k, q, &bad).n;
+    for (int q = 0; q < r; ++q) start += selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, ld, q, &bad).n;
     bool mine_bad = false;
-    const Sel me = selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, a.k, r, &mine_bad);
+    const Sel me = selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, ld, r, &mine_bad);
     if (threadIdx.x == 0) {
       if (mine_bad) raise_flag(a.err_flag, MSA_FLAG_INDEX_OOB);
       if (r == a.k - 1) {
@@ -106,7 +108,77 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a, int row_vecs)
   }
 }
 
+// Segment plan for the index-driven attention: one warp per query walks its k
+// selected documents 32 at a time (a lane per document), prefix-sums their
+// chunk counts across the warp to find where each document's rows start (rows
+// past Mmax are dropped), and writes the document's rows as segments of at
+// most kSegRows consecutive bank rows.  Entries past the query's last segment
+// are padding: row C (past the end of the bank, which a TMA load reads as
+// zeros) and count 0.
+__global__ void __launch_bounds__(128) plan_kernel(PlanArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t b = (int64_t)blockIdx.x * 4 + warp;
+  if (b >= a.B) return;
+  int32_t* row = a.seg_row + b * a.Smax;
+  uint8_t* cnt = a.seg_cnt + b * a.Smax;
+  const int ld = a.idx_ld > 0 ? a.idx_ld : a.k;
+  int64_t rows_before = 0;  // selected rows of the earlier ranks (not truncated)
+  int segs_before = 0;
+  bool any_bad = false;
+  for (int r0 = 0; r0 < a.k; r0 += 32) {
+    const int r = r0 + lane;
+    bool bad = false;
+    const Sel me = r < a.k ? selected(a.topk_idx, a.doc_chunk_off, a.D, a.C, b, ld, r, &bad) : Sel{0, 0};
+    any_bad |= bad;
+    // inclusive prefix sums over the lanes of the chunk counts
+    int64_t incl = me.n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int64_t start = rows_before + incl - me.n;
+    const int64_t kept = max((int64_t)0, min(me.n, (int64_t)a.Mmax - start));
+    const int segs = (int)((kept + kSegRows - 1) / kSegRows);
+    int sincl = segs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, sincl, o);
+      if (lane >= o) sincl += v;
+    }
+    const int s0 = segs_before + sincl - segs;
+    for (int q = 0; q < segs; ++q) {
+      const int si = s0 + q;
+      if (si < a.Smax) {  // always true for Smax >= ceil(Mmax / 8) + k
+        row[si] = (int32_t)(me.cs + (int64_t)q * kSegRows);
+        cnt[si] = (uint8_t)min((int64_t)kSegRows, kept - (int64_t)q * kSegRows);
+      }
+    }
+    rows_before += __shfl_sync(0xffffffffu, incl, 31);
+    segs_before += __shfl_sync(0xffffffffu, sincl, 31);
+  }
+  const int ns = min(segs_before, a.Smax);
+  for (int si = ns + lane; si < a.Smax; si += 32) {
+    row[si] = (int32_t)a.C;
+    cnt[si] = 0;
+  }
+  any_bad = __any_sync(0xffffffffu, any_bad);
+  if (lane == 0) {
+    if (any_bad) raise_flag(a.err_flag, MSA_FLAG_INDEX_OOB);
+    if (rows_before > a.Mmax) raise_flag(a.err_flag, MSA_FLAG_OVERFLOW);
+    a.nseg[b] = ns;
+    a.mem_len[b] = (int32_t)min(rows_before, (int64_t)a.Mmax);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s) {
+  if (a.B <= 0) return cudaSuccess;
+  count_launch();
+  plan_kernel<<<(unsigned)((a.B + 3) / 4), 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gather(msa_dtype dt, const GatherArgs& a, cudaStream_t s) {
   if (a.B <= 0) return cudaSuccess;

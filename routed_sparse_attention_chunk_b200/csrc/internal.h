@@ -147,9 +147,27 @@ struct TopkArgs {
   int32_t* topk_idx;
   float* topk_score;
   float* doc_scores;
+  int out_ld;  // row stride of topk_idx / topk_score (0: k)
 };
 int topk_num_slices(int64_t D, int k);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+// Documents excl[b, 0..n) (row stride ld) of each query get key 0 (score -inf), so the
+// top-k that follows passes them over while other documents remain; out-of-range
+// entries are ignored.
+cudaError_t launch_exclude(uint32_t* doc_key, int64_t B, int64_t D, const int32_t* excl, int ld, int n,
+                           cudaStream_t s);
+
+// Gated delta rule of the linear (DGA) layers' query path (gdr.cu), chunks of 64 tokens,
+// one CTA per (value head, query); d = dk = dv = 128.
+cudaError_t launch_gdr(msa_dtype dt, const void* q, const void* k, const void* v, const float* g, const float* beta,
+                       int64_t B, int T, int Hk, int Hv, int d, const float* h0, float scale, void* o, float* hT,
+                       cudaStream_t s);
+
+// Round-to-round map of the memory interleave: out[r, :] = in[r, :] x W for rows
+// r < rows (in [rows, K], W [K, N], out [rows, N]; fp32 accumulation, the
+// result rounded to the storage type).
+cudaError_t launch_project(msa_dtype dt, const void* in, const void* W, void* out, int64_t rows, int K, int N,
+                           cudaStream_t s);
 
 struct GatherArgs {
   const int32_t* topk_idx;
@@ -163,10 +181,40 @@ struct GatherArgs {
   int32_t* mem_len;
   int32_t* err_flag;
   bool host_src;  // Kbar / Vbar in page-locked host memory: few CTAs, many loads in flight each
+  int idx_ld;     // row stride of topk_idx (0: k)
 };
 cudaError_t launch_gather(msa_dtype dt, const GatherArgs& a, cudaStream_t s);
 
-// Memory rows are dense [B, Mmax, Hkv, d] tensors (Kmem/Vmem), rows [0, mem_len[b]) used.
+// Segment plan of the index-driven attention (gather fused into attention):
+// query b's selected chunks, in rank order, cut into segments of at most
+// kSegRows consecutive chunk rows of one document.  Segment s of query b starts
+// at bank row seg_row[b, s] and holds seg_cnt[b, s] valid rows; segments
+// [nseg[b], Smax) are padding (row C, past the bank; count 0).  mem_len[b] is
+// the number of selected rows kept (at most Mmax; more raises MSA_FLAG_OVERFLOW).
+constexpr int kSegRows = 8;
+struct PlanArgs {
+  const int32_t* topk_idx;
+  int64_t B;
+  int k;
+  const int64_t* doc_chunk_off;
+  int64_t D, C;
+  int Mmax, Smax;  // Smax: a multiple of 16, at least ceil(Mmax / 8) + k
+  int32_t* seg_row;  // [B, Smax]
+  uint8_t* seg_cnt;  // [B, Smax]
+  int32_t* nseg;     // [B]
+  int32_t* mem_len;  // [B]
+  int32_t* err_flag;
+  int idx_ld;        // row stride of topk_idx (0: k)
+};
+inline int plan_smax(int Mmax, int k) {
+  const int s = (Mmax + kSegRows - 1) / kSegRows + k;
+  return (s + 15) / 16 * 16;
+}
+cudaError_t launch_plan(const PlanArgs& a, cudaStream_t s);
+
+// Memory rows are either dense [B, Mmax, Hkv, d] tensors (Kmem/Vmem), rows
+// [0, mem_len[b]) used, or (seg_row != null) read in place from the bank
+// K̄ / V̄ [C, Hkv, d] through a segment plan (Kmem/Vmem then point at the bank).
 struct AttnArgs {
   const void *Q, *Kloc, *Vloc;
   int64_t B;
@@ -180,8 +228,21 @@ struct AttnArgs {
   void* ws;
   size_t ws_bytes;
   int32_t* err_flag;
+  // index-driven memory rows (all null / 0 for dense Kmem / Vmem)
+  const int32_t* seg_row;
+  const uint8_t* seg_cnt;
+  const int32_t* nseg;
+  int Smax;
+  int64_t C;  // bank rows
 };
 size_t attn_workspace_size(msa_dtype dt, int64_t B, int Tq, int Lloc, int Hq, int Hkv, int d, int Mmax);
 cudaError_t launch_attn(msa_dtype dt, const AttnArgs& a, cudaStream_t s);
+// Test hook of the prefill attention kernel's bounded waits (msa_testing_set_wait_polls).
+void attn_tc_set_test_polls(int64_t polls);
+// Whether a tensor-core kernel reads memory rows through a segment plan for this shape
+// (bf16, d = 128, a decode or prefill shape those kernels take).
+bool attn_indexed_applies(msa_dtype dt, const AttnArgs& a);
+// Workspace of the decode kernel when the memory rows come through a plan of Smax segments.
+size_t attn_indexed_workspace_size(int64_t B, int Tq, int Lloc, int Hq, int Hkv, int Smax);
 
 }  // namespace msa

@@ -182,7 +182,7 @@ __device__ bool slice_topk_filter(uint64_t* s, int* cnt, uint64_t* tau_s, const 
 
 __global__ void __launch_bounds__(kSortThreads)
 topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, uint64_t* cand,
-            uint32_t* counters, int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
+            uint32_t* counters, int32_t* __restrict__ out_idx, float* __restrict__ out_score, int out_ld) {
   __shared__ uint64_t s[kSortN];
   __shared__ uint64_t tau_s;
   __shared__ int last, cnt;
@@ -224,8 +224,17 @@ topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, 
   }
   for (int i = threadIdx.x; i < k; i += blockDim.x) {
     const uint64_t key = s[i];
-    out_idx[b * k + i] = (int32_t)(0xffffffffu - (uint32_t)(key & 0xffffffffu));
-    if (out_score) out_score[b * k + i] = key_to_float((uint32_t)(key >> 32));
+    out_idx[b * out_ld + i] = (int32_t)(0xffffffffu - (uint32_t)(key & 0xffffffffu));
+    if (out_score) out_score[b * out_ld + i] = key_to_float((uint32_t)(key >> 32));
+  }
+}
+
+__global__ void exclude_kernel(uint32_t* __restrict__ doc_key, int64_t D, const int32_t* __restrict__ excl, int ld,
+                               int n) {
+  const int64_t b = blockIdx.x;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int32_t j = __ldg(excl + b * ld + i);
+    if (j >= 0 && (int64_t)j < D) doc_key[b * D + j] = 0u;
   }
 }
 
@@ -255,7 +264,15 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   }
   count_launch();
   return launch_pdl(topk_kernel, dim3(a.nslice, (unsigned)a.B), dim3(kSortThreads), 0, s, a.doc_key, a.D, a.k,
-                    a.nslice, a.cand, a.counters, a.topk_idx, a.topk_score);
+                    a.nslice, a.cand, a.counters, a.topk_idx, a.topk_score, a.out_ld > 0 ? a.out_ld : a.k);
+}
+
+cudaError_t launch_exclude(uint32_t* doc_key, int64_t B, int64_t D, const int32_t* excl, int ld, int n,
+                           cudaStream_t s) {
+  if (B <= 0 || n <= 0) return cudaSuccess;
+  count_launch();
+  exclude_kernel<<<(unsigned)B, 128, 0, s>>>(doc_key, D, excl, ld, n);
+  return cudaGetLastError();
 }
 
 }  // namespace msa

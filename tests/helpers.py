@@ -112,3 +112,42 @@ def attn_on_gpu(Q, Kl, Vl, Km, Vm, mem_len, scale=0.0, want_lse=True):
     flag = torch.zeros(1, dtype=torch.int32, device=dev)
     msa.sparse_attn(Q, Kl, Vl, Km, Vm, mem_len, O, lse, scale, ws, flag)
     return O, lse, flag
+
+
+def pool_bank_slabs(cfg: synth.Config, device, seed: int = 0, Qr0=None):
+    """The bank of a whole workload pooled slab by slab on the device, as a large corpus is encoded
+    (each slab's raw tokens drawn, pooled with slab-relative offsets, then freed).
+    Returns (Kbar, Vbar, Krbar, doc_chunk_off, kr_rnorm, flag)."""
+    tok = synth.doc_tok_offsets(cfg)
+    coff = msa.chunk_offsets(tok, cfg.P)
+    C = int(coff[-1])
+    dt = cfg.torch_dtype
+    rope = msa.rope_table(cfg.theta, cfg.d, int(np.diff(tok).max())).to(device)
+    Kb = torch.empty((C, cfg.Hkv, cfg.d), dtype=dt, device=device)
+    Vb = torch.empty_like(Kb)
+    Krb = torch.empty((C, cfg.Hr, cfg.dr), dtype=dt, device=device)
+    rn = torch.empty((C, cfg.Hr), dtype=torch.float32, device=device)
+    flag = torch.zeros(1, dtype=torch.int32, device=device)
+    for lo, hi in synth.slab_bounds(cfg):
+        K, V, Kr = synth.gen_raw_slab(cfg, lo, hi, device, seed, Qr0=Qr0)
+        t = torch.from_numpy(tok[lo:hi + 1] - tok[lo]).to(device)
+        cs, ce = int(coff[lo]), int(coff[hi])
+        ch = torch.from_numpy(coff[lo:hi + 1] - coff[lo]).to(device)
+        msa.pool(K, V, Kr, t, ch, cfg.P, rope, Kb[cs:ce], Vb[cs:ce], Krb[cs:ce], rn[cs:ce], flag)
+        del K, V, Kr
+    return Kb, Vb, Krb, coff, rn, flag
+
+
+def oracle_route_by_slabs(Qr64: np.ndarray, Krb: torch.Tensor, coff: np.ndarray, docs_per_slab: int) -> np.ndarray:
+    """The oracle's document scores [B, D] over a device bank of any size: a document's score
+    depends only on its own chunks, so the oracle's route runs on one slab of whole documents at
+    a time (their stored bank bytes copied to the host and widened to fp64)."""
+    from oracle import msa_oracle as O
+    D = len(coff) - 1
+    out = np.empty((Qr64.shape[0], D))
+    for lo in range(0, D, docs_per_slab):
+        hi = min(lo + docs_per_slab, D)
+        cs, ce = int(coff[lo]), int(coff[hi])
+        kb = Krb[cs:ce].to("cpu", torch.float64).numpy()
+        out[:, lo:hi] = O.route(Qr64, kb, coff[lo:hi + 1] - cs)
+    return out
