@@ -515,6 +515,30 @@ def workload_extra(name: str, device, seed: int, peaks: dict, peak_kind: str, st
            "l2": "inputs larger than L2" if flush is None else "L2 flushed between steps (not timed)",
            "stages": {s: stage_entry(s, v, cfg, counts, peaks, peak_kind, long_region, clocks, step_sum)
                       for s, v in stage_ms.items() if v}}
+    if cfg.Tq > 1 and cfg.layers > 1:
+        # the attention kernel alone: every layer's msa_sparse_attn_indexed back to back (its clock is
+        # not the one the routing scan leaves it inside the step), W warm-up rounds, then K timed rounds
+        stream = torch.cuda.current_stream()
+        for _ in range(warmup):
+            for l in range(cfg.layers):
+                w.sparse_attn(l)
+        torch.cuda.synchronize()
+        sampler = ClockSampler(device)
+        sampler.start()
+        ev = []
+        for _ in range(steps):
+            for l in range(cfg.layers):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                w.sparse_attn(l)
+                e1.record(stream)
+                ev.append((e0, e1))
+        torch.cuda.synchronize()
+        aclocks = sampler.stop()
+        at = [a.elapsed_time(b) for a, b in ev]
+        out["sparse_attn_alone"] = stage_entry("sparse_attn", at, cfg, counts, peaks, peak_kind,
+                                               sustained_region(float(np.sum(at)), aclocks), aclocks)
+        out["sparse_attn_alone"]["clocks"] = aclocks
     if w.raw is not None:
         n = 3 if raw_bytes(cfg) > 20e9 else 10
         ptimes, pclocks = timed_pool(w, n, 2, device)

@@ -6,9 +6,9 @@
 // Flash-style forward, one CTA per (query block, KV head, batch row):
 //   * the CTA's 128 rows are the GQA group's G q-heads x (128 / G) tokens, so one
 //     K/V tile serves every head of the group;
-//   * key tiles of 128 rows: first the memory rows (all visible; rows past
-//     mem_len are masked), then the local rows up to the block's last causal
-//     position (bottom-right aligned: token i sits at Lloc - Tq + i);
+//   * key tiles of 128 rows: the local rows up to the block's last causal
+//     position (bottom-right aligned: token i sits at Lloc - Tq + i), then the
+//     memory rows (all visible; rows past mem_len are masked);
 //   * S = Q K^T by tcgen05.mma into one of two TMEM buffers (the tensor core
 //     computes S_{j+1} while the softmax warps work on S_j); P = exp2(S - m)
 //     is rounded to bf16 and written back over its own S tile in TMEM (two
@@ -73,10 +73,9 @@ struct ALayout {
   static constexpr int kBoxes = DH / 64;
   static constexpr int kQ = kRows * DH * 2;
   static constexpr int kK = kKeys * DH * 2;  // one K (or V) tile
-  static constexpr int kBar = 8 * 24;  // 23 barriers and the TMEM address
+  static constexpr int kBar = 8 * 24;
   static constexpr int kSmem = 1024 + kQ + 2 * kKV * kK + kBar;  // Q, K[kKV], V[kKV]
-  static constexpr uint32_t kTmemCols = 512;  // S0, S1 (128 each), O0, O1 (DH each)
-  static_assert(2 * kKeys + 2 * DH <= (int)kTmemCols, "two S buffers and two accumulators");
+  static constexpr uint32_t kTmemCols = 512;  // S0, S1 (128 each), O (DH)
   static_assert(kSmem <= 232448, "shared memory of one CTA");
 };
 
@@ -112,44 +111,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// One work item: a block of TB query tokens (x G q-heads = 128 rows) of one KV
-// head of one batch row, with its key tiles: memory rows first, then the local
-// rows up to the block's last causal position.
-struct Item {
-  int qb, g, b, t0, M, NM, T;
-};
-
-__device__ __forceinline__ Item item_at(const AttnTcParams& p, int64_t w) {
-  // longest items first: w runs over query blocks from the last one down, then KV heads, then batch rows
-  Item it;
-  const int64_t per_qb = (int64_t)p.Hkv * p.B;
-  const int qr = (int)(w / per_qb);
-  const int rem = (int)(w - (int64_t)qr * per_qb);
-  it.qb = p.n_qblk - 1 - qr;
-  it.g = rem % p.Hkv;
-  it.b = rem / p.Hkv;
-  it.t0 = it.qb * p.TB;
-  const int tlast = min(it.t0 + p.TB, p.Tq) - 1;
-  if (p.seg_row) {
-    // memory rows read in place from the bank: nseg segments of kSegRows rows
-    // each, the rows past a segment's count masked like rows past mem_len
-    it.M = min(max(__ldg(p.nseg + it.b), 0), p.Smax) * kSegRows;
-  } else {
-    const int M = __ldg(p.mem_len + it.b);
-    it.M = M < 0 ? 0 : (M > p.Mmax ? p.Mmax : M);
-  }
-  it.NM = (it.M + kKeys - 1) / kKeys;
-  it.T = it.NM + (p.Lloc - p.Tq + tlast + kKeys) / kKeys;  // + local tiles up to the last causal position
-  return it;
-}
-
-// The r-th item of this CTA: items are dealt to the CTAs in rounds of gridDim.x,
-// in alternating directions, so every CTA's total of tiles is about the same.
-__device__ __forceinline__ int64_t item_of(int r) {
-  const int64_t G = gridDim.x, c = blockIdx.x;
-  return (int64_t)r * G + ((r & 1) ? (G - 1 - c) : c);
-}
-
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKm,
@@ -162,27 +123,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* Ks = Qs + L::kQ;          // [kKV] K tiles
   uint8_t* Vs = Ks + kKV * L::kK;    // [kKV] V tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(Vs + kKV * L::kK);
-  uint64_t* q_full = bars + 0;             // TMA -> MMA (one Q tile per item)
-  uint64_t* q_empty = bars + 1;            // the item's last S MMA done -> TMA (next item's Q)
-  uint64_t* k_full = bars + 2;             // [kKV] TMA -> MMA
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;             // [kKV] TMA -> MMA
   uint64_t* k_empty = k_full + kKV;        // [kKV] S MMA done -> TMA
   uint64_t* v_full = k_empty + kKV;        // [kKV]
   uint64_t* v_empty = v_full + kKV;        // [kKV] PV MMA done -> TMA
   uint64_t* s_full = v_empty + kKV;        // [2] S MMA done -> softmax
   uint64_t* p_full = s_full + 2;           // [2] P written over S -> MMA
   uint64_t* p_free = p_full + 2;           // [2] PV MMA done -> softmax (O up to date)
-  uint64_t* o_free = p_free + 2;           // [2] an item's output read from O buffer i -> MMA
-  uint64_t* drain = o_free + 2;
+  uint64_t* drain = p_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // longest blocks first: block index 0 takes the last query block
+  const int qb = p.n_qblk - 1 - (int)blockIdx.x;
+  const int g = blockIdx.y;
+  const int b = blockIdx.z;
+  const int t0 = qb * p.TB;
+  const int tlast = min(t0 + p.TB, p.Tq) - 1;
   const bool bank = p.seg_row != nullptr;
   constexpr int kSegs = kKeys / kSegRows;  // segments per memory tile
-  const int64_t n_items = (int64_t)p.n_qblk * p.Hkv * p.B;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
     for (int i = 0; i < kKV; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
@@ -193,7 +156,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
       mbar_init(&p_free[i], 1);
-      mbar_init(&o_free[i], 128);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -206,93 +168,106 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S0, S1 (128 each), then the output accumulators O0, O1 (DH each), one per item parity
-  const uint32_t tS0 = tmem, tO0 = tmem + 2 * kKeys;
+  const uint32_t tS0 = tmem, tO = tmem + 2 * kKeys;
   bool timed_out = false;
+  if (warp == 0 && lane == 0) {
+    // the query rows do not depend on the kernel this one may overlap
+    tma_prefetch_desc(&tmQ);
+    mbar_arrive_expect_tx(q_full, L::kQ);
+    for (int hh = 0; hh < p.G; ++hh)
+#pragma unroll
+      for (int dc = 0; dc < L::kBoxes; ++dc)
+        tma_load_2d(Qs + dc * (kRows * 128) + hh * p.TB * 128, &tmQ, (g * p.G + hh) * DH + dc * 64,
+                    b * p.Tq + t0, q_full);
+  }
+  // With memory rows read from the bank, this kernel is a programmatic
+  // dependent of the plan kernel: everything above overlapped it, and the plan
+  // is read only after this wait (a no-op for an ordinary launch).
+  pdl_wait();
+  // the query's memory row count and (producer lanes) the first memory tile's run rows, both
+  // loaded before either is used so their latencies overlap
+  const int Mraw = bank ? __ldg(p.nseg + b) : __ldg(p.mem_len + b);
+  const int seg0 = (bank && warp == 0 && lane < kSegs) ? __ldg(p.seg_row + (int64_t)b * p.Smax + lane) : 0;
+  int M;
+  if (bank) {
+    // memory rows read in place from the bank: nseg segments of kSegRows rows
+    // each, the rows past a segment's count masked like rows past mem_len
+    M = min(max(Mraw, 0), p.Smax) * kSegRows;
+  } else {
+    M = Mraw;
+    if (M < 0 || M > p.Mmax) {
+      if (threadIdx.x == 0 && qb == 0 && g == 0) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
+      M = M < 0 ? 0 : p.Mmax;
+    }
+  }
+  const int NM = (M + kKeys - 1) / kKeys;                       // memory tiles
+  const int pos_last = p.Lloc - p.Tq + tlast;
+  const int NL = (pos_last + kKeys) / kKeys;                     // local tiles up to pos_last
+  const int T = NL + NM;
+  // Tile order: the local tiles first, then the memory tiles.  Local tile 0
+  // holds a key every row sees (local row 0), so each row's running maximum is
+  // finite from the first tile on; and a memory tile read from the bank (16
+  // small boxes per half) is issued while earlier tiles are in flight.
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    // Per item: its Q tile (once the previous item's S MMAs are done with the
-    // single Q buffer), then K and V tiles in the order their stages free up:
-    // K_j is free once S_j is done, V_j once PV_j is, and the tensor core runs
-    // S_{j+1} before PV_j, so the loads go K0, K1, K2, V0, K3, V1, ... and an
-    // item's last V tiles are issued before the next item's Q.  Stage indices
-    // and phases count tiles over all of the CTA's items.  Lane 0 waits and
-    // arms the barriers; a memory tile read from the bank is kSegs boxes of
-    // kSegRows rows, one per lane (each lands on a 1 KB swizzle atom, so the
-    // tile's layout is that of one 128-row box).
-    if (lane == 0) tma_prefetch_desc(&tmQ);
-    int nk = 0, nv = 0, nq = 0;  // loads issued over all items: K tiles, V tiles, Q tiles
-    bool ok = true;
-    auto load = [&](const Item& I, int j, int gidx, bool is_v) -> bool {
-      const int st = gidx % kKV;
-      uint64_t* empty = is_v ? &v_empty[st] : &k_empty[st];
-      uint64_t* full = is_v ? &v_full[st] : &k_full[st];
-      const int w = lane == 0 ? (int)mbar_wait(empty, ((gidx / kKV) & 1) ^ 1, p.polls) : 1;
-      if (!__shfl_sync(0xffffffffu, w, 0)) return false;
-      uint8_t* dst = (is_v ? Vs : Ks) + st * L::kK;
-      if (lane == 0) mbar_arrive_expect_tx(full, L::kK);
-      __syncwarp();
-      const bool mem = j < I.NM;
-      const CUtensorMap* map = is_v ? (mem ? &tmVm : &tmVl) : (mem ? &tmKm : &tmKl);
-      if (mem && bank) {
-        if (lane < kSegs) {
-          const int y = __ldg(p.seg_row + (int64_t)I.b * p.Smax + j * kSegs + lane);
-#pragma unroll
-          for (int dc = 0; dc < L::kBoxes; ++dc)
-            tma_load_2d(dst + dc * (kKeys * 128) + lane * (kSegRows * 128), map, I.g * DH + dc * 64, y, full);
-        }
-      } else if (lane == 0) {
-        const int y = mem ? I.b * p.Mmax + j * kKeys : I.b * p.Lloc + (j - I.NM) * kKeys;
-#pragma unroll
-        for (int dc = 0; dc < L::kBoxes; ++dc) tma_load_2d(dst + dc * (kKeys * 128), map, I.g * DH + dc * 64, y, full);
-      }
-      return true;
-    };
-    for (int r = 0; ok; ++r) {
-      const int64_t wi = item_of(r);
-      if (wi >= n_items) break;
-      const Item I = item_at(p, wi);
-      const int base = nv;  // global index of the item's first tile (every earlier V tile is issued)
-      // Q of the item, once the previous item's S MMAs no longer read the Q buffer
-      int w = 1;
-      if (lane == 0) {
-        w = r == 0 || mbar_wait(q_empty, (r - 1) & 1, p.polls);
-        if (w) {
-          mbar_arrive_expect_tx(q_full, L::kQ);
-          for (int hh = 0; hh < p.G; ++hh)
+    // K and V tiles have their own stages: K_j is free once S_j is done, V_j
+    // once PV_j is, and the tensor core runs S_{j+1} before PV_j, so the loads
+    // go K0, K1, K2, V0, K3, V1, K4, ... in the order their stages free up.
+    // Lane 0 waits and arms the barriers; a memory tile read from the bank is
+    // kSegs boxes of kSegRows rows, one per lane (each lands on a 1 KB
+    // swizzle atom, so the tile's layout is that of one 128-row box).
+    {
+      auto load = [&](int j, bool is_v) -> bool {
+        const int st = j % kKV;
+        uint64_t* empty = is_v ? &v_empty[st] : &k_empty[st];
+        uint64_t* full = is_v ? &v_full[st] : &k_full[st];
+        const int ok = lane == 0 ? (int)mbar_wait(empty, ((j / kKV) & 1) ^ 1, p.polls) : 1;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+        uint8_t* dst = (is_v ? Vs : Ks) + st * L::kK;
+        if (lane == 0) mbar_arrive_expect_tx(full, L::kK);
+        __syncwarp();
+        const bool mem = j >= NL;
+        const int jm = j - NL;  // memory tile index
+        const CUtensorMap* map = is_v ? (mem ? &tmVm : &tmVl) : (mem ? &tmKm : &tmKl);
+        if (mem && bank) {
+          if (lane < kSegs) {
+            const int y = jm == 0 ? seg0 : __ldg(p.seg_row + (int64_t)b * p.Smax + jm * kSegs + lane);
 #pragma unroll
             for (int dc = 0; dc < L::kBoxes; ++dc)
-              tma_load_2d(Qs + dc * (kRows * 128) + hh * p.TB * 128, &tmQ, (I.g * p.G + hh) * DH + dc * 64,
-                          I.b * p.Tq + I.t0, q_full);
+              tma_load_2d(dst + dc * (kKeys * 128) + lane * (kSegRows * 128), map, g * DH + dc * 64, y, full);
+          }
+        } else if (lane == 0) {
+          const int y = mem ? b * p.Mmax + jm * kKeys : b * p.Lloc + j * kKeys;
+#pragma unroll
+          for (int dc = 0; dc < L::kBoxes; ++dc)
+            tma_load_2d(dst + dc * (kKeys * 128), map, g * DH + dc * 64, y, full);
         }
-      }
-      if (!__shfl_sync(0xffffffffu, w, 0)) {
-        ok = false;
-        break;
-      }
-      ++nq;
-      for (int j = 0; ok && j < kKV && j < I.T; ++j) {
-        if (!(ok = load(I, j, base + j, false))) break;
+        return true;
+      };
+      int nk = 0, nv = 0;
+      bool ok = true;
+      while (ok && nk < kKV && nk < T) {
+        if (!(ok = load(nk, false))) break;
         ++nk;
       }
-      for (int j = 0; ok && j < I.T; ++j) {
-        if (!(ok = load(I, j, base + j, true))) break;
+      for (int j = 0; ok && j < T; ++j) {
+        if (!(ok = load(j, true))) break;
         ++nv;
-        if (j + kKV < I.T) {
-          if (!(ok = load(I, j + kKV, base + j + kKV, false))) break;
+        if (nk < T) {
+          if (!(ok = load(nk, false))) break;
           ++nk;
         }
       }
-    }
-    if (!ok) timed_out = true;
-    // drain the copies this warp issued
-    if (lane == 0) {
-      if (nq > 0 && !mbar_wait(q_full, (nq - 1) & 1, kWaitPolls)) timed_out = true;
-      for (int st = 0; st < kKV; ++st) {
-        // the last fill of stage st is fill (n - 1 - st) / kKV of it
-        if (st < nk && !mbar_wait(&k_full[st], ((nk - 1 - st) / kKV) & 1, kWaitPolls)) timed_out = true;
-        if (st < nv && !mbar_wait(&v_full[st], ((nv - 1 - st) / kKV) & 1, kWaitPolls)) timed_out = true;
+      if (!ok) timed_out = true;
+      // drain the copies this warp issued
+      if (lane == 0) {
+        if (!mbar_wait(q_full, 0, kWaitPolls)) timed_out = true;
+        for (int st = 0; st < kKV; ++st) {
+          // the last fill of stage st is fill (n - 1 - st) / kKV of it
+          if (st < nk && !mbar_wait(&k_full[st], ((nk - 1 - st) / kKV) & 1, kWaitPolls)) timed_out = true;
+          if (st < nv && !mbar_wait(&v_full[st], ((nv - 1 - st) / kKV) & 1, kWaitPolls)) timed_out = true;
+        }
       }
     }
   } else if (warp == 1) {
@@ -305,9 +280,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // the field never carries)
       const uint64_t dq = desc_k_sw128(smem_u32(Qs));
       const uint64_t dk0 = desc_k_sw128(smem_u32(Ks)), dv0 = desc_mn_sw128(smem_u32(Vs), kKeys * 128);
-      // S of tile j (counted over all items) goes to TMEM buffer j & 1, which
-      // holds P of tile j - 2 until its PV has read it; that PV was issued
-      // earlier, and the MMAs run in issue order.
+      // S_j goes to TMEM buffer j & 1, which holds P_{j-2} until PV_{j-2} has
+      // read it; PV_{j-2} was issued earlier, and the MMAs run in issue order.
       auto issue_S = [&](int j) -> bool {
         const int ks = j % kKV;
         if (!mbar_wait(&k_full[ks], (j / kKV) & 1, p.polls)) return false;
@@ -323,183 +297,155 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mma_commit(&k_empty[ks]);
         return true;
       };
-      bool ok = true;
-      int jt = 0;  // tiles over all items
-      for (int r = 0; ok; ++r) {
-        const int64_t wi = item_of(r);
-        if (wi >= n_items) break;
-        const Item I = item_at(p, wi);
-        const int ob = r & 1;
-        const uint32_t tO = tO0 + ob * DH;
-        // the item's first S needs its Q; its last S frees the Q buffer for the next item
-        if (!(ok = mbar_wait(q_full, r & 1, p.polls) && issue_S(jt))) break;
-        if (I.T == 1) mma_commit(q_empty);
-        for (int j = 0; j < I.T; ++j, ++jt) {
-          const int st = jt & 1, vs = jt % kKV;
-          if (j + 1 < I.T) {
-            if (!(ok = issue_S(jt + 1))) break;
-            if (j + 2 == I.T) mma_commit(q_empty);
-          }
-          if (!mbar_wait(&p_full[st], (jt >> 1) & 1, p.polls) || !mbar_wait(&v_full[vs], (jt / kKV) & 1, p.polls) ||
-              (j == 0 && r >= 2 && !mbar_wait(&o_free[ob], ((r >> 1) - 1) & 1, p.polls))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t dv = dv0 + (uint64_t)((vs * L::kK) >> 4);
-          // A = P from TMEM: 16 keys of bf16 per step are 8 columns
-#pragma unroll
-          for (int k = 0; k < kKeys / 16; ++k)
-            mma_bf16_ts(tO, tS0 + st * kKeys + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idO,
-                        (j > 0 || k > 0) ? 1u : 0u);
-          mma_commit(&p_free[st]);
-          mma_commit(&v_empty[vs]);
+      bool ok = mbar_wait(q_full, 0, p.polls) && issue_S(0);
+      for (int j = 0; ok && j < T; ++j) {
+        const int st = j & 1, vs = j % kKV;
+        if (j + 1 < T && !issue_S(j + 1)) {
+          ok = false;
+          break;
         }
+        if (!mbar_wait(&p_full[st], (j >> 1) & 1, p.polls) || !mbar_wait(&v_full[vs], (j / kKV) & 1, p.polls)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t dv = dv0 + (uint64_t)((vs * L::kK) >> 4);
+        // A = P_j from TMEM: 16 keys of bf16 per step are 8 columns
+#pragma unroll
+        for (int k = 0; k < kKeys / 16; ++k)
+          mma_bf16_ts(tO, tS0 + st * kKeys + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idO,
+                      (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&p_free[st]);
+        mma_commit(&v_empty[vs]);
       }
       if (!ok) timed_out = true;
       mma_commit(drain);
       if (!mbar_wait(drain, 0, kWaitPolls)) timed_out = true;
     }
   } else {
-    // ---------------------------------------------------------------- softmax / output
+    // ---------------------------------------------------------------- softmax
     const int q = warp & 3;
-    const int row = q * 32 + lane;                    // this thread's row (TMEM lane)
-    const int hh = row / p.TB, tl = row - hh * p.TB;
+    const int r = q * 32 + lane;                      // this thread's row (TMEM lane)
+    const int hh = r / p.TB, tl = r - hh * p.TB;
+    const int t = t0 + tl;
+    const int pos = p.Lloc - p.Tq + t;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float sl2 = p.scale_log2;
-    int jt = 0;  // tiles over all items
-    for (int r = 0; !timed_out; ++r) {
-      const int64_t wi = item_of(r);
-      if (wi >= n_items) break;
-      const Item I = item_at(p, wi);
-      if (!bank && row == 0 && I.qb == 0 && I.g == 0) {
-        const int M0 = __ldg(p.mem_len + I.b);
-        if (M0 < 0 || M0 > p.Mmax) raise_flag(p.err_flag, MSA_FLAG_INDEX_OOB);
-      }
-      const int ob = r & 1;
-      const uint32_t tO = tO0 + ob * DH;
-      const int t = I.t0 + tl;
-      const int pos = p.Lloc - p.Tq + t;
-      float m_run = -INFINITY, l_run = 0.f;  // running max in the scaled log2 domain
-      for (int j = 0; j < I.T; ++j, ++jt) {
-        const int st = jt & 1;
-        // a bank tile's segment counts (one byte per segment), loaded before the wait
-        uint4 segc = make_uint4(0u, 0u, 0u, 0u);
-        if (bank && j < I.NM)
-          segc = __ldg(reinterpret_cast<const uint4*>(p.seg_cnt + (int64_t)I.b * p.Smax + j * kSegs));
-        // waits are decided warp-wide so the warp-collective tcgen05 ops are never split
-        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (jt >> 1) & 1, p.polls))) {
-          timed_out = true;
-          break;
-        }
-        tc_fence_after();
-        float s[kKeys];
-#pragma unroll
-        for (int c = 0; c < kKeys; c += 16)
-          tmem_ld16(tmem + lane_off + st * kKeys + c, *reinterpret_cast<float(*)[16]>(&s[c]));
-        tmem_ld_wait();
-        // keys [0, lim) of this tile are visible to this row; most tiles are whole
-        const bool memt = j < I.NM;
-        if (memt && bank) {
-          // key c of the tile is row c % kSegRows of segment c / kSegRows
-          static_assert(kSegs == 16 && kSegRows == 8, "four segment counts per word");
-          const uint32_t full8 = 0x08080808u;
-          if (!(segc.x == full8 && segc.y == full8 && segc.z == full8 && segc.w == full8)) {
-            const uint32_t cw[4] = {segc.x, segc.y, segc.z, segc.w};
-#pragma unroll
-            for (int c = 0; c < kKeys; ++c) {
-              const uint32_t n = (cw[c >> 5] >> (((c >> 3) & 3) * 8)) & 0xffu;
-              s[c] = (uint32_t)(c & 7) < n ? s[c] : -INFINITY;
-            }
-          }
-        } else {
-          const int base = memt ? j * kKeys : (j - I.NM) * kKeys;
-          const int lim = memt ? I.M - base : pos - base + 1;
-          const bool whole = __all_sync(0xffffffffu, lim >= kKeys);
-          if (!whole) {
-#pragma unroll
-            for (int c = 0; c < kKeys; ++c) s[c] = c < lim ? s[c] : -INFINITY;
-          }
-        }
-        // eight independent chains of three-input maxima (max is exact in any order)
-        static_assert(kKeys == 128, "the chains cover 128 keys");
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = fmax3(s[i], s[i + 8], s[i + 16]);
-#pragma unroll
-        for (int c = 24; c < 120; c += 16)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[c + i], s[c + 8 + i]);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[120 + i]);
-        const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-        // move the max (and rescale O) only when it grows by more than 2^8
-        const float mt = mx * sl2;
-        const bool first = m_run == -INFINITY;
-        const bool grow = mt > m_run + kRescaleLog2;
-        float corr = 1.f;
-        if (grow) {
-          corr = first ? 0.f : fast_exp2(m_run - mt);
-          m_run = mt;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
-          // O must hold every earlier PV of the item before it is rescaled
-          const int jp = jt - 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(&p_free[jp & 1], (jp >> 1) & 1, p.polls))) {
-            timed_out = true;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < DH; c += 16) {
-            float o[16];
-            tmem_ld16(tO + lane_off + c, o);
-            tmem_ld_wait();
-            uint32_t w[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(o[i] * corr);
-            tmem_st16(tO + lane_off + c, w);
-          }
-          tmem_st_wait();
-        }
-        l_run *= corr;
-        const float nm = -m_run;
-        // P over S: 32 keys (16 columns of bf16 pairs) per store; the scaled arguments and the row
-        // sums in packed pairs (one f32x2 instruction for two keys)
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), nmx2 = f2_pack(nm, nm);
-        uint64_t lsa2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-#pragma unroll
-        for (int c0 = 0; c0 < kKeys; c0 += 32) {
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(s[c0 + 2 * i], s[c0 + 2 * i + 1]), sl2x2, nmx2), x0, x1);
-            const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-            lsa2[i & 1] = f2_add(lsa2[i & 1], f2_pack(e0, e1));
-            w[i] = pack_bf16x2(e0, e1);
-          }
-          tmem_st16(tmem + lane_off + st * kKeys + c0 / 2, w);
-        }
-        float lsa[4];
-        f2_unpack(lsa2[0], lsa[0], lsa[1]);
-        f2_unpack(lsa2[1], lsa[2], lsa[3]);
-        l_run += (lsa[0] + lsa[1]) + (lsa[2] + lsa[3]);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&p_full[st]);
-      }
-      if (timed_out) break;
-      // output of the item: O / l, lse = (m + log2 l) ln 2; then O buffer ob is free for item r + 2
-      const int jl = jt - 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&p_free[jl & 1], (jl >> 1) & 1, p.polls))) {
+    float m_run = -INFINITY, l_run = 0.f;  // running max in the scaled log2 domain
+    for (int j = 0; j < T; ++j) {
+      const int st = j & 1;
+      // a bank tile's segment counts (one byte per segment), loaded before the wait
+      uint4 segc = make_uint4(0u, 0u, 0u, 0u);
+      if (bank && j >= NL)
+        segc = __ldg(reinterpret_cast<const uint4*>(p.seg_cnt + (int64_t)b * p.Smax + (j - NL) * kSegs));
+      // waits are decided warp-wide so the warp-collective tcgen05 ops are never split
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1, p.polls))) {
         timed_out = true;
         break;
       }
       tc_fence_after();
+      float s[kKeys];
+#pragma unroll
+      for (int c = 0; c < kKeys; c += 16) tmem_ld16(tmem + lane_off + st * kKeys + c, *reinterpret_cast<float(*)[16]>(&s[c]));
+      tmem_ld_wait();
+      // keys [0, lim) of this tile are visible to this row; most tiles are whole
+      const bool memt = j >= NL;
+      if (memt && bank) {
+        // key c of the tile is row c % kSegRows of segment c / kSegRows
+        static_assert(kSegs == 16 && kSegRows == 8, "four segment counts per word");
+        const uint32_t full8 = 0x08080808u;
+        if (!(segc.x == full8 && segc.y == full8 && segc.z == full8 && segc.w == full8)) {
+          const uint32_t cw[4] = {segc.x, segc.y, segc.z, segc.w};
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c) {
+            const uint32_t n = (cw[c >> 5] >> (((c >> 3) & 3) * 8)) & 0xffu;
+            s[c] = (uint32_t)(c & 7) < n ? s[c] : -INFINITY;
+          }
+        }
+      } else {
+        const int base = memt ? (j - NL) * kKeys : j * kKeys;
+        const int lim = memt ? M - base : pos - base + 1;
+        const bool whole = __all_sync(0xffffffffu, lim >= kKeys);
+        if (!whole) {
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c) s[c] = c < lim ? s[c] : -INFINITY;
+        }
+      }
+      // eight independent chains of three-input maxima (max is exact in any order)
+      static_assert(kKeys == 128, "the chains cover 128 keys");
+      float m8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = fmax3(s[i], s[i + 8], s[i + 16]);
+#pragma unroll
+      for (int c = 24; c < 120; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[120 + i]);
+      const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+      // move the max (and rescale O) only when it grows by more than 2^8
+      const float mt = mx * sl2;
+      const bool first = m_run == -INFINITY;
+      const bool grow = mt > m_run + kRescaleLog2;
+      float corr = 1.f;
+      if (grow) {
+        corr = first ? 0.f : fast_exp2(m_run - mt);
+        m_run = mt;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O must hold every earlier PV before it is rescaled
+        const int jp = j - 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&p_free[jp & 1], (jp >> 1) & 1, p.polls))) {
+          timed_out = true;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < DH; c += 16) {
+          float o[16];
+          tmem_ld16(tO + lane_off + c, o);
+          tmem_ld_wait();
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(o[i] * corr);
+          tmem_st16(tO + lane_off + c, w);
+        }
+        tmem_st_wait();
+      }
+      l_run *= corr;
+      const float nm = -m_run;
+      // P_j over S_j: 32 keys (16 columns of bf16 pairs) per store; the scaled arguments and the row
+      // sums in packed pairs (one f32x2 instruction for two keys)
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), nmx2 = f2_pack(nm, nm);
+      uint64_t lsa2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+      for (int c0 = 0; c0 < kKeys; c0 += 32) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[c0 + 2 * i], s[c0 + 2 * i + 1]), sl2x2, nmx2), x0, x1);
+          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+          lsa2[i & 1] = f2_add(lsa2[i & 1], f2_pack(e0, e1));
+          w[i] = pack_bf16x2(e0, e1);
+        }
+        tmem_st16(tmem + lane_off + st * kKeys + c0 / 2, w);
+      }
+      float lsa[4];
+      f2_unpack(lsa2[0], lsa[0], lsa[1]);
+      f2_unpack(lsa2[1], lsa[2], lsa[3]);
+      l_run += (lsa[0] + lsa[1]) + (lsa[2] + lsa[3]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[st]);
+    }
+    // output: O / l, lse = (m + log2 l) ln 2
+    const int jl = T - 1;
+    if (!timed_out && __all_sync(0xffffffffu, mbar_wait(&p_free[jl & 1], (jl >> 1) & 1, p.polls))) {
+      tc_fence_after();
       const float inv = 1.f / l_run;
       const bool rvalid = t < p.Tq;
-      __nv_bfloat16* orow = p.O + (((int64_t)I.b * p.Tq + t) * p.Hq + I.g * p.G + hh) * DH;
+      __nv_bfloat16* orow = p.O + (((int64_t)b * p.Tq + t) * p.Hq + g * p.G + hh) * DH;
 #pragma unroll
       for (int c = 0; c < DH; c += 16) {
         float o[16];
@@ -515,9 +461,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
       }
       if (rvalid && p.lse)
-        p.lse[((int64_t)I.b * p.Hq + I.g * p.G + hh) * p.Tq + t] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-      tc_fence_before();
-      mbar_arrive(&o_free[ob]);
+        p.lse[((int64_t)b * p.Hq + g * p.G + hh) * p.Tq + t] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    } else {
+      timed_out = true;
     }
   }
 
@@ -575,11 +521,11 @@ cudaError_t launch_dh(const AttnArgs& a, cudaStream_t s) {
   p.polls = tp < 0 ? kWaitPolls : (uint32_t)(tp < (int64_t)kWaitPolls ? tp : kWaitPolls);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
   if (e != cudaSuccess) return e;
-  // persistent: one CTA per SM (shared memory allows no more) walks its share of the items
-  const int64_t n_items = (int64_t)p.n_qblk * a.Hkv * a.B;
-  const int64_t grid = n_items < sm_count() ? n_items : sm_count();
+  dim3 grid((unsigned)p.n_qblk, (unsigned)a.Hkv, (unsigned)a.B);
   count_launch();
-  attn_tc_kernel<DH><<<(unsigned)grid, kThreads, L::kSmem, s>>>(tq, tkm, tvm, tkl, tvl, p);
+  if (a.seg_row)  // overlaps the plan kernel just before it on the stream
+    return launch_pdl(attn_tc_kernel<DH>, grid, dim3(kThreads), (size_t)L::kSmem, s, tq, tkm, tvm, tkl, tvl, p);
+  attn_tc_kernel<DH><<<grid, kThreads, L::kSmem, s>>>(tq, tkm, tvm, tkl, tvl, p);
   return cudaGetLastError();
 }
 

@@ -116,6 +116,9 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a, int row_vecs)
 // are padding: row C (past the end of the bank, which a TMA load reads as
 // zeros) and count 0.
 __global__ void __launch_bounds__(128) plan_kernel(PlanArgs a) {
+  // the prefill attention kernel that reads the plan is launched as a programmatic
+  // dependent: let it start its set-up now (it waits for this grid before reading)
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t b = (int64_t)blockIdx.x * 4 + warp;
   if (b >= a.B) return;
