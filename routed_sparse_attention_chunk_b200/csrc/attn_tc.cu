@@ -75,7 +75,8 @@ struct ALayout {
   static constexpr int kK = kKeys * DH * 2;  // one K (or V) tile
   static constexpr int kBar = 8 * 24;
   static constexpr int kSmem = 1024 + kQ + 2 * kKV * kK + kBar;  // Q, K[kKV], V[kKV]
-  static constexpr uint32_t kTmemCols = 512;  // S0, S1 (128 each), O (DH)
+  static constexpr uint32_t kTmemCols = 512;  // S0, S1 (128 each), O (DH), Q (DH / 2)
+  static_assert(2 * kKeys + DH + DH / 2 <= (int)kTmemCols, "tensor memory columns");
   static_assert(kSmem <= 232448, "shared memory of one CTA");
 };
 
@@ -132,7 +133,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* p_full = s_full + 2;           // [2] P written over S -> MMA
   uint64_t* p_free = p_full + 2;           // [2] PV MMA done -> softmax (O up to date)
   uint64_t* drain = p_free + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* q_tmem = drain + 1;            // Q copied into tensor memory (softmax threads) -> MMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_tmem + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // longest blocks first: block index 0 takes the last query block
@@ -158,6 +160,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&p_free[i], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(q_tmem, 128);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -168,7 +171,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS0 = tmem, tO = tmem + 2 * kKeys;
+  // TMEM columns: S0, S1 (128 each), O (DH), then Q as the S MMAs' A operand (DH / 2: bf16 pairs)
+  const uint32_t tS0 = tmem, tO = tmem + 2 * kKeys, tQ = tmem + 2 * kKeys + DH;
   bool timed_out = false;
   if (warp == 0 && lane == 0) {
     // the query rows do not depend on the kernel this one may overlap
@@ -278,7 +282,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // descriptors of the operand bases; a k-step adds its byte offset / 16 to
       // the 14-bit start-address field (shared addresses stay below 256 KB, so
       // the field never carries)
-      const uint64_t dq = desc_k_sw128(smem_u32(Qs));
       const uint64_t dk0 = desc_k_sw128(smem_u32(Ks)), dv0 = desc_mn_sw128(smem_u32(Vs), kKeys * 128);
       // S_j goes to TMEM buffer j & 1, which holds P_{j-2} until PV_{j-2} has
       // read it; PV_{j-2} was issued earlier, and the MMAs run in issue order.
@@ -289,15 +292,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const uint64_t dk = dk0 + (uint64_t)((ks * L::kK) >> 4);
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
+          // A = Q from TMEM (16 elements of bf16 per step are 8 columns), B = K from its tile
           const int box = k >> 2, kk = k & 3;
-          mma_bf16_ss(tS0 + (j & 1) * kKeys, dq + (uint64_t)((box * kRows * 128 + kk * 32) >> 4),
-                      dk + (uint64_t)((box * kKeys * 128 + kk * 32) >> 4), idS, k > 0 ? 1u : 0u);
+          mma_bf16_ts(tS0 + (j & 1) * kKeys, tQ + k * 8, dk + (uint64_t)((box * kKeys * 128 + kk * 32) >> 4), idS,
+                      k > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[j & 1]);
         mma_commit(&k_empty[ks]);
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, p.polls) && issue_S(0);
+      // the S MMAs read Q from tensor memory once the softmax threads have put it there
+      bool ok = mbar_wait(q_tmem, 0, p.polls) && issue_S(0);
       for (int j = 0; ok && j < T; ++j) {
         const int st = j & 1, vs = j % kKV;
         if (j + 1 < T && !issue_S(j + 1)) {
@@ -331,6 +336,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int pos = p.Lloc - p.Tq + t;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float sl2 = p.scale_log2;
+    // This row of Q into tensor memory: S = Q K^T then takes Q from TMEM and
+    // reads only K from shared memory (both operands from shared memory would
+    // use its whole read bandwidth while the TMA writes the next tiles).  The
+    // row's 16-byte pieces sit in the 128-byte-swizzled layout of the TMA tile.
+    if (!__all_sync(0xffffffffu, mbar_wait(q_full, 0, p.polls))) timed_out = true;
+    if (!timed_out) {
+      uint32_t w[DH / 2];
+#pragma unroll
+      for (int box = 0; box < DH / 64; ++box)
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint4 v = *reinterpret_cast<const uint4*>(Qs + box * (kRows * 128) + r * 128 + ((c8 ^ (r & 7)) << 4));
+          w[box * 32 + c8 * 4 + 0] = v.x;
+          w[box * 32 + c8 * 4 + 1] = v.y;
+          w[box * 32 + c8 * 4 + 2] = v.z;
+          w[box * 32 + c8 * 4 + 3] = v.w;
+        }
+#pragma unroll
+      for (int c = 0; c < DH / 2; c += 16) tmem_st16(tQ + lane_off + c, *reinterpret_cast<const uint32_t(*)[16]>(&w[c]));
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    mbar_arrive(q_tmem);
     float m_run = -INFINITY, l_run = 0.f;  // running max in the scaled log2 domain
     for (int j = 0; j < T; ++j) {
       const int st = j & 1;

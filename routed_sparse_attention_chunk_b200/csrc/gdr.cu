@@ -327,8 +327,68 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_kernel(GdrParams p) {
   }
 }
 
+// Few tokens (decoding): the recurrence itself, token by token.  One CTA per
+// (value head, query); value column c is kept by two threads, each holding
+// half of h[:, c] in registers (the columns evolve independently):
+//   u = k . h[:, c];  h[:, c] = g' h[:, c] + beta k (v_c - g' u)  (g' = exp(g));  o_c = scale q . h[:, c]
+// the two halves' partial dot products meet in shared memory.
+constexpr int kTokenMax = 16;  // sequences up to this length take this kernel
+
+template <typename T, int DH>
+__global__ void __launch_bounds__(2 * DH) gdr_token_kernel(GdrParams p) {
+  constexpr int HR = DH / 2;  // rows of h per thread
+  __shared__ float ks[DH], qs[DH], part[2][DH];
+  const int half = threadIdx.x / DH, c = threadIdx.x % DH, r0 = half * HR;
+  const int hv = blockIdx.x;
+  const int64_t b = blockIdx.y;
+  const int hk = hv / (p.Hv / p.Hk);
+  const T* q = static_cast<const T*>(p.q);
+  const T* k = static_cast<const T*>(p.k);
+  const T* v = static_cast<const T*>(p.v);
+  T* o = static_cast<T*>(p.o);
+  const float* h0 = p.h0 ? p.h0 + ((int64_t)b * p.Hv + hv) * DH * DH : nullptr;
+  float h[HR];
+#pragma unroll
+  for (int i = 0; i < HR; ++i) h[i] = h0 ? h0[(int64_t)(r0 + i) * DH + c] : 0.f;  // a row: consecutive over c
+  for (int t = 0; t < p.T; ++t) {
+    const int64_t tok = (int64_t)b * p.T + t;
+    const int64_t gi = tok * p.Hv + hv;
+    __syncthreads();  // the previous token is done with ks, qs, part
+    if (half == 0) ks[c] = to_f32(k[(tok * p.Hk + hk) * DH + c]);
+    else qs[c] = to_f32(q[(tok * p.Hk + hk) * DH + c]);
+    __syncthreads();
+    float u = 0.f;
+#pragma unroll
+    for (int i = 0; i < HR; ++i) u = fmaf(ks[r0 + i], h[i], u);
+    part[half][c] = u;
+    __syncthreads();
+    const float a = expf(p.g[gi]), be = p.beta[gi];
+    const float w = be * (to_f32(v[gi * DH + c]) - a * (part[0][c] + part[1][c]));
+    float oc = 0.f;
+#pragma unroll
+    for (int i = 0; i < HR; ++i) {
+      h[i] = fmaf(a, h[i], ks[r0 + i] * w);
+      oc = fmaf(qs[r0 + i], h[i], oc);
+    }
+    __syncthreads();  // every thread has read part[.][c] before it is rewritten
+    part[half][c] = oc;
+    __syncthreads();
+    if (half == 0) o[gi * DH + c] = from_f32<T>(p.scale * (part[0][c] + part[1][c]));
+  }
+  if (p.hT) {
+    float* hT = p.hT + ((int64_t)b * p.Hv + hv) * DH * DH;
+#pragma unroll
+    for (int i = 0; i < HR; ++i) hT[(int64_t)(r0 + i) * DH + c] = h[i];
+  }
+}
+
 template <typename T, int DH>
 cudaError_t launch_t(const GdrParams& p, cudaStream_t s) {
+  if (p.T <= kTokenMax) {
+    count_launch();
+    gdr_token_kernel<T, DH><<<dim3((unsigned)p.Hv, (unsigned)p.B), 2 * DH, 0, s>>>(p);
+    return cudaGetLastError();
+  }
   constexpr int NV = 32;
   using L = GLayout<DH, NV>;
   cudaError_t e =

@@ -43,7 +43,9 @@ def _gpu(q, k, v, lg, beta, h0, scale=0.0):
 @pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("B,T,Hk,Hv", [(2, 150, 2, 4),    # three chunks, the last one ragged (22 tokens)
                                        (1, 64, 1, 1),     # exactly one chunk
-                                       (3, 1, 2, 2),      # one decode token
+                                       (3, 1, 2, 2),      # one decode token (the token-by-token kernel)
+                                       (2, 16, 2, 4),     # the token-by-token kernel's longest sequence
+                                       (1, 17, 1, 2),     # one token more: a single ragged chunk
                                        (1, 1000, 1, 2)])  # sixteen chunks
 def test_chunked_rule_matches_the_recurrence(dt, B, T, Hk, Hv):
     q, k, v, lg, beta, h0 = _inputs(B, T, Hk, Hv, dt, seed=T + Hv)
