@@ -16,17 +16,27 @@
 //     MMA's A operand straight from tensor memory and V MN-major from its TMA
 //     tile.  The tensor core runs its MMAs in issue order, so S_{j+2} (issued
 //     after PV_j) never overwrites P_j before PV_j has read it;
-//   * K and V tiles have separate three-deep stages: K_j is released when S_j
-//     is done and V_j when PV_j is, which keeps three loads in flight against
-//     the latency of a TMA tile;
+//   * key tile j's K and V share one of three stages and one barrier, so the
+//     MMA warp waits once per tile for both operands (each of its waits costs
+//     ~100-200 cycles on the critical path; separate K and V barriers made the
+//     dense-memory kernel 2.4% slower); the stage is released when PV_j is done;
+//   * S = Q K^T runs at N = 128, where one CTA's tensor core does a
+//     128 x 128 x 128 product in ~705 cycles with B K-major and ~853 with B
+//     MN-major (V), against 512 at N = 256 (a clock64 probe of back-to-back
+//     MMAs); a CTA pair (cta_group::2, M = 256, each CTA half of B) takes ~947,
+//     so the pair's halved tile loads did not pay: it ran 2-5% slower than one
+//     CTA.  An N = 256 S tile would need 2 x 256 TMEM columns for S alone;
 //   * the running max is only moved (and O rescaled in TMEM) when it grows by
 //     more than 2^8, so most tiles skip the rescale; the final 1/l and the
 //     log-sum-exp use the same max, which keeps the result exact;
-//   * the softmax warps are the critical path (one warp per SM sub-partition,
-//     bound by instruction issue; the two that share a sub-partition with the
-//     TMA and MMA warps finish last): the row max runs as eight independent
-//     chains of three-input maxima, the scaled arguments and row sums use
-//     packed f32x2 math, and the MMA warp reuses its operand descriptors.
+//   * a tile's pace is set by the MMA warp's serial chain (issue S_{j+1}, wait
+//     for P_j, issue PV_j; the tensor core takes in a group of MMAs about as
+//     fast as it runs them) and by the softmax warps (one per SM
+//     sub-partition): the row max runs as eight independent chains of
+//     three-input maxima, the scaled arguments and row sums use packed f32x2
+//     math, four of every sixteen key pairs take a polynomial 2^x on the FMA
+//     pipe instead of the transcendental unit (1-2% faster; eight of sixteen
+//     was slower), and the MMA warp reuses its operand descriptors.
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
 // issuer, warps 2..5 softmax / correction / output (one row per thread).
 // Every wait is bounded and ends the CTA with MSA_FLAG_TIMEOUT on expiry.
@@ -47,7 +57,7 @@ constexpr int kKeys = 128;   // keys per tile
 constexpr int kThreads = 192;
 constexpr uint32_t kWaitPolls = 1u << 24;
 constexpr float kRescaleLog2 = 8.0f;  // move the running max only when it grows by more than this
-constexpr int kKV = 3;                // K and V stages
+constexpr int kKV = 3;                // K + V stages
 
 struct AttnTcParams {
   const int32_t* mem_len;
@@ -112,6 +122,37 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
+// 2^x for a pair of arguments on the FMA and integer pipes, leaving the
+// transcendental unit (whose ex2 throughput bounds the softmax) to the other
+// keys: x = j + f with j = round(x) (read from the mantissa of x + 1.5 * 2^23)
+// and f in [-1/2, 1/2]; 2^f by a cubic whose coefficients are a weighted
+// least-squares fit of 2^f on [-1/2, 1/2] at Chebyshev nodes refined by Lawson
+// iterations toward equal relative error (max relative error 7.5e-5, far below
+// the bf16 rounding of P); 2^j is added to the exponent field.  Arguments below
+// -126 are clamped there (weights below 2^-126 instead of 0; masked keys give
+// 2^-126 * 2^f, which vanishes in the bf16 P and in the row sum's fp32).
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float& e1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = f2_add(x, f2_pack(kMagic, kMagic));         // round(x) in the low mantissa bits
+  const uint64_t jf = f2_add(t, f2_pack(-kMagic, -kMagic));      // round(x) as a float
+  const uint64_t f = f2_fma(jf, f2_pack(-1.0f, -1.0f), x);        // x - round(x)
+  uint64_t q = f2_fma(f, f2_pack(0.0551716648f, 0.0551716648f), f2_pack(0.2426111251f, 0.2426111251f));
+  q = f2_fma(q, f, f2_pack(0.6932609677f, 0.6932609677f));
+  q = f2_fma(q, f, f2_pack(0.9999280572f, 0.9999280572f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  // the low bits of t hold round(x); shifted by 23 they add it to the exponent
+  e0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  e1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// Of each 16 key pairs of a 32-key store, this many take exp2_poly2 (spread
+// evenly); the rest take the transcendental unit's ex2.
+constexpr int kPolyPairs = 4;
+__host__ __device__ constexpr bool poly_pair(int i) { return (i * kPolyPairs) / 16 != ((i + 1) * kPolyPairs) / 16; }
+
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKm,
@@ -122,14 +163,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* Qs = smem;
   uint8_t* Ks = Qs + L::kQ;          // [kKV] K tiles
-  uint8_t* Vs = Ks + kKV * L::kK;    // [kKV] V tiles
+  uint8_t* Vs = Ks + kKV * L::kK;    // [kKV] V tiles (stage st holds K_j and V_j of one key tile j)
   uint64_t* bars = reinterpret_cast<uint64_t*>(Vs + kKV * L::kK);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;             // [kKV] TMA -> MMA
-  uint64_t* k_empty = k_full + kKV;        // [kKV] S MMA done -> TMA
-  uint64_t* v_full = k_empty + kKV;        // [kKV]
-  uint64_t* v_empty = v_full + kKV;        // [kKV] PV MMA done -> TMA
-  uint64_t* s_full = v_empty + kKV;        // [2] S MMA done -> softmax
+  uint64_t* kv_full = bars + 1;            // [kKV] K and V of a key tile landed -> MMA
+  uint64_t* kv_empty = kv_full + kKV;      // [kKV] PV MMA done with the stage -> TMA
+  uint64_t* s_full = kv_empty + kKV;       // [2] S MMA done -> softmax
   uint64_t* p_full = s_full + 2;           // [2] P written over S -> MMA
   uint64_t* p_free = p_full + 2;           // [2] PV MMA done -> softmax (O up to date)
   uint64_t* drain = p_free + 2;
@@ -149,10 +188,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < kKV; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -215,62 +252,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    // K and V tiles have their own stages: K_j is free once S_j is done, V_j
-    // once PV_j is, and the tensor core runs S_{j+1} before PV_j, so the loads
-    // go K0, K1, K2, V0, K3, V1, K4, ... in the order their stages free up.
-    // Lane 0 waits and arms the barriers; a memory tile read from the bank is
-    // kSegs boxes of kSegRows rows, one per lane (each lands on a 1 KB
-    // swizzle atom, so the tile's layout is that of one 128-row box).
+    // Key tile j's K and V share stage j % kKV and one barrier, so the MMA
+    // warp waits once per tile for its operands; the stage is free once PV_j
+    // is done.  Lane 0 waits and arms the barrier; a memory tile read from the
+    // bank is kSegs boxes of kSegRows rows per matrix, one per lane (each lands
+    // on a 1 KB swizzle atom, so the tile's layout is that of one 128-row box).
     {
-      auto load = [&](int j, bool is_v) -> bool {
+      auto load = [&](int j) -> bool {
         const int st = j % kKV;
-        uint64_t* empty = is_v ? &v_empty[st] : &k_empty[st];
-        uint64_t* full = is_v ? &v_full[st] : &k_full[st];
-        const int ok = lane == 0 ? (int)mbar_wait(empty, ((j / kKV) & 1) ^ 1, p.polls) : 1;
+        const int ok = lane == 0 ? (int)mbar_wait(&kv_empty[st], ((j / kKV) & 1) ^ 1, p.polls) : 1;
         if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
-        uint8_t* dst = (is_v ? Vs : Ks) + st * L::kK;
-        if (lane == 0) mbar_arrive_expect_tx(full, L::kK);
+        uint8_t* dk = Ks + st * L::kK;
+        uint8_t* dv = Vs + st * L::kK;
+        uint64_t* full = &kv_full[st];
+        if (lane == 0) mbar_arrive_expect_tx(full, 2 * L::kK);
         __syncwarp();
         const bool mem = j >= NL;
         const int jm = j - NL;  // memory tile index
-        const CUtensorMap* map = is_v ? (mem ? &tmVm : &tmVl) : (mem ? &tmKm : &tmKl);
+        const CUtensorMap* mk = mem ? &tmKm : &tmKl;
+        const CUtensorMap* mv = mem ? &tmVm : &tmVl;
         if (mem && bank) {
           if (lane < kSegs) {
             const int y = jm == 0 ? seg0 : __ldg(p.seg_row + (int64_t)b * p.Smax + jm * kSegs + lane);
 #pragma unroll
-            for (int dc = 0; dc < L::kBoxes; ++dc)
-              tma_load_2d(dst + dc * (kKeys * 128) + lane * (kSegRows * 128), map, g * DH + dc * 64, y, full);
+            for (int dc = 0; dc < L::kBoxes; ++dc) {
+              tma_load_2d(dk + dc * (kKeys * 128) + lane * (kSegRows * 128), mk, g * DH + dc * 64, y, full);
+              tma_load_2d(dv + dc * (kKeys * 128) + lane * (kSegRows * 128), mv, g * DH + dc * 64, y, full);
+            }
           }
         } else if (lane == 0) {
           const int y = mem ? b * p.Mmax + jm * kKeys : b * p.Lloc + j * kKeys;
 #pragma unroll
-          for (int dc = 0; dc < L::kBoxes; ++dc)
-            tma_load_2d(dst + dc * (kKeys * 128), map, g * DH + dc * 64, y, full);
+          for (int dc = 0; dc < L::kBoxes; ++dc) {
+            tma_load_2d(dk + dc * (kKeys * 128), mk, g * DH + dc * 64, y, full);
+            tma_load_2d(dv + dc * (kKeys * 128), mv, g * DH + dc * 64, y, full);
+          }
         }
         return true;
       };
-      int nk = 0, nv = 0;
+      int n = 0;
       bool ok = true;
-      while (ok && nk < kKV && nk < T) {
-        if (!(ok = load(nk, false))) break;
-        ++nk;
-      }
-      for (int j = 0; ok && j < T; ++j) {
-        if (!(ok = load(j, true))) break;
-        ++nv;
-        if (nk < T) {
-          if (!(ok = load(nk, false))) break;
-          ++nk;
-        }
-      }
+      for (; n < T; ++n)
+        if (!(ok = load(n))) break;
       if (!ok) timed_out = true;
       // drain the copies this warp issued
       if (lane == 0) {
         if (!mbar_wait(q_full, 0, kWaitPolls)) timed_out = true;
         for (int st = 0; st < kKV; ++st) {
           // the last fill of stage st is fill (n - 1 - st) / kKV of it
-          if (st < nk && !mbar_wait(&k_full[st], ((nk - 1 - st) / kKV) & 1, kWaitPolls)) timed_out = true;
-          if (st < nv && !mbar_wait(&v_full[st], ((nv - 1 - st) / kKV) & 1, kWaitPolls)) timed_out = true;
+          if (st < n && !mbar_wait(&kv_full[st], ((n - 1 - st) / kKV) & 1, kWaitPolls)) timed_out = true;
         }
       }
     }
@@ -287,7 +317,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // read it; PV_{j-2} was issued earlier, and the MMAs run in issue order.
       auto issue_S = [&](int j) -> bool {
         const int ks = j % kKV;
-        if (!mbar_wait(&k_full[ks], (j / kKV) & 1, p.polls)) return false;
+        if (!mbar_wait(&kv_full[ks], (j / kKV) & 1, p.polls)) return false;
         tc_fence_after();
         const uint64_t dk = dk0 + (uint64_t)((ks * L::kK) >> 4);
 #pragma unroll
@@ -298,7 +328,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                       k > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[j & 1]);
-        mma_commit(&k_empty[ks]);
         return true;
       };
       // the S MMAs read Q from tensor memory once the softmax threads have put it there
@@ -309,7 +338,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           ok = false;
           break;
         }
-        if (!mbar_wait(&p_full[st], (j >> 1) & 1, p.polls) || !mbar_wait(&v_full[vs], (j / kKV) & 1, p.polls)) {
+        // V_j landed with K_j (S_j waited for both)
+        if (!mbar_wait(&p_full[st], (j >> 1) & 1, p.polls)) {
           ok = false;
           break;
         }
@@ -321,7 +351,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           mma_bf16_ts(tO, tS0 + st * kKeys + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idO,
                       (j > 0 || k > 0) ? 1u : 0u);
         mma_commit(&p_free[st]);
-        mma_commit(&v_empty[vs]);
+        mma_commit(&kv_empty[vs]);
       }
       if (!ok) timed_out = true;
       mma_commit(drain);
@@ -451,9 +481,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float x0, x1;
+          float x0, x1, e0, e1;
           f2_unpack(f2_fma(f2_pack(s[c0 + 2 * i], s[c0 + 2 * i + 1]), sl2x2, nmx2), x0, x1);
-          const float e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+          if (poly_pair(i)) {
+            exp2_poly2(x0, x1, e0, e1);
+          } else {
+            e0 = fast_exp2(x0);
+            e1 = fast_exp2(x1);
+          }
           lsa2[i & 1] = f2_add(lsa2[i & 1], f2_pack(e0, e1));
           w[i] = pack_bf16x2(e0, e1);
         }

@@ -79,6 +79,8 @@ def _oracle(Q, Kl, Vl, idx, coff, Kb, Vb, Mmax, D):
     (6, 1, 300, 32, 8, 16, 300, 3),       # decode, 4 query rows per KV head
     (3, 2, 260, 32, 8, 5, 80, 4),         # decode, 8 rows per KV head, overflow
     (2, 16, 48, 8, 8, 7, 64, 5),          # prefill MHA (G = 1: 8-token blocks)
+    (3, 24, 90, 32, 8, 11, 256, 6),       # one ragged block of rows per KV head, two memory tiles
+    (1, 160, 160, 64, 8, 16, 512, 7),     # G = 8: ten 16-token blocks, four memory tiles
 ])
 def test_indexed_attention_ragged_documents(B, Tq, Lloc, Hq, Hkv, k, Mmax, seed):
     rng = np.random.default_rng(seed)

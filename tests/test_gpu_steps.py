@@ -338,6 +338,8 @@ def test_attention_bf16(B, Tq, Lloc, Hq, Hkv, d, Mmax, mem_lens):
     (2, 1100, 1300, 32, 8, 256, [256, 37]),       # local history longer than the query, partial last block
     (1, 600, 600, 64, 8, 128, [128]),             # G=8: 16 tokens per tile, many tiles
     (2, 512, 512, 40, 40, 64, [64, 30]),          # G=1 with 40 heads: 128 tokens per tile
+    (2, 20, 300, 32, 8, 128, [128, 50]),          # one ragged block of rows per KV head
+    (1, 33, 33, 32, 8, 0, [0]),                   # two blocks, the second with one token, no memory
 ])
 def test_attention_bf16_tensor_core_tiling(B, Tq, Lloc, Hq, Hkv, Mmax, mem_lens):
     Q, Kl, Vl, Km, Vm, ml = _attn_inputs(B, Tq, Lloc, Hq, Hkv, 128, Mmax, mem_lens, torch.bfloat16, 4)

@@ -16,9 +16,10 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def test_expired_waits_raise_the_timeout_flag_and_the_next_call_is_correct():
+@pytest.mark.parametrize("Tq", [128, 24])  # four blocks of rows per KV head; one ragged block
+def test_expired_waits_raise_the_timeout_flag_and_the_next_call_is_correct(Tq):
     g = torch.Generator(device=DEV).manual_seed(5)
-    B, Tq, Lloc, Hq, Hkv, M = 1, 128, 256, 32, 8, 64
+    B, Lloc, Hq, Hkv, M = 1, 256, 32, 8, 64
     r = lambda *s: (0.5 * torch.randn(s, generator=g, device=DEV)).bfloat16()
     Q, Kl, Vl, Km, Vm = r(B, Tq, Hq, 128), r(B, Lloc, Hkv, 128), r(B, Lloc, Hkv, 128), r(B, M, Hkv, 128), \
         r(B, M, Hkv, 128)
