@@ -764,6 +764,9 @@ EXTRA_STEPS = {"decode16m": 30, "stack10m": 8, "1m": 30}
 DGA_HEADS = (16, 32)  # key heads, value heads of the linear layers (d = 128); the pages give no head counts
 
 
+GDR_TOKEN_MAX = 16  # msa_gated_delta_rule takes its token-by-token kernel up to this many query tokens
+
+
 def run_dga(args, rank, local_rank, world):
     """The linear (DGA) layers' memory path for the workload's queries: per step, the sum of each
     query's k selected documents' recurrent states (msa_state_gather_sum, S_ext) and the gated delta
@@ -847,7 +850,8 @@ def run_dga(args, rank, local_rank, world):
                            f"query tokens x {B} queries ({Hk} key heads, {Hv} value heads, d = {d})",
                    "l2": "flushed before every step", "parallelism": "single GPU"},
         "roofline": {"bound": "alu", "achieved": round(flops / per / 1e9, 2), "peak": round(peak, 1),
-                     "unit": "TFLOP/s", "kernel": "gdr_chunk_kernel (msa_gated_delta_rule)",
+                     "unit": "TFLOP/s",
+                     "kernel": ("gdr_token_kernel" if T <= GDR_TOKEN_MAX else "gdr_chunk_kernel") + " (msa_gated_delta_rule)",
                      "alg_flops_per_launch": flops,
                      "peak_source": "derived: SMs x 128 fp32 lanes x 2 x max SM clock",
                      "frac": round(flops / per / 1e9 / peak, 4), "avg_launch_ms": round(per, 4), "traffic": None},
