@@ -115,7 +115,9 @@ __device__ __forceinline__ int64_t warp_owner_doc(const int64_t* __restrict__ of
 // a document in [0, D) whatever the offsets hold.
 __device__ __forceinline__ int64_t warp_owner_doc_near(const int64_t* __restrict__ off, int64_t D, int64_t C,
                                                        int64_t c, int lane) {
-  int64_t g = (C > 0 ? (int64_t)((double)c * (double)D / (double)C) : 0) - 16;
+  // a guess only (a miss falls back to the full search): fp32 keeps it within a
+  // document for D up to ~2^24, without a double-precision division
+  int64_t g = (C > 0 ? (int64_t)((float)c * ((float)D / (float)C)) : 0) - 16;
   if (g > D - 32) g = D - 32;
   if (g < 0) g = 0;
   const int64_t j = g + lane;
@@ -131,7 +133,9 @@ __device__ __forceinline__ int64_t warp_owner_doc_near(const int64_t* __restrict
 // Owning document of chunk c0 + lane for the 32 consecutive chunks of a warp
 // (-1 for chunks >= C).  One warp-wide search for c0, then each lane counts the
 // document boundaries at or below its chunk among the next 32 (documents with no
-// chunks are boundaries too); falls back to a per-lane search when 32
+// chunks are boundaries too) by a binary search over the lanes' boundaries,
+// which valid offsets leave sorted (invalid ones give some count in [0, 32],
+// never an index outside the window); falls back to a per-lane search when 32
 // boundaries do not cover the warp's chunks.  All 32 lanes must call it.
 __device__ __forceinline__ int warp_chunk_docs(const int64_t* __restrict__ off, int64_t D, int64_t C, int64_t c0,
                                                int lane) {
@@ -140,9 +144,14 @@ __device__ __forceinline__ int warp_chunk_docs(const int64_t* __restrict__ off, 
   const int64_t c = c0 + lane;
   const int64_t bidx = j0 + 1 + lane;
   const int64_t b = __ldg(off + (bidx < D ? bidx : D));
-  int cnt = 0;
+  // boundary l relative to c0, clamped to [0, 32]: a 32-bit sorted list
+  const int64_t rb = b - c0;
+  const int r = rb < 0 ? 0 : (rb > 32 ? 32 : (int)rb);
+  int cnt = 0;  // boundaries r_l <= lane
 #pragma unroll
-  for (int l = 0; l < 32; ++l) cnt += __shfl_sync(0xffffffffu, b, l) <= c ? 1 : 0;
+  for (int step = 16; step > 0; step >>= 1)
+    if (__shfl_sync(0xffffffffu, r, cnt + step - 1) <= lane) cnt += step;
+  if (__shfl_sync(0xffffffffu, r, cnt & 31) <= lane && cnt == 31) cnt = 32;
   const int64_t b31 = __shfl_sync(0xffffffffu, b, 31);
   const bool covered = b31 > c0 + 31 || j0 + 32 >= D;
   if (c >= C) return -1;

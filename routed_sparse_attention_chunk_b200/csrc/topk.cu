@@ -7,18 +7,22 @@
 // so that one unsigned comparison orders by score descending and, for equal
 // scores, by lower document index first; padding is key 0, below every real key.
 //
-// One launch, grid (slices, B).  A slice of up to 8192 documents is held in
-// registers, 32 keys per thread.  The threshold tau is the k-th largest of the
-// 256 per-thread maxima: the k largest keys of the slice are all >= tau (k
-// distinct thread maxima already are), and only the k threads whose maximum
-// passes hold keys >= tau, so at most 32 k keys survive.  For k <= 32 the work
-// stays in warps: each warp sorts its 32 maxima across lanes with shuffles,
-// warp 0 merges the eight sorted lists (bitonic top-32 merges) to find tau, and
-// up to 32 survivors are sorted in one warp's registers; larger k or more
-// survivors take shared-memory bitonic sorts (and more than 2048 survivors,
-// which needs k > 64, a block sort streamed over the slice).  The slice's
-// top-k goes to the workspace; the last CTA of the row to finish (an atomic
-// counter, no waiting) merges the slices' sorted lists and writes the result.
+// One launch, grid (slices, B), 256 threads.  A slice of up to 8192 documents
+// is held in registers, 32 keys per thread.  The threshold tau is the k-th
+// largest of the 256 per-thread maxima: the k largest keys of the slice are all
+// >= tau (k distinct thread maxima already are), and only the k threads whose
+// maximum passes hold keys >= tau, so at most 32 k keys survive.  For k <= 32:
+// each warp sorts its 32 maxima across lanes with shuffles and the eight sorted
+// lists merge pairwise in three rounds (bitonic top-32 merges, half the warps
+// per round) to give tau; larger k sorts the 256 maxima in shared memory.  The
+// survivors are placed by a block-wide prefix sum of the threads' counts (one
+// scan instead of a ballot and a shared atomic per key position); up to 32 are
+// sorted in one warp's registers, more by a shared-memory bitonic sort, and
+// more than 2048 (which needs k > 64) fall back to a block sort streamed over
+// the slice.  With several slices, each slice's top-k goes to the workspace and
+// the last CTA of the row to finish (an atomic counter, no waiting) merges the
+// sorted lists.  (1024 threads and slices of 32768, one CTA per query of a 16M-
+// token bank with no merge, ran slower: 64 busy SMs and register spills.)
 // The top-k of a union is contained in the union of the parts' top-k, so the
 // result is exact.
 #include "common.cuh"
@@ -107,63 +111,91 @@ __device__ __forceinline__ uint64_t warp_merge_top(uint64_t a, uint64_t b, int l
 }
 
 // Top-k of keys row[lo, lo + n), n <= kSlice, left sorted in s[0, k); false
-// when more than kSortN keys pass the filter (s is then clobbered).
-__device__ bool slice_topk_filter(uint64_t* s, int* cnt, uint64_t* tau_s, const uint32_t* row, int64_t lo,
-                                  int64_t n, int k) {
+// when more than kSortN keys pass the filter (s is then clobbered).  wsum holds
+// kSortThreads / 32 ints.
+__device__ bool slice_topk_filter(uint64_t* s, int* wsum, const uint32_t* row, int64_t lo, int64_t n, int k) {
+  constexpr int kWarps = kSortThreads / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // n <= kSlice: 32-bit indices; a key keeps only the low 32 bits of its document
+  const int nn = (int)n;
+  const uint32_t lo32 = (uint32_t)lo;
+  auto key_of = [&](uint32_t sk, int i) -> uint64_t {
+    return ((uint64_t)sk << 32) | (uint64_t)(0xffffffffu - (lo32 + (uint32_t)i));
+  };
   // all 32 keys of this thread in registers from one round of loads
   uint32_t v[kPer];
 #pragma unroll
   for (int m = 0; m < kPer; ++m) {
-    const int64_t i = tid + (int64_t)m * kSortThreads;
-    v[m] = i < n ? __ldg(row + lo + i) : 0u;
+    const int i = tid + m * kSortThreads;
+    v[m] = i < nn ? __ldg(row + lo + i) : 0u;
   }
   uint64_t mx = 0ull;
 #pragma unroll
   for (int m = 0; m < kPer; ++m) {
-    const int64_t i = tid + (int64_t)m * kSortThreads;
-    if (i < n) mx = max(mx, doc_key64(v[m], lo + i));
+    const int i = tid + m * kSortThreads;
+    if (i < nn) mx = max(mx, key_of(v[m], i));
   }
-  // tau = the k-th largest of the 256 thread maxima
+  // tau = the k-th largest of the thread maxima
   uint64_t tau;
   if (k <= 32) {
-    // each warp sorts its maxima; warp 0 merges the eight sorted lists
-    s[tid] = warp_sort_desc(mx, lane);
-    if (tid == 0) *cnt = 0;
+    // each warp sorts its maxima; the sorted lists merge pairwise, half the warps a round
+    uint64_t x = warp_sort_desc(mx, lane);
+    s[tid] = x;
     __syncthreads();
-    if (warp == 0) {
-      uint64_t m = s[lane];
-      for (int w = 1; w < kSortThreads / 32; ++w) m = warp_merge_top(m, s[w * 32 + lane], lane);
-      const uint64_t t = __shfl_sync(0xffffffffu, m, k - 1);
-      if (lane == 0) *tau_s = t;
+#pragma unroll
+    for (int half = kWarps / 2; half >= 1; half >>= 1) {
+      if (warp < half) x = warp_merge_top(x, s[(warp + half) * 32 + lane], lane);
+      __syncthreads();
+      if (warp < half) s[tid] = x;
+      __syncthreads();
     }
-    __syncthreads();
-    tau = *tau_s;
+    tau = s[k - 1];
   } else {
     s[tid] = mx;
-    if (tid == 0) *cnt = 0;
     __syncthreads();
     bitonic_desc(s, kSortThreads);
     tau = s[k - 1];
-    __syncthreads();
   }
-  // keep the keys >= tau (the k thread maxima and what else their threads hold)
+  // keep the keys >= tau (the k thread maxima and what else their threads hold):
+  // each thread counts its own, a block-wide exclusive prefix of the counts
+  // gives where it writes them
+  int c = 0;
 #pragma unroll
   for (int m = 0; m < kPer; ++m) {
-    const int64_t i = tid + (int64_t)m * kSortThreads;
-    const uint64_t key = i < n ? doc_key64(v[m], lo + i) : 0ull;
-    const bool pass = i < n && key >= tau;
-    const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-    if (bal) {
-      int base = 0;
-      if (lane == 0) base = atomicAdd(cnt, __popc(bal));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      const int pos = base + __popc(bal & ((1u << lane) - 1u));
-      if (pass && pos < kSortN) s[pos] = key;
+    const int i = tid + m * kSortThreads;
+    c += (i < nn && key_of(v[m], i) >= tau) ? 1 : 0;
+  }
+  int inc = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();  // every thread has read tau from s, so s may be overwritten below
+  int before = 0, total = 0;
+  {
+    const int w = lane < kWarps ? wsum[lane] : 0;
+    int winc = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, winc, o);
+      if (lane >= o) winc += t;
+    }
+    before = __shfl_sync(0xffffffffu, winc - w, warp & 31);
+    total = __shfl_sync(0xffffffffu, winc, 31);
+  }
+  int pos = before + inc - c;
+#pragma unroll
+  for (int m = 0; m < kPer; ++m) {
+    const int i = tid + m * kSortThreads;
+    const uint64_t key = key_of(v[m], i);
+    if (i < nn && key >= tau) {
+      if (pos < kSortN) s[pos] = key;
+      ++pos;
     }
   }
   __syncthreads();
-  const int total = *cnt;
   if (total > kSortN) return false;
   if (total <= 32) {  // one warp sorts the survivors in registers
     if (warp == 0) {
@@ -184,8 +216,8 @@ __global__ void __launch_bounds__(kSortThreads)
 topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, uint64_t* cand,
             uint32_t* counters, int32_t* __restrict__ out_idx, float* __restrict__ out_score, int out_ld) {
   __shared__ uint64_t s[kSortN];
-  __shared__ uint64_t tau_s;
-  __shared__ int last, cnt;
+  __shared__ int wsum[kSortThreads / 32];
+  __shared__ int last;
   pdl_wait();  // the scan's keys (launched as a programmatic dependent of it)
   const int64_t b = blockIdx.y;
   const int slice = blockIdx.x;
@@ -194,7 +226,7 @@ topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, 
   const int64_t n = max((int64_t)0, min(D, lo + per) - lo);
   const uint32_t* row = doc_key + b * D;
   // (the branch is uniform over the CTA)
-  if (n > kSlice || !slice_topk_filter(s, &cnt, &tau_s, row, lo, n, k)) {
+  if (n > kSlice || !slice_topk_filter(s, wsum, row, lo, n, k)) {
     __syncthreads();
     block_topk(s, n, k, [&](int64_t i) -> uint64_t { return doc_key64(__ldg(row + lo + i), lo + i); });
   }

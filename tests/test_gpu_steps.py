@@ -132,6 +132,7 @@ def _bank_case(C_docs, Hr, dr, seed):
     (4, 2, 8, 128, 20000, 32),    # largest k of the warp-level top-k, three slices merged
     (3, 3, 8, 128, 17000, 33),    # smallest k of the block-level top-k, three slices
     (2, 5, 2, 64, 9000, 1),       # k = 1 over two slices
+    (64, 1, 2, 64, 32768, 16),    # four whole slices per query (256 threads x 32 documents each)
     (1, 4, 2, 64, 20, 20),        # fewer documents than a warp, k = D
     (1, 512, 8, 128, 9000, 16),   # ~40K chunks, 4 blocks of 128 query rows
     (2, 300, 1, 128, 9000, 16),   # blocks that span two queries, ragged last block
@@ -185,13 +186,15 @@ def test_topk_many_slices_merge():
 
 
 def test_topk_filter_overflow_takes_streaming_path():
-    # k = 100 over one slice of 32768 one-chunk documents.  The documents held
-    # by the first 100 threads of the filter (index mod 1024 < 100) all score
-    # high and rise with (thread, item), so several thousand keys pass the
-    # threshold and the slice falls back to the streamed block sort.
-    D, k, dr = 32768, 100, 64
+    # k = 100 over four slices of 8192 one-chunk documents; in a slice the
+    # filter's 256 threads hold 32 documents each (document i of the slice is
+    # item i // 256 of thread i % 256).  In every slice the documents of threads
+    # 0..99 score high and rise with (thread, item), so several thousand keys
+    # pass the threshold and each slice falls back to the streamed block sort.
+    D, k, dr, S, T = 4 * 8192, 100, 64, 8192, 256
     idx_all = np.arange(D)
-    t, m = idx_all % 1024, idx_all // 1024
+    local = idx_all % S
+    t, m = local % T, local // T
     heavy = t < k
     a = np.where(heavy, 1.0 + (t * 32 + m) / 4096.0, -1.0)
     bank = np.zeros((D, 1, dr), dtype=np.float32)
@@ -209,14 +212,16 @@ def test_topk_filter_overflow_takes_streaming_path():
     oi, _ = O.topk(ods, k)
     torch.cuda.synchronize()
     assert flag.item() == 0
-    # the filter's survivor count, from the oracle's scores: keys >= the k-th
+    # each slice's survivor count, from the oracle's scores: keys >= the k-th
     # largest per-thread maximum, keys ordered by (score, lower index)
-    order = np.lexsort((idx_all, -ods[0]))             # rank 0 = largest key
-    rank = np.empty(D, dtype=np.int64)
-    rank[order] = np.arange(D)
-    thread_best = np.array([rank[t == i].min() for i in range(1024)])
-    tau_rank = np.sort(thread_best)[k - 1]
-    assert int((rank <= tau_rank).sum()) > 2048
+    for sl in range(D // S):
+        sc_sl, ix_sl, t_sl = ods[0, sl * S:(sl + 1) * S], idx_all[sl * S:(sl + 1) * S], t[sl * S:(sl + 1) * S]
+        order = np.lexsort((ix_sl, -sc_sl))            # rank 0 = largest key
+        rank = np.empty(S, dtype=np.int64)
+        rank[order] = np.arange(S)
+        thread_best = np.array([rank[t_sl == i].min() for i in range(T)])
+        tau_rank = np.sort(thread_best)[k - 1]
+        assert int((rank <= tau_rank).sum()) > 2048
     assert np.array_equal(idx.cpu().numpy(), oi)
 
 
