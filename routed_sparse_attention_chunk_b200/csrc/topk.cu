@@ -241,14 +241,30 @@ topk_kernel(const uint32_t* __restrict__ doc_key, int64_t D, int k, int nslice, 
     __threadfence();
     const uint64_t* c = cand + b * nslice * k;
     if (k <= 32) {
-      // every slice's list is sorted: warp 0 merges them pairwise in registers
-      if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        uint64_t m = lane < k ? __ldcg(c + lane) : 0ull;
-        for (int sl = 1; sl < nslice; ++sl) m = warp_merge_top(m, lane < k ? __ldcg(c + sl * k + lane) : 0ull, lane);
-        s[lane] = m;
+      // every slice's list is sorted: the lists merge pairwise in rounds (half of them a
+      // round, one warp per pair), up to kSortN / 32 lists at a time in shared memory
+      constexpr int kLists = kSortN / 32;
+      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+      int have = 0, held = 0;  // slices merged so far; 1 once s[0, 32) holds their top list
+      while (have < nslice) {
+        const int take = min(nslice - have, kLists - held);
+        for (int i = threadIdx.x; i < take * 32; i += kSortThreads) {
+          const int l = i >> 5, e = i & 31;
+          s[(held + l) * 32 + e] = e < k ? __ldcg(c + (int64_t)(have + l) * k + e) : 0ull;
+        }
+        __syncthreads();
+        for (int L = held + take; L > 1;) {
+          const int half = (L + 1) >> 1;
+          // pairs (w, w + half); with L odd the middle list waits a round.  A warp writes only
+          // list w < half, which no other warp of the round reads.
+          for (int w = warp; w < L - half; w += kSortThreads / 32)
+            s[w * 32 + lane] = warp_merge_top(s[w * 32 + lane], s[(w + half) * 32 + lane], lane);
+          __syncthreads();
+          L = half;
+        }
+        have += take;
+        held = 1;
       }
-      __syncthreads();
     } else {
       block_topk(s, (int64_t)nslice * k, k, [&](int64_t i) -> uint64_t { return __ldcg(c + i); });
     }

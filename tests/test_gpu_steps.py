@@ -185,6 +185,23 @@ def test_topk_many_slices_merge():
     check_topk(idx.cpu().numpy(), to64(sc), ods, 16, TOL_SCORE_ABS)
 
 
+def test_topk_more_slices_than_one_merge_round():
+    # 600,000 one-chunk documents: 74 slices of 8192, more lists than the last CTA
+    # merges at once in shared memory (64), so the merge runs in two batches
+    D, k = 600000, 16
+    g = torch.Generator(device=DEV).manual_seed(31)
+    Krb = (torch.randn((D, 1, 64), generator=g, device=DEV)).bfloat16()
+    rn = torch.empty((D, 1), dtype=torch.float32, device=DEV)
+    msa.bank_rnorm(Krb, rn)
+    coff = np.arange(D + 1, dtype=np.int64)
+    Qr = torch.randn((1, 1, 1, 64), generator=g, device=DEV).bfloat16()
+    idx, sc, ds, flag = route_on_gpu(Qr, Krb, rn, coff, k)
+    ods = O.route(to64(Qr), to64(Krb), coff)
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    check_topk(idx.cpu().numpy(), to64(sc), ods, k, TOL_SCORE_ABS)
+
+
 def test_topk_filter_overflow_takes_streaming_path():
     # k = 100 over four slices of 8192 one-chunk documents; in a slice the
     # filter's 256 threads hold 32 documents each (document i of the slice is
