@@ -14,31 +14,37 @@
 //     is rounded to bf16 and written back over its own S tile in TMEM (two
 //     values per 32-bit column, one row per lane), and O += P V takes P as the
 //     MMA's A operand straight from tensor memory and V MN-major from its TMA
-//     tile.  The tensor core runs its MMAs in issue order, so S_{j+2} (issued
-//     after PV_j) never overwrites P_j before PV_j has read it;
+//     tile.  S and PV have their own issuing threads: PV_j waits only for P_j,
+//     and S_{j+2} waits for PV_j's commit before it overwrites P_j's buffer;
 //   * key tile j's K and V share one of three stages and one barrier, so the
 //     MMA warp waits once per tile for both operands (each of its waits costs
 //     ~100-200 cycles on the critical path; separate K and V barriers made the
 //     dense-memory kernel 2.4% slower); the stage is released when PV_j is done;
-//   * S = Q K^T runs at N = 128, where one CTA's tensor core does a
-//     128 x 128 x 128 product in ~705 cycles with B K-major and ~853 with B
-//     MN-major (V), against 512 at N = 256 (a clock64 probe of back-to-back
-//     MMAs); a CTA pair (cta_group::2, M = 256, each CTA half of B) takes ~947,
-//     so the pair's halved tile loads did not pay: it ran 2-5% slower than one
-//     CTA.  An N = 256 S tile would need 2 x 256 TMEM columns for S alone;
+//   * a tile's MMAs (S and PV, 128 x 128 x 128 each) run at the tensor core's
+//     full rate in isolation (~513 cycles each, B K-major or MN-major; a
+//     clock64 probe of back-to-back MMAs), but the issuing thread cannot queue
+//     ahead of them: issuing a group of 8 blocks about as long as it runs, and
+//     each hand-off through a barrier costs a few hundred cycles.  Inside this
+//     kernel PV's MMAs enter every ~79 cycles and S's every ~65; with one
+//     issuer its chain per tile (issue S_{j+1}, wait for P_j, issue PV_j, wait
+//     for K_{j+2}) was ~2,000 cycles, so S and PV now have one issuer each
+//     (1% faster: the softmax's own ~1,800-cycle chain paces the tile next).
+//     Tried and slower:
+//     CTA pairs (cta_group::2, M = 256, each CTA half of every K and V tile),
+//     P in its own TMEM columns so that PV_j goes before S_{j+2}, two softmax
+//     warpgroups splitting the keys;
 //   * the running max is only moved (and O rescaled in TMEM) when it grows by
 //     more than 2^8, so most tiles skip the rescale; the final 1/l and the
 //     log-sum-exp use the same max, which keeps the result exact;
-//   * a tile's pace is set by the MMA warp's serial chain (issue S_{j+1}, wait
-//     for P_j, issue PV_j; the tensor core takes in a group of MMAs about as
-//     fast as it runs them) and by the softmax warps (one per SM
-//     sub-partition): the row max runs as eight independent chains of
-//     three-input maxima, the scaled arguments and row sums use packed f32x2
-//     math, four of every sixteen key pairs take a polynomial 2^x on the FMA
-//     pipe instead of the transcendental unit (1-2% faster; eight of sixteen
-//     was slower), and the MMA warp reuses its operand descriptors.
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2..5 softmax / correction / output (one row per thread).
+//   * the softmax warps (one per SM sub-partition): the row max runs as eight
+//     independent chains of three-input maxima, the scaled arguments and row
+//     sums use packed f32x2 math, four of every sixteen key pairs take a
+//     polynomial 2^x on the FMA pipe instead of the transcendental unit (1-2%
+//     faster; eight of sixteen was slower), and the MMA warp reuses its
+//     operand descriptors.
+// Warp roles (224 threads): warp 0 TMA producer, warp 1 TMEM owner + S MMA
+// issuer, warps 2..5 softmax / correction / output (one row per thread),
+// warp 6 PV MMA issuer.
 // Every wait is bounded and ends the CTA with MSA_FLAG_TIMEOUT on expiry.
 #include <atomic>
 
@@ -54,7 +60,7 @@ using namespace sm100;
 
 constexpr int kRows = 128;   // MMA M: query rows per CTA
 constexpr int kKeys = 128;   // keys per tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;  // producer, S issuer, four softmax warps, PV issuer
 constexpr uint32_t kWaitPolls = 1u << 24;
 constexpr float kRescaleLog2 = 8.0f;  // move the running max only when it grows by more than this
 constexpr int kKV = 3;                // K + V stages
@@ -173,7 +179,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint64_t* p_free = p_full + 2;           // [2] PV MMA done -> softmax (O up to date)
   uint64_t* drain = p_free + 2;
   uint64_t* q_tmem = drain + 1;            // Q copied into tensor memory (softmax threads) -> MMA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_tmem + 1);
+  uint64_t* drain_pv = q_tmem + 1;         // the PV issuer's own drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_pv + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // longest blocks first: block index 0 takes the last query block
@@ -198,6 +205,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     mbar_init(drain, 1);
     mbar_init(q_tmem, 128);
+    mbar_init(drain_pv, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -305,16 +313,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+    // ---------------------------------------------------------------- S MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(kRows, kKeys);
-      constexpr uint32_t idO = idesc_bf16_f32(kRows, DH, /*b_mn_major=*/true);
       // descriptors of the operand bases; a k-step adds its byte offset / 16 to
       // the 14-bit start-address field (shared addresses stay below 256 KB, so
       // the field never carries)
-      const uint64_t dk0 = desc_k_sw128(smem_u32(Ks)), dv0 = desc_mn_sw128(smem_u32(Vs), kKeys * 128);
-      // S_j goes to TMEM buffer j & 1, which holds P_{j-2} until PV_{j-2} has
-      // read it; PV_{j-2} was issued earlier, and the MMAs run in issue order.
+      const uint64_t dk0 = desc_k_sw128(smem_u32(Ks));
       auto issue_S = [&](int j) -> bool {
         const int ks = j % kKV;
         if (!mbar_wait(&kv_full[ks], (j / kKV) & 1, p.polls)) return false;
@@ -330,16 +335,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mma_commit(&s_full[j & 1]);
         return true;
       };
-      // the S MMAs read Q from tensor memory once the softmax threads have put it there
-      bool ok = mbar_wait(q_tmem, 0, p.polls) && issue_S(0);
+      // the S MMAs read Q from tensor memory once the softmax threads have put it there; S_j
+      // (j >= 2) goes into buffer j & 1 once PV_{j-2} has read P_{j-2} from it (PV is issued
+      // by another thread, so the order comes from PV_{j-2}'s commit)
+      bool ok = mbar_wait(q_tmem, 0, p.polls);
       for (int j = 0; ok && j < T; ++j) {
-        const int st = j & 1, vs = j % kKV;
-        if (j + 1 < T && !issue_S(j + 1)) {
+        if (j >= 2 && !mbar_wait(&p_free[j & 1], ((j - 2) >> 1) & 1, p.polls)) {
           ok = false;
           break;
         }
-        // V_j landed with K_j (S_j waited for both)
-        if (!mbar_wait(&p_full[st], (j >> 1) & 1, p.polls)) {
+        if (!issue_S(j)) {
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) timed_out = true;
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0, kWaitPolls)) timed_out = true;
+    }
+  } else if (warp == 6) {
+    // ---------------------------------------------------------------- PV issuer
+    if (lane == 0) {
+      constexpr uint32_t idO = idesc_bf16_f32(kRows, DH, /*b_mn_major=*/true);
+      const uint64_t dv0 = desc_mn_sw128(smem_u32(Vs), kKeys * 128);
+      bool ok = true;
+      for (int j = 0; ok && j < T; ++j) {
+        const int st = j & 1, vs = j % kKV;
+        // P_j written over S_j; V_j landed with K_j
+        if (!mbar_wait(&p_full[st], (j >> 1) & 1, p.polls) || !mbar_wait(&kv_full[vs], (j / kKV) & 1, p.polls)) {
           ok = false;
           break;
         }
@@ -354,8 +377,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mma_commit(&kv_empty[vs]);
       }
       if (!ok) timed_out = true;
-      mma_commit(drain);
-      if (!mbar_wait(drain, 0, kWaitPolls)) timed_out = true;
+      mma_commit(drain_pv);
+      if (!mbar_wait(drain_pv, 0, kWaitPolls)) timed_out = true;
     }
   } else {
     // ---------------------------------------------------------------- softmax
