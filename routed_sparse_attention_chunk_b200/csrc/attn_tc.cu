@@ -28,7 +28,9 @@
 //     kernel PV's MMAs enter every ~79 cycles and S's every ~65; with one
 //     issuer its chain per tile (issue S_{j+1}, wait for P_j, issue PV_j, wait
 //     for K_{j+2}) was ~2,000 cycles, so S and PV now have one issuer each
-//     (1% faster: the softmax's own ~1,800-cycle chain paces the tile next).
+//     (1% faster); the softmax warps' chain (S load, row max, exponentials,
+//     P stores: ~1,975 cycles a tile) now paces the tile, both issuers idle
+//     about half of it.
 //     Tried and slower:
 //     CTA pairs (cta_group::2, M = 256, each CTA half of every K and V tile),
 //     P in its own TMEM columns so that PV_j goes before S_{j+2}, two softmax
