@@ -40,10 +40,10 @@
 //     log-sum-exp use the same max, which keeps the result exact;
 //   * the softmax warps (one per SM sub-partition): the row max runs as eight
 //     independent chains of three-input maxima, the scaled arguments and row
-//     sums use packed f32x2 math, four of every sixteen key pairs take a
-//     polynomial 2^x on the FMA pipe instead of the transcendental unit (1-2%
-//     faster; eight of sixteen was slower), and the MMA warp reuses its
-//     operand descriptors.
+//     sums use packed f32x2 math, six of every sixteen key pairs take a
+//     polynomial 2^x on the FMA pipe instead of the transcendental unit (2-3%
+//     faster than none; eight of sixteen was no better), and the MMA warps
+//     reuse their operand descriptors.
 // Warp roles (224 threads): warp 0 TMA producer, warp 1 TMEM owner + S MMA
 // issuer, warps 2..5 softmax / correction / output (one row per thread),
 // warp 6 PV MMA issuer.
@@ -158,7 +158,7 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float&
 
 // Of each 16 key pairs of a 32-key store, this many take exp2_poly2 (spread
 // evenly); the rest take the transcendental unit's ex2.
-constexpr int kPolyPairs = 4;
+constexpr int kPolyPairs = 6;
 __host__ __device__ constexpr bool poly_pair(int i) { return (i * kPolyPairs) / 16 != ((i + 1) * kPolyPairs) / 16; }
 
 template <int DH>
