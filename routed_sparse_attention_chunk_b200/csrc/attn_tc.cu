@@ -16,9 +16,8 @@
 //     MMA's A operand straight from tensor memory and V MN-major from its TMA
 //     tile.  S and PV have their own issuing threads: PV_j waits only for P_j,
 //     and S_{j+2} waits for PV_j's commit before it overwrites P_j's buffer;
-//   * key tile j's K and V share one of three stages and one barrier, so the
-//     MMA warp waits once per tile for both operands (each of its waits costs
-//     ~100-200 cycles on the critical path; separate K and V barriers made the
+//   * key tile j's K and V share one of three stages and one barrier (one
+//     wait per tile for both operands; separate K and V barriers made the
 //     dense-memory kernel 2.4% slower); the stage is released when PV_j is done;
 //   * a tile's MMAs (S and PV, 128 x 128 x 128 each) run at the tensor core's
 //     full rate in isolation (~513 cycles each, B K-major or MN-major; a
@@ -29,12 +28,11 @@
 //     issuer its chain per tile (issue S_{j+1}, wait for P_j, issue PV_j, wait
 //     for K_{j+2}) was ~2,000 cycles, so S and PV now have one issuer each
 //     (1% faster); the softmax warps' chain (S load, row max, exponentials,
-//     P stores: ~1,975 cycles a tile) now paces the tile, both issuers idle
-//     about half of it.
-//     Tried and slower:
-//     CTA pairs (cta_group::2, M = 256, each CTA half of every K and V tile),
-//     P in its own TMEM columns so that PV_j goes before S_{j+2}, two softmax
-//     warpgroups splitting the keys;
+//     P stores: ~1,975 cycles a tile) now paces the tile, and both issuers
+//     idle about half of it.  Tried and slower: CTA pairs (cta_group::2,
+//     M = 256, each CTA half of every K and V tile), P in its own TMEM columns
+//     so that PV_j goes before S_{j+2}, two softmax warpgroups splitting the
+//     keys;
 //   * the running max is only moved (and O rescaled in TMEM) when it grows by
 //     more than 2^8, so most tiles skip the rescale; the final 1/l and the
 //     log-sum-exp use the same max, which keeps the result exact;
