@@ -70,7 +70,7 @@ typedef struct CUstream_st* msa_stream_t; /* the same type as cudaStream_t */
 typedef enum {
   MSA_OK = 0,
   MSA_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned pointer */
-  MSA_ERR_UNSUPPORTED = -2, /* a shape or dtype this build has no kernel for */
+  MSA_ERR_UNSUPPORTED = -2, /* a shape or dtype the library has no kernel for */
   MSA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than *_workspace_size */
   MSA_ERR_CUDA = -4,        /* a CUDA launch or runtime call failed */
   MSA_ERR_TOO_LARGE = -5,   /* the problem needs more scratch than msa_route_topk_noalloc holds */
