@@ -73,3 +73,23 @@ def test_traffic_records_are_well_formed():
         got = bench.traffic_record(kernel_file, workload)
         assert got is None or got["dram_bytes_per_launch"] == r["dram_bytes_per_launch"]
     assert bench.traffic_record("pool.cu", "no-such-workload") is None
+
+
+def test_reference_arm_prints_the_contract_line():
+    # the oracle arm on a bounded sample of the 1M workload: one JSON line with the
+    # same metric and unit as the GPU arm, tagged impl=reference, e2e without copies
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "1m",
+                          "--steps", "1", "--warmup", "0", "--ref-budget", "1"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    r = json.loads(lines[0])
+    assert r["impl"] == "reference" and r["metric"] == bench.METRIC and r["unit"] == bench.UNIT
+    assert r["higher_is_better"] is True and r["steps"] == 1 and r["value"] > 0
+    assert r["config"]["workload"].startswith("1m")
+    cb = r["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == r["value"] and cb["sample"]
+    assert r["e2e"] == {"value": r["value"], "unit": r["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
