@@ -396,6 +396,7 @@ struct PairLayout {
   static constexpr int kStage = kA + kB;
   static constexpr int kStages = (192 * 1024) / kStage > 6 ? 6 : (192 * 1024) / kStage;
   static constexpr int kNH = kN / 2;                      // columns per epilogue warpgroup
+  static_assert(kNH % 64 == 0, "the epilogue reads its columns 64 at a time and frees the accumulator after the last 64");
   static constexpr int kRq = 8 * 8 * kNH * 4;             // per epilogue warp: rq of its columns, Hr <= 8
   static constexpr int kBar = 8 * (2 * kStages + 2 * 2 + 1) + 16;
   static constexpr int kSmem = 1024 + kStages * kStage + kRq + kBar;
@@ -608,6 +609,13 @@ route_tc_pair_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < 64; c += 16) tmem_regs_ready(*reinterpret_cast<float(*)[16]>(&v[c]));
+          if (j0 + 64 == NH) {
+            // the whole accumulator is in registers: the leader's MMA may reuse it
+            // while this half's products are summed
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acce0 + 8u * buf);
+          }
 #pragma unroll
           for (int j4 = 0; j4 < 64; j4 += 4) {
             const float4 w = *reinterpret_cast<const float4*>(rqh + j0 + j4);
@@ -621,9 +629,6 @@ route_tc_pair_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             S_[j0 + j4 + 3] = fmaf(v[j4 + 3], k3, S_[j0 + j4 + 3]);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(acce0 + 8u * buf);  // the leader's MMA may reuse it
       }
       if (timed_out) break;
       if (nvalid == 0) continue;
