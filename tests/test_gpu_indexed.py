@@ -81,6 +81,8 @@ def _oracle(Q, Kl, Vl, idx, coff, Kb, Vb, Mmax, D):
     (2, 16, 48, 8, 8, 7, 64, 5),          # prefill MHA (G = 1: 8-token blocks)
     (3, 24, 90, 32, 8, 11, 256, 6),       # one ragged block of rows per KV head, two memory tiles
     (1, 160, 160, 64, 8, 16, 512, 7),     # G = 8: ten 16-token blocks, four memory tiles
+    (2, 60, 120, 40, 8, 10, 200, 8),      # G = 5: no tensor-core tiling, the gathered path (no overflow)
+    (2, 8, 300, 32, 8, 12, 256, 9),       # 8 tokens x G = 4: neither a prefill block nor decode rows
 ])
 def test_indexed_attention_ragged_documents(B, Tq, Lloc, Hq, Hkv, k, Mmax, seed):
     rng = np.random.default_rng(seed)

@@ -389,6 +389,24 @@ def test_attention_bf16_decode_shapes(B, Tq, Lloc, Hq, Hkv, Mmax, mem_lens):
     close_abs(to64(lse), olse, 2e-3, "lse")
 
 
+@pytest.mark.parametrize("B,Tq,Lloc,Hq,Hkv,Mmax,mem_lens,dtype", [
+    (2, 8, 300, 32, 8, 128, [128, 40], torch.bfloat16),      # 8 tokens x G=4: too few for a tensor-core block, too many rows to decode
+    (1, 70, 150, 40, 8, 64, [50], torch.bfloat16),           # G=5 does not divide a block of 128 rows
+    (3, 1, 500, 40, 8, 128, [128, 0, 60], torch.bfloat16),   # G=5 decode: 5 real rows of the 8-row kernel
+    (2, 40, 100, 32, 1, 32, [32, 7], torch.bfloat16),        # G=32: 4 tokens per block, under the tensor-core minimum
+    (1, 50, 90, 8, 2, 40, [40], torch.float32),              # fp32 at d = 128
+])
+def test_attention_shapes_outside_the_tensor_core_tiles(B, Tq, Lloc, Hq, Hkv, Mmax, mem_lens, dtype):
+    Q, Kl, Vl, Km, Vm, ml = _attn_inputs(B, Tq, Lloc, Hq, Hkv, 128, Mmax, mem_lens, dtype, 6)
+    Og, lse, flag = attn_on_gpu(Q, Kl, Vl, Km, Vm, ml)
+    Oo, olse = O.attention(to64(Q), to64(Kl), to64(Vl), to64(Km), to64(Vm), mem_lens)
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    tol = TOL_F32_ATTN if dtype == torch.float32 else TOL_BF16_ABS
+    close_abs(to64(Og), Oo, tol, "O")
+    close_abs(to64(lse), olse, TOL_F32_ATTN if dtype == torch.float32 else 2e-3, "lse")
+
+
 def test_attention_bad_mem_len_is_flagged_not_faulted():
     Q, Kl, Vl, Km, Vm, ml = _attn_inputs(1, 4, 4, 2, 1, 64, 8, [9999], torch.bfloat16, 3)
     Og, lse, flag = attn_on_gpu(Q, Kl, Vl, Km, Vm, ml)
