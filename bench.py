@@ -863,6 +863,114 @@ def run_dga(args, rank, local_rank, world):
     }
 
 
+def interleave_roofline(cfg: synth.Config, counts: dict, rounds: int, ms: float, peaks: dict, peak_kind: str,
+                        long_region: bool) -> dict:
+    """Roofline of one msa_interleave_forward call, taken against its `rounds` routing scans of the bank
+    (the dominant work): the call is one C-ABI launch sequence, so the attention rounds and the
+    router-query projections run inside the same time and the figure is a lower bound on the scans'
+    rate.  The bound (HBM or tensor) is the routing stage's for the workload."""
+    r = stage_roofline("route_topk", ms / rounds, cfg, counts, peaks, peak_kind, long_region)
+    key = "alg_bytes_per_launch" if r["bound"] == "hbm" else "alg_flops_per_launch"
+    r[key] = r[key] * rounds
+    r["kernel"] = (f"msa_interleave_forward ({rounds} rounds: routing scans of the bank, plus the attention rounds "
+                   "and router-query projections in the same time)")
+    r["achieved"] = round(r["achieved"], 2)
+    r["frac"] = round(r["achieved"] / r["peak"], 4)
+    r["avg_launch_ms"] = round(ms, 4)
+    r["traffic"] = None
+    return r
+
+
+def run_interleave(args, rank, local_rank, world):
+    """Memory Interleave of the query path: per layer one msa_interleave_forward call of `--rounds`
+    rounds (route, the k best documents no earlier round chose, attention over every round's documents
+    ++ the local KV; the next round's router query is the round's output times a seeded W_route) over
+    a bank pooled before timing."""
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    import routed_sparse_attention_chunk_b200 as msa
+    cfg = workload_config(args)
+    R = args.rounds
+    if R < 1:
+        raise SystemExit("--rounds must be >= 1")
+    counts = workload_counts(cfg)
+    w = MSAWorkload(cfg, device, seed=1000 * rank, step_kind="query")
+    B, c = cfg.B, cfg
+    dt = cfg.torch_dtype
+    Mmax = R * c.Mmax  # every round's k documents fill Mmax rows in these workloads
+    g = torch.Generator(device=device).manual_seed(77 + 1000 * rank)
+    W = (torch.randn((c.Hq * c.d, c.Hr * c.dr), generator=g, device=device) / 64).to(dt) if R > 1 else None
+    ws = torch.empty(max(256, msa.interleave_workspace_size(B, c.Tq, c.Lloc, c.Hq, c.Hkv, c.d, c.Hr, c.dr, w.D, w.C,
+                                                            c.k, R, Mmax)), dtype=torch.uint8, device=device)
+    idx = [torch.empty((B, R * c.k), dtype=torch.int32, device=device) for _ in w.layers]
+    lse = torch.empty((B, c.Hq, c.Tq), dtype=torch.float32, device=device)
+    in_bytes = w.Krb.numel() * w.Krb.element_size()  # every round scans the whole bank
+    flush = None if in_bytes > L2_BYTES else torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(marks=None):
+        for l, L in enumerate(w.layers):
+            e0 = torch.cuda.Event(enable_timing=True) if marks is not None else None
+            if e0 is not None:
+                e0.record(stream)
+            msa.interleave_forward(L["Qr"], w.Krb, w.rn, w.coff_d, c.k, R, W, L["Q"], L["Kloc"], L["Vloc"], w.Kb,
+                                   w.Vb, Mmax, w.O[l], idx[l], ws, lse=lse, err_flag=w.flag)
+            if e0 is not None:
+                e1 = torch.cuda.Event(enable_timing=True)
+                e1.record(stream)
+                marks.append((e0, e1))
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    sampler = ClockSampler(device)
+    sampler.start()
+    n0 = msa.kernel_launch_count()
+    marks = []
+    for _ in range(args.steps):
+        if flush is not None:
+            flush.fill_(1.0)
+        step(marks)
+    torch.cuda.synchronize()
+    launches = msa.kernel_launch_count() - n0
+    clocks = sampler.stop()
+    call_ms = [a.elapsed_time(b) for a, b in marks]
+    step_sum = float(np.sum(call_ms))
+    flag = int(w.flag.item())
+    barrier(world, device)
+    ms_per_step = max_over_ranks(step_sum, world, device) / args.steps
+    value = B * c.Tq * world / (ms_per_step / 1e3)
+    peaks, peak_kind = load_peaks()
+    per = float(np.mean(call_ms))
+    roofline = interleave_roofline(cfg, counts, R, per, peaks, peak_kind, sustained_region(step_sum, clocks))
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded generators; see workloads/synth.py)",
+        "config": {"workload": workload_label(cfg),
+                   "step": f"Memory Interleave: per layer one msa_interleave_forward of {R} rounds (route + top-k of "
+                           f"{c.k} new documents, attention over all rounds' documents ++ local KV; next router "
+                           f"query = output x seeded W_route) over a bank pooled before timing",
+                   "l2": "inputs larger than L2" if flush is None else "L2 flushed between steps (not timed)",
+                   "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "stages": {"interleave_forward": {"ms_per_launch": round(per, 4), "launches": len(call_ms)}},
+        "gpu_launches": int(launches), "clocks": clocks, "err_flag": flag,
+    }
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world, device)
+        dist.destroy_process_group()
+    return result
+
+
 def run_gpu(args, rank, local_rank, world):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -1230,9 +1338,12 @@ def main():
     ap.add_argument("--step", choices=["full", "query"], default=None,
                     help="full: pool + query path per step; query: bank pooled before timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which_pass", choices=["forward", "backward", "state", "dga"], default="forward",
+    ap.add_argument("--pass", dest="which_pass", choices=["forward", "backward", "state", "dga", "interleave"],
+                    default="forward",
                     help="backward: time the backward of the query path instead of the forward step; "
-                         "state: the linear layers' memory injection (sum of the selected documents' states)")
+                         "state: the linear layers' memory injection (sum of the selected documents' states); "
+                         "dga: that injection and the gated delta rule; interleave: Memory Interleave rounds")
+    ap.add_argument("--rounds", type=int, default=2, help="Memory Interleave rounds (with --pass interleave)")
     ap.add_argument("--bank-kv", choices=["device", "host"], default="device",
                     help="where the pooled K̄ / V̄ live (host: page-locked host memory, the query path only)")
     ap.add_argument("--pipeline", action="store_true",
@@ -1253,6 +1364,8 @@ def main():
         res = run_state(args, rank, local_rank, world)
     elif args.which_pass == "dga":
         res = run_dga(args, rank, local_rank, world)
+    elif args.which_pass == "interleave":
+        res = run_interleave(args, rank, local_rank, world)
     else:
         res = run_gpu(args, rank, local_rank, world)
     if rank == 0 and res is not None:

@@ -58,6 +58,23 @@ def test_stage_roofline_bound_and_peak(name, stage, bound, unit):
         assert r["achieved"] == pytest.approx(work / (1e6 if unit == "GB/s" else 1e9))
 
 
+@pytest.mark.parametrize("name,bound,key", [
+    ("100m", "hbm", "route_bytes"),
+    ("stack10m", "tensor", "route_flops"),
+])
+def test_interleave_roofline_counts_every_rounds_scan(name, bound, key):
+    cfg = synth.get_config(name)
+    counts = bench.workload_counts(cfg)
+    for rounds in (1, 3):
+        r = bench.interleave_roofline(cfg, counts, rounds, 2.0, PEAKS, "measured", False)
+        work = r.get("alg_bytes_per_launch", r.get("alg_flops_per_launch"))
+        assert r["bound"] == bound and work == counts[key] * rounds
+        # achieved = all rounds' scan work / the whole call's time (2 ms here)
+        assert r["achieved"] == pytest.approx(work / 2.0 / (1e6 if bound == "hbm" else 1e9), rel=1e-3)
+        assert r["frac"] == pytest.approx(r["achieved"] / r["peak"], rel=1e-3)
+        assert r["avg_launch_ms"] == 2.0 and r["traffic"] is None
+
+
 def test_traffic_records_are_well_formed():
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
         rec = json.load(f)
