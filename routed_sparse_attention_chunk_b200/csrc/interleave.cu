@@ -10,7 +10,9 @@
 // The map is a small dense product (rows = B * Tq query tokens, K = Hq * d,
 // N = Hr * dr): a CUDA-core tiled kernel with fp32 accumulation, one CTA per
 // BM x 64 output tile, operands staged through shared memory in steps of 32.
-// It is a few percent of a round next to the routing scan of a large bank.
+// With few rows (64 query tokens) that is 64 CTAs, each walking all of K in
+// dependent steps, so the map is latency-bound: a few hundred microseconds for
+// K = 4096, N = 1024, against the routing scan's ~0.5 ms on a 100M-token bank.
 #include <math.h>
 
 #include "common.cuh"
