@@ -210,3 +210,32 @@ def test_noalloc_checks_arguments_before_its_size():
     assert call(None, 128, k) == INVALID         # no Qr
     assert call(FAKE, 128, D + 1) == INVALID     # k > D
     assert call(FAKE, 128, k) == -5              # MSA_ERR_TOO_LARGE
+
+
+def _largest_fitting_docs(B, Tq, Hr, chunks_per_doc, k):
+    lo, hi = 1, 1 << 26
+    while lo < hi:
+        m = (lo + hi + 1) // 2
+        if msa.route_topk_workspace_size(B, Tq, Hr, m, chunks_per_doc * m, k) <= msa.NOALLOC_SCRATCH_BYTES:
+            lo = m
+        else:
+            hi = m - 1
+    return lo
+
+
+def test_noalloc_bounds_in_the_header_are_exact():
+    # msa.h states the largest document counts the allocation-free entry point takes for two
+    # shapes (documents of 8 chunks, Hr = 8, k = 16); they are the exact boundary of the library's
+    # own size function, and its size formula holds to the 256-byte rounding of each part
+    text = open(os.path.join(ROOT, "include", "msa.h")).read()
+    text = re.sub(r"\s+", " ", re.sub(r"\n\s*\*", " ", text))  # comment lines joined
+    one = int(re.search(r"fits up to ([0-9,]+) documents", text).group(1).replace(",", ""))
+    many = int(re.search(r"64 one-token queries up to ([0-9,]+) documents", text).group(1).replace(",", ""))
+    assert _largest_fitting_docs(1, 64, 8, 8, 16) == one
+    assert _largest_fitting_docs(64, 1, 8, 8, 16) == many
+    for B, Tq, D in ((1, 64, one), (64, 1, many), (3, 7, 9000), (2, 1, 100)):
+        Hr, k, C = 8, 16, 8 * D
+        nslice = -(-D // 8192)
+        formula = 4 * (B * D + B) + 4 * C + 4 * B * Tq * Hr + (8 * B * k * nslice if D > 8192 else 0)
+        got = msa.route_topk_workspace_size(B, Tq, Hr, D, C, k)
+        assert formula <= got <= formula + 4 * 255
