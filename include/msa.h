@@ -292,8 +292,10 @@ msa_status msa_sparse_attn(msa_dtype dt, const void* Q, const void* Kloc, const 
  *   topk_idx int32 [B, k];  doc_chunk_off int64 [D+1];
  *   Kbar, Vbar [C, Hkv, d] dtype dt (device memory, or page-locked host memory
  *   as for msa_gather).
- * For bf16, d = 128 and the shapes the tensor-core kernels take (decode: up to
- * 16 query rows per KV head; prefill: a GQA group that divides 128 rows), a
+ * For bf16, d = 128 and the shapes the tensor-core kernels take (decode: at most
+ * 4 query tokens and 16 query rows per KV head; prefill: a GQA group G that
+ * divides 128 with at least 8 tokens per block of 128 rows, and at least
+ * min(16, 64 / G) query tokens), a
  * small plan kernel cuts every query's selection into runs of at most 8
  * consecutive chunk rows of one document, and the attention kernel loads those
  * runs straight from the bank with TMA.  A run shorter than 8 rows is padded
@@ -367,7 +369,7 @@ msa_status msa_gather_backward(const int32_t* topk_idx, int64_t B, int k, const 
  * cosine s(t, c) = (1/Hr) sum_h cos(Qr[b, t, h], Krbar[c, h]) ("MSA: Memory
  * Sparse Attention" README, "Architecture"); the model card's auxiliary
  * routing loss is not defined on the pages, so its gradient with respect to
- * each selected document's score, d_score (fp32 [B, k], host layout as
+ * each selected document's score, d_score (fp32 [B, k], laid out as
  * topk_idx), is the input.  The max passes it to its argmax pair (t*, c*),
  * the first in (chunk, token) order on exact ties, with s computed as
  * msa_route_topk computes it (kr_rnorm for the key norms); then for every
