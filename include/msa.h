@@ -473,8 +473,8 @@ msa_status msa_interleave_forward(msa_dtype dt, const void* Qr0, int Hr, int dr,
  *   e.g. heads x key dim x value dim);  topk_idx int32 [B, k];  S_ext fp32 [B, S]
  * S must make a state a whole number of 16-byte vectors (S % 8 == 0 for bf16,
  * S % 4 == 0 for fp32), else MSA_ERR_UNSUPPORTED; B <= 65535.  How the states
- * are produced, and the delta rule that consumes S_ext, are not part of this
- * library.  Device flag: MSA_FLAG_INDEX_OOB for an index outside [0, D); that
+ * are produced is not part of this library (msa_gated_delta_rule below
+ * consumes S_ext).  Device flag: MSA_FLAG_INDEX_OOB for an index outside [0, D); that
  * selection adds nothing.
  * ---------------------------------------------------------------------- */
 msa_status msa_state_gather_sum(msa_dtype dt, const void* states, int64_t D, int64_t S,
@@ -496,9 +496,11 @@ msa_status msa_state_gather_sum(msa_dtype dt, const void* states, int64_t D, int
  *   g (log gates, <= 0), beta [B, T, Hv] fp32;  h0, hT fp32 [B, Hv, dk, dv]
  *   (hT, the state after the last token, may be NULL).
  * Keys are used as given (the model normalises them before the rule).
- * Computed chunk by chunk (64 tokens) in fp32 on the CUDA cores, one CTA per
- * (value head, query): the within-chunk products, a unit lower-triangular
- * solve for the chunk's new values, then the state update.
+ * Computed in fp32 on the CUDA cores, one CTA per (value head, query):
+ * sequences of up to 16 tokens (decode) in the token-by-token form with the
+ * state in registers; longer ones chunk by chunk (64 tokens): the within-chunk
+ * products, a unit lower-triangular solve for the chunk's new values, then the
+ * state update.
  * Supported: dk = dv = 128, Hv % Hk == 0, B <= 65535.  No workspace.
  * ---------------------------------------------------------------------- */
 msa_status msa_gated_delta_rule(msa_dtype dt, const void* q, const void* k, const void* v, const float* g,
