@@ -1,8 +1,10 @@
 """Python binding of the MSA memory-path library (include/msa.h) for B200.
 
 Argument marshalling only: every function takes caller-allocated torch tensors,
-checks that they are contiguous CUDA tensors of the right dtype, and passes raw
-pointers and sizes to the C ABI in libmsa.so on the current (or given) stream.
+checks that they are contiguous CUDA tensors of the right dtype (the bank's
+K̄ / V̄ may instead be pinned host tensors: the host tier, read in place), and
+passes raw pointers and sizes to the C ABI in libmsa.so on the current (or
+given) stream.
 All computation happens in the library's CUDA kernels; there is no fallback.
 """
 from __future__ import annotations
