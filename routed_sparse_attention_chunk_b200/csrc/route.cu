@@ -14,7 +14,9 @@
 //
 // This file holds the CUDA-core kernel used for fp32 banks and for shapes the
 // tensor-core kernel does not take: one CTA per tile of 32 chunks, one warp per
-// router head, lane = chunk, the chunk's router key held in registers.
+// router head, lane = chunk, the chunk's router key held in registers.  It also
+// holds the routing prelude that every scan starts from: the per-document keys
+// zeroed, the chunk -> document map, and the query norms of the tensor-core scan.
 #include "common.cuh"
 #include "internal.h"
 
